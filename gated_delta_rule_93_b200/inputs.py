@@ -1,0 +1,118 @@
+"""Seeded synthetic inputs for the gated delta-rule mixer.
+
+This module only draws random numbers and shapes them; it holds none of the
+method's arithmetic, so both the CUDA path and the fp64 oracle consume the
+exact same values from here.
+
+Recipe (every workload, one CPU ``torch.Generator`` per call):
+  * q, k ~ N(0, 1) in fp32, L2-normalised over d_k for each (b, t, h), then
+    cast to the input dtype;
+  * v ~ N(0, 1), cast to the input dtype;
+  * g = log(alpha) = -0.1 * softplus(N(0, 1)), fp32, shape [B,T,H] for a
+    scalar per-head gate or [B,T,H,d_k] for a per-channel gate;
+  * beta = sigmoid(N(0, 1)), fp32;
+  * S0 = N(0, 0.02^2) fp32 [B,H,d_v,d_k] where the workload has one, else None.
+Draw order: q, k, v, g, beta, S0.  The decode workload draws its initial
+state first, then q, k, v, g, beta of each step in step order.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+import torch.nn.functional as F
+
+
+@dataclass(frozen=True)
+class Workload:
+    """A named shape + dtype recipe."""
+
+    name: str
+    kind: str  # "chunk" (gdr_chunk_fwd) or "step" (gdr_step)
+    B: int
+    T: int
+    H: int
+    dk: int
+    dv: int
+    dtype: torch.dtype
+    gate: str  # "scalar" or "channel"
+    with_S0: bool
+    want_S_T: bool
+    steps: int = 1  # decode workloads: consecutive steps
+    C: int = 64
+    note: str = field(default="", compare=False)
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.T if self.kind == "chunk" else self.B * self.steps
+
+
+# The five workloads, named by what they are.
+WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("tiny_fp32", "chunk", 1, 256, 2, 32, 32, torch.float32, "scalar", False, True,
+                 note="tiny Gated DeltaNet forward, fp32"),
+        Workload("gdn_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16, "scalar",
+                 False, True, note="Gated DeltaNet layer forward at 350M-model shape"),
+        Workload("gdn_b1_t65536_h16_d128", "chunk", 1, 65536, 16, 128, 128, torch.bfloat16,
+                 "scalar", True, True, note="long-sequence Gated DeltaNet forward"),
+        Workload("kda_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
+                 "channel", False, True, note="per-channel (Kimi-Delta-style) gate forward"),
+        Workload("decode_n256_h16_d128_x1024", "step", 256, 1, 16, 128, 128, torch.bfloat16,
+                 "scalar", True, True, steps=1024,
+                 note="recurrent decode step, 256 sequences, 1024 consecutive steps"),
+    ]
+}
+
+
+def _unit_rows(x: torch.Tensor) -> torch.Tensor:
+    return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+
+
+def make_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, gate="scalar", with_S0=False,
+                      seed=0):
+    """Inputs for ``gdr_chunk_fwd`` on the CPU: dict of q,k,v,g,beta,S0 (S0 may be None)."""
+    gen = torch.Generator().manual_seed(seed)
+    q = _unit_rows(torch.randn(B, T, H, dk, generator=gen)).to(dtype)
+    k = _unit_rows(torch.randn(B, T, H, dk, generator=gen)).to(dtype)
+    v = torch.randn(B, T, H, dv, generator=gen).to(dtype)
+    gshape = (B, T, H, dk) if gate == "channel" else (B, T, H)
+    g = -0.1 * F.softplus(torch.randn(*gshape, generator=gen))
+    beta = torch.sigmoid(torch.randn(B, T, H, generator=gen))
+    S0 = 0.02 * torch.randn(B, H, dv, dk, generator=gen) if with_S0 else None
+    return dict(q=q, k=k, v=v, g=g.float(), beta=beta.float(), S0=S0)
+
+
+def make_step_inputs(N, H, dk, dv, steps, dtype=torch.bfloat16, gate="scalar", seed=0):
+    """Inputs for ``steps`` consecutive ``gdr_step`` calls.
+
+    Returns dict with S0 [N,H,dv,dk] fp32 and per-step stacks q,k [steps,N,H,dk],
+    v [steps,N,H,dv], g [steps,N,H] (or [steps,N,H,dk]), beta [steps,N,H].
+    """
+    gen = torch.Generator().manual_seed(seed)
+    S0 = 0.02 * torch.randn(N, H, dv, dk, generator=gen)
+    qs, ks, vs, gs, bs = [], [], [], [], []
+    gshape = (N, H, dk) if gate == "channel" else (N, H)
+    for _ in range(steps):
+        qs.append(_unit_rows(torch.randn(N, H, dk, generator=gen)).to(dtype))
+        ks.append(_unit_rows(torch.randn(N, H, dk, generator=gen)).to(dtype))
+        vs.append(torch.randn(N, H, dv, generator=gen).to(dtype))
+        gs.append(-0.1 * F.softplus(torch.randn(*gshape, generator=gen)))
+        bs.append(torch.sigmoid(torch.randn(N, H, generator=gen)))
+    return dict(S0=S0.float(), q=torch.stack(qs), k=torch.stack(ks), v=torch.stack(vs),
+                g=torch.stack(gs).float(), beta=torch.stack(bs).float())
+
+
+def make_workload_inputs(w: Workload, seed=0, steps=None):
+    if w.kind == "chunk":
+        return make_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.gate, w.with_S0, seed)
+    return make_step_inputs(w.B, w.H, w.dk, w.dv, steps or w.steps, w.dtype, w.gate, seed)
+
+
+def to_numpy_input(t: torch.Tensor):
+    """CPU tensor -> numpy array the oracle accepts (float32, or uint16 bf16 bits)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view("uint16")
+    return t.float().numpy()

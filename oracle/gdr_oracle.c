@@ -1,0 +1,193 @@
+/*
+ * Gated delta-rule oracle: plain fp64 token-by-token recurrence on the CPU.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline use it.  It shares no code, header or constant with the CUDA
+ * library.
+ *
+ * What it computes (state S has shape d_v x d_k, row i = value channel,
+ * column j = key channel):
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t
+ *
+ * with alpha_t = exp(g_t).  g_t is a scalar per head or a vector over the key
+ * channels.  Sources:
+ *   - "Decoding Hybrid Linear Attention Architectures", section 3, items 2
+ *     (delta rule), 3 (gated delta rule, scalar gate) and 6 (Gated Delta
+ *     Attention, per-channel gate), plus the single-step pseudocode under
+ *     item 6, which fixes the order: decay, then erase along k_t, then write.
+ *   - "Linear Attention Variants (RetNet, GLA, DeltaNet, Based)", section
+ *     "DeltaNet: Error-Correcting Writes": the update written as
+ *     S + beta v k^T - beta (S k) k^T, i.e. read what k_t maps to, subtract
+ *     it, write the new value.  That is the form coded below.
+ *   - "Decoding Hybrid Linear Attention Architectures", section 5 (the
+ *     gates are accumulated in log space): the gate enters as g = log alpha.
+ *
+ * Readings where the pages are loose (each also listed in the design notes):
+ *   - the output reads the state after the write (o_t = S_t q_t);
+ *   - no 1/sqrt(d_k) query scale (no page applies one);
+ *   - for a per-channel gate the decay scales the key axis of S and comes
+ *     before the erase (pseudocode order under section 3 item 6).
+ *
+ * Inputs q, k, v are either fp32 or bf16 (raw 16-bit patterns); bf16 is
+ * widened exactly (bit shift) and all arithmetic is in double.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { OR_F32 = 0, OR_BF16 = 1 };
+enum { OR_GATE_SCALAR = 0, OR_GATE_PER_CHANNEL = 1 };
+
+/* Exact widening of one input element to double. */
+static double load_elem(const void *base, size_t idx, int dtype) {
+    if (dtype == OR_F32) return (double)((const float *)base)[idx];
+    uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    const void *q, *k, *v;
+    int in_dtype;
+    const float *g;
+    int gate_kind;
+    const float *beta;
+    const double *S0; /* may be NULL: zero initial state */
+    double *o;
+    double *S_T;      /* may be NULL */
+    int B, T, H, dk, dv;
+    int next;         /* shared work counter over (b, h) */
+    pthread_mutex_t lock;
+} job_t;
+
+/*
+ * One (b, h) pair: the recurrence over t = 0..T-1.
+ * Layouts: q,k [B,T,H,dk]; v,o [B,T,H,dv]; g [B,T,H] or [B,T,H,dk];
+ * beta [B,T,H]; S0,S_T [B,H,dv,dk].
+ */
+static void run_head(job_t *J, int b, int h) {
+    const int T = J->T, H = J->H, dk = J->dk, dv = J->dv;
+    double *S = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *kk = (double *)malloc(sizeof(double) * dk);
+    double *qq = (double *)malloc(sizeof(double) * dk);
+    double *alpha = (double *)malloc(sizeof(double) * dk);
+    double *p = (double *)malloc(sizeof(double) * dv);
+    const size_t sidx = ((size_t)b * H + h) * (size_t)dv * dk;
+    if (J->S0)
+        memcpy(S, J->S0 + sidx, sizeof(double) * (size_t)dv * dk);
+    else
+        memset(S, 0, sizeof(double) * (size_t)dv * dk);
+
+    for (int t = 0; t < T; ++t) {
+        const size_t tok = ((size_t)b * T + t) * H + h;
+        for (int j = 0; j < dk; ++j) {
+            kk[j] = load_elem(J->k, tok * dk + j, J->in_dtype);
+            qq[j] = load_elem(J->q, tok * dk + j, J->in_dtype);
+        }
+        if (J->gate_kind == OR_GATE_PER_CHANNEL) {
+            for (int j = 0; j < dk; ++j) alpha[j] = exp((double)J->g[tok * dk + j]);
+        } else {
+            const double a = exp((double)J->g[tok]);
+            for (int j = 0; j < dk; ++j) alpha[j] = a;
+        }
+        const double beta = (double)J->beta[tok];
+
+        /* 1. decay: S <- S Diag(alpha)  (scales the key axis) */
+        for (int i = 0; i < dv; ++i)
+            for (int j = 0; j < dk; ++j) S[(size_t)i * dk + j] *= alpha[j];
+
+        /* 2. read what k_t currently maps to: p = S k */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * kk[j];
+            p[i] = acc;
+        }
+
+        /* 3. erase-and-write: S <- S + beta (v - p) k^T */
+        for (int i = 0; i < dv; ++i) {
+            const double vi = load_elem(J->v, tok * dv + i, J->in_dtype);
+            const double c = beta * (vi - p[i]);
+            for (int j = 0; j < dk; ++j) S[(size_t)i * dk + j] += c * kk[j];
+        }
+
+        /* 4. read-out after the write: o = S q */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * qq[j];
+            J->o[tok * dv + i] = acc;
+        }
+    }
+    if (J->S_T) memcpy(J->S_T + sidx, S, sizeof(double) * (size_t)dv * dk);
+    free(S);
+    free(kk);
+    free(qq);
+    free(alpha);
+    free(p);
+}
+
+static void *worker(void *arg) {
+    job_t *J = (job_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int w = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (w >= J->B * J->H) break;
+        run_head(J, w / J->H, w % J->H);
+    }
+    return NULL;
+}
+
+/*
+ * Forward over a whole sequence.  Returns 0 on success, -1 on a bad
+ * argument.  nthreads <= 0 means one thread per online core.
+ */
+int oracle_gdr_fwd(const void *q, const void *k, const void *v, int in_dtype,
+                   const float *g, int gate_kind, const float *beta,
+                   const double *S0, double *o, double *S_T, int B, int T,
+                   int H, int dk, int dv, int nthreads) {
+    if (!q || !k || !v || !g || !beta || !o) return -1;
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (in_dtype != OR_F32 && in_dtype != OR_BF16) return -1;
+    if (gate_kind != OR_GATE_SCALAR && gate_kind != OR_GATE_PER_CHANNEL) return -1;
+    job_t J;
+    J.q = q; J.k = k; J.v = v; J.in_dtype = in_dtype;
+    J.g = g; J.gate_kind = gate_kind; J.beta = beta;
+    J.S0 = S0; J.o = o; J.S_T = S_T;
+    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+    J.next = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    int n = nthreads;
+    if (n <= 0) n = 1;
+    if (n > B * H) n = B * H;
+    if (n <= 1) {
+        worker(&J);
+    } else {
+        pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * n);
+        for (int i = 0; i < n; ++i) pthread_create(&th[i], NULL, worker, &J);
+        for (int i = 0; i < n; ++i) pthread_join(th[i], NULL);
+        free(th);
+    }
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
+
+/*
+ * One recurrent step for N independent states ("Decoding Hybrid Linear
+ * Attention Architectures", section 6: a constant-cost update of the
+ * fixed-size state per decoded token).  S [N,H,dv,dk] is updated in place;
+ * q,k [N,H,dk]; v,o [N,H,dv]; g [N,H] or [N,H,dk]; beta [N,H].
+ * It is the forward above with T = 1 and S_T aliasing S0.
+ */
+int oracle_gdr_step(const void *q, const void *k, const void *v, int in_dtype,
+                    const float *g, int gate_kind, const float *beta, double *S,
+                    double *o, int N, int H, int dk, int dv, int nthreads) {
+    if (!S) return -1;
+    return oracle_gdr_fwd(q, k, v, in_dtype, g, gate_kind, beta, S, o, S, N, 1,
+                          H, dk, dv, nthreads);
+}
