@@ -1,0 +1,396 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta-rule chunked forward on B200.
+
+Prints ONE JSON line on rank 0.  Default workload: the Gated DeltaNet layer
+forward at 350M-model shape (B=8, T=4096, H=16, d_k=d_v=128, C=64, bf16
+q/k/v, fp32 gates and state, S0 = 0, S_T returned).  A "step" is one
+gdr_chunk_fwd call over that batch.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
+
+Multi-GPU (launched by torchrun): every rank runs the same per-GPU workload
+on its own seeded batch (independent (b, h) problems, no collective on the
+data path) -> weak scaling; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from gated_delta_rule_93_b200.inputs import WORKLOADS, make_workload_inputs  # noqa: E402
+
+METRIC = "tokens/s and TFLOP/s per gated-delta layer fwd (1 B200), % of roofline"
+DEFAULT_WORKLOAD = "gdn_b8_t4096_h16_d128"
+L2_BYTES = 126 * 1024 * 1024
+CHUNK_KERNEL_SOURCES = ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
+                        "gated_delta_rule_93_b200/csrc/gdr_chunk_simt.cu",
+                        "gated_delta_rule_93_b200/csrc/gdr_abi.cu"]
+
+
+# ------------------------------------------------------------------ work model
+def algorithmic_bytes(w):
+    """HBM bytes a perfect fused kernel must move for one step (per GPU)."""
+    e_in = 2 if w.dtype == torch.bfloat16 else 4
+    gate_elems = w.dk if w.gate == "channel" else 1
+    per_tok = (2 * w.dk + w.dv) * e_in + w.dv * e_in + 4 * gate_elems + 4
+    state = 4 * w.dk * w.dv * w.B * w.H
+    return w.B * w.T * w.H * per_tok + state * (int(w.with_S0) + int(w.want_S_T))
+
+
+def algorithmic_flops(w, C=64):
+    """Chunked-method flops per step, counting masked products as triangles:
+    6 d_k d_v + C (3 d_k + 2 d_v) + C^2 / 3 per token-head."""
+    per = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0
+    return w.B * w.T * w.H * per
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in CHUNK_KERNEL_SOURCES:
+        p = os.path.join(ROOT, rel)
+        if os.path.exists(p):
+            with open(p, "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    cur = kernel_source_hash()
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == workload:
+                if parts[2] == cur:
+                    return float(parts[1])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    from gated_delta_rule_93_b200 import binding
+
+    w = WORKLOADS[args.workload]
+    if w.kind != "chunk":
+        raise SystemExit("bench.py times the chunked forward; the decode workload is a "
+                         "parity case")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    host = make_workload_inputs(w, seed=rank)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
+    o = torch.empty(w.B, w.T, w.H, w.dv, dtype=w.dtype, device=dev)
+    S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev) if w.want_S_T \
+        else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o, S_T=S_T,
+                          output_final_state=S_T is not None)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if binding.device_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+
+    # ---- device-timed region: inputs resident in HBM, one launch per step
+    vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    clocks = ClockSampler(vis[local_rank].strip() if local_rank < len(vis) else local_rank)
+    clocks.start()
+    time.sleep(0.15)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    per_launch_ms = [a.elapsed_time(b) for a, b in ev]
+    if binding.device_status() != 0:
+        raise RuntimeError("device status word set during the timed region")
+
+    # ---- end to end through the same API with host buffers (pinned)
+    pin = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory() if S_T is not None else None
+    h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
+    d2h = o_h.numel() * o_h.element_size() + (S_h.numel() * 4 if S_h is not None else 0)
+
+    def e2e_step():
+        for kk, v in pin.items():
+            if v is not None:
+                d[kk].copy_(v, non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        if S_h is not None:
+            S_h.copy_(S_T, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+
+    # ---- max over ranks
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, e2e_ms = t.tolist()
+
+    if rank != 0:
+        return None
+    ms_step = total_ms / args.steps
+    tokens_step = w.tokens
+    value = world * tokens_step * args.steps / (total_ms / 1e3)
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    abytes = algorithmic_bytes(w)
+    aflops = algorithmic_flops(w, w.C)
+    avg_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
+    achieved = abytes / (avg_launch_ms / 1e3) / 1e9
+    roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (tc_peak * 1e12)) * 1e3
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+        "data": "synthetic (seeded; q,k L2-normalised N(0,1), v N(0,1), "
+                "beta=sigmoid(N(0,1)), log alpha=-0.1 softplus(N(0,1)))",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                   "chunk": w.C, "gate": w.gate, "S0": w.with_S0, "S_T": w.want_S_T,
+                   "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"independent (b,h) shards x{world}",
+                   "l2": "inputs exceed L2 (%.0f MB > 126 MB); no flush" %
+                         (algorithmic_bytes(w) / 1e6)},
+        "tflops": aflops * world * args.steps / (total_ms / 1e3) / 1e12,
+        "roofline_time_ms": roof_ms,
+        "roofline_fraction": roof_ms / ms_step,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name),
+                     "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
+                     "kernel": "gdr_chunk_fwd"},
+        "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    return line
+
+
+# ------------------------------------------------------------------ oracle arm
+def cpu_baseline(w, target_s=12.0):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the workload:
+    all B*H heads over the first T' tokens, T' grown until a run takes a few
+    seconds, then tokens/s = B*T'/elapsed."""
+    import oracle
+    from gated_delta_rule_93_b200.inputs import to_numpy_input
+
+    oracle.build()
+    inp = make_workload_inputs(w)
+    n = min(oracle.default_threads(), w.B * w.H)
+    Tp = 16
+    while True:
+        sl = {k: (v[:, :Tp].contiguous() if (v is not None and k != "S0") else v)
+              for k, v in inp.items()}
+        args = [to_numpy_input(sl["q"]), to_numpy_input(sl["k"]), to_numpy_input(sl["v"]),
+                sl["g"].numpy(), sl["beta"].numpy(),
+                None if sl["S0"] is None else sl["S0"].double().numpy()]
+        t = time.perf_counter()
+        oracle.gdr_fwd(*args, gate=w.gate, nthreads=n)
+        el = time.perf_counter() - t
+        if el >= target_s / 4 or Tp >= w.T:
+            break
+        Tp = min(w.T, max(Tp * 2, int(Tp * (target_s / 3) / max(el, 1e-3))))
+    return {"value": w.B * Tp / el, "unit": "tokens/s", "cores": n, "kind": "oracle",
+            "sample": f"all {w.B}x{w.H} (b,h) pairs, first {Tp} of {w.T} tokens "
+                      f"({el:.2f} s wall, fp64 C recurrence, {n} threads)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    import oracle
+    from gated_delta_rule_93_b200.inputs import to_numpy_input
+
+    oracle.build()
+    inp = make_workload_inputs(w)
+    n = min(oracle.default_threads(), w.B * w.H)
+    # bounded per-step sample: first Tp tokens of every (b, h)
+    Tp = max(1, min(w.T, args.ref_tokens))
+    sl = {k: (v[:, :Tp].contiguous() if (v is not None and k != "S0") else v)
+          for k, v in inp.items()}
+    a = [to_numpy_input(sl["q"]), to_numpy_input(sl["k"]), to_numpy_input(sl["v"]),
+         sl["g"].numpy(), sl["beta"].numpy(),
+         None if sl["S0"] is None else sl["S0"].double().numpy()]
+    for _ in range(args.warmup):
+        oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)
+    el = time.perf_counter() - t
+    val = w.B * Tp * args.steps / el
+    sample = (f"all {w.B}x{w.H} (b,h) pairs, first {Tp} of {w.T} tokens per step "
+              f"(fp64 C recurrence, {n} threads)")
+    return {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk,
+                       "d_v": w.dv, "chunk": w.C, "gate": w.gate},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": n, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-tokens", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,18 @@
+"""Gated delta-rule sequence mixer for NVIDIA B200 (sm_100a).
+
+The computation lives in ``libgdr.so`` (CUDA kernels behind the C ABI in
+``include/gdr.h``); ``binding`` is a ctypes front-end with the same names.
+Importing this package does not load the library; the first call does.
+"""
+from .binding import (  # noqa: F401
+    GdrError,
+    chunk_fwd,
+    chunk_fwd_workspace_bytes,
+    device_status,
+    lib,
+    status_string,
+    step,
+)
+
+__all__ = ["chunk_fwd", "chunk_fwd_workspace_bytes", "step", "device_status", "lib",
+           "status_string", "GdrError"]

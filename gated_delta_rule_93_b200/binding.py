@@ -1,0 +1,195 @@
+"""Thin Python binding of ``libgdr.so`` (argument marshalling only).
+
+Every step of the computation runs in the library's CUDA kernels; this
+module checks tensor devices, dtypes, shapes and contiguity, then passes
+raw device pointers and the current CUDA stream through ctypes.  There is no
+CPU fallback: if the library is missing, or a tensor is not on a CUDA
+device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdr.so")
+_lib = None
+_lock = threading.Lock()
+
+GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_WORKSPACE, GDR_ERR_CUDA, \
+    GDR_ERR_TIMEOUT = range(6)
+GDR_F32, GDR_BF16 = 0, 1
+GDR_GATE_SCALAR, GDR_GATE_PER_CHANNEL = 0, 1
+
+EXPORTS = (
+    "gdr_chunk_fwd_workspace_bytes",
+    "gdr_chunk_fwd",
+    "gdr_step",
+    "gdr_get_device_status",
+    "gdr_status_string",
+    "gdr_last_error_message",
+    "gdr_version",
+)
+
+
+class GdrError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{status_string(status)}: {msg}")
+        self.status = status
+
+
+def lib():
+    """Load ``libgdr.so`` once; raise if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m gated_delta_rule_93_b200.build` (no CPU fallback exists)")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            L.gdr_chunk_fwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
+            L.gdr_chunk_fwd_workspace_bytes.restype = sz
+            L.gdr_chunk_fwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, i, i, i, i, i, i,
+                                        vp, sz, vp]
+            L.gdr_chunk_fwd.restype = i
+            L.gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp]
+            L.gdr_step.restype = i
+            L.gdr_get_device_status.argtypes = [vp]
+            L.gdr_get_device_status.restype = i
+            L.gdr_status_string.argtypes = [i]
+            L.gdr_status_string.restype = ctypes.c_char_p
+            L.gdr_last_error_message.argtypes = []
+            L.gdr_last_error_message.restype = ctypes.c_char_p
+            L.gdr_version.argtypes = []
+            L.gdr_version.restype = i
+            _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().gdr_status_string(int(s)).decode()
+
+
+def _check(rc):
+    if rc != GDR_OK:
+        raise GdrError(rc, lib().gdr_last_error_message().decode())
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device (no CPU path exists)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _in_dtype(dt):
+    if dt == torch.bfloat16:
+        return GDR_BF16
+    if dt == torch.float32:
+        return GDR_F32
+    raise TypeError(f"q/k/v dtype must be bfloat16 or float32, got {dt}")
+
+
+def chunk_fwd_workspace_bytes(B, T, H, dk, dv, C=64, dtype=torch.bfloat16, gate="scalar"):
+    gk = GDR_GATE_PER_CHANNEL if gate == "channel" else GDR_GATE_SCALAR
+    return int(lib().gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, _in_dtype(dtype), gk))
+
+
+def chunk_fwd(q, k, v, g, beta, S0=None, *, output_final_state=True, o=None, S_T=None, C=64,
+              workspace=None, stream=None):
+    """Chunkwise forward, ``gdr_chunk_fwd``.  Returns (o, S_T or None).
+
+    q, k [B,T,H,dk]; v [B,T,H,dv] (bf16 or fp32, one dtype); g [B,T,H] (scalar
+    gate) or [B,T,H,dk] (per-channel gate) fp32 log alpha; beta [B,T,H] fp32;
+    S0 [B,H,dv,dk] fp32 or None.
+    """
+    _need(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (B, T, H, dk), dev)
+    _need(v, "v", dt, (B, T, H, dv), dev)
+    if g.dim() == 4:
+        _need(g, "g", torch.float32, (B, T, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (B, T, H), dev)
+        gk = GDR_GATE_SCALAR
+    _need(beta, "beta", torch.float32, (B, T, H), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _need(o, "o", dt, (B, T, H, dv), dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
+    ws = chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, dt, "channel" if gk else "scalar")
+    if ws and workspace is None:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk,
+                                 _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, C,
+                                 _ptr(workspace), workspace.numel() if workspace is not None
+                                 else 0, _stream_handle(stream))
+    _check(rc)
+    return o, S_T
+
+
+def step(q, k, v, g, beta, S, *, o=None, stream=None):
+    """One decode step, ``gdr_step``: S [N,H,dv,dk] fp32 is updated in place.
+
+    q, k [N,H,dk]; v [N,H,dv]; g [N,H] or [N,H,dk]; beta [N,H].  Returns o.
+    """
+    _need(q, "q")
+    dev = q.device
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (N, H, dk), dev)
+    _need(v, "v", dt, (N, H, dv), dev)
+    if g.dim() == 3:
+        _need(g, "g", torch.float32, (N, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (N, H), dev)
+        gk = GDR_GATE_SCALAR
+    _need(beta, "beta", torch.float32, (N, H), dev)
+    _need(S, "S", torch.float32, (N, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=dt, device=dev)
+    _need(o, "o", dt, (N, H, dv), dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_step(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk, _ptr(beta),
+                            _ptr(S), _ptr(o), N, H, dk, dv, _stream_handle(stream))
+    _check(rc)
+    return o
+
+
+def device_status(stream=None):
+    """Synchronise and read/clear the library's device status word (0 = OK)."""
+    return int(lib().gdr_get_device_status(_stream_handle(stream)))

@@ -1,0 +1,172 @@
+// C ABI of the gated delta-rule library: argument validation, dispatch to
+// the kernels, status reporting.  See include/gdr.h for the contract.
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "gdr_internal.cuh"
+
+namespace gdr {
+__device__ unsigned int g_device_status = 0;
+}
+
+namespace {
+
+thread_local char t_msg[512] = "";
+
+gdr_status fail(gdr_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_msg, sizeof t_msg, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+gdr_status ok() {
+  t_msg[0] = '\0';
+  return GDR_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+gdr_status from_cuda(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return ok();
+  return fail(GDR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Device address of the status word on the current device (cached per device).
+cudaError_t status_word(unsigned int **out) {
+  static unsigned int *cache[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!cache[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, gdr::g_device_status);
+    if (e != cudaSuccess) return e;
+    cache[dev] = static_cast<unsigned int *>(p);
+  }
+  *out = cache[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr_version(void) { return 100; }
+
+const char *gdr_status_string(gdr_status s) {
+  switch (s) {
+    case GDR_OK: return "GDR_OK";
+    case GDR_ERR_INVALID_ARG: return "GDR_ERR_INVALID_ARG";
+    case GDR_ERR_UNSUPPORTED: return "GDR_ERR_UNSUPPORTED";
+    case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
+    case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
+    case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+  }
+  return "GDR_ERR_UNKNOWN";
+}
+
+const char *gdr_last_error_message(void) { return t_msg; }
+
+size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int C,
+                                     gdr_dtype in_dtype, gdr_gate_kind gate) {
+  (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)C; (void)in_dtype; (void)gate;
+  return 0;  // every chunked-forward kernel keeps its intermediates on chip
+}
+
+gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                         const float *g, gdr_gate_kind gate, const float *beta,
+                         const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
+                         int dv, int C, void *workspace, size_t ws_bytes,
+                         gdr_stream_t stream) {
+  if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "negative B/T/H");
+  if (in_dtype != GDR_F32 && in_dtype != GDR_BF16)
+    return fail(GDR_ERR_INVALID_ARG, "in_dtype must be GDR_F32 or GDR_BF16");
+  if (gate != GDR_GATE_SCALAR && gate != GDR_GATE_PER_CHANNEL)
+    return fail(GDR_ERR_INVALID_ARG, "unknown gate kind");
+  if (C != 64) return fail(GDR_ERR_UNSUPPORTED, "chunk size C=%d (only 64 is built)", C);
+  if (!head_dim_ok(dk) || !head_dim_ok(dv))
+    return fail(GDR_ERR_UNSUPPORTED, "head dims dk=%d dv=%d (need 32, 64 or 128)", dk, dv);
+  const size_t need_ws = gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, in_dtype, gate);
+  if (ws_bytes < need_ws || (need_ws && !workspace))
+    return fail(GDR_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need_ws);
+  if ((size_t)B * (size_t)H * (size_t)T > (size_t)1 << 40)
+    return fail(GDR_ERR_INVALID_ARG, "problem too large");
+  const bool empty_tokens = (size_t)B * H * T == 0;
+  const bool empty_state = (size_t)B * H == 0;
+  if (!empty_tokens) {
+    if (!q || !k || !v || !g || !beta || !o)
+      return fail(GDR_ERR_INVALID_ARG, "null q/k/v/g/beta/o");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
+        !aligned16(o))
+      return fail(GDR_ERR_INVALID_ARG, "q/k/v/g/beta/o must be 16-byte aligned");
+  }
+  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+    return fail(GDR_ERR_INVALID_ARG, "S0/S_T must be 16-byte aligned");
+  if (empty_state) return ok();
+
+  gdr::ChunkArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.S_T = S_T;
+  a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+  a.bf16 = in_dtype == GDR_BF16;
+  a.per_channel = gate == GDR_GATE_PER_CHANNEL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = status_word(&a.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd status word");
+  if (gdr::chunk_tc_supports(a))
+    e = gdr::launch_chunk_tc(a, s);
+  else
+    e = gdr::launch_chunk_simt(a, s);
+  return from_cuda(e, "gdr_chunk_fwd launch");
+}
+
+gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                    const float *g, gdr_gate_kind gate, const float *beta, float *S, void *o,
+                    int N, int H, int dk, int dv, gdr_stream_t stream) {
+  if (N < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "negative N/H");
+  if (in_dtype != GDR_F32 && in_dtype != GDR_BF16)
+    return fail(GDR_ERR_INVALID_ARG, "in_dtype must be GDR_F32 or GDR_BF16");
+  if (gate != GDR_GATE_SCALAR && gate != GDR_GATE_PER_CHANNEL)
+    return fail(GDR_ERR_INVALID_ARG, "unknown gate kind");
+  if (!head_dim_ok(dk) || !head_dim_ok(dv))
+    return fail(GDR_ERR_UNSUPPORTED, "head dims dk=%d dv=%d (need 32, 64 or 128)", dk, dv);
+  if ((size_t)N * H == 0) return ok();
+  if (!q || !k || !v || !g || !beta || !S || !o)
+    return fail(GDR_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
+      !aligned16(S) || !aligned16(o))
+    return fail(GDR_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((size_t)N * H > (size_t)1 << 31) return fail(GDR_ERR_INVALID_ARG, "N*H too large");
+  gdr::StepArgs a;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S = S; a.o = o;
+  a.N = N; a.H = H; a.dk = dk; a.dv = dv;
+  a.bf16 = in_dtype == GDR_BF16;
+  a.per_channel = gate == GDR_GATE_PER_CHANNEL;
+  cudaError_t e = status_word(&a.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_step status word");
+  return from_cuda(gdr::launch_step(a, reinterpret_cast<cudaStream_t>(stream)),
+                   "gdr_step launch");
+}
+
+gdr_status gdr_get_device_status(gdr_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int word = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&word, gdr::g_device_status, sizeof word, 0,
+                                            cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyToSymbolAsync(gdr::g_device_status, &zero, sizeof zero, 0,
+                                cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_get_device_status");
+  if (word & gdr::kStatusTimeout)
+    return fail(GDR_ERR_TIMEOUT, "a kernel gave up a bounded wait (status word 0x%x)", word);
+  return ok();
+}
+
+}  // extern "C"

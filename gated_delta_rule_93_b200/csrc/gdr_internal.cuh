@@ -1,0 +1,62 @@
+// Internal declarations shared by the gated delta-rule CUDA sources.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdr.h"
+
+namespace gdr {
+
+// Kernels OR error bits into a device status word (they never trap).  The
+// word lives in gdr_abi.cu; launchers receive its device address.
+constexpr unsigned int kStatusTimeout = 1u;
+
+struct ChunkArgs {
+  const void *q, *k, *v;
+  const float *g;
+  const float *beta;
+  const float *S0;
+  void *o;
+  float *S_T;
+  int B, T, H, dk, dv;
+  int bf16;          // 1: q, k, v, o are bf16; 0: fp32
+  int per_channel;   // 1: g is [B,T,H,dk]
+  unsigned int *status;  // device status word
+};
+
+struct StepArgs {
+  const void *q, *k, *v;
+  const float *g;
+  const float *beta;
+  float *S;
+  void *o;
+  int N, H, dk, dv;
+  int bf16;
+  int per_channel;
+  unsigned int *status;
+};
+
+// Launchers return cudaSuccess or the launch error.
+cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
+cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
+// Tensor-core (tcgen05) chunked forward; returns cudaErrorNotSupported when
+// the shape is outside what it handles, so the caller can pick another path.
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
+bool chunk_tc_supports(const ChunkArgs &a);
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ float load_in(const void *p, size_t i, int bf16) {
+  if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+  return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ void store_out(void *p, size_t i, float x, int bf16) {
+  if (bf16)
+    reinterpret_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+  else
+    reinterpret_cast<float *>(p)[i] = x;
+}
+
+}  // namespace gdr

@@ -13,7 +13,7 @@ Recipe (every workload, one CPU ``torch.Generator`` per call):
   * beta = sigmoid(N(0, 1)), fp32;
   * S0 = N(0, 0.02^2) fp32 [B,H,d_v,d_k] where the workload has one, else None.
 Draw order: q, k, v, g, beta, S0.  The decode workload draws its initial
-state first, then q, k, v, g, beta of each step in step order.
+state first, then the q, k, v, g, beta stacks of all steps (step-major).
 """
 from __future__ import annotations
 
@@ -89,19 +89,17 @@ def make_step_inputs(N, H, dk, dv, steps, dtype=torch.bfloat16, gate="scalar", s
 
     Returns dict with S0 [N,H,dv,dk] fp32 and per-step stacks q,k [steps,N,H,dk],
     v [steps,N,H,dv], g [steps,N,H] (or [steps,N,H,dk]), beta [steps,N,H].
+    Draw order: S0, then the q, k, v, g, beta stacks (step-major).
     """
     gen = torch.Generator().manual_seed(seed)
     S0 = 0.02 * torch.randn(N, H, dv, dk, generator=gen)
-    qs, ks, vs, gs, bs = [], [], [], [], []
-    gshape = (N, H, dk) if gate == "channel" else (N, H)
-    for _ in range(steps):
-        qs.append(_unit_rows(torch.randn(N, H, dk, generator=gen)).to(dtype))
-        ks.append(_unit_rows(torch.randn(N, H, dk, generator=gen)).to(dtype))
-        vs.append(torch.randn(N, H, dv, generator=gen).to(dtype))
-        gs.append(-0.1 * F.softplus(torch.randn(*gshape, generator=gen)))
-        bs.append(torch.sigmoid(torch.randn(N, H, generator=gen)))
-    return dict(S0=S0.float(), q=torch.stack(qs), k=torch.stack(ks), v=torch.stack(vs),
-                g=torch.stack(gs).float(), beta=torch.stack(bs).float())
+    q = _unit_rows(torch.randn(steps, N, H, dk, generator=gen)).to(dtype)
+    k = _unit_rows(torch.randn(steps, N, H, dk, generator=gen)).to(dtype)
+    v = torch.randn(steps, N, H, dv, generator=gen).to(dtype)
+    gshape = (steps, N, H, dk) if gate == "channel" else (steps, N, H)
+    g = -0.1 * F.softplus(torch.randn(*gshape, generator=gen))
+    beta = torch.sigmoid(torch.randn(steps, N, H, generator=gen))
+    return dict(S0=S0.float(), q=q, k=k, v=v, g=g.float(), beta=beta.float())
 
 
 def make_workload_inputs(w: Workload, seed=0, steps=None):

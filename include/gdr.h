@@ -1,0 +1,142 @@
+/*
+ * gdr.h -- C ABI of the gated delta-rule sequence mixer for NVIDIA B200
+ * (sm_100a).
+ *
+ * The mixer keeps a matrix state S (d_v x d_k, row i = value channel,
+ * column j = key channel) and, for every token t,
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t
+ *
+ * Sources:
+ *   "Decoding Hybrid Linear Attention Architectures", section 3 (state
+ *   update equations: item 3 Gated Delta Rule with a scalar gate, item 6
+ *   Gated Delta Attention with a per-channel gate and the decay -> erase ->
+ *   write pseudocode), section 4 (the two gates), section 5 (chunkwise
+ *   algorithm: inter-chunk state recursion, intra-chunk output, gates
+ *   accumulated in log space) and section 6 (constant-cost decode step);
+ *   "Linear Attention Variants (RetNet, GLA, DeltaNet, Based)", section
+ *   "DeltaNet: Error-Correcting Writes" (the delta rule and its WY-based
+ *   chunked parallel form).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every pointer is a CUDA device pointer owned by the caller.  The library
+ *   allocates no device memory in any call and keeps no per-call state.
+ * - All device work is enqueued on `stream` (a cudaStream_t; NULL means the
+ *   legacy default stream) and runs asynchronously.
+ * - Argument errors are detected on the host, before anything is enqueued:
+ *   the call returns GDR_ERR_INVALID_ARG or GDR_ERR_UNSUPPORTED and launches
+ *   nothing; gdr_last_error_message() then describes the problem.
+ * - A kernel that gives up a bounded wait records GDR_ERR_TIMEOUT in a
+ *   device status word; gdr_get_device_status() reads and clears it.
+ * - Gate: `g` holds log(alpha) in fp32 (finite, <= 0).  A scalar gate has one
+ *   value per (token, head); a per-channel gate has d_k values.
+ * - Dtypes: q, k, v and o share `in_dtype` (fp32 or bf16); g, beta and the
+ *   state are always fp32.  All arithmetic accumulates in fp32.
+ * - No query scale is applied: o_t = S_t q_t exactly as written above.
+ * - Supported head sizes: d_k, d_v in {32, 64, 128}.  Chunk size C = 64.
+ * - Pointers must be 16-byte aligned; every tensor is dense row-major
+ *   (contiguous) in the layout given below.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDR_OK = 0,
+  GDR_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad enum   */
+  GDR_ERR_UNSUPPORTED = 2, /* valid request this build does not implement   */
+  GDR_ERR_WORKSPACE = 3,   /* workspace pointer/size too small              */
+  GDR_ERR_CUDA = 4,        /* a CUDA runtime call failed                    */
+  GDR_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (device word) */
+} gdr_status;
+
+typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+typedef enum { GDR_GATE_SCALAR = 0, GDR_GATE_PER_CHANNEL = 1 } gdr_gate_kind;
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *gdr_stream_t;
+
+/*
+ * Workspace the chunked forward needs for this problem, in bytes (0 if none).
+ * Pass at least this much (16-byte aligned) to gdr_chunk_fwd.
+ */
+size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int C,
+                                     gdr_dtype in_dtype, gdr_gate_kind gate);
+
+/*
+ * Chunkwise-parallel forward over whole sequences (prefill / training
+ * forward).  Source: "Decoding Hybrid Linear Attention Architectures",
+ * section 5; the per-token result it reproduces is the recurrence above.
+ *
+ *   q, k  [B, T, H, dk]  in_dtype      queries / keys (the caller normalises)
+ *   v     [B, T, H, dv]  in_dtype      values
+ *   g     [B, T, H]      fp32          log alpha, scalar gate, or
+ *         [B, T, H, dk]  fp32          log alpha, per-channel gate
+ *   beta  [B, T, H]      fp32          write strength in [0, 1]
+ *   S0    [B, H, dv, dk] fp32 or NULL  initial state (NULL = zero state)
+ *   o     [B, T, H, dv]  in_dtype      output (written)
+ *   S_T   [B, H, dv, dk] fp32 or NULL  final state (written if not NULL)
+ *   C     chunk length; must be 64
+ *   workspace, ws_bytes: see gdr_chunk_fwd_workspace_bytes (may be NULL/0
+ *         when that returns 0)
+ *
+ * T may be any value >= 0 (a ragged last chunk is masked); B*H may be 0.
+ * S0 may alias S_T (each (b, h) reads all of S0 before writing S_T); o must
+ * not alias any input.  Per-channel gates must keep the decay accumulated
+ * over one chunk within about 80 (|sum of g| per channel) so that the
+ * intermediate exp(-sum g) stays finite in fp32; scalar gates have no limit.
+ */
+gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                         const float *g, gdr_gate_kind gate, const float *beta,
+                         const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
+                         int dv, int C, void *workspace, size_t ws_bytes,
+                         gdr_stream_t stream);
+
+/*
+ * One recurrent decode step for N independent states, S updated in place.
+ * Source: "Decoding Hybrid Linear Attention Architectures", section 6
+ * (constant-cost update of the fixed-size state per decoded token) with the
+ * step order of section 3 item 6.
+ *
+ *   q, k  [N, H, dk]     in_dtype
+ *   v     [N, H, dv]     in_dtype
+ *   g     [N, H] or [N, H, dk]  fp32   log alpha (scalar / per-channel gate)
+ *   beta  [N, H]         fp32
+ *   S     [N, H, dv, dk] fp32          state, read and overwritten
+ *   o     [N, H, dv]     in_dtype      output (written)
+ *
+ * o must not alias S or any input.
+ */
+gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                    const float *g, gdr_gate_kind gate, const float *beta, float *S, void *o,
+                    int N, int H, int dk, int dv, gdr_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word.
+ * Returns GDR_OK, GDR_ERR_TIMEOUT (a kernel gave up a bounded wait since the
+ * last call) or GDR_ERR_CUDA (the synchronisation itself failed).
+ */
+gdr_status gdr_get_device_status(gdr_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *gdr_status_string(gdr_status s);
+
+/* Detail of the last error returned on this host thread ("" if none). */
+const char *gdr_last_error_message(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

@@ -1,0 +1,104 @@
+"""Host-side checks of the C-ABI library (no GPU, no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_93_b200 import binding
+from gated_delta_rule_93_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return binding.lib()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"\b(gdr_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert "gdr_chunk_fwd" in declared and "gdr_step" in declared
+    for name in declared:
+        assert hasattr(L, name), f"{name} declared in include/ but not exported"
+    assert set(binding.EXPORTS) <= set(declared)
+
+
+def test_no_driver_dependency(L):
+    """The library links the CUDA runtime statically and needs no libcuda at
+    load time (it loads on this GPU-less host)."""
+    assert L.gdr_version() == 100
+
+
+def test_status_strings(L):
+    for code, name in enumerate(["GDR_OK", "GDR_ERR_INVALID_ARG", "GDR_ERR_UNSUPPORTED",
+                                 "GDR_ERR_WORKSPACE", "GDR_ERR_CUDA", "GDR_ERR_TIMEOUT"]):
+        assert binding.status_string(code) == name
+
+
+def test_workspace_query(L):
+    assert L.gdr_chunk_fwd_workspace_bytes(8, 4096, 16, 128, 128, 64, 1, 0) == 0
+
+
+def _fake_ptr(off=0):
+    return ctypes.c_void_p(0x10000 + off)
+
+
+def test_validation_rejects_before_any_launch(L):
+    p = _fake_ptr()
+    args = lambda **kw: dict(dict(q=p, k=p, v=p, dt=1, g=p, gate=0, beta=p, S0=None, o=p,
+                                  ST=None, B=1, T=64, H=1, dk=128, dv=128, C=64, ws=None,
+                                  wsb=0, st=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return L.gdr_chunk_fwd(a["q"], a["k"], a["v"], a["dt"], a["g"], a["gate"], a["beta"],
+                               a["S0"], a["o"], a["ST"], a["B"], a["T"], a["H"], a["dk"],
+                               a["dv"], a["C"], a["ws"], a["wsb"], a["st"])
+
+    assert call(C=32) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dk=48) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dv=256) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dt=7) == binding.GDR_ERR_INVALID_ARG
+    assert call(gate=3) == binding.GDR_ERR_INVALID_ARG
+    assert call(B=-1) == binding.GDR_ERR_INVALID_ARG
+    assert call(q=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(o=_fake_ptr(4)) == binding.GDR_ERR_INVALID_ARG
+    assert "aligned" in L.gdr_last_error_message().decode()
+    assert call(S0=_fake_ptr(8)) == binding.GDR_ERR_INVALID_ARG
+    # empty problems succeed without touching the device
+    assert call(B=0) == binding.GDR_OK
+    assert call(H=0) == binding.GDR_OK
+
+    def step(**kw):
+        d = dict(q=p, k=p, v=p, dt=1, g=p, gate=0, beta=p, S=p, o=p, N=4, H=2, dk=128, dv=128,
+                 st=None)
+        d.update(kw)
+        return L.gdr_step(d["q"], d["k"], d["v"], d["dt"], d["g"], d["gate"], d["beta"],
+                          d["S"], d["o"], d["N"], d["H"], d["dk"], d["dv"], d["st"])
+
+    assert step(dk=100) == binding.GDR_ERR_UNSUPPORTED
+    assert step(S=None) == binding.GDR_ERR_INVALID_ARG
+    assert step(S=_fake_ptr(4)) == binding.GDR_ERR_INVALID_ARG
+    assert step(N=-2) == binding.GDR_ERR_INVALID_ARG
+    assert step(N=0) == binding.GDR_OK
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+
+    x = torch.zeros(1, 64, 1, 32)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.chunk_fwd(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1))
