@@ -31,6 +31,7 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 from gated_delta_rule_93_b200.inputs import WORKLOADS, make_workload_inputs  # noqa: E402
+from gated_delta_rule_93_b200.sharding import max_over_ranks  # noqa: E402
 
 METRIC = "tokens/s and TFLOP/s per gated-delta layer fwd (1 B200), % of roofline"
 DEFAULT_WORKLOAD = "gdn_b8_t4096_h16_d128"
@@ -233,10 +234,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1)
 
     # ---- max over ranks
-    if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, e2e_ms = t.tolist()
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
 
     if rank != 0:
         return None
