@@ -46,6 +46,9 @@ def algorithmic_bytes(w):
     """HBM bytes a perfect fused kernel must move for one step (per GPU)."""
     e_in = 2 if w.dtype == torch.bfloat16 else 4
     gate_elems = w.dk if w.gate == "channel" else 1
+    if w.kind == "step":  # one decode step: S read + written once, q/k/v/g/beta in, o out
+        return w.B * w.H * (8 * w.dk * w.dv + (2 * w.dk + w.dv) * e_in + w.dv * e_in
+                            + 4 * gate_elems + 4)
     per_tok = (2 * w.dk + w.dv) * e_in + w.dv * e_in + 4 * gate_elems + 4
     state = 4 * w.dk * w.dv * w.B * w.H
     return w.B * w.T * w.H * per_tok + state * (int(w.with_S0) + int(w.want_S_T))
@@ -53,7 +56,10 @@ def algorithmic_bytes(w):
 
 def algorithmic_flops(w, C=64):
     """Chunked-method flops per step, counting masked products as triangles:
-    6 d_k d_v + C (3 d_k + 2 d_v) + C^2 / 3 per token-head."""
+    6 d_k d_v + C (3 d_k + 2 d_v) + C^2 / 3 per token-head (decode step:
+    about 7 d_k d_v per state, CUDA cores)."""
+    if w.kind == "step":
+        return w.B * w.H * 7.0 * w.dk * w.dv
     per = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0
     return w.B * w.T * w.H * per
 
@@ -152,21 +158,35 @@ def run_ours(args, rank, world, local_rank):
     from gated_delta_rule_93_b200 import binding
 
     w = WORKLOADS[args.workload]
-    if w.kind != "chunk":
-        raise SystemExit("bench.py times the chunked forward; the decode workload is a "
-                         "parity case")
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    host = make_workload_inputs(w, seed=rank)
-    d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
-    o = torch.empty(w.B, w.T, w.H, w.dv, dtype=w.dtype, device=dev)
-    S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev) if w.want_S_T \
-        else None
     stream = torch.cuda.current_stream(dev)
+    if w.kind == "step":
+        # decode: one gdr_step over all N x H states per step, inputs of the
+        # first (warmup + steps) steps resident, the state updated in place
+        nsteps = args.warmup + args.steps + 3
+        host = make_workload_inputs(w, seed=rank, steps=nsteps)
+        d = {k: v.to(dev) for k, v in host.items()}
+        S = d["S0"].clone()
+        o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
+        it = [0]
 
-    def step():
-        binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o, S_T=S_T,
-                          output_final_state=S_T is not None)
+        def step():
+            i = it[0] % nsteps
+            it[0] += 1
+            binding.step(d["q"][i], d["k"][i], d["v"][i], d["g"][i], d["beta"][i], S, o=o)
+
+        S_T = None
+    else:
+        host = make_workload_inputs(w, seed=rank)
+        d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
+        o = torch.empty(w.B, w.T, w.H, w.dv, dtype=w.dtype, device=dev)
+        S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev) \
+            if w.want_S_T else None
+
+        def step():
+            binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o,
+                              S_T=S_T, output_final_state=S_T is not None)
 
     def barrier():
         if world > 1:
@@ -204,7 +224,14 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device status word set during the timed region")
 
     # ---- end to end through the same API with host buffers (pinned)
-    pin = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+    if w.kind == "step":
+        # per step: that step's q, k, v, g, beta go host -> device, o comes back;
+        # the state stays resident (it is the decoder's cache)
+        pin = {k: host[k][0].pin_memory() for k in ("q", "k", "v", "g", "beta")}
+        dev_in = {k: torch.empty_like(v, device=dev) for k, v in pin.items()}
+    else:
+        pin = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+        dev_in = d
     o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     S_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory() if S_T is not None else None
     h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
@@ -213,8 +240,12 @@ def run_ours(args, rank, world, local_rank):
     def e2e_step():
         for kk, v in pin.items():
             if v is not None:
-                d[kk].copy_(v, non_blocking=True)
-        step()
+                dev_in[kk].copy_(v, non_blocking=True)
+        if w.kind == "step":
+            binding.step(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"], dev_in["beta"], S,
+                         o=o)
+        else:
+            step()
         o_h.copy_(o, non_blocking=True)
         if S_h is not None:
             S_h.copy_(S_T, non_blocking=True)
@@ -239,7 +270,7 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return None
     ms_step = total_ms / args.steps
-    tokens_step = w.tokens
+    tokens_step = w.B * w.T if w.kind == "chunk" else w.B  # tokens one step processes
     value = world * tokens_step * args.steps / (total_ms / 1e3)
     hbm_peak, tc_peak, peak_kind = measured_peaks()
     abytes = algorithmic_bytes(w)
@@ -261,9 +292,10 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
         "data": "synthetic (seeded; q,k L2-normalised N(0,1), v N(0,1), "
                 "beta=sigmoid(N(0,1)), log alpha=-0.1 softplus(N(0,1)))",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+        "config": {"workload": w.name, "B": w.B, "T": w.T if w.kind == "chunk" else 1,
+                   "H": w.H, "d_k": w.dk, "d_v": w.dv,
                    "chunk": w.C, "gate": w.gate, "S0": w.with_S0, "S_T": w.want_S_T,
-                   "global_batch": w.B * world, "seq_len": w.T,
+                   "global_batch": w.B * world, "seq_len": w.T if w.kind == "chunk" else 1,
                    "parallelism": f"independent (b,h) shards x{world}",
                    "l2": "inputs exceed L2 (%.0f MB > 126 MB); no flush" %
                          (algorithmic_bytes(w) / 1e6)},
@@ -273,14 +305,14 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
-                     "kernel": "gdr_chunk_fwd"},
+                     "kernel": "gdr_chunk_fwd" if w.kind == "chunk" else "gdr_step"},
         "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": args.steps,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.kind == "chunk":
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return line
 
