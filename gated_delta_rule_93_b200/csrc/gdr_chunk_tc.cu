@@ -15,10 +15,9 @@
 //   Y    = (I + A)^{-1}  (16x16 diagonal blocks by forward substitution,
 //                          off-diagonal blocks with mma.sync TF32)
 //   T    = Y Diag(beta),  T' = T Diag(e^{gc})            -> bf16, smem
-//   Q~   = Diag(e^{gc}) Q                                -> in place, smem
 //   U^T  = V^T T^T,  W^T = K^T T'^T        (tcgen05, M=128 N=64 K=64)
 //   V'^T = U^T + S_b (-W)^T                (tcgen05, A = S_b from TMEM)
-//   O^T  = S_b Q~^T + V'^T P^T             (tcgen05, one accumulator)
+//   O^T  = (S_b Q^T) Diag(e^{gc}) + V'^T P^T   (tcgen05, two accumulators)
 //   S    = e^{gc_last} S + (V'^T Diag(e^{gc_last - gc})) K   (fp32 TMEM acc)
 //
 // S_b is the bf16 copy of the fp32 state, kept in TMEM as the A operand.
@@ -26,10 +25,10 @@
 // decay keeps e^{-gc} finite, else pairwise, so no scalar gate overflows.
 //
 // Warp roles (one CTA per (b, h), 320 threads):
-//   warps 0-3  "state" group: V'^T -> bf16 operands, O epilogue + TMA store,
+//   warps 0-3  "state" group: V'^T -> bf16 operands, O epilogue (direct stores),
 //              S -> S_b and the per-chunk state decay (TMEM lanes 0-127);
 //   warps 4-7  "prep" group, one chunk ahead: gate cumsum, A/P epilogue,
-//              (I + A)^{-1}, T/T', Q~, W^T -> bf16 operand;
+//              (I + A)^{-1}, T/T', W^T -> bf16 operand;
 //   warp 8     TMA producer (two input stages, no multicast) + g/beta loads;
 //   warp 9     MMA issuer (one thread).
 // Hand-offs are mbarriers; every wait is bounded (time-out -> device status
@@ -47,12 +46,18 @@ namespace {
 using namespace sm100;
 
 constexpr int C = 64, DK = 128, DV = 128;
-constexpr int kThreads = 320;
+constexpr int kPrepWarps = 4;
+constexpr int kPrepThreads = 32 * kPrepWarps;
+constexpr int kThreads = 320;  // 4 state + 4 prep + producer + MMA warps
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kStages = 2;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr uint32_t kTileBytes = 64 * 128;    // one 64 x 64 bf16 tile
 constexpr uint32_t kStageTx = 6 * kTileBytes;
 constexpr float kSafeDecay = 80.f;  // e^{80} is finite in fp32
+// Row stride (floats) of the fp32 A/Y matrix: rows stay 16-byte aligned, and
+// mma.sync A-fragment loads hit distinct banks.
+constexpr int LDA = 68;
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
 struct Lay {
@@ -62,13 +67,14 @@ struct Lay {
   static constexpr uint32_t TP = T + kTileBytes;                // T'  K-major [r][s]
   static constexpr uint32_t P = TP + kTileBytes;                // P   K-major [r][s], x2
   static constexpr uint32_t WT = P + 2 * kTileBytes;            // -W^T MN-major [dk][C]
-  static constexpr uint32_t VP = WT + 2 * kTileBytes;           // V'^T K-major [dv][C]; O staging
+  static constexpr uint32_t VP = WT + 2 * kTileBytes;           // V'^T K-major [dv][C]
   static constexpr uint32_t VPD = VP + 2 * kTileBytes;          // decayed V'^T
-  static constexpr uint32_t AF = VPD + 2 * kTileBytes;          // fp32 A/Y [64][65]
-  static constexpr uint32_t R = AF + 64 * 65 * 4;               // fp32 [16][49]
-  static constexpr uint32_t GS = R + 16 * 49 * 4;               // per stage g[64], beta[64]
+  static constexpr uint32_t AF = VPD + 2 * kTileBytes;          // fp32 A, then Y [64][LDA]
+  static constexpr uint32_t SCR = AF + 64 * LDA * 4;            // fp32 inverse scratch 4 x [16][8]
+  static constexpr uint32_t GS = SCR + 4 * 128 * 4;             // per stage g[64], beta[64]
   static constexpr uint32_t VEC = GS + kStages * 512;           // x3: gc, eg, ieg, egl [64] each
-  static constexpr uint32_t BAR = VEC + 3 * 1024;               // mbarriers
+  static constexpr uint32_t SVEC = VEC + 3 * 1024;              // x2: eg, egl [64] (state group)
+  static constexpr uint32_t BAR = SVEC + 2 * 512;               // mbarriers
   static constexpr uint32_t MISC = BAR + 16 * 8;                // tmem base, abort flag, consumed
   static constexpr uint32_t END = MISC + 16;
 };
@@ -81,20 +87,22 @@ enum {
   B_FULL = 0,   // [2] TMA + g/beta of a stage landed          (count 1 + tx)
   B_EMPTY = 2,  // [2] stage may be refilled: MMA commit + prep  (count 2)
   B_D1F = 4,    // D1 written                                   (commit)
-  B_D1E,        // D1 read by the prep group                    (128)
-  B_TRDY,       // T, T', Q~, P, gate vectors of a chunk ready  (128)
+  B_D1E,        // D1 read by the prep group                    (256)
+  B_TRDY,       // T, T', P, gate vectors of a chunk ready      (256)
   B_WTF,        // U^T, W^T written                             (commit)
-  B_WTB,        // -W^T bf16 operand written                    (128)
+  B_WTB,        // -W^T bf16 operand written                    (256)
   B_SBR,        // S_b in TMEM and the decayed S ready          (128)
   B_VPF,        // V'^T and O_a written                         (commit)
   B_VPR,        // V'^T bf16 operands written                   (128)
-  B_OF,         // O and the updated S written                  (commit)
+  B_SF,         // the updated S written                        (commit)
+  B_OF,         // O_a and O_b written                          (commit)
   B_FIN,        // final drain of the MMA pipe                  (commit)
   B_COUNT
 };
 
 // TMEM column map (512 allocated; 1 CTA per SM).
-constexpr uint32_t TM_S = 0, TM_SB = 128, TM_D1 = 192, TM_UV = 256, TM_WT = 320, TM_O = 384;
+constexpr uint32_t TM_S = 0, TM_SB = 128, TM_D1 = 192, TM_UV = 256, TM_WT = 320, TM_O = 384,
+                   TM_OA = 448;
 
 constexpr uint32_t ID_D1 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t ID_U = idesc_bf16(128, 64, 1, 0);
@@ -133,6 +141,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   }
 }
 
+// 64 consecutive TMEM columns of this thread's lane: four loads, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  float a0[16], a1[16], a2[16], a3[16];
+  tmem_ld16(taddr, a0);
+  tmem_ld16(taddr + 16, a1);
+  tmem_ld16(taddr + 32, a2);
+  tmem_ld16(taddr + 48, a3);
+  tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    v[e] = a0[e];
+    v[16 + e] = a1[e];
+    v[32 + e] = a2[e];
+    v[48 + e] = a3[e];
+  }
+}
+
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -153,26 +178,35 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// Barrier over one 128-thread group that also ORs a predicate.
+// Warp-group barriers: id 2 = state group (128 threads), id 3 = prep group
+// (kPrepThreads).
+__device__ __forceinline__ uint32_t group_threads(uint32_t bar_id) {
+  return bar_id == 3 ? (uint32_t)kPrepThreads : 128u;
+}
+
+// Barrier over one warp group that also ORs a predicate.
 __device__ __forceinline__ bool group_any(uint32_t bar_id, bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred), "r"(bar_id)
+      : "r"((uint32_t)pred), "r"(bar_id), "r"(group_threads(bar_id))
       : "memory");
   return r != 0;
 }
 
-__device__ __forceinline__ void group_bar(uint32_t bar_id) { named_bar_sync(bar_id, 128); }
+__device__ __forceinline__ void group_bar(uint32_t bar_id) {
+  named_bar_sync(bar_id, group_threads(bar_id));
+}
 
 // Bounded wait that also gives up as soon as another role has aborted.
+// The thread sleeps inside try_wait (suspend hint) between checks.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
                                               volatile int *abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, 20000)) {
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitNs) {
       *abort_flag = 1;
@@ -180,6 +214,16 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
     }
   }
   return true;
+}
+
+// Group-wide wait: lane 0 of each warp polls, the warp shares its result,
+// and the group agrees (any failure -> every thread sees failure).
+__device__ __forceinline__ bool group_wait(uint32_t bar_id, uint64_t *bar, uint32_t parity,
+                                           volatile int *abort_flag, int lane) {
+  bool ok = true;
+  if (lane == 0) ok = wait_or_abort(bar, parity, abort_flag);
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return !group_any(bar_id, !ok);
 }
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
@@ -198,11 +242,21 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// (I + A)^{-1} in place for a strictly lower 64x64 fp32 matrix (row stride
-// 65) with one 128-thread group (local thread id t, warp w = t / 32):
-// diagonal 16x16 blocks by forward substitution (warp w owns block w), then
-// for block rows b = 1..3: R_b = sum_{k<b} A_bk Y_k and Y_b = -D_bb R_b,
-// 8-column tiles on mma.sync (TF32 operands rounded to nearest).
+// (I + A)^{-1} in place for a strictly lower 64x64 fp32 matrix A (row stride
+// LDA, zero on and above the diagonal) with the 4-warp prep group (local
+// thread t, warp w = t / 32), in 16x16 blocks:
+//  1. diagonal blocks D_bb = (I + A_bb)^{-1} by forward substitution (warp b);
+//  2. every 8-column strip of a column block j is independent:
+//       Y_jj = D_jj,   Y_bj = -D_bb sum_{k=j}^{b-1} A_bk Y_kj   (b > j),
+//     so each warp sweeps its strips down the block rows with mma.sync
+//     (TF32 operands rounded to nearest, fp32 accumulation), keeping the
+//     strip's finished blocks in registers and re-laying accumulator
+//     fragments as B fragments through a warp-private scratch;
+//  3. after a group barrier the off-diagonal blocks overwrite A.
+// Strips (column block j, half hf): warp 0 -> (0,0); warp 1 -> (0,1);
+// warp 2 -> (1,0), (2,0); warp 3 -> (1,1), (2,1).  (The measured in-kernel
+// time of this form beat an fp32 CUDA-core strip sweep, although mma.sync
+// queues behind concurrent tcgen05 work.)
 __device__ void invert_unit_lower(float *AF, float *R, int t, uint32_t bar_id) {
   const int warp = t >> 5, lane = t & 31;
   {
@@ -210,69 +264,132 @@ __device__ void invert_unit_lower(float *AF, float *R, int t, uint32_t bar_id) {
     float x[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
-    const float *Ab = AF + (16 * w) * 65 + 16 * w;
+    const float *Ab = AF + (16 * w) * LDA + 16 * w;
 #pragma unroll
     for (int i = 1; i < 16; ++i) {
       float acc = 0.f;
 #pragma unroll
-      for (int k = 0; k < i; ++k) acc += Ab[i * 65 + k] * x[k];
+      for (int k4 = 0; k4 < (i + 3) / 4; ++k4) {
+        const float4 av = *reinterpret_cast<const float4 *>(Ab + i * LDA + 4 * k4);
+        if (4 * k4 + 0 < i) acc += av.x * x[4 * k4 + 0];
+        if (4 * k4 + 1 < i) acc += av.y * x[4 * k4 + 1];
+        if (4 * k4 + 2 < i) acc += av.z * x[4 * k4 + 2];
+        if (4 * k4 + 3 < i) acc += av.w * x[4 * k4 + 3];
+      }
       if (i > c) x[i] = -acc;
     }
     __syncwarp();
     if (lane < 16) {
-      float *Yb = AF + (16 * w) * 65 + 16 * w;
+      float *Yb = AF + (16 * w) * LDA + 16 * w;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) Yb[i * 65 + c] = x[i];
+      for (int i = 0; i < 16; ++i) Yb[i * LDA + c] = x[i];
     }
   }
   group_bar(bar_id);
   const int g = lane >> 2, tq = lane & 3;
+  float *scr = R + warp * 128;  // [16][8] per warp
+  // accumulator fragment (16x8) -> B fragments of two k-steps (rows 0-7, 8-15)
+  auto to_bfrag = [&](const float (&cf)[4], uint32_t (&bf)[2][2]) {
+    scr[g * 8 + 2 * tq] = cf[0];
+    scr[g * 8 + 2 * tq + 1] = cf[1];
+    scr[(g + 8) * 8 + 2 * tq] = cf[2];
+    scr[(g + 8) * 8 + 2 * tq + 1] = cf[3];
+    __syncwarp();
 #pragma unroll
-  for (int b = 1; b < 4; ++b) {
-    const int ntiles = 2 * b;
-    for (int nt = warp; nt < ntiles; nt += 4) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int k = nt >> 1; k < b; ++k) {
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const int col = 16 * k + 8 * ks;
-          uint32_t af[4], bf[2];
-          af[0] = to_tf32(AF[(16 * b + g) * 65 + col + tq]);
-          af[1] = to_tf32(AF[(16 * b + g + 8) * 65 + col + tq]);
-          af[2] = to_tf32(AF[(16 * b + g) * 65 + col + tq + 4]);
-          af[3] = to_tf32(AF[(16 * b + g + 8) * 65 + col + tq + 4]);
-          bf[0] = to_tf32(AF[(col + tq) * 65 + 8 * nt + g]);
-          bf[1] = to_tf32(AF[(col + tq + 4) * 65 + 8 * nt + g]);
-          mma_tf32_16x8x8(acc, af, bf);
-        }
-      }
-      R[g * 49 + 8 * nt + 2 * tq] = acc[0];
-      R[g * 49 + 8 * nt + 2 * tq + 1] = acc[1];
-      R[(g + 8) * 49 + 8 * nt + 2 * tq] = acc[2];
-      R[(g + 8) * 49 + 8 * nt + 2 * tq + 1] = acc[3];
+    for (int ks = 0; ks < 2; ++ks) {
+      bf[ks][0] = to_tf32(scr[(8 * ks + tq) * 8 + g]);
+      bf[ks][1] = to_tf32(scr[(8 * ks + tq + 4) * 8 + g]);
     }
-    group_bar(bar_id);
-    for (int nt = warp; nt < ntiles; nt += 4) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    __syncwarp();
+  };
+  auto afrag = [&](int row0, int col0, uint32_t (&af)[4]) {
+    af[0] = to_tf32(AF[(row0 + g) * LDA + col0 + tq]);
+    af[1] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq]);
+    af[2] = to_tf32(AF[(row0 + g) * LDA + col0 + tq + 4]);
+    af[3] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq + 4]);
+  };
+  float yout[2][4][4];  // finished blocks: [strip slot][block row]
+  const int nstrip = warp < 2 ? 1 : 2;
+#pragma unroll
+  for (int si = 0; si < 2; ++si) {
+    if (si >= nstrip) break;
+    const int j = warp < 2 ? 0 : 1 + si, hf = warp & 1;
+    const int col = 16 * j + 8 * hf;  // first column of the strip
+    uint32_t yb[4][2][2];             // B fragments of Y_kj
+#pragma unroll
+    for (int jj = 0; jj < 3; ++jj) {  // Y_jj strip = D_jj (static indices only)
+      if (jj != j) continue;
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
-        const int col = 16 * b + 8 * ks;
-        uint32_t af[4], bf[2];
-        af[0] = to_tf32(AF[(16 * b + g) * 65 + col + tq]);
-        af[1] = to_tf32(AF[(16 * b + g + 8) * 65 + col + tq]);
-        af[2] = to_tf32(AF[(16 * b + g) * 65 + col + tq + 4]);
-        af[3] = to_tf32(AF[(16 * b + g + 8) * 65 + col + tq + 4]);
-        bf[0] = to_tf32(R[(8 * ks + tq) * 49 + 8 * nt + g]);
-        bf[1] = to_tf32(R[(8 * ks + tq + 4) * 49 + 8 * nt + g]);
-        mma_tf32_16x8x8(acc, af, bf);
+        yb[jj][ks][0] = to_tf32(AF[(16 * jj + 8 * ks + tq) * LDA + col + g]);
+        yb[jj][ks][1] = to_tf32(AF[(16 * jj + 8 * ks + tq + 4) * LDA + col + g]);
       }
-      AF[(16 * b + g) * 65 + 8 * nt + 2 * tq] = -acc[0];
-      AF[(16 * b + g) * 65 + 8 * nt + 2 * tq + 1] = -acc[1];
-      AF[(16 * b + g + 8) * 65 + 8 * nt + 2 * tq] = -acc[2];
-      AF[(16 * b + g + 8) * 65 + 8 * nt + 2 * tq + 1] = -acc[3];
     }
-    group_bar(bar_id);
+#pragma unroll
+    for (int bb = 1; bb < 4; ++bb) {
+      if (bb <= j) continue;
+      float racc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        if (k < j || k >= bb) continue;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          uint32_t af[4];
+          afrag(16 * bb, 16 * k + 8 * ks, af);
+          mma_tf32_16x8x8(racc, af, yb[k][ks]);
+        }
+      }
+      uint32_t rb[2][2];
+      to_bfrag(racc, rb);
+      float yacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        uint32_t af[4];
+        afrag(16 * bb, 16 * bb + 8 * ks, af);
+        mma_tf32_16x8x8(yacc, af, rb[ks]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        yacc[e] = -yacc[e];
+        yout[si][bb][e] = yacc[e];
+      }
+      if (bb < 3) to_bfrag(yacc, yb[bb]);
+    }
   }
+  group_bar(bar_id);  // every read of A is done: store the off-diagonal blocks
+#pragma unroll
+  for (int si = 0; si < 2; ++si) {
+    if (si >= nstrip) break;
+    const int j = warp < 2 ? 0 : 1 + si, hf = warp & 1;
+    const int col = 16 * j + 8 * hf;
+#pragma unroll
+    for (int bb = 1; bb < 4; ++bb) {
+      if (bb <= j) continue;
+      AF[(16 * bb + g) * LDA + col + 2 * tq] = yout[si][bb][0];
+      AF[(16 * bb + g) * LDA + col + 2 * tq + 1] = yout[si][bb][1];
+      AF[(16 * bb + g + 8) * LDA + col + 2 * tq] = yout[si][bb][2];
+      AF[(16 * bb + g + 8) * LDA + col + 2 * tq + 1] = yout[si][bb][3];
+    }
+  }
+  group_bar(bar_id);
+}
+
+// One warp: cumulative log decay of a chunk (g[64] -> gc[64] in log space,
+// inclusive prefix sum) held as lanes r and r + 32; returns the chunk total.
+__device__ __forceinline__ float chunk_cumsum(const float *g, int lane, float &x0, float &x1) {
+  x0 = g[lane];
+  x1 = g[lane + 32];
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+    const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+    if (lane >= off) {
+      x0 += y0;
+      x1 += y1;
+    }
+  }
+  x1 += __shfl_sync(0xffffffffu, x0, 31);
+  return __shfl_sync(0xffffffffu, x1, 31);
 }
 
 #ifdef GDR_TC_DEBUG
@@ -290,13 +407,12 @@ __device__ int g_dbg_chunk = 0;
   } while (0)
 #endif
 
-// 10 warps leave three warps on some SM sub-partitions, whose register file
-// is a quarter of the SM's: the launch bound caps registers accordingly.
+// Each SM sub-partition holds a quarter of the register file and up to three
+// of the block's ten warps: the launch bound caps registers at 168.
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV,
-                        const __grid_constant__ CUtensorMap tmO, ChunkArgs a) {
+                        const __grid_constant__ CUtensorMap tmV, ChunkArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~uintptr_t(1023));
@@ -310,7 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lay::MISC + 4);
   volatile int *consumed = reinterpret_cast<volatile int *>(sm + Lay::MISC + 8);
   float *AF = reinterpret_cast<float *>(sm + Lay::AF);
-  float *Rs = reinterpret_cast<float *>(sm + Lay::R);
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -318,13 +433,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[B_EMPTY + s], 2);
     }
     mbar_init(&bars[B_D1F], 1);
-    mbar_init(&bars[B_D1E], 128);
-    mbar_init(&bars[B_TRDY], 128);
+    mbar_init(&bars[B_D1E], kPrepThreads);
+    mbar_init(&bars[B_TRDY], kPrepThreads);
     mbar_init(&bars[B_WTF], 1);
-    mbar_init(&bars[B_WTB], 128);
+    mbar_init(&bars[B_WTB], kPrepThreads);
     mbar_init(&bars[B_SBR], 128);
     mbar_init(&bars[B_VPF], 1);
     mbar_init(&bars[B_VPR], 128);
+    mbar_init(&bars[B_SF], 1);
     mbar_init(&bars[B_OF], 1);
     mbar_init(&bars[B_FIN], 1);
     *abort_flag = 0;
@@ -341,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tm = *tmem_slot;
   const uint32_t lane_base = tm + ((uint32_t)((warp & 3) * 32) << 16);
 
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ================================================================ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -385,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = *consumed; c < issued; ++c)
         mbar_wait_bounded(&bars[B_FULL + (c & 1)], (c >> 1) & 1, kWaitNs);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_v = smem_u32(sm + Lay::V);
@@ -425,41 +541,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_d1(0);
         if (!(ok = W(B_TRDY, 0))) break;
         issue_uw(0);
-        // Each barrier below completes once per chunk and is waited on by
-        // parity, so no producer may run two phases ahead of a waiter.  D1 of
-        // chunk c+1 is issued only after S_b of chunk c is ready, i.e. after
-        // the state group has consumed the gate vectors of chunk c; this
-        // bounds the prep group's lead to one chunk.
+        if (n > 1) {
+          if (!(ok = W(B_D1E, 0) && W(B_FULL + 1, 0))) break;
+          issue_d1(1);
+        }
+        // Each barrier completes once per chunk and is waited on by parity,
+        // so no arrival may run two phases ahead of its waiter: every
+        // producer of a phase first waits, directly or through this thread's
+        // program order, for its consumer's previous phase.
         for (int c = 0; c < n && ok; ++c) {
           const uint32_t ph = c & 1;
           const uint32_t kq = a_kq + (c & 1) * 4 * kTileBytes;
-          // V'^T = U^T + S_b (-W)^T ;  O = S_b Q~^T
+          // V'^T = U^T + S_b (-W)^T
           if (!(ok = W(B_WTB, ph) && W(B_SBR, ph))) break;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             mma_bf16_ts(tm + TM_UV, tm + TM_SB + 8 * kk,
                         sdesc_sw128(a_wt + kk * 2048, 2 * kTileBytes, 1024), ID_VP, 1);
           }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t boff = kTileBytes + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32;
-            mma_bf16_ts(tm + TM_O, tm + TM_SB + 8 * kk, sdesc_sw128(kq + boff, 16, 1024), ID_O,
-                        kk > 0);
-          }
           mma_commit(&bars[B_VPF]);
-          if (c + 1 < n) {
-            if (!(ok = W(B_D1E, ph) && W(B_FULL + ((c + 1) & 1), ((c + 1) >> 1) & 1))) break;
-            issue_d1(c + 1);
-          }
-          // O += V'^T P^T ;  S += (V'^T decayed) K
+          // O_a = S_b Q^T ;  S += (V'^T decayed) K ;  O_b = V'^T P^T.  O_a is
+          // issued before the SF commit: SF then also covers the last read
+          // of S_b, which the state group overwrites once SF completes.
           if (!(ok = W(B_VPR, ph))) break;
           const uint32_t pp = a_p + (c & 1) * kTileBytes;
 #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t boff = kTileBytes + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32;
+            mma_bf16_ts(tm + TM_OA, tm + TM_SB + 8 * kk, sdesc_sw128(kq + boff, 16, 1024), ID_O,
+                        kk > 0);
+          }
+#pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_ss(tm + TM_O, sdesc_sw128(a_vp + kk * 32, 16, 1024),
-                        sdesc_sw128(pp + kk * 32, 16, 1024), ID_O, 1);
             mma_bf16_ss(tm + TM_S, sdesc_sw128(a_vpd + kk * 32, 16, 1024),
                         sdesc_sw128(kq + kk * 2048, 2 * kTileBytes, 1024), ID_S, 1);
+          }
+          mma_commit(&bars[B_SF]);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_bf16_ss(tm + TM_O, sdesc_sw128(a_vp + kk * 32, 16, 1024),
+                        sdesc_sw128(pp + kk * 32, 16, 1024), ID_O, kk > 0);
           }
           mma_commit(&bars[B_OF]);
           mma_commit(&bars[B_EMPTY + (c & 1)]);
@@ -468,6 +589,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = W(B_TRDY, (c + 1) & 1))) break;
             issue_uw(c + 1);
           }
+          if (c + 2 < n) {
+            if (!(ok = W(B_D1E, (c + 1) & 1) && W(B_FULL + (c & 1), ((c + 2) >> 1) & 1))) break;
+            issue_d1(c + 2);
+          }
         }
       } while (0);
       // Drain: all issued MMAs complete before TMEM is released.
@@ -475,10 +600,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_bounded(&bars[B_FIN], 0, kWaitNs);
       if (!ok) atomicOr(a.status, kStatusTimeout);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 4 + kPrepWarps) {
     // ================================================================ prep group
-    const int t = tid - 128;  // 0..127, also the TMEM lane
-    const int lrow = t;
+    // TMEM lane rl = pt; each thread handles both 32-column halves hp of
+    // its 64-column rows.
+    const int pt = tid - 128, rl = pt & 127, hp0 = 0, pw = pt >> 5;
+    constexpr int kHalfStep = 1;
+    const int lrow = rl;
     (void)lrow;
     constexpr uint32_t kBar = 3;
     for (int c = 0; c < n; ++c) {
@@ -486,19 +614,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = c & 1;
       float *vec = reinterpret_cast<float *>(sm + Lay::VEC + (c % 3) * 1024);
       float *gcv = vec, *egv = vec + 64, *iegv = vec + 128, *eglv = vec + 192;
-      if (group_any(kBar, !wait_or_abort(&bars[B_FULL + s], (c >> 1) & 1, abort_flag))) break;
+      if (!group_wait(kBar, &bars[B_FULL + s], (c >> 1) & 1, abort_flag, lane)) break;
       const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + s * 512);
       const float *bs = gs + 64;
-      if (warp == 4) {  // cumulative log decay and the derived factors
-        float x0 = gs[lane], x1 = gs[lane + 32];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
-          const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
-          if (lane >= off) { x0 += y0; x1 += y1; }
-        }
-        x1 += __shfl_sync(0xffffffffu, x0, 31);
-        const float gl = __shfl_sync(0xffffffffu, x1, 31);
+      if (pw == 0) {  // cumulative log decay and the derived factors
+        float x0, x1;
+        const float gl = chunk_cumsum(gs, lane, x0, x1);
         gcv[lane] = x0;
         gcv[lane + 32] = x1;
         egv[lane] = __expf(x0);
@@ -510,119 +631,135 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       group_bar(kBar);
       const bool factored = -gcv[63] < kSafeDecay;
-      // ---- A (lanes 0-63) and P (lanes 64-127) from D1
-      if (group_any(kBar, !wait_or_abort(&bars[B_D1F], ph, abort_flag))) break;
+      // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns each
+      if (!group_wait(kBar, &bars[B_D1F], ph, abort_flag, lane)) break;
       tc_fence_after();
-      {
-        const int r = t & 63;
+      for (int hp = hp0; hp < 2; hp += kHalfStep) {
+        const int r = rl & 63;
         const float gr = gcv[r];
-        const float br = t < 64 ? bs[r] : 1.f;
+        const float br = rl < 64 ? bs[r] : 1.f;
         const float fr = br * egv[r];
-        uint8_t *ptile = sm + Lay::P + s * kTileBytes;
+        float x[32];
+        tmem_ld32(lane_base + TM_D1 + 32 * hp, x);
+        DBG_ROW(32 * hp, 64, x);
+        const int lim = (rl < 64 ? r : r + 1) - 32 * hp;  // A: s < r, P: s <= r
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float x[32];
-          tmem_ld32(lane_base + TM_D1 + 32 * q, x);
-          DBG_ROW(32 * q, 64, x);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int s2 = 32 * q + e;
-            const float d = factored ? fr * iegv[s2] : br * __expf(gr - gcv[s2]);
-            x[e] = (t < 64 ? (s2 < r) : (s2 <= r)) ? x[e] * d : 0.f;
-          }
-          if (t < 64) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) AF[r * 65 + 32 * q + e] = x[e];
+        for (int s4 = 0; s4 < 8; ++s4) {
+          float4 dv;
+          if (factored) {
+            const float4 ie = *reinterpret_cast<const float4 *>(iegv + 32 * hp + 4 * s4);
+            dv = make_float4(fr * ie.x, fr * ie.y, fr * ie.z, fr * ie.w);
           } else {
-            st_row32_sw128(ptile, r, q, x);
+            const float4 gg = *reinterpret_cast<const float4 *>(gcv + 32 * hp + 4 * s4);
+            dv = make_float4(br * __expf(gr - gg.x), br * __expf(gr - gg.y),
+                             br * __expf(gr - gg.z), br * __expf(gr - gg.w));
           }
+          const int s2 = 4 * s4;
+          x[s2 + 0] = (s2 + 0 < lim) ? x[s2 + 0] * dv.x : 0.f;
+          x[s2 + 1] = (s2 + 1 < lim) ? x[s2 + 1] * dv.y : 0.f;
+          x[s2 + 2] = (s2 + 2 < lim) ? x[s2 + 2] * dv.z : 0.f;
+          x[s2 + 3] = (s2 + 3 < lim) ? x[s2 + 3] * dv.w : 0.f;
+        }
+        if (rl < 64) {
+          float4 *dst = reinterpret_cast<float4 *>(AF + r * LDA + 32 * hp);
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4)
+            dst[s4] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
+        } else {
+          st_row32_sw128(sm + Lay::P + s * kTileBytes, r, hp, x);
         }
       }
       tc_fence_before();
       mbar_arrive(&bars[B_D1E]);
       group_bar(kBar);
       // ---- Y = (I + A)^{-1}
-      invert_unit_lower(AF, Rs, t, kBar);
+      invert_unit_lower(AF, reinterpret_cast<float *>(sm + Lay::SCR), pt, kBar);
 #ifdef GDR_TC_DEBUG
-      if (t < 64) {
-        DBG_ROW(12288, 64, AF + t * 65);
-        DBG_ROW(12288 + 32, 64, AF + t * 65 + 32);
-      }
+      for (int hp = hp0; hp < 2; hp += kHalfStep)
+        if (rl < 64) DBG_ROW(12288 + 32 * hp, 64, AF + rl * LDA + 32 * hp);
 #endif
       // ---- T (lanes 0-63) and T' (lanes 64-127) as bf16 operands
-      {
-        const int r = t & 63;
-        uint8_t *tile = sm + (t < 64 ? Lay::T : Lay::TP);
+      for (int hp = hp0; hp < 2; hp += kHalfStep) {
+        const int r = rl & 63;
+        uint8_t *tile = sm + (rl < 64 ? Lay::T : Lay::TP);
+        float x[32];
+        const float4 *yr = reinterpret_cast<const float4 *>(AF + r * LDA + 32 * hp);
+        const float4 *b4 = reinterpret_cast<const float4 *>(bs + 32 * hp);
+        const float4 *e4 = reinterpret_cast<const float4 *>(egv + 32 * hp);
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float x[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int s2 = 32 * q + e;
-            x[e] = AF[r * 65 + s2] * bs[s2] * (t < 64 ? 1.f : egv[s2]);
+        for (int s4 = 0; s4 < 8; ++s4) {
+          const float4 y = yr[s4], bb = b4[s4];
+          float4 f = make_float4(bb.x, bb.y, bb.z, bb.w);
+          if (rl >= 64) {
+            const float4 ee = e4[s4];
+            f = make_float4(f.x * ee.x, f.y * ee.y, f.z * ee.z, f.w * ee.w);
           }
-          st_row32_sw128(tile, r, q, x);
+          x[4 * s4 + 0] = y.x * f.x;
+          x[4 * s4 + 1] = y.y * f.y;
+          x[4 * s4 + 2] = y.z * f.z;
+          x[4 * s4 + 3] = y.w * f.w;
         }
-      }
-      // ---- Q~ = Diag(e^{gc}) Q in place (both 64-column halves)
-      {
-        uint8_t *kq = sm + Lay::KQ + s * 4 * kTileBytes;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int idx = t + 128 * m;  // 16-byte chunk index over 2 x 64 rows x 8
-          const int half = idx >> 9, row = (idx >> 3) & 63, ch = idx & 7;
-          uint4 *p = reinterpret_cast<uint4 *>(kq + kTileBytes + half * 2 * kTileBytes +
-                                               row * 128 + ch * 16);
-          uint4 u = *p;
-          const float e = egv[row];
-          uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162 *>(&w[j]);
-            float2 f = __bfloat1622float2(v2);
-            w[j] = pack_bf16(f.x * e, f.y * e);
-          }
-          *p = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+        st_row32_sw128(tile, r, hp, x);
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_TRDY]);
       group_bar(kBar);
-      if (t == 0) mbar_arrive(&bars[B_EMPTY + s]);  // g, beta of this stage no longer read
+      if (pt == 0) mbar_arrive(&bars[B_EMPTY + s]);  // g, beta of this stage no longer read
       // ---- -W^T -> bf16 MN-major operand (row j = this thread's lane)
-      if (group_any(kBar, !wait_or_abort(&bars[B_WTF], ph, abort_flag))) break;
+      if (!group_wait(kBar, &bars[B_WTF], ph, abort_flag, lane)) break;
       tc_fence_after();
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
+      for (int hp = hp0; hp < 2; hp += kHalfStep) {
         float x[32];
-        tmem_ld32(lane_base + TM_WT + 32 * q, x);
-        DBG_ROW(16384 + 32 * q, 64, x);
+        tmem_ld32(lane_base + TM_WT + 32 * hp, x);
+        DBG_ROW(16384 + 32 * hp, 64, x);
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[e] = -x[e];
-        st_row32_sw128(sm + Lay::WT, t, q, x);
+        st_row32_sw128(sm + Lay::WT, rl, hp, x);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_WTB]);
     }
-  } else {
+  } else if (warp < 4) {
     // ================================================================ state group
     const int i = tid;  // TMEM lane = value channel
     const int lrow = i;
     (void)lrow;
     constexpr uint32_t kBar = 2;
     bool ok = true;
-    // Initial state: S = S0 e^{gc_last(0)} (fp32), S_b = bf16(S0).
-    if (group_any(kBar, !wait_or_abort(&bars[B_TRDY], 0, abort_flag))) ok = false;
-    if (ok) {
-      const float *vec = reinterpret_cast<const float *>(sm + Lay::VEC);
-      const float dl = vec[64 + 63];  // e^{gc_last} of chunk 0
+    // Gate factors of chunk c for this group: e^{gc_r} and e^{gc_last - gc_r}
+    // into SVEC[c & 1], and the chunk's total decay e^{gc_last}.  Computed
+    // from the staged g with the prep group's scan (bit-identical values);
+    // the stage's TMA barrier cannot run ahead of this group.
+    auto chunk_vectors = [&](int c, float &dl) -> bool {
+      if (!group_wait(kBar, &bars[B_FULL + (c & 1)], (c >> 1) & 1, abort_flag, lane))
+        return false;
+      float *sv = reinterpret_cast<float *>(sm + Lay::SVEC + (c & 1) * 512);
+      if (warp == 0) {
+        const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + (c & 1) * 512);
+        float x0, x1;
+        const float gl = chunk_cumsum(gs, lane, x0, x1);
+        sv[lane] = __expf(x0);
+        sv[lane + 32] = __expf(x1);
+        sv[64 + lane] = __expf(gl - x0);
+        sv[64 + lane + 32] = __expf(gl - x1);
+      }
+      group_bar(kBar);
+      dl = sv[63];
+      return true;
+    };
+    // S_b = bf16(S) for the next chunk's MMAs, and S <- S * dl (that chunk's
+    // decay, applied before its state update accumulates onto S).
+    auto state_pass = [&](const float *src_global, float dl) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float x[32];
+        if (src_global) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          x[e] = a.S0 ? a.S0[((size_t)bh * DV + i) * DK + 32 * q + e] : 0.f;
+          for (int e = 0; e < 32; ++e) x[e] = src_global[32 * q + e];
+        } else {
+          tmem_ld32(lane_base + TM_S + 32 * q, x);
+        }
         uint32_t u[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
@@ -639,88 +776,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[B_SBR]);
-    }
-    for (int c = 0; ok && c < n; ++c) {
-      const uint32_t ph = c & 1;
-      const float *vec = reinterpret_cast<const float *>(sm + Lay::VEC + (c % 3) * 1024);
-      const float *eglv = vec + 192;
-      // ---- V'^T -> bf16 operands (plain and decayed to the chunk end)
-      if (group_any(kBar, !wait_or_abort(&bars[B_VPF], ph, abort_flag))) { ok = false; break; }
-      tc_fence_after();
-      if (i == 0) tma_store_wait_read0();  // previous O staging (aliases VP) is free
-      group_bar(kBar);
+    };
+    {
+      float dl;
+      if (!chunk_vectors(0, dl)) {
+        ok = false;
+      } else if (a.S0) {
+        state_pass(a.S0 + ((size_t)bh * DV + i) * DK, dl);
+      } else {
+        // zero initial state: write zeros through the same path
+        float z[32];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float x[32];
-        tmem_ld32(lane_base + TM_UV + 32 * q, x);
-        DBG_ROW(40960 + 32 * q, 64, x);
-        st_row32_sw128(sm + Lay::VP, i, q, x);
+        for (int e = 0; e < 32; ++e) z[e] = 0.f;
+        uint32_t u[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] *= eglv[32 * q + e];
-        st_row32_sw128(sm + Lay::VPD, i, q, x);
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars[B_VPR]);
-      // ---- O -> bf16 -> staging (VP region) -> TMA store
-      if (group_any(kBar, !wait_or_abort(&bars[B_OF], ph, abort_flag))) { ok = false; break; }
-      tc_fence_after();
-      {
-        uint32_t *stg = reinterpret_cast<uint32_t *>(sm + Lay::VP + (i >> 6) * kTileBytes);
-        const int col = i & 63;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float x[32];
-          tmem_ld32(lane_base + TM_O + 32 * q, x);
-          DBG_ROW(49152 + 32 * q, 64, x);
-          // lanes i, i^1 swap so each writes two adjacent channels of one token
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float lo = x[2 * e], hi = x[2 * e + 1];  // tokens 32q+2e, +1
-            const float send = (i & 1) ? lo : hi;
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-            const int r = 32 * q + 2 * e + (i & 1);
-            const uint32_t w = (i & 1) ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
-            stg[(r * 64 + (col & ~1)) >> 1] = w;
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      group_bar(kBar);
-      if (i == 0) {
-        tma_store_4d(&tmO, sm + Lay::VP, 0, h, c * C, b);
-        tma_store_4d(&tmO, sm + Lay::VP + kTileBytes, 64, h, c * C, b);
-        tma_store_commit();
-      }
-      if (c + 1 < n) {
-        // ---- S (= state after this chunk) -> S_b; pre-decay by the next chunk
-        if (group_any(kBar, !wait_or_abort(&bars[B_TRDY], (c + 1) & 1, abort_flag))) {
-          ok = false;
-          break;
-        }
-        const float *vn = reinterpret_cast<const float *>(sm + Lay::VEC + ((c + 1) % 3) * 1024);
-        const float dl = vn[64 + 63];
+        for (int e = 0; e < 16; ++e) u[e] = 0u;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float x[32];
-          tmem_ld32(lane_base + TM_S + 32 * q, x);
-          DBG_ROW(57344 + 32 * q, 128, x);
-          uint32_t u[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
           tmem_st16u(lane_base + TM_SB + 16 * q, u);
-          float y0[16], y1[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            y0[e] = x[e] * dl;
-            y1[e] = x[16 + e] * dl;
-          }
-          tmem_st16(lane_base + TM_S + 32 * q, y0);
-          tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
+          tmem_st16(lane_base + TM_S + 32 * q, *reinterpret_cast<float(*)[16]>(z));
+          tmem_st16(lane_base + TM_S + 32 * q + 16, *reinterpret_cast<float(*)[16]>(z + 16));
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[B_SBR]);
+      }
+    }
+    for (int c = 0; ok && c < n; ++c) {
+      const uint32_t ph = c & 1;
+      const float *sv = reinterpret_cast<const float *>(sm + Lay::SVEC + (c & 1) * 512);
+      const float *egv = sv, *eglv = sv + 64;
+      // ---- V'^T -> bf16 operands (plain and decayed to the chunk end)
+      if (!group_wait(kBar, &bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
+      tc_fence_after();
+      {
+        float x[64];
+        tmem_ld64(lane_base + TM_UV, x);
+        DBG_ROW(40960, 64, x);
+        DBG_ROW(40960 + 32, 64, x + 32);
+        st_row32_sw128(sm + Lay::VP, i, 0, x);
+        st_row32_sw128(sm + Lay::VP, i, 1, x + 32);
+        const float4 *e4 = reinterpret_cast<const float4 *>(eglv);
+#pragma unroll
+        for (int s4 = 0; s4 < 16; ++s4) {
+          const float4 e = e4[s4];
+          x[4 * s4] *= e.x;
+          x[4 * s4 + 1] *= e.y;
+          x[4 * s4 + 2] *= e.z;
+          x[4 * s4 + 3] *= e.w;
+        }
+        st_row32_sw128(sm + Lay::VPD, i, 0, x);
+        st_row32_sw128(sm + Lay::VPD, i, 1, x + 32);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[B_VPR]);
+      // ---- updated S -> S_b and the next chunk's decay, or the final state
+      if (!group_wait(kBar, &bars[B_SF], ph, abort_flag, lane)) { ok = false; break; }
+      tc_fence_after();
+      if (c + 1 < n) {
+        float dl;
+        if (!chunk_vectors(c + 1, dl)) { ok = false; break; }
+#ifdef GDR_TC_DEBUG
+        for (int q = 0; q < 4; ++q) {
+          float x[32];
+          tmem_ld32(lane_base + TM_S + 32 * q, x);
+          DBG_ROW(57344 + 32 * q, 128, x);
+        }
+#endif
+        state_pass(nullptr, dl);
       } else if (a.S_T) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -733,8 +857,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
         }
       }
+      // ---- O = O_a Diag(e^{gc}) + O_b -> bf16, stored straight to o: lanes
+      //      i, i^1 swap values so each lane writes two adjacent channels of
+      //      one token (a warp writes 2 tokens x 64 contiguous bytes)
+      if (!group_wait(kBar, &bars[B_OF], ph, abort_flag, lane)) { ok = false; break; }
+      tc_fence_after();
+      {
+        const int t0 = c * C;
+        const size_t tok0 = ((size_t)b * T + t0) * H + h;
+        uint32_t *o32 = reinterpret_cast<uint32_t *>(a.o);
+        const int chpair = i & ~1;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          float xa[32], xb[32];
+          {
+            float a0[16], a1[16], b0[16], b1[16];
+            tmem_ld16(lane_base + TM_OA + 32 * q, a0);
+            tmem_ld16(lane_base + TM_OA + 32 * q + 16, a1);
+            tmem_ld16(lane_base + TM_O + 32 * q, b0);
+            tmem_ld16(lane_base + TM_O + 32 * q + 16, b1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              xa[e] = a0[e];
+              xa[16 + e] = a1[e];
+              xb[e] = b0[e];
+              xb[16 + e] = b1[e];
+            }
+          }
+          const float4 *e4 = reinterpret_cast<const float4 *>(egv + 32 * q);
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const float4 ev = e4[s4];
+            xa[4 * s4 + 0] = ev.x * xa[4 * s4 + 0] + xb[4 * s4 + 0];
+            xa[4 * s4 + 1] = ev.y * xa[4 * s4 + 1] + xb[4 * s4 + 1];
+            xa[4 * s4 + 2] = ev.z * xa[4 * s4 + 2] + xb[4 * s4 + 2];
+            xa[4 * s4 + 3] = ev.w * xa[4 * s4 + 3] + xb[4 * s4 + 3];
+          }
+          DBG_ROW(49152 + 32 * q, 64, xa);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float lo = xa[2 * e], hi = xa[2 * e + 1];  // tokens 32q+2e, +1
+            const float send = (i & 1) ? lo : hi;
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+            const int r = 32 * q + 2 * e + (i & 1);
+            const uint32_t w = (i & 1) ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
+            if (t0 + r < T) __stcs(o32 + (((tok0 + (size_t)r * H) * DV + chpair) >> 1), w);
+          }
+        }
+      }
+      tc_fence_before();
     }
-    if (i == 0) tma_store_wait0();
     if (!ok && i == 0) atomicOr(a.status, kStatusTimeout);
   }
 
@@ -759,8 +932,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D map over a [B, T, H, d] bf16 tensor, box = 64 tokens x 64 channels.
-bool make_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, bool swizzle) {
+// 4-D map over a [B, T, H, d] bf16 tensor, box = 64 tokens x 64 channels,
+// 128-byte swizzle (the layout the MMA descriptors expect).
+bool make_map(CUtensorMap *m, const void *base, int B, int T, int H, int d) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -769,7 +943,7 @@ bool make_map(CUtensorMap *m, const void *base, int B, int T, int H, int d, bool
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -783,16 +957,16 @@ bool chunk_tc_supports(const ChunkArgs &a) {
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
   if (!chunk_tc_supports(a)) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv, mo;
-  if (!make_map(&mq, a.q, a.B, a.T, a.H, DK, true) || !make_map(&mk, a.k, a.B, a.T, a.H, DK, true) ||
-      !make_map(&mv, a.v, a.B, a.T, a.H, DV, true) || !make_map(&mo, a.o, a.B, a.T, a.H, DV, false))
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, a.B, a.T, a.H, DK) ||
+      !make_map(&mv, a.v, a.B, a.T, a.H, DV))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   gdr_chunk_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, kSmemBytes, stream>>>(mq, mk, mv,
-                                                                                       mo, a);
+                                                                                       a);
   return cudaGetLastError();
 }
 
