@@ -36,9 +36,14 @@ from gated_delta_rule_93_b200.sharding import max_over_ranks  # noqa: E402
 METRIC = "tokens/s and TFLOP/s per gated-delta layer fwd (1 B200), % of roofline"
 DEFAULT_WORKLOAD = "gdn_b8_t4096_h16_d128"
 L2_BYTES = 126 * 1024 * 1024
-CHUNK_KERNEL_SOURCES = ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
-                        "gated_delta_rule_93_b200/csrc/gdr_chunk_simt.cu",
-                        "gated_delta_rule_93_b200/csrc/gdr_abi.cu"]
+KERNEL_SOURCES = {
+    "chunk": ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
+              "gated_delta_rule_93_b200/csrc/gdr_chunk_simt.cu",
+              "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh",
+              "gated_delta_rule_93_b200/csrc/gdr_abi.cu"],
+    "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu",
+             "gated_delta_rule_93_b200/csrc/gdr_abi.cu"],
+}
 
 
 # ------------------------------------------------------------------ work model
@@ -73,9 +78,10 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kind="chunk"):
+    """Hash of the sources of the kernel a workload times (profiles record it)."""
     h = hashlib.sha256()
-    for rel in CHUNK_KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kind]:
         p = os.path.join(ROOT, rel)
         if os.path.exists(p):
             with open(p, "rb") as f:
@@ -83,13 +89,13 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload):
+def recorded_traffic(workload, kind="chunk"):
     """dram read+write bytes per launch from the committed ncu summary, if it
     was taken on the current kernel sources (else None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
-    cur = kernel_source_hash()
+    cur = kernel_source_hash(kind)
     with open(p) as f:
         for line in f:
             parts = line.split()
@@ -303,7 +309,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline_time_ms": roof_ms,
         "roofline_fraction": roof_ms / ms_step,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name),
+                     "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
                      "kernel": "gdr_chunk_fwd" if w.kind == "chunk" else "gdr_step"},
         "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",

@@ -32,6 +32,7 @@ EXPORTS = (
     "gdr_status_string",
     "gdr_last_error_message",
     "gdr_version",
+    "gdr_testing_skip_stage_load",
 )
 
 
@@ -67,6 +68,8 @@ def lib():
             L.gdr_last_error_message.restype = ctypes.c_char_p
             L.gdr_version.argtypes = []
             L.gdr_version.restype = i
+            L.gdr_testing_skip_stage_load.argtypes = [i]
+            L.gdr_testing_skip_stage_load.restype = i
             _lib = L
     return _lib
 
@@ -188,6 +191,12 @@ def step(q, k, v, g, beta, S, *, o=None, stream=None):
                             _ptr(S), _ptr(o), N, H, dk, dv, _stream_handle(stream))
     _check(rc)
     return o
+
+
+def testing_skip_stage_load(chunk):
+    """Test-only: the next tensor-core chunked forward on this thread skips the
+    input load of `chunk`, so its bounded waits time out (see gdr_testing.h)."""
+    _check(lib().gdr_testing_skip_stage_load(int(chunk)))
 
 
 def device_status(stream=None):

@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "gdr_internal.cuh"
+#include "gdr_testing.h"
 
 namespace gdr {
 __device__ unsigned int g_device_status = 0;
@@ -14,6 +15,7 @@ __device__ unsigned int g_device_status = 0;
 namespace {
 
 thread_local char t_msg[512] = "";
+thread_local int t_skip_stage_chunk = -1;  // testing hook, consumed by the next call
 
 gdr_status fail(gdr_status s, const char *fmt, ...) {
   va_list ap;
@@ -116,6 +118,8 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
   a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
   a.bf16 = in_dtype == GDR_BF16;
   a.per_channel = gate == GDR_GATE_PER_CHANNEL;
+  a.skip_stage_chunk = t_skip_stage_chunk;
+  t_skip_stage_chunk = -1;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = status_word(&a.status);
   if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd status word");
@@ -152,6 +156,12 @@ gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dt
   if (e != cudaSuccess) return from_cuda(e, "gdr_step status word");
   return from_cuda(gdr::launch_step(a, reinterpret_cast<cudaStream_t>(stream)),
                    "gdr_step launch");
+}
+
+gdr_status gdr_testing_skip_stage_load(int chunk) {
+  if (chunk < 0) return fail(GDR_ERR_INVALID_ARG, "chunk must be >= 0");
+  t_skip_stage_chunk = chunk;
+  return ok();
 }
 
 gdr_status gdr_get_device_status(gdr_stream_t stream) {

@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    int issued = 0;
+    int last_issued[kStages] = {-1, -1};  // latest chunk loaded into each stage
     for (int c = 0; c < n; ++c) {
       const int s = c & 1;
       if (c >= kStages) {
@@ -472,6 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) ok = wait_or_abort(&bars[B_EMPTY + s], ((c >> 1) - 1) & 1, abort_flag);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
+      // Testing hook: this chunk's load is never issued, so its consumers'
+      // bounded waits run out and the kernel unwinds (no trap, no hang).
+      if (c == a.skip_stage_chunk) continue;
       const int t0 = c * C;
       float *gs = reinterpret_cast<float *>(sm + Lay::GS + s * 512);
 #pragma unroll
@@ -494,12 +497,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(vv + 0 * kTileBytes, &tmV, fb, 0, h, t0, b);
         tma_load_4d(vv + 1 * kTileBytes, &tmV, fb, 64, h, t0, b);
       }
-      ++issued;
+      last_issued[s] = c;
     }
-    // Loads issued but never consumed exist only after an abort: let them land.
+    // A load issued but never consumed exists only after an abort: let it land
+    // before the CTA exits.
     if (lane == 0) {
-      for (int c = *consumed; c < issued; ++c)
-        mbar_wait_bounded(&bars[B_FULL + (c & 1)], (c >> 1) & 1, kWaitNs);
+      for (int s = 0; s < kStages; ++s) {
+        const int c = last_issued[s];
+        if (c >= 0 && c >= *consumed)
+          mbar_wait_bounded(&bars[B_FULL + s], (c >> 1) & 1, kWaitNs);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer

@@ -24,6 +24,7 @@ struct ChunkArgs {
   int bf16;          // 1: q, k, v, o are bf16; 0: fp32
   int per_channel;   // 1: g is [B,T,H,dk]
   unsigned int *status;  // device status word
+  int skip_stage_chunk;  // testing: chunk whose input load is never issued (-1: none)
 };
 
 struct StepArgs {
