@@ -242,16 +242,93 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// Helpers of the blocked inverse below (one warp, mma.sync m16n8k8 TF32
+// fragments: g = lane / 4, tq = lane % 4).
+struct Frag {
+  int g, tq;
+  float *scr;  // warp-private [16][8] fp32 scratch
+  // A fragment of the 16x8 block of AF at (row0, col0).
+  __device__ __forceinline__ void a(const float *AF, int row0, int col0, uint32_t (&af)[4]) const {
+    af[0] = to_tf32(AF[(row0 + g) * LDA + col0 + tq]);
+    af[1] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq]);
+    af[2] = to_tf32(AF[(row0 + g) * LDA + col0 + tq + 4]);
+    af[3] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq + 4]);
+  }
+  // 16x8 accumulator fragment -> B fragments of two k-steps (rows 0-7, 8-15).
+  __device__ __forceinline__ void to_b(const float (&cf)[4], uint32_t (&bf)[2][2]) const {
+    scr[g * 8 + 2 * tq] = cf[0];
+    scr[g * 8 + 2 * tq + 1] = cf[1];
+    scr[(g + 8) * 8 + 2 * tq] = cf[2];
+    scr[(g + 8) * 8 + 2 * tq + 1] = cf[3];
+    __syncwarp();
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      bf[ks][0] = to_tf32(scr[(8 * ks + tq) * 8 + g]);
+      bf[ks][1] = to_tf32(scr[(8 * ks + tq + 4) * 8 + g]);
+    }
+    __syncwarp();
+  }
+};
+
+// One 8-column strip (first column `col`) of column block J of Y = (I + A)^{-1}:
+// Y_JJ = D_JJ (already in AF), Y_bJ = -D_bb sum_{k=J}^{b-1} A_bk Y_kJ for
+// b > J, swept down the block rows; the finished blocks stay in `yout[b]`.
+// J is a template parameter so that every loop is fully static.
+template <int J>
+__device__ __forceinline__ void inverse_strip(const float *AF, const Frag &f, int col,
+                                              float (&yout)[4][4]) {
+  uint32_t yb[4][2][2];
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    yb[J][ks][0] = to_tf32(AF[(16 * J + 8 * ks + f.tq) * LDA + col + f.g]);
+    yb[J][ks][1] = to_tf32(AF[(16 * J + 8 * ks + f.tq + 4) * LDA + col + f.g]);
+  }
+#pragma unroll
+  for (int bb = J + 1; bb < 4; ++bb) {
+    float racc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = J; k < bb; ++k) {
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        uint32_t af[4];
+        f.a(AF, 16 * bb, 16 * k + 8 * ks, af);
+        mma_tf32_16x8x8(racc, af, yb[k][ks]);
+      }
+    }
+    uint32_t rb[2][2];
+    f.to_b(racc, rb);
+    float yacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t af[4];
+      f.a(AF, 16 * bb, 16 * bb + 8 * ks, af);
+      mma_tf32_16x8x8(yacc, af, rb[ks]);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) yout[bb][e] = -yacc[e];
+    if (bb < 3) f.to_b(yout[bb], yb[bb]);
+  }
+}
+
+template <int J>
+__device__ __forceinline__ void store_strip(float *AF, const Frag &f, int col,
+                                            const float (&yout)[4][4]) {
+#pragma unroll
+  for (int bb = J + 1; bb < 4; ++bb) {
+    AF[(16 * bb + f.g) * LDA + col + 2 * f.tq] = yout[bb][0];
+    AF[(16 * bb + f.g) * LDA + col + 2 * f.tq + 1] = yout[bb][1];
+    AF[(16 * bb + f.g + 8) * LDA + col + 2 * f.tq] = yout[bb][2];
+    AF[(16 * bb + f.g + 8) * LDA + col + 2 * f.tq + 1] = yout[bb][3];
+  }
+}
+
 // (I + A)^{-1} in place for a strictly lower 64x64 fp32 matrix A (row stride
-// LDA, zero on and above the diagonal) with the 4-warp prep group (local
+// LDA, zero above the diagonal blocks) with the 4-warp prep group (local
 // thread t, warp w = t / 32), in 16x16 blocks:
 //  1. diagonal blocks D_bb = (I + A_bb)^{-1} by forward substitution (warp b);
-//  2. every 8-column strip of a column block j is independent:
-//       Y_jj = D_jj,   Y_bj = -D_bb sum_{k=j}^{b-1} A_bk Y_kj   (b > j),
-//     so each warp sweeps its strips down the block rows with mma.sync
-//     (TF32 operands rounded to nearest, fp32 accumulation), keeping the
-//     strip's finished blocks in registers and re-laying accumulator
-//     fragments as B fragments through a warp-private scratch;
+//  2. every 8-column strip of a column block is independent, so each warp
+//     sweeps its strips down the block rows with mma.sync (TF32 operands
+//     rounded to nearest, fp32 accumulation);
 //  3. after a group barrier the off-diagonal blocks overwrite A.
 // Strips (column block j, half hf): warp 0 -> (0,0); warp 1 -> (0,1);
 // warp 2 -> (1,0), (2,0); warp 3 -> (1,1), (2,1).  (The measured in-kernel
@@ -276,7 +353,7 @@ __device__ void invert_unit_lower(float *AF, float *R, int t, uint32_t bar_id) {
         if (4 * k4 + 2 < i) acc += av.z * x[4 * k4 + 2];
         if (4 * k4 + 3 < i) acc += av.w * x[4 * k4 + 3];
       }
-      if (i > c) x[i] = -acc;
+      x[i] = (i > c) ? -acc : x[i];
     }
     __syncwarp();
     if (lane < 16) {
@@ -286,90 +363,21 @@ __device__ void invert_unit_lower(float *AF, float *R, int t, uint32_t bar_id) {
     }
   }
   group_bar(bar_id);
-  const int g = lane >> 2, tq = lane & 3;
-  float *scr = R + warp * 128;  // [16][8] per warp
-  // accumulator fragment (16x8) -> B fragments of two k-steps (rows 0-7, 8-15)
-  auto to_bfrag = [&](const float (&cf)[4], uint32_t (&bf)[2][2]) {
-    scr[g * 8 + 2 * tq] = cf[0];
-    scr[g * 8 + 2 * tq + 1] = cf[1];
-    scr[(g + 8) * 8 + 2 * tq] = cf[2];
-    scr[(g + 8) * 8 + 2 * tq + 1] = cf[3];
-    __syncwarp();
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      bf[ks][0] = to_tf32(scr[(8 * ks + tq) * 8 + g]);
-      bf[ks][1] = to_tf32(scr[(8 * ks + tq + 4) * 8 + g]);
-    }
-    __syncwarp();
-  };
-  auto afrag = [&](int row0, int col0, uint32_t (&af)[4]) {
-    af[0] = to_tf32(AF[(row0 + g) * LDA + col0 + tq]);
-    af[1] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq]);
-    af[2] = to_tf32(AF[(row0 + g) * LDA + col0 + tq + 4]);
-    af[3] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq + 4]);
-  };
-  float yout[2][4][4];  // finished blocks: [strip slot][block row]
-  const int nstrip = warp < 2 ? 1 : 2;
-#pragma unroll
-  for (int si = 0; si < 2; ++si) {
-    if (si >= nstrip) break;
-    const int j = warp < 2 ? 0 : 1 + si, hf = warp & 1;
-    const int col = 16 * j + 8 * hf;  // first column of the strip
-    uint32_t yb[4][2][2];             // B fragments of Y_kj
-#pragma unroll
-    for (int jj = 0; jj < 3; ++jj) {  // Y_jj strip = D_jj (static indices only)
-      if (jj != j) continue;
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        yb[jj][ks][0] = to_tf32(AF[(16 * jj + 8 * ks + tq) * LDA + col + g]);
-        yb[jj][ks][1] = to_tf32(AF[(16 * jj + 8 * ks + tq + 4) * LDA + col + g]);
-      }
-    }
-#pragma unroll
-    for (int bb = 1; bb < 4; ++bb) {
-      if (bb <= j) continue;
-      float racc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < 3; ++k) {
-        if (k < j || k >= bb) continue;
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          uint32_t af[4];
-          afrag(16 * bb, 16 * k + 8 * ks, af);
-          mma_tf32_16x8x8(racc, af, yb[k][ks]);
-        }
-      }
-      uint32_t rb[2][2];
-      to_bfrag(racc, rb);
-      float yacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        uint32_t af[4];
-        afrag(16 * bb, 16 * bb + 8 * ks, af);
-        mma_tf32_16x8x8(yacc, af, rb[ks]);
-      }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        yacc[e] = -yacc[e];
-        yout[si][bb][e] = yacc[e];
-      }
-      if (bb < 3) to_bfrag(yacc, yb[bb]);
-    }
+  const Frag f{lane >> 2, lane & 3, R + warp * 128};
+  const int hf = warp & 1;
+  float y0[4][4], y1[4][4];
+  if (warp < 2) {
+    inverse_strip<0>(AF, f, 8 * hf, y0);
+  } else {
+    inverse_strip<1>(AF, f, 16 + 8 * hf, y0);
+    inverse_strip<2>(AF, f, 32 + 8 * hf, y1);
   }
   group_bar(bar_id);  // every read of A is done: store the off-diagonal blocks
-#pragma unroll
-  for (int si = 0; si < 2; ++si) {
-    if (si >= nstrip) break;
-    const int j = warp < 2 ? 0 : 1 + si, hf = warp & 1;
-    const int col = 16 * j + 8 * hf;
-#pragma unroll
-    for (int bb = 1; bb < 4; ++bb) {
-      if (bb <= j) continue;
-      AF[(16 * bb + g) * LDA + col + 2 * tq] = yout[si][bb][0];
-      AF[(16 * bb + g) * LDA + col + 2 * tq + 1] = yout[si][bb][1];
-      AF[(16 * bb + g + 8) * LDA + col + 2 * tq] = yout[si][bb][2];
-      AF[(16 * bb + g + 8) * LDA + col + 2 * tq + 1] = yout[si][bb][3];
-    }
+  if (warp < 2) {
+    store_strip<0>(AF, f, 8 * hf, y0);
+  } else {
+    store_strip<1>(AF, f, 16 + 8 * hf, y0);
+    store_strip<2>(AF, f, 32 + 8 * hf, y1);
   }
   group_bar(bar_id);
 }
@@ -650,23 +658,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + TM_D1 + 32 * hp, x);
         DBG_ROW(32 * hp, 64, x);
         const int lim = (rl < 64 ? r : r + 1) - 32 * hp;  // A: s < r, P: s <= r
+        // The decay form is chosen once per chunk, outside the unrolled loops
+        // (a branch inside them costs even when it is never taken).
+        float dvs[32];
+        if (factored) {
 #pragma unroll
-        for (int s4 = 0; s4 < 8; ++s4) {
-          float4 dv;
-          if (factored) {
+          for (int s4 = 0; s4 < 8; ++s4) {
             const float4 ie = *reinterpret_cast<const float4 *>(iegv + 32 * hp + 4 * s4);
-            dv = make_float4(fr * ie.x, fr * ie.y, fr * ie.z, fr * ie.w);
-          } else {
-            const float4 gg = *reinterpret_cast<const float4 *>(gcv + 32 * hp + 4 * s4);
-            dv = make_float4(br * __expf(gr - gg.x), br * __expf(gr - gg.y),
-                             br * __expf(gr - gg.z), br * __expf(gr - gg.w));
+            dvs[4 * s4 + 0] = fr * ie.x;
+            dvs[4 * s4 + 1] = fr * ie.y;
+            dvs[4 * s4 + 2] = fr * ie.z;
+            dvs[4 * s4 + 3] = fr * ie.w;
           }
-          const int s2 = 4 * s4;
-          x[s2 + 0] = (s2 + 0 < lim) ? x[s2 + 0] * dv.x : 0.f;
-          x[s2 + 1] = (s2 + 1 < lim) ? x[s2 + 1] * dv.y : 0.f;
-          x[s2 + 2] = (s2 + 2 < lim) ? x[s2 + 2] * dv.z : 0.f;
-          x[s2 + 3] = (s2 + 3 < lim) ? x[s2 + 3] * dv.w : 0.f;
+        } else {
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const float4 gg = *reinterpret_cast<const float4 *>(gcv + 32 * hp + 4 * s4);
+            dvs[4 * s4 + 0] = br * __expf(gr - gg.x);
+            dvs[4 * s4 + 1] = br * __expf(gr - gg.y);
+            dvs[4 * s4 + 2] = br * __expf(gr - gg.z);
+            dvs[4 * s4 + 3] = br * __expf(gr - gg.w);
+          }
         }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = (e < lim) ? x[e] * dvs[e] : 0.f;
         if (rl < 64) {
           float4 *dst = reinterpret_cast<float4 *>(AF + r * LDA + 32 * hp);
 #pragma unroll
@@ -693,18 +708,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 *yr = reinterpret_cast<const float4 *>(AF + r * LDA + 32 * hp);
         const float4 *b4 = reinterpret_cast<const float4 *>(bs + 32 * hp);
         const float4 *e4 = reinterpret_cast<const float4 *>(egv + 32 * hp);
+        if (rl < 64) {
 #pragma unroll
-        for (int s4 = 0; s4 < 8; ++s4) {
-          const float4 y = yr[s4], bb = b4[s4];
-          float4 f = make_float4(bb.x, bb.y, bb.z, bb.w);
-          if (rl >= 64) {
-            const float4 ee = e4[s4];
-            f = make_float4(f.x * ee.x, f.y * ee.y, f.z * ee.z, f.w * ee.w);
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const float4 y = yr[s4], bb = b4[s4];
+            x[4 * s4 + 0] = y.x * bb.x;
+            x[4 * s4 + 1] = y.y * bb.y;
+            x[4 * s4 + 2] = y.z * bb.z;
+            x[4 * s4 + 3] = y.w * bb.w;
           }
-          x[4 * s4 + 0] = y.x * f.x;
-          x[4 * s4 + 1] = y.y * f.y;
-          x[4 * s4 + 2] = y.z * f.z;
-          x[4 * s4 + 3] = y.w * f.w;
+        } else {
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const float4 y = yr[s4], bb = b4[s4], ee = e4[s4];
+            x[4 * s4 + 0] = y.x * (bb.x * ee.x);
+            x[4 * s4 + 1] = y.y * (bb.y * ee.y);
+            x[4 * s4 + 2] = y.z * (bb.z * ee.z);
+            x[4 * s4 + 3] = y.w * (bb.w * ee.w);
+          }
         }
         st_row32_sw128(tile, r, hp, x);
       }
@@ -756,29 +777,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     // S_b = bf16(S) for the next chunk's MMAs, and S <- S * dl (that chunk's
-    // decay, applied before its state update accumulates onto S).
+    // decay, applied before its state update accumulates onto S).  The
+    // source (S0 in global memory, or S in TMEM) is chosen outside the
+    // unrolled loops.
+    auto state_cols = [&](int q, const float (&x)[32], float dl) {
+      uint32_t u[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+      tmem_st16u(lane_base + TM_SB + 16 * q, u);
+      float y0[16], y1[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        y0[e] = x[e] * dl;
+        y1[e] = x[16 + e] * dl;
+      }
+      tmem_st16(lane_base + TM_S + 32 * q, y0);
+      tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
+    };
     auto state_pass = [&](const float *src_global, float dl) {
+      if (src_global) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float x[32];
-        if (src_global) {
+        for (int q = 0; q < 4; ++q) {
+          float x[32];
+          const float4 *s4 = reinterpret_cast<const float4 *>(src_global + 32 * q);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = src_global[32 * q + e];
-        } else {
+          for (int e = 0; e < 8; ++e) {
+            const float4 v = s4[e];
+            x[4 * e] = v.x;
+            x[4 * e + 1] = v.y;
+            x[4 * e + 2] = v.z;
+            x[4 * e + 3] = v.w;
+          }
+          state_cols(q, x, dl);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float x[32];
           tmem_ld32(lane_base + TM_S + 32 * q, x);
+          state_cols(q, x, dl);
         }
-        uint32_t u[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
-        tmem_st16u(lane_base + TM_SB + 16 * q, u);
-        float y0[16], y1[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          y0[e] = x[e] * dl;
-          y1[e] = x[16 + e] * dl;
-        }
-        tmem_st16(lane_base + TM_S + 32 * q, y0);
-        tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -874,6 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t tok0 = ((size_t)b * T + t0) * H + h;
         uint32_t *o32 = reinterpret_cast<uint32_t *>(a.o);
         const int chpair = i & ~1;
+        const bool full = t0 + C <= T;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           float xa[32], xb[32];
@@ -902,14 +941,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             xa[4 * s4 + 3] = ev.w * xa[4 * s4 + 3] + xb[4 * s4 + 3];
           }
           DBG_ROW(49152 + 32 * q, 64, xa);
+          // full chunks store unconditionally; only a ragged last chunk
+          // takes the guarded loop (chosen outside the unrolled loops)
+          uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float lo = xa[2 * e], hi = xa[2 * e + 1];  // tokens 32q+2e, +1
             const float send = (i & 1) ? lo : hi;
             const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-            const int r = 32 * q + 2 * e + (i & 1);
-            const uint32_t w = (i & 1) ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
-            if (t0 + r < T) __stcs(o32 + (((tok0 + (size_t)r * H) * DV + chpair) >> 1), w);
+            w[e] = (i & 1) ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
+          }
+          uint32_t *dst = o32 + (((tok0 + (size_t)(32 * q + (i & 1)) * H) * DV + chpair) >> 1);
+          const size_t tstep = (size_t)H * DV;  // 32-bit words between tokens t and t + 2
+          if (full) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) __stcs(dst + e * tstep, w[e]);
+          } else {
+            const int rem = T - t0 - 32 * q - (i & 1);  // tokens left for this lane's parity
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (2 * e < rem) __stcs(dst + e * tstep, w[e]);
           }
         }
       }
