@@ -11,28 +11,39 @@
 //
 //   D1   = [K; Q] K^T                      (tcgen05, M=128 N=64 K=128)
 //   A    = strict_tril(beta_r D1_KK[r][s] e^{gc_r - gc_s})
-//   P    = tril_incl(D1_QK[r][s] e^{gc_r - gc_s})       -> bf16, smem
+//   P    = tril_incl(D1_QK[r][s] e^{gc_r - gc_s})        -> bf16, smem
 //   Y    = (I + A)^{-1}  (16x16 diagonal blocks by forward substitution,
 //                          off-diagonal blocks with mma.sync TF32)
-//   T    = Y Diag(beta),  T' = T Diag(e^{gc})            -> bf16, smem
-//   U^T  = V^T T^T,  W^T = K^T T'^T        (tcgen05, M=128 N=64 K=64)
-//   V'^T = U^T + S_b (-W)^T                (tcgen05, A = S_b from TMEM)
-//   O^T  = (S_b Q^T) Diag(e^{gc}) + V'^T P^T   (tcgen05, two accumulators)
+//   T    = Y Diag(beta),  T' = T Diag(e^{gc})             -> bf16, smem
+//   Z    = S_b K^T                          (tcgen05, A = S_b from TMEM)
+//   V'^T = V^T T^T - Z T'^T                 (= U^T - S_b W^T with W = T' K)
+//   O^T  = (S_b Q^T) Diag(e^{gc}) + V'^T P^T
 //   S    = e^{gc_last} S + (V'^T Diag(e^{gc_last - gc})) K   (fp32 TMEM acc)
 //
-// S_b is the bf16 copy of the fp32 state, kept in TMEM as the A operand.
-// e^{gc_r - gc_s} is formed as e^{gc_r} e^{-gc_s} while the chunk's total
-// decay keeps e^{-gc} finite, else pairwise, so no scalar gate overflows.
+// W is never formed: S_b W^T = (S_b K^T) T'^T moves that product onto the
+// state side, where it costs one small MMA and one TMEM conversion.  S_b is
+// the bf16 copy of the fp32 state, kept in TMEM as the A operand.
 //
-// Warp roles (one CTA per (b, h), 320 threads):
-//   warps 0-3  "state" group: V'^T -> bf16 operands, O epilogue (direct stores),
-//              S -> S_b and the per-chunk state decay (TMEM lanes 0-127);
+// The fp32 state is held as S = sigma * S_tmem.  A chunk's decay only
+// changes sigma (and scales the next update by 1 / sigma), so S_tmem is
+// rewritten only when sigma falls below 2^-40, where the decay is folded
+// back into it; the bf16 copy is always formed at the true scale.
+//
+// Warp roles (one CTA per (b, h), 352 threads):
+//   warps 0-3  "state" group (TMEM lanes = value channels): -Z -> bf16 in
+//              TMEM, V'^T -> bf16 operands, S -> S_b, O epilogue (direct
+//              stores of o);
 //   warps 4-7  "prep" group, one chunk ahead: gate cumsum, A/P epilogue,
-//              (I + A)^{-1}, T/T', W^T -> bf16 operand;
-//   warp 8     TMA producer (two input stages, no multicast) + g/beta loads;
-//   warp 9     MMA issuer (one thread).
-// Hand-offs are mbarriers; every wait is bounded (time-out -> device status
-// word, abort flag, orderly unwind, TMEM freed).
+//              (I + A)^{-1} with T/T' written straight from it;
+//   warp 8     TMA producer of the K/Q stages (three) + g/beta loads;
+//   warp 9     state-side MMA issuer (one thread);
+//   warp 10    TMA producer of V (one stage);
+//   warp 11    prep-side MMA issuer (D1 and U^T = V^T T^T, one thread): an
+//              issue can stall while the tensor core's queue is full, which
+//              must not hold up the prep group.
+// No TMA load uses cluster multicast.  Hand-offs are mbarriers; every wait
+// is bounded (time-out -> device status word, abort flag, orderly unwind,
+// TMEM freed).
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -46,68 +57,77 @@ namespace {
 using namespace sm100;
 
 constexpr int C = 64, DK = 128, DV = 128;
-constexpr int kPrepWarps = 4;
-constexpr int kPrepThreads = 32 * kPrepWarps;
-constexpr int kThreads = 320;  // 4 state + 4 prep + producer + MMA warps
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kStages = 2;
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
-constexpr uint32_t kTileBytes = 64 * 128;    // one 64 x 64 bf16 tile
-constexpr uint32_t kStageTx = 6 * kTileBytes;
-constexpr float kSafeDecay = 80.f;  // e^{80} is finite in fp32
-// Row stride (floats) of the fp32 A/Y matrix: rows stay 16-byte aligned, and
-// mma.sync A-fragment loads hit distinct banks.
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kVWarp = 10, kPrepMmaWarp = 11;
+constexpr int kStages = 3;                    // K/Q stages
+constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
+constexpr uint32_t kTileBytes = 64 * 128;     // one 64 x 64 bf16 tile
+constexpr uint32_t kKQTx = 4 * kTileBytes, kVTx = 2 * kTileBytes;
+constexpr float kSafeDecay = 80.f;            // e^{80} is finite in fp32
+constexpr float kScaleFloor = 0x1p-40f;       // smallest state scale sigma kept
+// Per prep warp: [16][8] product scratch and [48][8] finished strip blocks.
+constexpr int kScrFloats = 16 * 8 + 48 * 8;
+// Row stride (floats) of the fp32 A matrix: rows stay 16-byte aligned and
+// 16 consecutive rows hit distinct 16-byte bank groups pairwise.
 constexpr int LDA = 68;
 
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
 struct Lay {
   static constexpr uint32_t KQ = 0;                             // per stage [K_h0|Q_h0|K_h1|Q_h1]
-  static constexpr uint32_t V = KQ + kStages * 4 * kTileBytes;  // per stage [V_h0|V_h1]
-  static constexpr uint32_t T = V + kStages * 2 * kTileBytes;   // T   K-major [r][s]
-  static constexpr uint32_t TP = T + kTileBytes;                // T'  K-major [r][s]
-  static constexpr uint32_t P = TP + kTileBytes;                // P   K-major [r][s], x2
-  static constexpr uint32_t WT = P + 2 * kTileBytes;            // -W^T MN-major [dk][C]
-  static constexpr uint32_t VP = WT + 2 * kTileBytes;           // V'^T K-major [dv][C]
-  static constexpr uint32_t VPD = VP + 2 * kTileBytes;          // decayed V'^T
-  static constexpr uint32_t AF = VPD + 2 * kTileBytes;          // fp32 A, then Y [64][LDA]
-  static constexpr uint32_t SCR = AF + 64 * LDA * 4;            // fp32 inverse scratch 4 x [16][8]
-  static constexpr uint32_t GS = SCR + 4 * 128 * 4;             // per stage g[64], beta[64]
-  static constexpr uint32_t VEC = GS + kStages * 512;           // x3: gc, eg, ieg, egl [64] each
-  static constexpr uint32_t SVEC = VEC + 3 * 1024;              // x2: eg, egl [64] (state group)
+  static constexpr uint32_t V = KQ + kStages * 4 * kTileBytes;  // [V_h0|V_h1]
+  static constexpr uint32_t T = V + 2 * kTileBytes;             // T  K-major [r][s]
+  static constexpr uint32_t TP = T + kTileBytes;                // T' K-major [r][s], x2
+  static constexpr uint32_t P = TP + 2 * kTileBytes;            // P  K-major [r][s], x2
+  static constexpr uint32_t VP = P + 2 * kTileBytes;            // V'^T K-major [dv][C]
+  static constexpr uint32_t VPD = VP + 2 * kTileBytes;          // decayed, rescaled V'^T
+  static constexpr uint32_t AF = VPD + 2 * kTileBytes;          // fp32 A, diagonal blocks -> D
+  static constexpr uint32_t SCR = AF + 64 * LDA * 4;            // 4 x kScrFloats fp32
+  static constexpr uint32_t GS = SCR + 4 * kScrFloats * 4;      // per stage g[64], beta[64]
+  static constexpr uint32_t VEC = GS + kStages * 512;           // x2 (prep): gc, eg, ieg [64]
+  static constexpr uint32_t SVEC = VEC + 2 * 1024;              // x2 (state): eg, egl [64]
   static constexpr uint32_t BAR = SVEC + 2 * 512;               // mbarriers
-  static constexpr uint32_t MISC = BAR + 16 * 8;                // tmem base, abort flag, consumed
+  static constexpr uint32_t MISC = BAR + 32 * 8;                // tmem base, abort flag
   static constexpr uint32_t END = MISC + 16;
 };
-static_assert(Lay::AF % 1024 == 0, "tile alignment");
+static_assert(Lay::V % 1024 == 0 && Lay::T % 1024 == 0 && Lay::VPD % 1024 == 0 &&
+                  Lay::AF % 1024 == 0,
+              "tile alignment");
 constexpr size_t kSmemBytes = Lay::END + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // mbarrier slots
 enum {
-  B_FULL = 0,   // [2] TMA + g/beta of a stage landed          (count 1 + tx)
-  B_EMPTY = 2,  // [2] stage may be refilled: MMA commit + prep  (count 2)
-  B_D1F = 4,    // D1 written                                   (commit)
-  B_D1E,        // D1 read by the prep group                    (256)
-  B_TRDY,       // T, T', P, gate vectors of a chunk ready      (256)
-  B_WTF,        // U^T, W^T written                             (commit)
-  B_WTB,        // -W^T bf16 operand written                    (256)
-  B_SBR,        // S_b in TMEM and the decayed S ready          (128)
-  B_VPF,        // V'^T and O_a written                         (commit)
-  B_VPR,        // V'^T bf16 operands written                   (128)
-  B_SF,         // the updated S written                        (commit)
-  B_OF,         // O_a and O_b written                          (commit)
-  B_FIN,        // final drain of the MMA pipe                  (commit)
+  B_FULL = 0,          // [3] K/Q + g/beta of a stage landed            (1 + tx)
+  B_EMPTY = 3,         // [3] K/Q stage free (state MMA commit)         (commit)
+  B_VFULL = 6,         // V landed                                      (1 + tx)
+  B_VEMPTY,            // V free (prep commit after U)                  (commit)
+  B_D1F,               // D1 written                                    (commit, prep side)
+  B_D1E,               // D1 read by the prep group                     (1)
+  B_TRDY,              // T, T' and P of a chunk written                (1)
+  B_UF,                // U^T written (T read)                          (commit, prep side)
+  B_ZF,                // Z written                                     (commit)
+  B_ZR,                // -Z bf16 operand in TMEM                       (128)
+  B_VPF,               // V'^T complete                                 (commit)
+  B_VPR,               // V'^T bf16 operands in smem                    (128)
+  B_SF,                // state update complete                         (commit)
+  B_OF,                // O_a, O_b complete                             (commit)
+  B_SBR,               // S_b in TMEM for the next chunk                (128)
+  B_OE,                // O_a, O_b read by the epilogue                 (128)
+  B_PE,                // [2] P buffer free (after O_b)                 (commit)
+  B_TPE = B_PE + 2,    // [2] T' buffer free (after V')                 (commit)
+  B_FIN = B_TPE + 2,   // final drain, state-side issuer                (commit)
+  B_FIN2,              // final drain, prep-side issuer                 (commit)
   B_COUNT
 };
+static_assert(B_COUNT <= 32, "barrier slots");
 
 // TMEM column map (512 allocated; 1 CTA per SM).
-constexpr uint32_t TM_S = 0, TM_SB = 128, TM_D1 = 192, TM_UV = 256, TM_WT = 320, TM_O = 384,
-                   TM_OA = 448;
+constexpr uint32_t TM_S = 0, TM_SB = 128, TM_Z = 192, TM_UV = 256, TM_O = 320, TM_OA = 384,
+                   TM_D1 = 448;
 
 constexpr uint32_t ID_D1 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t ID_U = idesc_bf16(128, 64, 1, 0);
-constexpr uint32_t ID_VP = idesc_bf16(128, 64, 0, 1);
-constexpr uint32_t ID_O = idesc_bf16(128, 64, 0, 0);
+constexpr uint32_t ID_N64 = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t ID_S = idesc_bf16(128, 128, 0, 1);
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -158,7 +178,7 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   }
 }
 
-__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16]) {
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t *v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
       "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
@@ -178,27 +198,19 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// Warp-group barriers: id 2 = state group (128 threads), id 3 = prep group
-// (kPrepThreads).
-__device__ __forceinline__ uint32_t group_threads(uint32_t bar_id) {
-  return bar_id == 3 ? (uint32_t)kPrepThreads : 128u;
-}
-
-// Barrier over one warp group that also ORs a predicate.
+// Warp-group barriers (128 threads each): id 2 = state group, id 3 = prep.
 __device__ __forceinline__ bool group_any(uint32_t bar_id, bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      "bar.red.or.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)pred), "r"(bar_id), "r"(group_threads(bar_id))
+      : "r"((uint32_t)pred), "r"(bar_id)
       : "memory");
   return r != 0;
 }
 
-__device__ __forceinline__ void group_bar(uint32_t bar_id) {
-  named_bar_sync(bar_id, group_threads(bar_id));
-}
+__device__ __forceinline__ void group_bar(uint32_t bar_id) { named_bar_sync(bar_id, 128); }
 
 // Bounded wait that also gives up as soon as another role has aborted.
 // The thread sleeps inside try_wait (suspend hint) between checks.
@@ -216,15 +228,42 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
   return true;
 }
 
-// Group-wide wait: lane 0 of each warp polls, the warp shares its result,
-// and the group agrees (any failure -> every thread sees failure).
+// Group-wide wait and abort check: lane 0 of each warp polls, the warp
+// shares its result, and the group agrees (any failure, or an abort raised
+// anywhere in the CTA, -> every thread sees failure).
 __device__ __forceinline__ bool group_wait(uint32_t bar_id, uint64_t *bar, uint32_t parity,
                                            volatile int *abort_flag, int lane) {
   bool ok = true;
-  if (lane == 0) ok = wait_or_abort(bar, parity, abort_flag);
+  if (lane == 0) ok = wait_or_abort(bar, parity, abort_flag) && !*abort_flag;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return !group_any(bar_id, !ok);
 }
+
+// One warp: cumulative log decay of a chunk (g[64] -> gc[64] in log space,
+// inclusive prefix sum) held as lanes r and r + 32; returns the chunk total.
+__device__ __forceinline__ float chunk_cumsum(const float *g, int lane, float &x0, float &x1) {
+  x0 = g[lane];
+  x1 = g[lane + 32];
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+    const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+    if (lane >= off) {
+      x0 += y0;
+      x1 += y1;
+    }
+  }
+  x1 += __shfl_sync(0xffffffffu, x0, 31);
+  return __shfl_sync(0xffffffffu, x1, 31);
+}
+
+// ---------------------------------------------------------------- inverse
+// Output of the inverse: T = Y Diag(beta) and T' = T Diag(e^{gc}) as bf16
+// K-major 128B-swizzled tiles [r][s].
+struct TOut {
+  uint8_t *t, *tp;
+  const float *beta, *eg;  // [64]
+};
 
 __device__ __forceinline__ uint32_t to_tf32(float x) {
   uint32_t r;
@@ -242,8 +281,7 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
-// Helpers of the blocked inverse below (one warp, mma.sync m16n8k8 TF32
-// fragments: g = lane / 4, tq = lane % 4).
+// mma.sync m16n8k8 TF32 fragments of one warp (g = lane / 4, tq = lane % 4).
 struct Frag {
   int g, tq;
   float *scr;  // warp-private [16][8] fp32 scratch
@@ -270,29 +308,50 @@ struct Frag {
   }
 };
 
-// One 8-column strip (first column `col`) of column block J of Y = (I + A)^{-1}:
-// Y_JJ = D_JJ (already in AF), Y_bJ = -D_bb sum_{k=J}^{b-1} A_bk Y_kJ for
-// b > J, swept down the block rows; the finished blocks stay in `yout[b]`.
-// J is a template parameter so that every loop is fully static.
-template <int J>
-__device__ __forceinline__ void inverse_strip(const float *AF, const Frag &f, int col,
-                                              float (&yout)[4][4]) {
-  uint32_t yb[4][2][2];
+// Two adjacent columns s, s + 1 (s even) of row r of T and T'.
+__device__ __forceinline__ void store_t2(const TOut &o, int r, int s, float y0, float y1) {
+  const float2 b = *reinterpret_cast<const float2 *>(o.beta + s);
+  const float2 e = *reinterpret_cast<const float2 *>(o.eg + s);
+  const float t0 = y0 * b.x, t1 = y1 * b.y;
+  const uint32_t off = sw128_off(r, s);
+  *reinterpret_cast<uint32_t *>(o.t + off) = pack_bf16(t0, t1);
+  *reinterpret_cast<uint32_t *>(o.tp + off) = pack_bf16(t0 * e.x, t1 * e.y);
+}
+
+// B fragments (two k-steps) of a 16x8 fp32 block stored row-major with
+// row stride `ld` floats.
+__device__ __forceinline__ void load_bfrag(const float *blk, int ld, const Frag &f,
+                                           uint32_t (&bf)[2][2]) {
 #pragma unroll
   for (int ks = 0; ks < 2; ++ks) {
-    yb[J][ks][0] = to_tf32(AF[(16 * J + 8 * ks + f.tq) * LDA + col + f.g]);
-    yb[J][ks][1] = to_tf32(AF[(16 * J + 8 * ks + f.tq + 4) * LDA + col + f.g]);
+    bf[ks][0] = to_tf32(blk[(8 * ks + f.tq) * ld + f.g]);
+    bf[ks][1] = to_tf32(blk[(8 * ks + f.tq + 4) * ld + f.g]);
   }
-#pragma unroll
-  for (int bb = J + 1; bb < 4; ++bb) {
+}
+
+// One 8-column strip (first column col0) of column block j of
+// Y = (I + A)^{-1}.  With D_bb = (I + A_bb)^{-1} already in the diagonal
+// blocks of AF:  Y_jj = D_jj,  Y_bj = -D_bb sum_{k=j}^{b-1} A_bk Y_kj (b > j),
+// swept down the block rows with mma.sync (TF32 operands rounded to
+// nearest, fp32 accumulation).  Finished blocks go to the warp's scratch
+// `ys` ([48][8], block row b at rows 16 (b - j - 1)) for the rows below,
+// and, scaled, to T and T'.  Runtime loops keep the code small: every warp
+// of the SM runs it each chunk next to the state group's code.
+__device__ __forceinline__ void inverse_strip(const float *AF, float *ys, const Frag &f,
+                                              const TOut &o, int j, int col0) {
+#pragma unroll 1
+  for (int bb = j + 1; bb < 4; ++bb) {
     float racc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int k = J; k < bb; ++k) {
+#pragma unroll 1
+    for (int k = j; k < bb; ++k) {
+      const float *yblk = (k == j) ? AF + (16 * j) * LDA + col0 : ys + 16 * (k - j - 1) * 8;
+      uint32_t bf[2][2];
+      load_bfrag(yblk, (k == j) ? LDA : 8, f, bf);
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
         uint32_t af[4];
         f.a(AF, 16 * bb, 16 * k + 8 * ks, af);
-        mma_tf32_16x8x8(racc, af, yb[k][ks]);
+        mma_tf32_16x8x8(racc, af, bf[ks]);
       }
     }
     uint32_t rb[2][2];
@@ -304,37 +363,29 @@ __device__ __forceinline__ void inverse_strip(const float *AF, const Frag &f, in
       f.a(AF, 16 * bb, 16 * bb + 8 * ks, af);
       mma_tf32_16x8x8(yacc, af, rb[ks]);
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) yout[bb][e] = -yacc[e];
-    if (bb < 3) f.to_b(yout[bb], yb[bb]);
+    const float y0 = -yacc[0], y1 = -yacc[1], y2 = -yacc[2], y3 = -yacc[3];
+    float *yo = ys + 16 * (bb - j - 1) * 8;
+    yo[f.g * 8 + 2 * f.tq] = y0;
+    yo[f.g * 8 + 2 * f.tq + 1] = y1;
+    yo[(f.g + 8) * 8 + 2 * f.tq] = y2;
+    yo[(f.g + 8) * 8 + 2 * f.tq + 1] = y3;
+    __syncwarp();
+    store_t2(o, 16 * bb + f.g, col0 + 2 * f.tq, y0, y1);
+    store_t2(o, 16 * bb + f.g + 8, col0 + 2 * f.tq, y2, y3);
   }
 }
 
-template <int J>
-__device__ __forceinline__ void store_strip(float *AF, const Frag &f, int col,
-                                            const float (&yout)[4][4]) {
-#pragma unroll
-  for (int bb = J + 1; bb < 4; ++bb) {
-    AF[(16 * bb + f.g) * LDA + col + 2 * f.tq] = yout[bb][0];
-    AF[(16 * bb + f.g) * LDA + col + 2 * f.tq + 1] = yout[bb][1];
-    AF[(16 * bb + f.g + 8) * LDA + col + 2 * f.tq] = yout[bb][2];
-    AF[(16 * bb + f.g + 8) * LDA + col + 2 * f.tq + 1] = yout[bb][3];
-  }
-}
-
-// (I + A)^{-1} in place for a strictly lower 64x64 fp32 matrix A (row stride
-// LDA, zero above the diagonal blocks) with the 4-warp prep group (local
-// thread t, warp w = t / 32), in 16x16 blocks:
-//  1. diagonal blocks D_bb = (I + A_bb)^{-1} by forward substitution (warp b);
-//  2. every 8-column strip of a column block is independent, so each warp
-//     sweeps its strips down the block rows with mma.sync (TF32 operands
-//     rounded to nearest, fp32 accumulation);
-//  3. after a group barrier the off-diagonal blocks overwrite A.
-// Strips (column block j, half hf): warp 0 -> (0,0); warp 1 -> (0,1);
-// warp 2 -> (1,0), (2,0); warp 3 -> (1,1), (2,1).  (The measured in-kernel
-// time of this form beat an fp32 CUDA-core strip sweep, although mma.sync
-// queues behind concurrent tcgen05 work.)
-__device__ void invert_unit_lower(float *AF, float *R, int t, uint32_t bar_id) {
+// (I + A)^{-1} for the strictly lower 64x64 fp32 A in AF (row stride LDA,
+// zero above the diagonal) with the 4-warp prep group (local thread t),
+// written as T and T' (their blocks above the block diagonal stay zero from
+// the kernel's start):
+//  1. warp b: D_bb = (I + A_bb)^{-1} by forward substitution (lane c % 16
+//     owns column c), stored over A_bb in AF and, scaled, into T and T';
+//  2. strips (column block j, half hf): warp 0 -> (0,0); warp 1 -> (0,1);
+//     warp 2 -> (1,0), (2,0); warp 3 -> (1,1), (2,1).  (An fp32 CUDA-core
+//     strip sweep was faster alone but, competing for issue slots with the
+//     state group, slower in the kernel.)
+__device__ void invert_to_t(float *AF, float *scr, const TOut &o, int t, uint32_t bar_id) {
   const int warp = t >> 5, lane = t & 31;
   {
     const int w = warp, c = lane & 15;
@@ -344,60 +395,49 @@ __device__ void invert_unit_lower(float *AF, float *R, int t, uint32_t bar_id) {
     const float *Ab = AF + (16 * w) * LDA + 16 * w;
 #pragma unroll
     for (int i = 1; i < 16; ++i) {
-      float acc = 0.f;
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
       for (int k4 = 0; k4 < (i + 3) / 4; ++k4) {
         const float4 av = *reinterpret_cast<const float4 *>(Ab + i * LDA + 4 * k4);
-        if (4 * k4 + 0 < i) acc += av.x * x[4 * k4 + 0];
-        if (4 * k4 + 1 < i) acc += av.y * x[4 * k4 + 1];
-        if (4 * k4 + 2 < i) acc += av.z * x[4 * k4 + 2];
-        if (4 * k4 + 3 < i) acc += av.w * x[4 * k4 + 3];
+        if (4 * k4 + 0 < i) acc0 += av.x * x[4 * k4 + 0];
+        if (4 * k4 + 1 < i) acc1 += av.y * x[4 * k4 + 1];
+        if (4 * k4 + 2 < i) acc0 += av.z * x[4 * k4 + 2];
+        if (4 * k4 + 3 < i) acc1 += av.w * x[4 * k4 + 3];
       }
-      x[i] = (i > c) ? -acc : x[i];
+      x[i] = (i > c) ? -(acc0 + acc1) : x[i];
     }
-    __syncwarp();
+    __syncwarp();  // every lane has read A_ww
     if (lane < 16) {
       float *Yb = AF + (16 * w) * LDA + 16 * w;
 #pragma unroll
       for (int i = 0; i < 16; ++i) Yb[i * LDA + c] = x[i];
     }
-  }
-  group_bar(bar_id);
-  const Frag f{lane >> 2, lane & 3, R + warp * 128};
-  const int hf = warp & 1;
-  float y0[4][4], y1[4][4];
-  if (warp < 2) {
-    inverse_strip<0>(AF, f, 8 * hf, y0);
-  } else {
-    inverse_strip<1>(AF, f, 16 + 8 * hf, y0);
-    inverse_strip<2>(AF, f, 32 + 8 * hf, y1);
-  }
-  group_bar(bar_id);  // every read of A is done: store the off-diagonal blocks
-  if (warp < 2) {
-    store_strip<0>(AF, f, 8 * hf, y0);
-  } else {
-    store_strip<1>(AF, f, 16 + 8 * hf, y0);
-    store_strip<2>(AF, f, 32 + 8 * hf, y1);
-  }
-  group_bar(bar_id);
-}
-
-// One warp: cumulative log decay of a chunk (g[64] -> gc[64] in log space,
-// inclusive prefix sum) held as lanes r and r + 32; returns the chunk total.
-__device__ __forceinline__ float chunk_cumsum(const float *g, int lane, float &x0, float &x1) {
-  x0 = g[lane];
-  x1 = g[lane + 32];
+    // T (lanes 0-15) and T' (lanes 16-31) of the diagonal block: lanes c and
+    // c ^ 1 pair up so that each writes two adjacent columns of every other
+    // row.
+    const int col = 16 * w + c;
+    const float sc = (lane < 16) ? o.beta[col] : o.beta[col] * o.eg[col];
+    uint8_t *tile = (lane < 16) ? o.t : o.tp;
+    const int odd = c & 1;
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
-    const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
-    if (lane >= off) {
-      x0 += y0;
-      x1 += y1;
+    for (int i = 0; i < 16; ++i) {
+      const float mine = x[i] * sc;
+      const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+      if ((i & 1) == odd) {
+        const uint32_t v = odd ? pack_bf16(other, mine) : pack_bf16(mine, other);
+        *reinterpret_cast<uint32_t *>(tile + sw128_off(16 * w + i, col & ~1)) = v;
+      }
     }
   }
-  x1 += __shfl_sync(0xffffffffu, x0, 31);
-  return __shfl_sync(0xffffffffu, x1, 31);
+  group_bar(bar_id);
+  float *ws = scr + warp * kScrFloats;  // [16][8] product scratch, then [48][8] strip blocks
+  const Frag f{lane >> 2, lane & 3, ws};
+  const int hf = warp & 1;
+#pragma unroll 1
+  for (int si = 0; si < (warp < 2 ? 1 : 2); ++si) {
+    const int j = warp < 2 ? 0 : 1 + si;
+    inverse_strip(AF, ws + 128, f, o, j, 16 * j + 8 * hf);
+  }
 }
 
 #ifdef GDR_TC_DEBUG
@@ -415,8 +455,8 @@ __device__ int g_dbg_chunk = 0;
   } while (0)
 #endif
 
-// Each SM sub-partition holds a quarter of the register file and up to three
-// of the block's ten warps: the launch bound caps registers at 168.
+// Each SM sub-partition holds a quarter of the register file and three of
+// the block's twelve warps: the launch bound caps registers at 168.
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -432,29 +472,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lay::MISC + 4);
-  volatile int *consumed = reinterpret_cast<volatile int *>(sm + Lay::MISC + 8);
   float *AF = reinterpret_cast<float *>(sm + Lay::AF);
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars[B_FULL + s], 1);
-      mbar_init(&bars[B_EMPTY + s], 2);
+      mbar_init(&bars[B_EMPTY + s], 1);
     }
+    mbar_init(&bars[B_VFULL], 1);
+    mbar_init(&bars[B_VEMPTY], 1);
     mbar_init(&bars[B_D1F], 1);
-    mbar_init(&bars[B_D1E], kPrepThreads);
-    mbar_init(&bars[B_TRDY], kPrepThreads);
-    mbar_init(&bars[B_WTF], 1);
-    mbar_init(&bars[B_WTB], kPrepThreads);
-    mbar_init(&bars[B_SBR], 128);
+    mbar_init(&bars[B_D1E], 1);
+    mbar_init(&bars[B_TRDY], 1);
+    mbar_init(&bars[B_UF], 1);
+    mbar_init(&bars[B_ZF], 1);
+    mbar_init(&bars[B_ZR], 128);
     mbar_init(&bars[B_VPF], 1);
     mbar_init(&bars[B_VPR], 128);
     mbar_init(&bars[B_SF], 1);
     mbar_init(&bars[B_OF], 1);
+    mbar_init(&bars[B_SBR], 128);
+    mbar_init(&bars[B_OE], 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[B_PE + s], 1);
+      mbar_init(&bars[B_TPE + s], 1);
+    }
     mbar_init(&bars[B_FIN], 1);
+    mbar_init(&bars[B_FIN2], 1);
     *abort_flag = 0;
-    *consumed = 0;
     fence_mbar_init();
   }
+  // T and both T' tiles start at zero: their blocks above the block diagonal
+  // are never written afterwards.
+  for (uint32_t off = 16 * tid; off < 3 * kTileBytes; off += 16 * kThreads)
+    *reinterpret_cast<uint4 *>(sm + Lay::T + off) = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -466,18 +518,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t lane_base = tm + ((uint32_t)((warp & 3) * 32) << 16);
 
   if (warp == kProducerWarp) {
-    // ================================================================ producer
+    // ================================================================ K/Q producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
     }
-    int last_issued[kStages] = {-1, -1};  // latest chunk loaded into each stage
+    int last_issued[kStages] = {-1, -1, -1};  // latest chunk loaded into each stage
     for (int c = 0; c < n; ++c) {
-      const int s = c & 1;
+      const int s = c % kStages;
       if (c >= kStages) {
         bool ok = true;
-        if (lane == 0) ok = wait_or_abort(&bars[B_EMPTY + s], ((c >> 1) - 1) & 1, abort_flag);
+        if (lane == 0)
+          ok = wait_or_abort(&bars[B_EMPTY + s], ((c / kStages) - 1) & 1, abort_flag);
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
       // Testing hook: this chunk's load is never issued, so its consumers'
@@ -495,42 +547,119 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         uint64_t *fb = &bars[B_FULL + s];
-        mbar_arrive_expect_tx(fb, kStageTx);
+        mbar_arrive_expect_tx(fb, kKQTx);
         uint8_t *kq = sm + Lay::KQ + s * 4 * kTileBytes;
-        uint8_t *vv = sm + Lay::V + s * 2 * kTileBytes;
         tma_load_4d(kq + 0 * kTileBytes, &tmK, fb, 0, h, t0, b);
         tma_load_4d(kq + 1 * kTileBytes, &tmQ, fb, 0, h, t0, b);
         tma_load_4d(kq + 2 * kTileBytes, &tmK, fb, 64, h, t0, b);
         tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, t0, b);
-        tma_load_4d(vv + 0 * kTileBytes, &tmV, fb, 0, h, t0, b);
-        tma_load_4d(vv + 1 * kTileBytes, &tmV, fb, 64, h, t0, b);
       }
       last_issued[s] = c;
     }
-    // A load issued but never consumed exists only after an abort: let it land
-    // before the CTA exits.
+    // Loads still in flight after an abort land before the CTA exits (a
+    // phase that has already completed passes at once).
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) {
         const int c = last_issued[s];
-        if (c >= 0 && c >= *consumed)
-          mbar_wait_bounded(&bars[B_FULL + s], (c >> 1) & 1, kWaitNs);
+        if (c >= 0) mbar_wait_bounded(&bars[B_FULL + s], (c / kStages) & 1, kWaitNs);
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ================================================================ MMA issuer
+  } else if (warp == kVWarp) {
+    // ================================================================ V producer
     if (lane == 0) {
-      const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_v = smem_u32(sm + Lay::V);
-      const uint32_t a_t = smem_u32(sm + Lay::T), a_tp = smem_u32(sm + Lay::TP);
-      const uint32_t a_p = smem_u32(sm + Lay::P), a_wt = smem_u32(sm + Lay::WT);
+      tma_prefetch_desc(&tmV);
+      int last = -1;
+      for (int c = 0; c < n; ++c) {
+        if (c >= 1 && !wait_or_abort(&bars[B_VEMPTY], (c - 1) & 1, abort_flag)) break;
+        uint8_t *vv = sm + Lay::V;
+        mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
+        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, c * C, b);
+        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, c * C, b);
+        last = c;
+      }
+      if (last >= 0) mbar_wait_bounded(&bars[B_VFULL], last & 1, kWaitNs);
+    }
+  } else if (warp == kMmaWarp) {
+    // ================================================================ state-side MMAs
+    if (lane == 0) {
+      const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_tp = smem_u32(sm + Lay::TP);
+      const uint32_t a_p = smem_u32(sm + Lay::P);
       const uint32_t a_vp = smem_u32(sm + Lay::VP), a_vpd = smem_u32(sm + Lay::VPD);
       auto W = [&](int slot, uint32_t parity) {
         const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
         tc_fence_after();
         return ok;
       };
+      // Each barrier completes once per chunk (per buffer for PE / TPE) and
+      // is waited on by parity, so no arrival may run two phases ahead of
+      // its waiter: every producer of a phase first depends, directly or
+      // through this thread's program order, on its consumer's previous one.
+      bool ok = true;
+      for (int c = 0; c < n && ok; ++c) {
+        const uint32_t ph = c & 1;
+        const int st = c % kStages;
+        const uint32_t kq = a_kq + st * 4 * kTileBytes;
+        // Z = S_b K^T
+        if (!(ok = W(B_SBR, ph) && W(B_FULL + st, (c / kStages) & 1))) break;
+#pragma unroll 1
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tm + TM_Z, tm + TM_SB + 8 * kk,
+                      sdesc_sw128(kq + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32, 16, 1024),
+                      ID_N64, kk > 0);
+        mma_commit(&bars[B_ZF]);
+        // V'^T = U^T + (-Z) T'^T   (U^T from the prep-side issuer)
+        if (!(ok = W(B_ZR, ph) && W(B_UF, ph))) break;
+        const uint32_t tp = a_tp + (c & 1) * kTileBytes;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ts(tm + TM_UV, tm + TM_Z + 8 * kk, sdesc_sw128(tp + kk * 32, 16, 1024), ID_N64,
+                      1);
+        mma_commit(&bars[B_VPF]);
+        mma_commit(&bars[B_TPE + (c & 1)]);
+        // O_a = S_b Q^T, once the epilogue has read the previous chunk's O.
+        // Issued before the SF commit, which then also covers this last read
+        // of S_b (the state group overwrites S_b once SF completes).
+        if (c >= 1 && !(ok = W(B_OE, (c - 1) & 1))) break;
+#pragma unroll 1
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tm + TM_OA, tm + TM_SB + 8 * kk,
+                      sdesc_sw128(kq + kTileBytes + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32,
+                                  16, 1024),
+                      ID_N64, kk > 0);
+        // S_tmem += (V'^T decayed / sigma) K ;  O_b = V'^T P^T
+        if (!(ok = W(B_VPR, ph))) break;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tm + TM_S, sdesc_sw128(a_vpd + kk * 32, 16, 1024),
+                      sdesc_sw128(kq + kk * 2048, 2 * kTileBytes, 1024), ID_S, 1);
+        mma_commit(&bars[B_SF]);
+        const uint32_t pp = a_p + (c & 1) * kTileBytes;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tm + TM_O, sdesc_sw128(a_vp + kk * 32, 16, 1024),
+                      sdesc_sw128(pp + kk * 32, 16, 1024), ID_N64, kk > 0);
+        mma_commit(&bars[B_OF]);
+        mma_commit(&bars[B_PE + (c & 1)]);
+        mma_commit(&bars[B_EMPTY + st]);
+      }
+      // Drain: all issued MMAs complete before TMEM is released.
+      mma_commit(&bars[B_FIN]);
+      mbar_wait_bounded(&bars[B_FIN], 0, kWaitNs);
+      if (!ok) atomicOr(a.status, kStatusTimeout);
+    }
+  } else if (warp == kPrepMmaWarp) {
+    // ================================================================ prep-side MMAs
+    if (lane == 0) {
+      const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_v = smem_u32(sm + Lay::V);
+      const uint32_t a_t = smem_u32(sm + Lay::T);
+      auto W = [&](int slot, uint32_t parity) {
+        const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
+        tc_fence_after();
+        return ok;
+      };
       auto issue_d1 = [&](int c) {  // D1 = [K; Q] K^T
-        const uint32_t kq = a_kq + (c & 1) * 4 * kTileBytes;
-#pragma unroll
+        const uint32_t kq = a_kq + (c % kStages) * 4 * kTileBytes;
+#pragma unroll 1
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32;
           mma_bf16_ss(tm + TM_D1, sdesc_sw128(kq + off, 16, 1024),
@@ -538,118 +667,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars[B_D1F]);
       };
-      auto issue_uw = [&](int c) {  // U^T = V^T T^T, W^T = K^T T'^T
-        const uint32_t kq = a_kq + (c & 1) * 4 * kTileBytes;
-        const uint32_t vv = a_v + (c & 1) * 2 * kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16_ss(tm + TM_UV, sdesc_sw128(vv + kk * 2048, kTileBytes, 1024),
+      // D1 of chunk c + 1 goes out as soon as the prep group has read D1 of
+      // chunk c; U^T of chunk c once T is written and the state group has
+      // converted the previous V'^T (the accumulator is shared).
+      bool ok = W(B_FULL, 0);
+      if (ok) issue_d1(0);
+      for (int c = 0; c < n && ok; ++c) {
+        if (c + 1 < n) {
+          if (!(ok = W(B_D1E, c & 1) &&
+                     W(B_FULL + (c + 1) % kStages, ((c + 1) / kStages) & 1)))
+            break;
+          issue_d1(c + 1);
+        }
+        if (!(ok = W(B_TRDY, c & 1) && (c < 1 || W(B_VPR, (c - 1) & 1)) && W(B_VFULL, c & 1)))
+          break;
+#pragma unroll 1
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tm + TM_UV, sdesc_sw128(a_v + kk * 2048, kTileBytes, 1024),
                       sdesc_sw128(a_t + kk * 32, 16, 1024), ID_U, kk > 0);
-          mma_bf16_ss(tm + TM_WT, sdesc_sw128(kq + kk * 2048, 2 * kTileBytes, 1024),
-                      sdesc_sw128(a_tp + kk * 32, 16, 1024), ID_U, kk > 0);
-        }
-        mma_commit(&bars[B_WTF]);
-      };
-      bool ok = true;
-      do {
-        if (!(ok = W(B_FULL, 0))) break;
-        issue_d1(0);
-        if (!(ok = W(B_TRDY, 0))) break;
-        issue_uw(0);
-        if (n > 1) {
-          if (!(ok = W(B_D1E, 0) && W(B_FULL + 1, 0))) break;
-          issue_d1(1);
-        }
-        // Each barrier completes once per chunk and is waited on by parity,
-        // so no arrival may run two phases ahead of its waiter: every
-        // producer of a phase first waits, directly or through this thread's
-        // program order, for its consumer's previous phase.
-        for (int c = 0; c < n && ok; ++c) {
-          const uint32_t ph = c & 1;
-          const uint32_t kq = a_kq + (c & 1) * 4 * kTileBytes;
-          // V'^T = U^T + S_b (-W)^T
-          if (!(ok = W(B_WTB, ph) && W(B_SBR, ph))) break;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            mma_bf16_ts(tm + TM_UV, tm + TM_SB + 8 * kk,
-                        sdesc_sw128(a_wt + kk * 2048, 2 * kTileBytes, 1024), ID_VP, 1);
-          }
-          mma_commit(&bars[B_VPF]);
-          // O_a = S_b Q^T ;  S += (V'^T decayed) K ;  O_b = V'^T P^T.  O_a is
-          // issued before the SF commit: SF then also covers the last read
-          // of S_b, which the state group overwrites once SF completes.
-          if (!(ok = W(B_VPR, ph))) break;
-          const uint32_t pp = a_p + (c & 1) * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t boff = kTileBytes + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32;
-            mma_bf16_ts(tm + TM_OA, tm + TM_SB + 8 * kk, sdesc_sw128(kq + boff, 16, 1024), ID_O,
-                        kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_ss(tm + TM_S, sdesc_sw128(a_vpd + kk * 32, 16, 1024),
-                        sdesc_sw128(kq + kk * 2048, 2 * kTileBytes, 1024), ID_S, 1);
-          }
-          mma_commit(&bars[B_SF]);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_bf16_ss(tm + TM_O, sdesc_sw128(a_vp + kk * 32, 16, 1024),
-                        sdesc_sw128(pp + kk * 32, 16, 1024), ID_O, kk > 0);
-          }
-          mma_commit(&bars[B_OF]);
-          mma_commit(&bars[B_EMPTY + (c & 1)]);
-          *consumed = c + 1;
-          if (c + 1 < n) {
-            if (!(ok = W(B_TRDY, (c + 1) & 1))) break;
-            issue_uw(c + 1);
-          }
-          if (c + 2 < n) {
-            if (!(ok = W(B_D1E, (c + 1) & 1) && W(B_FULL + (c & 1), ((c + 2) >> 1) & 1))) break;
-            issue_d1(c + 2);
-          }
-        }
-      } while (0);
-      // Drain: all issued MMAs complete before TMEM is released.
-      mma_commit(&bars[B_FIN]);
-      mbar_wait_bounded(&bars[B_FIN], 0, kWaitNs);
+        mma_commit(&bars[B_UF]);
+        mma_commit(&bars[B_VEMPTY]);
+      }
+      mma_commit(&bars[B_FIN2]);
+      mbar_wait_bounded(&bars[B_FIN2], 0, kWaitNs);
       if (!ok) atomicOr(a.status, kStatusTimeout);
     }
-  } else if (warp >= 4 && warp < 4 + kPrepWarps) {
+  } else if (warp >= 4 && warp < 8) {
     // ================================================================ prep group
-    // TMEM lane rl = pt; each thread handles both 32-column halves hp of
-    // its 64-column rows.
-    const int pt = tid - 128, rl = pt & 127, hp0 = 0, pw = pt >> 5;
-    constexpr int kHalfStep = 1;
+    const int pt = tid - 128, rl = pt, pw = pt >> 5;
     const int lrow = rl;
     (void)lrow;
     constexpr uint32_t kBar = 3;
+    bool ok = true;
     for (int c = 0; c < n; ++c) {
-      const int s = c & 1;
+      const int st = c % kStages;
       const uint32_t ph = c & 1;
-      float *vec = reinterpret_cast<float *>(sm + Lay::VEC + (c % 3) * 1024);
-      float *gcv = vec, *egv = vec + 64, *iegv = vec + 128, *eglv = vec + 192;
-      if (!group_wait(kBar, &bars[B_FULL + s], (c >> 1) & 1, abort_flag, lane)) break;
-      const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + s * 512);
+      float *vec = reinterpret_cast<float *>(sm + Lay::VEC + (c & 1) * 1024);
+      float *gcv = vec, *egv = vec + 64, *iegv = vec + 128;
+      if (!(ok = group_wait(kBar, &bars[B_FULL + st], (c / kStages) & 1, abort_flag, lane))) break;
+      const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + st * 512);
       const float *bs = gs + 64;
       if (pw == 0) {  // cumulative log decay and the derived factors
         float x0, x1;
-        const float gl = chunk_cumsum(gs, lane, x0, x1);
+        chunk_cumsum(gs, lane, x0, x1);
         gcv[lane] = x0;
         gcv[lane + 32] = x1;
         egv[lane] = __expf(x0);
         egv[lane + 32] = __expf(x1);
         iegv[lane] = __expf(-x0);
         iegv[lane + 32] = __expf(-x1);
-        eglv[lane] = __expf(gl - x0);
-        eglv[lane + 32] = __expf(gl - x1);
       }
       group_bar(kBar);
       const bool factored = -gcv[63] < kSafeDecay;
-      // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns each
-      if (!group_wait(kBar, &bars[B_D1F], ph, abort_flag, lane)) break;
+      // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns at a time
+      if (!(ok = group_wait(kBar, &bars[B_D1F], ph, abort_flag, lane))) break;
+      if (c >= 2 &&
+          !(ok = group_wait(kBar, &bars[B_PE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane)))
+        break;
       tc_fence_after();
-      for (int hp = hp0; hp < 2; hp += kHalfStep) {
+#pragma unroll 1
+      for (int hp = 0; hp < 2; ++hp) {
         const int r = rl & 63;
         const float gr = gcv[r];
         const float br = rl < 64 ? bs[r] : 1.f;
@@ -688,66 +765,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int s4 = 0; s4 < 8; ++s4)
             dst[s4] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
         } else {
-          st_row32_sw128(sm + Lay::P + s * kTileBytes, r, hp, x);
+          st_row32_sw128(sm + Lay::P + (c & 1) * kTileBytes, r, hp, x);
         }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[B_D1E]);
-      group_bar(kBar);
-      // ---- Y = (I + A)^{-1}
-      invert_unit_lower(AF, reinterpret_cast<float *>(sm + Lay::SCR), pt, kBar);
-#ifdef GDR_TC_DEBUG
-      for (int hp = hp0; hp < 2; hp += kHalfStep)
-        if (rl < 64) DBG_ROW(12288 + 32 * hp, 64, AF + rl * LDA + 32 * hp);
-#endif
-      // ---- T (lanes 0-63) and T' (lanes 64-127) as bf16 operands
-      for (int hp = hp0; hp < 2; hp += kHalfStep) {
-        const int r = rl & 63;
-        uint8_t *tile = sm + (rl < 64 ? Lay::T : Lay::TP);
-        float x[32];
-        const float4 *yr = reinterpret_cast<const float4 *>(AF + r * LDA + 32 * hp);
-        const float4 *b4 = reinterpret_cast<const float4 *>(bs + 32 * hp);
-        const float4 *e4 = reinterpret_cast<const float4 *>(egv + 32 * hp);
-        if (rl < 64) {
-#pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4) {
-            const float4 y = yr[s4], bb = b4[s4];
-            x[4 * s4 + 0] = y.x * bb.x;
-            x[4 * s4 + 1] = y.y * bb.y;
-            x[4 * s4 + 2] = y.z * bb.z;
-            x[4 * s4 + 3] = y.w * bb.w;
-          }
-        } else {
-#pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4) {
-            const float4 y = yr[s4], bb = b4[s4], ee = e4[s4];
-            x[4 * s4 + 0] = y.x * (bb.x * ee.x);
-            x[4 * s4 + 1] = y.y * (bb.y * ee.y);
-            x[4 * s4 + 2] = y.z * (bb.z * ee.z);
-            x[4 * s4 + 3] = y.w * (bb.w * ee.w);
-          }
-        }
-        st_row32_sw128(tile, r, hp, x);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&bars[B_TRDY]);
-      group_bar(kBar);
-      if (pt == 0) mbar_arrive(&bars[B_EMPTY + s]);  // g, beta of this stage no longer read
-      // ---- -W^T -> bf16 MN-major operand (row j = this thread's lane)
-      if (!group_wait(kBar, &bars[B_WTF], ph, abort_flag, lane)) break;
-      tc_fence_after();
-      for (int hp = hp0; hp < 2; hp += kHalfStep) {
-        float x[32];
-        tmem_ld32(lane_base + TM_WT + 32 * hp, x);
-        DBG_ROW(16384 + 32 * hp, 64, x);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = -x[e];
-        st_row32_sw128(sm + Lay::WT, rl, hp, x);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars[B_WTB]);
+      group_bar(kBar);
+      if (pt == 0) mbar_arrive(&bars[B_D1E]);  // D1 may be overwritten
+      // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
+      //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
+      if (c >= 1 && !(ok = group_wait(kBar, &bars[B_UF], (c - 1) & 1, abort_flag, lane))) break;
+      if (c >= 2 &&
+          !(ok = group_wait(kBar, &bars[B_TPE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane)))
+        break;
+      {
+        const TOut to{sm + Lay::T, sm + Lay::TP + (c & 1) * kTileBytes, bs, egv};
+        invert_to_t(AF, reinterpret_cast<float *>(sm + Lay::SCR), to, pt, kBar);
+      }
+      fence_proxy_async_smem();
+      group_bar(kBar);
+      if (pt == 0) mbar_arrive(&bars[B_TRDY]);  // T, T', P of chunk c written
     }
+    if (!ok && pt == 0) atomicOr(a.status, kStatusTimeout);
   } else if (warp < 4) {
     // ================================================================ state group
     const int i = tid;  // TMEM lane = value channel
@@ -756,15 +795,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t kBar = 2;
     bool ok = true;
     // Gate factors of chunk c for this group: e^{gc_r} and e^{gc_last - gc_r}
-    // into SVEC[c & 1], and the chunk's total decay e^{gc_last}.  Computed
-    // from the staged g with the prep group's scan (bit-identical values);
-    // the stage's TMA barrier cannot run ahead of this group.
+    // into SVEC[c & 1]; returns the chunk's total decay e^{gc_last}.
+    // Computed from the staged g with the prep group's scan (bit-identical).
     auto chunk_vectors = [&](int c, float &dl) -> bool {
-      if (!group_wait(kBar, &bars[B_FULL + (c & 1)], (c >> 1) & 1, abort_flag, lane))
+      if (!group_wait(kBar, &bars[B_FULL + c % kStages], (c / kStages) & 1, abort_flag, lane))
         return false;
       float *sv = reinterpret_cast<float *>(sm + Lay::SVEC + (c & 1) * 512);
       if (warp == 0) {
-        const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + (c & 1) * 512);
+        const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * 512);
         float x0, x1;
         const float gl = chunk_cumsum(gs, lane, x0, x1);
         sv[lane] = __expf(x0);
@@ -776,71 +814,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       dl = sv[63];
       return true;
     };
-    // S_b = bf16(S) for the next chunk's MMAs, and S <- S * dl (that chunk's
-    // decay, applied before its state update accumulates onto S).  The
-    // source (S0 in global memory, or S in TMEM) is chosen outside the
-    // unrolled loops.
-    auto state_cols = [&](int q, const float (&x)[32], float dl) {
-      uint32_t u[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
-      tmem_st16u(lane_base + TM_SB + 16 * q, u);
-      float y0[16], y1[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        y0[e] = x[e] * dl;
-        y1[e] = x[16 + e] * dl;
-      }
-      tmem_st16(lane_base + TM_S + 32 * q, y0);
-      tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
-    };
-    auto state_pass = [&](const float *src_global, float dl) {
-      if (src_global) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float x[32];
-          const float4 *s4 = reinterpret_cast<const float4 *>(src_global + 32 * q);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 v = s4[e];
-            x[4 * e] = v.x;
-            x[4 * e + 1] = v.y;
-            x[4 * e + 2] = v.z;
-            x[4 * e + 3] = v.w;
-          }
-          state_cols(q, x, dl);
-        }
-      } else {
+    // S_b = bf16(sigma S_tmem) for the chunk's MMAs.  While sigma * dl (dl:
+    // the chunk's decay) stays above the floor only sigma changes; otherwise
+    // (fold) S_tmem <- f S_tmem with f = sigma * dl and sigma restarts at 1.
+    // The branch is taken outside the unrolled loops.
+    auto pass_from_tmem = [&](float sig, bool fold, float f) {
+      if (fold) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float x[32];
           tmem_ld32(lane_base + TM_S + 32 * q, x);
-          state_cols(q, x, dl);
+          uint32_t u[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e] * sig, x[2 * e + 1] * sig);
+          tmem_st16u(lane_base + TM_SB + 16 * q, u);
+          float y0[16], y1[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            y0[e] = x[e] * f;
+            y1[e] = x[16 + e] * f;
+          }
+          tmem_st16(lane_base + TM_S + 32 * q, y0);
+          tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
+        }
+      } else {
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+          float x[64];
+          tmem_ld64(lane_base + TM_S + 64 * q, x);
+          uint32_t u[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) u[e] = pack_bf16(x[2 * e] * sig, x[2 * e + 1] * sig);
+          tmem_st16u(lane_base + TM_SB + 32 * q, u);
+          tmem_st16u(lane_base + TM_SB + 32 * q + 16, u + 16);
         }
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[B_SBR]);
     };
+    // sig: the scale of S_tmem at the next state pass; inv: 1 / the scale
+    // after the chunk in flight, applied to that chunk's state update.
+    float sig = 1.f, inv = 1.f;
     {
       float dl;
       if (!chunk_vectors(0, dl)) {
         ok = false;
-      } else if (a.S0) {
-        state_pass(a.S0 + ((size_t)bh * DV + i) * DK, dl);
       } else {
-        // zero initial state: write zeros through the same path
-        float z[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) z[e] = 0.f;
-        uint32_t u[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = 0u;
+        // S_b = bf16(S0); S_tmem = e^{gc_last} S0; sigma = 1 afterwards.
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
+          float x[32];
+          if (a.S0) {
+            const float4 *s4 =
+                reinterpret_cast<const float4 *>(a.S0 + ((size_t)bh * DV + i) * DK + 32 * q);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float4 v = s4[e];
+              x[4 * e] = v.x;
+              x[4 * e + 1] = v.y;
+              x[4 * e + 2] = v.z;
+              x[4 * e + 3] = v.w;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = 0.f;
+          }
+          uint32_t u[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
           tmem_st16u(lane_base + TM_SB + 16 * q, u);
-          tmem_st16(lane_base + TM_S + 32 * q, *reinterpret_cast<float(*)[16]>(z));
-          tmem_st16(lane_base + TM_S + 32 * q + 16, *reinterpret_cast<float(*)[16]>(z + 16));
+          float y0[16], y1[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            y0[e] = x[e] * dl;
+            y1[e] = x[16 + e] * dl;
+          }
+          tmem_st16(lane_base + TM_S + 32 * q, y0);
+          tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -851,32 +902,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = c & 1;
       const float *sv = reinterpret_cast<const float *>(sm + Lay::SVEC + (c & 1) * 512);
       const float *egv = sv, *eglv = sv + 64;
-      // ---- V'^T -> bf16 operands (plain and decayed to the chunk end)
-      if (!group_wait(kBar, &bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
+      // ---- -Z -> bf16 A operand, in place in TMEM
+      if (!group_wait(kBar, &bars[B_ZF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
-        float x[64];
-        tmem_ld64(lane_base + TM_UV, x);
-        DBG_ROW(40960, 64, x);
-        DBG_ROW(40960 + 32, 64, x + 32);
-        st_row32_sw128(sm + Lay::VP, i, 0, x);
-        st_row32_sw128(sm + Lay::VP, i, 1, x + 32);
-        const float4 *e4 = reinterpret_cast<const float4 *>(eglv);
+        // both halves are loaded before either is overwritten in place
+        float z0[32], z1[32];
+        tmem_ld32(lane_base + TM_Z, z0);
+        tmem_ld32(lane_base + TM_Z + 32, z1);
+        DBG_ROW(16384, 64, z0);
+        DBG_ROW(16384 + 32, 64, z1);
+        uint32_t u[16];
 #pragma unroll
-        for (int s4 = 0; s4 < 16; ++s4) {
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(-z0[2 * e], -z0[2 * e + 1]);
+        tmem_st16u(lane_base + TM_Z, u);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(-z1[2 * e], -z1[2 * e + 1]);
+        tmem_st16u(lane_base + TM_Z + 16, u);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_ZR]);
+      // ---- V'^T -> bf16 operands (plain, and decayed to the chunk end / sigma)
+      if (!group_wait(kBar, &bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int q = 0; q < 2; ++q) {
+        float x[32];
+        tmem_ld32(lane_base + TM_UV + 32 * q, x);
+        DBG_ROW(40960 + 32 * q, 64, x);
+        st_row32_sw128(sm + Lay::VP, i, q, x);
+        const float4 *e4 = reinterpret_cast<const float4 *>(eglv + 32 * q);
+#pragma unroll
+        for (int s4 = 0; s4 < 8; ++s4) {
           const float4 e = e4[s4];
-          x[4 * s4] *= e.x;
-          x[4 * s4 + 1] *= e.y;
-          x[4 * s4 + 2] *= e.z;
-          x[4 * s4 + 3] *= e.w;
+          x[4 * s4] *= e.x * inv;
+          x[4 * s4 + 1] *= e.y * inv;
+          x[4 * s4 + 2] *= e.z * inv;
+          x[4 * s4 + 3] *= e.w * inv;
         }
-        st_row32_sw128(sm + Lay::VPD, i, 0, x);
-        st_row32_sw128(sm + Lay::VPD, i, 1, x + 32);
+        st_row32_sw128(sm + Lay::VPD, i, q, x);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_VPR]);
-      // ---- updated S -> S_b and the next chunk's decay, or the final state
+      // ---- updated S -> S_b for the next chunk, or the final state
       if (!group_wait(kBar, &bars[B_SF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       if (c + 1 < n) {
@@ -886,15 +956,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < 4; ++q) {
           float x[32];
           tmem_ld32(lane_base + TM_S + 32 * q, x);
+          for (int e = 0; e < 32; ++e) x[e] *= sig;
           DBG_ROW(57344 + 32 * q, 128, x);
         }
 #endif
-        state_pass(nullptr, dl);
+        const float nxt = sig * dl;
+        const bool fold = !(nxt >= kScaleFloor);  // also when dl underflows to 0
+        pass_from_tmem(sig, fold, nxt);
+        sig = fold ? 1.f : nxt;
+        inv = 1.f / sig;
       } else if (a.S_T) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float x[32];
           tmem_ld32(lane_base + TM_S + 32 * q, x);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= sig;
           DBG_ROW(57344 + 32 * q, 128, x);
           float4 *dst = reinterpret_cast<float4 *>(a.S_T + ((size_t)bh * DV + i) * DK + 32 * q);
 #pragma unroll
@@ -913,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t *o32 = reinterpret_cast<uint32_t *>(a.o);
         const int chpair = i & ~1;
         const bool full = t0 + C <= T;
-#pragma unroll
+#pragma unroll 1
         for (int q = 0; q < 2; ++q) {
           float xa[32], xb[32];
           {
@@ -930,6 +1007,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               xb[e] = b0[e];
               xb[16 + e] = b1[e];
             }
+          }
+          if (q == 1) {  // every read of O_a / O_b is done
+            tc_fence_before();
+            mbar_arrive(&bars[B_OE]);
           }
           const float4 *e4 = reinterpret_cast<const float4 *>(egv + 32 * q);
 #pragma unroll
@@ -964,7 +1045,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      tc_fence_before();
     }
     if (!ok && i == 0) atomicOr(a.status, kStatusTimeout);
   }
