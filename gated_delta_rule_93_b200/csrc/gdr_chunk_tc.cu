@@ -71,6 +71,12 @@ constexpr int kScrFloats = 16 * 8 + 48 * 8;
 // 16 consecutive rows hit distinct 16-byte bank groups pairwise.
 constexpr int LDA = 68;
 
+// Gate vectors of a stage, written by the K/Q producer (float offsets):
+// gc = cumulative log decay from the chunk start, e^{gc}, e^{-gc},
+// e^{gc_last - gc}, beta.
+constexpr int kGateGc = 0, kGateEg = 64, kGateIeg = 128, kGateEgl = 192, kGateBeta = 256;
+constexpr uint32_t kGateBytes = 320 * 4;
+
 // Shared-memory layout (byte offsets from a 1024-byte aligned base).
 struct Lay {
   static constexpr uint32_t KQ = 0;                             // per stage [K_h0|Q_h0|K_h1|Q_h1]
@@ -82,9 +88,8 @@ struct Lay {
   static constexpr uint32_t VPD = VP + 2 * kTileBytes;          // decayed, rescaled V'^T
   static constexpr uint32_t AF = VPD + 2 * kTileBytes;          // fp32 A, diagonal blocks -> D
   static constexpr uint32_t SCR = AF + 64 * LDA * 4;            // 4 x kScrFloats fp32
-  static constexpr uint32_t GS = SCR + 4 * kScrFloats * 4;      // per stage g[64], beta[64]
-  static constexpr uint32_t VEC = GS + kStages * 512;           // x2 (prep): gc, eg, ieg [64]
-  static constexpr uint32_t SVEC = VEC + 2 * 1024;              // x2 (state): eg, egl [64]
+  static constexpr uint32_t GS = SCR + 4 * kScrFloats * 4;      // per stage, see kGate*
+  static constexpr uint32_t SVEC = GS + kStages * kGateBytes;   // x2 (state): eg, egl [64]
   static constexpr uint32_t BAR = SVEC + 2 * 512;               // mbarriers
   static constexpr uint32_t MISC = BAR + 32 * 8;                // tmem base, abort flag
   static constexpr uint32_t END = MISC + 16;
@@ -102,8 +107,8 @@ enum {
   B_VFULL = 6,         // V landed                                      (1 + tx)
   B_VEMPTY,            // V free (prep commit after U)                  (commit)
   B_D1F,               // D1 written                                    (commit, prep side)
-  B_D1E,               // D1 read by the prep group                     (1)
-  B_TRDY,              // T, T' and P of a chunk written                (1)
+  B_D1E,               // D1 read by the prep group                     (128)
+  B_TRDY,              // T, T' and P of a chunk written                (128)
   B_UF,                // U^T written (T read)                          (commit, prep side)
   B_ZF,                // Z written                                     (commit)
   B_ZR,                // -Z bf16 operand in TMEM                       (128)
@@ -198,7 +203,9 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// Warp-group barriers (128 threads each): id 2 = state group, id 3 = prep.
+// Barrier over the prep warpgroup (id 3, 128 threads) that also ORs a
+// failure flag, so that the group leaves its loop together (a warp left
+// behind at a named barrier would never return).
 __device__ __forceinline__ bool group_any(uint32_t bar_id, bool pred) {
   uint32_t r;
   asm volatile(
@@ -210,7 +217,6 @@ __device__ __forceinline__ bool group_any(uint32_t bar_id, bool pred) {
   return r != 0;
 }
 
-__device__ __forceinline__ void group_bar(uint32_t bar_id) { named_bar_sync(bar_id, 128); }
 
 // Bounded wait that also gives up as soon as another role has aborted.
 // The thread sleeps inside try_wait (suspend hint) between checks.
@@ -228,19 +234,21 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
   return true;
 }
 
-// Group-wide wait and abort check: lane 0 of each warp polls, the warp
-// shares its result, and the group agrees (any failure, or an abort raised
-// anywhere in the CTA, -> every thread sees failure).
-__device__ __forceinline__ bool group_wait(uint32_t bar_id, uint64_t *bar, uint32_t parity,
-                                           volatile int *abort_flag, int lane) {
-  bool ok = true;
-  if (lane == 0) ok = wait_or_abort(bar, parity, abort_flag) && !*abort_flag;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  return !group_any(bar_id, !ok);
+// Warp-wide wait and abort check (false on time-out or once an abort was
+// raised anywhere in the CTA).  Every lane polls the same barrier, flag and
+// timer, so the result is warp-uniform without a shuffle (chained shuffles
+// were measured at several hundred cycles each in this kernel).  Warps wait
+// on their own: a group barrier after every wait would make each warp wait
+// for the slowest one as well.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
+                                          volatile int *abort_flag, int lane) {
+  (void)lane;
+  return wait_or_abort(bar, parity, abort_flag) && !*abort_flag;
 }
 
 // One warp: cumulative log decay of a chunk (g[64] -> gc[64] in log space,
 // inclusive prefix sum) held as lanes r and r + 32; returns the chunk total.
+// Used by the K/Q producer only, which runs chunks ahead of its consumers.
 __device__ __forceinline__ float chunk_cumsum(const float *g, int lane, float &x0, float &x1) {
   x0 = g[lane];
   x1 = g[lane + 32];
@@ -378,14 +386,14 @@ __device__ __forceinline__ void inverse_strip(const float *AF, float *ys, const 
 // (I + A)^{-1} for the strictly lower 64x64 fp32 A in AF (row stride LDA,
 // zero above the diagonal) with the 4-warp prep group (local thread t),
 // written as T and T' (their blocks above the block diagonal stay zero from
-// the kernel's start):
+// the kernel's start), in two steps with a group barrier between them:
 //  1. warp b: D_bb = (I + A_bb)^{-1} by forward substitution (lane c % 16
 //     owns column c), stored over A_bb in AF and, scaled, into T and T';
 //  2. strips (column block j, half hf): warp 0 -> (0,0); warp 1 -> (0,1);
 //     warp 2 -> (1,0), (2,0); warp 3 -> (1,1), (2,1).  (An fp32 CUDA-core
 //     strip sweep was faster alone but, competing for issue slots with the
 //     state group, slower in the kernel.)
-__device__ void invert_to_t(float *AF, float *scr, const TOut &o, int t, uint32_t bar_id) {
+__device__ void invert_diag(float *AF, const TOut &o, int t) {
   const int warp = t >> 5, lane = t & 31;
   {
     const int w = warp, c = lane & 15;
@@ -412,24 +420,21 @@ __device__ void invert_to_t(float *AF, float *scr, const TOut &o, int t, uint32_
 #pragma unroll
       for (int i = 0; i < 16; ++i) Yb[i * LDA + c] = x[i];
     }
-    // T (lanes 0-15) and T' (lanes 16-31) of the diagonal block: lanes c and
-    // c ^ 1 pair up so that each writes two adjacent columns of every other
-    // row.
+    // T (lanes 0-15) and T' (lanes 16-31) of the diagonal block, one bf16
+    // per store (no shuffles).
     const int col = 16 * w + c;
     const float sc = (lane < 16) ? o.beta[col] : o.beta[col] * o.eg[col];
     uint8_t *tile = (lane < 16) ? o.t : o.tp;
-    const int odd = c & 1;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float mine = x[i] * sc;
-      const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-      if ((i & 1) == odd) {
-        const uint32_t v = odd ? pack_bf16(other, mine) : pack_bf16(mine, other);
-        *reinterpret_cast<uint32_t *>(tile + sw128_off(16 * w + i, col & ~1)) = v;
-      }
-    }
+    for (int i = 0; i < 16; ++i)
+      *reinterpret_cast<__nv_bfloat16 *>(tile + sw128_off(16 * w + i, col)) =
+          __float2bfloat16_rn(x[i] * sc);
   }
-  group_bar(bar_id);
+}
+
+// Step 2 of the inverse (after a group barrier: every D_bb is in AF).
+__device__ void invert_strips(const float *AF, float *scr, const TOut &o, int t) {
+  const int warp = t >> 5, lane = t & 31;
   float *ws = scr + warp * kScrFloats;  // [16][8] product scratch, then [48][8] strip blocks
   const Frag f{lane >> 2, lane & 3, ws};
   const int hf = warp & 1;
@@ -482,8 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[B_VFULL], 1);
     mbar_init(&bars[B_VEMPTY], 1);
     mbar_init(&bars[B_D1F], 1);
-    mbar_init(&bars[B_D1E], 1);
-    mbar_init(&bars[B_TRDY], 1);
+    mbar_init(&bars[B_D1E], 128);
+    mbar_init(&bars[B_TRDY], 128);
     mbar_init(&bars[B_UF], 1);
     mbar_init(&bars[B_ZF], 1);
     mbar_init(&bars[B_ZR], 128);
@@ -526,23 +531,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     int last_issued[kStages] = {-1, -1, -1};  // latest chunk loaded into each stage
     for (int c = 0; c < n; ++c) {
       const int s = c % kStages;
-      if (c >= kStages) {
-        bool ok = true;
-        if (lane == 0)
-          ok = wait_or_abort(&bars[B_EMPTY + s], ((c / kStages) - 1) & 1, abort_flag);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      }
+      if (c >= kStages &&
+          !wait_or_abort(&bars[B_EMPTY + s], ((c / kStages) - 1) & 1, abort_flag))
+        break;
       // Testing hook: this chunk's load is never issued, so its consumers'
       // bounded waits run out and the kernel unwinds (no trap, no hang).
       if (c == a.skip_stage_chunk) continue;
       const int t0 = c * C;
-      float *gs = reinterpret_cast<float *>(sm + Lay::GS + s * 512);
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int r = lane + 32 * q, t = t0 + r;
-        const size_t tok = ((size_t)b * T + t) * H + h;
-        gs[r] = t < T ? a.g[tok] : 0.f;
-        gs[64 + r] = t < T ? a.beta[tok] : 0.f;
+      float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
+      {
+        float gl0 = 0.f, gl1 = 0.f, b0 = 0.f, b1 = 0.f;
+        const size_t tok = ((size_t)b * T + t0 + lane) * H + h;
+        if (t0 + lane < T) {
+          gl0 = a.g[tok];
+          b0 = a.beta[tok];
+        }
+        if (t0 + lane + 32 < T) {
+          gl1 = a.g[tok + (size_t)32 * H];
+          b1 = a.beta[tok + (size_t)32 * H];
+        }
+        float* gc = gv + kGateGc;
+        gc[lane] = gl0;
+        gc[lane + 32] = gl1;
+        __syncwarp();
+        float x0, x1;
+        const float gl = chunk_cumsum(gc, lane, x0, x1);
+        __syncwarp();
+        gc[lane] = x0;
+        gc[lane + 32] = x1;
+        gv[kGateEg + lane] = __expf(x0);
+        gv[kGateEg + lane + 32] = __expf(x1);
+        gv[kGateIeg + lane] = __expf(-x0);
+        gv[kGateIeg + lane + 32] = __expf(-x1);
+        gv[kGateEgl + lane] = __expf(gl - x0);
+        gv[kGateEgl + lane + 32] = __expf(gl - x1);
+        gv[kGateBeta + lane] = b0;
+        gv[kGateBeta + lane + 32] = b1;
       }
       __syncwarp();
       if (lane == 0) {
@@ -694,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 4 && warp < 8) {
     // ================================================================ prep group
-    const int pt = tid - 128, rl = pt, pw = pt >> 5;
+    const int pt = tid - 128, rl = pt;
     const int lrow = rl;
     (void)lrow;
     constexpr uint32_t kBar = 3;
@@ -702,89 +726,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < n; ++c) {
       const int st = c % kStages;
       const uint32_t ph = c & 1;
-      float *vec = reinterpret_cast<float *>(sm + Lay::VEC + (c & 1) * 1024);
-      float *gcv = vec, *egv = vec + 64, *iegv = vec + 128;
-      if (!(ok = group_wait(kBar, &bars[B_FULL + st], (c / kStages) & 1, abort_flag, lane))) break;
-      const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + st * 512);
-      const float *bs = gs + 64;
-      if (pw == 0) {  // cumulative log decay and the derived factors
-        float x0, x1;
-        chunk_cumsum(gs, lane, x0, x1);
-        gcv[lane] = x0;
-        gcv[lane + 32] = x1;
-        egv[lane] = __expf(x0);
-        egv[lane + 32] = __expf(x1);
-        iegv[lane] = __expf(-x0);
-        iegv[lane + 32] = __expf(-x1);
-      }
-      group_bar(kBar);
-      const bool factored = -gcv[63] < kSafeDecay;
-      // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns at a time
-      if (!(ok = group_wait(kBar, &bars[B_D1F], ph, abort_flag, lane))) break;
-      if (c >= 2 &&
-          !(ok = group_wait(kBar, &bars[B_PE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane)))
-        break;
-      tc_fence_after();
+      const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + st * kGateBytes);
+      const float *gcv = gv + kGateGc, *egv = gv + kGateEg, *iegv = gv + kGateIeg;
+      const float *bs = gv + kGateBeta;
+      // This warp's waits: the stage, D1, (c >= 2) this P buffer free, and
+      // for the warps writing A (rows 0-63), every strip of the previous
+      // chunk done reading AF (TRDY counts all 128 prep threads).
+      bool bad = !warp_wait(&bars[B_FULL + st], (c / kStages) & 1, abort_flag, lane) ||
+                 !warp_wait(&bars[B_D1F], ph, abort_flag, lane) ||
+                 (c >= 2 &&
+                  !warp_wait(&bars[B_PE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane)) ||
+                 (c >= 1 && pt < 64 && !warp_wait(&bars[B_TRDY], (c - 1) & 1, abort_flag, lane));
+      if (!bad) {
+        const bool factored = -gcv[63] < kSafeDecay;
+        // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns at a time
+        tc_fence_after();
 #pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
-        const int r = rl & 63;
-        const float gr = gcv[r];
-        const float br = rl < 64 ? bs[r] : 1.f;
-        const float fr = br * egv[r];
-        float x[32];
-        tmem_ld32(lane_base + TM_D1 + 32 * hp, x);
-        DBG_ROW(32 * hp, 64, x);
-        const int lim = (rl < 64 ? r : r + 1) - 32 * hp;  // A: s < r, P: s <= r
-        // The decay form is chosen once per chunk, outside the unrolled loops
-        // (a branch inside them costs even when it is never taken).
-        float dvs[32];
-        if (factored) {
+        for (int hp = 0; hp < 2; ++hp) {
+          const int r = rl & 63;
+          const float gr = gcv[r];
+          const float br = rl < 64 ? bs[r] : 1.f;
+          const float fr = br * egv[r];
+          float x[32];
+          tmem_ld32(lane_base + TM_D1 + 32 * hp, x);
+          DBG_ROW(32 * hp, 64, x);
+          const int lim = (rl < 64 ? r : r + 1) - 32 * hp;  // A: s < r, P: s <= r
+          // The decay form is chosen once per chunk, outside the unrolled
+          // loops (a branch inside them costs even when it is never taken).
+          float dvs[32];
+          if (factored) {
 #pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4) {
-            const float4 ie = *reinterpret_cast<const float4 *>(iegv + 32 * hp + 4 * s4);
-            dvs[4 * s4 + 0] = fr * ie.x;
-            dvs[4 * s4 + 1] = fr * ie.y;
-            dvs[4 * s4 + 2] = fr * ie.z;
-            dvs[4 * s4 + 3] = fr * ie.w;
+            for (int s4 = 0; s4 < 8; ++s4) {
+              const float4 ie = *reinterpret_cast<const float4 *>(iegv + 32 * hp + 4 * s4);
+              dvs[4 * s4 + 0] = fr * ie.x;
+              dvs[4 * s4 + 1] = fr * ie.y;
+              dvs[4 * s4 + 2] = fr * ie.z;
+              dvs[4 * s4 + 3] = fr * ie.w;
+            }
+          } else {
+#pragma unroll
+            for (int s4 = 0; s4 < 8; ++s4) {
+              const float4 gg = *reinterpret_cast<const float4 *>(gcv + 32 * hp + 4 * s4);
+              dvs[4 * s4 + 0] = br * __expf(gr - gg.x);
+              dvs[4 * s4 + 1] = br * __expf(gr - gg.y);
+              dvs[4 * s4 + 2] = br * __expf(gr - gg.z);
+              dvs[4 * s4 + 3] = br * __expf(gr - gg.w);
+            }
           }
-        } else {
 #pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4) {
-            const float4 gg = *reinterpret_cast<const float4 *>(gcv + 32 * hp + 4 * s4);
-            dvs[4 * s4 + 0] = br * __expf(gr - gg.x);
-            dvs[4 * s4 + 1] = br * __expf(gr - gg.y);
-            dvs[4 * s4 + 2] = br * __expf(gr - gg.z);
-            dvs[4 * s4 + 3] = br * __expf(gr - gg.w);
+          for (int e = 0; e < 32; ++e) x[e] = (e < lim) ? x[e] * dvs[e] : 0.f;
+          if (rl < 64) {
+            float4 *dst = reinterpret_cast<float4 *>(AF + r * LDA + 32 * hp);
+#pragma unroll
+            for (int s4 = 0; s4 < 8; ++s4)
+              dst[s4] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
+          } else {
+            st_row32_sw128(sm + Lay::P + (c & 1) * kTileBytes, r, hp, x);
           }
         }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = (e < lim) ? x[e] * dvs[e] : 0.f;
-        if (rl < 64) {
-          float4 *dst = reinterpret_cast<float4 *>(AF + r * LDA + 32 * hp);
-#pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4)
-            dst[s4] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
-        } else {
-          st_row32_sw128(sm + Lay::P + (c & 1) * kTileBytes, r, hp, x);
-        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars[B_D1E]);  // this thread's D1 reads are done
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      group_bar(kBar);
-      if (pt == 0) mbar_arrive(&bars[B_D1E]);  // D1 may be overwritten
+      // A complete in AF before the inverse; the group agrees on failure.
+      if (group_any(kBar, bad)) { ok = false; break; }
       // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
-      if (c >= 1 && !(ok = group_wait(kBar, &bars[B_UF], (c - 1) & 1, abort_flag, lane))) break;
-      if (c >= 2 &&
-          !(ok = group_wait(kBar, &bars[B_TPE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane)))
-        break;
-      {
-        const TOut to{sm + Lay::T, sm + Lay::TP + (c & 1) * kTileBytes, bs, egv};
-        invert_to_t(AF, reinterpret_cast<float *>(sm + Lay::SCR), to, pt, kBar);
-      }
+      const TOut to{sm + Lay::T, sm + Lay::TP + (c & 1) * kTileBytes, bs, egv};
+      bad = (c >= 1 && !warp_wait(&bars[B_UF], (c - 1) & 1, abort_flag, lane)) ||
+            (c >= 2 &&
+             !warp_wait(&bars[B_TPE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane));
+      if (!bad) invert_diag(AF, to, pt);
+      if (group_any(kBar, bad)) { ok = false; break; }
+      invert_strips(AF, reinterpret_cast<float *>(sm + Lay::SCR), to, pt);
       fence_proxy_async_smem();
-      group_bar(kBar);
-      if (pt == 0) mbar_arrive(&bars[B_TRDY]);  // T, T', P of chunk c written
+      mbar_arrive(&bars[B_TRDY]);  // this thread's T, T', P writes are done
     }
     if (!ok && pt == 0) atomicOr(a.status, kStatusTimeout);
   } else if (warp < 4) {
@@ -792,25 +808,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = tid;  // TMEM lane = value channel
     const int lrow = i;
     (void)lrow;
-    constexpr uint32_t kBar = 2;
     bool ok = true;
     // Gate factors of chunk c for this group: e^{gc_r} and e^{gc_last - gc_r}
     // into SVEC[c & 1]; returns the chunk's total decay e^{gc_last}.
-    // Computed from the staged g with the prep group's scan (bit-identical).
+    // Every warp writes the same values and reads them after its own writes
+    // (no group barrier).  A warp cannot run a whole chunk ahead of another:
+    // the count-128 barriers it waits for need the other warps' arrivals.
     auto chunk_vectors = [&](int c, float &dl) -> bool {
-      if (!group_wait(kBar, &bars[B_FULL + c % kStages], (c / kStages) & 1, abort_flag, lane))
+      if (!warp_wait(&bars[B_FULL + c % kStages], (c / kStages) & 1, abort_flag, lane))
         return false;
+      // The stage can be refilled while this chunk's O epilogue still runs,
+      // so the group keeps its own copy of e^{gc} and e^{gc_last - gc}.
       float *sv = reinterpret_cast<float *>(sm + Lay::SVEC + (c & 1) * 512);
-      if (warp == 0) {
-        const float *gs = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * 512);
-        float x0, x1;
-        const float gl = chunk_cumsum(gs, lane, x0, x1);
-        sv[lane] = __expf(x0);
-        sv[lane + 32] = __expf(x1);
-        sv[64 + lane] = __expf(gl - x0);
-        sv[64 + lane + 32] = __expf(gl - x1);
-      }
-      group_bar(kBar);
+      const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * kGateBytes);
+      sv[lane] = gv[kGateEg + lane];
+      sv[lane + 32] = gv[kGateEg + lane + 32];
+      sv[64 + lane] = gv[kGateEgl + lane];
+      sv[64 + lane + 32] = gv[kGateEgl + lane + 32];
+      __syncwarp();
       dl = sv[63];
       return true;
     };
@@ -903,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *sv = reinterpret_cast<const float *>(sm + Lay::SVEC + (c & 1) * 512);
       const float *egv = sv, *eglv = sv + 64;
       // ---- -Z -> bf16 A operand, in place in TMEM
-      if (!group_wait(kBar, &bars[B_ZF], ph, abort_flag, lane)) { ok = false; break; }
+      if (!warp_wait(&bars[B_ZF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
         // both halves are loaded before either is overwritten in place
@@ -924,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars[B_ZR]);
       // ---- V'^T -> bf16 operands (plain, and decayed to the chunk end / sigma)
-      if (!group_wait(kBar, &bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
+      if (!warp_wait(&bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {
@@ -947,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars[B_VPR]);
       // ---- updated S -> S_b for the next chunk, or the final state
-      if (!group_wait(kBar, &bars[B_SF], ph, abort_flag, lane)) { ok = false; break; }
+      if (!warp_wait(&bars[B_SF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       if (c + 1 < n) {
         float dl;
@@ -979,16 +994,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
         }
       }
-      // ---- O = O_a Diag(e^{gc}) + O_b -> bf16, stored straight to o: lanes
-      //      i, i^1 swap values so each lane writes two adjacent channels of
-      //      one token (a warp writes 2 tokens x 64 contiguous bytes)
-      if (!group_wait(kBar, &bars[B_OF], ph, abort_flag, lane)) { ok = false; break; }
+      // ---- O = O_a Diag(e^{gc}) + O_b -> bf16, stored straight to o
+      if (!warp_wait(&bars[B_OF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
         const int t0 = c * C;
         const size_t tok0 = ((size_t)b * T + t0) * H + h;
-        uint32_t *o32 = reinterpret_cast<uint32_t *>(a.o);
-        const int chpair = i & ~1;
         const bool full = t0 + C <= T;
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
@@ -1022,31 +1033,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             xa[4 * s4 + 3] = ev.w * xa[4 * s4 + 3] + xb[4 * s4 + 3];
           }
           DBG_ROW(49152 + 32 * q, 64, xa);
-          // full chunks store unconditionally; only a ragged last chunk
-          // takes the guarded loop (chosen outside the unrolled loops)
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float lo = xa[2 * e], hi = xa[2 * e + 1];  // tokens 32q+2e, +1
-            const float send = (i & 1) ? lo : hi;
-            const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-            w[e] = (i & 1) ? pack_bf16(recv, hi) : pack_bf16(lo, recv);
-          }
-          uint32_t *dst = o32 + (((tok0 + (size_t)(32 * q + (i & 1)) * H) * DV + chpair) >> 1);
-          const size_t tstep = (size_t)H * DV;  // 32-bit words between tokens t and t + 2
+          // one bf16 per store: a warp writes 32 adjacent channels (64 bytes)
+          // of one token; full chunks store unconditionally, only a ragged
+          // last chunk takes the guarded loop (chosen outside the loops)
+          __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.o) +
+                               (tok0 + (size_t)(32 * q) * H) * DV + i;
+          const size_t tstep = (size_t)H * DV;  // elements between tokens t and t + 1
           if (full) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) __stcs(dst + e * tstep, w[e]);
+            for (int e = 0; e < 32; ++e) {
+              __stcs(dst, __float2bfloat16_rn(xa[e]));
+              dst += tstep;
+            }
           } else {
-            const int rem = T - t0 - 32 * q - (i & 1);  // tokens left for this lane's parity
+            const int rem = T - t0 - 32 * q;
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (2 * e < rem) __stcs(dst + e * tstep, w[e]);
+            for (int e = 0; e < 32; ++e) {
+              if (e < rem) __stcs(dst, __float2bfloat16_rn(xa[e]));
+              dst += tstep;
+            }
           }
         }
       }
     }
-    if (!ok && i == 0) atomicOr(a.status, kStatusTimeout);
+    if (!ok && lane == 0) atomicOr(a.status, kStatusTimeout);
   }
 
   tc_fence_before();
