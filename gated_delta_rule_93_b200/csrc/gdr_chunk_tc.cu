@@ -290,15 +290,29 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
 }
 
 // mma.sync m16n8k8 TF32 fragments of one warp (g = lane / 4, tq = lane % 4).
+// The k index is permuted identically in A and B (fragment slot tq holds
+// k = 2 tq, slot tq + 4 holds k = 2 tq + 1), which leaves the product
+// unchanged and makes each lane's two A elements of a row adjacent.
 struct Frag {
   int g, tq;
   float *scr;  // warp-private [16][8] fp32 scratch
   // A fragment of the 16x8 block of AF at (row0, col0).
   __device__ __forceinline__ void a(const float *AF, int row0, int col0, uint32_t (&af)[4]) const {
-    af[0] = to_tf32(AF[(row0 + g) * LDA + col0 + tq]);
-    af[1] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq]);
-    af[2] = to_tf32(AF[(row0 + g) * LDA + col0 + tq + 4]);
-    af[3] = to_tf32(AF[(row0 + g + 8) * LDA + col0 + tq + 4]);
+    const float2 lo = *reinterpret_cast<const float2 *>(AF + (row0 + g) * LDA + col0 + 2 * tq);
+    const float2 hi = *reinterpret_cast<const float2 *>(AF + (row0 + g + 8) * LDA + col0 + 2 * tq);
+    af[0] = to_tf32(lo.x);
+    af[1] = to_tf32(hi.x);
+    af[2] = to_tf32(lo.y);
+    af[3] = to_tf32(hi.y);
+  }
+  // B fragments (two k-steps) of a 16x8 fp32 block stored row-major with
+  // row stride ld floats.
+  __device__ __forceinline__ void b(const float *blk, int ld, uint32_t (&bf)[2][2]) const {
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      bf[ks][0] = to_tf32(blk[(8 * ks + 2 * tq) * ld + g]);
+      bf[ks][1] = to_tf32(blk[(8 * ks + 2 * tq + 1) * ld + g]);
+    }
   }
   // 16x8 accumulator fragment -> B fragments of two k-steps (rows 0-7, 8-15).
   __device__ __forceinline__ void to_b(const float (&cf)[4], uint32_t (&bf)[2][2]) const {
@@ -307,11 +321,7 @@ struct Frag {
     scr[(g + 8) * 8 + 2 * tq] = cf[2];
     scr[(g + 8) * 8 + 2 * tq + 1] = cf[3];
     __syncwarp();
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      bf[ks][0] = to_tf32(scr[(8 * ks + tq) * 8 + g]);
-      bf[ks][1] = to_tf32(scr[(8 * ks + tq + 4) * 8 + g]);
-    }
+    b(scr, 8, bf);
     __syncwarp();
   }
 };
@@ -324,17 +334,6 @@ __device__ __forceinline__ void store_t2(const TOut &o, int r, int s, float y0, 
   const uint32_t off = sw128_off(r, s);
   *reinterpret_cast<uint32_t *>(o.t + off) = pack_bf16(t0, t1);
   *reinterpret_cast<uint32_t *>(o.tp + off) = pack_bf16(t0 * e.x, t1 * e.y);
-}
-
-// B fragments (two k-steps) of a 16x8 fp32 block stored row-major with
-// row stride `ld` floats.
-__device__ __forceinline__ void load_bfrag(const float *blk, int ld, const Frag &f,
-                                           uint32_t (&bf)[2][2]) {
-#pragma unroll
-  for (int ks = 0; ks < 2; ++ks) {
-    bf[ks][0] = to_tf32(blk[(8 * ks + f.tq) * ld + f.g]);
-    bf[ks][1] = to_tf32(blk[(8 * ks + f.tq + 4) * ld + f.g]);
-  }
 }
 
 // One 8-column strip (first column col0) of column block j of
@@ -354,7 +353,7 @@ __device__ __forceinline__ void inverse_strip(const float *AF, float *ys, const 
     for (int k = j; k < bb; ++k) {
       const float *yblk = (k == j) ? AF + (16 * j) * LDA + col0 : ys + 16 * (k - j - 1) * 8;
       uint32_t bf[2][2];
-      load_bfrag(yblk, (k == j) ? LDA : 8, f, bf);
+      f.b(yblk, (k == j) ? LDA : 8, bf);
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
         uint32_t af[4];
@@ -387,48 +386,47 @@ __device__ __forceinline__ void inverse_strip(const float *AF, float *ys, const 
 // zero above the diagonal) with the 4-warp prep group (local thread t),
 // written as T and T' (their blocks above the block diagonal stay zero from
 // the kernel's start), in two steps with a group barrier between them:
-//  1. warp b: D_bb = (I + A_bb)^{-1} by forward substitution (lane c % 16
-//     owns column c), stored over A_bb in AF and, scaled, into T and T';
+//  1. D_bb = (I + A_bb)^{-1} by forward substitution, in the two warps
+//     that wrote A (two blocks each), stored over A_bb in AF and, scaled,
+//     into T and T';
 //  2. strips (column block j, half hf): warp 0 -> (0,0); warp 1 -> (0,1);
 //     warp 2 -> (1,0), (2,0); warp 3 -> (1,1), (2,1).  (An fp32 CUDA-core
 //     strip sweep was faster alone but, competing for issue slots with the
 //     state group, slower in the kernel.)
-__device__ void invert_diag(float *AF, const TOut &o, int t) {
-  const int warp = t >> 5, lane = t & 31;
-  {
-    const int w = warp, c = lane & 15;
-    float x[16];
+__device__ void invert_diag(float *AF, const TOut &o, int pw, int lane) {
+  // warp pw (0 or 1) has just written A rows 32 pw .. 32 pw + 31: lanes
+  // 0-15 invert block 2 pw, lanes 16-31 block 2 pw + 1 (lane c % 16 owns
+  // column c of its block)
+  const int w = 2 * pw + (lane >> 4), c = lane & 15;
+  float x[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
-    const float *Ab = AF + (16 * w) * LDA + 16 * w;
+  for (int i = 0; i < 16; ++i) x[i] = (i == c) ? 1.f : 0.f;
+  const float *Ab = AF + (16 * w) * LDA + 16 * w;
 #pragma unroll
-    for (int i = 1; i < 16; ++i) {
-      float acc0 = 0.f, acc1 = 0.f;
+  for (int i = 1; i < 16; ++i) {
+    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int k4 = 0; k4 < (i + 3) / 4; ++k4) {
-        const float4 av = *reinterpret_cast<const float4 *>(Ab + i * LDA + 4 * k4);
-        if (4 * k4 + 0 < i) acc0 += av.x * x[4 * k4 + 0];
-        if (4 * k4 + 1 < i) acc1 += av.y * x[4 * k4 + 1];
-        if (4 * k4 + 2 < i) acc0 += av.z * x[4 * k4 + 2];
-        if (4 * k4 + 3 < i) acc1 += av.w * x[4 * k4 + 3];
-      }
-      x[i] = (i > c) ? -(acc0 + acc1) : x[i];
+    for (int k4 = 0; k4 < (i + 3) / 4; ++k4) {
+      const float4 av = *reinterpret_cast<const float4 *>(Ab + i * LDA + 4 * k4);
+      if (4 * k4 + 0 < i) acc0 += av.x * x[4 * k4 + 0];
+      if (4 * k4 + 1 < i) acc1 += av.y * x[4 * k4 + 1];
+      if (4 * k4 + 2 < i) acc0 += av.z * x[4 * k4 + 2];
+      if (4 * k4 + 3 < i) acc1 += av.w * x[4 * k4 + 3];
     }
-    __syncwarp();  // every lane has read A_ww
-    if (lane < 16) {
-      float *Yb = AF + (16 * w) * LDA + 16 * w;
+    x[i] = (i > c) ? -(acc0 + acc1) : x[i];
+  }
+  __syncwarp();  // every lane has read its A_ww
+  float *Yb = AF + (16 * w) * LDA + 16 * w;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) Yb[i * LDA + c] = x[i];
-    }
-    // T (lanes 0-15) and T' (lanes 16-31) of the diagonal block, one bf16
-    // per store (no shuffles).
-    const int col = 16 * w + c;
-    const float sc = (lane < 16) ? o.beta[col] : o.beta[col] * o.eg[col];
-    uint8_t *tile = (lane < 16) ? o.t : o.tp;
+  for (int i = 0; i < 16; ++i) Yb[i * LDA + c] = x[i];
+  // T and T' of the diagonal block, one bf16 per store
+  const int col = 16 * w + c;
+  const float bt = o.beta[col], bte = bt * o.eg[col];
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      *reinterpret_cast<__nv_bfloat16 *>(tile + sw128_off(16 * w + i, col)) =
-          __float2bfloat16_rn(x[i] * sc);
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t off = sw128_off(16 * w + i, col);
+    *reinterpret_cast<__nv_bfloat16 *>(o.t + off) = __float2bfloat16_rn(x[i] * bt);
+    *reinterpret_cast<__nv_bfloat16 *>(o.tp + off) = __float2bfloat16_rn(x[i] * bte);
   }
 }
 
@@ -788,15 +786,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&bars[B_D1E]);  // this thread's D1 reads are done
       }
-      // A complete in AF before the inverse; the group agrees on failure.
-      if (group_any(kBar, bad)) { ok = false; break; }
       // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
       const TOut to{sm + Lay::T, sm + Lay::TP + (c & 1) * kTileBytes, bs, egv};
-      bad = (c >= 1 && !warp_wait(&bars[B_UF], (c - 1) & 1, abort_flag, lane)) ||
+      bad = bad || (c >= 1 && !warp_wait(&bars[B_UF], (c - 1) & 1, abort_flag, lane)) ||
             (c >= 2 &&
              !warp_wait(&bars[B_TPE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane));
-      if (!bad) invert_diag(AF, to, pt);
+      if (!bad && rl < 64) {  // the warps that wrote A invert its diagonal blocks
+        __syncwarp();
+        invert_diag(AF, to, rl >> 5, lane);
+      }
+      // A and every D_bb complete in AF; the group agrees on failure.
       if (group_any(kBar, bad)) { ok = false; break; }
       invert_strips(AF, reinterpret_cast<float *>(sm + Lay::SCR), to, pt);
       fence_proxy_async_smem();
