@@ -65,8 +65,6 @@ constexpr uint32_t kTileBytes = 64 * 128;     // one 64 x 64 bf16 tile
 constexpr uint32_t kKQTx = 4 * kTileBytes, kVTx = 2 * kTileBytes;
 constexpr float kSafeDecay = 80.f;            // e^{80} is finite in fp32
 constexpr float kScaleFloor = 0x1p-40f;       // smallest state scale sigma kept
-// Per prep warp: [16][8] product scratch and [48][8] finished strip blocks.
-constexpr int kScrFloats = 16 * 8 + 48 * 8;
 // Row stride (floats) of the fp32 A matrix: rows stay 16-byte aligned and
 // 16 consecutive rows hit distinct 16-byte bank groups pairwise.
 constexpr int LDA = 68;
@@ -87,8 +85,8 @@ struct Lay {
   static constexpr uint32_t VP = P + 2 * kTileBytes;            // V'^T K-major [dv][C]
   static constexpr uint32_t VPD = VP + 2 * kTileBytes;          // decayed, rescaled V'^T
   static constexpr uint32_t AF = VPD + 2 * kTileBytes;          // fp32 A, diagonal blocks -> D
-  static constexpr uint32_t SCR = AF + 64 * LDA * 4;            // 4 x kScrFloats fp32
-  static constexpr uint32_t GS = SCR + 4 * kScrFloats * 4;      // per stage, see kGate*
+  static constexpr uint32_t SCR = AF + 64 * LDA * 4;            // inverse scratch (6 KB)
+  static constexpr uint32_t GS = SCR + (512 + 4 * 256) * 4;     // per stage, see kGate*
   static constexpr uint32_t SVEC = GS + kStages * kGateBytes;   // x2 (state): eg, egl [64]
   static constexpr uint32_t BAR = SVEC + 2 * 512;               // mbarriers
   static constexpr uint32_t MISC = BAR + 32 * 8;                // tmem base, abort flag
@@ -219,10 +217,10 @@ __device__ __forceinline__ bool group_any(uint32_t bar_id, bool pred) {
 
 
 // Bounded wait that also gives up as soon as another role has aborted.
-// The thread sleeps inside try_wait (suspend hint) between checks.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
-                                              volatile int *abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The thread sleeps inside try_wait (suspend hint) between checks.  The
+// slow path is out of line: it is reached rarely and would otherwise be
+// copied into every wait site of the hot loops.
+__device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait_sleep(bar, parity, 20000)) {
     if (*abort_flag) return false;
@@ -232,6 +230,17 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
     }
   }
   return true;
+}
+
+// End-of-kernel drains (bounded, cold): out of line as well.
+__device__ __noinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
+  return mbar_wait_bounded(bar, parity, kWaitNs);
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
+                                              volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, abort_flag);
 }
 
 // Warp-wide wait and abort check (false on time-out or once an abort was
@@ -295,18 +304,18 @@ __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&
 // unchanged and makes each lane's two A elements of a row adjacent.
 struct Frag {
   int g, tq;
-  float *scr;  // warp-private [16][8] fp32 scratch
-  // A fragment of the 16x8 block of AF at (row0, col0).
-  __device__ __forceinline__ void a(const float *AF, int row0, int col0, uint32_t (&af)[4]) const {
-    const float2 lo = *reinterpret_cast<const float2 *>(AF + (row0 + g) * LDA + col0 + 2 * tq);
-    const float2 hi = *reinterpret_cast<const float2 *>(AF + (row0 + g + 8) * LDA + col0 + 2 * tq);
+  float *scr;  // warp-private 2 x [16][8] fp32 scratch
+  // A fragment of the 16x8 block at (row0, col0) of a row-major matrix.
+  __device__ __forceinline__ void a(const float *M, int ld, int row0, int col0,
+                                    uint32_t (&af)[4]) const {
+    const float2 lo = *reinterpret_cast<const float2 *>(M + (row0 + g) * ld + col0 + 2 * tq);
+    const float2 hi = *reinterpret_cast<const float2 *>(M + (row0 + g + 8) * ld + col0 + 2 * tq);
     af[0] = to_tf32(lo.x);
     af[1] = to_tf32(hi.x);
     af[2] = to_tf32(lo.y);
     af[3] = to_tf32(hi.y);
   }
-  // B fragments (two k-steps) of a 16x8 fp32 block stored row-major with
-  // row stride ld floats.
+  // B fragments (two k-steps) of a 16x8 block of a row-major matrix.
   __device__ __forceinline__ void b(const float *blk, int ld, uint32_t (&bf)[2][2]) const {
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
@@ -314,17 +323,42 @@ struct Frag {
       bf[ks][1] = to_tf32(blk[(8 * ks + 2 * tq + 1) * ld + g]);
     }
   }
-  // 16x8 accumulator fragment -> B fragments of two k-steps (rows 0-7, 8-15).
-  __device__ __forceinline__ void to_b(const float (&cf)[4], uint32_t (&bf)[2][2]) const {
-    scr[g * 8 + 2 * tq] = cf[0];
-    scr[g * 8 + 2 * tq + 1] = cf[1];
-    scr[(g + 8) * 8 + 2 * tq] = cf[2];
-    scr[(g + 8) * 8 + 2 * tq + 1] = cf[3];
+  // 16x8 accumulator fragments -> B fragments, through the scratch (one
+  // shared-memory round trip, for one or two fragments).
+  __device__ __forceinline__ void put(float *m, const float (&cf)[4]) const {
+    m[g * 8 + 2 * tq] = cf[0];
+    m[g * 8 + 2 * tq + 1] = cf[1];
+    m[(g + 8) * 8 + 2 * tq] = cf[2];
+    m[(g + 8) * 8 + 2 * tq + 1] = cf[3];
+  }
+  __device__ __forceinline__ void to_b(const float (&c0)[4], uint32_t (&b0)[2][2]) const {
+    put(scr, c0);
     __syncwarp();
-    b(scr, 8, bf);
+    b(scr, 8, b0);
+    __syncwarp();
+  }
+  __device__ __forceinline__ void to_b2(const float (&c0)[4], const float (&c1)[4],
+                                        uint32_t (&b0)[2][2], uint32_t (&b1)[2][2]) const {
+    put(scr, c0);
+    put(scr + 128, c1);
+    __syncwarp();
+    b(scr, 8, b0);
+    b(scr + 128, 8, b1);
     __syncwarp();
   }
 };
+
+// acc (+)= A (16 x 16 block at (row0, col0), two k-steps) * B (16 x 8), with
+// one accumulator per k-step (the caller sums them).
+__device__ __forceinline__ void mma_blk(const Frag &f, const float *M, int ld, int row0, int col0,
+                                        const uint32_t (&bf)[2][2], float (&acc0)[4],
+                                        float (&acc1)[4]) {
+  uint32_t a0[4], a1[4];
+  f.a(M, ld, row0, col0, a0);
+  f.a(M, ld, row0, col0 + 8, a1);
+  mma_tf32_16x8x8(acc0, a0, bf[0]);
+  mma_tf32_16x8x8(acc1, a1, bf[1]);
+}
 
 // Two adjacent columns s, s + 1 (s even) of row r of T and T'.
 __device__ __forceinline__ void store_t2(const TOut &o, int r, int s, float y0, float y1) {
@@ -336,52 +370,6 @@ __device__ __forceinline__ void store_t2(const TOut &o, int r, int s, float y0, 
   *reinterpret_cast<uint32_t *>(o.tp + off) = pack_bf16(t0 * e.x, t1 * e.y);
 }
 
-// One 8-column strip (first column col0) of column block j of
-// Y = (I + A)^{-1}.  With D_bb = (I + A_bb)^{-1} already in the diagonal
-// blocks of AF:  Y_jj = D_jj,  Y_bj = -D_bb sum_{k=j}^{b-1} A_bk Y_kj (b > j),
-// swept down the block rows with mma.sync (TF32 operands rounded to
-// nearest, fp32 accumulation).  Finished blocks go to the warp's scratch
-// `ys` ([48][8], block row b at rows 16 (b - j - 1)) for the rows below,
-// and, scaled, to T and T'.  Runtime loops keep the code small: every warp
-// of the SM runs it each chunk next to the state group's code.
-__device__ __forceinline__ void inverse_strip(const float *AF, float *ys, const Frag &f,
-                                              const TOut &o, int j, int col0) {
-#pragma unroll 1
-  for (int bb = j + 1; bb < 4; ++bb) {
-    float racc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-    for (int k = j; k < bb; ++k) {
-      const float *yblk = (k == j) ? AF + (16 * j) * LDA + col0 : ys + 16 * (k - j - 1) * 8;
-      uint32_t bf[2][2];
-      f.b(yblk, (k == j) ? LDA : 8, bf);
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        uint32_t af[4];
-        f.a(AF, 16 * bb, 16 * k + 8 * ks, af);
-        mma_tf32_16x8x8(racc, af, bf[ks]);
-      }
-    }
-    uint32_t rb[2][2];
-    f.to_b(racc, rb);
-    float yacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t af[4];
-      f.a(AF, 16 * bb, 16 * bb + 8 * ks, af);
-      mma_tf32_16x8x8(yacc, af, rb[ks]);
-    }
-    const float y0 = -yacc[0], y1 = -yacc[1], y2 = -yacc[2], y3 = -yacc[3];
-    float *yo = ys + 16 * (bb - j - 1) * 8;
-    yo[f.g * 8 + 2 * f.tq] = y0;
-    yo[f.g * 8 + 2 * f.tq + 1] = y1;
-    yo[(f.g + 8) * 8 + 2 * f.tq] = y2;
-    yo[(f.g + 8) * 8 + 2 * f.tq + 1] = y3;
-    __syncwarp();
-    store_t2(o, 16 * bb + f.g, col0 + 2 * f.tq, y0, y1);
-    store_t2(o, 16 * bb + f.g + 8, col0 + 2 * f.tq, y2, y3);
-  }
-}
-
 // (I + A)^{-1} for the strictly lower 64x64 fp32 A in AF (row stride LDA,
 // zero above the diagonal) with the 4-warp prep group (local thread t),
 // written as T and T' (their blocks above the block diagonal stay zero from
@@ -389,10 +377,9 @@ __device__ __forceinline__ void inverse_strip(const float *AF, float *ys, const 
 //  1. D_bb = (I + A_bb)^{-1} by forward substitution, in the two warps
 //     that wrote A (two blocks each), stored over A_bb in AF and, scaled,
 //     into T and T';
-//  2. strips (column block j, half hf): warp 0 -> (0,0); warp 1 -> (0,1);
-//     warp 2 -> (1,0), (2,0); warp 3 -> (1,1), (2,1).  (An fp32 CUDA-core
-//     strip sweep was faster alone but, competing for issue slots with the
-//     state group, slower in the kernel.)
+//  2. the off-diagonal blocks in two doubling levels (below), with mma.sync.
+//     (An fp32 CUDA-core sweep was faster alone but, competing for issue
+//     slots with the state group, slower in the kernel.)
 __device__ void invert_diag(float *AF, const TOut &o, int pw, int lane) {
   // warp pw (0 or 1) has just written A rows 32 pw .. 32 pw + 31: lanes
   // 0-15 invert block 2 pw, lanes 16-31 block 2 pw + 1 (lane c % 16 owns
@@ -430,17 +417,68 @@ __device__ void invert_diag(float *AF, const TOut &o, int pw, int lane) {
   }
 }
 
-// Step 2 of the inverse (after a group barrier: every D_bb is in AF).
-__device__ void invert_strips(const float *AF, float *scr, const TOut &o, int t) {
+// Off-diagonal blocks of Y by two doubling levels (with every D_bb in AF):
+//  level 1:  Y_10 = -D_11 A_10 D_00,   Y_32 = -D_33 A_32 D_22;
+//  level 2:  [Y_20 Y_21; Y_30 Y_31] = -[D_22 0; Y_32 D_33] R,
+//            R = [A_20 A_21; A_30 A_31] [D_00 0; Y_10 D_11].
+// Each warp takes one 8-column strip per level (mma.sync TF32, fp32
+// accumulation); Y_10 and Y_32 reach level 2 through the shared scratch
+// `ysc` ([2][16][16]); every block is written, scaled, to T and T'.
+__device__ void invert_level1(const float *AF, float *ysc, float *scr, const TOut &o, int t) {
   const int warp = t >> 5, lane = t & 31;
-  float *ws = scr + warp * kScrFloats;  // [16][8] product scratch, then [48][8] strip blocks
-  const Frag f{lane >> 2, lane & 3, ws};
-  const int hf = warp & 1;
-#pragma unroll 1
-  for (int si = 0; si < (warp < 2 ? 1 : 2); ++si) {
-    const int j = warp < 2 ? 0 : 1 + si;
-    inverse_strip(AF, ws + 128, f, o, j, 16 * j + 8 * hf);
+  const Frag f{lane >> 2, lane & 3, scr + warp * 256};
+  const int jb = warp < 2 ? 0 : 2, blk = jb + 1, cs = 8 * (warp & 1);
+  uint32_t bf[2][2], rb[2][2];
+  f.b(AF + (16 * jb) * LDA + 16 * jb + cs, LDA, bf);  // D_jj strip
+  float r0[4] = {0.f, 0.f, 0.f, 0.f}, r1[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_blk(f, AF, LDA, 16 * blk, 16 * jb, bf, r0, r1);  // A_{blk,jb} D_jj
+  const float r[4] = {r0[0] + r1[0], r0[1] + r1[1], r0[2] + r1[2], r0[3] + r1[3]};
+  f.to_b(r, rb);
+  float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_blk(f, AF, LDA, 16 * blk, 16 * blk, rb, y0, y1);  // D_{blk,blk} R
+  const float y[4] = {-(y0[0] + y1[0]), -(y0[1] + y1[1]), -(y0[2] + y1[2]), -(y0[3] + y1[3])};
+  float *yo = ysc + (jb >> 1) * 256 + cs;  // [16][16]
+  yo[f.g * 16 + 2 * f.tq] = y[0];
+  yo[f.g * 16 + 2 * f.tq + 1] = y[1];
+  yo[(f.g + 8) * 16 + 2 * f.tq] = y[2];
+  yo[(f.g + 8) * 16 + 2 * f.tq + 1] = y[3];
+  store_t2(o, 16 * blk + f.g, 16 * jb + cs + 2 * f.tq, y[0], y[1]);
+  store_t2(o, 16 * blk + f.g + 8, 16 * jb + cs + 2 * f.tq, y[2], y[3]);
+}
+
+// Level 2, after a group barrier (Y_10 and Y_32 in ysc): warp w takes the
+// columns 8 w .. 8 w + 7 of the lower-left 32x32 block.
+__device__ void invert_level2(const float *AF, const float *ysc, float *scr, const TOut &o,
+                              int t) {
+  const int warp = t >> 5, lane = t & 31;
+  const Frag f{lane >> 2, lane & 3, scr + warp * 256};
+  const int jb = warp >> 1, cs = 8 * (warp & 1), col = 16 * jb + cs;
+  float p0[4] = {0.f, 0.f, 0.f, 0.f}, p1[4] = {0.f, 0.f, 0.f, 0.f};  // R_2 (block row 2)
+  float q0[4] = {0.f, 0.f, 0.f, 0.f}, q1[4] = {0.f, 0.f, 0.f, 0.f};  // R_3 (block row 3)
+  uint32_t bf[2][2];
+  if (jb == 0) {  // strip of [D_00; Y_10]
+    f.b(AF + cs, LDA, bf);
+    mma_blk(f, AF, LDA, 32, 0, bf, p0, p1);
+    mma_blk(f, AF, LDA, 48, 0, bf, q0, q1);
+    f.b(ysc + cs, 16, bf);
+  } else {  // strip of [0; D_11]
+    f.b(AF + 16 * LDA + 16 + cs, LDA, bf);
   }
+  mma_blk(f, AF, LDA, 32, 16, bf, p0, p1);
+  mma_blk(f, AF, LDA, 48, 16, bf, q0, q1);
+  const float r2[4] = {p0[0] + p1[0], p0[1] + p1[1], p0[2] + p1[2], p0[3] + p1[3]};
+  const float r3[4] = {q0[0] + q1[0], q0[1] + q1[1], q0[2] + q1[2], q0[3] + q1[3]};
+  uint32_t b2[2][2], b3[2][2];
+  f.to_b2(r2, r3, b2, b3);
+  float u0[4] = {0.f, 0.f, 0.f, 0.f}, u1[4] = {0.f, 0.f, 0.f, 0.f};
+  float v0[4] = {0.f, 0.f, 0.f, 0.f}, v1[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_blk(f, AF, LDA, 32, 32, b2, u0, u1);      // D_22 R_2
+  mma_blk(f, ysc + 256, 16, 0, 0, b2, v0, v1);  // Y_32 R_2
+  mma_blk(f, AF, LDA, 48, 48, b3, v0, v1);      // + D_33 R_3
+  store_t2(o, 32 + f.g, col + 2 * f.tq, -(u0[0] + u1[0]), -(u0[1] + u1[1]));
+  store_t2(o, 40 + f.g, col + 2 * f.tq, -(u0[2] + u1[2]), -(u0[3] + u1[3]));
+  store_t2(o, 48 + f.g, col + 2 * f.tq, -(v0[0] + v1[0]), -(v0[1] + v1[1]));
+  store_t2(o, 56 + f.g, col + 2 * f.tq, -(v0[2] + v1[2]), -(v0[3] + v1[3]));
 }
 
 #ifdef GDR_TC_DEBUG
@@ -583,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) {
         const int c = last_issued[s];
-        if (c >= 0) mbar_wait_bounded(&bars[B_FULL + s], (c / kStages) & 1, kWaitNs);
+        if (c >= 0) drain_wait(&bars[B_FULL + s], (c / kStages) & 1);
       }
     }
   } else if (warp == kVWarp) {
@@ -599,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, c * C, b);
         last = c;
       }
-      if (last >= 0) mbar_wait_bounded(&bars[B_VFULL], last & 1, kWaitNs);
+      if (last >= 0) drain_wait(&bars[B_VFULL], last & 1);
     }
   } else if (warp == kMmaWarp) {
     // ================================================================ state-side MMAs
@@ -666,7 +704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // Drain: all issued MMAs complete before TMEM is released.
       mma_commit(&bars[B_FIN]);
-      mbar_wait_bounded(&bars[B_FIN], 0, kWaitNs);
+      drain_wait(&bars[B_FIN], 0);
       if (!ok) atomicOr(a.status, kStatusTimeout);
     }
   } else if (warp == kPrepMmaWarp) {
@@ -711,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars[B_VEMPTY]);
       }
       mma_commit(&bars[B_FIN2]);
-      mbar_wait_bounded(&bars[B_FIN2], 0, kWaitNs);
+      drain_wait(&bars[B_FIN2], 0);
       if (!ok) atomicOr(a.status, kStatusTimeout);
     }
   } else if (warp >= 4 && warp < 8) {
@@ -761,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               dvs[4 * s4 + 2] = fr * ie.z;
               dvs[4 * s4 + 3] = fr * ie.w;
             }
-          } else {
+          } else {  // rare: chunks whose total decay is beyond e^{-80}
 #pragma unroll
             for (int s4 = 0; s4 < 8; ++s4) {
               const float4 gg = *reinterpret_cast<const float4 *>(gcv + 32 * hp + 4 * s4);
@@ -798,7 +836,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // A and every D_bb complete in AF; the group agrees on failure.
       if (group_any(kBar, bad)) { ok = false; break; }
-      invert_strips(AF, reinterpret_cast<float *>(sm + Lay::SCR), to, pt);
+      {
+        float *ysc = reinterpret_cast<float *>(sm + Lay::SCR);  // [2][16][16]
+        float *wscr = ysc + 512;                                 // 4 warps x 2 x [16][8]
+        invert_level1(AF, ysc, wscr, to, pt);
+        if (group_any(kBar, false)) { ok = false; break; }  // Y_10, Y_32 in ysc
+        invert_level2(AF, ysc, wscr, to, pt);
+      }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_TRDY]);  // this thread's T, T', P writes are done
     }
@@ -832,36 +876,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // S_b = bf16(sigma S_tmem) for the chunk's MMAs.  While sigma * dl (dl:
     // the chunk's decay) stays above the floor only sigma changes; otherwise
     // (fold) S_tmem <- f S_tmem with f = sigma * dl and sigma restarts at 1.
-    // The branch is taken outside the unrolled loops.
     auto pass_from_tmem = [&](float sig, bool fold, float f) {
-      if (fold) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float x[32];
-          tmem_ld32(lane_base + TM_S + 32 * q, x);
-          uint32_t u[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e] * sig, x[2 * e + 1] * sig);
-          tmem_st16u(lane_base + TM_SB + 16 * q, u);
-          float y0[16], y1[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            y0[e] = x[e] * f;
-            y1[e] = x[16 + e] * f;
-          }
-          tmem_st16(lane_base + TM_S + 32 * q, y0);
-          tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
-        }
-      } else {
 #pragma unroll 1
-        for (int q = 0; q < 2; ++q) {
-          float x[64];
-          tmem_ld64(lane_base + TM_S + 64 * q, x);
-          uint32_t u[32];
+      for (int q = 0; q < 4; ++q) {
+        float x[32];
+        tmem_ld32(lane_base + TM_S + 32 * q, x);
+        uint32_t u[16];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = pack_bf16(x[2 * e] * sig, x[2 * e + 1] * sig);
-          tmem_st16u(lane_base + TM_SB + 32 * q, u);
-          tmem_st16u(lane_base + TM_SB + 32 * q + 16, u + 16);
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e] * sig, x[2 * e + 1] * sig);
+        tmem_st16u(lane_base + TM_SB + 16 * q, u);
+        if (fold) {  // rare: write back S_tmem * f
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x[e] *= f;
+          tmem_st16(lane_base + TM_S + 32 * q, *reinterpret_cast<float(*)[16]>(x));
+          tmem_st16(lane_base + TM_S + 32 * q + 16, *reinterpret_cast<float(*)[16]>(x + 16));
         }
       }
       tmem_wait_st();
@@ -877,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
       } else {
         // S_b = bf16(S0); S_tmem = e^{gc_last} S0; sigma = 1 afterwards.
-#pragma unroll
+#pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           float x[32];
           if (a.S0) {
@@ -961,12 +989,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars[B_VPR]);
+      // next chunk's gate factors, while the state update runs
+      float dl = 1.f;
+      if (c + 1 < n && !chunk_vectors(c + 1, dl)) { ok = false; break; }
       // ---- updated S -> S_b for the next chunk, or the final state
       if (!warp_wait(&bars[B_SF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       if (c + 1 < n) {
-        float dl;
-        if (!chunk_vectors(c + 1, dl)) { ok = false; break; }
 #ifdef GDR_TC_DEBUG
         for (int q = 0; q < 4; ++q) {
           float x[32];
@@ -981,7 +1010,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sig = fold ? 1.f : nxt;
         inv = 1.f / sig;
       } else if (a.S_T) {
-#pragma unroll
+#pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           float x[32];
           tmem_ld32(lane_base + TM_S + 32 * q, x);
