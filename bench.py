@@ -39,10 +39,8 @@ L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = {
     "chunk": ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
               "gated_delta_rule_93_b200/csrc/gdr_chunk_simt.cu",
-              "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh",
-              "gated_delta_rule_93_b200/csrc/gdr_abi.cu"],
-    "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu",
-             "gated_delta_rule_93_b200/csrc/gdr_abi.cu"],
+              "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
+    "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu"],
 }
 
 
