@@ -59,7 +59,6 @@ using namespace sm100;
 constexpr int C = 64, DK = 128, DV = 128;
 constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8, kMmaWarp = 9, kVWarp = 10, kPrepMmaWarp = 11;
-constexpr int kStages = 3;                    // K/Q stages
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per wait
 constexpr uint32_t kTileBytes = 64 * 128;     // one 64 x 64 bf16 tile
 constexpr uint32_t kKQTx = 4 * kTileBytes, kVTx = 2 * kTileBytes;
@@ -71,32 +70,47 @@ constexpr int LDA = 68;
 
 // Gate vectors of a stage, written by the K/Q producer (float offsets):
 // gc = cumulative log decay from the chunk start, e^{gc}, e^{-gc},
-// e^{gc_last - gc}, beta.
-constexpr int kGateGc = 0, kGateEg = 64, kGateIeg = 128, kGateEgl = 192, kGateBeta = 256;
-constexpr uint32_t kGateBytes = 320 * 4;
+// e^{gc_last - gc}, beta.  Per-channel gates (PC) use gc = 0 and factors 1
+// here (the decay is inside the scaled K/Q tiles) and add, per key channel,
+// e^{m} and e^{gc_last - m} (m = the cumulative decay at row 31).
+constexpr int kGateGc = 0, kGateEg = 64, kGateIeg = 128, kGateEgl = 192, kGateBeta = 256,
+              kGateEm = 320, kGateEgm = 448;
+// The state group's copy per chunk (float offsets): e^{gc}, e^{gc_last - gc};
+// PC adds e^{m}, e^{gc_last - m} and the state's per-column factor.
+constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256, kSvF = 384;
 
-// Shared-memory layout (byte offsets from a 1024-byte aligned base).
-struct Lay {
-  static constexpr uint32_t KQ = 0;                             // per stage [K_h0|Q_h0|K_h1|Q_h1]
-  static constexpr uint32_t V = KQ + kStages * 4 * kTileBytes;  // [V_h0|V_h1]
-  static constexpr uint32_t T = V + 2 * kTileBytes;             // T  K-major [r][s]
-  static constexpr uint32_t TP = T + kTileBytes;                // T' K-major [r][s], x2
-  static constexpr uint32_t P = TP + 2 * kTileBytes;            // P  K-major [r][s], x2
-  static constexpr uint32_t VP = P + 2 * kTileBytes;            // V'^T K-major [dv][C]
-  static constexpr uint32_t VPD = VP + 2 * kTileBytes;          // decayed, rescaled V'^T
-  static constexpr uint32_t AF = VPD + 2 * kTileBytes;          // fp32 A, diagonal blocks -> D
-  static constexpr uint32_t SCR = AF + 64 * LDA * 4;            // inverse scratch (6 KB)
-  static constexpr uint32_t GS = SCR + (512 + 4 * 256) * 4;     // per stage, see kGate*
-  static constexpr uint32_t SVEC = GS + kStages * kGateBytes;   // x2 (state): eg, egl [64]
-  static constexpr uint32_t BAR = SVEC + 2 * 512;               // mbarriers
-  static constexpr uint32_t MISC = BAR + 32 * 8;                // tmem base, abort flag
+// Per-variant configuration: K/Q stages and the shared-memory layout (byte
+// offsets from a 1024-byte aligned base).  PC (per-channel gates) holds, per
+// stage, the scaled K~, Q~ tiles in place of K, Q and K^ in its own tiles,
+// the fp32 gate tile of the chunk being scaled, and shares T with T' and
+// V'^T with its decayed copy (both identical without a scalar decay).
+template <bool PC>
+struct Cfg {
+  static constexpr int kStages = PC ? 2 : 3;
+  static constexpr uint32_t kGateBytes = (PC ? 576 : 320) * 4;
+  static constexpr uint32_t kSvecBytes = (PC ? 512 : 128) * 4;
+  static constexpr uint32_t KQ = 0;                                          // [K_h0|Q_h0|K_h1|Q_h1]
+  static constexpr uint32_t KH = KQ + kStages * 4 * kTileBytes;              // PC: [Kh_h0|Kh_h1]
+  static constexpr uint32_t GT = KH + (PC ? kStages * 2 * kTileBytes : 0);   // PC: g [64][128]
+  static constexpr uint32_t V = GT + (PC ? 64 * 128 * 4 : 0);                // [V_h0|V_h1]
+  static constexpr uint32_t T = V + 2 * kTileBytes;                          // T  K-major [r][s]
+  static constexpr uint32_t TP = T + (PC ? 0 : kTileBytes);                  // T' K-major, x2
+  static constexpr uint32_t P = TP + 2 * kTileBytes;                         // P  K-major, x2
+  static constexpr uint32_t VP = P + 2 * kTileBytes;                         // V'^T K-major [dv][C]
+  static constexpr uint32_t VPD = VP + (PC ? 0 : 2 * kTileBytes);            // decayed / sigma
+  static constexpr uint32_t AF = VPD + 2 * kTileBytes;                       // fp32 A, D blocks
+  static constexpr uint32_t SCR = AF + 64 * LDA * 4;                         // inverse scratch
+  static constexpr uint32_t GS = SCR + (512 + 4 * 256) * 4;                  // gate vectors
+  static constexpr uint32_t SVEC = GS + kStages * kGateBytes;                // x2 (state group)
+  static constexpr uint32_t BAR = SVEC + 2 * kSvecBytes;                     // mbarriers
+  static constexpr uint32_t MISC = BAR + 32 * 8;                             // tmem base, abort
   static constexpr uint32_t END = MISC + 16;
+  static constexpr size_t kSmemBytes = END + 1024;
+  static_assert(V % 1024 == 0 && T % 1024 == 0 && VPD % 1024 == 0 && AF % 1024 == 0 &&
+                    GT % 1024 == 0,
+                "tile alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
-static_assert(Lay::V % 1024 == 0 && Lay::T % 1024 == 0 && Lay::VPD % 1024 == 0 &&
-                  Lay::AF % 1024 == 0,
-              "tile alignment");
-constexpr size_t kSmemBytes = Lay::END + 1024;
-static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 // mbarrier slots
 enum {
@@ -120,7 +134,8 @@ enum {
   B_TPE = B_PE + 2,    // [2] T' buffer free (after V')                 (commit)
   B_FIN = B_TPE + 2,   // final drain, state-side issuer                (commit)
   B_FIN2,              // final drain, prep-side issuer                 (commit)
-  B_COUNT
+  B_SCALED,            // [2] PC: scaled K~, Q~, K^ of a stage written  (64)
+  B_COUNT = B_SCALED + 2
 };
 static_assert(B_COUNT <= 32, "barrier slots");
 
@@ -496,12 +511,70 @@ __device__ int g_dbg_chunk = 0;
   } while (0)
 #endif
 
+// 2^x with the hardware approximation (ex2.approx, the instruction __expf is
+// built on); the per-channel scaling keeps its logs in base 2.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Per-channel gates, one warp, channels j0 .. j0 + 63 (lane l: the adjacent
+// pair j0 + 2 l, j0 + 2 l + 1): cumulative log decay gc over the chunk (kept
+// in place in the fp32 gate tile gt [64][128], in log2 units), the
+// reference m = gc at row 31, e^{m} and e^{gc_last - m} into the stage's gate
+// vectors, and the operand tiles scaled in place:
+//   K~ = K e^{gc - m},  Q~ = Q e^{gc - m},  K^ = K e^{m - gc}  (bf16),
+// so that K~ K^T, Q~ K^T carry e^{gc_r - gc_s} per channel, and with the
+// state kept as S Diag(e^{m}), Z and O_a carry e^{gc} (decay from the chunk
+// start) and the update V'^T K^ carries e^{m - gc}.  The factors stay within
+// e^{|gc_last| / 2}.
+__device__ void scale_channels(uint8_t *kq, uint8_t *kh, float *gt, float *gv, int j0,
+                               int lane) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int j = j0 + 2 * lane, hh = j >> 6, jc = j & 63;
+  float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 8
+  for (int t = 0; t < 64; ++t) {
+    float2 *p = reinterpret_cast<float2 *>(gt + t * 128 + j);
+    const float2 x = *p;
+    acc.x += x.x * kLog2e;
+    acc.y += x.y * kLog2e;
+    *p = acc;
+  }
+  const float2 m = *reinterpret_cast<const float2 *>(gt + 31 * 128 + j);
+  gv[kGateEm + j] = ex2(m.x);
+  gv[kGateEm + j + 1] = ex2(m.y);
+  gv[kGateEgm + j] = ex2(acc.x - m.x);
+  gv[kGateEgm + j + 1] = ex2(acc.y - m.y);
+  uint8_t *kt = kq + (2 * hh) * kTileBytes, *qt = kt + kTileBytes, *ht = kh + hh * kTileBytes;
+#pragma unroll 4
+  for (int t = 0; t < 64; ++t) {
+    const float2 gl = *reinterpret_cast<const float2 *>(gt + t * 128 + j);
+    const float dx = gl.x - m.x, dy = gl.y - m.y;
+    const float ux = ex2(dx), uy = ex2(dy), vx = ex2(-dx), vy = ex2(-dy);
+    const uint32_t off = sw128_off(t, jc);
+    uint32_t *kp = reinterpret_cast<uint32_t *>(kt + off);
+    uint32_t *qp = reinterpret_cast<uint32_t *>(qt + off);
+    const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(kp));
+    const float2 qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(qp));
+    *kp = pack_bf16(kv.x * ux, kv.y * uy);
+    *qp = pack_bf16(qv.x * ux, qv.y * uy);
+    *reinterpret_cast<uint32_t *>(ht + off) = pack_bf16(kv.x * vx, kv.y * vy);
+  }
+}
+
 // Each SM sub-partition holds a quarter of the register file and three of
 // the block's twelve warps: the launch bound caps registers at 168.
+template <bool PC>
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, ChunkArgs a) {
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmG, ChunkArgs a) {
+  using Lay = Cfg<PC>;
+  constexpr int kStages = Lay::kStages;
+  constexpr uint32_t kGateBytes = Lay::kGateBytes;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~uintptr_t(1023));
@@ -540,13 +613,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&bars[B_FIN], 1);
     mbar_init(&bars[B_FIN2], 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&bars[B_SCALED + s], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
   // T and both T' tiles start at zero: their blocks above the block diagonal
   // are never written afterwards.
-  for (uint32_t off = 16 * tid; off < 3 * kTileBytes; off += 16 * kThreads)
+  for (uint32_t off = 16 * tid; off < (PC ? 2 : 3) * kTileBytes; off += 16 * kThreads)
     *reinterpret_cast<uint4 *>(sm + Lay::T + off) = make_uint4(0u, 0u, 0u, 0u);
+  if (PC) {  // per-channel gates: the scalar gate vectors are constants
+    for (int i = tid; i < kStages * 256; i += kThreads) {
+      float *gv = reinterpret_cast<float *>(sm + Lay::GS + (i >> 8) * kGateBytes);
+      const int k = i & 255;
+      gv[k] = k < 64 ? 0.f : 1.f;  // gc = 0; e^{gc}, e^{-gc}, e^{gc_last - gc} = 1
+    }
+  }
   fence_proxy_async_smem();
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
@@ -564,18 +645,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
     }
-    int last_issued[kStages] = {-1, -1, -1};  // latest chunk loaded into each stage
+    int last_issued[3] = {-1, -1, -1};  // latest chunk loaded into each stage
     for (int c = 0; c < n; ++c) {
       const int s = c % kStages;
       if (c >= kStages &&
           !wait_or_abort(&bars[B_EMPTY + s], ((c / kStages) - 1) & 1, abort_flag))
+        break;
+      // PC: the gate tile is single-buffered; both scaling warps must be done
+      // with the previous chunk's (its barrier is per stage parity, so it
+      // cannot be two phases ahead of this wait).
+      if (PC && c >= 1 &&
+          !wait_or_abort(&bars[B_SCALED + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag))
         break;
       // Testing hook: this chunk's load is never issued, so its consumers'
       // bounded waits run out and the kernel unwinds (no trap, no hang).
       if (c == a.skip_stage_chunk) continue;
       const int t0 = c * C;
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
-      {
+      if (PC) {  // beta only; the gate tile comes with the K/Q loads
+        const size_t tok = ((size_t)b * T + t0 + lane) * H + h;
+        gv[kGateBeta + lane] = t0 + lane < T ? a.beta[tok] : 0.f;
+        gv[kGateBeta + lane + 32] = t0 + lane + 32 < T ? a.beta[tok + (size_t)32 * H] : 0.f;
+      } else {
         float gl0 = 0.f, gl1 = 0.f, b0 = 0.f, b1 = 0.f;
         const size_t tok = ((size_t)b * T + t0 + lane) * H + h;
         if (t0 + lane < T) {
@@ -607,14 +698,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         uint64_t *fb = &bars[B_FULL + s];
-        mbar_arrive_expect_tx(fb, kKQTx);
+        mbar_arrive_expect_tx(fb, kKQTx + (PC ? 64 * 128 * 4 : 0));
         uint8_t *kq = sm + Lay::KQ + s * 4 * kTileBytes;
         tma_load_4d(kq + 0 * kTileBytes, &tmK, fb, 0, h, t0, b);
         tma_load_4d(kq + 1 * kTileBytes, &tmQ, fb, 0, h, t0, b);
         tma_load_4d(kq + 2 * kTileBytes, &tmK, fb, 64, h, t0, b);
         tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, t0, b);
+        if (PC) tma_load_4d(sm + Lay::GT, &tmG, fb, 0, h, t0, b);
       }
       last_issued[s] = c;
+      if (PC) {  // channels 0-63 of this stage's per-channel scaling
+        if (!warp_wait(&bars[B_FULL + s], (c / kStages) & 1, abort_flag, lane)) break;
+        scale_channels(sm + Lay::KQ + s * 4 * kTileBytes, sm + Lay::KH + s * 2 * kTileBytes,
+                       reinterpret_cast<float *>(sm + Lay::GT), gv, 0, lane);
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[B_SCALED + (c & 1)]);
+      }
     }
     // Loads still in flight after an abort land before the CTA exits (a
     // phase that has already completed passes at once).
@@ -624,6 +723,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c >= 0) drain_wait(&bars[B_FULL + s], (c / kStages) & 1);
       }
     }
+  } else if (warp == kVWarp && PC) {
+    // ================================================================ V producer + PC scaling
+    if (lane == 0) tma_prefetch_desc(&tmV);
+    int last = -1;
+    for (int c = 0; c < n; ++c) {
+      const int s = c % kStages;
+      if (!warp_wait(&bars[B_FULL + s], (c / kStages) & 1, abort_flag, lane)) break;
+      float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
+      scale_channels(sm + Lay::KQ + s * 4 * kTileBytes, sm + Lay::KH + s * 2 * kTileBytes,
+                     reinterpret_cast<float *>(sm + Lay::GT), gv, 64, lane);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[B_SCALED + (c & 1)]);
+      if (c >= 1 && !warp_wait(&bars[B_VEMPTY], (c - 1) & 1, abort_flag, lane)) break;
+      if (lane == 0) {
+        uint8_t *vv = sm + Lay::V;
+        mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
+        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, c * C, b);
+        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, c * C, b);
+      }
+      __syncwarp();
+      last = c;
+    }
+    if (lane == 0 && last >= 0) drain_wait(&bars[B_VFULL], last & 1);
   } else if (warp == kVWarp) {
     // ================================================================ V producer
     if (lane == 0) {
@@ -645,6 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_tp = smem_u32(sm + Lay::TP);
       const uint32_t a_p = smem_u32(sm + Lay::P);
       const uint32_t a_vp = smem_u32(sm + Lay::VP), a_vpd = smem_u32(sm + Lay::VPD);
+      const uint32_t a_kh = smem_u32(sm + Lay::KH);
       auto W = [&](int slot, uint32_t parity) {
         const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
         tc_fence_after();
@@ -688,10 +811,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                       ID_N64, kk > 0);
         // S_tmem += (V'^T decayed / sigma) K ;  O_b = V'^T P^T
         if (!(ok = W(B_VPR, ph))) break;
+        // B = K (MN-major); PC: K^ of the stage
+        const uint32_t kb = PC ? a_kh + st * 2 * kTileBytes : kq;
+        const uint32_t kb_lbo = PC ? kTileBytes : 2 * kTileBytes;
 #pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ss(tm + TM_S, sdesc_sw128(a_vpd + kk * 32, 16, 1024),
-                      sdesc_sw128(kq + kk * 2048, 2 * kTileBytes, 1024), ID_S, 1);
+                      sdesc_sw128(kb + kk * 2048, kb_lbo, 1024), ID_S, 1);
         mma_commit(&bars[B_SF]);
         const uint32_t pp = a_p + (c & 1) * kTileBytes;
 #pragma unroll 1
@@ -711,40 +837,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ prep-side MMAs
     if (lane == 0) {
       const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_v = smem_u32(sm + Lay::V);
-      const uint32_t a_t = smem_u32(sm + Lay::T);
+      const uint32_t a_t = smem_u32(sm + Lay::T), a_kh = smem_u32(sm + Lay::KH);
       auto W = [&](int slot, uint32_t parity) {
         const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
         tc_fence_after();
         return ok;
       };
-      auto issue_d1 = [&](int c) {  // D1 = [K; Q] K^T
+      // chunk c's operands ready: K/Q landed, or (PC) scaled
+      auto ready = [&](int c) {
+        return PC ? W(B_SCALED + (c & 1), (c >> 1) & 1)
+                  : W(B_FULL + c % kStages, (c / kStages) & 1);
+      };
+      auto issue_d1 = [&](int c) {  // D1 = [K; Q] K^T   (PC: [K~; Q~] K^T)
         const uint32_t kq = a_kq + (c % kStages) * 4 * kTileBytes;
+        const uint32_t kh = a_kh + (c % kStages) * 2 * kTileBytes;
 #pragma unroll 1
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32;
-          mma_bf16_ss(tm + TM_D1, sdesc_sw128(kq + off, 16, 1024),
-                      sdesc_sw128(kq + off, 16, 1024), ID_D1, kk > 0);
+          const uint32_t boff = PC ? kh + (kk >> 2) * kTileBytes + (kk & 3) * 32 : kq + off;
+          mma_bf16_ss(tm + TM_D1, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(boff, 16, 1024),
+                      ID_D1, kk > 0);
         }
         mma_commit(&bars[B_D1F]);
       };
       // D1 of chunk c + 1 goes out as soon as the prep group has read D1 of
       // chunk c; U^T of chunk c once T is written and the state group has
       // converted the previous V'^T (the accumulator is shared).
-      bool ok = W(B_FULL, 0);
+      bool ok = ready(0);
       if (ok) issue_d1(0);
       for (int c = 0; c < n && ok; ++c) {
         if (c + 1 < n) {
-          if (!(ok = W(B_D1E, c & 1) &&
-                     W(B_FULL + (c + 1) % kStages, ((c + 1) / kStages) & 1)))
-            break;
+          if (!(ok = W(B_D1E, c & 1) && ready(c + 1))) break;
           issue_d1(c + 1);
         }
         if (!(ok = W(B_TRDY, c & 1) && (c < 1 || W(B_VPR, (c - 1) & 1)) && W(B_VFULL, c & 1)))
           break;
+        // PC: T is written into the T' buffer of the chunk
+        const uint32_t tt = PC ? smem_u32(sm + Lay::TP) + (c & 1) * kTileBytes : a_t;
 #pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ss(tm + TM_UV, sdesc_sw128(a_v + kk * 2048, kTileBytes, 1024),
-                      sdesc_sw128(a_t + kk * 32, 16, 1024), ID_U, kk > 0);
+                      sdesc_sw128(tt + kk * 32, 16, 1024), ID_U, kk > 0);
         mma_commit(&bars[B_UF]);
         mma_commit(&bars[B_VEMPTY]);
       }
@@ -826,7 +959,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
-      const TOut to{sm + Lay::T, sm + Lay::TP + (c & 1) * kTileBytes, bs, egv};
+      uint8_t *tpc = sm + Lay::TP + (c & 1) * kTileBytes;
+      const TOut to{PC ? tpc : sm + Lay::T, tpc, bs, egv};
       bad = bad || (c >= 1 && !warp_wait(&bars[B_UF], (c - 1) & 1, abort_flag, lane)) ||
             (c >= 2 &&
              !warp_wait(&bars[B_TPE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane));
@@ -859,19 +993,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     // (no group barrier).  A warp cannot run a whole chunk ahead of another:
     // the count-128 barriers it waits for need the other warps' arrivals.
     auto chunk_vectors = [&](int c, float &dl) -> bool {
-      if (!warp_wait(&bars[B_FULL + c % kStages], (c / kStages) & 1, abort_flag, lane))
-        return false;
+      const bool got =
+          PC ? warp_wait(&bars[B_SCALED + (c & 1)], (c >> 1) & 1, abort_flag, lane)
+             : warp_wait(&bars[B_FULL + c % kStages], (c / kStages) & 1, abort_flag, lane);
+      if (!got) return false;
       // The stage can be refilled while this chunk's O epilogue still runs,
       // so the group keeps its own copy of e^{gc} and e^{gc_last - gc}.
-      float *sv = reinterpret_cast<float *>(sm + Lay::SVEC + (c & 1) * 512);
+      float *sv = reinterpret_cast<float *>(sm + Lay::SVEC + (c & 1) * Lay::kSvecBytes);
       const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * kGateBytes);
-      sv[lane] = gv[kGateEg + lane];
-      sv[lane + 32] = gv[kGateEg + lane + 32];
-      sv[64 + lane] = gv[kGateEgl + lane];
-      sv[64 + lane + 32] = gv[kGateEgl + lane + 32];
+      sv[kSvEg + lane] = gv[kGateEg + lane];
+      sv[kSvEg + lane + 32] = gv[kGateEg + lane + 32];
+      sv[kSvEgl + lane] = gv[kGateEgl + lane];
+      sv[kSvEgl + lane + 32] = gv[kGateEgl + lane + 32];
+      if (PC) {  // per-column factors; the previous chunk's copy is in the other slot
+        const float *pv =
+            reinterpret_cast<const float *>(sm + Lay::SVEC + ((c + 1) & 1) * Lay::kSvecBytes);
+#pragma unroll
+        for (int k = lane; k < 128; k += 32) {
+          const float em = gv[kGateEm + k];
+          sv[kSvEm + k] = em;
+          sv[kSvEgm + k] = gv[kGateEgm + k];
+          // S_tmem after chunk c - 1's update -> S Diag(e^{m_c}) for chunk c
+          sv[kSvF + k] = c == 0 ? em : pv[kSvEgm + k] * em;
+        }
+      }
       __syncwarp();
-      dl = sv[63];
+      dl = sv[kSvEg + 63];
       return true;
+    };
+    // PC: S_tmem <- S_tmem Diag(f) and S_b = bf16 of the result (f: per-column
+    // factors, broadcast from shared memory).
+    auto pass_vec = [&](const float *fv) {
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float x[32];
+        tmem_ld32(lane_base + TM_S + 32 * q, x);
+        const float4 *f4 = reinterpret_cast<const float4 *>(fv + 32 * q);
+#pragma unroll
+        for (int s4 = 0; s4 < 8; ++s4) {
+          const float4 f = f4[s4];
+          x[4 * s4] *= f.x;
+          x[4 * s4 + 1] *= f.y;
+          x[4 * s4 + 2] *= f.z;
+          x[4 * s4 + 3] *= f.w;
+        }
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
+        tmem_st16u(lane_base + TM_SB + 16 * q, u);
+        tmem_st16(lane_base + TM_S + 32 * q, *reinterpret_cast<float(*)[16]>(x));
+        tmem_st16(lane_base + TM_S + 32 * q + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[B_SBR]);
     };
     // S_b = bf16(sigma S_tmem) for the chunk's MMAs.  While sigma * dl (dl:
     // the chunk's decay) stays above the floor only sigma changes; otherwise
@@ -923,15 +1098,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) x[e] = 0.f;
           }
+          if (PC) {  // S Diag(e^{m_0})
+            const float *fv = reinterpret_cast<const float *>(sm + Lay::SVEC) + kSvF + 32 * q;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= fv[e];
+          }
           uint32_t u[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
           tmem_st16u(lane_base + TM_SB + 16 * q, u);
           float y0[16], y1[16];
+          const float dl0 = PC ? 1.f : dl;
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            y0[e] = x[e] * dl;
-            y1[e] = x[16 + e] * dl;
+            y0[e] = x[e] * dl0;
+            y1[e] = x[16 + e] * dl0;
           }
           tmem_st16(lane_base + TM_S + 32 * q, y0);
           tmem_st16(lane_base + TM_S + 32 * q + 16, y1);
@@ -943,8 +1124,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int c = 0; ok && c < n; ++c) {
       const uint32_t ph = c & 1;
-      const float *sv = reinterpret_cast<const float *>(sm + Lay::SVEC + (c & 1) * 512);
-      const float *egv = sv, *eglv = sv + 64;
+      const float *sv = reinterpret_cast<const float *>(sm + Lay::SVEC + (c & 1) * Lay::kSvecBytes);
+      const float *egv = sv + kSvEg, *eglv = sv + kSvEgl;
       // ---- -Z -> bf16 A operand, in place in TMEM
       if (!warp_wait(&bars[B_ZF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
@@ -1004,18 +1185,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           DBG_ROW(57344 + 32 * q, 128, x);
         }
 #endif
-        const float nxt = sig * dl;
-        const bool fold = !(nxt >= kScaleFloor);  // also when dl underflows to 0
-        pass_from_tmem(sig, fold, nxt);
-        sig = fold ? 1.f : nxt;
-        inv = 1.f / sig;
+        if (PC) {
+          pass_vec(reinterpret_cast<const float *>(sm + Lay::SVEC +
+                                                   ((c + 1) & 1) * Lay::kSvecBytes) +
+                   kSvF);
+        } else {
+          const float nxt = sig * dl;
+          const bool fold = !(nxt >= kScaleFloor);  // also when dl underflows to 0
+          pass_from_tmem(sig, fold, nxt);
+          sig = fold ? 1.f : nxt;
+          inv = 1.f / sig;
+        }
       } else if (a.S_T) {
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           float x[32];
           tmem_ld32(lane_base + TM_S + 32 * q, x);
+          if (PC) {  // S = S_tmem Diag(e^{gc_last - m})
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] *= sig;
+            for (int e = 0; e < 32; ++e) x[e] *= sv[kSvEgm + 32 * q + e];
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= sig;
+          }
           DBG_ROW(57344 + 32 * q, 128, x);
           float4 *dst = reinterpret_cast<float4 *>(a.S_T + ((size_t)bh * DV + i) * DK + 32 * q);
 #pragma unroll
@@ -1125,26 +1317,50 @@ bool make_map(CUtensorMap *m, const void *base, int B, int T, int H, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// 4-D map over the per-channel gate g [B, T, H, d] fp32, box = 64 tokens x
+// all 128 channels (512-byte rows, no swizzle).
+bool make_map_gate(CUtensorMap *m, const float *base, int B, int T, int H, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)T * H * d * 4};
+  cuuint32_t box[4] = {(cuuint32_t)d, 1, 64, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool PC>
+cudaError_t launch_variant(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                           const CUtensorMap &mv, const CUtensorMap &mg, cudaStream_t stream) {
+  constexpr size_t smem = Cfg<PC>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gdr_chunk_tc_kernel<PC>
+      <<<(unsigned)((size_t)a.B * a.H), kThreads, smem, stream>>>(mq, mk, mv, mg, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool chunk_tc_supports(const ChunkArgs &a) {
-  return a.bf16 && !a.per_channel && a.dk == DK && a.dv == DV && a.T > 0 &&
-         (size_t)a.B * a.H <= 0x7fffffffu;
+  return a.bf16 && a.dk == DK && a.dv == DV && a.T > 0 && (size_t)a.B * a.H <= 0x7fffffffu;
 }
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
   if (!chunk_tc_supports(a)) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mg;
   if (!make_map(&mq, a.q, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, a.B, a.T, a.H, DK) ||
       !make_map(&mv, a.v, a.B, a.T, a.H, DV))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  gdr_chunk_tc_kernel<<<(unsigned)((size_t)a.B * a.H), kThreads, kSmemBytes, stream>>>(mq, mk, mv,
-                                                                                       a);
-  return cudaGetLastError();
+  if (a.per_channel) {
+    if (!make_map_gate(&mg, a.g, a.B, a.T, a.H, DK)) return cudaErrorInvalidValue;
+    return launch_variant<true>(a, mq, mk, mv, mg, stream);
+  }
+  return launch_variant<false>(a, mq, mk, mv, mq, stream);  // 4th map unused
 }
 
 }  // namespace gdr
