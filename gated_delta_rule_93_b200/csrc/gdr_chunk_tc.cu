@@ -31,8 +31,8 @@
 //
 // Warp roles (one CTA per (b, h), 352 threads):
 //   warps 0-3  "state" group (TMEM lanes = value channels): -Z -> bf16 in
-//              TMEM, V'^T -> bf16 operands, S -> S_b, O epilogue (direct
-//              stores of o);
+//              TMEM, V'^T -> bf16 operands, S -> S_b, O epilogue (each warp
+//              stages its 32 channels and stores them with one TMA store);
 //   warps 4-7  "prep" group, one chunk ahead: gate cumsum, A/P epilogue,
 //              (I + A)^{-1} with T/T' written straight from it;
 //   warp 8     TMA producer of the K/Q stages (three) + g/beta loads;
@@ -571,7 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     gdr_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
-                        const __grid_constant__ CUtensorMap tmG, ChunkArgs a) {
+                        const __grid_constant__ CUtensorMap tmG,
+                        const __grid_constant__ CUtensorMap tmO, ChunkArgs a) {
   using Lay = Cfg<PC>;
   constexpr int kStages = Lay::kStages;
   constexpr uint32_t kGateBytes = Lay::kGateBytes;
@@ -1150,6 +1151,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- V'^T -> bf16 operands (plain, and decayed to the chunk end / sigma)
       if (!warp_wait(&bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
+      if (lane == 0) tma_store_wait_read0();  // the previous o store has read VPD
+      __syncwarp();
 #pragma unroll 1
       for (int q = 0; q < 2; ++q) {
         float x[32];
@@ -1219,9 +1222,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars[B_OF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
-        const int t0 = c * C;
-        const size_t tok0 = ((size_t)b * T + t0) * H + h;
-        const bool full = t0 + C <= T;
+        // The warp stages its 32 channels x 64 tokens (bf16, 64-byte rows)
+        // in its own rows of VPD, free once the state update has read them,
+        // and one lane stores the box with TMA (rows past T are clipped).
+        __nv_bfloat16 *stg = reinterpret_cast<__nv_bfloat16 *>(sm + Lay::VPD + 4096 * warp);
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
           float xa[32], xb[32];
@@ -1254,29 +1258,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             xa[4 * s4 + 3] = ev.w * xa[4 * s4 + 3] + xb[4 * s4 + 3];
           }
           DBG_ROW(49152 + 32 * q, 64, xa);
-          // one bf16 per store: a warp writes 32 adjacent channels (64 bytes)
-          // of one token; full chunks store unconditionally, only a ragged
-          // last chunk takes the guarded loop (chosen outside the loops)
-          __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.o) +
-                               (tok0 + (size_t)(32 * q) * H) * DV + i;
-          const size_t tstep = (size_t)H * DV;  // elements between tokens t and t + 1
-          if (full) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              __stcs(dst, __float2bfloat16_rn(xa[e]));
-              dst += tstep;
-            }
-          } else {
-            const int rem = T - t0 - 32 * q;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (e < rem) __stcs(dst, __float2bfloat16_rn(xa[e]));
-              dst += tstep;
-            }
-          }
+          for (int e = 0; e < 32; ++e) stg[(32 * q + e) * 32 + lane] = __float2bfloat16_rn(xa[e]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(&tmO, stg, 32 * warp, h, c * C, b);
+          tma_store_commit();
         }
       }
     }
+    // stores still reading shared memory or in flight complete before exit
+    if (lane == 0) tma_store_wait0();
     if (!ok && lane == 0) atomicOr(a.status, kStatusTimeout);
   }
 
@@ -1317,6 +1311,21 @@ bool make_map(CUtensorMap *m, const void *base, int B, int T, int H, int d) {
   return r == CUDA_SUCCESS;
 }
 
+// 4-D map over the output o [B, T, H, d] bf16 for the epilogue's stores:
+// box = 64 tokens x 32 channels (one state warp's), 64-byte rows, no swizzle.
+bool make_map_out(CUtensorMap *m, void *base, int B, int T, int H, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+  cuuint32_t box[4] = {32, 1, 64, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 4-D map over the per-channel gate g [B, T, H, d] fp32, box = 64 tokens x
 // all 128 channels (512-byte rows, no swizzle).
 bool make_map_gate(CUtensorMap *m, const float *base, int B, int T, int H, int d) {
@@ -1334,13 +1343,14 @@ bool make_map_gate(CUtensorMap *m, const float *base, int B, int T, int H, int d
 
 template <bool PC>
 cudaError_t launch_variant(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
-                           const CUtensorMap &mv, const CUtensorMap &mg, cudaStream_t stream) {
+                           const CUtensorMap &mv, const CUtensorMap &mg, const CUtensorMap &mo,
+                           cudaStream_t stream) {
   constexpr size_t smem = Cfg<PC>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   gdr_chunk_tc_kernel<PC>
-      <<<(unsigned)((size_t)a.B * a.H), kThreads, smem, stream>>>(mq, mk, mv, mg, a);
+      <<<(unsigned)((size_t)a.B * a.H), kThreads, smem, stream>>>(mq, mk, mv, mg, mo, a);
   return cudaGetLastError();
 }
 
@@ -1352,15 +1362,15 @@ bool chunk_tc_supports(const ChunkArgs &a) {
 
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
   if (!chunk_tc_supports(a)) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv, mg;
+  CUtensorMap mq, mk, mv, mg, mo;
   if (!make_map(&mq, a.q, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, a.B, a.T, a.H, DK) ||
-      !make_map(&mv, a.v, a.B, a.T, a.H, DV))
+      !make_map(&mv, a.v, a.B, a.T, a.H, DV) || !make_map_out(&mo, a.o, a.B, a.T, a.H, DV))
     return cudaErrorInvalidValue;
   if (a.per_channel) {
     if (!make_map_gate(&mg, a.g, a.B, a.T, a.H, DK)) return cudaErrorInvalidValue;
-    return launch_variant<true>(a, mq, mk, mv, mg, stream);
+    return launch_variant<true>(a, mq, mk, mv, mg, mo, stream);
   }
-  return launch_variant<false>(a, mq, mk, mv, mq, stream);  // 4th map unused
+  return launch_variant<false>(a, mq, mk, mv, mq, mo, stream);  // gate map unused
 }
 
 }  // namespace gdr
