@@ -421,14 +421,19 @@ __device__ void invert_diag(float *AF, const TOut &o, int pw, int lane) {
   float *Yb = AF + (16 * w) * LDA + 16 * w;
 #pragma unroll
   for (int i = 0; i < 16; ++i) Yb[i * LDA + c] = x[i];
-  // T and T' of the diagonal block, one bf16 per store
-  const int col = 16 * w + c;
-  const float bt = o.beta[col], bte = bt * o.eg[col];
+  (void)o;  // T and T' of the diagonal blocks: diag_to_t, after the barrier
+}
+
+// T and T' of the four diagonal blocks from D_bb in AF, spread over the 128
+// prep threads (one row pair of four columns each, paired bf16 stores).
+__device__ __forceinline__ void diag_to_t(const float *AF, const TOut &o, int t) {
+  const int blk = t >> 5, r = (t >> 1) & 15, c0 = 8 * (t & 1);  // 8 columns per thread
+  const int row = 16 * blk + r, col = 16 * blk + c0;
+  const float *src = AF + row * LDA + col;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t off = sw128_off(16 * w + i, col);
-    *reinterpret_cast<__nv_bfloat16 *>(o.t + off) = __float2bfloat16_rn(x[i] * bt);
-    *reinterpret_cast<__nv_bfloat16 *>(o.tp + off) = __float2bfloat16_rn(x[i] * bte);
+  for (int p = 0; p < 4; ++p) {
+    const float2 y = *reinterpret_cast<const float2 *>(src + 2 * p);
+    store_t2(o, row, col + 2 * p, y.x, y.y);
   }
 }
 
@@ -971,6 +976,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // A and every D_bb complete in AF; the group agrees on failure.
       if (group_any(kBar, bad)) { ok = false; break; }
+      diag_to_t(AF, to, pt);
       {
         float *ysc = reinterpret_cast<float *>(sm + Lay::SCR);  // [2][16][16]
         float *wscr = ysc + 512;                                 // 4 warps x 2 x [16][8]
