@@ -179,23 +179,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   }
 }
 
-// 64 consecutive TMEM columns of this thread's lane: four loads, one wait.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  float a0[16], a1[16], a2[16], a3[16];
-  tmem_ld16(taddr, a0);
-  tmem_ld16(taddr + 16, a1);
-  tmem_ld16(taddr + 32, a2);
-  tmem_ld16(taddr + 48, a3);
-  tmem_wait_ld();
-#pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    v[e] = a0[e];
-    v[16 + e] = a1[e];
-    v[32 + e] = a2[e];
-    v[48 + e] = a3[e];
-  }
-}
-
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t *v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -258,16 +241,39 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity,
   return wait_slow(bar, parity, abort_flag);
 }
 
-// Warp-wide wait and abort check (false on time-out or once an abort was
-// raised anywhere in the CTA).  Every lane polls the same barrier, flag and
-// timer, so the result is warp-uniform without a shuffle (chained shuffles
+// Waits for N phases at once.  The non-blocking probes are independent, so
+// their latencies overlap (a chain of single waits costs each probe's full
+// latency in turn); only when one of them is incomplete does the thread take
+// the bounded, abort-aware path barrier by barrier.  Uniform per warp when
+// every lane calls it.  A parity of 1 on a barrier that has not completed
+// its first phase passes at once: the first chunks' "previous phase" waits
+// rely on that.
+template <int N>
+__device__ __forceinline__ bool wait_all(uint64_t *const (&bar)[N], const uint32_t (&parity)[N],
+                                         volatile int *abort_flag) {
+  bool done = true;
+#pragma unroll
+  for (int j = 0; j < N; ++j) done &= mbar_test_wait(bar[j], parity[j]);
+  if (done) return true;
+#pragma unroll
+  for (int j = 0; j < N; ++j)
+    if (!wait_or_abort(bar[j], parity[j], abort_flag)) return false;
+  return true;
+}
+
+// Warp-wide wait for one phase (false on time-out or once an abort was
+// raised anywhere in the CTA while waiting).  Every lane polls the same
+// barrier, so the result is warp-uniform without a shuffle (chained shuffles
 // were measured at several hundred cycles each in this kernel).  Warps wait
 // on their own: a group barrier after every wait would make each warp wait
-// for the slowest one as well.
+// for the slowest one as well.  A phase that is already complete returns at
+// once without reading the abort flag (that read, on every hand-off, cost
+// about 4 % of the kernel): a role that keeps finding its phases complete
+// goes on, and the first wait that has to sleep sees the flag.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort_flag, int lane) {
   (void)lane;
-  return wait_or_abort(bar, parity, abort_flag) && !*abort_flag;
+  return wait_or_abort(bar, parity, abort_flag);
 }
 
 // One warp: cumulative log decay of a chunk (g[64] -> gc[64] in log space,
@@ -297,11 +303,10 @@ struct TOut {
   const float *beta, *eg;  // [64]
 };
 
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
+// The tensor core reads the top 19 bits of a tf32 operand register, i.e.
+// fp32 truncated toward zero (error below 2^-10 relative, under the bf16
+// rounding T and T' get afterwards), so no conversion instruction is spent.
+__device__ __forceinline__ uint32_t to_tf32(float x) { return __float_as_uint(x); }
 
 // D += A(16x8, row) * B(8x8, col), tf32 inputs, fp32 accumulate.
 __device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
@@ -904,14 +909,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + st * kGateBytes);
       const float *gcv = gv + kGateGc, *egv = gv + kGateEg, *iegv = gv + kGateIeg;
       const float *bs = gv + kGateBeta;
-      // This warp's waits: the stage, D1, (c >= 2) this P buffer free, and
-      // for the warps writing A (rows 0-63), every strip of the previous
-      // chunk done reading AF (TRDY counts all 128 prep threads).
-      bool bad = !warp_wait(&bars[B_FULL + st], (c / kStages) & 1, abort_flag, lane) ||
-                 !warp_wait(&bars[B_D1F], ph, abort_flag, lane) ||
-                 (c >= 2 &&
-                  !warp_wait(&bars[B_PE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane)) ||
-                 (c >= 1 && pt < 64 && !warp_wait(&bars[B_TRDY], (c - 1) & 1, abort_flag, lane));
+      // This warp's waits, probed together: the stage, D1, this P buffer
+      // free (O_b of chunk c - 2), and for the warps writing A (rows 0-63)
+      // every strip of the previous chunk done reading AF (TRDY counts all
+      // 128 prep threads; the P warps probe D1 again in its place).
+      const bool a_rows = pt < 64;
+      bool bad = !wait_all<4>({&bars[B_FULL + st], &bars[B_D1F], &bars[B_PE + (c & 1)],
+                               a_rows ? &bars[B_TRDY] : &bars[B_D1F]},
+                              {uint32_t((c / kStages) & 1), ph, uint32_t(((c >> 1) - 1) & 1),
+                               a_rows ? uint32_t((c - 1) & 1) : ph},
+                              abort_flag);
       if (!bad) {
         const bool factored = -gcv[63] < kSafeDecay;
         // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns at a time
@@ -959,7 +966,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             st_row32_sw128(sm + Lay::P + (c & 1) * kTileBytes, r, hp, x);
           }
         }
-        fence_proxy_async_smem();
+        if (rl >= 64) fence_proxy_async_smem();  // P is read by the tensor core
         tc_fence_before();
         mbar_arrive(&bars[B_D1E]);  // this thread's D1 reads are done
       }
@@ -967,9 +974,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
       uint8_t *tpc = sm + Lay::TP + (c & 1) * kTileBytes;
       const TOut to{PC ? tpc : sm + Lay::T, tpc, bs, egv};
-      bad = bad || (c >= 1 && !warp_wait(&bars[B_UF], (c - 1) & 1, abort_flag, lane)) ||
-            (c >= 2 &&
-             !warp_wait(&bars[B_TPE + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane));
+      bad = bad || !wait_all<2>({&bars[B_UF], &bars[B_TPE + (c & 1)]},
+                                {uint32_t((c - 1) & 1), uint32_t(((c >> 1) - 1) & 1)}, abort_flag);
       if (!bad && rl < 64) {  // the warps that wrote A invert its diagonal blocks
         __syncwarp();
         invert_diag(AF, to, rl >> 5, lane);
