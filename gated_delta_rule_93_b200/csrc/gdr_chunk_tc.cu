@@ -17,6 +17,7 @@
 //   T    = Y Diag(beta),  T' = T Diag(e^{gc})             -> bf16, smem
 //   Z    = S_b K^T                          (tcgen05, A = S_b from TMEM)
 //   V'^T = V^T T^T - Z T'^T                 (= U^T - S_b W^T with W = T' K)
+//          (scalar gates: T' is stored negated and Z enters as it is)
 //   O^T  = (S_b Q^T) Diag(e^{gc}) + V'^T P^T
 //   S    = e^{gc_last} S + (V'^T Diag(e^{gc_last - gc})) K   (fp32 TMEM acc)
 //
@@ -30,7 +31,7 @@
 // back into it; the bf16 copy is always formed at the true scale.
 //
 // Warp roles (one CTA per (b, h), 352 threads):
-//   warps 0-3  "state" group (TMEM lanes = value channels): -Z -> bf16 in
+//   warps 0-3  "state" group (TMEM lanes = value channels): Z -> bf16 in
 //              TMEM, V'^T -> bf16 operands, S -> S_b, O epilogue (each warp
 //              stages its 32 channels and stores them with one TMA store);
 //   warps 4-7  "prep" group, one chunk ahead: gate cumsum, A/P epilogue,
@@ -123,7 +124,7 @@ enum {
   B_TRDY,              // T, T' and P of a chunk written                (128)
   B_UF,                // U^T written (T read)                          (commit, prep side)
   B_ZF,                // Z written                                     (commit)
-  B_ZR,                // -Z bf16 operand in TMEM                       (128)
+  B_ZR,                // Z (or -Z) bf16 operand in TMEM                (128)
   B_VPF,               // V'^T complete                                 (commit)
   B_VPR,               // V'^T bf16 operands in smem                    (128)
   B_SF,                // state update complete                         (commit)
@@ -380,14 +381,17 @@ __device__ __forceinline__ void mma_blk(const Frag &f, const float *M, int ld, i
   mma_tf32_16x8x8(acc1, a1, bf[1]);
 }
 
-// Two adjacent columns s, s + 1 (s even) of row r of T and T'.
+// Two adjacent columns s, s + 1 (s even) of row r of T and T' (kNegTp: -T',
+// which lets the state side use +Z as its operand).
+template <bool kNegTp>
 __device__ __forceinline__ void store_t2(const TOut &o, int r, int s, float y0, float y1) {
   const float2 b = *reinterpret_cast<const float2 *>(o.beta + s);
   const float2 e = *reinterpret_cast<const float2 *>(o.eg + s);
   const float t0 = y0 * b.x, t1 = y1 * b.y;
   const uint32_t off = sw128_off(r, s);
   *reinterpret_cast<uint32_t *>(o.t + off) = pack_bf16(t0, t1);
-  *reinterpret_cast<uint32_t *>(o.tp + off) = pack_bf16(t0 * e.x, t1 * e.y);
+  const float ex = kNegTp ? -e.x : e.x, ey = kNegTp ? -e.y : e.y;
+  *reinterpret_cast<uint32_t *>(o.tp + off) = pack_bf16(t0 * ex, t1 * ey);
 }
 
 // (I + A)^{-1} for the strictly lower 64x64 fp32 A in AF (row stride LDA,
@@ -431,6 +435,7 @@ __device__ void invert_diag(float *AF, const TOut &o, int pw, int lane) {
 
 // T and T' of the four diagonal blocks from D_bb in AF, spread over the 128
 // prep threads (one row pair of four columns each, paired bf16 stores).
+template <bool kNegTp>
 __device__ __forceinline__ void diag_to_t(const float *AF, const TOut &o, int t) {
   const int blk = t >> 5, r = (t >> 1) & 15, c0 = 8 * (t & 1);  // 8 columns per thread
   const int row = 16 * blk + r, col = 16 * blk + c0;
@@ -438,7 +443,7 @@ __device__ __forceinline__ void diag_to_t(const float *AF, const TOut &o, int t)
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const float2 y = *reinterpret_cast<const float2 *>(src + 2 * p);
-    store_t2(o, row, col + 2 * p, y.x, y.y);
+    store_t2<kNegTp>(o, row, col + 2 * p, y.x, y.y);
   }
 }
 
@@ -449,6 +454,7 @@ __device__ __forceinline__ void diag_to_t(const float *AF, const TOut &o, int t)
 // Each warp takes one 8-column strip per level (mma.sync TF32, fp32
 // accumulation); Y_10 and Y_32 reach level 2 through the shared scratch
 // `ysc` ([2][16][16]); every block is written, scaled, to T and T'.
+template <bool kNegTp>
 __device__ void invert_level1(const float *AF, float *ysc, float *scr, const TOut &o, int t) {
   const int warp = t >> 5, lane = t & 31;
   const Frag f{lane >> 2, lane & 3, scr + warp * 256};
@@ -467,12 +473,13 @@ __device__ void invert_level1(const float *AF, float *ysc, float *scr, const TOu
   yo[f.g * 16 + 2 * f.tq + 1] = y[1];
   yo[(f.g + 8) * 16 + 2 * f.tq] = y[2];
   yo[(f.g + 8) * 16 + 2 * f.tq + 1] = y[3];
-  store_t2(o, 16 * blk + f.g, 16 * jb + cs + 2 * f.tq, y[0], y[1]);
-  store_t2(o, 16 * blk + f.g + 8, 16 * jb + cs + 2 * f.tq, y[2], y[3]);
+  store_t2<kNegTp>(o, 16 * blk + f.g, 16 * jb + cs + 2 * f.tq, y[0], y[1]);
+  store_t2<kNegTp>(o, 16 * blk + f.g + 8, 16 * jb + cs + 2 * f.tq, y[2], y[3]);
 }
 
 // Level 2, after a group barrier (Y_10 and Y_32 in ysc): warp w takes the
 // columns 8 w .. 8 w + 7 of the lower-left 32x32 block.
+template <bool kNegTp>
 __device__ void invert_level2(const float *AF, const float *ysc, float *scr, const TOut &o,
                               int t) {
   const int warp = t >> 5, lane = t & 31;
@@ -500,10 +507,10 @@ __device__ void invert_level2(const float *AF, const float *ysc, float *scr, con
   mma_blk(f, AF, LDA, 32, 32, b2, u0, u1);      // D_22 R_2
   mma_blk(f, ysc + 256, 16, 0, 0, b2, v0, v1);  // Y_32 R_2
   mma_blk(f, AF, LDA, 48, 48, b3, v0, v1);      // + D_33 R_3
-  store_t2(o, 32 + f.g, col + 2 * f.tq, -(u0[0] + u1[0]), -(u0[1] + u1[1]));
-  store_t2(o, 40 + f.g, col + 2 * f.tq, -(u0[2] + u1[2]), -(u0[3] + u1[3]));
-  store_t2(o, 48 + f.g, col + 2 * f.tq, -(v0[0] + v1[0]), -(v0[1] + v1[1]));
-  store_t2(o, 56 + f.g, col + 2 * f.tq, -(v0[2] + v1[2]), -(v0[3] + v1[3]));
+  store_t2<kNegTp>(o, 32 + f.g, col + 2 * f.tq, -(u0[0] + u1[0]), -(u0[1] + u1[1]));
+  store_t2<kNegTp>(o, 40 + f.g, col + 2 * f.tq, -(u0[2] + u1[2]), -(u0[3] + u1[3]));
+  store_t2<kNegTp>(o, 48 + f.g, col + 2 * f.tq, -(v0[0] + v1[0]), -(v0[1] + v1[1]));
+  store_t2<kNegTp>(o, 56 + f.g, col + 2 * f.tq, -(v0[2] + v1[2]), -(v0[3] + v1[3]));
 }
 
 #ifdef GDR_TC_DEBUG
@@ -801,7 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       sdesc_sw128(kq + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32, 16, 1024),
                       ID_N64, kk > 0);
         mma_commit(&bars[B_ZF]);
-        // V'^T = U^T + (-Z) T'^T   (U^T from the prep-side issuer)
+        // V'^T = U^T + Z (-T')^T, or (-Z) T'^T   (U^T from the prep-side issuer)
         if (!(ok = W(B_ZR, ph) && W(B_UF, ph))) break;
         const uint32_t tp = a_tp + (c & 1) * kTileBytes;
 #pragma unroll 1
@@ -932,7 +939,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float x[32];
           tmem_ld32(lane_base + TM_D1 + 32 * hp, x);
           DBG_ROW(32 * hp, 64, x);
-          const int lim = (rl < 64 ? r : r + 1) - 32 * hp;  // A: s < r, P: s <= r
+          const int lim = r + 1 - 32 * hp;  // P: s <= r
           // The decay form is chosen once per chunk, outside the unrolled
           // loops (a branch inside them costs even when it is never taken).
           float dvs[32];
@@ -955,14 +962,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               dvs[4 * s4 + 3] = br * __expf(gr - gg.w);
             }
           }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = (e < lim) ? x[e] * dvs[e] : 0.f;
           if (rl < 64) {
+            // A is not masked: what lands at or above its diagonal is never
+            // read (the diagonal blocks are replaced by their inverses before
+            // any other use, the blocks above them are not used).
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] *= dvs[e];
             float4 *dst = reinterpret_cast<float4 *>(AF + r * LDA + 32 * hp);
 #pragma unroll
             for (int s4 = 0; s4 < 8; ++s4)
               dst[s4] = make_float4(x[4 * s4], x[4 * s4 + 1], x[4 * s4 + 2], x[4 * s4 + 3]);
           } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = (e < lim) ? x[e] * dvs[e] : 0.f;
             st_row32_sw128(sm + Lay::P + (c & 1) * kTileBytes, r, hp, x);
           }
         }
@@ -982,13 +994,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // A and every D_bb complete in AF; the group agrees on failure.
       if (group_any(kBar, bad)) { ok = false; break; }
-      diag_to_t(AF, to, pt);
+      diag_to_t<!PC>(AF, to, pt);
       {
         float *ysc = reinterpret_cast<float *>(sm + Lay::SCR);  // [2][16][16]
         float *wscr = ysc + 512;                                 // 4 warps x 2 x [16][8]
-        invert_level1(AF, ysc, wscr, to, pt);
+        invert_level1<!PC>(AF, ysc, wscr, to, pt);
         if (group_any(kBar, false)) { ok = false; break; }  // Y_10, Y_32 in ysc
-        invert_level2(AF, ysc, wscr, to, pt);
+        invert_level2<!PC>(AF, ysc, wscr, to, pt);
       }
       fence_proxy_async_smem();
       mbar_arrive(&bars[B_TRDY]);  // this thread's T, T', P writes are done
@@ -1016,8 +1028,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * kGateBytes);
       sv[kSvEg + lane] = gv[kGateEg + lane];
       sv[kSvEg + lane + 32] = gv[kGateEg + lane + 32];
-      sv[kSvEgl + lane] = gv[kGateEgl + lane];
-      sv[kSvEgl + lane + 32] = gv[kGateEgl + lane + 32];
+      if (PC || c == 0) {  // scalar gates, c >= 1: written with 1 / sigma by the pass
+        sv[kSvEgl + lane] = gv[kGateEgl + lane];
+        sv[kSvEgl + lane + 32] = gv[kGateEgl + lane + 32];
+      }
       if (PC) {  // per-column factors; the previous chunk's copy is in the other slot
         const float *pv =
             reinterpret_cast<const float *>(sm + Lay::SVEC + ((c + 1) & 1) * Lay::kSvecBytes);
@@ -1084,9 +1098,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars[B_SBR]);
     };
-    // sig: the scale of S_tmem at the next state pass; inv: 1 / the scale
-    // after the chunk in flight, applied to that chunk's state update.
-    float sig = 1.f, inv = 1.f;
+    // sig: the scale of S_tmem at the next state pass.  1 / the scale after
+    // the chunk in flight is applied to that chunk's state update through the
+    // group's copy of e^{gc_last - gc}.
+    float sig = 1.f;
     {
       float dl;
       if (!chunk_vectors(0, dl)) {
@@ -1139,7 +1154,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = c & 1;
       const float *sv = reinterpret_cast<const float *>(sm + Lay::SVEC + (c & 1) * Lay::kSvecBytes);
       const float *egv = sv + kSvEg, *eglv = sv + kSvEgl;
-      // ---- -Z -> bf16 A operand, in place in TMEM
+      // ---- Z (scalar gates: T' is stored negated) or -Z (per-channel gates,
+      //      whose T' buffer is T itself) -> bf16 A operand, in place in TMEM
       if (!warp_wait(&bars[B_ZF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
@@ -1151,10 +1167,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         DBG_ROW(16384 + 32, 64, z1);
         uint32_t u[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(-z0[2 * e], -z0[2 * e + 1]);
+        for (int e = 0; e < 16; ++e)
+          u[e] = PC ? pack_bf16(-z0[2 * e], -z0[2 * e + 1]) : pack_bf16(z0[2 * e], z0[2 * e + 1]);
         tmem_st16u(lane_base + TM_Z, u);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(-z1[2 * e], -z1[2 * e + 1]);
+        for (int e = 0; e < 16; ++e)
+          u[e] = PC ? pack_bf16(-z1[2 * e], -z1[2 * e + 1]) : pack_bf16(z1[2 * e], z1[2 * e + 1]);
         tmem_st16u(lane_base + TM_Z + 16, u);
         tmem_wait_st();
       }
@@ -1175,10 +1193,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int s4 = 0; s4 < 8; ++s4) {
           const float4 e = e4[s4];
-          x[4 * s4] *= e.x * inv;
-          x[4 * s4 + 1] *= e.y * inv;
-          x[4 * s4 + 2] *= e.z * inv;
-          x[4 * s4 + 3] *= e.w * inv;
+          x[4 * s4] *= e.x;
+          x[4 * s4 + 1] *= e.y;
+          x[4 * s4 + 2] *= e.z;
+          x[4 * s4 + 3] *= e.w;
         }
         st_row32_sw128(sm + Lay::VPD, i, q, x);
       }
@@ -1209,7 +1227,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool fold = !(nxt >= kScaleFloor);  // also when dl underflows to 0
           pass_from_tmem(sig, fold, nxt);
           sig = fold ? 1.f : nxt;
-          inv = 1.f / sig;
+          // next chunk's e^{gc_last - gc} / sigma for its update (every warp
+          // writes the same values, from the stage, after its own pass)
+          const float inv = 1.f / sig;
+          const float *gn = reinterpret_cast<const float *>(sm + Lay::GS +
+                                                            ((c + 1) % kStages) * kGateBytes);
+          float *svn = reinterpret_cast<float *>(sm + Lay::SVEC + ((c + 1) & 1) * Lay::kSvecBytes);
+          svn[kSvEgl + lane] = gn[kGateEgl + lane] * inv;
+          svn[kSvEgl + lane + 32] = gn[kGateEgl + lane + 32] * inv;
+          __syncwarp();
         }
       } else if (a.S_T) {
 #pragma unroll 1
