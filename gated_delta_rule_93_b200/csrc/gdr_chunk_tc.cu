@@ -15,6 +15,7 @@
 //   Y    = (I + A)^{-1}  (16x16 diagonal blocks by forward substitution,
 //                          off-diagonal blocks with mma.sync TF32)
 //   T    = Y Diag(beta),  T' = T Diag(e^{gc})             -> bf16, smem
+//          (scalar gates: T' also carries the scale sigma of S_b, below)
 //   Z    = S_b K^T                          (tcgen05, A = S_b from TMEM)
 //   V'^T = V^T T^T - Z T'^T                 (= U^T - S_b W^T with W = T' K)
 //          (scalar gates: T' is stored negated and Z enters as it is)
@@ -28,9 +29,12 @@
 // The fp32 state is held as S = sigma * S_tmem.  A chunk's decay only
 // changes sigma (and scales the next update by 1 / sigma), so S_tmem is
 // rewritten only when sigma falls below 2^-40, where the decay is folded
-// back into it; the bf16 copy is always formed at the true scale.
+// back into it.  The bf16 copy is S_b = bf16(S_tmem); sigma enters through
+// T' and the O epilogue's e^{gc}, which the K/Q producer writes as
+// sigma e^{gc} from the same scale sequence (replayed in the same fp32
+// operations from the chunk decays).
 //
-// Warp roles (one CTA per (b, h), 352 threads):
+// Warp roles (one CTA per (b, h), 384 threads):
 //   warps 0-3  "state" group (TMEM lanes = value channels): Z -> bf16 in
 //              TMEM, V'^T -> bf16 operands, S -> S_b, O epilogue (each warp
 //              stages its 32 channels and stores them with one TMA store);
@@ -76,6 +80,10 @@ constexpr int LDA = 68;
 // e^{m} and e^{gc_last - m} (m = the cumulative decay at row 31).
 constexpr int kGateGc = 0, kGateEg = 64, kGateIeg = 128, kGateEgl = 192, kGateBeta = 256,
               kGateEm = 320, kGateEgm = 448;
+// Scalar gates only (PC keeps e^{m} there): sigma_c e^{gc}, where sigma_c is
+// the scale of the bf16 state copy S_b the chunk's MMAs read (the state
+// group forms S_b from S_tmem unscaled; T' and the O epilogue carry sigma).
+constexpr int kGateSEg = 320;
 // The state group's copy per chunk (float offsets): e^{gc}, e^{gc_last - gc};
 // PC adds e^{m}, e^{gc_last - m} and the state's per-column factor.
 constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256, kSvF = 384;
@@ -88,7 +96,7 @@ constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256, kSvF = 384;
 template <bool PC>
 struct Cfg {
   static constexpr int kStages = PC ? 2 : 3;
-  static constexpr uint32_t kGateBytes = (PC ? 576 : 320) * 4;
+  static constexpr uint32_t kGateBytes = (PC ? 576 : 384) * 4;
   static constexpr uint32_t kSvecBytes = (PC ? 512 : 128) * 4;
   static constexpr uint32_t KQ = 0;                                          // [K_h0|Q_h0|K_h1|Q_h1]
   static constexpr uint32_t KH = KQ + kStages * 4 * kTileBytes;              // PC: [Kh_h0|Kh_h1]
@@ -297,8 +305,8 @@ __device__ __forceinline__ float chunk_cumsum(const float *g, int lane, float &x
 }
 
 // ---------------------------------------------------------------- inverse
-// Output of the inverse: T = Y Diag(beta) and T' = T Diag(e^{gc}) as bf16
-// K-major 128B-swizzled tiles [r][s].
+// Output of the inverse: T = Y Diag(beta) and T' = T Diag(eg) as bf16
+// K-major 128B-swizzled tiles [r][s] (eg: e^{gc}, scalar gates sigma e^{gc}).
 struct TOut {
   uint8_t *t, *tp;
   const float *beta, *eg;  // [64]
@@ -664,6 +672,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmK);
     }
     int last_issued[3] = {-1, -1, -1};  // latest chunk loaded into each stage
+    // Scalar gates: the state group's scale sequence, replayed with the same
+    // fp32 operations: sig = the scale of S_b for the chunk being produced.
+    float sig = 1.f;
     for (int c = 0; c < n; ++c) {
       const int s = c % kStages;
       if (c >= kStages &&
@@ -712,6 +723,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         gv[kGateEgl + lane + 32] = __expf(gl - x1);
         gv[kGateBeta + lane] = b0;
         gv[kGateBeta + lane + 32] = b1;
+        gv[kGateSEg + lane] = sig * __expf(x0);
+        gv[kGateSEg + lane + 32] = sig * __expf(x1);
+        // the scale after this chunk: 1 after chunk 0 (its decay goes into
+        // S_tmem), else sig * decay unless that falls below the floor
+        const float nxt = sig * __expf(gl);  // the decay e^{gc_last} as stored above
+        sig = (c == 0 || !(nxt >= kScaleFloor)) ? 1.f : nxt;
       }
       __syncwarp();
       if (lane == 0) {
@@ -985,7 +1002,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
       uint8_t *tpc = sm + Lay::TP + (c & 1) * kTileBytes;
-      const TOut to{PC ? tpc : sm + Lay::T, tpc, bs, egv};
+      const TOut to{PC ? tpc : sm + Lay::T, tpc, bs, PC ? egv : gv + kGateSEg};
       bad = bad || !wait_all<2>({&bars[B_UF], &bars[B_TPE + (c & 1)]},
                                 {uint32_t((c - 1) & 1), uint32_t(((c >> 1) - 1) & 1)}, abort_flag);
       if (!bad && rl < 64) {  // the warps that wrote A invert its diagonal blocks
@@ -1026,8 +1043,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // so the group keeps its own copy of e^{gc} and e^{gc_last - gc}.
       float *sv = reinterpret_cast<float *>(sm + Lay::SVEC + (c & 1) * Lay::kSvecBytes);
       const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * kGateBytes);
-      sv[kSvEg + lane] = gv[kGateEg + lane];
-      sv[kSvEg + lane + 32] = gv[kGateEg + lane + 32];
+      constexpr int kEg = PC ? kGateEg : kGateSEg;  // O epilogue: sigma e^{gc}
+      sv[kSvEg + lane] = gv[kEg + lane];
+      sv[kSvEg + lane + 32] = gv[kEg + lane + 32];
       if (PC || c == 0) {  // scalar gates, c >= 1: written with 1 / sigma by the pass
         sv[kSvEgl + lane] = gv[kGateEgl + lane];
         sv[kSvEgl + lane + 32] = gv[kGateEgl + lane + 32];
@@ -1045,7 +1063,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      dl = sv[kSvEg + 63];
+      dl = gv[kGateEg + 63];
       return true;
     };
     // PC: S_tmem <- S_tmem Diag(f) and S_b = bf16 of the result (f: per-column
@@ -1075,17 +1093,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&bars[B_SBR]);
     };
-    // S_b = bf16(sigma S_tmem) for the chunk's MMAs.  While sigma * dl (dl:
-    // the chunk's decay) stays above the floor only sigma changes; otherwise
-    // (fold) S_tmem <- f S_tmem with f = sigma * dl and sigma restarts at 1.
-    auto pass_from_tmem = [&](float sig, bool fold, float f) {
+    // S_b = bf16(S_tmem) for the chunk's MMAs (true state / sigma: T' and
+    // the O epilogue carry sigma).  While sigma * dl (dl: the chunk's decay)
+    // stays above the floor only sigma changes; otherwise (fold) S_tmem <-
+    // f S_tmem with f = sigma * dl and sigma restarts at 1.
+    auto pass_from_tmem = [&](bool fold, float f) {
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float x[32];
         tmem_ld32(lane_base + TM_S + 32 * q, x);
         uint32_t u[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e] * sig, x[2 * e + 1] * sig);
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
         tmem_st16u(lane_base + TM_SB + 16 * q, u);
         if (fold) {  // rare: write back S_tmem * f
 #pragma unroll
@@ -1225,7 +1244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const float nxt = sig * dl;
           const bool fold = !(nxt >= kScaleFloor);  // also when dl underflows to 0
-          pass_from_tmem(sig, fold, nxt);
+          pass_from_tmem(fold, nxt);
           sig = fold ? 1.f : nxt;
           // next chunk's e^{gc_last - gc} / sigma for its update (every warp
           // writes the same values, from the stage, after its own pass)
