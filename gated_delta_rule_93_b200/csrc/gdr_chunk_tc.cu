@@ -188,6 +188,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   }
 }
 
+// 16 TMEM lanes x 32 columns (shape 16x256b, 4 repeats): for column group
+// k (8 columns), thread t holds lane t / 4 at columns 8 k + 2 (t % 4) and
+// + 1 (v[4 k], v[4 k + 1]) and lane t / 4 + 8 at the same columns
+// (v[4 k + 2], v[4 k + 3]).  No wait.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Four 8x8 b16 matrices stored transposed: register j of thread t holds
+// elements (t / 4, 2 (t % 4)) and (t / 4, 2 (t % 4) + 1) of matrix j, which
+// land in memory rows 2 (t % 4) and 2 (t % 4) + 1, column t / 4; threads
+// 8 j .. 8 j + 7 give the 16-byte aligned row addresses of matrix j.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1,
+                                                  uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t *v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -1279,49 +1307,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(&bars[B_OF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
-        // The warp stages its 32 channels x 64 tokens (bf16, 64-byte rows)
-        // in its own rows of VPD, free once the state update has read them,
-        // and one lane stores the box with TMA (rows past T are clipped).
-        __nv_bfloat16 *stg = reinterpret_cast<__nv_bfloat16 *>(sm + Lay::VPD + 4096 * warp);
+        // The warp stages its 32 channels x 64 tokens (bf16, [token][channel],
+        // 64-byte rows) in its own rows of VPD, free once the state update
+        // has read them, and one lane stores the box with TMA (rows past T
+        // are clipped).  O is read in the 16-lane shape, which gives each
+        // thread two adjacent tokens of a channel, so one transposing matrix
+        // store writes 8 tokens x 32 channels per warp.
+        const uint32_t stg = smem_u32(sm + Lay::VPD + 4096 * warp);
+        // row address of this thread in a matrix store: token 8 k + lane % 8
+        // of channel group lane / 8 (matrix j = lane / 8 holds channels
+        // 8 j .. 8 j + 7)
+        const uint32_t row_addr = stg + (lane & 7) * 64 + 16 * (lane >> 3);
+        const int tq = lane & 3;
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
-          float xa[32], xb[32];
-          {
-            float a0[16], a1[16], b0[16], b1[16];
-            tmem_ld16(lane_base + TM_OA + 32 * q, a0);
-            tmem_ld16(lane_base + TM_OA + 32 * q + 16, a1);
-            tmem_ld16(lane_base + TM_O + 32 * q, b0);
-            tmem_ld16(lane_base + TM_O + 32 * q + 16, b1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              xa[e] = a0[e];
-              xa[16 + e] = a1[e];
-              xb[e] = b0[e];
-              xb[16 + e] = b1[e];
-            }
-          }
+          // lanes 0-15 / 16-31 of the warp's quarter, tokens 32 q .. 32 q + 31
+          float a0[16], a1[16], b0[16], b1[16];
+          tmem_ld16x256b_x4(lane_base + TM_OA + 32 * q, a0);
+          tmem_ld16x256b_x4(lane_base + (16u << 16) + TM_OA + 32 * q, a1);
+          tmem_ld16x256b_x4(lane_base + TM_O + 32 * q, b0);
+          tmem_ld16x256b_x4(lane_base + (16u << 16) + TM_O + 32 * q, b1);
+          tmem_wait_ld();
           if (q == 1) {  // every read of O_a / O_b is done
             tc_fence_before();
             mbar_arrive(&bars[B_OE]);
           }
-          const float4 *e4 = reinterpret_cast<const float4 *>(egv + 32 * q);
 #pragma unroll
-          for (int s4 = 0; s4 < 8; ++s4) {
-            const float4 ev = e4[s4];
-            xa[4 * s4 + 0] = ev.x * xa[4 * s4 + 0] + xb[4 * s4 + 0];
-            xa[4 * s4 + 1] = ev.y * xa[4 * s4 + 1] + xb[4 * s4 + 1];
-            xa[4 * s4 + 2] = ev.z * xa[4 * s4 + 2] + xb[4 * s4 + 2];
-            xa[4 * s4 + 3] = ev.w * xa[4 * s4 + 3] + xb[4 * s4 + 3];
+          for (int k = 0; k < 4; ++k) {  // tokens 32 q + 8 k + 2 tq, + 1
+            const float2 ev = *reinterpret_cast<const float2 *>(egv + 32 * q + 8 * k + 2 * tq);
+            const int e = 4 * k;
+            stmatrix_x4_trans(
+                row_addr + (4 * q + k) * 512,
+                pack_bf16(ev.x * a0[e] + b0[e], ev.y * a0[e + 1] + b0[e + 1]),
+                pack_bf16(ev.x * a0[e + 2] + b0[e + 2], ev.y * a0[e + 3] + b0[e + 3]),
+                pack_bf16(ev.x * a1[e] + b1[e], ev.y * a1[e + 1] + b1[e + 1]),
+                pack_bf16(ev.x * a1[e + 2] + b1[e + 2], ev.y * a1[e + 3] + b1[e + 3]));
           }
-          DBG_ROW(49152 + 32 * q, 64, xa);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) stg[(32 * q + e) * 32 + lane] = __float2bfloat16_rn(xa[e]);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_4d(&tmO, stg, 32 * warp, h, c * C, b);
+          tma_store_4d(&tmO, sm + Lay::VPD + 4096 * warp, 32 * warp, h, c * C, b);
           tma_store_commit();
         }
       }
