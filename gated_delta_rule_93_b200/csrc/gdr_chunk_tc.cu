@@ -128,22 +128,22 @@ enum {
   B_VFULL = 6,         // V landed                                      (1 + tx)
   B_VEMPTY,            // V free (prep commit after U)                  (commit)
   B_D1F,               // D1 written                                    (commit, prep side)
-  B_D1E,               // D1 read by the prep group                     (128)
-  B_TRDY,              // T, T' and P of a chunk written                (128)
+  B_D1E,               // D1 read by the prep group                     (4 warps)
+  B_TRDY,              // T, T' and P of a chunk written                (4 warps)
   B_UF,                // U^T written (T read)                          (commit, prep side)
   B_ZF,                // Z written                                     (commit)
-  B_ZR,                // Z (or -Z) bf16 operand in TMEM                (128)
+  B_ZR,                // Z (or -Z) bf16 operand in TMEM                (4 warps)
   B_VPF,               // V'^T complete                                 (commit)
-  B_VPR,               // V'^T bf16 operands in smem                    (128)
+  B_VPR,               // V'^T bf16 operands in smem                    (4 warps)
   B_SF,                // state update complete                         (commit)
   B_OF,                // O_a, O_b complete                             (commit)
-  B_SBR,               // S_b in TMEM for the next chunk                (128)
-  B_OE,                // O_a, O_b read by the epilogue                 (128)
+  B_SBR,               // S_b in TMEM for the next chunk                (4 warps)
+  B_OE,                // O_a, O_b read by the epilogue                 (4 warps)
   B_PE,                // [2] P buffer free (after O_b)                 (commit)
   B_TPE = B_PE + 2,    // [2] T' buffer free (after V')                 (commit)
   B_FIN = B_TPE + 2,   // final drain, state-side issuer                (commit)
   B_FIN2,              // final drain, prep-side issuer                 (commit)
-  B_SCALED,            // [2] PC: scaled K~, Q~, K^ of a stage written  (64)
+  B_SCALED,            // [2] PC: scaled K~, Q~, K^ of a stage written  (2 warps)
   B_COUNT = B_SCALED + 2
 };
 static_assert(B_COUNT <= 32, "barrier slots");
@@ -252,12 +252,13 @@ __device__ __forceinline__ bool group_any(uint32_t bar_id, bool pred) {
 
 
 // Bounded wait that also gives up as soon as another role has aborted.
-// The thread sleeps inside try_wait (suspend hint) between checks.  The
-// slow path is out of line: it is reached rarely and would otherwise be
+// The thread blocks inside try_wait (for the hardware's default time)
+// between checks; a long suspend hint was measured to wake it later after
+// the phase completes.  The slow path is out of line: it would otherwise be
 // copied into every wait site of the hot loops.
 __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait_sleep(bar, parity, 20000)) {
+  while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > kWaitNs) {
       *abort_flag = 1;
@@ -311,6 +312,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity,
                                           volatile int *abort_flag, int lane) {
   (void)lane;
   return wait_or_abort(bar, parity, abort_flag);
+}
+
+// One arrival per warp: every lane's earlier writes and fences are ordered
+// before lane 0's (release) arrive by the warp barrier.  Per-thread
+// arrivals on one barrier word serialise: a group of 128 was measured at
+// several hundred cycles per hand-off.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // One warp: cumulative log decay of a chunk (g[64] -> gc[64] in log space,
@@ -650,24 +660,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[B_VFULL], 1);
     mbar_init(&bars[B_VEMPTY], 1);
     mbar_init(&bars[B_D1F], 1);
-    mbar_init(&bars[B_D1E], 128);
-    mbar_init(&bars[B_TRDY], 128);
+    mbar_init(&bars[B_D1E], 4);
+    mbar_init(&bars[B_TRDY], 4);
     mbar_init(&bars[B_UF], 1);
     mbar_init(&bars[B_ZF], 1);
-    mbar_init(&bars[B_ZR], 128);
+    mbar_init(&bars[B_ZR], 4);
     mbar_init(&bars[B_VPF], 1);
-    mbar_init(&bars[B_VPR], 128);
+    mbar_init(&bars[B_VPR], 4);
     mbar_init(&bars[B_SF], 1);
     mbar_init(&bars[B_OF], 1);
-    mbar_init(&bars[B_SBR], 128);
-    mbar_init(&bars[B_OE], 128);
+    mbar_init(&bars[B_SBR], 4);
+    mbar_init(&bars[B_OE], 4);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_PE + s], 1);
       mbar_init(&bars[B_TPE + s], 1);
     }
     mbar_init(&bars[B_FIN], 1);
     mbar_init(&bars[B_FIN2], 1);
-    for (int s = 0; s < 2; ++s) mbar_init(&bars[B_SCALED + s], 64);
+    for (int s = 0; s < 2; ++s) mbar_init(&bars[B_SCALED + s], 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -775,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         scale_channels(sm + Lay::KQ + s * 4 * kTileBytes, sm + Lay::KH + s * 2 * kTileBytes,
                        reinterpret_cast<float *>(sm + Lay::GT), gv, 0, lane);
         fence_proxy_async_smem();
-        mbar_arrive(&bars[B_SCALED + (c & 1)]);
+        warp_arrive(&bars[B_SCALED + (c & 1)]);
       }
     }
     // Loads still in flight after an abort land before the CTA exits (a
@@ -797,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       scale_channels(sm + Lay::KQ + s * 4 * kTileBytes, sm + Lay::KH + s * 2 * kTileBytes,
                      reinterpret_cast<float *>(sm + Lay::GT), gv, 64, lane);
       fence_proxy_async_smem();
-      mbar_arrive(&bars[B_SCALED + (c & 1)]);
+      warp_arrive(&bars[B_SCALED + (c & 1)]);
       if (c >= 1 && !warp_wait(&bars[B_VEMPTY], (c - 1) & 1, abort_flag, lane)) break;
       if (lane == 0) {
         uint8_t *vv = sm + Lay::V;
@@ -964,7 +974,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // This warp's waits, probed together: the stage, D1, this P buffer
       // free (O_b of chunk c - 2), and for the warps writing A (rows 0-63)
       // every strip of the previous chunk done reading AF (TRDY counts all
-      // 128 prep threads; the P warps probe D1 again in its place).
+      // four prep warps; the P warps probe D1 again in its place).
       const bool a_rows = pt < 64;
       bool bad = !wait_all<4>({&bars[B_FULL + st], &bars[B_D1F], &bars[B_PE + (c & 1)],
                                a_rows ? &bars[B_TRDY] : &bars[B_D1F]},
@@ -1025,7 +1035,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (rl >= 64) fence_proxy_async_smem();  // P is read by the tensor core
         tc_fence_before();
-        mbar_arrive(&bars[B_D1E]);  // this thread's D1 reads are done
+        warp_arrive(&bars[B_D1E]);  // this thread's D1 reads are done
       }
       // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
@@ -1048,7 +1058,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         invert_level2<!PC>(AF, ysc, wscr, to, pt);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bars[B_TRDY]);  // this thread's T, T', P writes are done
+      warp_arrive(&bars[B_TRDY]);  // this thread's T, T', P writes are done
     }
     if (!ok && pt == 0) atomicOr(a.status, kStatusTimeout);
   } else if (warp < 4) {
@@ -1061,7 +1071,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // into SVEC[c & 1]; returns the chunk's total decay e^{gc_last}.
     // Every warp writes the same values and reads them after its own writes
     // (no group barrier).  A warp cannot run a whole chunk ahead of another:
-    // the count-128 barriers it waits for need the other warps' arrivals.
+    // the four-warp barriers it waits for need the other warps' arrivals.
     auto chunk_vectors = [&](int c, float &dl) -> bool {
       const bool got =
           PC ? warp_wait(&bars[B_SCALED + (c & 1)], (c >> 1) & 1, abort_flag, lane)
@@ -1119,7 +1129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_SBR]);
+      warp_arrive(&bars[B_SBR]);
     };
     // S_b = bf16(S_tmem) for the chunk's MMAs (true state / sigma: T' and
     // the O epilogue carry sigma).  While sigma * dl (dl: the chunk's decay)
@@ -1143,7 +1153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_SBR]);
+      warp_arrive(&bars[B_SBR]);
     };
     // sig: the scale of S_tmem at the next state pass.  1 / the scale after
     // the chunk in flight is applied to that chunk's state update through the
@@ -1194,7 +1204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[B_SBR]);
+        warp_arrive(&bars[B_SBR]);
       }
     }
     for (int c = 0; ok && c < n; ++c) {
@@ -1224,7 +1234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&bars[B_ZR]);
+      warp_arrive(&bars[B_ZR]);
       // ---- V'^T -> bf16 operands (plain, and decayed to the chunk end / sigma)
       if (!warp_wait(&bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
@@ -1249,7 +1259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars[B_VPR]);
+      warp_arrive(&bars[B_VPR]);
       // next chunk's gate factors, while the state update runs
       float dl = 1.f;
       if (c + 1 < n && !chunk_vectors(c + 1, dl)) { ok = false; break; }
@@ -1330,7 +1340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           if (q == 1) {  // every read of O_a / O_b is done
             tc_fence_before();
-            mbar_arrive(&bars[B_OE]);
+            warp_arrive(&bars[B_OE]);
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k) {  // tokens 32 q + 8 k + 2 tq, + 1
