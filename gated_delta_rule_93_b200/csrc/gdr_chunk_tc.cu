@@ -1326,8 +1326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t stg = smem_u32(sm + Lay::VPD + 4096 * warp);
         // row address of this thread in a matrix store: token 8 k + lane % 8
         // of channel group lane / 8 (matrix j = lane / 8 holds channels
-        // 8 j .. 8 j + 7)
-        const uint32_t row_addr = stg + (lane & 7) * 64 + 16 * (lane >> 3);
+        // 8 j .. 8 j + 7).  The staging tile is 64-byte swizzled (16-byte
+        // chunk j of row r at chunk j ^ ((r / 2) % 4), as the TMA store
+        // expects), so the 8 rows of a matrix fall in distinct banks.
+        const int r8 = lane & 7;
+        const uint32_t row_addr = stg + r8 * 64 + 16 * ((lane >> 3) ^ ((r8 >> 1) & 3));
         const int tq = lane & 3;
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
@@ -1405,7 +1408,8 @@ bool make_map(CUtensorMap *m, const void *base, int B, int T, int H, int d) {
 }
 
 // 4-D map over the output o [B, T, H, d] bf16 for the epilogue's stores:
-// box = 64 tokens x 32 channels (one state warp's), 64-byte rows, no swizzle.
+// box = 64 tokens x 32 channels (one state warp's), 64-byte rows, 64-byte
+// swizzle (16-byte chunk j of row r lands at chunk j ^ ((r / 2) % 4)).
 bool make_map_out(CUtensorMap *m, void *base, int B, int T, int H, int d) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -1414,7 +1418,7 @@ bool make_map_out(CUtensorMap *m, void *base, int B, int T, int H, int d) {
   cuuint32_t box[4] = {32, 1, 64, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
