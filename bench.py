@@ -39,6 +39,7 @@ L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = {
     "chunk": ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
               "gated_delta_rule_93_b200/csrc/gdr_chunk_simt.cu",
+              "gated_delta_rule_93_b200/csrc/gdr_segments.cu",
               "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
     "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu"],
 }
@@ -174,6 +175,7 @@ def run_ours(args, rank, world, local_rank):
         S = d["S0"].clone()
         o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
         it = [0]
+        launches_per_step = 1
 
         def step():
             i = it[0] % nsteps
@@ -187,10 +189,16 @@ def run_ours(args, rank, world, local_rank):
         o = torch.empty(w.B, w.T, w.H, w.dv, dtype=w.dtype, device=dev)
         S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev) \
             if w.want_S_T else None
+        # scratch of the segment path (long sequences with few heads), if any
+        ws_bytes = binding.chunk_fwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.C, w.dtype,
+                                                     w.gate)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+        launches_per_step = binding.chunk_fwd_kernel_launches(w.B, w.T, w.H, w.dk, w.dv, w.C,
+                                                              w.dtype, w.gate)
 
         def step():
             binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o,
-                              S_T=S_T, output_final_state=S_T is not None)
+                              S_T=S_T, output_final_state=S_T is not None, workspace=ws)
 
     def barrier():
         if world > 1:
@@ -313,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline and w.kind == "chunk":

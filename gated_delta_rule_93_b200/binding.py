@@ -26,6 +26,7 @@ GDR_GATE_SCALAR, GDR_GATE_PER_CHANNEL = 0, 1
 
 EXPORTS = (
     "gdr_chunk_fwd_workspace_bytes",
+    "gdr_chunk_fwd_kernel_launches",
     "gdr_chunk_fwd",
     "gdr_step",
     "gdr_get_device_status",
@@ -55,6 +56,8 @@ def lib():
             vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
             L.gdr_chunk_fwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i, i]
             L.gdr_chunk_fwd_workspace_bytes.restype = sz
+            L.gdr_chunk_fwd_kernel_launches.argtypes = [i, i, i, i, i, i, i, i]
+            L.gdr_chunk_fwd_kernel_launches.restype = i
             L.gdr_chunk_fwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, i, i, i, i, i, i,
                                         vp, sz, vp]
             L.gdr_chunk_fwd.restype = i
@@ -118,6 +121,12 @@ def _in_dtype(dt):
 def chunk_fwd_workspace_bytes(B, T, H, dk, dv, C=64, dtype=torch.bfloat16, gate="scalar"):
     gk = GDR_GATE_PER_CHANNEL if gate == "channel" else GDR_GATE_SCALAR
     return int(lib().gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, _in_dtype(dtype), gk))
+
+
+def chunk_fwd_kernel_launches(B, T, H, dk, dv, C=64, dtype=torch.bfloat16, gate="scalar"):
+    """Kernels one ``chunk_fwd`` call launches on the current device."""
+    gk = GDR_GATE_PER_CHANNEL if gate == "channel" else GDR_GATE_SCALAR
+    return int(lib().gdr_chunk_fwd_kernel_launches(B, T, H, dk, dv, C, _in_dtype(dtype), gk))
 
 
 def chunk_fwd(q, k, v, g, beta, S0=None, *, output_final_state=True, o=None, S_T=None, C=64,

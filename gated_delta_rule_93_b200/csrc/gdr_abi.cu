@@ -39,6 +39,48 @@ gdr_status from_cuda(cudaError_t e, const char *what) {
   return fail(GDR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// Number of SMs of the current device (cached per device; 0 if unknown).
+int device_sms() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// The arguments as the kernels see them (no pointers).
+gdr::ChunkArgs chunk_shape(int B, int T, int H, int dk, int dv, gdr_dtype in_dtype,
+                           gdr_gate_kind gate) {
+  gdr::ChunkArgs a{};
+  a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
+  a.bf16 = in_dtype == GDR_BF16;
+  a.per_channel = gate == GDR_GATE_PER_CHANNEL;
+  a.skip_stage_chunk = -1;
+  a.s0_seg = 0;
+  a.s0_identity = 0;
+  a.write_o = 1;
+  return a;
+}
+
+// Segments per sequence for this problem on the current device (1: none).
+int segments_for(int B, int T, int H, int dk, int dv, int C, gdr_dtype in_dtype,
+                 gdr_gate_kind gate) {
+  if (B <= 0 || T <= 0 || H <= 0 || C != 64) return 1;
+  if (in_dtype != GDR_F32 && in_dtype != GDR_BF16) return 1;
+  if (gate != GDR_GATE_SCALAR && gate != GDR_GATE_PER_CHANNEL) return 1;
+  return gdr::chunk_segments(chunk_shape(B, T, H, dk, dv, in_dtype, gate), device_sms());
+}
+
 // Device address of the status word on the current device (cached per device).
 cudaError_t status_word(unsigned int **out) {
   static unsigned int *cache[64] = {};
@@ -78,8 +120,17 @@ const char *gdr_last_error_message(void) { return t_msg; }
 
 size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int C,
                                      gdr_dtype in_dtype, gdr_gate_kind gate) {
-  (void)B; (void)T; (void)H; (void)dk; (void)dv; (void)C; (void)in_dtype; (void)gate;
-  return 0;  // every chunked-forward kernel keeps its intermediates on chip
+  // Only the segment path of long sequences with few (b, h) needs scratch
+  // (one fp32 state per segment and head, three sets); every kernel keeps its
+  // intermediates on chip.
+  const int P = segments_for(B, T, H, dk, dv, C, in_dtype, gate);
+  return gdr::chunk_segments_ws_bytes(chunk_shape(B, T, H, dk, dv, in_dtype, gate), P);
+}
+
+int gdr_chunk_fwd_kernel_launches(int B, int T, int H, int dk, int dv, int C,
+                                  gdr_dtype in_dtype, gdr_gate_kind gate) {
+  if (B <= 0 || H <= 0 || T < 0) return 0;
+  return segments_for(B, T, H, dk, dv, C, in_dtype, gate) > 1 ? 4 : 1;
 }
 
 gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
@@ -113,17 +164,18 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
     return fail(GDR_ERR_INVALID_ARG, "S0/S_T must be 16-byte aligned");
   if (empty_state) return ok();
 
-  gdr::ChunkArgs a;
+  gdr::ChunkArgs a = chunk_shape(B, T, H, dk, dv, in_dtype, gate);
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.S_T = S_T;
-  a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv;
-  a.bf16 = in_dtype == GDR_BF16;
-  a.per_channel = gate == GDR_GATE_PER_CHANNEL;
   a.skip_stage_chunk = t_skip_stage_chunk;
   t_skip_stage_chunk = -1;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = status_word(&a.status);
   if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd status word");
-  if (gdr::chunk_tc_supports(a))
+  // (an armed load-skip test hook keeps the single-pass kernel)
+  const int P = a.skip_stage_chunk >= 0 ? 1 : segments_for(B, T, H, dk, dv, C, in_dtype, gate);
+  if (P > 1)
+    e = gdr::launch_chunk_segments(a, P, workspace, s);
+  else if (gdr::chunk_tc_supports(a))
     e = gdr::launch_chunk_tc(a, s);
   else
     e = gdr::launch_chunk_simt(a, s);

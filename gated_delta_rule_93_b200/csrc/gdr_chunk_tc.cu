@@ -1165,12 +1165,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
       } else {
         // S_b = bf16(S0); S_tmem = e^{gc_last} S0; sigma = 1 afterwards.
+        // Segment passes: S0 of the first segment of each sequence only
+        // (a.s0_seg segments per sequence, S0 indexed by sequence), or the
+        // identity (the run that yields a segment's transition).
+        const float *s0 = nullptr;
+        if (a.S0 && a.s0_seg == 0) {
+          s0 = a.S0 + ((size_t)bh * DV + i) * DK;
+        } else if (a.S0 && b % a.s0_seg == 0) {
+          s0 = a.S0 + (((size_t)(b / a.s0_seg) * H + h) * DV + i) * DK;
+        }
 #pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           float x[32];
-          if (a.S0) {
-            const float4 *s4 =
-                reinterpret_cast<const float4 *>(a.S0 + ((size_t)bh * DV + i) * DK + 32 * q);
+          if (s0) {
+            const float4 *s4 = reinterpret_cast<const float4 *>(s0 + 32 * q);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float4 v = s4[e];
@@ -1180,8 +1188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               x[4 * e + 3] = v.w;
             }
           } else {
+            const float one = a.s0_identity ? 1.f : 0.f;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = 0.f;
+            for (int e = 0; e < 32; ++e) x[e] = (32 * q + e == i) ? one : 0.f;
           }
           if (PC) {  // S Diag(e^{m_0})
             const float *fv = reinterpret_cast<const float *>(sm + Lay::SVEC) + kSvF + 32 * q;
@@ -1360,7 +1369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_4d(&tmO, sm + Lay::VPD + 4096 * warp, 32 * warp, h, c * C, b);
+          if (a.write_o) tma_store_4d(&tmO, sm + Lay::VPD + 4096 * warp, 32 * warp, h, c * C, b);
           tma_store_commit();
         }
       }
@@ -1460,8 +1469,11 @@ bool chunk_tc_supports(const ChunkArgs &a) {
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
   if (!chunk_tc_supports(a)) return cudaErrorNotSupported;
   CUtensorMap mq, mk, mv, mg, mo;
+  // Without an output (segment passes) the output map is never used; it is
+  // built over q so that it is a valid map.
   if (!make_map(&mq, a.q, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, a.B, a.T, a.H, DK) ||
-      !make_map(&mv, a.v, a.B, a.T, a.H, DV) || !make_map_out(&mo, a.o, a.B, a.T, a.H, DV))
+      !make_map(&mv, a.v, a.B, a.T, a.H, DV) ||
+      !make_map_out(&mo, a.write_o ? a.o : const_cast<void *>(a.q), a.B, a.T, a.H, DV))
     return cudaErrorInvalidValue;
   if (a.per_channel) {
     if (!make_map_gate(&mg, a.g, a.B, a.T, a.H, DK)) return cudaErrorInvalidValue;

@@ -25,6 +25,11 @@ struct ChunkArgs {
   int per_channel;   // 1: g is [B,T,H,dk]
   unsigned int *status;  // device status word
   int skip_stage_chunk;  // testing: chunk whose input load is never issued (-1: none)
+  // Segment passes of a long sequence (tensor-core kernel only; 0 / 0 / 1
+  // for an ordinary call):
+  int s0_seg;       // > 0: sequence b reads S0[b / s0_seg] if b % s0_seg == 0, else starts at 0
+  int s0_identity;  // 1: sequences without an S0 start from the identity (d_v == d_k)
+  int write_o;      // 0: o is not written (may be null)
 };
 
 struct StepArgs {
@@ -46,6 +51,13 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 // the shape is outside what it handles, so the caller can pick another path.
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 bool chunk_tc_supports(const ChunkArgs &a);
+
+// Long sequences with few (b, h): each sequence is cut into P segments that
+// run as separate (b, h) units (two passes of the tensor-core kernel, a
+// combine of the segments' states, a final pass).  P = 1: not used.
+int chunk_segments(const ChunkArgs &a, int num_sms);
+size_t chunk_segments_ws_bytes(const ChunkArgs &a, int P);
+cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStream_t stream);
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float load_in(const void *p, size_t i, int bf16) {

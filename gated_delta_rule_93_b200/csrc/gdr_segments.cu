@@ -1,0 +1,167 @@
+// Long sequences with few (b, h): the sequence is cut into P equal segments
+// that run as separate (b, h) units of the tensor-core chunked forward, so
+// that B * H * P CTAs share the work of B * H.
+//
+// Source: "Decoding Hybrid Linear Attention Architectures", section 5: the
+// state after a stretch of tokens is linear in the state before it,
+//   S_end = S_start M + E,
+// M = the product of the per-token transitions (decay times I - beta k k^T)
+// over the stretch, E = the state the stretch writes from a zero start.  The
+// section applies this per chunk; here it is applied per segment:
+//   pass 1a: every segment from zero (the first from S0): E_p, and for the
+//            first segment its true end state;
+//   pass 1b: every segment from the identity: end state M_p + E_p (d_v = d_k);
+//   combine: S_start(1) = end of segment 0, S_start(p + 1) = S_start(p) M_p +
+//            E_p, in fp32; the last product is the final state S_T;
+//   pass 2:  every segment from its true start state: the output o.
+// The passes reuse the kernel on the same tensors: [B, T, H, d] is
+// [B * P, T / P, H, d] with segment p of sequence b as sequence b * P + p.
+#include "gdr_internal.cuh"
+
+namespace gdr {
+namespace {
+
+constexpr int kDim = 128;                   // d_k = d_v of the tensor-core kernel
+constexpr int kRows = 16;                   // state rows per combine CTA
+constexpr int kRowBlocks = kDim / kRows;
+constexpr int kCombineThreads = 256;        // 16 rows x 16 column groups of 8
+constexpr size_t kCombineSmem = (size_t)(kDim * kDim + kRows * kDim) * sizeof(float);
+
+// One CTA per (b, h) and block of 16 state rows (rows of S are independent
+// under S <- S M + E).  E_a: end states of pass 1a, E_b: of pass 1b, X: the
+// start state of every segment (written), S_T: the final state (optional),
+// all [B * P, H, 128, 128] except S0 / S_T [B, H, 128, 128].
+__global__ void __launch_bounds__(kCombineThreads)
+    combine_segments(const float *__restrict__ S0, const float *__restrict__ Ea,
+                     const float *__restrict__ Eb, float *__restrict__ X, float *S_T, int H,
+                     int P) {
+  extern __shared__ float smem[];
+  float *M = smem;                // [128][128] transition of the current segment
+  float *R = smem + kDim * kDim;  // [16][128] rows of the running start state
+  const int bh = blockIdx.x, b = bh / H, h = bh % H, r0 = blockIdx.y * kRows;
+  const int t = threadIdx.x;
+  const size_t st = (size_t)kDim * kDim;
+  auto seg = [&](int p) { return ((size_t)(b * P + p) * H + h) * st; };
+
+  // segment 0 starts from S0 (or 0); segment 1 from segment 0's end state
+  for (int i = t; i < kRows * kDim; i += kCombineThreads) {
+    const size_t off = (size_t)r0 * kDim + i;
+    X[seg(0) + off] = S0 ? S0[(size_t)bh * st + off] : 0.f;
+    const float e0 = Ea[seg(0) + off];
+    R[i] = e0;
+    X[seg(1) + off] = e0;
+  }
+  const int r = t / 16, c0 = (t % 16) * 8;
+  for (int p = 1; p < P; ++p) {
+    __syncthreads();  // R written, M free
+    const float4 *ea4 = reinterpret_cast<const float4 *>(Ea + seg(p));
+    const float4 *eb4 = reinterpret_cast<const float4 *>(Eb + seg(p));
+    float4 *m4 = reinterpret_cast<float4 *>(M);
+    for (int i = t; i < kDim * kDim / 4; i += kCombineThreads) {
+      const float4 x = eb4[i], y = ea4[i];
+      m4[i] = make_float4(x.x - y.x, x.y - y.y, x.z - y.z, x.w - y.w);
+    }
+    __syncthreads();
+    float acc[8];
+    const float *er = Ea + seg(p) + (size_t)(r0 + r) * kDim + c0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = er[j];
+#pragma unroll 4
+    for (int k = 0; k < kDim; ++k) {
+      const float s = R[r * kDim + k];
+      const float4 ma = *reinterpret_cast<const float4 *>(M + k * kDim + c0);
+      const float4 mb = *reinterpret_cast<const float4 *>(M + k * kDim + c0 + 4);
+      acc[0] = fmaf(s, ma.x, acc[0]);
+      acc[1] = fmaf(s, ma.y, acc[1]);
+      acc[2] = fmaf(s, ma.z, acc[2]);
+      acc[3] = fmaf(s, ma.w, acc[3]);
+      acc[4] = fmaf(s, mb.x, acc[4]);
+      acc[5] = fmaf(s, mb.y, acc[5]);
+      acc[6] = fmaf(s, mb.z, acc[6]);
+      acc[7] = fmaf(s, mb.w, acc[7]);
+    }
+    __syncthreads();  // every thread has read R
+    float *dst = nullptr;
+    if (p + 1 < P)
+      dst = X + seg(p + 1);
+    else if (S_T)
+      dst = S_T + (size_t)bh * st;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) R[r * kDim + c0 + j] = acc[j];
+    if (dst) {
+      float4 *d4 = reinterpret_cast<float4 *>(dst + (size_t)(r0 + r) * kDim + c0);
+      d4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      d4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    }
+  }
+}
+
+}  // namespace
+
+int chunk_segments(const ChunkArgs &a, int num_sms) {
+  if (!chunk_tc_supports(a) || a.dk != kDim || a.dv != kDim || a.skip_stage_chunk >= 0)
+    return 1;
+  const long long bh = (long long)a.B * a.H;
+  if (bh <= 0 || num_sms <= 0) return 1;
+  // Largest power of two P with B * H * P CTAs in one wave, segments of whole
+  // chunks, at least 16 chunks each; three passes pay off only from P = 4.
+  int P = 1;
+  while (P < 64 && bh * 2 * P <= num_sms && a.T % (64 * 2 * P) == 0 &&
+         a.T / (64 * 2 * P) >= 16)
+    P *= 2;
+  return P >= 4 ? P : 1;
+}
+
+size_t chunk_segments_ws_bytes(const ChunkArgs &a, int P) {
+  if (P <= 1) return 0;
+  // X, E_a, E_b: one fp32 state per segment and head each
+  return 3 * (size_t)a.B * P * a.H * a.dv * a.dk * sizeof(float);
+}
+
+cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStream_t stream) {
+  static bool smem_set[64] = {};  // per device
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!smem_set[dev]) {
+    e0 = cudaFuncSetAttribute(combine_segments, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kCombineSmem);
+    if (e0 != cudaSuccess) return e0;
+    smem_set[dev] = true;
+  }
+  const size_t n_state = (size_t)a.B * P * a.H * a.dv * a.dk;
+  float *X = static_cast<float *>(ws), *Ea = X + n_state, *Eb = Ea + n_state;
+  ChunkArgs s = a;
+  s.B = a.B * P;
+  s.T = a.T / P;
+  // pass 1a: zero start (the first segment of a sequence from S0), end states
+  s.S0 = a.S0;
+  s.s0_seg = P;
+  s.s0_identity = 0;
+  s.S_T = Ea;
+  s.o = nullptr;
+  s.write_o = 0;
+  cudaError_t e = launch_chunk_tc(s, stream);
+  if (e != cudaSuccess) return e;
+  // pass 1b: identity start, end states = transition + the same writes
+  s.S0 = nullptr;
+  s.s0_seg = 0;
+  s.s0_identity = 1;
+  s.S_T = Eb;
+  e = launch_chunk_tc(s, stream);
+  if (e != cudaSuccess) return e;
+  combine_segments<<<dim3(a.B * a.H, kRowBlocks), kCombineThreads, kCombineSmem, stream>>>(
+      a.S0, Ea, Eb, X, a.S_T, a.H, P);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // pass 2: every segment from its true start state; the output
+  s.S0 = X;
+  s.s0_identity = 0;
+  s.S_T = nullptr;
+  s.o = a.o;
+  s.write_o = 1;
+  return launch_chunk_tc(s, stream);
+}
+
+}  // namespace gdr

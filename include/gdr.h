@@ -65,11 +65,26 @@ typedef enum { GDR_GATE_SCALAR = 0, GDR_GATE_PER_CHANNEL = 1 } gdr_gate_kind;
 typedef struct CUstream_st *gdr_stream_t;
 
 /*
- * Workspace the chunked forward needs for this problem, in bytes (0 if none).
- * Pass at least this much (16-byte aligned) to gdr_chunk_fwd.
+ * Workspace the chunked forward needs for this problem on the current
+ * device, in bytes (0 if none).  Pass at least this much (16-byte aligned,
+ * device memory owned by the caller) to gdr_chunk_fwd.  Only long sequences
+ * with few (b, h) use it: with B*H*P <= the device's SM count for a power of
+ * two P >= 4 and T a multiple of 64*P with at least 16 chunks per segment,
+ * each sequence runs as P segments (section 5 of "Decoding Hybrid Linear
+ * Attention Architectures": a stretch's end state is its start state times
+ * the stretch's transition plus what the stretch writes), which needs
+ * 3 * B*P*H * dv*dk fp32 values of scratch.
  */
 size_t gdr_chunk_fwd_workspace_bytes(int B, int T, int H, int dk, int dv, int C,
                                      gdr_dtype in_dtype, gdr_gate_kind gate);
+
+/*
+ * Number of kernels one gdr_chunk_fwd call with these arguments launches on
+ * the current device (4 on the segment path, 1 otherwise, 0 if B*H == 0),
+ * for sizing CUDA graphs and counting launches.
+ */
+int gdr_chunk_fwd_kernel_launches(int B, int T, int H, int dk, int dv, int C,
+                                  gdr_dtype in_dtype, gdr_gate_kind gate);
 
 /*
  * Chunkwise-parallel forward over whole sequences (prefill / training

@@ -50,6 +50,10 @@ def test_status_strings(L):
 
 def test_workspace_query(L):
     assert L.gdr_chunk_fwd_workspace_bytes(8, 4096, 16, 128, 128, 64, 1, 0) == 0
+    # the segment path depends on the device's SM count: none without a GPU
+    assert L.gdr_chunk_fwd_workspace_bytes(1, 65536, 16, 128, 128, 64, 1, 0) == 0
+    assert L.gdr_chunk_fwd_kernel_launches(8, 4096, 16, 128, 128, 64, 1, 0) == 1
+    assert L.gdr_chunk_fwd_kernel_launches(0, 4096, 16, 128, 128, 64, 1, 0) == 0
 
 
 def _fake_ptr(off=0):

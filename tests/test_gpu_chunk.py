@@ -149,3 +149,51 @@ def test_misaligned_pointer_is_rejected(cuda_device):
     with pytest.raises(binding.GdrError, match="aligned"):
         binding.chunk_fwd(q_bad, d["k"], d["v"], d["g"], d["beta"])
     assert binding.device_status() == 0
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("with_S0", [True, False])
+def test_segment_path_matches_oracle(cuda_device, gate, with_S0):
+    """A long sequence with few heads runs as segments (two passes, a combine
+    of the segments' states, a final pass): B1 H2 T4096 d128 is 4 segments of
+    16 chunks on a B200."""
+    B, T, H, d = 1, 4096, 2, 128
+    assert binding.chunk_fwd_kernel_launches(B, T, H, d, d, gate=gate) == 4
+    assert binding.chunk_fwd_workspace_bytes(B, T, H, d, d, gate=gate) == 3 * B * 4 * H * d * d * 4
+    inp = make_chunk_inputs(B, T, H, d, d, torch.bfloat16, gate, with_S0, seed=11)
+    o, S_T = gpu_chunk(inp, cuda_device)
+    assert binding.device_status() == 0
+    ro, rS = oracle_chunk(inp)
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S_T, rS, 2e-2, "S_T")
+
+
+def test_segment_path_initial_state_may_alias_final_state(cuda_device):
+    inp = make_chunk_inputs(1, 4096, 2, 128, 128, torch.bfloat16, "scalar", True, seed=12)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    S = d["S0"].clone()
+    o, S_T = binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S, S_T=S)
+    torch.cuda.synchronize()
+    ro, rS = oracle_chunk(inp)
+    assert S_T.data_ptr() == S.data_ptr()
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S, rS, 2e-2, "S_T (aliased)")
+
+
+def test_segment_path_rejects_short_workspace(cuda_device):
+    inp = make_chunk_inputs(1, 4096, 2, 128, 128, torch.bfloat16, "scalar", False, seed=13)
+    d = {k: (v.to(cuda_device) if v is not None else None) for k, v in inp.items()}
+    small = torch.empty(16, dtype=torch.uint8, device=cuda_device)
+    with pytest.raises(binding.GdrError) as ei:
+        binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, workspace=small)
+    assert ei.value.status == binding.GDR_ERR_WORKSPACE
+
+
+def test_segment_rule_leaves_wide_batches_alone(cuda_device):
+    """B*H large enough to fill the SMs, short sequences, fp32 inputs or other
+    head sizes: one launch, no workspace."""
+    for args, kw in [((8, 4096, 16, 128, 128), {}), ((1, 512, 2, 128, 128), {}),
+                     ((1, 65536, 16, 128, 128), {"dtype": torch.float32}),
+                     ((1, 65536, 2, 64, 64), {})]:
+        assert binding.chunk_fwd_kernel_launches(*args, **kw) == 1, args
+        assert binding.chunk_fwd_workspace_bytes(*args, **kw) == 0, args
