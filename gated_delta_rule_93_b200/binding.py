@@ -28,6 +28,7 @@ EXPORTS = (
     "gdr_chunk_fwd_workspace_bytes",
     "gdr_chunk_fwd_kernel_launches",
     "gdr_chunk_fwd",
+    "gdr_chunk_fwd_segmented",
     "gdr_step",
     "gdr_get_device_status",
     "gdr_status_string",
@@ -61,6 +62,9 @@ def lib():
             L.gdr_chunk_fwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, i, i, i, i, i, i,
                                         vp, sz, vp]
             L.gdr_chunk_fwd.restype = i
+            L.gdr_chunk_fwd_segmented.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, i, i, i, i,
+                                                  i, i, i, vp, sz, vp]
+            L.gdr_chunk_fwd_segmented.restype = i
             L.gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp]
             L.gdr_step.restype = i
             L.gdr_get_device_status.argtypes = [vp]
@@ -211,3 +215,42 @@ def testing_skip_stage_load(chunk):
 def device_status(stream=None):
     """Synchronise and read/clear the library's device status word (0 = OK)."""
     return int(lib().gdr_get_device_status(_stream_handle(stream)))
+
+
+def chunk_fwd_segmented(q, k, v, g, beta, S0=None, *, segments, workspace,
+                        output_final_state=True, o=None, S_T=None, C=64, stream=None):
+    """``gdr_chunk_fwd_segmented``: the chunked forward as ``segments`` segments
+    per sequence in the caller's ``workspace`` (a uint8 CUDA tensor of at least
+    3*B*segments*H*dv*dk*4 bytes).  Returns (o, S_T or None)."""
+    _need(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (B, T, H, dk), dev)
+    _need(v, "v", dt, (B, T, H, dv), dev)
+    if g.dim() == 4:
+        _need(g, "g", torch.float32, (B, T, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (B, T, H), dev)
+        gk = GDR_GATE_SCALAR
+    _need(beta, "beta", torch.float32, (B, T, H), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    if not isinstance(workspace, torch.Tensor) or workspace.device != dev:
+        raise ValueError("workspace must be a tensor on the inputs' device")
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _need(o, "o", dt, (B, T, H, dv), dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_chunk_fwd_segmented(
+            _ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk, _ptr(beta), _ptr(S0),
+            _ptr(o), _ptr(S_T), B, T, H, dk, dv, C, int(segments), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc)
+    return o, S_T

@@ -133,11 +133,16 @@ int gdr_chunk_fwd_kernel_launches(int B, int T, int H, int dk, int dv, int C,
   return segments_for(B, T, H, dk, dv, C, in_dtype, gate) > 1 ? 4 : 1;
 }
 
-gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
-                         const float *g, gdr_gate_kind gate, const float *beta,
-                         const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
-                         int dv, int C, void *workspace, size_t ws_bytes,
-                         gdr_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the chunked-forward entry points (everything but the
+// workspace); fills the kernel arguments.  Returns GDR_OK or the error.
+gdr_status check_chunk(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                       const float *g, gdr_gate_kind gate, const float *beta, const float *S0,
+                       void *o, float *S_T, int B, int T, int H, int dk, int dv, int C,
+                       gdr::ChunkArgs *out) {
   if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "negative B/T/H");
   if (in_dtype != GDR_F32 && in_dtype != GDR_BF16)
     return fail(GDR_ERR_INVALID_ARG, "in_dtype must be GDR_F32 or GDR_BF16");
@@ -146,13 +151,9 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
   if (C != 64) return fail(GDR_ERR_UNSUPPORTED, "chunk size C=%d (only 64 is built)", C);
   if (!head_dim_ok(dk) || !head_dim_ok(dv))
     return fail(GDR_ERR_UNSUPPORTED, "head dims dk=%d dv=%d (need 32, 64 or 128)", dk, dv);
-  const size_t need_ws = gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, in_dtype, gate);
-  if (ws_bytes < need_ws || (need_ws && !workspace))
-    return fail(GDR_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need_ws);
   if ((size_t)B * (size_t)H * (size_t)T > (size_t)1 << 40)
     return fail(GDR_ERR_INVALID_ARG, "problem too large");
   const bool empty_tokens = (size_t)B * H * T == 0;
-  const bool empty_state = (size_t)B * H == 0;
   if (!empty_tokens) {
     if (!q || !k || !v || !g || !beta || !o)
       return fail(GDR_ERR_INVALID_ARG, "null q/k/v/g/beta/o");
@@ -162,10 +163,31 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
   }
   if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
     return fail(GDR_ERR_INVALID_ARG, "S0/S_T must be 16-byte aligned");
-  if (empty_state) return ok();
-
   gdr::ChunkArgs a = chunk_shape(B, T, H, dk, dv, in_dtype, gate);
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.S0 = S0; a.o = o; a.S_T = S_T;
+  *out = a;
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                         const float *g, gdr_gate_kind gate, const float *beta,
+                         const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
+                         int dv, int C, void *workspace, size_t ws_bytes,
+                         gdr_stream_t stream) {
+  gdr::ChunkArgs a;
+  gdr_status st = check_chunk(q, k, v, in_dtype, g, gate, beta, S0, o, S_T, B, T, H, dk, dv, C,
+                              &a);
+  if (st != GDR_OK) return st;
+  const size_t need_ws = gdr_chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, in_dtype, gate);
+  if (ws_bytes < need_ws || (need_ws && !workspace))
+    return fail(GDR_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need_ws);
+  if (need_ws && !aligned16(workspace))
+    return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((size_t)B * H == 0) return ok();
   a.skip_stage_chunk = t_skip_stage_chunk;
   t_skip_stage_chunk = -1;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -180,6 +202,33 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
   else
     e = gdr::launch_chunk_simt(a, s);
   return from_cuda(e, "gdr_chunk_fwd launch");
+}
+
+gdr_status gdr_chunk_fwd_segmented(const void *q, const void *k, const void *v,
+                                   gdr_dtype in_dtype, const float *g, gdr_gate_kind gate,
+                                   const float *beta, const float *S0, void *o, float *S_T,
+                                   int B, int T, int H, int dk, int dv, int C, int P,
+                                   void *workspace, size_t ws_bytes, gdr_stream_t stream) {
+  gdr::ChunkArgs a;
+  gdr_status st = check_chunk(q, k, v, in_dtype, g, gate, beta, S0, o, S_T, B, T, H, dk, dv, C,
+                              &a);
+  if (st != GDR_OK) return st;
+  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128)
+    return fail(GDR_ERR_UNSUPPORTED, "segments need bf16 inputs and dk = dv = 128");
+  if (P < 2 || T <= 0 || T % (64 * P) != 0)
+    return fail(GDR_ERR_UNSUPPORTED, "P=%d segments of whole 64-token chunks (T=%d)", P, T);
+  if ((size_t)B * P * H > (size_t)1 << 31) return fail(GDR_ERR_INVALID_ARG, "B*P*H too large");
+  const size_t need_ws = gdr::chunk_segments_ws_bytes(a, P);
+  if (ws_bytes < need_ws || !workspace)
+    return fail(GDR_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need_ws);
+  if (!aligned16(workspace)) return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((size_t)B * H == 0) return ok();
+  a.skip_stage_chunk = -1;
+  cudaError_t e = status_word(&a.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd_segmented status word");
+  return from_cuda(gdr::launch_chunk_segments(a, P, workspace,
+                                              reinterpret_cast<cudaStream_t>(stream)),
+                   "gdr_chunk_fwd_segmented launch");
 }
 
 gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dtype,

@@ -116,6 +116,33 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
                          gdr_stream_t stream);
 
 /*
+ * The chunked forward as P segments per sequence, with P chosen by the
+ * caller, allocating nothing: every intermediate lives in the caller's
+ * workspace.  Source: "Decoding Hybrid Linear Attention Architectures",
+ * section 5, whose inter-chunk recursion (end state = start state times the
+ * chunk's transition plus what the chunk writes) is applied per segment:
+ * every segment runs from a zero state (the first from S0) and from the
+ * identity, the segments' start states follow in fp32
+ * (S_start(p+1) = S_start(p) M_p + E_p, M_p = the identity run's end state
+ * minus the zero run's), and a last pass writes o.  gdr_chunk_fwd takes
+ * this path by itself for long sequences with few heads; this entry point
+ * fixes P (for example to capture a fixed shape in a CUDA graph).
+ *
+ * Arguments as gdr_chunk_fwd, plus
+ *   P          segments per sequence, >= 2, T a multiple of 64*P
+ *   workspace  device memory of at least 3*B*P*H*dv*dk*4 bytes, 16-byte
+ *              aligned, owned by the caller (overwritten)
+ * Needs bf16 inputs and dk = dv = 128 (GDR_ERR_UNSUPPORTED otherwise, also
+ * for a P that does not split T into whole chunks); GDR_ERR_WORKSPACE if
+ * the workspace is missing or too small.  Launches 4 kernels on `stream`.
+ */
+gdr_status gdr_chunk_fwd_segmented(const void *q, const void *k, const void *v,
+                                   gdr_dtype in_dtype, const float *g, gdr_gate_kind gate,
+                                   const float *beta, const float *S0, void *o, float *S_T,
+                                   int B, int T, int H, int dk, int dv, int C, int P,
+                                   void *workspace, size_t ws_bytes, gdr_stream_t stream);
+
+/*
  * One recurrent decode step for N independent states, S updated in place.
  * Source: "Decoding Hybrid Linear Attention Architectures", section 6
  * (constant-cost update of the fixed-size state per decoded token) with the

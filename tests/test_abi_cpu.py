@@ -100,6 +100,32 @@ def test_validation_rejects_before_any_launch(L):
     assert step(N=0) == binding.GDR_OK
 
 
+def test_segmented_validation_rejects_before_any_launch(L):
+    """gdr_chunk_fwd_segmented: caller-chosen segments, caller's workspace."""
+    p = _fake_ptr()
+    need = 3 * 2 * 4 * 3 * 128 * 128 * 4  # B=2, P=4, H=3
+
+    def call(**kw):
+        a = dict(q=p, k=p, v=p, dt=1, g=p, gate=0, beta=p, S0=None, o=p, ST=None, B=2, T=1024,
+                 H=3, dk=128, dv=128, C=64, P=4, ws=p, wsb=need, st=None)
+        a.update(kw)
+        return L.gdr_chunk_fwd_segmented(a["q"], a["k"], a["v"], a["dt"], a["g"], a["gate"],
+                                         a["beta"], a["S0"], a["o"], a["ST"], a["B"], a["T"],
+                                         a["H"], a["dk"], a["dv"], a["C"], a["P"], a["ws"],
+                                         a["wsb"], a["st"])
+
+    assert call(P=1) == binding.GDR_ERR_UNSUPPORTED
+    assert call(P=3) == binding.GDR_ERR_UNSUPPORTED      # 1024 is not 3 x whole chunks
+    assert call(T=1000) == binding.GDR_ERR_UNSUPPORTED   # ragged segments
+    assert call(dt=0) == binding.GDR_ERR_UNSUPPORTED     # fp32 inputs: single pass only
+    assert call(dk=64, dv=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(wsb=need - 1) == binding.GDR_ERR_WORKSPACE
+    assert call(ws=None) == binding.GDR_ERR_WORKSPACE
+    assert call(ws=_fake_ptr(8)) == binding.GDR_ERR_INVALID_ARG
+    assert call(q=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(B=0) == binding.GDR_OK
+
+
 def test_binding_refuses_cpu_tensors(L):
     import torch
 

@@ -197,3 +197,31 @@ def test_segment_rule_leaves_wide_batches_alone(cuda_device):
                      ((1, 65536, 2, 64, 64), {})]:
         assert binding.chunk_fwd_kernel_launches(*args, **kw) == 1, args
         assert binding.chunk_fwd_workspace_bytes(*args, **kw) == 0, args
+
+
+@pytest.mark.parametrize("gate,P", [("scalar", 2), ("scalar", 8), ("channel", 4),
+                                    ("scalar", 3)])
+def test_segmented_entry_point_matches_oracle(cuda_device, gate, P):
+    """gdr_chunk_fwd_segmented with the caller's P and workspace (nothing is
+    allocated by the call): B2 H2 T1536 (24 chunks) with S0."""
+    B, T, H, d = 2, 1536, 2, 128
+    inp = make_chunk_inputs(B, T, H, d, d, torch.bfloat16, gate, True, seed=20 + P)
+    dd = {k: v.to(cuda_device) for k, v in inp.items()}
+    ws = torch.empty(3 * B * P * H * d * d * 4, dtype=torch.uint8, device=cuda_device)
+    o, S_T = binding.chunk_fwd_segmented(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
+                                         dd["S0"], segments=P, workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    ro, rS = oracle_chunk(inp)
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S_T, rS, 2e-2, "S_T")
+
+
+def test_segmented_entry_point_rejects_short_workspace(cuda_device):
+    inp = make_chunk_inputs(1, 1024, 2, 128, 128, torch.bfloat16, "scalar", False, seed=30)
+    dd = {k: (v.to(cuda_device) if v is not None else None) for k, v in inp.items()}
+    ws = torch.empty(3 * 4 * 2 * 128 * 128 * 4 - 16, dtype=torch.uint8, device=cuda_device)
+    with pytest.raises(binding.GdrError) as ei:
+        binding.chunk_fwd_segmented(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], None,
+                                    segments=4, workspace=ws)
+    assert ei.value.status == binding.GDR_ERR_WORKSPACE
