@@ -91,8 +91,10 @@ constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256, kSvF = 384;
 // Per-variant configuration: K/Q stages and the shared-memory layout (byte
 // offsets from a 1024-byte aligned base).  PC (per-channel gates) holds, per
 // stage, the scaled K~, Q~ tiles in place of K, Q and K^ in its own tiles,
-// the fp32 gate tile of the chunk being scaled, and shares T with T' and
-// V'^T with its decayed copy (both identical without a scalar decay).
+// each scaling warp's fp32 gate rows (its 64 channels, rows 0-31 and 32-63
+// of the chunk being scaled, each half refilled with the next chunk's as
+// soon as it has been read), and shares T with T' and V'^T with its decayed
+// copy (both identical without a scalar decay).
 template <bool PC>
 struct Cfg {
   static constexpr int kStages = PC ? 2 : 3;
@@ -100,7 +102,7 @@ struct Cfg {
   static constexpr uint32_t kSvecBytes = (PC ? 512 : 128) * 4;
   static constexpr uint32_t KQ = 0;                                          // [K_h0|Q_h0|K_h1|Q_h1]
   static constexpr uint32_t KH = KQ + kStages * 4 * kTileBytes;              // PC: [Kh_h0|Kh_h1]
-  static constexpr uint32_t GT = KH + (PC ? kStages * 2 * kTileBytes : 0);   // PC: g [64][128]
+  static constexpr uint32_t GT = KH + (PC ? kStages * 2 * kTileBytes : 0);   // PC: g [2][2][32][64]
   static constexpr uint32_t V = GT + (PC ? 64 * 128 * 4 : 0);                // [V_h0|V_h1]
   static constexpr uint32_t T = V + 2 * kTileBytes;                          // T  K-major [r][s]
   static constexpr uint32_t TP = T + (PC ? 0 : kTileBytes);                  // T' K-major, x2
@@ -144,7 +146,9 @@ enum {
   B_FIN = B_TPE + 2,   // final drain, state-side issuer                (commit)
   B_FIN2,              // final drain, prep-side issuer                 (commit)
   B_SCALED,            // [2] PC: scaled K~, Q~, K^ of a stage written  (2 warps)
-  B_COUNT = B_SCALED + 2
+  B_GF = B_SCALED + 2, // [4] PC: gate rows of a scaling warp landed    (1 + tx)
+                       //     (warp w, rows 0-31 / 32-63: 2 w + half)
+  B_COUNT = B_GF + 4
 };
 static_assert(B_COUNT <= 32, "barrier slots");
 
@@ -582,49 +586,81 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Per-channel gates, one warp, channels j0 .. j0 + 63 (lane l: the adjacent
-// pair j0 + 2 l, j0 + 2 l + 1): cumulative log decay gc over the chunk (kept
-// in place in the fp32 gate tile gt [64][128], in log2 units), the
-// reference m = gc at row 31, e^{m} and e^{gc_last - m} into the stage's gate
-// vectors, and the operand tiles scaled in place:
+// Per-channel gates, one warp, channels j0 .. j0 + 63 of a chunk (lane l:
+// the adjacent pair j0 + 2 l, j0 + 2 l + 1).  g0 / g1: the warp's gate rows
+// 0-31 / 32-63 of the chunk ([32][64] fp32 log decay, zero past T), landed
+// on gf[0] / gf[1] (phase parity ph).  The cumulative log decay gc (log2
+// units) of rows 0-31 is formed in place; the reference m = gc at row 31,
+// e^{m} and e^{gc_last - m} go into the stage's gate vectors, and the
+// operand tiles are scaled in place:
 //   K~ = K e^{gc - m},  Q~ = Q e^{gc - m},  K^ = K e^{m - gc}  (bf16),
 // so that K~ K^T, Q~ K^T carry e^{gc_r - gc_s} per channel, and with the
 // state kept as S Diag(e^{m}), Z and O_a carry e^{gc} (decay from the chunk
 // start) and the update V'^T K^ carries e^{m - gc}.  The factors stay within
-// e^{|gc_last| / 2}.
-__device__ void scale_channels(uint8_t *kq, uint8_t *kh, float *gt, float *gv, int j0,
-                               int lane) {
+// e^{|gc_last| / 2}.  Each half is refilled with rows of the chunk at token
+// t0n (none if t0n < 0) as soon as the warp has read it, so the load runs
+// under the other half's work.  Returns 2 when done, 1 if the wait for rows
+// 32-63 gave up (rows 0-31 already refilled), 0 if the first wait gave up.
+__device__ __forceinline__ void scale_row(uint8_t *kt, uint8_t *qt, uint8_t *ht, int t, int jc,
+                                          float dx, float dy) {
+  const float ux = ex2(dx), uy = ex2(dy), vx = ex2(-dx), vy = ex2(-dy);
+  const uint32_t off = sw128_off(t, jc);
+  uint32_t *kp = reinterpret_cast<uint32_t *>(kt + off);
+  uint32_t *qp = reinterpret_cast<uint32_t *>(qt + off);
+  const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(kp));
+  const float2 qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(qp));
+  *kp = pack_bf16(kv.x * ux, kv.y * uy);
+  *qp = pack_bf16(qv.x * ux, qv.y * uy);
+  *reinterpret_cast<uint32_t *>(ht + off) = pack_bf16(kv.x * vx, kv.y * vy);
+}
+
+__device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, uint64_t *gf,
+                              uint32_t ph, const CUtensorMap *tmG, int h, int b, int t0n,
+                              float *gv, int j0, int lane, volatile int *abort_flag) {
   constexpr float kLog2e = 1.4426950408889634f;
-  const int j = j0 + 2 * lane, hh = j >> 6, jc = j & 63;
+  const int jl = 2 * lane, j = j0 + jl, hh = j >> 6, jc = j & 63;
+  uint8_t *kt = kq + (2 * hh) * kTileBytes, *qt = kt + kTileBytes, *ht = kh + hh * kTileBytes;
+  if (!warp_wait(&gf[0], ph, abort_flag, lane)) return 0;
   float2 acc = make_float2(0.f, 0.f);
 #pragma unroll 8
-  for (int t = 0; t < 64; ++t) {
-    float2 *p = reinterpret_cast<float2 *>(gt + t * 128 + j);
+  for (int t = 0; t < 32; ++t) {
+    float2 *p = reinterpret_cast<float2 *>(g0 + t * 64 + jl);
     const float2 x = *p;
     acc.x += x.x * kLog2e;
     acc.y += x.y * kLog2e;
     *p = acc;
   }
-  const float2 m = *reinterpret_cast<const float2 *>(gt + 31 * 128 + j);
+  const float2 m = acc;
   gv[kGateEm + j] = ex2(m.x);
   gv[kGateEm + j + 1] = ex2(m.y);
+#pragma unroll 4
+  for (int t = 0; t < 32; ++t) {
+    const float2 gl = *reinterpret_cast<const float2 *>(g0 + t * 64 + jl);
+    scale_row(kt, qt, ht, t, jc, gl.x - m.x, gl.y - m.y);
+  }
+  // rows 0-31 read (and written, by the generic proxy): refill
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && t0n >= 0) {
+    mbar_arrive_expect_tx(&gf[0], 32 * 64 * 4);
+    tma_load_4d(g0, tmG, &gf[0], j0, h, t0n, b);
+  }
+  if (!warp_wait(&gf[1], ph, abort_flag, lane)) return 1;
+#pragma unroll 4
+  for (int t = 32; t < 64; ++t) {
+    const float2 x = *reinterpret_cast<const float2 *>(g1 + (t - 32) * 64 + jl);
+    acc.x += x.x * kLog2e;
+    acc.y += x.y * kLog2e;
+    scale_row(kt, qt, ht, t, jc, acc.x - m.x, acc.y - m.y);
+  }
+  __syncwarp();
+  if (lane == 0 && t0n >= 0) {
+    mbar_arrive_expect_tx(&gf[1], 32 * 64 * 4);
+    tma_load_4d(g1, tmG, &gf[1], j0, h, t0n + 32, b);
+  }
   gv[kGateEgm + j] = ex2(acc.x - m.x);
   gv[kGateEgm + j + 1] = ex2(acc.y - m.y);
-  uint8_t *kt = kq + (2 * hh) * kTileBytes, *qt = kt + kTileBytes, *ht = kh + hh * kTileBytes;
-#pragma unroll 4
-  for (int t = 0; t < 64; ++t) {
-    const float2 gl = *reinterpret_cast<const float2 *>(gt + t * 128 + j);
-    const float dx = gl.x - m.x, dy = gl.y - m.y;
-    const float ux = ex2(dx), uy = ex2(dy), vx = ex2(-dx), vy = ex2(-dy);
-    const uint32_t off = sw128_off(t, jc);
-    uint32_t *kp = reinterpret_cast<uint32_t *>(kt + off);
-    uint32_t *qp = reinterpret_cast<uint32_t *>(qt + off);
-    const float2 kv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(kp));
-    const float2 qv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(qp));
-    *kp = pack_bf16(kv.x * ux, kv.y * uy);
-    *qp = pack_bf16(qv.x * ux, qv.y * uy);
-    *reinterpret_cast<uint32_t *>(ht + off) = pack_bf16(kv.x * vx, kv.y * vy);
-  }
+  return 2;
 }
 
 // Each SM sub-partition holds a quarter of the register file and three of
@@ -678,6 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[B_FIN], 1);
     mbar_init(&bars[B_FIN2], 1);
     for (int s = 0; s < 2; ++s) mbar_init(&bars[B_SCALED + s], 2);
+    for (int s = 0; s < 4; ++s) mbar_init(&bars[B_GF + s], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -710,6 +747,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmK);
     }
     int last_issued[3] = {-1, -1, -1};  // latest chunk loaded into each stage
+    int gate_req[2] = {0, 0};              // PC: latest chunk of gate rows requested, per half
+    if (PC && lane == 0) {  // this warp's gate rows of chunk 0
+      float *gt = reinterpret_cast<float *>(sm + Lay::GT);
+      mbar_arrive_expect_tx(&bars[B_GF + 0], 32 * 64 * 4);
+      tma_load_4d(gt, &tmG, &bars[B_GF + 0], 0, h, 0, b);
+      mbar_arrive_expect_tx(&bars[B_GF + 1], 32 * 64 * 4);
+      tma_load_4d(gt + 32 * 64, &tmG, &bars[B_GF + 1], 0, h, 32, b);
+    }
     // Scalar gates: the state group's scale sequence, replayed with the same
     // fp32 operations: sig = the scale of S_b for the chunk being produced.
     float sig = 1.f;
@@ -718,18 +763,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (c >= kStages &&
           !wait_or_abort(&bars[B_EMPTY + s], ((c / kStages) - 1) & 1, abort_flag))
         break;
-      // PC: the gate tile is single-buffered; both scaling warps must be done
-      // with the previous chunk's (its barrier is per stage parity, so it
-      // cannot be two phases ahead of this wait).
-      if (PC && c >= 1 &&
-          !wait_or_abort(&bars[B_SCALED + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag))
-        break;
       // Testing hook: this chunk's load is never issued, so its consumers'
       // bounded waits run out and the kernel unwinds (no trap, no hang).
       if (c == a.skip_stage_chunk) continue;
       const int t0 = c * C;
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
-      if (PC) {  // beta only; the gate tile comes with the K/Q loads
+      if (PC) {  // beta only; each scaling warp loads its own gate rows
         const size_t tok = ((size_t)b * T + t0 + lane) * H + h;
         gv[kGateBeta + lane] = t0 + lane < T ? a.beta[tok] : 0.f;
         gv[kGateBeta + lane + 32] = t0 + lane + 32 < T ? a.beta[tok + (size_t)32 * H] : 0.f;
@@ -771,19 +810,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         uint64_t *fb = &bars[B_FULL + s];
-        mbar_arrive_expect_tx(fb, kKQTx + (PC ? 64 * 128 * 4 : 0));
+        mbar_arrive_expect_tx(fb, kKQTx);
         uint8_t *kq = sm + Lay::KQ + s * 4 * kTileBytes;
         tma_load_4d(kq + 0 * kTileBytes, &tmK, fb, 0, h, t0, b);
         tma_load_4d(kq + 1 * kTileBytes, &tmQ, fb, 0, h, t0, b);
         tma_load_4d(kq + 2 * kTileBytes, &tmK, fb, 64, h, t0, b);
         tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, t0, b);
-        if (PC) tma_load_4d(sm + Lay::GT, &tmG, fb, 0, h, t0, b);
       }
       last_issued[s] = c;
       if (PC) {  // channels 0-63 of this stage's per-channel scaling
         if (!warp_wait(&bars[B_FULL + s], (c / kStages) & 1, abort_flag, lane)) break;
-        scale_channels(sm + Lay::KQ + s * 4 * kTileBytes, sm + Lay::KH + s * 2 * kTileBytes,
-                       reinterpret_cast<float *>(sm + Lay::GT), gv, 0, lane);
+        float *gt = reinterpret_cast<float *>(sm + Lay::GT);
+        const int r = scale_channels(sm + Lay::KQ + s * 4 * kTileBytes,
+                                     sm + Lay::KH + s * 2 * kTileBytes, gt, gt + 32 * 64,
+                                     &bars[B_GF], c & 1, &tmG, h, b, c + 1 < n ? t0 + C : -1,
+                                     gv, 0, lane, abort_flag);
+        if (c + 1 < n && r >= 1) gate_req[0] = c + 1;
+        if (c + 1 < n && r == 2) gate_req[1] = c + 1;
+        if (r < 2) break;
         fence_proxy_async_smem();
         warp_arrive(&bars[B_SCALED + (c & 1)]);
       }
@@ -795,17 +839,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c = last_issued[s];
         if (c >= 0) drain_wait(&bars[B_FULL + s], (c / kStages) & 1);
       }
+      if (PC) {
+        drain_wait(&bars[B_GF + 0], gate_req[0] & 1);
+        drain_wait(&bars[B_GF + 1], gate_req[1] & 1);
+      }
     }
   } else if (warp == kVWarp && PC) {
     // ================================================================ V producer + PC scaling
-    if (lane == 0) tma_prefetch_desc(&tmV);
-    int last = -1;
+    float *gt = reinterpret_cast<float *>(sm + Lay::GT) + 2 * 32 * 64;  // this warp's rows
+    if (lane == 0) {
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&bars[B_GF + 2], 32 * 64 * 4);
+      tma_load_4d(gt, &tmG, &bars[B_GF + 2], 64, h, 0, b);
+      mbar_arrive_expect_tx(&bars[B_GF + 3], 32 * 64 * 4);
+      tma_load_4d(gt + 32 * 64, &tmG, &bars[B_GF + 3], 64, h, 32, b);
+    }
+    int last = -1, gate_req[2] = {0, 0};
     for (int c = 0; c < n; ++c) {
       const int s = c % kStages;
       if (!warp_wait(&bars[B_FULL + s], (c / kStages) & 1, abort_flag, lane)) break;
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
-      scale_channels(sm + Lay::KQ + s * 4 * kTileBytes, sm + Lay::KH + s * 2 * kTileBytes,
-                     reinterpret_cast<float *>(sm + Lay::GT), gv, 64, lane);
+      const int r = scale_channels(sm + Lay::KQ + s * 4 * kTileBytes,
+                                   sm + Lay::KH + s * 2 * kTileBytes, gt, gt + 32 * 64,
+                                   &bars[B_GF + 2], c & 1, &tmG, h, b,
+                                   c + 1 < n ? (c + 1) * C : -1, gv, 64, lane, abort_flag);
+      if (c + 1 < n && r >= 1) gate_req[0] = c + 1;
+      if (c + 1 < n && r == 2) gate_req[1] = c + 1;
+      if (r < 2) break;
       fence_proxy_async_smem();
       warp_arrive(&bars[B_SCALED + (c & 1)]);
       if (c >= 1 && !warp_wait(&bars[B_VEMPTY], (c - 1) & 1, abort_flag, lane)) break;
@@ -819,6 +879,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       last = c;
     }
     if (lane == 0 && last >= 0) drain_wait(&bars[B_VFULL], last & 1);
+    if (lane == 0) {
+      drain_wait(&bars[B_GF + 2], gate_req[0] & 1);
+      drain_wait(&bars[B_GF + 3], gate_req[1] & 1);
+    }
   } else if (warp == kVWarp) {
     // ================================================================ V producer
     if (lane == 0) {
@@ -1432,14 +1496,14 @@ bool make_map_out(CUtensorMap *m, void *base, int B, int T, int H, int d) {
   return r == CUDA_SUCCESS;
 }
 
-// 4-D map over the per-channel gate g [B, T, H, d] fp32, box = 64 tokens x
-// all 128 channels (512-byte rows, no swizzle).
+// 4-D map over the per-channel gate g [B, T, H, d] fp32, box = 32 tokens x
+// 64 channels (one scaling warp's half chunk: 256-byte rows, no swizzle).
 bool make_map_gate(CUtensorMap *m, const float *base, int B, int T, int H, int d) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)T * H * d * 4};
-  cuuint32_t box[4] = {(cuuint32_t)d, 1, 64, 1};
+  cuuint32_t box[4] = {64, 1, 32, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float *>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
