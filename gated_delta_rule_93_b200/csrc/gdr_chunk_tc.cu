@@ -41,11 +41,12 @@
 //   warps 4-7  "prep" group, one chunk ahead: gate cumsum, A/P epilogue,
 //              (I + A)^{-1} with T/T' written straight from it;
 //   warp 8     TMA producer of the K/Q stages (three) + g/beta loads;
-//   warp 9     state-side MMA issuer (one thread);
+//   warp 9     state-side MMA issuer (U^T = V^T T^T, Z, V'^T, O_a, S, O_b;
+//              one thread);
 //   warp 10    TMA producer of V (one stage);
-//   warp 11    prep-side MMA issuer (D1 and U^T = V^T T^T, one thread): an
-//              issue can stall while the tensor core's queue is full, which
-//              must not hold up the prep group.
+//   warp 11    prep-side MMA issuer (D1, one thread): an issue can stall
+//              while the tensor core's queue is full, which must not hold up
+//              the prep group.
 // No TMA load uses cluster multicast.  Hand-offs are mbarriers; every wait
 // is bounded (time-out -> device status word, abort flag, orderly unwind,
 // TMEM freed).
@@ -128,11 +129,11 @@ enum {
   B_FULL = 0,          // [3] K/Q + g/beta of a stage landed            (1 + tx)
   B_EMPTY = 3,         // [3] K/Q stage free (state MMA commit)         (commit)
   B_VFULL = 6,         // V landed                                      (1 + tx)
-  B_VEMPTY,            // V free (prep commit after U)                  (commit)
+  B_VEMPTY,            // V free (commit after U)                       (commit)
   B_D1F,               // D1 written                                    (commit, prep side)
   B_D1E,               // D1 read by the prep group                     (4 warps)
   B_TRDY,              // T, T' and P of a chunk written                (4 warps)
-  B_UF,                // U^T written (T read)                          (commit, prep side)
+  B_UF,                // U^T written (T read)                          (commit)
   B_ZF,                // Z written                                     (commit)
   B_ZR,                // Z (or -Z) bf16 operand in TMEM                (4 warps)
   B_VPF,               // V'^T complete                                 (commit)
@@ -767,6 +768,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // bounded waits run out and the kernel unwinds (no trap, no hang).
       if (c == a.skip_stage_chunk) continue;
       const int t0 = c * C;
+      // The K/Q loads go out first; the phase's one arrival follows once the
+      // gate vectors are written, so whoever sees the phase sees both.
+      if (lane == 0) {
+        uint64_t *fb = &bars[B_FULL + s];
+        mbar_expect_tx(fb, kKQTx);
+        uint8_t *kq = sm + Lay::KQ + s * 4 * kTileBytes;
+        tma_load_4d(kq + 0 * kTileBytes, &tmK, fb, 0, h, t0, b);
+        tma_load_4d(kq + 1 * kTileBytes, &tmQ, fb, 0, h, t0, b);
+        tma_load_4d(kq + 2 * kTileBytes, &tmK, fb, 64, h, t0, b);
+        tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, t0, b);
+      }
+      last_issued[s] = c;
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
       if (PC) {  // beta only; each scaling warp loads its own gate rows
         const size_t tok = ((size_t)b * T + t0 + lane) * H + h;
@@ -808,16 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sig = (c == 0 || !(nxt >= kScaleFloor)) ? 1.f : nxt;
       }
       __syncwarp();
-      if (lane == 0) {
-        uint64_t *fb = &bars[B_FULL + s];
-        mbar_arrive_expect_tx(fb, kKQTx);
-        uint8_t *kq = sm + Lay::KQ + s * 4 * kTileBytes;
-        tma_load_4d(kq + 0 * kTileBytes, &tmK, fb, 0, h, t0, b);
-        tma_load_4d(kq + 1 * kTileBytes, &tmQ, fb, 0, h, t0, b);
-        tma_load_4d(kq + 2 * kTileBytes, &tmK, fb, 64, h, t0, b);
-        tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, t0, b);
-      }
-      last_issued[s] = c;
+      if (lane == 0) mbar_arrive(&bars[B_FULL + s]);
       if (PC) {  // channels 0-63 of this stage's per-channel scaling
         if (!warp_wait(&bars[B_FULL + s], (c / kStages) & 1, abort_flag, lane)) break;
         float *gt = reinterpret_cast<float *>(sm + Lay::GT);
@@ -904,7 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_tp = smem_u32(sm + Lay::TP);
       const uint32_t a_p = smem_u32(sm + Lay::P);
       const uint32_t a_vp = smem_u32(sm + Lay::VP), a_vpd = smem_u32(sm + Lay::VPD);
-      const uint32_t a_kh = smem_u32(sm + Lay::KH);
+      const uint32_t a_kh = smem_u32(sm + Lay::KH), a_v = smem_u32(sm + Lay::V);
+      const uint32_t a_t = smem_u32(sm + Lay::T);
       auto W = [&](int slot, uint32_t parity) {
         const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
         tc_fence_after();
@@ -927,8 +932,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                       sdesc_sw128(kq + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32, 16, 1024),
                       ID_N64, kk > 0);
         mma_commit(&bars[B_ZF]);
-        // V'^T = U^T + Z (-T')^T, or (-Z) T'^T   (U^T from the prep-side issuer)
-        if (!(ok = W(B_ZR, ph) && W(B_UF, ph))) break;
+        // U^T = V^T T^T into the V' accumulator, once T of the chunk is
+        // written and V has landed (the previous V' was converted: its VPR
+        // wait precedes in this thread).  PC: T is in the T' buffer.
+        if (!(ok = W(B_TRDY, ph) && W(B_VFULL, ph))) break;
+        {
+          const uint32_t tt = PC ? a_tp + (c & 1) * kTileBytes : a_t;
+#pragma unroll 1
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tm + TM_UV, sdesc_sw128(a_v + kk * 2048, kTileBytes, 1024),
+                        sdesc_sw128(tt + kk * 32, 16, 1024), ID_U, kk > 0);
+          mma_commit(&bars[B_UF]);      // T read: the prep group may write the next T
+          mma_commit(&bars[B_VEMPTY]);  // V read
+        }
+        // V'^T = U^T + Z (-T')^T, or (-Z) T'^T
+        if (!(ok = W(B_ZR, ph))) break;
         const uint32_t tp = a_tp + (c & 1) * kTileBytes;
 #pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
@@ -973,8 +991,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kPrepMmaWarp) {
     // ================================================================ prep-side MMAs
     if (lane == 0) {
-      const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_v = smem_u32(sm + Lay::V);
-      const uint32_t a_t = smem_u32(sm + Lay::T), a_kh = smem_u32(sm + Lay::KH);
+      const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_kh = smem_u32(sm + Lay::KH);
       auto W = [&](int slot, uint32_t parity) {
         const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
         tc_fence_after();
@@ -998,25 +1015,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bars[B_D1F]);
       };
       // D1 of chunk c + 1 goes out as soon as the prep group has read D1 of
-      // chunk c; U^T of chunk c once T is written and the state group has
-      // converted the previous V'^T (the accumulator is shared).
+      // chunk c and the chunk's operands are ready.
       bool ok = ready(0);
       if (ok) issue_d1(0);
-      for (int c = 0; c < n && ok; ++c) {
-        if (c + 1 < n) {
-          if (!(ok = W(B_D1E, c & 1) && ready(c + 1))) break;
-          issue_d1(c + 1);
-        }
-        if (!(ok = W(B_TRDY, c & 1) && (c < 1 || W(B_VPR, (c - 1) & 1)) && W(B_VFULL, c & 1)))
-          break;
-        // PC: T is written into the T' buffer of the chunk
-        const uint32_t tt = PC ? smem_u32(sm + Lay::TP) + (c & 1) * kTileBytes : a_t;
-#pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tm + TM_UV, sdesc_sw128(a_v + kk * 2048, kTileBytes, 1024),
-                      sdesc_sw128(tt + kk * 32, 16, 1024), ID_U, kk > 0);
-        mma_commit(&bars[B_UF]);
-        mma_commit(&bars[B_VEMPTY]);
+      for (int c = 0; c + 1 < n && ok; ++c) {
+        if (!(ok = W(B_D1E, c & 1) && ready(c + 1))) break;
+        issue_d1(c + 1);
       }
       mma_commit(&bars[B_FIN2]);
       drain_wait(&bars[B_FIN2], 0);
