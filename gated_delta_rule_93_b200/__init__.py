@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     chunk_fwd,
     chunk_fwd_kernel_launches,
     chunk_fwd_segmented,
+    chunk_fwd_varlen,
     chunk_fwd_workspace_bytes,
     device_status,
     lib,
@@ -16,6 +17,6 @@ from .binding import (  # noqa: F401
     step,
 )
 
-__all__ = ["chunk_fwd", "chunk_fwd_kernel_launches", "chunk_fwd_segmented",
+__all__ = ["chunk_fwd", "chunk_fwd_kernel_launches", "chunk_fwd_segmented", "chunk_fwd_varlen",
            "chunk_fwd_workspace_bytes", "step", "device_status", "lib", "status_string",
            "GdrError"]

@@ -29,6 +29,7 @@ EXPORTS = (
     "gdr_chunk_fwd_kernel_launches",
     "gdr_chunk_fwd",
     "gdr_chunk_fwd_segmented",
+    "gdr_chunk_fwd_varlen",
     "gdr_step",
     "gdr_get_device_status",
     "gdr_status_string",
@@ -65,6 +66,9 @@ def lib():
             L.gdr_chunk_fwd_segmented.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, i, i, i, i,
                                                   i, i, i, vp, sz, vp]
             L.gdr_chunk_fwd_segmented.restype = i
+            L.gdr_chunk_fwd_varlen.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, i, i, i,
+                                               i, i, i, vp]
+            L.gdr_chunk_fwd_varlen.restype = i
             L.gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp]
             L.gdr_step.restype = i
             L.gdr_get_device_status.argtypes = [vp]
@@ -252,5 +256,49 @@ def chunk_fwd_segmented(q, k, v, g, beta, S0=None, *, segments, workspace,
             _ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk, _ptr(beta), _ptr(S0),
             _ptr(o), _ptr(S_T), B, T, H, dk, dv, C, int(segments), _ptr(workspace),
             workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc)
+    return o, S_T
+
+
+def chunk_fwd_varlen(q, k, v, g, beta, cu_seqlens, S0=None, *, output_final_state=True, o=None,
+                     S_T=None, C=64, stream=None):
+    """``gdr_chunk_fwd_varlen``: N packed sequences of different lengths.
+
+    q, k [total, H, dk]; v [total, H, dv] (bf16); g [total, H] or
+    [total, H, dk] fp32; beta [total, H] fp32; cu_seqlens int32 CUDA tensor
+    [N + 1] (sequence i = tokens cu_seqlens[i] .. cu_seqlens[i + 1] - 1);
+    S0 [N, H, dv, dk] fp32 or None.  Returns (o [total, H, dv], S_T or None).
+    """
+    _need(q, "q")
+    dev = q.device
+    total, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (total, H, dk), dev)
+    _need(v, "v", dt, (total, H, dv), dev)
+    if g.dim() == 3:
+        _need(g, "g", torch.float32, (total, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (total, H), dev)
+        gk = GDR_GATE_SCALAR
+    _need(beta, "beta", torch.float32, (total, H), dev)
+    if not isinstance(cu_seqlens, torch.Tensor) or cu_seqlens.dtype != torch.int32 or \
+            cu_seqlens.device != dev or cu_seqlens.dim() != 1 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor [N + 1] on the inputs' device")
+    N = cu_seqlens.numel() - 1
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (N, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((total, H, dv), dtype=dt, device=dev)
+    _need(o, "o", dt, (total, H, dv), dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (N, H, dv, dk), dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_chunk_fwd_varlen(
+            _ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk, _ptr(beta), _ptr(cu_seqlens),
+            _ptr(S0), _ptr(o), _ptr(S_T), N, total, H, dk, dv, C, _stream_handle(stream))
     _check(rc)
     return o, S_T

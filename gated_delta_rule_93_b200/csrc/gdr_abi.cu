@@ -231,6 +231,37 @@ gdr_status gdr_chunk_fwd_segmented(const void *q, const void *k, const void *v,
                    "gdr_chunk_fwd_segmented launch");
 }
 
+gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                                const float *g, gdr_gate_kind gate, const float *beta,
+                                const int *cu_seqlens, const float *S0, void *o, float *S_T,
+                                int N, int total_T, int H, int dk, int dv, int C,
+                                gdr_stream_t stream) {
+  if (N < 0) return fail(GDR_ERR_INVALID_ARG, "negative N");
+  gdr::ChunkArgs a;
+  gdr_status st = check_chunk(q, k, v, in_dtype, g, gate, beta, S0, o, S_T, 1, total_T, H, dk,
+                              dv, C, &a);
+  if (st != GDR_OK) return st;
+  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128)
+    return fail(GDR_ERR_UNSUPPORTED, "packed sequences need bf16 inputs and dk = dv = 128");
+  if ((size_t)N * H == 0) return ok();
+  if (!cu_seqlens) return fail(GDR_ERR_INVALID_ARG, "null cu_seqlens");
+  if ((size_t)N * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "N*H too large");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = status_word(&a.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd_varlen status word");
+  if (total_T == 0) {  // every sequence is empty: S_T = S0 (or 0)
+    const size_t bytes = (size_t)N * H * dv * dk * sizeof(float);
+    if (S_T && S0 && S_T != S0)
+      e = cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s);
+    else if (S_T && !S0)
+      e = cudaMemsetAsync(S_T, 0, bytes, s);
+    return from_cuda(e, "gdr_chunk_fwd_varlen copy");
+  }
+  a.B = N;
+  a.cu_seqlens = cu_seqlens;
+  return from_cuda(gdr::launch_chunk_tc(a, s), "gdr_chunk_fwd_varlen launch");
+}
+
 gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                     const float *g, gdr_gate_kind gate, const float *beta, float *S, void *o,
                     int N, int H, int dk, int dv, gdr_stream_t stream) {

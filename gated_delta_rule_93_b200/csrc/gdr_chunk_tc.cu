@@ -589,7 +589,8 @@ __device__ __forceinline__ float ex2(float x) {
 
 // Per-channel gates, one warp, channels j0 .. j0 + 63 of a chunk (lane l:
 // the adjacent pair j0 + 2 l, j0 + 2 l + 1).  g0 / g1: the warp's gate rows
-// 0-31 / 32-63 of the chunk ([32][64] fp32 log decay, zero past T), landed
+// 0-31 / 32-63 of the chunk ([32][64] fp32 log decay; rows from nv on read as
+// zero: past the end of the sequence), landed
 // on gf[0] / gf[1] (phase parity ph).  The cumulative log decay gc (log2
 // units) of rows 0-31 is formed in place; the reference m = gc at row 31,
 // e^{m} and e^{gc_last - m} go into the stage's gate vectors, and the
@@ -599,7 +600,8 @@ __device__ __forceinline__ float ex2(float x) {
 // state kept as S Diag(e^{m}), Z and O_a carry e^{gc} (decay from the chunk
 // start) and the update V'^T K^ carries e^{m - gc}.  The factors stay within
 // e^{|gc_last| / 2}.  Each half is refilled with rows of the chunk at token
-// t0n (none if t0n < 0) as soon as the warp has read it, so the load runs
+// t0n of tensor row bt (none if t0n < 0) as soon as the warp has read it, so
+// the load runs
 // under the other half's work.  Returns 2 when done, 1 if the wait for rows
 // 32-63 gave up (rows 0-31 already refilled), 0 if the first wait gave up.
 __device__ __forceinline__ void scale_row(uint8_t *kt, uint8_t *qt, uint8_t *ht, int t, int jc,
@@ -616,8 +618,8 @@ __device__ __forceinline__ void scale_row(uint8_t *kt, uint8_t *qt, uint8_t *ht,
 }
 
 __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, uint64_t *gf,
-                              uint32_t ph, const CUtensorMap *tmG, int h, int b, int t0n,
-                              float *gv, int j0, int lane, volatile int *abort_flag) {
+                              uint32_t ph, const CUtensorMap *tmG, int h, int bt, int t0n,
+                              int nv, float *gv, int j0, int lane, volatile int *abort_flag) {
   constexpr float kLog2e = 1.4426950408889634f;
   const int jl = 2 * lane, j = j0 + jl, hh = j >> 6, jc = j & 63;
   uint8_t *kt = kq + (2 * hh) * kTileBytes, *qt = kt + kTileBytes, *ht = kh + hh * kTileBytes;
@@ -626,7 +628,7 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
 #pragma unroll 8
   for (int t = 0; t < 32; ++t) {
     float2 *p = reinterpret_cast<float2 *>(g0 + t * 64 + jl);
-    const float2 x = *p;
+    const float2 x = t < nv ? *p : make_float2(0.f, 0.f);
     acc.x += x.x * kLog2e;
     acc.y += x.y * kLog2e;
     *p = acc;
@@ -644,12 +646,13 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
   __syncwarp();
   if (lane == 0 && t0n >= 0) {
     mbar_arrive_expect_tx(&gf[0], 32 * 64 * 4);
-    tma_load_4d(g0, tmG, &gf[0], j0, h, t0n, b);
+    tma_load_4d(g0, tmG, &gf[0], j0, h, t0n, bt);
   }
   if (!warp_wait(&gf[1], ph, abort_flag, lane)) return 1;
 #pragma unroll 4
   for (int t = 32; t < 64; ++t) {
-    const float2 x = *reinterpret_cast<const float2 *>(g1 + (t - 32) * 64 + jl);
+    const float2 x = t < nv ? *reinterpret_cast<const float2 *>(g1 + (t - 32) * 64 + jl)
+                            : make_float2(0.f, 0.f);
     acc.x += x.x * kLog2e;
     acc.y += x.y * kLog2e;
     scale_row(kt, qt, ht, t, jc, acc.x - m.x, acc.y - m.y);
@@ -657,7 +660,7 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
   __syncwarp();
   if (lane == 0 && t0n >= 0) {
     mbar_arrive_expect_tx(&gf[1], 32 * 64 * 4);
-    tma_load_4d(g1, tmG, &gf[1], j0, h, t0n + 32, b);
+    tma_load_4d(g1, tmG, &gf[1], j0, h, t0n + 32, bt);
   }
   gv[kGateEgm + j] = ex2(acc.x - m.x);
   gv[kGateEgm + j + 1] = ex2(acc.y - m.y);
@@ -681,7 +684,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-  const int T = a.T, H = a.H;
+  const int H = a.H;
+  // Dense: sequence b is row b of the [B, T, H, d] tensors.  Packed
+  // (cu_seqlens): sequence b is tokens [cu[b], cu[b + 1]) of row 0 of the
+  // [1, total, H, d] tensors.  tb: its first token, bt: its row, T: its
+  // length (clamped into the tensor).
+  int tb = 0, bt = b, T = a.T;
+  if (a.cu_seqlens) {
+    const int s0 = min(max(a.cu_seqlens[b], 0), a.T);
+    const int s1 = min(max(a.cu_seqlens[b + 1], s0), a.T);
+    tb = s0;
+    bt = 0;
+    T = s1 - s0;
+  }
   const int n = (T + C - 1) / C;
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + Lay::BAR);
@@ -741,7 +756,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tm = *tmem_slot;
   const uint32_t lane_base = tm + ((uint32_t)((warp & 3) * 32) << 16);
 
-  if (warp == kProducerWarp) {
+  if (n == 0) {
+    // ================================================================ empty packed sequence
+    if (warp < 4 && a.S_T) {  // S_T = S0 (or 0); row i of the state per thread
+      const float4 *src = a.S0 ? reinterpret_cast<const float4 *>(a.S0 + ((size_t)bh * DV + tid) * DK)
+                               : nullptr;
+      float4 *dst = reinterpret_cast<float4 *>(a.S_T + ((size_t)bh * DV + tid) * DK);
+      for (int e = 0; e < DK / 4; ++e) dst[e] = src ? src[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  } else if (warp == kProducerWarp) {
     // ================================================================ K/Q producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -752,9 +775,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (PC && lane == 0) {  // this warp's gate rows of chunk 0
       float *gt = reinterpret_cast<float *>(sm + Lay::GT);
       mbar_arrive_expect_tx(&bars[B_GF + 0], 32 * 64 * 4);
-      tma_load_4d(gt, &tmG, &bars[B_GF + 0], 0, h, 0, b);
+      tma_load_4d(gt, &tmG, &bars[B_GF + 0], 0, h, tb, bt);
       mbar_arrive_expect_tx(&bars[B_GF + 1], 32 * 64 * 4);
-      tma_load_4d(gt + 32 * 64, &tmG, &bars[B_GF + 1], 0, h, 32, b);
+      tma_load_4d(gt + 32 * 64, &tmG, &bars[B_GF + 1], 0, h, tb + 32, bt);
     }
     // Scalar gates: the state group's scale sequence, replayed with the same
     // fp32 operations: sig = the scale of S_b for the chunk being produced.
@@ -774,20 +797,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t *fb = &bars[B_FULL + s];
         mbar_expect_tx(fb, kKQTx);
         uint8_t *kq = sm + Lay::KQ + s * 4 * kTileBytes;
-        tma_load_4d(kq + 0 * kTileBytes, &tmK, fb, 0, h, t0, b);
-        tma_load_4d(kq + 1 * kTileBytes, &tmQ, fb, 0, h, t0, b);
-        tma_load_4d(kq + 2 * kTileBytes, &tmK, fb, 64, h, t0, b);
-        tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, t0, b);
+        tma_load_4d(kq + 0 * kTileBytes, &tmK, fb, 0, h, tb + t0, bt);
+        tma_load_4d(kq + 1 * kTileBytes, &tmQ, fb, 0, h, tb + t0, bt);
+        tma_load_4d(kq + 2 * kTileBytes, &tmK, fb, 64, h, tb + t0, bt);
+        tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, tb + t0, bt);
       }
       last_issued[s] = c;
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
       if (PC) {  // beta only; each scaling warp loads its own gate rows
-        const size_t tok = ((size_t)b * T + t0 + lane) * H + h;
+        const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
         gv[kGateBeta + lane] = t0 + lane < T ? a.beta[tok] : 0.f;
         gv[kGateBeta + lane + 32] = t0 + lane + 32 < T ? a.beta[tok + (size_t)32 * H] : 0.f;
       } else {
         float gl0 = 0.f, gl1 = 0.f, b0 = 0.f, b1 = 0.f;
-        const size_t tok = ((size_t)b * T + t0 + lane) * H + h;
+        const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
         if (t0 + lane < T) {
           gl0 = a.g[tok];
           b0 = a.beta[tok];
@@ -827,8 +850,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float *gt = reinterpret_cast<float *>(sm + Lay::GT);
         const int r = scale_channels(sm + Lay::KQ + s * 4 * kTileBytes,
                                      sm + Lay::KH + s * 2 * kTileBytes, gt, gt + 32 * 64,
-                                     &bars[B_GF], c & 1, &tmG, h, b, c + 1 < n ? t0 + C : -1,
-                                     gv, 0, lane, abort_flag);
+                                     &bars[B_GF], c & 1, &tmG, h, bt,
+                                     c + 1 < n ? tb + t0 + C : -1, T - t0, gv, 0, lane,
+                                     abort_flag);
         if (c + 1 < n && r >= 1) gate_req[0] = c + 1;
         if (c + 1 < n && r == 2) gate_req[1] = c + 1;
         if (r < 2) break;
@@ -854,9 +878,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmV);
       mbar_arrive_expect_tx(&bars[B_GF + 2], 32 * 64 * 4);
-      tma_load_4d(gt, &tmG, &bars[B_GF + 2], 64, h, 0, b);
+      tma_load_4d(gt, &tmG, &bars[B_GF + 2], 64, h, tb, bt);
       mbar_arrive_expect_tx(&bars[B_GF + 3], 32 * 64 * 4);
-      tma_load_4d(gt + 32 * 64, &tmG, &bars[B_GF + 3], 64, h, 32, b);
+      tma_load_4d(gt + 32 * 64, &tmG, &bars[B_GF + 3], 64, h, tb + 32, bt);
     }
     int last = -1, gate_req[2] = {0, 0};
     for (int c = 0; c < n; ++c) {
@@ -865,8 +889,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
       const int r = scale_channels(sm + Lay::KQ + s * 4 * kTileBytes,
                                    sm + Lay::KH + s * 2 * kTileBytes, gt, gt + 32 * 64,
-                                   &bars[B_GF + 2], c & 1, &tmG, h, b,
-                                   c + 1 < n ? (c + 1) * C : -1, gv, 64, lane, abort_flag);
+                                   &bars[B_GF + 2], c & 1, &tmG, h, bt,
+                                   c + 1 < n ? tb + (c + 1) * C : -1, T - c * C, gv, 64, lane,
+                                   abort_flag);
       if (c + 1 < n && r >= 1) gate_req[0] = c + 1;
       if (c + 1 < n && r == 2) gate_req[1] = c + 1;
       if (r < 2) break;
@@ -876,8 +901,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         uint8_t *vv = sm + Lay::V;
         mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
-        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, c * C, b);
-        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, c * C, b);
+        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, tb + c * C, bt);
+        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, tb + c * C, bt);
       }
       __syncwarp();
       last = c;
@@ -896,8 +921,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c >= 1 && !wait_or_abort(&bars[B_VEMPTY], (c - 1) & 1, abort_flag)) break;
         uint8_t *vv = sm + Lay::V;
         mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
-        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, c * C, b);
-        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, c * C, b);
+        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, tb + c * C, bt);
+        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, tb + c * C, bt);
         last = c;
       }
       if (last >= 0) drain_wait(&bars[B_VFULL], last & 1);
@@ -1436,8 +1461,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          if (a.write_o) tma_store_4d(&tmO, sm + Lay::VPD + 4096 * warp, 32 * warp, h, c * C, b);
+        const int rows = T - c * C;  // valid rows of the chunk
+        if (a.cu_seqlens && rows < C) {
+          // The last chunk of a packed sequence: the TMA box would run into
+          // the next sequence's rows, so the valid rows go out with plain
+          // 16-byte stores (chunk j of staging row r sits at j ^ ((r / 2) % 4)).
+          if (a.write_o) {
+            const uint8_t *st = sm + Lay::VPD + 4096 * warp;
+            for (int r = lane; r < rows; r += 32) {
+              uint4 *dst = reinterpret_cast<uint4 *>(
+                  reinterpret_cast<__nv_bfloat16 *>(a.o) +
+                  (((size_t)bt * a.T + tb + c * C + r) * H + h) * DV + 32 * warp);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                dst[j] = *reinterpret_cast<const uint4 *>(st + r * 64 + 16 * (j ^ ((r >> 1) & 3)));
+            }
+          }
+        } else if (lane == 0) {
+          if (a.write_o)
+            tma_store_4d(&tmO, sm + Lay::VPD + 4096 * warp, 32 * warp, h, tb + c * C, bt);
           tma_store_commit();
         }
       }
@@ -1539,12 +1581,14 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
   CUtensorMap mq, mk, mv, mg, mo;
   // Without an output (segment passes) the output map is never used; it is
   // built over q so that it is a valid map.
-  if (!make_map(&mq, a.q, a.B, a.T, a.H, DK) || !make_map(&mk, a.k, a.B, a.T, a.H, DK) ||
-      !make_map(&mv, a.v, a.B, a.T, a.H, DV) ||
-      !make_map_out(&mo, a.write_o ? a.o : const_cast<void *>(a.q), a.B, a.T, a.H, DV))
+  // (packed sequences: the tensors are [1, total, H, d]; one CTA per sequence and head)
+  const int mb = a.cu_seqlens ? 1 : a.B;
+  if (!make_map(&mq, a.q, mb, a.T, a.H, DK) || !make_map(&mk, a.k, mb, a.T, a.H, DK) ||
+      !make_map(&mv, a.v, mb, a.T, a.H, DV) ||
+      !make_map_out(&mo, a.write_o ? a.o : const_cast<void *>(a.q), mb, a.T, a.H, DV))
     return cudaErrorInvalidValue;
   if (a.per_channel) {
-    if (!make_map_gate(&mg, a.g, a.B, a.T, a.H, DK)) return cudaErrorInvalidValue;
+    if (!make_map_gate(&mg, a.g, mb, a.T, a.H, DK)) return cudaErrorInvalidValue;
     return launch_variant<true>(a, mq, mk, mv, mg, mo, stream);
   }
   return launch_variant<false>(a, mq, mk, mv, mq, mo, stream);  // gate map unused

@@ -30,6 +30,10 @@ struct ChunkArgs {
   int s0_seg;       // > 0: sequence b reads S0[b / s0_seg] if b % s0_seg == 0, else starts at 0
   int s0_identity;  // 1: sequences without an S0 start from the identity (d_v == d_k)
   int write_o;      // 0: o is not written (may be null)
+  // Packed sequences (tensor-core kernel only): B sequences, sequence b is
+  // tokens [cu_seqlens[b], cu_seqlens[b + 1]) of the [1, T, H, d] tensors
+  // (device int32 [B + 1]); null: dense [B, T, H, d].
+  const int *cu_seqlens;
 };
 
 struct StepArgs {

@@ -84,6 +84,27 @@ def make_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, gate="scalar", with
     return dict(q=q, k=k, v=v, g=g.float(), beta=beta.float(), S0=S0)
 
 
+def make_varlen_inputs(lens, H, dk, dv, dtype=torch.bfloat16, gate="scalar", with_S0=True,
+                       seed=0):
+    """Packed inputs for ``gdr_chunk_fwd_varlen``: len(lens) sequences back to back.
+
+    Returns dict of q, k [total,H,dk], v [total,H,dv], g [total,H] (or
+    [total,H,dk]), beta [total,H], S0 [N,H,dv,dk] fp32 (or None) and
+    cu_seqlens int32 [N+1] (all on the CPU).  Token draws as
+    ``make_chunk_inputs(1, total, ...)``; S0 from its own stream.
+    """
+    total = int(sum(lens))
+    d = make_chunk_inputs(1, total, H, dk, dv, dtype, gate, False, seed=seed)
+    out = {key: d[key][0] for key in ("q", "k", "v", "g", "beta")}
+    gen = torch.Generator().manual_seed(seed + 7919)
+    out["S0"] = 0.02 * torch.randn(len(lens), H, dv, dk, generator=gen) if with_S0 else None
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + int(n))
+    out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32)
+    return out
+
+
 def make_step_inputs(N, H, dk, dv, steps, dtype=torch.bfloat16, gate="scalar", seed=0):
     """Inputs for ``steps`` consecutive ``gdr_step`` calls.
 

@@ -143,6 +143,32 @@ gdr_status gdr_chunk_fwd_segmented(const void *q, const void *k, const void *v,
                                    void *workspace, size_t ws_bytes, gdr_stream_t stream);
 
 /*
+ * The chunked forward over N packed sequences of different lengths (a
+ * variable-length batch), one state per sequence and head.  Source as
+ * gdr_chunk_fwd: each sequence runs the recurrence of "Decoding Hybrid
+ * Linear Attention Architectures", sections 3 and 5, from its own S0.
+ *
+ *   q, k        [total_T, H, dk]  bf16     the sequences back to back
+ *   v, o        [total_T, H, dv]  bf16
+ *   g           [total_T, H] fp32 (scalar gate) or [total_T, H, dk] (per
+ *               channel); beta [total_T, H] fp32
+ *   cu_seqlens  device int32 [N + 1]: sequence i is tokens
+ *               [cu_seqlens[i], cu_seqlens[i + 1]); non-decreasing from 0 to
+ *               total_T (values outside [0, total_T] are clamped into it)
+ *   S0, S_T     [N, H, dv, dk] fp32 or NULL, as in gdr_chunk_fwd (S0 may
+ *               alias S_T); an empty sequence gets S_T = S0 (or 0)
+ *
+ * S_T feeds gdr_step directly (same layout): prefill, then decode.  Needs
+ * bf16 inputs and dk = dv = 128 (GDR_ERR_UNSUPPORTED otherwise).  One
+ * launch; no workspace.
+ */
+gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                                const float *g, gdr_gate_kind gate, const float *beta,
+                                const int *cu_seqlens, const float *S0, void *o, float *S_T,
+                                int N, int total_T, int H, int dk, int dv, int C,
+                                gdr_stream_t stream);
+
+/*
  * One recurrent decode step for N independent states, S updated in place.
  * Source: "Decoding Hybrid Linear Attention Architectures", section 6
  * (constant-cost update of the fixed-size state per decoded token) with the

@@ -132,3 +132,25 @@ def test_binding_refuses_cpu_tensors(L):
     x = torch.zeros(1, 64, 1, 32)
     with pytest.raises(ValueError, match="CUDA"):
         binding.chunk_fwd(x, x, x, torch.zeros(1, 64, 1), torch.zeros(1, 64, 1))
+
+
+def test_varlen_validation_rejects_before_any_launch(L):
+    """gdr_chunk_fwd_varlen: packed sequences, tensor-core shapes only."""
+    p = _fake_ptr()
+
+    def call(**kw):
+        a = dict(q=p, k=p, v=p, dt=1, g=p, gate=0, beta=p, cu=p, S0=None, o=p, ST=None, N=3,
+                 total=500, H=2, dk=128, dv=128, C=64, st=None)
+        a.update(kw)
+        return L.gdr_chunk_fwd_varlen(a["q"], a["k"], a["v"], a["dt"], a["g"], a["gate"],
+                                      a["beta"], a["cu"], a["S0"], a["o"], a["ST"], a["N"],
+                                      a["total"], a["H"], a["dk"], a["dv"], a["C"], a["st"])
+
+    assert call(N=-1) == binding.GDR_ERR_INVALID_ARG
+    assert call(cu=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(dt=0) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dk=64, dv=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(C=32) == binding.GDR_ERR_UNSUPPORTED
+    assert call(q=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(o=_fake_ptr(2)) == binding.GDR_ERR_INVALID_ARG
+    assert call(N=0) == binding.GDR_OK
