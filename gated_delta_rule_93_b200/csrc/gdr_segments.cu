@@ -24,61 +24,89 @@ namespace {
 constexpr int kDim = 128;                   // d_k = d_v of the tensor-core kernel
 constexpr int kRows = 16;                   // state rows per combine CTA
 constexpr int kRowBlocks = kDim / kRows;
-constexpr int kCombineThreads = 256;        // 16 rows x 16 column groups of 8
-constexpr size_t kCombineSmem = (size_t)(kDim * kDim + kRows * kDim) * sizeof(float);
+constexpr int kCombineThreads = 256;        // 4 row groups x 64 column pairs
+// M, E_a of the current segment and the running rows
+constexpr size_t kCombineSmem = (size_t)(2 * kDim * kDim + kRows * kDim) * sizeof(float);
+
+// 16-byte global -> shared copy that bypasses the registers (many in flight
+// per thread), and the wait for all of this thread's copies.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                   (uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
 
 // One CTA per (b, h) and block of 16 state rows (rows of S are independent
 // under S <- S M + E).  E_a: end states of pass 1a, E_b: of pass 1b, X: the
 // start state of every segment (written), S_T: the final state (optional),
-// all [B * P, H, 128, 128] except S0 / S_T [B, H, 128, 128].
+// all [B * P, H, 128, 128] except S0 / S_T [B, H, 128, 128].  Each thread
+// forms 4 rows x 2 columns of the product (a warp shares its rows), so every
+// column pair of M read from shared memory serves four rows.
 __global__ void __launch_bounds__(kCombineThreads)
     combine_segments(const float *__restrict__ S0, const float *__restrict__ Ea,
                      const float *__restrict__ Eb, float *__restrict__ X, float *S_T, int H,
                      int P) {
   extern __shared__ float smem[];
-  float *M = smem;                // [128][128] transition of the current segment
-  float *R = smem + kDim * kDim;  // [16][128] rows of the running start state
+  float *M = smem;                    // [128][128] transition of the current segment
+  float *MA = smem + kDim * kDim;     // [128][128] its E_a
+  float *R = smem + 2 * kDim * kDim;  // [16][128] rows of the running start state
   const int bh = blockIdx.x, b = bh / H, h = bh % H, r0 = blockIdx.y * kRows;
   const int t = threadIdx.x;
   const size_t st = (size_t)kDim * kDim;
   auto seg = [&](int p) { return ((size_t)(b * P + p) * H + h) * st; };
 
   // segment 0 starts from S0 (or 0); segment 1 from segment 0's end state
-  for (int i = t; i < kRows * kDim; i += kCombineThreads) {
-    const size_t off = (size_t)r0 * kDim + i;
-    X[seg(0) + off] = S0 ? S0[(size_t)bh * st + off] : 0.f;
-    const float e0 = Ea[seg(0) + off];
-    R[i] = e0;
-    X[seg(1) + off] = e0;
+#pragma unroll
+  for (int j = 0; j < kRows * kDim / 4 / kCombineThreads; ++j) {
+    const int i = t + j * kCombineThreads;  // float4 index in the row block
+    const size_t off = (size_t)r0 * kDim + 4 * i;
+    const float4 s0 = S0 ? *reinterpret_cast<const float4 *>(S0 + (size_t)bh * st + off)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 e0 = *reinterpret_cast<const float4 *>(Ea + seg(0) + off);
+    *reinterpret_cast<float4 *>(X + seg(0) + off) = s0;
+    *reinterpret_cast<float4 *>(X + seg(1) + off) = e0;
+    reinterpret_cast<float4 *>(R)[i] = e0;
   }
-  const int r = t / 16, c0 = (t % 16) * 8;
+  const int rg = t >> 6, c0 = (t & 63) * 2;  // rows 4 rg .. 4 rg + 3, columns c0, c0 + 1
   for (int p = 1; p < P; ++p) {
     __syncthreads();  // R written, M free
     const float4 *ea4 = reinterpret_cast<const float4 *>(Ea + seg(p));
     const float4 *eb4 = reinterpret_cast<const float4 *>(Eb + seg(p));
-    float4 *m4 = reinterpret_cast<float4 *>(M);
-    for (int i = t; i < kDim * kDim / 4; i += kCombineThreads) {
-      const float4 x = eb4[i], y = ea4[i];
+    float4 *m4 = reinterpret_cast<float4 *>(M), *a4 = reinterpret_cast<float4 *>(MA);
+    // E_b and E_a of the segment into shared memory, every copy in flight at
+    // once, then M = E_b - E_a in place
+#pragma unroll 8
+    for (int j = 0; j < kDim * kDim / 4 / kCombineThreads; ++j) {
+      const int i = t + j * kCombineThreads;
+      cp_async16(m4 + i, eb4 + i);
+      cp_async16(a4 + i, ea4 + i);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll 8
+    for (int j = 0; j < kDim * kDim / 4 / kCombineThreads; ++j) {
+      const int i = t + j * kCombineThreads;
+      const float4 x = m4[i], y = a4[i];
       m4[i] = make_float4(x.x - y.x, x.y - y.y, x.z - y.z, x.w - y.w);
     }
     __syncthreads();
-    float acc[8];
-    const float *er = Ea + seg(p) + (size_t)(r0 + r) * kDim + c0;
+    float2 acc[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = er[j];
-#pragma unroll 4
+    for (int i = 0; i < 4; ++i)
+      acc[i] = *reinterpret_cast<const float2 *>(MA + (size_t)(r0 + 4 * rg + i) * kDim + c0);
+#pragma unroll 8
     for (int k = 0; k < kDim; ++k) {
-      const float s = R[r * kDim + k];
-      const float4 ma = *reinterpret_cast<const float4 *>(M + k * kDim + c0);
-      const float4 mb = *reinterpret_cast<const float4 *>(M + k * kDim + c0 + 4);
-      acc[0] = fmaf(s, ma.x, acc[0]);
-      acc[1] = fmaf(s, ma.y, acc[1]);
-      acc[2] = fmaf(s, ma.z, acc[2]);
-      acc[3] = fmaf(s, ma.w, acc[3]);
-      acc[4] = fmaf(s, mb.x, acc[4]);
-      acc[5] = fmaf(s, mb.y, acc[5]);
-      acc[6] = fmaf(s, mb.z, acc[6]);
-      acc[7] = fmaf(s, mb.w, acc[7]);
+      const float2 m = *reinterpret_cast<const float2 *>(M + k * kDim + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float s = R[(4 * rg + i) * kDim + k];
+        acc[i].x = fmaf(s, m.x, acc[i].x);
+        acc[i].y = fmaf(s, m.y, acc[i].y);
+      }
     }
     __syncthreads();  // every thread has read R
     float *dst = nullptr;
@@ -87,11 +115,10 @@ __global__ void __launch_bounds__(kCombineThreads)
     else if (S_T)
       dst = S_T + (size_t)bh * st;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) R[r * kDim + c0 + j] = acc[j];
-    if (dst) {
-      float4 *d4 = reinterpret_cast<float4 *>(dst + (size_t)(r0 + r) * kDim + c0);
-      d4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      d4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    for (int i = 0; i < 4; ++i) {
+      const int rr = 4 * rg + i;
+      *reinterpret_cast<float2 *>(R + rr * kDim + c0) = acc[i];
+      if (dst) *reinterpret_cast<float2 *>(dst + (size_t)(r0 + rr) * kDim + c0) = acc[i];
     }
   }
 }
