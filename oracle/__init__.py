@@ -14,6 +14,12 @@ Contents
     ("Decoding Hybrid Linear Attention Architectures", section 3 items 3 and
     6 with the single-step pseudocode; "Linear Attention Variants", section
     "DeltaNet: Error-Correcting Writes".)
+``gla_fwd``
+    The gated-linear-attention recurrence S_t = S_{t-1} Diag(alpha_t) +
+    v_t k_t^T, o_t = S_t q_t (additive write, no erase), from its own plain
+    loop in ``gdr_oracle.c`` ("Decoding Hybrid Linear Attention
+    Architectures", section 3 item 4; "Linear Attention Variants", GLA
+    section).
 ``chunked``
     A staged fp64 NumPy restatement of the chunkwise algorithm ("Decoding
     Hybrid Linear Attention Architectures", section 5, inter-chunk recursion
@@ -66,6 +72,8 @@ def _load():
             lib.oracle_gdr_fwd.restype = i
             lib.oracle_gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, i]
             lib.oracle_gdr_step.restype = i
+            lib.oracle_gla_fwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, i, i]
+            lib.oracle_gla_fwd.restype = i
             _lib = lib
     return _lib
 
@@ -130,6 +138,42 @@ def gdr_fwd(q, k, v, g, beta, S0=None, gate="scalar", nthreads=None):
                                 _ptr(S0d), _ptr(o), _ptr(S_T), B, T, H, dk, dv, n)
     if rc != 0:
         raise ValueError("oracle_gdr_fwd rejected its arguments")
+    return o, S_T
+
+
+def gla_fwd(q, k, v, g, S0=None, gate="scalar", nthreads=None):
+    """fp64 gated linear attention over a whole sequence (additive write).
+
+    q, k: [B,T,H,dk]; v: [B,T,H,dv] (float32 or uint16 bf16 bits); g = log
+    alpha: [B,T,H] or [B,T,H,dk] float32; S0: [B,H,dv,dk] or None.  Returns
+    (o [B,T,H,dv] float64, S_T [B,H,dv,dk] float64).
+    """
+    q, dt = _as_input(q, "q")
+    k, dt2 = _as_input(k, "k")
+    v, dt3 = _as_input(v, "v")
+    if not (dt == dt2 == dt3):
+        raise TypeError("q, k, v must share one dtype")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != (B, T, H, dk) or v.shape != (B, T, H, dv):
+        raise ValueError("shape mismatch among q, k, v")
+    gk = GATE_PER_CHANNEL if gate in ("channel", "per_channel", GATE_PER_CHANNEL) else GATE_SCALAR
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    want_g = (B, T, H, dk) if gk == GATE_PER_CHANNEL else (B, T, H)
+    if g.shape != want_g:
+        raise ValueError(f"g has shape {g.shape}, expected {want_g}")
+    S0d = None
+    if S0 is not None:
+        S0d = np.ascontiguousarray(S0, dtype=np.float64)
+        if S0d.shape != (B, H, dv, dk):
+            raise ValueError("S0 must be [B,H,dv,dk]")
+    o = np.zeros((B, T, H, dv), np.float64)
+    S_T = np.zeros((B, H, dv, dk), np.float64)
+    n = nthreads or default_threads()
+    rc = _load().oracle_gla_fwd(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), gk, _ptr(S0d), _ptr(o),
+                                _ptr(S_T), B, T, H, dk, dv, n)
+    if rc != 0:
+        raise ValueError("oracle_gla_fwd rejected its arguments")
     return o, S_T
 
 

@@ -191,3 +191,100 @@ int oracle_gdr_step(const void *q, const void *k, const void *v, int in_dtype,
     return oracle_gdr_fwd(q, k, v, in_dtype, g, gate_kind, beta, S, o, S, N, 1,
                           H, dk, dv, nthreads);
 }
+
+/*
+ * Gated linear attention (additive write, no erase):
+ *
+ *     S_t = S_{t-1} Diag(alpha_t) + v_t k_t^T,    o_t = S_t q_t
+ *
+ * Source: "Decoding Hybrid Linear Attention Architectures", section 3 item 4
+ * (GLA family: channel-wise forgetting, the write reverts to accumulation);
+ * "Linear Attention Variants", GLA section (the same recurrence in the
+ * transposed convention).  The gate enters as g = log alpha, scalar per head
+ * or per key channel as above; the output reads the state after the write.
+ * A separate plain loop: it shares nothing with the delta-rule one.
+ */
+typedef struct {
+    const void *q, *k, *v;
+    int in_dtype;
+    const float *g;
+    int gate_kind;
+    const double *S0;
+    double *o;
+    double *S_T;
+    int B, T, H, dk, dv;
+    int next;
+    pthread_mutex_t lock;
+} gla_job_t;
+
+static void gla_head(gla_job_t *J, int b, int h) {
+    const int T = J->T, H = J->H, dk = J->dk, dv = J->dv;
+    double *S = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *kk = (double *)malloc(sizeof(double) * dk);
+    double *qq = (double *)malloc(sizeof(double) * dk);
+    double *alpha = (double *)malloc(sizeof(double) * dk);
+    const size_t sidx = ((size_t)b * H + h) * (size_t)dv * dk;
+    if (J->S0)
+        memcpy(S, J->S0 + sidx, sizeof(double) * (size_t)dv * dk);
+    else
+        memset(S, 0, sizeof(double) * (size_t)dv * dk);
+    for (int t = 0; t < T; ++t) {
+        const size_t tok = ((size_t)b * T + t) * H + h;
+        for (int j = 0; j < dk; ++j) {
+            kk[j] = load_elem(J->k, tok * dk + j, J->in_dtype);
+            qq[j] = load_elem(J->q, tok * dk + j, J->in_dtype);
+            alpha[j] = exp((double)(J->gate_kind == OR_GATE_PER_CHANNEL ? J->g[tok * dk + j]
+                                                                        : J->g[tok]));
+        }
+        /* decay the key axis, then add the outer product v_t k_t^T */
+        for (int i = 0; i < dv; ++i) {
+            const double vi = load_elem(J->v, tok * dv + i, J->in_dtype);
+            for (int j = 0; j < dk; ++j)
+                S[(size_t)i * dk + j] = S[(size_t)i * dk + j] * alpha[j] + vi * kk[j];
+        }
+        /* read-out after the write */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(size_t)i * dk + j] * qq[j];
+            J->o[tok * dv + i] = acc;
+        }
+    }
+    if (J->S_T) memcpy(J->S_T + sidx, S, sizeof(double) * (size_t)dv * dk);
+    free(S);
+    free(kk);
+    free(qq);
+    free(alpha);
+}
+
+static void *gla_worker(void *arg) {
+    gla_job_t *J = (gla_job_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int w = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (w >= J->B * J->H) break;
+        gla_head(J, w / J->H, w % J->H);
+    }
+    return NULL;
+}
+
+int oracle_gla_fwd(const void *q, const void *k, const void *v, int in_dtype, const float *g,
+                   int gate_kind, const double *S0, double *o, double *S_T, int B, int T, int H,
+                   int dk, int dv, int nthreads) {
+    if (!q || !k || !v || !g || !o || B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (in_dtype != OR_F32 && in_dtype != OR_BF16) return -1;
+    if (gate_kind != OR_GATE_SCALAR && gate_kind != OR_GATE_PER_CHANNEL) return -1;
+    gla_job_t J;
+    J.q = q; J.k = k; J.v = v; J.in_dtype = in_dtype; J.g = g; J.gate_kind = gate_kind;
+    J.S0 = S0; J.o = o; J.S_T = S_T;
+    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv; J.next = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    int nt = nthreads > 0 ? nthreads : 1;
+    if (nt > B * H) nt = B * H > 0 ? B * H : 1;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * nt);
+    for (int i = 0; i < nt; ++i) pthread_create(&th[i], NULL, gla_worker, &J);
+    for (int i = 0; i < nt; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}

@@ -352,3 +352,77 @@ def test_oracle_regression_fixture():
                                 arr["S0"].astype(np.float64), gate=c["gate"], nthreads=1)
         assert np.allclose(o, np.array(c["o"]), rtol=0, atol=1e-14)
         assert np.allclose(S_T, np.array(c["S_T"]), rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------- gated linear attention
+# [HLA] section 3 item 4: S_t = S_{t-1} Diag(alpha_t) + v_t k_t^T, o_t = S_t q_t.
+
+def _gla_closed_form(q, k, v, g, S0, gate):
+    """Unrolled: S_t[i, j] = S0[i, j] e^{G_t[j]} + sum_{s<=t} v_s[i] k_s[j] e^{G_t[j] - G_s[j]}
+    with G_t = sum of g up to t (per key channel), computed from cumulative
+    sums, independently of the oracle's loop."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    gg = g.astype(np.float64)
+    if gate == "scalar":
+        gg = np.repeat(gg[..., None], dk, axis=-1)
+    G = np.cumsum(gg, axis=1)  # [B,T,H,dk]
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dv, dk))
+    for b in range(B):
+        for h in range(H):
+            for t in range(T):
+                S = np.zeros((dv, dk)) if S0 is None else S0[b, h] * np.exp(G[b, t, h])[None, :]
+                for s_ in range(t + 1):
+                    S = S + np.outer(v[b, s_, h], k[b, s_, h] * np.exp(G[b, t, h] - G[b, s_, h]))
+                o[b, t, h] = S @ q[b, t, h]
+                if t == T - 1:
+                    ST[b, h] = S
+    return o, ST
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_gla_oracle_matches_closed_form(gate):
+    q, k, v, g, _, s0 = _rand_inputs(2, 9, 2, 5, 3, gate)
+    o, ST = oracle.gla_fwd(q, k, v, g, s0, gate=gate)
+    ro, rS = _gla_closed_form(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64),
+                              g, s0, gate)
+    assert rel_err(o, ro) < 1e-12 and rel_err(ST, rS) < 1e-12
+
+
+def test_gla_without_decay_is_linear_attention():
+    """alpha = 1, S0 = 0: o_t = sum_{s<=t} v_s (k_s . q_t)  (causal linear
+    attention without normaliser, [LAV] linear attention recurrence)."""
+    q, k, v, g, _, _ = _rand_inputs(1, 12, 2, 6, 4, "scalar", S0=False)
+    g[:] = 0.0
+    o, _ = oracle.gla_fwd(q, k, v, g, None)
+    qd, kd, vd = (x.astype(np.float64) for x in (q, k, v))
+    scores = np.einsum("bthd,bshd->bhts", qd, kd)
+    scores = np.tril(scores)
+    want = np.einsum("bhts,bshv->bthv", scores, vd)
+    assert rel_err(o, want) < 1e-12
+
+
+def test_gla_write_is_additive_not_erasing():
+    """Writing the same (k, v) twice with alpha = 1 doubles the state (the
+    delta rule would overwrite: its second write adds nothing)."""
+    q, k, v, g, beta, _ = _rand_inputs(1, 2, 1, 4, 3, "scalar", S0=False)
+    k[0, 1] = k[0, 0]
+    v[0, 1] = v[0, 0]
+    g[:] = 0.0
+    _, ST = oracle.gla_fwd(q, k, v, g, None)
+    one = np.outer(v[0, 0, 0].astype(np.float64), k[0, 0, 0].astype(np.float64))
+    assert rel_err(ST[0, 0], 2 * one) < 1e-12
+    beta[:] = 1.0
+    _, SD = oracle.gdr_fwd(q, k, v, g, beta, None)
+    # k is unit length up to its fp32 rounding, so the erase is exact to ~1e-7
+    assert rel_err(SD[0, 0], one) < 1e-6
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_gla_split_and_resume(gate):
+    q, k, v, g, _, s0 = _rand_inputs(1, 20, 2, 8, 5, gate)
+    o, ST = oracle.gla_fwd(q, k, v, g, s0, gate=gate)
+    oa, Sa = oracle.gla_fwd(q[:, :7], k[:, :7], v[:, :7], g[:, :7], s0, gate=gate)
+    ob, Sb = oracle.gla_fwd(q[:, 7:], k[:, 7:], v[:, 7:], g[:, 7:], Sa, gate=gate)
+    assert rel_err(np.concatenate([oa, ob], axis=1), o) < 1e-12 and rel_err(Sb, ST) < 1e-12
