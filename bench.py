@@ -53,7 +53,8 @@ def algorithmic_bytes(w):
     if w.kind == "step":  # one decode step: S read + written once, q/k/v/g/beta in, o out
         return w.B * w.H * (8 * w.dk * w.dv + (2 * w.dk + w.dv) * e_in + w.dv * e_in
                             + 4 * gate_elems + 4)
-    per_tok = (2 * w.dk + w.dv) * e_in + w.dv * e_in + 4 * gate_elems + 4
+    beta = 0 if w.mixer == "gla" else 4
+    per_tok = (2 * w.dk + w.dv) * e_in + w.dv * e_in + 4 * gate_elems + beta
     state = 4 * w.dk * w.dv * w.B * w.H
     return w.B * w.T * w.H * per_tok + state * (int(w.with_S0) + int(w.want_S_T))
 
@@ -64,6 +65,8 @@ def algorithmic_flops(w, C=64):
     about 7 d_k d_v per state, CUDA cores)."""
     if w.kind == "step":
         return w.B * w.H * 7.0 * w.dk * w.dv
+    if w.mixer == "gla":  # no correction: state update, S q, masked Q K^T and P V
+        return w.B * w.T * w.H * (4 * w.dk * w.dv + C * (w.dk + w.dv))
     per = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0
     return w.B * w.T * w.H * per
 
@@ -200,6 +203,15 @@ def run_ours(args, rank, world, local_rank):
             binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o,
                               S_T=S_T, output_final_state=S_T is not None, workspace=ws)
 
+        if w.mixer == "gla":  # gated linear attention: one launch, no beta, no workspace
+            host.pop("beta")
+            d.pop("beta")
+            launches_per_step = 1
+
+            def step():
+                binding.chunk_fwd_gla(d["q"], d["k"], d["v"], d["g"], d["S0"], o=o, S_T=S_T,
+                                      output_final_state=S_T is not None)
+
     def barrier():
         if world > 1:
             torch.distributed.barrier()
@@ -317,7 +329,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
-                     "kernel": "gdr_chunk_fwd" if w.kind == "chunk" else "gdr_step"},
+                     "kernel": ("gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
+                     if w.kind == "chunk" else "gdr_step"},
         "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
@@ -330,6 +343,13 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------ oracle arm
+def _oracle_fwd(oracle, w, a, n):
+    """The oracle's forward for the workload's mixer; a = q, k, v, g, beta, S0."""
+    if w.mixer == "gla":
+        return oracle.gla_fwd(a[0], a[1], a[2], a[3], a[5], gate=w.gate, nthreads=n)
+    return oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)
+
+
 def cpu_baseline(w, target_s=12.0):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload:
     all B*H heads over the first T' tokens, T' grown until a run takes a few
@@ -348,7 +368,7 @@ def cpu_baseline(w, target_s=12.0):
                 sl["g"].numpy(), sl["beta"].numpy(),
                 None if sl["S0"] is None else sl["S0"].double().numpy()]
         t = time.perf_counter()
-        oracle.gdr_fwd(*args, gate=w.gate, nthreads=n)
+        _oracle_fwd(oracle, w, args, n)
         el = time.perf_counter() - t
         if el >= target_s / 4 or Tp >= w.T:
             break
@@ -376,10 +396,10 @@ def run_reference(args, rank, world):
          sl["g"].numpy(), sl["beta"].numpy(),
          None if sl["S0"] is None else sl["S0"].double().numpy()]
     for _ in range(args.warmup):
-        oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)
+        _oracle_fwd(oracle, w, a, n)
     t = time.perf_counter()
     for _ in range(args.steps):
-        oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)
+        _oracle_fwd(oracle, w, a, n)
     el = time.perf_counter() - t
     val = w.B * Tp * args.steps / el
     sample = (f"all {w.B}x{w.H} (b,h) pairs, first {Tp} of {w.T} tokens per step "

@@ -30,6 +30,7 @@ EXPORTS = (
     "gdr_chunk_fwd",
     "gdr_chunk_fwd_segmented",
     "gdr_chunk_fwd_varlen",
+    "gdr_chunk_fwd_gla",
     "gdr_step",
     "gdr_get_device_status",
     "gdr_status_string",
@@ -69,6 +70,9 @@ def lib():
             L.gdr_chunk_fwd_varlen.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, i, i, i,
                                                i, i, i, vp]
             L.gdr_chunk_fwd_varlen.restype = i
+            L.gdr_chunk_fwd_gla.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, i, i,
+                                            vp]
+            L.gdr_chunk_fwd_gla.restype = i
             L.gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp]
             L.gdr_step.restype = i
             L.gdr_get_device_status.argtypes = [vp]
@@ -300,5 +304,41 @@ def chunk_fwd_varlen(q, k, v, g, beta, cu_seqlens, S0=None, *, output_final_stat
         rc = lib().gdr_chunk_fwd_varlen(
             _ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk, _ptr(beta), _ptr(cu_seqlens),
             _ptr(S0), _ptr(o), _ptr(S_T), N, total, H, dk, dv, C, _stream_handle(stream))
+    _check(rc)
+    return o, S_T
+
+
+def chunk_fwd_gla(q, k, v, g, S0=None, *, output_final_state=True, o=None, S_T=None, C=64,
+                  stream=None):
+    """``gdr_chunk_fwd_gla``: gated linear attention, S_t = S_{t-1} Diag(alpha_t)
+    + v_t k_t^T, o_t = S_t q_t (no beta).  q, k [B,T,H,dk]; v [B,T,H,dv] (bf16);
+    g [B,T,H] or [B,T,H,dk] fp32 log alpha; S0 [B,H,dv,dk] fp32 or None.
+    Returns (o, S_T or None)."""
+    _need(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (B, T, H, dk), dev)
+    _need(v, "v", dt, (B, T, H, dv), dev)
+    if g.dim() == 4:
+        _need(g, "g", torch.float32, (B, T, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (B, T, H), dev)
+        gk = GDR_GATE_SCALAR
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _need(o, "o", dt, (B, T, H, dv), dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_chunk_fwd_gla(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk,
+                                     _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, C,
+                                     _stream_handle(stream))
     _check(rc)
     return o, S_T

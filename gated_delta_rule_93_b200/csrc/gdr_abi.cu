@@ -139,10 +139,11 @@ namespace {
 
 // Checks shared by the chunked-forward entry points (everything but the
 // workspace); fills the kernel arguments.  Returns GDR_OK or the error.
+// (need_beta = false: beta is not read and may be null)
 gdr_status check_chunk(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                        const float *g, gdr_gate_kind gate, const float *beta, const float *S0,
                        void *o, float *S_T, int B, int T, int H, int dk, int dv, int C,
-                       gdr::ChunkArgs *out) {
+                       gdr::ChunkArgs *out, bool need_beta = true) {
   if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "negative B/T/H");
   if (in_dtype != GDR_F32 && in_dtype != GDR_BF16)
     return fail(GDR_ERR_INVALID_ARG, "in_dtype must be GDR_F32 or GDR_BF16");
@@ -155,10 +156,10 @@ gdr_status check_chunk(const void *q, const void *k, const void *v, gdr_dtype in
     return fail(GDR_ERR_INVALID_ARG, "problem too large");
   const bool empty_tokens = (size_t)B * H * T == 0;
   if (!empty_tokens) {
-    if (!q || !k || !v || !g || !beta || !o)
-      return fail(GDR_ERR_INVALID_ARG, "null q/k/v/g/beta/o");
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(beta) ||
-        !aligned16(o))
+    if (!q || !k || !v || !g || (need_beta && !beta) || !o)
+      return fail(GDR_ERR_INVALID_ARG, need_beta ? "null q/k/v/g/beta/o" : "null q/k/v/g/o");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) ||
+        (need_beta && !aligned16(beta)) || !aligned16(o))
       return fail(GDR_ERR_INVALID_ARG, "q/k/v/g/beta/o must be 16-byte aligned");
   }
   if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
@@ -260,6 +261,34 @@ gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr
   a.B = N;
   a.cu_seqlens = cu_seqlens;
   return from_cuda(gdr::launch_chunk_tc(a, s), "gdr_chunk_fwd_varlen launch");
+}
+
+gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                             const float *g, gdr_gate_kind gate, const float *S0, void *o,
+                             float *S_T, int B, int T, int H, int dk, int dv, int C,
+                             gdr_stream_t stream) {
+  gdr::ChunkArgs a;
+  gdr_status st = check_chunk(q, k, v, in_dtype, g, gate, nullptr, S0, o, S_T, B, T, H, dk, dv,
+                              C, &a, false);
+  if (st != GDR_OK) return st;
+  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128)
+    return fail(GDR_ERR_UNSUPPORTED, "gated linear attention needs bf16 inputs and dk = dv = 128");
+  if ((size_t)B * H == 0) return ok();
+  if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "B*H too large");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = status_word(&a.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd_gla status word");
+  if (T == 0) {  // no tokens: S_T = S0 (or 0)
+    const size_t bytes = (size_t)B * H * dv * dk * sizeof(float);
+    if (S_T && S0 && S_T != S0)
+      e = cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s);
+    else if (S_T && !S0)
+      e = cudaMemsetAsync(S_T, 0, bytes, s);
+    return from_cuda(e, "gdr_chunk_fwd_gla copy");
+  }
+  a.beta = nullptr;
+  a.additive = 1;
+  return from_cuda(gdr::launch_chunk_tc(a, s), "gdr_chunk_fwd_gla launch");
 }
 
 gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dtype,

@@ -86,8 +86,8 @@ constexpr int kGateGc = 0, kGateEg = 64, kGateIeg = 128, kGateEgl = 192, kGateBe
 // group forms S_b from S_tmem unscaled; T' and the O epilogue carry sigma).
 constexpr int kGateSEg = 320;
 // The state group's copy per chunk (float offsets): e^{gc}, e^{gc_last - gc};
-// PC adds e^{m}, e^{gc_last - m} and the state's per-column factor.
-constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256, kSvF = 384;
+// PC adds e^{m} and e^{gc_last - m}.
+constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256;
 
 // Per-variant configuration: K/Q stages and the shared-memory layout (byte
 // offsets from a 1024-byte aligned base).  PC (per-channel gates) holds, per
@@ -113,8 +113,8 @@ struct Cfg {
   static constexpr uint32_t AF = VPD + 2 * kTileBytes;                       // fp32 A, D blocks
   static constexpr uint32_t SCR = AF + 64 * LDA * 4;                         // inverse scratch
   static constexpr uint32_t GS = SCR + (512 + 4 * 256) * 4;                  // gate vectors
-  static constexpr uint32_t SVEC = GS + kStages * kGateBytes;                // x2 (state group)
-  static constexpr uint32_t BAR = SVEC + 2 * kSvecBytes;                     // mbarriers
+  static constexpr uint32_t SVEC = GS + kStages * kGateBytes;                // x3 (state group)
+  static constexpr uint32_t BAR = SVEC + 3 * kSvecBytes;                     // mbarriers
   static constexpr uint32_t MISC = BAR + 32 * 8;                             // tmem base, abort
   static constexpr uint32_t END = MISC + 16;
   static constexpr size_t kSmemBytes = END + 1024;
@@ -669,7 +669,7 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
 
 // Each SM sub-partition holds a quarter of the register file and three of
 // the block's twelve warps: the launch bound caps registers at 168.
-template <bool PC>
+template <bool PC, bool ADD>
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -735,9 +735,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   // T and both T' tiles start at zero: their blocks above the block diagonal
-  // are never written afterwards.
-  for (uint32_t off = 16 * tid; off < (PC ? 2 : 3) * kTileBytes; off += 16 * kThreads)
-    *reinterpret_cast<uint4 *>(sm + Lay::T + off) = make_uint4(0u, 0u, 0u, 0u);
+  // are never written afterwards.  Additive writes (ADD): T = I for good (in
+  // the T tile, or both T' tiles that per-channel gates use for T), so that
+  // the U MMA yields V'^T = V^T.
+  for (uint32_t off = 16 * tid; off < (PC ? 2 : 3) * kTileBytes; off += 16 * kThreads) {
+    uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t tile = off / kTileBytes, row = (off % kTileBytes) / 128;
+    if (ADD && (PC ? tile < 2 : tile == 0) && ((off % 128) / 16 ^ (row & 7)) == row / 8) {
+      // this 16-byte chunk holds columns 8 (row / 8) .. + 7 of its row: the
+      // diagonal element is number row % 8 (bf16 1.0 = 0x3f80)
+      const uint32_t e = row & 7, one = 0x3f80u << (16 * (e & 1));
+      (&z.x)[e >> 1] = one;
+    }
+    *reinterpret_cast<uint4 *>(sm + Lay::T + off) = z;
+  }
   if (PC) {  // per-channel gates: the scalar gate vectors are constants
     for (int i = tid; i < kStages * 256; i += kThreads) {
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + (i >> 8) * kGateBytes);
@@ -805,19 +816,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       last_issued[s] = c;
       float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
       if (PC) {  // beta only; each scaling warp loads its own gate rows
-        const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
-        gv[kGateBeta + lane] = t0 + lane < T ? a.beta[tok] : 0.f;
-        gv[kGateBeta + lane + 32] = t0 + lane + 32 < T ? a.beta[tok + (size_t)32 * H] : 0.f;
+        if (!ADD) {
+          const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
+          gv[kGateBeta + lane] = t0 + lane < T ? a.beta[tok] : 0.f;
+          gv[kGateBeta + lane + 32] = t0 + lane + 32 < T ? a.beta[tok + (size_t)32 * H] : 0.f;
+        }
       } else {
         float gl0 = 0.f, gl1 = 0.f, b0 = 0.f, b1 = 0.f;
         const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
         if (t0 + lane < T) {
           gl0 = a.g[tok];
-          b0 = a.beta[tok];
+          if (!ADD) b0 = a.beta[tok];
         }
         if (t0 + lane + 32 < T) {
           gl1 = a.g[tok + (size_t)32 * H];
-          b1 = a.beta[tok + (size_t)32 * H];
+          if (!ADD) b1 = a.beta[tok + (size_t)32 * H];
         }
         float* gc = gv + kGateGc;
         gc[lane] = gl0;
@@ -949,14 +962,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = c & 1;
         const int st = c % kStages;
         const uint32_t kq = a_kq + st * 4 * kTileBytes;
-        // Z = S_b K^T
+        // Z = S_b K^T  (ADD: no correction, no Z)
         if (!(ok = W(B_SBR, ph) && W(B_FULL + st, (c / kStages) & 1))) break;
+        if (!ADD) {
 #pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tm + TM_Z, tm + TM_SB + 8 * kk,
-                      sdesc_sw128(kq + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32, 16, 1024),
-                      ID_N64, kk > 0);
-        mma_commit(&bars[B_ZF]);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_bf16_ts(tm + TM_Z, tm + TM_SB + 8 * kk,
+                        sdesc_sw128(kq + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32, 16, 1024),
+                        ID_N64, kk > 0);
+          mma_commit(&bars[B_ZF]);
+        }
         // U^T = V^T T^T into the V' accumulator, once T of the chunk is
         // written and V has landed (the previous V' was converted: its VPR
         // wait precedes in this thread).  PC: T is in the T' buffer.
@@ -970,15 +985,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&bars[B_UF]);      // T read: the prep group may write the next T
           mma_commit(&bars[B_VEMPTY]);  // V read
         }
-        // V'^T = U^T + Z (-T')^T, or (-Z) T'^T
-        if (!(ok = W(B_ZR, ph))) break;
-        const uint32_t tp = a_tp + (c & 1) * kTileBytes;
+        // V'^T = U^T + Z (-T')^T, or (-Z) T'^T  (ADD: V'^T = U^T = V^T)
+        if (!ADD) {
+          if (!(ok = W(B_ZR, ph))) break;
+          const uint32_t tp = a_tp + (c & 1) * kTileBytes;
 #pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ts(tm + TM_UV, tm + TM_Z + 8 * kk, sdesc_sw128(tp + kk * 32, 16, 1024), ID_N64,
-                      1);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tm + TM_UV, tm + TM_Z + 8 * kk, sdesc_sw128(tp + kk * 32, 16, 1024),
+                        ID_N64, 1);
+        }
         mma_commit(&bars[B_VPF]);
-        mma_commit(&bars[B_TPE + (c & 1)]);
+        if (!ADD) mma_commit(&bars[B_TPE + (c & 1)]);
         // O_a = S_b Q^T, once the epilogue has read the previous chunk's O.
         // Issued before the SF commit, which then also covers this last read
         // of S_b (the state group overwrites S_b once SF completes).
@@ -1068,13 +1085,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // free (O_b of chunk c - 2), and for the warps writing A (rows 0-63)
       // every strip of the previous chunk done reading AF (TRDY counts all
       // four prep warps; the P warps probe D1 again in its place).
-      const bool a_rows = pt < 64;
+      // (ADD: no A, so no wait on AF)
+      const bool a_rows = !ADD && pt < 64;
       bool bad = !wait_all<4>({&bars[B_FULL + st], &bars[B_D1F], &bars[B_PE + (c & 1)],
                                a_rows ? &bars[B_TRDY] : &bars[B_D1F]},
                               {uint32_t((c / kStages) & 1), ph, uint32_t(((c >> 1) - 1) & 1),
                                a_rows ? uint32_t((c - 1) & 1) : ph},
                               abort_flag);
-      if (!bad) {
+      if (!bad && (!ADD || rl >= 64)) {
         const bool factored = -gcv[63] < kSafeDecay;
         // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns at a time
         tc_fence_after();
@@ -1127,8 +1145,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (rl >= 64) fence_proxy_async_smem();  // P is read by the tensor core
+      }
+      if (!bad) {
         tc_fence_before();
         warp_arrive(&bars[B_D1E]);  // this thread's D1 reads are done
+      }
+      if (ADD) {
+        // T = I throughout: only P is handed on, once U of the previous chunk
+        // has completed (which keeps TRDY within one phase of its waiter).
+        bad = bad || !warp_wait(&bars[B_UF], (c - 1) & 1, abort_flag, lane);
+        if (group_any(kBar, bad)) { ok = false; break; }
+        warp_arrive(&bars[B_TRDY]);
+        continue;
       }
       // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
@@ -1161,10 +1189,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     (void)lrow;
     bool ok = true;
     // Gate factors of chunk c for this group: e^{gc_r} and e^{gc_last - gc_r}
-    // into SVEC[c & 1]; returns the chunk's total decay e^{gc_last}.
+    // into its SVEC slot; returns the chunk's total decay e^{gc_last}.
     // Every warp writes the same values and reads them after its own writes
     // (no group barrier).  A warp cannot run a whole chunk ahead of another:
     // the four-warp barriers it waits for need the other warps' arrivals.
+    // With additive writes it can, however, write chunk c + 2's copy while
+    // another warp still reads chunk c's in its O epilogue (nothing ties V'
+    // of chunk c + 1 to that epilogue; otherwise the Z hand-off of chunk
+    // c + 1 does), hence three slots there, two otherwise.
+    auto svec = [&](int c) {
+      return sm + Lay::SVEC + (ADD ? c % 3 : c & 1) * Lay::kSvecBytes;
+    };
     auto chunk_vectors = [&](int c, float &dl) -> bool {
       const bool got =
           PC ? warp_wait(&bars[B_SCALED + (c & 1)], (c >> 1) & 1, abort_flag, lane)
@@ -1172,7 +1207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!got) return false;
       // The stage can be refilled while this chunk's O epilogue still runs,
       // so the group keeps its own copy of e^{gc} and e^{gc_last - gc}.
-      float *sv = reinterpret_cast<float *>(sm + Lay::SVEC + (c & 1) * Lay::kSvecBytes);
+      float *sv = reinterpret_cast<float *>(svec(c));
       const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * kGateBytes);
       constexpr int kEg = PC ? kGateEg : kGateSEg;  // O epilogue: sigma e^{gc}
       sv[kSvEg + lane] = gv[kEg + lane];
@@ -1181,37 +1216,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         sv[kSvEgl + lane] = gv[kGateEgl + lane];
         sv[kSvEgl + lane + 32] = gv[kGateEgl + lane + 32];
       }
-      if (PC) {  // per-column factors; the previous chunk's copy is in the other slot
-        const float *pv =
-            reinterpret_cast<const float *>(sm + Lay::SVEC + ((c + 1) & 1) * Lay::kSvecBytes);
+      if (PC) {  // per-column factors (the previous chunk's stay in the other slot)
 #pragma unroll
         for (int k = lane; k < 128; k += 32) {
-          const float em = gv[kGateEm + k];
-          sv[kSvEm + k] = em;
+          sv[kSvEm + k] = gv[kGateEm + k];
           sv[kSvEgm + k] = gv[kGateEgm + k];
-          // S_tmem after chunk c - 1's update -> S Diag(e^{m_c}) for chunk c
-          sv[kSvF + k] = c == 0 ? em : pv[kSvEgm + k] * em;
         }
       }
       __syncwarp();
       dl = gv[kGateEg + 63];
       return true;
     };
-    // PC: S_tmem <- S_tmem Diag(f) and S_b = bf16 of the result (f: per-column
-    // factors, broadcast from shared memory).
-    auto pass_vec = [&](const float *fv) {
+    // PC: S_tmem <- S_tmem Diag(f1) Diag(f2) and S_b = bf16 of the result
+    // (per-column factors, broadcast from shared memory).  f1 = e^{gc_last - m}
+    // of the chunk just done takes S_tmem to the true state, f2 = e^{m} of the
+    // next chunk to its frame; the two are applied one after the other because
+    // their product can underflow where neither frame does.
+    auto pass_vec = [&](const float *fv, const float *fv2) {
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float x[32];
         tmem_ld32(lane_base + TM_S + 32 * q, x);
         const float4 *f4 = reinterpret_cast<const float4 *>(fv + 32 * q);
+        const float4 *g4 = reinterpret_cast<const float4 *>(fv2 + 32 * q);
 #pragma unroll
         for (int s4 = 0; s4 < 8; ++s4) {
-          const float4 f = f4[s4];
-          x[4 * s4] *= f.x;
-          x[4 * s4 + 1] *= f.y;
-          x[4 * s4 + 2] *= f.z;
-          x[4 * s4 + 3] *= f.w;
+          const float4 f = f4[s4], f2 = g4[s4];
+          x[4 * s4] = x[4 * s4] * f.x * f2.x;
+          x[4 * s4 + 1] = x[4 * s4 + 1] * f.y * f2.y;
+          x[4 * s4 + 2] = x[4 * s4 + 2] * f.z * f2.z;
+          x[4 * s4 + 3] = x[4 * s4 + 3] * f.w * f2.w;
         }
         uint32_t u[16];
 #pragma unroll
@@ -1286,7 +1320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int e = 0; e < 32; ++e) x[e] = (32 * q + e == i) ? one : 0.f;
           }
           if (PC) {  // S Diag(e^{m_0})
-            const float *fv = reinterpret_cast<const float *>(sm + Lay::SVEC) + kSvF + 32 * q;
+            const float *fv = reinterpret_cast<const float *>(sm + Lay::SVEC) + kSvEm + 32 * q;
 #pragma unroll
             for (int e = 0; e < 32; ++e) x[e] *= fv[e];
           }
@@ -1311,10 +1345,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int c = 0; ok && c < n; ++c) {
       const uint32_t ph = c & 1;
-      const float *sv = reinterpret_cast<const float *>(sm + Lay::SVEC + (c & 1) * Lay::kSvecBytes);
+      const float *sv = reinterpret_cast<const float *>(svec(c));
       const float *egv = sv + kSvEg, *eglv = sv + kSvEgl;
       // ---- Z (scalar gates: T' is stored negated) or -Z (per-channel gates,
       //      whose T' buffer is T itself) -> bf16 A operand, in place in TMEM
+      if (!ADD) {
       if (!warp_wait(&bars[B_ZF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
@@ -1337,6 +1372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       warp_arrive(&bars[B_ZR]);
+      }
       // ---- V'^T -> bf16 operands (plain, and decayed to the chunk end / sigma)
       if (!warp_wait(&bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
@@ -1378,9 +1414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #endif
         if (PC) {
-          pass_vec(reinterpret_cast<const float *>(sm + Lay::SVEC +
-                                                   ((c + 1) & 1) * Lay::kSvecBytes) +
-                   kSvF);
+          pass_vec(sv + kSvEgm, reinterpret_cast<const float *>(svec(c + 1)) + kSvEm);
         } else {
           const float nxt = sig * dl;
           const bool fold = !(nxt >= kScaleFloor);  // also when dl underflows to 0
@@ -1391,7 +1425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float inv = 1.f / sig;
           const float *gn = reinterpret_cast<const float *>(sm + Lay::GS +
                                                             ((c + 1) % kStages) * kGateBytes);
-          float *svn = reinterpret_cast<float *>(sm + Lay::SVEC + ((c + 1) & 1) * Lay::kSvecBytes);
+          float *svn = reinterpret_cast<float *>(svec(c + 1));
           svn[kSvEgl + lane] = gn[kGateEgl + lane] * inv;
           svn[kSvEgl + lane + 32] = gn[kGateEgl + lane + 32] * inv;
           __syncwarp();
@@ -1557,17 +1591,25 @@ bool make_map_gate(CUtensorMap *m, const float *base, int B, int T, int H, int d
   return r == CUDA_SUCCESS;
 }
 
-template <bool PC>
+template <bool PC, bool ADD>
 cudaError_t launch_variant(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                            const CUtensorMap &mv, const CUtensorMap &mg, const CUtensorMap &mo,
                            cudaStream_t stream) {
   constexpr size_t smem = Cfg<PC>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC>,
+  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC, ADD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gdr_chunk_tc_kernel<PC>
+  gdr_chunk_tc_kernel<PC, ADD>
       <<<(unsigned)((size_t)a.B * a.H), kThreads, smem, stream>>>(mq, mk, mv, mg, mo, a);
   return cudaGetLastError();
+}
+
+template <bool PC>
+cudaError_t launch_pc(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                      const CUtensorMap &mv, const CUtensorMap &mg, const CUtensorMap &mo,
+                      cudaStream_t stream) {
+  return a.additive ? launch_variant<PC, true>(a, mq, mk, mv, mg, mo, stream)
+                    : launch_variant<PC, false>(a, mq, mk, mv, mg, mo, stream);
 }
 
 }  // namespace
@@ -1589,9 +1631,9 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
     return cudaErrorInvalidValue;
   if (a.per_channel) {
     if (!make_map_gate(&mg, a.g, mb, a.T, a.H, DK)) return cudaErrorInvalidValue;
-    return launch_variant<true>(a, mq, mk, mv, mg, mo, stream);
+    return launch_pc<true>(a, mq, mk, mv, mg, mo, stream);
   }
-  return launch_variant<false>(a, mq, mk, mv, mq, mo, stream);  // gate map unused
+  return launch_pc<false>(a, mq, mk, mv, mq, mo, stream);  // gate map unused
 }
 
 }  // namespace gdr

@@ -34,6 +34,9 @@ struct ChunkArgs {
   // tokens [cu_seqlens[b], cu_seqlens[b + 1]) of the [1, T, H, d] tensors
   // (device int32 [B + 1]); null: dense [B, T, H, d].
   const int *cu_seqlens;
+  // Additive writes (tensor-core kernel only): 1 runs gated linear attention,
+  // S_t = S_{t-1} Diag(alpha_t) + v_t k_t^T, with beta unused (may be null).
+  int additive;
 };
 
 struct StepArgs {

@@ -40,6 +40,7 @@ class Workload:
     want_S_T: bool
     steps: int = 1  # decode workloads: consecutive steps
     C: int = 64
+    mixer: str = "gdr"  # "gdr" (delta rule) or "gla" (gated linear attention, beta unused)
     note: str = field(default="", compare=False)
 
     @property
@@ -47,7 +48,7 @@ class Workload:
         return self.B * self.T if self.kind == "chunk" else self.B * self.steps
 
 
-# The five workloads, named by what they are.
+# The workloads, named by what they are.
 WORKLOADS = {
     w.name: w
     for w in [
@@ -62,6 +63,9 @@ WORKLOADS = {
         Workload("decode_n256_h16_d128_x1024", "step", 256, 1, 16, 128, 128, torch.bfloat16,
                  "scalar", True, True, steps=1024,
                  note="recurrent decode step, 256 sequences, 1024 consecutive steps"),
+        Workload("gla_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
+                 "scalar", False, True, mixer="gla",
+                 note="gated linear attention forward at the same shape (additive writes)"),
     ]
 }
 

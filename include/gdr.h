@@ -169,6 +169,31 @@ gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr
                                 gdr_stream_t stream);
 
 /*
+ * Chunked forward of gated linear attention, the delta rule's additive
+ * sibling: "Decoding Hybrid Linear Attention Architectures", section 3 item
+ * 4, and "Linear Attention Variants", gated linear attention:
+ *
+ *   S_t = S_{t-1} Diag(alpha_t) + v_t k_t^T,   o_t = S_t q_t,
+ *
+ * alpha_t = e^{g_t} (one value per head, or one per key channel), with no
+ * erase term and no beta.  Computed chunkwise as gdr_chunk_fwd with the
+ * correction W S dropped (T = I).
+ *
+ *   q, k   [B, T, H, dk] bf16;  v, o [B, T, H, dv] bf16
+ *   g      [B, T, H] fp32 (scalar gate) or [B, T, H, dk] (per channel)
+ *   S0     [B, H, dv, dk] fp32 or NULL (zero state); may alias S_T
+ *   S_T    [B, H, dv, dk] fp32 or NULL (not written)
+ *
+ * Needs dk = dv = 128, C = 64 and bf16 inputs (GDR_ERR_UNSUPPORTED
+ * otherwise).  T = 0 copies S0 (or zeros) to S_T.  One launch on `stream`,
+ * no workspace; o must not alias an input.
+ */
+gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                             const float *g, gdr_gate_kind gate, const float *S0, void *o,
+                             float *S_T, int B, int T, int H, int dk, int dv, int C,
+                             gdr_stream_t stream);
+
+/*
  * One recurrent decode step for N independent states, S updated in place.
  * Source: "Decoding Hybrid Linear Attention Architectures", section 6
  * (constant-cost update of the fixed-size state per decoded token) with the

@@ -154,3 +154,26 @@ def test_varlen_validation_rejects_before_any_launch(L):
     assert call(q=None) == binding.GDR_ERR_INVALID_ARG
     assert call(o=_fake_ptr(2)) == binding.GDR_ERR_INVALID_ARG
     assert call(N=0) == binding.GDR_OK
+
+
+def test_gla_validation_rejects_before_any_launch(L):
+    """gdr_chunk_fwd_gla: no beta; tensor-core shapes only."""
+    p = _fake_ptr()
+
+    def call(**kw):
+        a = dict(q=p, k=p, v=p, dt=1, g=p, gate=0, S0=None, o=p, ST=None, B=2, T=300, H=2,
+                 dk=128, dv=128, C=64, st=None)
+        a.update(kw)
+        return L.gdr_chunk_fwd_gla(a["q"], a["k"], a["v"], a["dt"], a["g"], a["gate"], a["S0"],
+                                   a["o"], a["ST"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                   a["C"], a["st"])
+
+    assert call(B=-1) == binding.GDR_ERR_INVALID_ARG
+    assert call(gate=7) == binding.GDR_ERR_INVALID_ARG
+    assert call(dt=0) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dk=64, dv=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(C=32) == binding.GDR_ERR_UNSUPPORTED
+    assert call(q=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(g=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(o=_fake_ptr(2)) == binding.GDR_ERR_INVALID_ARG
+    assert call(H=0) == binding.GDR_OK

@@ -98,6 +98,21 @@ def test_strong_scalar_forgetting_has_no_nan(cuda_device, dtype):
     assert_close(S_T, rS, TOL[dtype], "S_T")
 
 
+def test_strong_per_channel_decay_tensor_cores(cuda_device):
+    """Per-channel gates 20x the usual recipe (alpha ~ 0.2 per token): the
+    log decay over a 32-token half chunk reaches about -72 in some channel.
+    The operand factors e^{gc - m} stay inside bf16's range there, and the
+    state's change of frame between chunks is applied as two factors (their
+    product would underflow fp32)."""
+    inp = make_chunk_inputs(1, 512, 2, 128, 128, torch.bfloat16, "channel", True, seed=77)
+    inp["g"] = inp["g"] * 20.0
+    o, S_T = gpu_chunk(inp, cuda_device)
+    assert binding.device_status() == 0
+    ro, rS = oracle_chunk(inp)
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S_T, rS, 2e-2, "S_T")
+
+
 def test_beta_zero_is_pure_decay(cuda_device):
     """beta = 0: no write, so S_T = S0 Diag(exp(sum g)) (closed form)."""
     inp = make_chunk_inputs(1, 160, 2, 64, 32, torch.float32, "channel", True, seed=6)
