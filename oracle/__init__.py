@@ -20,6 +20,9 @@ Contents
     loop in ``gdr_oracle.c`` ("Decoding Hybrid Linear Attention
     Architectures", section 3 item 4; "Linear Attention Variants", GLA
     section).
+``gdr_fwd_f64`` / ``gdr_fwd_prologue``
+    The same recurrence on fp64 inputs, and on the output of ``prologue``
+    (raw q, k L2-normalised, beta = sigmoid(b), g = -s_h softplus(a)).
 ``chunked``
     A staged fp64 NumPy restatement of the chunkwise algorithm ("Decoding
     Hybrid Linear Attention Architectures", section 5, inter-chunk recursion
@@ -74,6 +77,9 @@ def _load():
             lib.oracle_gdr_step.restype = i
             lib.oracle_gla_fwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, i, i]
             lib.oracle_gla_fwd.restype = i
+            lib.oracle_gdr_fwd_f64.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp, i, i, i, i, i,
+                                               i]
+            lib.oracle_gdr_fwd_f64.restype = i
             _lib = lib
     return _lib
 
@@ -202,3 +208,40 @@ def gdr_step(q, k, v, g, beta, S, gate="scalar", nthreads=None):
     if rc != 0:
         raise ValueError("oracle_gdr_step rejected its arguments")
     return o
+
+
+def gdr_fwd_f64(q, k, v, g, beta, S0=None, gate="scalar", nthreads=None):
+    """``gdr_fwd`` with every input in float64 (same shapes)."""
+    q, k, v, g, beta = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != (B, T, H, dk) or v.shape != (B, T, H, dv):
+        raise ValueError("shape mismatch among q, k, v")
+    gk = GATE_PER_CHANNEL if gate in ("channel", "per_channel", GATE_PER_CHANNEL) else GATE_SCALAR
+    want_g = (B, T, H, dk) if gk == GATE_PER_CHANNEL else (B, T, H)
+    if g.shape != want_g or beta.shape != (B, T, H):
+        raise ValueError("g / beta shape mismatch")
+    S0d = None
+    if S0 is not None:
+        S0d = np.ascontiguousarray(S0, dtype=np.float64)
+        if S0d.shape != (B, H, dv, dk):
+            raise ValueError("S0 must be [B,H,dv,dk]")
+    o = np.zeros((B, T, H, dv), np.float64)
+    S_T = np.zeros((B, H, dv, dk), np.float64)
+    n = nthreads or default_threads()
+    rc = _load().oracle_gdr_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(g), gk, _ptr(beta),
+                                    _ptr(S0d), _ptr(o), _ptr(S_T), B, T, H, dk, dv, n)
+    if rc != 0:
+        raise ValueError("oracle_gdr_fwd_f64 rejected its arguments")
+    return o, S_T
+
+
+def gdr_fwd_prologue(q_raw, k_raw, v, a, b, gate_scale, S0=None, gate="scalar", norm_q=True,
+                     norm_k=True, nthreads=None):
+    """The forward from raw projections: ``prologue.prologue`` then
+    ``gdr_fwd_f64``.  q_raw, k_raw, v fp32 or uint16 (bf16 bits); a [B,T,H]
+    or [B,T,H,dk] and b [B,T,H] fp32 logits; gate_scale [H] > 0."""
+    from . import prologue as _pro
+
+    q, k, g, beta = _pro.prologue(q_raw, k_raw, a, b, gate_scale, norm_q, norm_k)
+    return gdr_fwd_f64(q, k, _pro.widen(v), g, beta, S0, gate=gate, nthreads=nthreads)

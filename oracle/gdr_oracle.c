@@ -40,11 +40,12 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { OR_F32 = 0, OR_BF16 = 1 };
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F64 = 2 };
 enum { OR_GATE_SCALAR = 0, OR_GATE_PER_CHANNEL = 1 };
 
 /* Exact widening of one input element to double. */
 static double load_elem(const void *base, size_t idx, int dtype) {
+    if (dtype == OR_F64) return ((const double *)base)[idx];
     if (dtype == OR_F32) return (double)((const float *)base)[idx];
     uint32_t bits = ((uint32_t)((const uint16_t *)base)[idx]) << 16;
     float f;
@@ -58,6 +59,7 @@ typedef struct {
     const float *g;
     int gate_kind;
     const float *beta;
+    const double *g64, *beta64; /* fp64 gates (take the place of g, beta when set) */
     const double *S0; /* may be NULL: zero initial state */
     double *o;
     double *S_T;      /* may be NULL */
@@ -65,6 +67,10 @@ typedef struct {
     int next;         /* shared work counter over (b, h) */
     pthread_mutex_t lock;
 } job_t;
+
+static double gate_at(const job_t *J, size_t idx) {
+    return J->g64 ? J->g64[idx] : (double)J->g[idx];
+}
 
 /*
  * One (b, h) pair: the recurrence over t = 0..T-1.
@@ -91,12 +97,12 @@ static void run_head(job_t *J, int b, int h) {
             qq[j] = load_elem(J->q, tok * dk + j, J->in_dtype);
         }
         if (J->gate_kind == OR_GATE_PER_CHANNEL) {
-            for (int j = 0; j < dk; ++j) alpha[j] = exp((double)J->g[tok * dk + j]);
+            for (int j = 0; j < dk; ++j) alpha[j] = exp(gate_at(J, tok * dk + j));
         } else {
-            const double a = exp((double)J->g[tok]);
+            const double a = exp(gate_at(J, tok));
             for (int j = 0; j < dk; ++j) alpha[j] = a;
         }
-        const double beta = (double)J->beta[tok];
+        const double beta = J->beta64 ? J->beta64[tok] : (double)J->beta[tok];
 
         /* 1. decay: S <- S Diag(alpha)  (scales the key axis) */
         for (int i = 0; i < dv; ++i)
@@ -147,6 +153,8 @@ static void *worker(void *arg) {
  * Forward over a whole sequence.  Returns 0 on success, -1 on a bad
  * argument.  nthreads <= 0 means one thread per online core.
  */
+static int run_job(job_t *Jp, int nthreads);
+
 int oracle_gdr_fwd(const void *q, const void *k, const void *v, int in_dtype,
                    const float *g, int gate_kind, const float *beta,
                    const double *S0, double *o, double *S_T, int B, int T,
@@ -158,8 +166,37 @@ int oracle_gdr_fwd(const void *q, const void *k, const void *v, int in_dtype,
     job_t J;
     J.q = q; J.k = k; J.v = v; J.in_dtype = in_dtype;
     J.g = g; J.gate_kind = gate_kind; J.beta = beta;
+    J.g64 = NULL; J.beta64 = NULL;
     J.S0 = S0; J.o = o; J.S_T = S_T;
     J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+    return run_job(&J, nthreads);
+}
+
+/*
+ * The same forward with every input in fp64 (q, k, v, g = log alpha, beta):
+ * for inputs that are themselves computed in fp64, such as the output of the
+ * prologue (normalised q, k and gates mapped from their logits).
+ */
+int oracle_gdr_fwd_f64(const double *q, const double *k, const double *v,
+                       const double *g, int gate_kind, const double *beta,
+                       const double *S0, double *o, double *S_T, int B, int T,
+                       int H, int dk, int dv, int nthreads) {
+    if (!q || !k || !v || !g || !beta || !o) return -1;
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (gate_kind != OR_GATE_SCALAR && gate_kind != OR_GATE_PER_CHANNEL) return -1;
+    job_t J;
+    J.q = q; J.k = k; J.v = v; J.in_dtype = OR_F64;
+    J.g = NULL; J.gate_kind = gate_kind; J.beta = NULL;
+    J.g64 = g; J.beta64 = beta;
+    J.S0 = S0; J.o = o; J.S_T = S_T;
+    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+    return run_job(&J, nthreads);
+}
+
+/* Runs every (b, h) of the job on nthreads threads (<= 0: one). */
+static int run_job(job_t *Jp, int nthreads) {
+    job_t J = *Jp;
+    const int B = J.B, H = J.H;
     J.next = 0;
     pthread_mutex_init(&J.lock, NULL);
     int n = nthreads;
