@@ -203,6 +203,14 @@ def run_ours(args, rank, world, local_rank):
             binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o,
                               S_T=S_T, output_final_state=S_T is not None, workspace=ws)
 
+        if w.prologue:  # raw projections in: one launch, no workspace
+            launches_per_step = 1
+
+            def step():
+                binding.chunk_fwd_prologue(d["q"], d["k"], d["v"], d["a"], d["b"],
+                                           d["gate_scale"], d["S0"], o=o, S_T=S_T,
+                                           output_final_state=S_T is not None)
+
         if w.mixer == "gla":  # gated linear attention: one launch, no beta, no workspace
             host.pop("beta")
             d.pop("beta")
@@ -329,7 +337,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
-                     "kernel": ("gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
+                     "kernel": ("gdr_chunk_fwd_prologue" if w.prologue else
+                                "gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
                      if w.kind == "chunk" else "gdr_step"},
         "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -343,8 +352,23 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------ oracle arm
+def _oracle_sample(w, inp, Tp):
+    """The oracle's arguments for the first Tp tokens of every (b, h)."""
+    from gated_delta_rule_93_b200.inputs import to_numpy_input
+
+    sl = {k: (v[:, :Tp].contiguous() if (v is not None and k not in ("S0", "gate_scale"))
+              else v) for k, v in inp.items()}
+    S0 = None if sl["S0"] is None else sl["S0"].double().numpy()
+    qkv = [to_numpy_input(sl["q"]), to_numpy_input(sl["k"]), to_numpy_input(sl["v"])]
+    if w.prologue:
+        return qkv + [sl["a"].numpy(), sl["b"].numpy(), sl["gate_scale"].numpy(), S0]
+    return qkv + [sl["g"].numpy(), sl["beta"].numpy(), S0]
+
+
 def _oracle_fwd(oracle, w, a, n):
-    """The oracle's forward for the workload's mixer; a = q, k, v, g, beta, S0."""
+    """The oracle's forward for the workload (arguments from _oracle_sample)."""
+    if w.prologue:
+        return oracle.gdr_fwd_prologue(*a, gate=w.gate, nthreads=n)
     if w.mixer == "gla":
         return oracle.gla_fwd(a[0], a[1], a[2], a[3], a[5], gate=w.gate, nthreads=n)
     return oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)
@@ -362,11 +386,7 @@ def cpu_baseline(w, target_s=12.0):
     n = min(oracle.default_threads(), w.B * w.H)
     Tp = 16
     while True:
-        sl = {k: (v[:, :Tp].contiguous() if (v is not None and k != "S0") else v)
-              for k, v in inp.items()}
-        args = [to_numpy_input(sl["q"]), to_numpy_input(sl["k"]), to_numpy_input(sl["v"]),
-                sl["g"].numpy(), sl["beta"].numpy(),
-                None if sl["S0"] is None else sl["S0"].double().numpy()]
+        args = _oracle_sample(w, inp, Tp)
         t = time.perf_counter()
         _oracle_fwd(oracle, w, args, n)
         el = time.perf_counter() - t
@@ -390,11 +410,7 @@ def run_reference(args, rank, world):
     n = min(oracle.default_threads(), w.B * w.H)
     # bounded per-step sample: first Tp tokens of every (b, h)
     Tp = max(1, min(w.T, args.ref_tokens))
-    sl = {k: (v[:, :Tp].contiguous() if (v is not None and k != "S0") else v)
-          for k, v in inp.items()}
-    a = [to_numpy_input(sl["q"]), to_numpy_input(sl["k"]), to_numpy_input(sl["v"]),
-         sl["g"].numpy(), sl["beta"].numpy(),
-         None if sl["S0"] is None else sl["S0"].double().numpy()]
+    a = _oracle_sample(w, inp, Tp)
     for _ in range(args.warmup):
         _oracle_fwd(oracle, w, a, n)
     t = time.perf_counter()

@@ -8,6 +8,7 @@ from .binding import (  # noqa: F401
     GdrError,
     chunk_fwd,
     chunk_fwd_gla,
+    chunk_fwd_prologue,
     chunk_fwd_kernel_launches,
     chunk_fwd_segmented,
     chunk_fwd_varlen,
@@ -18,6 +19,6 @@ from .binding import (  # noqa: F401
     step,
 )
 
-__all__ = ["chunk_fwd", "chunk_fwd_gla", "chunk_fwd_kernel_launches", "chunk_fwd_segmented", "chunk_fwd_varlen",
+__all__ = ["chunk_fwd", "chunk_fwd_gla", "chunk_fwd_prologue", "chunk_fwd_kernel_launches", "chunk_fwd_segmented", "chunk_fwd_varlen",
            "chunk_fwd_workspace_bytes", "step", "device_status", "lib", "status_string",
            "GdrError"]

@@ -31,6 +31,7 @@ EXPORTS = (
     "gdr_chunk_fwd_segmented",
     "gdr_chunk_fwd_varlen",
     "gdr_chunk_fwd_gla",
+    "gdr_chunk_fwd_prologue",
     "gdr_step",
     "gdr_get_device_status",
     "gdr_status_string",
@@ -73,6 +74,9 @@ def lib():
             L.gdr_chunk_fwd_gla.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, i, i,
                                             vp]
             L.gdr_chunk_fwd_gla.restype = i
+            L.gdr_chunk_fwd_prologue.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, i, i,
+                                                 i, i, i, i, i, vp]
+            L.gdr_chunk_fwd_prologue.restype = i
             L.gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp]
             L.gdr_step.restype = i
             L.gdr_get_device_status.argtypes = [vp]
@@ -340,5 +344,42 @@ def chunk_fwd_gla(q, k, v, g, S0=None, *, output_final_state=True, o=None, S_T=N
         rc = lib().gdr_chunk_fwd_gla(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk,
                                      _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, C,
                                      _stream_handle(stream))
+    _check(rc)
+    return o, S_T
+
+
+def chunk_fwd_prologue(q, k, v, a, b, gate_scale, S0=None, *, norm_q=True, norm_k=True,
+                       output_final_state=True, o=None, S_T=None, C=64, stream=None):
+    """``gdr_chunk_fwd_prologue``: the chunked forward from raw projections.
+
+    q, k [B,T,H,dk] (raw, bf16); v [B,T,H,dv]; a, b [B,T,H] fp32 gate and
+    beta logits; gate_scale [H] fp32.  In the kernel: q, k L2-normalised (per
+    the flags), beta = sigmoid(b), g = -gate_scale[h] softplus(a).
+    Returns (o, S_T or None)."""
+    _need(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (B, T, H, dk), dev)
+    _need(v, "v", dt, (B, T, H, dv), dev)
+    _need(a, "a", torch.float32, (B, T, H), dev)
+    _need(b, "b", torch.float32, (B, T, H), dev)
+    _need(gate_scale, "gate_scale", torch.float32, (H,), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _need(o, "o", dt, (B, T, H, dv), dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
+    flags = (1 if norm_q else 0) | (2 if norm_k else 0)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_chunk_fwd_prologue(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(a),
+                                          GDR_GATE_SCALAR, _ptr(gate_scale), _ptr(b), _ptr(S0),
+                                          _ptr(o), _ptr(S_T), B, T, H, dk, dv, C, flags,
+                                          _stream_handle(stream))
     _check(rc)
     return o, S_T

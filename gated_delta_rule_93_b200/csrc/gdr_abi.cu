@@ -291,6 +291,41 @@ gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dt
   return from_cuda(gdr::launch_chunk_tc(a, s), "gdr_chunk_fwd_gla launch");
 }
 
+gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
+                                  gdr_dtype in_dtype, const float *a, gdr_gate_kind gate,
+                                  const float *gate_scale, const float *b, const float *S0,
+                                  void *o, float *S_T, int B, int T, int H, int dk, int dv, int C,
+                                  int norm_qk, gdr_stream_t stream) {
+  gdr::ChunkArgs ca;
+  gdr_status st = check_chunk(q, k, v, in_dtype, a, gate, b, S0, o, S_T, B, T, H, dk, dv, C,
+                              &ca);
+  if (st != GDR_OK) return st;
+  if (norm_qk < 0 || norm_qk > 3) return fail(GDR_ERR_INVALID_ARG, "norm_qk must be 0..3");
+  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128 || gate != GDR_GATE_SCALAR)
+    return fail(GDR_ERR_UNSUPPORTED,
+                "the fused prologue needs bf16 inputs, dk = dv = 128 and a scalar gate");
+  if ((size_t)B * H == 0) return ok();
+  if (!gate_scale) return fail(GDR_ERR_INVALID_ARG, "null gate_scale");
+  if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "B*H too large");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = status_word(&ca.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd_prologue status word");
+  if (T == 0) {  // no tokens: S_T = S0 (or 0)
+    const size_t bytes = (size_t)B * H * dv * dk * sizeof(float);
+    if (S_T && S0 && S_T != S0)
+      e = cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s);
+    else if (S_T && !S0)
+      e = cudaMemsetAsync(S_T, 0, bytes, s);
+    return from_cuda(e, "gdr_chunk_fwd_prologue copy");
+  }
+  ca.prologue = 1;
+  ca.norm_qk = norm_qk;
+  ca.gate_scale = gate_scale;
+  ca.skip_stage_chunk = t_skip_stage_chunk;
+  t_skip_stage_chunk = -1;
+  return from_cuda(gdr::launch_chunk_tc(ca, s), "gdr_chunk_fwd_prologue launch");
+}
+
 gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                     const float *g, gdr_gate_kind gate, const float *beta, float *S, void *o,
                     int N, int H, int dk, int dv, gdr_stream_t stream) {

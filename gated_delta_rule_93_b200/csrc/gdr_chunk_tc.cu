@@ -85,6 +85,13 @@ constexpr int kGateGc = 0, kGateEg = 64, kGateIeg = 128, kGateEgl = 192, kGateBe
 // the scale of the bf16 state copy S_b the chunk's MMAs read (the state
 // group forms S_b from S_tmem unscaled; T' and the O epilogue carry sigma).
 constexpr int kGateSEg = 320;
+// Prologue instance only (scalar gates): the tiles hold raw K, Q, and each
+// token's 1 / |k| and 1 / |q| (rk, rq) ride on the per-token vectors instead:
+// once a stage has landed, Ieg and Egl are multiplied by rk in place
+// (columns of A and P, the state update's rows), T' takes sigma e^{gc} rk
+// (SEgK), the O epilogue sigma e^{gc} rq (SEgQ), and the A / P rows take
+// rk / rq from their own vectors.
+constexpr int kGateRk = 384, kGateRq = 448, kGateSEgQ = 512, kGateSEgK = 576;
 // The state group's copy per chunk (float offsets): e^{gc}, e^{gc_last - gc};
 // PC adds e^{m} and e^{gc_last - m}.
 constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256;
@@ -99,7 +106,7 @@ constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256;
 template <bool PC>
 struct Cfg {
   static constexpr int kStages = PC ? 2 : 3;
-  static constexpr uint32_t kGateBytes = (PC ? 576 : 384) * 4;
+  static constexpr uint32_t kGateBytes = (PC ? 576 : 640) * 4;
   static constexpr uint32_t kSvecBytes = (PC ? 512 : 128) * 4;
   static constexpr uint32_t KQ = 0;                                          // [K_h0|Q_h0|K_h1|Q_h1]
   static constexpr uint32_t KH = KQ + kStages * 4 * kTileBytes;              // PC: [Kh_h0|Kh_h1]
@@ -149,6 +156,8 @@ enum {
   B_SCALED,            // [2] PC: scaled K~, Q~, K^ of a stage written  (2 warps)
   B_GF = B_SCALED + 2, // [4] PC: gate rows of a scaling warp landed    (1 + tx)
                        //     (warp w, rows 0-31 / 32-63: 2 w + half)
+  B_NORM = B_GF,       // [3] prologue (scalar gates): token norms of a
+                       //     stage folded into its vectors (prep-side MMA warp)
   B_COUNT = B_GF + 4
 };
 static_assert(B_COUNT <= 32, "barrier slots");
@@ -587,6 +596,105 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// ---- prologue (raw projections in): "Decoding Hybrid Linear Attention
+// Architectures", section 3 item 2 (the erase is a projector along a unit
+// key) and section 4 (beta in (0, 1), alpha in (0, 1]):
+//   q, k <- x / sqrt(|x|^2 + eps),  beta = sigmoid(b),  g = -s_h softplus(a).
+constexpr float kNormEps = 1e-6f;
+
+__device__ __forceinline__ float softplus_f(float x) {
+  return fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+
+// L2-normalise the K rows (nk) and Q rows (nq) of a landed K/Q stage in
+// place, one warp: lane l takes row l and l + 32 of each.  A row's 128
+// channels are its 128-byte row in the h0 tile and in the h1 tile; the sum
+// of squares and the scaling do not depend on the order of the 16-byte
+// chunks, so the swizzle is ignored and each lane starts at chunk l % 8,
+// which puts the 8 lanes of a 16-byte access phase on distinct banks.
+// Rows past the sequence's end were filled with zeros and stay zero.
+__device__ __forceinline__ float sumsq_bf16x8(uint4 x, float ss) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[u]));
+    ss = fmaf(f.x, f.x, ss);
+    ss = fmaf(f.y, f.y, ss);
+  }
+  return ss;
+}
+
+// 1 / sqrt(|x|^2 + eps) of one 128-channel row of a landed K/Q stage: its
+// 128-byte row in the h0 tile (p0) and in the h1 tile (p0 + 2 tiles).  The
+// sum does not depend on the order of the 16-byte chunks, so the swizzle is
+// ignored and lane l starts at chunk l % 8, which puts the 8 lanes of a
+// 16-byte access phase on distinct banks.  Zero rows (past the sequence's
+// end) give a finite factor.
+__device__ __forceinline__ float row_inv_norm(const uint8_t *p0, int lane) {
+  const uint8_t *p1 = p0 + 2 * kTileBytes;
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int ch = ((p + lane) & 7) * 16;
+    s0 = sumsq_bf16x8(*reinterpret_cast<const uint4 *>(p0 + ch), s0);
+    s1 = sumsq_bf16x8(*reinterpret_cast<const uint4 *>(p1 + ch), s1);
+  }
+  return rsqrtf(s0 + s1 + kNormEps);
+}
+
+// Prologue, one warp, once a stage has landed (lane l: tokens l and l + 32):
+// 1 / |k| into Rk and folded into the vectors that meet K (Ieg, Egl in
+// place, SEgK = SEg rk), 1 / |q| into Rq and SEgQ = SEg rq.
+__device__ __forceinline__ void fold_token_norms(const uint8_t *kq, float *gv, int lane, bool nq,
+                                                 bool nk) {
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    const int t = lane + 32 * half;
+    const float rk = nk ? row_inv_norm(kq + t * 128, lane) : 1.f;
+    const float rq = nq ? row_inv_norm(kq + kTileBytes + t * 128, lane) : 1.f;
+    const float seg = gv[kGateSEg + t];
+    gv[kGateRk + t] = rk;
+    gv[kGateRq + t] = rq;
+    gv[kGateSEgK + t] = seg * rk;
+    gv[kGateSEgQ + t] = seg * rq;
+    gv[kGateIeg + t] *= rk;
+    gv[kGateEgl + t] *= rk;
+  }
+}
+
+// Scalar gates of one stage from the per-token log decays (gl0: token lane,
+// gl1: token lane + 32) and betas: the cumulative decay gc, e^{gc}, e^{-gc},
+// e^{gc_last - gc}, beta and sigma e^{gc} into gv; sig advances to the
+// state scale after the chunk (see the state group), replayed in the same
+// fp32 operations.  One warp.
+__device__ __forceinline__ void write_scalar_gates(float *gv, float gl0, float gl1, float b0,
+                                                   float b1, int lane, int c, float &sig) {
+  float *gc = gv + kGateGc;
+  gc[lane] = gl0;
+  gc[lane + 32] = gl1;
+  __syncwarp();
+  float x0, x1;
+  const float gl = chunk_cumsum(gc, lane, x0, x1);
+  __syncwarp();
+  gc[lane] = x0;
+  gc[lane + 32] = x1;
+  gv[kGateEg + lane] = __expf(x0);
+  gv[kGateEg + lane + 32] = __expf(x1);
+  gv[kGateIeg + lane] = __expf(-x0);
+  gv[kGateIeg + lane + 32] = __expf(-x1);
+  gv[kGateEgl + lane] = __expf(gl - x0);
+  gv[kGateEgl + lane + 32] = __expf(gl - x1);
+  gv[kGateBeta + lane] = b0;
+  gv[kGateBeta + lane + 32] = b1;
+  gv[kGateSEg + lane] = sig * __expf(x0);
+  gv[kGateSEg + lane + 32] = sig * __expf(x1);
+  // the scale after this chunk: 1 after chunk 0 (its decay goes into
+  // S_tmem), else sig * decay unless that falls below the floor
+  const float nxt = sig * __expf(gl);  // the decay e^{gc_last} as stored above
+  sig = (c == 0 || !(nxt >= kScaleFloor)) ? 1.f : nxt;
+}
+
 // Per-channel gates, one warp, channels j0 .. j0 + 63 of a chunk (lane l:
 // the adjacent pair j0 + 2 l, j0 + 2 l + 1).  g0 / g1: the warp's gate rows
 // 0-31 / 32-63 of the chunk ([32][64] fp32 log decay; rows from nv on read as
@@ -669,7 +777,7 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
 
 // Each SM sub-partition holds a quarter of the register file and three of
 // the block's twelve warps: the launch bound caps registers at 168.
-template <bool PC, bool ADD>
+template <bool PC, bool ADD, bool PRO>
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -703,6 +811,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Lay::MISC);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + Lay::MISC + 4);
   float *AF = reinterpret_cast<float *>(sm + Lay::AF);
+  // gate vectors of chunk c (one set per K/Q stage)
+  auto gate_slot = [&](int c) {
+    return reinterpret_cast<float *>(sm + Lay::GS + (c % kStages) * kGateBytes);
+  };
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -793,6 +905,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Scalar gates: the state group's scale sequence, replayed with the same
     // fp32 operations: sig = the scale of S_b for the chunk being produced.
     float sig = 1.f;
+    // Scalar gates of chunk j into its stage's vectors (prologue: g and
+    // beta arrive as logits).
+    auto gates = [&](int j) {
+      const int t0 = j * C;
+      float gl0 = 0.f, gl1 = 0.f, b0 = 0.f, b1 = 0.f;
+      const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
+      const float gsc = PRO ? a.gate_scale[h] : 0.f;
+      if (t0 + lane < T) {
+        gl0 = PRO ? -gsc * softplus_f(a.g[tok]) : a.g[tok];
+        if (!ADD) b0 = PRO ? sigmoid_f(a.beta[tok]) : a.beta[tok];
+      }
+      if (t0 + lane + 32 < T) {
+        gl1 = PRO ? -gsc * softplus_f(a.g[tok + (size_t)32 * H]) : a.g[tok + (size_t)32 * H];
+        if (!ADD) {
+          const float bl = a.beta[tok + (size_t)32 * H];
+          b1 = PRO ? sigmoid_f(bl) : bl;
+        }
+      }
+      write_scalar_gates(gate_slot(j), gl0, gl1, b0, b1, lane, j, sig);
+    };
     for (int c = 0; c < n; ++c) {
       const int s = c % kStages;
       if (c >= kStages &&
@@ -814,48 +946,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(kq + 3 * kTileBytes, &tmQ, fb, 64, h, tb + t0, bt);
       }
       last_issued[s] = c;
-      float *gv = reinterpret_cast<float *>(sm + Lay::GS + s * kGateBytes);
-      if (PC) {  // beta only; each scaling warp loads its own gate rows
-        if (!ADD) {
-          const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
-          gv[kGateBeta + lane] = t0 + lane < T ? a.beta[tok] : 0.f;
-          gv[kGateBeta + lane + 32] = t0 + lane + 32 < T ? a.beta[tok + (size_t)32 * H] : 0.f;
-        }
-      } else {
-        float gl0 = 0.f, gl1 = 0.f, b0 = 0.f, b1 = 0.f;
+      float *gv = gate_slot(c);
+      if (PC && !ADD) {  // beta only; each scaling warp loads its own gate rows
         const size_t tok = ((size_t)bt * a.T + tb + t0 + lane) * H + h;
-        if (t0 + lane < T) {
-          gl0 = a.g[tok];
-          if (!ADD) b0 = a.beta[tok];
-        }
-        if (t0 + lane + 32 < T) {
-          gl1 = a.g[tok + (size_t)32 * H];
-          if (!ADD) b1 = a.beta[tok + (size_t)32 * H];
-        }
-        float* gc = gv + kGateGc;
-        gc[lane] = gl0;
-        gc[lane + 32] = gl1;
-        __syncwarp();
-        float x0, x1;
-        const float gl = chunk_cumsum(gc, lane, x0, x1);
-        __syncwarp();
-        gc[lane] = x0;
-        gc[lane + 32] = x1;
-        gv[kGateEg + lane] = __expf(x0);
-        gv[kGateEg + lane + 32] = __expf(x1);
-        gv[kGateIeg + lane] = __expf(-x0);
-        gv[kGateIeg + lane + 32] = __expf(-x1);
-        gv[kGateEgl + lane] = __expf(gl - x0);
-        gv[kGateEgl + lane + 32] = __expf(gl - x1);
-        gv[kGateBeta + lane] = b0;
-        gv[kGateBeta + lane + 32] = b1;
-        gv[kGateSEg + lane] = sig * __expf(x0);
-        gv[kGateSEg + lane + 32] = sig * __expf(x1);
-        // the scale after this chunk: 1 after chunk 0 (its decay goes into
-        // S_tmem), else sig * decay unless that falls below the floor
-        const float nxt = sig * __expf(gl);  // the decay e^{gc_last} as stored above
-        sig = (c == 0 || !(nxt >= kScaleFloor)) ? 1.f : nxt;
+        gv[kGateBeta + lane] = t0 + lane < T ? a.beta[tok] : 0.f;
+        gv[kGateBeta + lane + 32] = t0 + lane + 32 < T ? a.beta[tok + (size_t)32 * H] : 0.f;
       }
+      if (!PC) gates(c);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_FULL + s]);
       if (PC) {  // channels 0-63 of this stage's per-channel scaling
@@ -1032,7 +1129,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kPrepMmaWarp) {
     // ================================================================ prep-side MMAs
-    if (lane == 0) {
+    // (prologue: after issuing D1 of a chunk, the whole warp folds the
+    // chunk's token norms into its vectors, off the K/Q load's path; the
+    // prep group next needs them about an inverse later)
+    if (PRO || lane == 0) {
       const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_kh = smem_u32(sm + Lay::KH);
       auto W = [&](int slot, uint32_t parity) {
         const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
@@ -1056,17 +1156,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars[B_D1F]);
       };
+      auto norms = [&](int c) {
+        if (!PRO) return;
+        __syncwarp();
+        const int s = c % kStages;
+        fold_token_norms(sm + Lay::KQ + s * 4 * kTileBytes, gate_slot(c), lane,
+                         (a.norm_qk & 1) != 0, (a.norm_qk & 2) != 0);
+        warp_arrive(&bars[B_NORM + s]);
+      };
       // D1 of chunk c + 1 goes out as soon as the prep group has read D1 of
       // chunk c and the chunk's operands are ready.
       bool ok = ready(0);
-      if (ok) issue_d1(0);
+      if (ok) {
+        if (lane == 0) issue_d1(0);
+        norms(0);
+      }
       for (int c = 0; c + 1 < n && ok; ++c) {
         if (!(ok = W(B_D1E, c & 1) && ready(c + 1))) break;
-        issue_d1(c + 1);
+        if (lane == 0) issue_d1(c + 1);
+        norms(c + 1);
       }
-      mma_commit(&bars[B_FIN2]);
-      drain_wait(&bars[B_FIN2], 0);
-      if (!ok) atomicOr(a.status, kStatusTimeout);
+      if (lane == 0) {
+        mma_commit(&bars[B_FIN2]);
+        drain_wait(&bars[B_FIN2], 0);
+        if (!ok) atomicOr(a.status, kStatusTimeout);
+      }
     }
   } else if (warp >= 4 && warp < 8) {
     // ================================================================ prep group
@@ -1078,7 +1192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < n; ++c) {
       const int st = c % kStages;
       const uint32_t ph = c & 1;
-      const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + st * kGateBytes);
+      const float *gv = gate_slot(c);
       const float *gcv = gv + kGateGc, *egv = gv + kGateEg, *iegv = gv + kGateIeg;
       const float *bs = gv + kGateBeta;
       // This warp's waits, probed together: the stage, D1, this P buffer
@@ -1087,8 +1201,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // four prep warps; the P warps probe D1 again in its place).
       // (ADD: no A, so no wait on AF)
       const bool a_rows = !ADD && pt < 64;
-      bool bad = !wait_all<4>({&bars[B_FULL + st], &bars[B_D1F], &bars[B_PE + (c & 1)],
-                               a_rows ? &bars[B_TRDY] : &bars[B_D1F]},
+      // (prologue: also the chunk's token norms, in place of the stage)
+      bool bad = !wait_all<4>({PRO ? &bars[B_NORM + st] : &bars[B_FULL + st], &bars[B_D1F],
+                               &bars[B_PE + (c & 1)], a_rows ? &bars[B_TRDY] : &bars[B_D1F]},
                               {uint32_t((c / kStages) & 1), ph, uint32_t(((c >> 1) - 1) & 1),
                                a_rows ? uint32_t((c - 1) & 1) : ph},
                               abort_flag);
@@ -1100,7 +1215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hp = 0; hp < 2; ++hp) {
           const int r = rl & 63;
           const float gr = gcv[r];
-          const float br = rl < 64 ? bs[r] : 1.f;
+          // (prologue: the row's 1 / |k| or 1 / |q| as well)
+          const float br = (rl < 64 ? bs[r] : 1.f) *
+                           (PRO ? gv[(rl < 64 ? kGateRk : kGateRq) + r] : 1.f);
           const float fr = br * egv[r];
           float x[32];
           tmem_ld32(lane_base + TM_D1 + 32 * hp, x);
@@ -1122,10 +1239,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int s4 = 0; s4 < 8; ++s4) {
               const float4 gg = *reinterpret_cast<const float4 *>(gcv + 32 * hp + 4 * s4);
-              dvs[4 * s4 + 0] = br * __expf(gr - gg.x);
-              dvs[4 * s4 + 1] = br * __expf(gr - gg.y);
-              dvs[4 * s4 + 2] = br * __expf(gr - gg.z);
-              dvs[4 * s4 + 3] = br * __expf(gr - gg.w);
+              // (prologue: the columns' 1 / |k|, which Ieg carries on the
+              // factored path)
+              const float4 rc = PRO ? *reinterpret_cast<const float4 *>(gv + kGateRk + 32 * hp +
+                                                                        4 * s4)
+                                    : make_float4(1.f, 1.f, 1.f, 1.f);
+              dvs[4 * s4 + 0] = br * __expf(gr - gg.x) * rc.x;
+              dvs[4 * s4 + 1] = br * __expf(gr - gg.y) * rc.y;
+              dvs[4 * s4 + 2] = br * __expf(gr - gg.z) * rc.z;
+              dvs[4 * s4 + 3] = br * __expf(gr - gg.w) * rc.w;
             }
           }
           if (rl < 64) {
@@ -1161,7 +1283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
       //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
       uint8_t *tpc = sm + Lay::TP + (c & 1) * kTileBytes;
-      const TOut to{PC ? tpc : sm + Lay::T, tpc, bs, PC ? egv : gv + kGateSEg};
+      const TOut to{PC ? tpc : sm + Lay::T, tpc, bs,
+                    PC ? egv : gv + (PRO ? kGateSEgK : kGateSEg)};
       bad = bad || !wait_all<2>({&bars[B_UF], &bars[B_TPE + (c & 1)]},
                                 {uint32_t((c - 1) & 1), uint32_t(((c >> 1) - 1) & 1)}, abort_flag);
       if (!bad && rl < 64) {  // the warps that wrote A invert its diagonal blocks
@@ -1201,15 +1324,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       return sm + Lay::SVEC + (ADD ? c % 3 : c & 1) * Lay::kSvecBytes;
     };
     auto chunk_vectors = [&](int c, float &dl) -> bool {
+      // (prologue: the stage's vectors are final once its norms are folded in)
       const bool got =
           PC ? warp_wait(&bars[B_SCALED + (c & 1)], (c >> 1) & 1, abort_flag, lane)
-             : warp_wait(&bars[B_FULL + c % kStages], (c / kStages) & 1, abort_flag, lane);
+             : warp_wait(&bars[(PRO ? B_NORM : B_FULL) + c % kStages], (c / kStages) & 1,
+                         abort_flag, lane);
       if (!got) return false;
       // The stage can be refilled while this chunk's O epilogue still runs,
       // so the group keeps its own copy of e^{gc} and e^{gc_last - gc}.
       float *sv = reinterpret_cast<float *>(svec(c));
-      const float *gv = reinterpret_cast<const float *>(sm + Lay::GS + (c % kStages) * kGateBytes);
-      constexpr int kEg = PC ? kGateEg : kGateSEg;  // O epilogue: sigma e^{gc}
+      const float *gv = gate_slot(c);
+      // O epilogue: sigma e^{gc} (prologue: times the token's 1 / |q|)
+      constexpr int kEg = PC ? kGateEg : (PRO ? kGateSEgQ : kGateSEg);
       sv[kSvEg + lane] = gv[kEg + lane];
       sv[kSvEg + lane + 32] = gv[kEg + lane + 32];
       if (PC || c == 0) {  // scalar gates, c >= 1: written with 1 / sigma by the pass
@@ -1423,8 +1549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // next chunk's e^{gc_last - gc} / sigma for its update (every warp
           // writes the same values, from the stage, after its own pass)
           const float inv = 1.f / sig;
-          const float *gn = reinterpret_cast<const float *>(sm + Lay::GS +
-                                                            ((c + 1) % kStages) * kGateBytes);
+          const float *gn = gate_slot(c + 1);
           float *svn = reinterpret_cast<float *>(svec(c + 1));
           svn[kSvEgl + lane] = gn[kGateEgl + lane] * inv;
           svn[kSvEgl + lane + 32] = gn[kGateEgl + lane + 32] * inv;
@@ -1591,15 +1716,15 @@ bool make_map_gate(CUtensorMap *m, const float *base, int B, int T, int H, int d
   return r == CUDA_SUCCESS;
 }
 
-template <bool PC, bool ADD>
+template <bool PC, bool ADD, bool PRO>
 cudaError_t launch_variant(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                            const CUtensorMap &mv, const CUtensorMap &mg, const CUtensorMap &mo,
                            cudaStream_t stream) {
   constexpr size_t smem = Cfg<PC>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC, ADD>,
+  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC, ADD, PRO>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gdr_chunk_tc_kernel<PC, ADD>
+  gdr_chunk_tc_kernel<PC, ADD, PRO>
       <<<(unsigned)((size_t)a.B * a.H), kThreads, smem, stream>>>(mq, mk, mv, mg, mo, a);
   return cudaGetLastError();
 }
@@ -1608,8 +1733,13 @@ template <bool PC>
 cudaError_t launch_pc(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                       const CUtensorMap &mv, const CUtensorMap &mg, const CUtensorMap &mo,
                       cudaStream_t stream) {
-  return a.additive ? launch_variant<PC, true>(a, mq, mk, mv, mg, mo, stream)
-                    : launch_variant<PC, false>(a, mq, mk, mv, mg, mo, stream);
+  if (a.additive) return launch_variant<PC, true, false>(a, mq, mk, mv, mg, mo, stream);
+  if constexpr (!PC) {  // the prologue instance exists for scalar gates only
+    if (a.prologue) return launch_variant<false, false, true>(a, mq, mk, mv, mg, mo, stream);
+  } else {
+    if (a.prologue) return cudaErrorNotSupported;
+  }
+  return launch_variant<PC, false, false>(a, mq, mk, mv, mg, mo, stream);
 }
 
 }  // namespace

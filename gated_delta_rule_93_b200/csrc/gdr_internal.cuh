@@ -37,6 +37,12 @@ struct ChunkArgs {
   // Additive writes (tensor-core kernel only): 1 runs gated linear attention,
   // S_t = S_{t-1} Diag(alpha_t) + v_t k_t^T, with beta unused (may be null).
   int additive;
+  // Prologue (tensor-core kernel, scalar gates): 1 reads g as gate logits a
+  // (g = -gate_scale[h] softplus(a)) and beta as logits b (beta = sigmoid(b))
+  // and L2-normalises q (norm_qk & 1) and k (norm_qk & 2) in the kernel.
+  int prologue;
+  int norm_qk;
+  const float *gate_scale;  // [H]
 };
 
 struct StepArgs {

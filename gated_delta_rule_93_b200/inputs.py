@@ -41,6 +41,7 @@ class Workload:
     steps: int = 1  # decode workloads: consecutive steps
     C: int = 64
     mixer: str = "gdr"  # "gdr" (delta rule) or "gla" (gated linear attention, beta unused)
+    prologue: bool = False  # raw projections in: q, k unnormalised, gate / beta logits
     note: str = field(default="", compare=False)
 
     @property
@@ -66,6 +67,10 @@ WORKLOADS = {
         Workload("gla_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
                  "scalar", False, True, mixer="gla",
                  note="gated linear attention forward at the same shape (additive writes)"),
+        Workload("gdn_prologue_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128,
+                 torch.bfloat16, "scalar", False, True, prologue=True,
+                 note="Gated DeltaNet forward at the 350M shape from raw projections "
+                      "(normalisation and gate maps inside the kernel)"),
     ]
 }
 
@@ -86,6 +91,29 @@ def make_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, gate="scalar", with
     beta = torch.sigmoid(torch.randn(B, T, H, generator=gen))
     S0 = 0.02 * torch.randn(B, H, dv, dk, generator=gen) if with_S0 else None
     return dict(q=q, k=k, v=v, g=g.float(), beta=beta.float(), S0=S0)
+
+
+def make_raw_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, with_S0=False, seed=0,
+                          gate_scale=None):
+    """Raw-projection inputs for ``gdr_chunk_fwd_prologue`` (scalar gate).
+
+    Returns dict of q, k [B,T,H,dk] ~ N(0,1) not normalised, v [B,T,H,dv], a
+    (gate logits) and b (beta logits) [B,T,H] ~ N(0,1) fp32, gate_scale [H]
+    fp32 (default 0.1 for every head) and S0 (or None).  Same draws, in the
+    same order, as ``make_chunk_inputs`` with the same seed, before its
+    normalisation and gate maps: with gate_scale 0.1 the prologue yields that
+    workload's distribution.
+    """
+    gen = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, T, H, dk, generator=gen).to(dtype)
+    k = torch.randn(B, T, H, dk, generator=gen).to(dtype)
+    v = torch.randn(B, T, H, dv, generator=gen).to(dtype)
+    a = torch.randn(B, T, H, generator=gen)
+    b = torch.randn(B, T, H, generator=gen)
+    S0 = 0.02 * torch.randn(B, H, dv, dk, generator=gen) if with_S0 else None
+    gs = torch.full((H,), 0.1) if gate_scale is None else torch.as_tensor(gate_scale).float()
+    return dict(q=q, k=k, v=v, a=a.float(), b=b.float(), gate_scale=gs.float().contiguous(),
+                S0=S0)
 
 
 def make_varlen_inputs(lens, H, dk, dv, dtype=torch.bfloat16, gate="scalar", with_S0=True,
@@ -128,6 +156,8 @@ def make_step_inputs(N, H, dk, dv, steps, dtype=torch.bfloat16, gate="scalar", s
 
 
 def make_workload_inputs(w: Workload, seed=0, steps=None):
+    if w.kind == "chunk" and w.prologue:
+        return make_raw_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.with_S0, seed)
     if w.kind == "chunk":
         return make_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.gate, w.with_S0, seed)
     return make_step_inputs(w.B, w.H, w.dk, w.dv, steps or w.steps, w.dtype, w.gate, seed)

@@ -193,6 +193,40 @@ gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dt
                              float *S_T, int B, int T, int H, int dk, int dv, int C,
                              gdr_stream_t stream);
 
+/* Bits of gdr_chunk_fwd_prologue's norm_qk. */
+#define GDR_NORM_Q 1
+#define GDR_NORM_K 2
+
+/*
+ * The chunked forward from raw projections: the prologue runs inside the
+ * kernel, so the normalised q, k and the gates never go through HBM.
+ * "Decoding Hybrid Linear Attention Architectures", section 3 item 2 (the
+ * erase is a projector along a unit key), section 4 (beta in (0, 1), alpha
+ * a forgetting rate in (0, 1]) and section 5 (gates in log space):
+ *
+ *   q <- q / sqrt(|q|^2 + 1e-6)   if norm_qk & GDR_NORM_Q   (per token, head)
+ *   k <- k / sqrt(|k|^2 + 1e-6)   if norm_qk & GDR_NORM_K
+ *   beta = 1 / (1 + e^{-b}),   g = log alpha = -gate_scale[h] * softplus(a)
+ *
+ * then the recurrence of gdr_chunk_fwd.
+ *
+ *   q, k        [B, T, H, dk] bf16   raw (not normalised) projections
+ *   v, o        [B, T, H, dv] bf16
+ *   a, b        [B, T, H] fp32       gate and write-strength logits
+ *   gate_scale  [H] fp32, > 0        per-head decay scale
+ *   S0, S_T     as gdr_chunk_fwd
+ *
+ * Needs bf16 inputs, dk = dv = 128, C = 64 and gate = GDR_GATE_SCALAR
+ * (GDR_ERR_UNSUPPORTED otherwise).  One launch, no workspace (long sequences
+ * with few heads are not split into segments on this entry).  The inputs
+ * are not modified.
+ */
+gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
+                                  gdr_dtype in_dtype, const float *a, gdr_gate_kind gate,
+                                  const float *gate_scale, const float *b, const float *S0,
+                                  void *o, float *S_T, int B, int T, int H, int dk, int dv, int C,
+                                  int norm_qk, gdr_stream_t stream);
+
 /*
  * One recurrent decode step for N independent states, S updated in place.
  * Source: "Decoding Hybrid Linear Attention Architectures", section 6

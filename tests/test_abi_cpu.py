@@ -177,3 +177,27 @@ def test_gla_validation_rejects_before_any_launch(L):
     assert call(g=None) == binding.GDR_ERR_INVALID_ARG
     assert call(o=_fake_ptr(2)) == binding.GDR_ERR_INVALID_ARG
     assert call(H=0) == binding.GDR_OK
+
+
+def test_prologue_validation_rejects_before_any_launch(L):
+    """gdr_chunk_fwd_prologue: raw projections; scalar gate, tensor-core shapes."""
+    p = _fake_ptr()
+
+    def call(**kw):
+        a = dict(q=p, k=p, v=p, dt=1, a=p, gate=0, gs=p, b=p, S0=None, o=p, ST=None, B=2, T=300,
+                 H=2, dk=128, dv=128, C=64, flags=3, st=None)
+        a.update(kw)
+        return L.gdr_chunk_fwd_prologue(a["q"], a["k"], a["v"], a["dt"], a["a"], a["gate"],
+                                        a["gs"], a["b"], a["S0"], a["o"], a["ST"], a["B"], a["T"],
+                                        a["H"], a["dk"], a["dv"], a["C"], a["flags"], a["st"])
+
+    assert call(B=-1) == binding.GDR_ERR_INVALID_ARG
+    assert call(flags=4) == binding.GDR_ERR_INVALID_ARG
+    assert call(dt=0) == binding.GDR_ERR_UNSUPPORTED
+    assert call(gate=1) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dk=64, dv=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(C=32) == binding.GDR_ERR_UNSUPPORTED
+    assert call(gs=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(b=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(q=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(H=0) == binding.GDR_OK
