@@ -23,6 +23,9 @@ Contents
 ``gdr_fwd_f64`` / ``gdr_fwd_prologue``
     The same recurrence on fp64 inputs, and on the output of ``prologue``
     (raw q, k L2-normalised, beta = sigmoid(b), g = -s_h softplus(a)).
+``gdr_bwd``
+    The backward of the recurrence (reverse mode over tokens, every state
+    kept): gradients of q, k, v, g, beta and S0 from dL/do and dL/dS_T.
 ``chunked``
     A staged fp64 NumPy restatement of the chunkwise algorithm ("Decoding
     Hybrid Linear Attention Architectures", section 5, inter-chunk recursion
@@ -80,6 +83,9 @@ def _load():
             lib.oracle_gdr_fwd_f64.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp, i, i, i, i, i,
                                                i]
             lib.oracle_gdr_fwd_f64.restype = i
+            lib.oracle_gdr_bwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, i, i, i, i, i, i]
+            lib.oracle_gdr_bwd.restype = i
             _lib = lib
     return _lib
 
@@ -245,3 +251,35 @@ def gdr_fwd_prologue(q_raw, k_raw, v, a, b, gate_scale, S0=None, gate="scalar", 
 
     q, k, g, beta = _pro.prologue(q_raw, k_raw, a, b, gate_scale, norm_q, norm_k)
     return gdr_fwd_f64(q, k, _pro.widen(v), g, beta, S0, gate=gate, nthreads=nthreads)
+
+
+def gdr_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, gate="scalar", nthreads=None):
+    """fp64 gradients of the forward ``gdr_fwd`` for upstream dout = dL/do
+    [B,T,H,dv] and dS_T = dL/dS_T [B,H,dv,dk] (None: 0).  Inputs as
+    ``gdr_fwd``.  Returns dict dq, dk [B,T,H,dk], dv [B,T,H,dv], dg (shape of
+    g), dbeta [B,T,H], dS0 [B,H,dv,dk] (float64)."""
+    q, dt = _as_input(q, "q")
+    k, dt2 = _as_input(k, "k")
+    v, dt3 = _as_input(v, "v")
+    if not (dt == dt2 == dt3):
+        raise TypeError("q, k, v must share one dtype")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    gk = GATE_PER_CHANNEL if gate in ("channel", "per_channel", GATE_PER_CHANNEL) else GATE_SCALAR
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    beta = np.ascontiguousarray(beta, dtype=np.float32)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    if dout.shape != (B, T, H, dv):
+        raise ValueError("dout must be [B,T,H,dv]")
+    S0d = None if S0 is None else np.ascontiguousarray(S0, dtype=np.float64)
+    dST = None if dS_T is None else np.ascontiguousarray(dS_T, dtype=np.float64)
+    out = dict(dq=np.zeros((B, T, H, dk)), dk=np.zeros((B, T, H, dk)), dv=np.zeros((B, T, H, dv)),
+               dg=np.zeros(g.shape), dbeta=np.zeros((B, T, H)), dS0=np.zeros((B, H, dv, dk)))
+    n = nthreads or default_threads()
+    rc = _load().oracle_gdr_bwd(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(g), gk, _ptr(beta),
+                                _ptr(S0d), _ptr(dout), _ptr(dST), _ptr(out["dq"]),
+                                _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                                _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk, dv, n)
+    if rc != 0:
+        raise ValueError("oracle_gdr_bwd rejected its arguments")
+    return out

@@ -325,3 +325,199 @@ int oracle_gla_fwd(const void *q, const void *k, const void *v, int in_dtype, co
     pthread_mutex_destroy(&J.lock);
     return 0;
 }
+
+/*
+ * Backward of the gated delta-rule recurrence (reverse mode over tokens),
+ * for training: given dL/do_t and dL/dS_T, the gradients of q, k, v,
+ * g = log alpha, beta and S0.  "Decoding Hybrid Linear Attention
+ * Architectures", section 5 (backpropagation through the same recurrence,
+ * with recomputation); here the plainest form: the forward is run once,
+ * keeping every state, then the steps are undone in reverse.
+ *
+ * One step, as in oracle_gdr_fwd:
+ *     S' = S_{t-1} Diag(alpha)          p = S' k        u = beta (v - p)
+ *     S_t = S' + u k^T                  o = S_t q
+ * With G = dL/dS_t (dS_T at t = T, plus each later step's contribution):
+ *     G   += do q^T,          dq = S_t^T do
+ *     du   = G k,             dk = G^T u (+ S'^T dp below)
+ *     dbeta = du . (v - p),   dv = beta du,   dp = -beta du
+ *     dS'  = G + dp k^T,      dk += S'^T dp
+ *     dg_j = sum_i S'[i][j] dS'[i][j]   (summed over j for a scalar gate)
+ *     dS_{t-1} = dS' Diag(alpha)
+ * dS0 = G after the first step.  Inputs as oracle_gdr_fwd; dout [B,T,H,dv]
+ * and dS_T [B,H,dv,dk] (NULL: zero) in double; outputs in double, same
+ * layouts as the inputs (dg [B,T,H] or [B,T,H,dk]).
+ */
+typedef struct {
+    const void *q, *k, *v;
+    int in_dtype;
+    const float *g;
+    int gate_kind;
+    const float *beta;
+    const double *S0, *dout, *dST;
+    double *dq, *dk, *dv, *dg, *dbeta, *dS0;
+    int B, T, H, dk_, dv_;
+    int next;
+    pthread_mutex_t lock;
+} bwd_job_t;
+
+static void bwd_head(bwd_job_t *J, int b, int h) {
+    const int T = J->T, H = J->H, dk = J->dk_, dv = J->dv_;
+    const size_t SS = (size_t)dv * dk;
+    /* all states S_0 .. S_T, and the decayed S'_t of every step */
+    double *St = (double *)malloc(sizeof(double) * SS * (size_t)(T + 1));
+    double *Sp = (double *)malloc(sizeof(double) * SS * (size_t)(T > 0 ? T : 1));
+    double *G = (double *)malloc(sizeof(double) * SS);
+    double *dSp = (double *)malloc(sizeof(double) * SS);
+    double *kk = (double *)malloc(sizeof(double) * dk);
+    double *qq = (double *)malloc(sizeof(double) * dk);
+    double *al = (double *)malloc(sizeof(double) * dk);
+    double *vv = (double *)malloc(sizeof(double) * dv);
+    double *pp = (double *)malloc(sizeof(double) * dv);
+    double *uu = (double *)malloc(sizeof(double) * dv);
+    double *du = (double *)malloc(sizeof(double) * dv);
+    double *dp = (double *)malloc(sizeof(double) * dv);
+    const size_t sidx = ((size_t)b * H + h) * SS;
+    if (J->S0)
+        memcpy(St, J->S0 + sidx, sizeof(double) * SS);
+    else
+        memset(St, 0, sizeof(double) * SS);
+
+#define LOAD_TOKEN(t)                                                          \
+    const size_t tok = ((size_t)b * T + (t)) * H + h;                          \
+    for (int j = 0; j < dk; ++j) {                                             \
+        kk[j] = load_elem(J->k, tok * dk + j, J->in_dtype);                    \
+        qq[j] = load_elem(J->q, tok * dk + j, J->in_dtype);                    \
+        al[j] = exp((double)(J->gate_kind == OR_GATE_PER_CHANNEL               \
+                                 ? J->g[tok * dk + j] : J->g[tok]));           \
+    }                                                                          \
+    for (int i = 0; i < dv; ++i) vv[i] = load_elem(J->v, tok * dv + i, J->in_dtype); \
+    const double be = (double)J->beta[tok];
+
+    /* forward, keeping the states */
+    for (int t = 0; t < T; ++t) {
+        LOAD_TOKEN(t)
+        const double *Sprev = St + SS * (size_t)t;
+        double *S1 = Sp + SS * (size_t)t, *S2 = St + SS * (size_t)(t + 1);
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) {
+                S1[(size_t)i * dk + j] = Sprev[(size_t)i * dk + j] * al[j];
+                acc += S1[(size_t)i * dk + j] * kk[j];
+            }
+            const double u = be * (vv[i] - acc);
+            for (int j = 0; j < dk; ++j) S2[(size_t)i * dk + j] = S1[(size_t)i * dk + j] + u * kk[j];
+        }
+        (void)qq;
+        (void)tok;
+    }
+
+    /* reverse */
+    if (J->dST)
+        memcpy(G, J->dST + sidx, sizeof(double) * SS);
+    else
+        memset(G, 0, sizeof(double) * SS);
+    for (int t = T - 1; t >= 0; --t) {
+        LOAD_TOKEN(t)
+        const double *S1 = Sp + SS * (size_t)t, *S2 = St + SS * (size_t)(t + 1);
+        const double *dO = J->dout + tok * dv;
+        /* o = S_t q */
+        for (int j = 0; j < dk; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < dv; ++i) acc += S2[(size_t)i * dk + j] * dO[i];
+            J->dq[tok * dk + j] = acc;
+        }
+        for (int i = 0; i < dv; ++i)
+            for (int j = 0; j < dk; ++j) G[(size_t)i * dk + j] += dO[i] * qq[j];
+        /* p and u of this step, recomputed from S' */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S1[(size_t)i * dk + j] * kk[j];
+            pp[i] = acc;
+            uu[i] = be * (vv[i] - acc);
+        }
+        /* S_t = S' + u k^T */
+        double dbeta = 0.0;
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += G[(size_t)i * dk + j] * kk[j];
+            du[i] = acc;
+            dbeta += acc * (vv[i] - pp[i]);
+            J->dv[tok * dv + i] = be * acc;
+            dp[i] = -be * acc;
+        }
+        J->dbeta[tok] = dbeta;
+        for (int j = 0; j < dk; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < dv; ++i)
+                acc += G[(size_t)i * dk + j] * uu[i] + S1[(size_t)i * dk + j] * dp[i];
+            J->dk[tok * dk + j] = acc;
+        }
+        /* dS' = G + dp k^T; dg; dS_{t-1} = dS' Diag(alpha) */
+        double dgs = 0.0;
+        for (int j = 0; j < dk; ++j) {
+            double acc = 0.0;
+            for (int i = 0; i < dv; ++i) {
+                const double d = G[(size_t)i * dk + j] + dp[i] * kk[j];
+                dSp[(size_t)i * dk + j] = d;
+                acc += S1[(size_t)i * dk + j] * d;
+            }
+            if (J->gate_kind == OR_GATE_PER_CHANNEL)
+                J->dg[tok * dk + j] = acc;
+            else
+                dgs += acc;
+        }
+        if (J->gate_kind != OR_GATE_PER_CHANNEL) J->dg[tok] = dgs;
+        for (int i = 0; i < dv; ++i)
+            for (int j = 0; j < dk; ++j) G[(size_t)i * dk + j] = dSp[(size_t)i * dk + j] * al[j];
+    }
+#undef LOAD_TOKEN
+    if (J->dS0) memcpy(J->dS0 + sidx, G, sizeof(double) * SS);
+    free(St); free(Sp); free(G); free(dSp); free(kk); free(qq); free(al);
+    free(vv); free(pp); free(uu); free(du); free(dp);
+}
+
+static void *bwd_worker(void *arg) {
+    bwd_job_t *J = (bwd_job_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int w = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (w >= J->B * J->H) break;
+        bwd_head(J, w / J->H, w % J->H);
+    }
+    return NULL;
+}
+
+int oracle_gdr_bwd(const void *q, const void *k, const void *v, int in_dtype,
+                   const float *g, int gate_kind, const float *beta, const double *S0,
+                   const double *dout, const double *dST, double *dq, double *dk,
+                   double *dv, double *dg, double *dbeta, double *dS0, int B, int T,
+                   int H, int dk_, int dv_, int nthreads) {
+    if (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta)
+        return -1;
+    if (B < 0 || T < 0 || H < 0 || dk_ <= 0 || dv_ <= 0) return -1;
+    if (in_dtype != OR_F32 && in_dtype != OR_BF16) return -1;
+    if (gate_kind != OR_GATE_SCALAR && gate_kind != OR_GATE_PER_CHANNEL) return -1;
+    bwd_job_t J;
+    J.q = q; J.k = k; J.v = v; J.in_dtype = in_dtype;
+    J.g = g; J.gate_kind = gate_kind; J.beta = beta;
+    J.S0 = S0; J.dout = dout; J.dST = dST;
+    J.dq = dq; J.dk = dk; J.dv = dv; J.dg = dg; J.dbeta = dbeta; J.dS0 = dS0;
+    J.B = B; J.T = T; J.H = H; J.dk_ = dk_; J.dv_ = dv_;
+    J.next = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    int n = nthreads;
+    if (n <= 0) n = 1;
+    if (n > B * H) n = B * H;
+    if (n <= 1) {
+        bwd_worker(&J);
+    } else {
+        pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * n);
+        for (int i = 0; i < n; ++i) pthread_create(&th[i], NULL, bwd_worker, &J);
+        for (int i = 0; i < n; ++i) pthread_join(th[i], NULL);
+        free(th);
+    }
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
