@@ -6,6 +6,8 @@ Importing this package does not load the library; the first call does.
 """
 from .binding import (  # noqa: F401
     GdrError,
+    chunk_bwd,
+    chunk_bwd_workspace_bytes,
     chunk_fwd,
     chunk_fwd_gla,
     chunk_fwd_prologue,
@@ -19,6 +21,6 @@ from .binding import (  # noqa: F401
     step,
 )
 
-__all__ = ["chunk_fwd", "chunk_fwd_gla", "chunk_fwd_prologue", "chunk_fwd_kernel_launches", "chunk_fwd_segmented", "chunk_fwd_varlen",
+__all__ = ["chunk_bwd", "chunk_bwd_workspace_bytes", "chunk_fwd", "chunk_fwd_gla", "chunk_fwd_prologue", "chunk_fwd_kernel_launches", "chunk_fwd_segmented", "chunk_fwd_varlen",
            "chunk_fwd_workspace_bytes", "step", "device_status", "lib", "status_string",
            "GdrError"]

@@ -32,6 +32,8 @@ EXPORTS = (
     "gdr_chunk_fwd_varlen",
     "gdr_chunk_fwd_gla",
     "gdr_chunk_fwd_prologue",
+    "gdr_chunk_bwd_workspace_bytes",
+    "gdr_chunk_bwd",
     "gdr_step",
     "gdr_get_device_status",
     "gdr_status_string",
@@ -77,6 +79,11 @@ def lib():
             L.gdr_chunk_fwd_prologue.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, i, i,
                                                  i, i, i, i, i, vp]
             L.gdr_chunk_fwd_prologue.restype = i
+            L.gdr_chunk_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+            L.gdr_chunk_bwd_workspace_bytes.restype = sz
+            L.gdr_chunk_bwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                        vp, i, i, i, i, i, vp, sz, vp]
+            L.gdr_chunk_bwd.restype = i
             L.gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp]
             L.gdr_step.restype = i
             L.gdr_get_device_status.argtypes = [vp]
@@ -383,3 +390,53 @@ def chunk_fwd_prologue(q, k, v, a, b, gate_scale, S0=None, *, norm_q=True, norm_
                                           _stream_handle(stream))
     _check(rc)
     return o, S_T
+
+
+def chunk_bwd_workspace_bytes(B, T, H, dk, dv):
+    return int(lib().gdr_chunk_bwd_workspace_bytes(B, T, H, dk, dv))
+
+
+def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, *, want_dS0=True, workspace=None,
+              stream=None):
+    """``gdr_chunk_bwd``: gradients of the chunked forward.
+
+    Inputs as ``chunk_fwd``; dout [B,T,H,dv] fp32; dS_T [B,H,dv,dk] fp32 or
+    None.  Returns dict dq, dk, dv, dg, dbeta, dS0 (fp32; dS0 None unless
+    want_dS0)."""
+    _need(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (B, T, H, dk), dev)
+    _need(v, "v", dt, (B, T, H, dv), dev)
+    if g.dim() == 4:
+        _need(g, "g", torch.float32, (B, T, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (B, T, H), dev)
+        gk = GDR_GATE_SCALAR
+    _need(beta, "beta", torch.float32, (B, T, H), dev)
+    _need(dout, "dout", torch.float32, (B, T, H, dv), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    if dS_T is not None:
+        _need(dS_T, "dS_T", torch.float32, (B, H, dv, dk), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+               dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty(tuple(g.shape), **f32),
+               dbeta=torch.empty((B, T, H), **f32),
+               dS0=torch.empty((B, H, dv, dk), **f32) if want_dS0 else None)
+    ws = chunk_bwd_workspace_bytes(B, T, H, dk, dv)
+    if workspace is None and ws:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk,
+                                 _ptr(beta), _ptr(S0), _ptr(dout), _ptr(dS_T), _ptr(out["dq"]),
+                                 _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                                 _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk, dv,
+                                 _ptr(workspace),
+                                 workspace.numel() * workspace.element_size()
+                                 if workspace is not None else 0, _stream_handle(stream))
+    _check(rc)
+    return out

@@ -326,6 +326,43 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
   return from_cuda(gdr::launch_chunk_tc(ca, s), "gdr_chunk_fwd_prologue launch");
 }
 
+size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+  if (dk != dv || (dk != 32 && dk != 64 && dk != 128)) return 0;
+  return gdr::bwd_ws_bytes(B, T, H, dk);
+}
+
+gdr_status gdr_chunk_bwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                         const float *g, gdr_gate_kind gate, const float *beta, const float *S0,
+                         const float *dout, const float *dS_T, float *dq, float *dk, float *dv,
+                         float *dg, float *dbeta, float *dS0, int B, int T, int H, int dk_,
+                         int dv_, void *workspace, size_t ws_bytes, gdr_stream_t stream) {
+  if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "negative B/T/H");
+  if (in_dtype != GDR_F32 && in_dtype != GDR_BF16)
+    return fail(GDR_ERR_INVALID_ARG, "in_dtype must be GDR_F32 or GDR_BF16");
+  if (gate != GDR_GATE_SCALAR && gate != GDR_GATE_PER_CHANNEL)
+    return fail(GDR_ERR_INVALID_ARG, "unknown gate kind");
+  if (dk_ != dv_ || (dk_ != 32 && dk_ != 64 && dk_ != 128))
+    return fail(GDR_ERR_UNSUPPORTED, "backward needs dk = dv in {32, 64, 128} (got %d, %d)", dk_,
+                dv_);
+  if ((size_t)B * (size_t)H * (size_t)T > (size_t)1 << 40)
+    return fail(GDR_ERR_INVALID_ARG, "problem too large");
+  if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "B*H too large");
+  if ((size_t)B * H * T != 0) {
+    if (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta)
+      return fail(GDR_ERR_INVALID_ARG, "null input or gradient pointer");
+  }
+  const size_t need = gdr::bwd_ws_bytes(B, T, H, dk_);
+  if ((size_t)B * H != 0 && (ws_bytes < need || !workspace))
+    return fail(GDR_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need);
+  if (workspace && !aligned16(workspace))
+    return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((size_t)B * H == 0) return ok();
+  return from_cuda(gdr::launch_bwd(q, k, v, in_dtype == GDR_BF16, g, gate == GDR_GATE_PER_CHANNEL,
+                                   beta, S0, dout, dS_T, dq, dk, dv, dg, dbeta, dS0, B, T, H,
+                                   dk_, workspace, reinterpret_cast<cudaStream_t>(stream)),
+                   "gdr_chunk_bwd launch");
+}
+
 gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                     const float *g, gdr_gate_kind gate, const float *beta, float *S, void *o,
                     int N, int H, int dk, int dv, gdr_stream_t stream) {

@@ -71,6 +71,13 @@ bool chunk_tc_supports(const ChunkArgs &a);
 int chunk_segments(const ChunkArgs &a, int num_sms);
 size_t chunk_segments_ws_bytes(const ChunkArgs &a, int P);
 cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStream_t stream);
+// Backward of the recurrence (CUDA cores, d_k = d_v = d in {32, 64, 128}).
+size_t bwd_ws_bytes(int B, int T, int H, int d);
+cudaError_t launch_bwd(const void *q, const void *k, const void *v, int bf16, const float *g,
+                       int per_channel, const float *beta, const float *S0, const float *dout,
+                       const float *dST, float *dq, float *dk, float *dv, float *dg,
+                       float *dbeta, float *dS0, int B, int T, int H, int d, void *ws,
+                       cudaStream_t stream);
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float load_in(const void *p, size_t i, int bf16) {

@@ -228,6 +228,39 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
                                   int norm_qk, gdr_stream_t stream);
 
 /*
+ * Backward of the chunked forward (training): the gradients of q, k, v,
+ * g = log alpha, beta and S0 from dL/do and dL/dS_T.  "Decoding Hybrid
+ * Linear Attention Architectures", section 5: backpropagation through the
+ * same recurrence, with recomputation.  Per step (S' = S_{t-1} Diag(alpha),
+ * p = S' k, u = beta (v - p), S_t = S' + u k^T, o = S_t q) and G = dL/dS_t:
+ *
+ *   G += do q^T;  dq = S_t^T do;  du = G k;  dbeta = du . (v - p);
+ *   dv = beta du;  dk = G^T u - beta S'^T du;  dS' = G - beta du k^T;
+ *   dg_j = sum_i S'[i][j] dS'[i][j] (summed over j for a scalar gate);
+ *   G <- dS' Diag(alpha);  dS0 = G at the start.
+ *
+ *   q, k, v, g, beta, S0   as gdr_chunk_fwd (S0 NULL: zero)
+ *   dout   [B, T, H, dv] fp32   dL/do
+ *   dS_T   [B, H, dv, dk] fp32 or NULL (zero)
+ *   dq, dk [B, T, H, dk] fp32;  dv [B, T, H, dv] fp32 (written)
+ *   dg     [B, T, H] fp32 (scalar gate) or [B, T, H, dk] (per channel)
+ *   dbeta  [B, T, H] fp32;  dS0 [B, H, dv, dk] fp32 or NULL (not written)
+ *   workspace  device memory of gdr_chunk_bwd_workspace_bytes() bytes,
+ *              16-byte aligned, owned by the caller (overwritten): the
+ *              state at every 64th token and a 64-token stash per (b, h)
+ *
+ * Needs dk = dv in {32, 64, 128} (GDR_ERR_UNSUPPORTED otherwise); fp32 or
+ * bf16 inputs; arithmetic in fp32 on CUDA cores, one CTA per (b, h).  One
+ * launch on `stream`.
+ */
+size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+gdr_status gdr_chunk_bwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
+                         const float *g, gdr_gate_kind gate, const float *beta, const float *S0,
+                         const float *dout, const float *dS_T, float *dq, float *dk, float *dv,
+                         float *dg, float *dbeta, float *dS0, int B, int T, int H, int dk_,
+                         int dv_, void *workspace, size_t ws_bytes, gdr_stream_t stream);
+
+/*
  * One recurrent decode step for N independent states, S updated in place.
  * Source: "Decoding Hybrid Linear Attention Architectures", section 6
  * (constant-cost update of the fixed-size state per decoded token) with the

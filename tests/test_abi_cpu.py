@@ -201,3 +201,33 @@ def test_prologue_validation_rejects_before_any_launch(L):
     assert call(b=None) == binding.GDR_ERR_INVALID_ARG
     assert call(q=None) == binding.GDR_ERR_INVALID_ARG
     assert call(H=0) == binding.GDR_OK
+
+
+def test_backward_validation_rejects_before_any_launch(L):
+    """gdr_chunk_bwd: square heads of 32, 64 or 128; workspace required."""
+    p = _fake_ptr()
+    ws = L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128)
+    assert ws == 2 * 2 * (5 + 1 + 64) * 128 * 128 * 4
+    assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 64) == 0
+
+    def call(**kw):
+        a = dict(q=p, k=p, v=p, dt=1, g=p, gate=0, beta=p, S0=None, do=p, dST=None, dq=p, dk=p,
+                 dv=p, dg=p, db=p, dS0=None, B=2, T=300, H=2, dk_=128, dv_=128, ws=p, wsb=ws,
+                 st=None)
+        a.update(kw)
+        return L.gdr_chunk_bwd(a["q"], a["k"], a["v"], a["dt"], a["g"], a["gate"], a["beta"],
+                               a["S0"], a["do"], a["dST"], a["dq"], a["dk"], a["dv"], a["dg"],
+                               a["db"], a["dS0"], a["B"], a["T"], a["H"], a["dk_"], a["dv_"],
+                               a["ws"], a["wsb"], a["st"])
+
+    assert call(B=-1) == binding.GDR_ERR_INVALID_ARG
+    assert call(dt=5) == binding.GDR_ERR_INVALID_ARG
+    assert call(gate=3) == binding.GDR_ERR_INVALID_ARG
+    assert call(dk_=128, dv_=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dk_=96, dv_=96) == binding.GDR_ERR_UNSUPPORTED
+    assert call(do=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(dg=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(wsb=ws - 1) == binding.GDR_ERR_WORKSPACE
+    assert call(ws=None) == binding.GDR_ERR_WORKSPACE
+    assert call(ws=_fake_ptr(4)) == binding.GDR_ERR_INVALID_ARG
+    assert call(H=0) == binding.GDR_OK
