@@ -42,6 +42,7 @@ KERNEL_SOURCES = {
               "gated_delta_rule_93_b200/csrc/gdr_segments.cu",
               "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
     "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu"],
+    "bwd": ["gated_delta_rule_93_b200/csrc/gdr_bwd.cu"],
 }
 
 
@@ -55,6 +56,9 @@ def algorithmic_bytes(w):
                             + 4 * gate_elems + 4)
     beta = 0 if w.mixer == "gla" else 4
     per_tok = (2 * w.dk + w.dv) * e_in + w.dv * e_in + 4 * gate_elems + beta
+    if w.backward:  # q, k, v, g, beta, dL/do in; dq, dk, dv, dg, dbeta out (fp32)
+        per_tok = ((2 * w.dk + w.dv) * e_in + 4 * gate_elems + 4 + 4 * w.dv
+                   + 4 * (2 * w.dk + w.dv) + 4 * gate_elems + 4)
     state = 4 * w.dk * w.dv * w.B * w.H
     return w.B * w.T * w.H * per_tok + state * (int(w.with_S0) + int(w.want_S_T))
 
@@ -65,6 +69,8 @@ def algorithmic_flops(w, C=64):
     about 7 d_k d_v per state, CUDA cores)."""
     if w.kind == "step":
         return w.B * w.H * 7.0 * w.dk * w.dv
+    if w.backward:  # one recomputed forward step (5 d^2) and its reverse (16 d^2)
+        return w.B * w.T * w.H * 21.0 * w.dk * w.dv
     if w.mixer == "gla":  # no correction: state update, S q, masked Q K^T and P V
         return w.B * w.T * w.H * (4 * w.dk * w.dv + C * (w.dk + w.dv))
     per = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0
@@ -128,6 +134,11 @@ class ClockSampler:
             self.t.start()
         except (FileNotFoundError, OSError):
             self.proc = None
+            return
+        # the first sample before the timed region starts (bounded)
+        t_end = time.time() + 5.0
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -136,6 +147,11 @@ class ClockSampler:
     def stop(self):
         if self.proc is None:
             return None
+        # one more sample after the timed region (a short region can fall
+        # between two samples), bounded
+        n0, t_end = len(self.lines), time.time() + 1.0
+        while len(self.lines) <= n0 and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.005)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -211,6 +227,22 @@ def run_ours(args, rank, world, local_rank):
                                            d["gate_scale"], d["S0"], o=o, S_T=S_T,
                                            output_final_state=S_T is not None)
 
+        if w.backward:  # gradients for a seeded dL/do; preallocated outputs and workspace
+            launches_per_step = 1
+            f32 = dict(dtype=torch.float32, device=dev)
+            grads = dict(dq=torch.empty(w.B, w.T, w.H, w.dk, **f32),
+                         dk=torch.empty(w.B, w.T, w.H, w.dk, **f32),
+                         dv=torch.empty(w.B, w.T, w.H, w.dv, **f32),
+                         dg=torch.empty(tuple(d["g"].shape), **f32),
+                         dbeta=torch.empty(w.B, w.T, w.H, **f32), dS0=None)
+            bws = torch.empty(binding.chunk_bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv),
+                              dtype=torch.uint8, device=dev)
+            o, S_T = grads["dq"], None
+
+            def step():
+                binding.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dout"], d["S0"],
+                                  None, want_dS0=False, workspace=bws, out=grads)
+
         if w.mixer == "gla":  # gated linear attention: one launch, no beta, no workspace
             host.pop("beta")
             d.pop("beta")
@@ -264,10 +296,12 @@ def run_ours(args, rank, world, local_rank):
     else:
         pin = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
         dev_in = d
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    S_h = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory() if S_T is not None else None
+    # the step's results read back: o (and S_T), or every gradient
+    results = [grads[n] for n in ("dq", "dk", "dv", "dg", "dbeta")] if w.backward else \
+        [o] + ([S_T] if S_T is not None else [])
+    res_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in results]
     h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
-    d2h = o_h.numel() * o_h.element_size() + (S_h.numel() * 4 if S_h is not None else 0)
+    d2h = sum(t.numel() * t.element_size() for t in res_h)
 
     def e2e_step():
         for kk, v in pin.items():
@@ -278,9 +312,8 @@ def run_ours(args, rank, world, local_rank):
                          o=o)
         else:
             step()
-        o_h.copy_(o, non_blocking=True)
-        if S_h is not None:
-            S_h.copy_(S_T, non_blocking=True)
+        for hb, t in zip(res_h, results):
+            hb.copy_(t, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
@@ -310,6 +343,9 @@ def run_ours(args, rank, world, local_rank):
     avg_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
     achieved = abytes / (avg_launch_ms / 1e3) / 1e9
     roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (tc_peak * 1e12)) * 1e3
+    if w.backward:  # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x SM clock
+        alu_peak = 148 * 128 * 2 * (clk.get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
+        roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (alu_peak * 1e12)) * 1e3
     line = {
         "metric": METRIC,
         "value": value,
@@ -334,12 +370,19 @@ def run_ours(args, rank, world, local_rank):
         "tflops": aflops * world * args.steps / (total_ms / 1e3) / 1e12,
         "roofline_time_ms": roof_ms,
         "roofline_fraction": roof_ms / ms_step,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+        "roofline": ({"bound": "alu", "achieved": aflops / (avg_launch_ms / 1e3) / 1e12,
+                      "peak": alu_peak, "unit": "TFLOP/s",
+                      "frac": aflops / (avg_launch_ms / 1e3) / 1e12 / alu_peak,
+                      "traffic": recorded_traffic(w.name, "bwd"),
+                      "peak_source": "CUDA-core fp32 FMA, 148 SMs x 128 lanes "
+                      "x 2 flop x max SM clock", "algorithmic_flops_per_launch": aflops,
+                      "kernel": "gdr_chunk_bwd"} if w.backward else
+                     {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
                      "kernel": ("gdr_chunk_fwd_prologue" if w.prologue else
                                 "gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
-                     if w.kind == "chunk" else "gdr_step"},
+                     if w.kind == "chunk" else "gdr_step"}),
         "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
@@ -362,6 +405,8 @@ def _oracle_sample(w, inp, Tp):
     qkv = [to_numpy_input(sl["q"]), to_numpy_input(sl["k"]), to_numpy_input(sl["v"])]
     if w.prologue:
         return qkv + [sl["a"].numpy(), sl["b"].numpy(), sl["gate_scale"].numpy(), S0]
+    if w.backward:
+        return qkv + [sl["g"].numpy(), sl["beta"].numpy(), sl["dout"].double().numpy(), S0]
     return qkv + [sl["g"].numpy(), sl["beta"].numpy(), S0]
 
 
@@ -369,6 +414,8 @@ def _oracle_fwd(oracle, w, a, n):
     """The oracle's forward for the workload (arguments from _oracle_sample)."""
     if w.prologue:
         return oracle.gdr_fwd_prologue(*a, gate=w.gate, nthreads=n)
+    if w.backward:
+        return oracle.gdr_bwd(*a, gate=w.gate, nthreads=n)
     if w.mixer == "gla":
         return oracle.gla_fwd(a[0], a[1], a[2], a[3], a[5], gate=w.gate, nthreads=n)
     return oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)

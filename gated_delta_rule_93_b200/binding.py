@@ -397,7 +397,7 @@ def chunk_bwd_workspace_bytes(B, T, H, dk, dv):
 
 
 def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, *, want_dS0=True, workspace=None,
-              stream=None):
+              out=None, stream=None):
     """``gdr_chunk_bwd``: gradients of the chunked forward.
 
     Inputs as ``chunk_fwd``; dout [B,T,H,dv] fp32; dS_T [B,H,dv,dk] fp32 or
@@ -423,10 +423,16 @@ def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, *, want_dS0=True, work
     if dS_T is not None:
         _need(dS_T, "dS_T", torch.float32, (B, H, dv, dk), dev)
     f32 = dict(dtype=torch.float32, device=dev)
-    out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
-               dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty(tuple(g.shape), **f32),
-               dbeta=torch.empty((B, T, H), **f32),
-               dS0=torch.empty((B, H, dv, dk), **f32) if want_dS0 else None)
+    if out is None:  # (or the caller's preallocated dict of the same tensors)
+        out = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+                   dv=torch.empty((B, T, H, dv), **f32), dg=torch.empty(tuple(g.shape), **f32),
+                   dbeta=torch.empty((B, T, H), **f32),
+                   dS0=torch.empty((B, H, dv, dk), **f32) if want_dS0 else None)
+    for name, shape in (("dq", (B, T, H, dk)), ("dk", (B, T, H, dk)), ("dv", (B, T, H, dv)),
+                        ("dg", tuple(g.shape)), ("dbeta", (B, T, H))):
+        _need(out[name], name, torch.float32, shape, dev)
+    if out.get("dS0") is not None:
+        _need(out["dS0"], "dS0", torch.float32, (B, H, dv, dk), dev)
     ws = chunk_bwd_workspace_bytes(B, T, H, dk, dv)
     if workspace is None and ws:
         workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
@@ -434,7 +440,7 @@ def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, *, want_dS0=True, work
         rc = lib().gdr_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk,
                                  _ptr(beta), _ptr(S0), _ptr(dout), _ptr(dS_T), _ptr(out["dq"]),
                                  _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
-                                 _ptr(out["dbeta"]), _ptr(out["dS0"]), B, T, H, dk, dv,
+                                 _ptr(out["dbeta"]), _ptr(out.get("dS0")), B, T, H, dk, dv,
                                  _ptr(workspace),
                                  workspace.numel() * workspace.element_size()
                                  if workspace is not None else 0, _stream_handle(stream))

@@ -15,11 +15,15 @@
 // l, l + 32, ..., so S and G stay in registers (32 floats each at d = 128)
 // and a row's dot products are warp reductions.  The sums over rows (dq, dk,
 // dg, dbeta) go through shared memory once per token.
-// Recomputation: a forward sweep stores the state at every 64th token
-// (checkpoints); then, chunk by chunk from the last, the chunk's states are
-// recomputed from its checkpoint into a stash and the chunk is walked in
-// reverse.  Both live in the caller's workspace, in a thread-major layout
-// (each thread reads back only what it wrote).
+// Recomputation: a forward sweep stores the state at every 8th token
+// (checkpoints); then, 8 tokens at a time from the last, the states are
+// recomputed from their checkpoint into a stash and walked in reverse.
+// Both live in the caller's workspace, element-major ([element][thread], so
+// a warp's access is one contiguous 128-byte line; each thread reads back
+// only what it wrote); the stashes of all CTAs (64 KB per token and head at
+// d = 128) stay within L2.  The token vectors of a 64-token
+// chunk (k, q, v, g, beta, dL/do) are staged in shared memory as fp32 by
+// the whole CTA with coalesced loads before the chunk is processed.
 #include "gdr_internal.cuh"
 
 namespace gdr {
@@ -27,7 +31,8 @@ namespace {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 64;
+constexpr int kChunk = 64;  // tokens staged in shared memory at a time
+constexpr int kSub = 8;     // tokens per checkpoint / stash
 
 struct BwdArgs {
   const void *q, *k, *v;
@@ -64,16 +69,23 @@ template <int NC, int RW>
 __global__ void __launch_bounds__(kThreads, 1) gdr_bwd_kernel(BwdArgs a) {
   constexpr int D = NC * 32;
   constexpr int E = NC * RW;  // state elements per thread
-  extern __shared__ float red_raw[];  // [2][kWarps][3 D + 1]: per-warp partial sums
-  float(*red)[kWarps][3 * D + 1] = reinterpret_cast<float(*)[kWarps][3 * D + 1]>(red_raw);
+  // shared memory: per-warp partial sums [2][kWarps][3 D + 1], then the
+  // staged chunk: k, q, v, dL/do [kChunk][D], g [kChunk][D or 1], beta [kChunk]
+  extern __shared__ float smem[];
+  float(*red)[kWarps][3 * D + 1] = reinterpret_cast<float(*)[kWarps][3 * D + 1]>(smem);
+  float *sk = smem + 2 * kWarps * (3 * D + 1);
+  float *sq = sk + kChunk * D, *sv = sq + kChunk * D, *sdo = sv + kChunk * D;
+  float *sg = sdo + kChunk * D;
+  float *sb = sg + kChunk * (a.per_channel ? D : 1);
   const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int T = a.T, H = a.H;
+  const int nsub = (T + kSub - 1) / kSub;
   const int nch = (T + kChunk - 1) / kChunk;
   const size_t SS = (size_t)D * D;
-  float *ckpt = a.ws + (size_t)bh * (nch + 1 + kChunk) * SS;  // [nch + 1][thread][E]
-  float *stash = ckpt + (size_t)(nch + 1) * SS;                // [64][thread][E]
-  auto at = [&](float *base, int slot) { return base + (size_t)slot * SS + (size_t)tid * E; };
+  float *ckpt = a.ws + (size_t)bh * (nsub + 1 + kSub) * SS;  // [nsub + 1][E][thread]
+  float *stash = ckpt + (size_t)(nsub + 1) * SS;              // [kSub][E][thread]
+  auto at = [&](float *base, int slot) { return base + (size_t)slot * SS + tid; };
   auto sidx = [&](int r, int c) { return (size_t)(w + 16 * r) * D + l + 32 * c; };
 
   float S[RW][NC], G[RW][NC];
@@ -85,19 +97,40 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_bwd_kernel(BwdArgs a) {
       for (int c = 0; c < NC; ++c) S[r][c] = s0 ? s0[sidx(r, c)] : 0.f;
   }
 
-  // per-token inputs of this thread: k, q, alpha at its channels, v at its rows
+  // tokens [t0, t1) of this (b, h) into shared memory (all threads;
+  // bracketed by barriers)
+  auto stage = [&](int t0, int t1, bool with_q, bool with_do) {
+    __syncthreads();  // the previous chunk's reads are done
+    const int n = (t1 - t0) * D;
+    for (int i = tid; i < n; i += kThreads) {
+      const int t = i / D, j = i - t * D;
+      const size_t x = (((size_t)b * T + t0 + t) * H + h) * D + j;
+      sk[i] = ld_in(a.k, x, a.bf16);
+      sv[i] = ld_in(a.v, x, a.bf16);
+      if (with_q) sq[i] = ld_in(a.q, x, a.bf16);
+      if (with_do) sdo[i] = a.dout[x];
+      if (a.per_channel) sg[i] = a.g[x];
+    }
+    for (int t = tid; t < t1 - t0; t += kThreads) {
+      const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+      if (!a.per_channel) sg[t] = a.g[tok];
+      sb[t] = a.beta[tok];
+    }
+    __syncthreads();
+  };
+  // per-token inputs of this thread: k, q, alpha at its channels, v at its
+  // rows (token tl of the staged chunk)
   float kk[NC], qq[NC], al[NC], vv[RW], be;
-  auto load = [&](int t) {
-    const size_t tok = ((size_t)b * T + t) * H + h;
+  auto load = [&](int tl) {
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-      kk[c] = ld_in(a.k, tok * D + l + 32 * c, a.bf16);
-      qq[c] = ld_in(a.q, tok * D + l + 32 * c, a.bf16);
-      al[c] = __expf(a.per_channel ? a.g[tok * D + l + 32 * c] : a.g[tok]);
+      kk[c] = sk[tl * D + l + 32 * c];
+      qq[c] = sq[tl * D + l + 32 * c];
+      al[c] = __expf(a.per_channel ? sg[tl * D + l + 32 * c] : sg[tl]);
     }
 #pragma unroll
-    for (int r = 0; r < RW; ++r) vv[r] = ld_in(a.v, tok * D + w + 16 * r, a.bf16);
-    be = a.beta[tok];
+    for (int r = 0; r < RW; ++r) vv[r] = sv[tl * D + w + 16 * r];
+    be = sb[tl];
   };
   // one forward step in place: S <- S Diag(alpha) + u k^T; returns nothing
   auto step = [&](float (&X)[RW][NC]) {
@@ -124,20 +157,24 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_bwd_kernel(BwdArgs a) {
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
-      for (int c = 0; c < NC; ++c) dst[r * NC + c] = X[r][c];
+      for (int c = 0; c < NC; ++c) dst[(r * NC + c) * kThreads] = X[r][c];
   };
   auto fetch = [&](const float *src, float (&X)[RW][NC]) {
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
-      for (int c = 0; c < NC; ++c) X[r][c] = src[r * NC + c];
+      for (int c = 0; c < NC; ++c) X[r][c] = src[(r * NC + c) * kThreads];
   };
 
-  // ---- forward sweep: checkpoints at every chunk start
-  for (int t = 0; t < T; ++t) {
-    if (t % kChunk == 0) store(at(ckpt, t / kChunk), S);
-    load(t);
-    step(S);
+  // ---- forward sweep: checkpoints at every kSub-th token
+  for (int ch = 0; ch < nch; ++ch) {
+    const int t0 = ch * kChunk, t1 = min(T, t0 + kChunk);
+    stage(t0, t1, false, false);
+    for (int t = t0; t < t1; ++t) {
+      if (t % kSub == 0) store(at(ckpt, t / kSub), S);
+      load(t - t0);
+      step(S);
+    }
   }
 
   // ---- reverse: G = dL/dS_T
@@ -149,15 +186,18 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_bwd_kernel(BwdArgs a) {
       for (int c = 0; c < NC; ++c) G[r][c] = d ? d[sidx(r, c)] : 0.f;
   }
   for (int ch = nch - 1; ch >= 0; --ch) {
-    const int t0 = ch * kChunk, t1 = min(T, t0 + kChunk);
-    fetch(at(ckpt, ch), S);
-    for (int t = t0; t < t1; ++t) {  // the chunk's states S_{t-1} into the stash
+    const int c0 = ch * kChunk, c1 = min(T, c0 + kChunk);
+    stage(c0, c1, true, true);
+    for (int t0 = c0 + ((c1 - 1 - c0) / kSub) * kSub; t0 >= c0; t0 -= kSub) {
+    const int t1 = min(c1, t0 + kSub);
+    fetch(at(ckpt, t0 / kSub), S);
+    for (int t = t0; t < t1; ++t) {  // the states S_{t-1} into the stash
       store(at(stash, t - t0), S);
-      load(t);
+      load(t - c0);
       step(S);
     }
     for (int t = t1 - 1; t >= t0; --t) {
-      load(t);
+      load(t - c0);
       const size_t tok = ((size_t)b * T + t) * H + h;
       float Sp[RW][NC];
       fetch(at(stash, t - t0), Sp);
@@ -177,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_bwd_kernel(BwdArgs a) {
 #pragma unroll
       for (int r = 0; r < RW; ++r) {
         u[r] = be * (vv[r] - p[r]);
-        dO[r] = a.dout[tok * D + w + 16 * r];
+        dO[r] = sdo[(t - c0) * D + w + 16 * r];
       }
       // dq = S_t^T do (partial over this warp's rows); G += do q^T
       float dqp[NC], dkp[NC], dgp[NC];
@@ -261,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_bwd_kernel(BwdArgs a) {
         }
       }
     }
+    }
   }
   if (a.dS0) {
 #pragma unroll
@@ -274,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_bwd_kernel(BwdArgs a) {
 
 size_t bwd_ws_bytes(int B, int T, int H, int d) {
   if (B <= 0 || H <= 0 || T < 0) return 0;
-  const size_t nch = (size_t)(T + kChunk - 1) / kChunk;
-  return (size_t)B * H * (nch + 1 + kChunk) * (size_t)d * d * sizeof(float);
+  const size_t nsub = (size_t)(T + kSub - 1) / kSub;
+  return (size_t)B * H * (nsub + 1 + kSub) * (size_t)d * d * sizeof(float);
 }
 
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, int bf16, const float *g,
@@ -286,7 +327,9 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, int bf16, co
   BwdArgs a{q, k, v, g, beta, S0, dout, dST, dq, dk, dv, dg, dbeta, dS0,
             static_cast<float *>(ws), B, T, H, d, bf16, per_channel};
   const unsigned grid = (unsigned)((size_t)B * H);
-  const size_t smem = 2 * kWarps * (3 * (size_t)d + 1) * sizeof(float);
+  const size_t smem = (2 * kWarps * (3 * (size_t)d + 1) + 4 * (size_t)kChunk * d +
+                      (size_t)kChunk * (per_channel ? d : 1) + kChunk) *
+                     sizeof(float);
   auto go = [&](auto kern) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -42,6 +42,7 @@ class Workload:
     C: int = 64
     mixer: str = "gdr"  # "gdr" (delta rule) or "gla" (gated linear attention, beta unused)
     prologue: bool = False  # raw projections in: q, k unnormalised, gate / beta logits
+    backward: bool = False  # gradients (gdr_chunk_bwd) for a seeded dL/do
     note: str = field(default="", compare=False)
 
     @property
@@ -67,6 +68,9 @@ WORKLOADS = {
         Workload("gla_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
                  "scalar", False, True, mixer="gla",
                  note="gated linear attention forward at the same shape (additive writes)"),
+        Workload("gdn_bwd_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
+                 "scalar", False, False, backward=True,
+                 note="Gated DeltaNet backward at the 350M shape (dL/do ~ N(0, 1) fp32)"),
         Workload("gdn_prologue_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128,
                  torch.bfloat16, "scalar", False, True, prologue=True,
                  note="Gated DeltaNet forward at the 350M shape from raw projections "
@@ -158,6 +162,11 @@ def make_step_inputs(N, H, dk, dv, steps, dtype=torch.bfloat16, gate="scalar", s
 def make_workload_inputs(w: Workload, seed=0, steps=None):
     if w.kind == "chunk" and w.prologue:
         return make_raw_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.with_S0, seed)
+    if w.kind == "chunk" and w.backward:
+        d = make_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.gate, w.with_S0, seed)
+        gen = torch.Generator().manual_seed(seed + 104729)
+        d["dout"] = torch.randn(w.B, w.T, w.H, w.dv, generator=gen)
+        return d
     if w.kind == "chunk":
         return make_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.gate, w.with_S0, seed)
     return make_step_inputs(w.B, w.H, w.dk, w.dv, steps or w.steps, w.dtype, w.gate, seed)

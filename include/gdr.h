@@ -247,7 +247,7 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
  *   dbeta  [B, T, H] fp32;  dS0 [B, H, dv, dk] fp32 or NULL (not written)
  *   workspace  device memory of gdr_chunk_bwd_workspace_bytes() bytes,
  *              16-byte aligned, owned by the caller (overwritten): the
- *              state at every 64th token and a 64-token stash per (b, h)
+ *              state at every 8th token and an 8-token stash per (b, h)
  *
  * Needs dk = dv in {32, 64, 128} (GDR_ERR_UNSUPPORTED otherwise); fp32 or
  * bf16 inputs; arithmetic in fp32 on CUDA cores, one CTA per (b, h).  One

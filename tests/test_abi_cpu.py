@@ -207,7 +207,7 @@ def test_backward_validation_rejects_before_any_launch(L):
     """gdr_chunk_bwd: square heads of 32, 64 or 128; workspace required."""
     p = _fake_ptr()
     ws = L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128)
-    assert ws == 2 * 2 * (5 + 1 + 64) * 128 * 128 * 4
+    assert ws == 2 * 2 * (38 + 1 + 8) * 128 * 128 * 4  # every 8th state + an 8-token stash
     assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 64) == 0
 
     def call(**kw):
