@@ -26,6 +26,10 @@ Contents
 ``gdr_bwd``
     The backward of the recurrence (reverse mode over tokens, every state
     kept): gradients of q, k, v, g, beta and S0 from dL/do and dL/dS_T.
+``dplr_fwd``
+    The diagonal-plus-low-rank transition S_t = S_{t-1}(Diag(alpha_t) +
+    a_t b_t^T) + v_t k_t^T, o_t = S_t q_t ("Decoding Hybrid Linear Attention
+    Architectures", section 3 item 5).
 ``chunked``
     A staged fp64 NumPy restatement of the chunkwise algorithm ("Decoding
     Hybrid Linear Attention Architectures", section 5, inter-chunk recursion
@@ -86,6 +90,9 @@ def _load():
             lib.oracle_gdr_bwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp, vp, vp,
                                            vp, vp, i, i, i, i, i, i]
             lib.oracle_gdr_bwd.restype = i
+            lib.oracle_dplr_fwd.argtypes = [vp, vp, vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i,
+                                            i, i]
+            lib.oracle_dplr_fwd.restype = i
             _lib = lib
     return _lib
 
@@ -283,3 +290,31 @@ def gdr_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, gate="scalar", nthreads=
     if rc != 0:
         raise ValueError("oracle_gdr_bwd rejected its arguments")
     return out
+
+
+def dplr_fwd(q, k, v, a, b, g, S0=None, gate="scalar", nthreads=None):
+    """fp64 DPLR recurrence S_t = S_{t-1}(Diag(alpha_t) + a_t b_t^T) + v_t k_t^T,
+    o_t = S_t q_t.  q, k, a, b [B,T,H,dk] and v [B,T,H,dv] (float32, or
+    uint16 bf16 bits, one dtype); g = log alpha [B,T,H] or [B,T,H,dk];
+    S0 [B,H,dv,dk] or None.  Returns (o, S_T) float64."""
+    arrs = [_as_input(x, n) for x, n in ((q, "q"), (k, "k"), (v, "v"), (a, "a"), (b, "b"))]
+    dts = {dt for _, dt in arrs}
+    if len(dts) != 1:
+        raise TypeError("q, k, v, a, b must share one dtype")
+    (q, dt), (k, _), (v, _), (a, _), (b, _) = arrs
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for x, n in ((k, "k"), (a, "a"), (b, "b")):
+        if x.shape != (B, T, H, dk):
+            raise ValueError(f"{n} must be [B,T,H,dk]")
+    gk = GATE_PER_CHANNEL if gate in ("channel", "per_channel", GATE_PER_CHANNEL) else GATE_SCALAR
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    S0d = None if S0 is None else np.ascontiguousarray(S0, dtype=np.float64)
+    o = np.zeros((B, T, H, dv), np.float64)
+    S_T = np.zeros((B, H, dv, dk), np.float64)
+    n = nthreads or default_threads()
+    rc = _load().oracle_dplr_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), dt, _ptr(g), gk,
+                                 _ptr(S0d), _ptr(o), _ptr(S_T), B, T, H, dk, dv, n)
+    if rc != 0:
+        raise ValueError("oracle_dplr_fwd rejected its arguments")
+    return o, S_T

@@ -521,3 +521,108 @@ int oracle_gdr_bwd(const void *q, const void *k, const void *v, int in_dtype,
     pthread_mutex_destroy(&J.lock);
     return 0;
 }
+
+/*
+ * Diagonal-plus-low-rank transition (DPLR), the generalised sibling of the
+ * delta rule: "Decoding Hybrid Linear Attention Architectures", section 3
+ * item 5:
+ *
+ *     S_t = S_{t-1} (Diag(alpha_t) + a_t b_t^T) + v_t k_t^T,    o_t = S_t q_t
+ *
+ * (the transition acts on the key axis; the write accumulates).  With
+ * a = -beta (alpha . k), b = k and v scaled by beta it is the gated delta
+ * rule with a per-channel gate.  q, k, a, b [B,T,H,dk]; v, o [B,T,H,dv];
+ * g = log alpha [B,T,H] or [B,T,H,dk]; S0, S_T [B,H,dv,dk].  Per row i of S:
+ *     x_i = S_i . a;   S_i <- S_i Diag(alpha) + x_i b^T + v_i k^T;   o_i = S_i . q
+ */
+typedef struct {
+    const void *q, *k, *v, *a, *b;
+    int in_dtype;
+    const float *g;
+    int gate_kind;
+    const double *S0;
+    double *o, *S_T;
+    int B, T, H, dk, dv;
+    int next;
+    pthread_mutex_t lock;
+} dplr_job_t;
+
+static void dplr_head(dplr_job_t *J, int b_, int h) {
+    const int T = J->T, H = J->H, dk = J->dk, dv = J->dv;
+    double *S = (double *)malloc(sizeof(double) * (size_t)dv * dk);
+    double *kk = (double *)malloc(sizeof(double) * dk);
+    double *qq = (double *)malloc(sizeof(double) * dk);
+    double *aa = (double *)malloc(sizeof(double) * dk);
+    double *bb = (double *)malloc(sizeof(double) * dk);
+    double *al = (double *)malloc(sizeof(double) * dk);
+    const size_t sidx = ((size_t)b_ * H + h) * (size_t)dv * dk;
+    if (J->S0)
+        memcpy(S, J->S0 + sidx, sizeof(double) * (size_t)dv * dk);
+    else
+        memset(S, 0, sizeof(double) * (size_t)dv * dk);
+    for (int t = 0; t < T; ++t) {
+        const size_t tok = ((size_t)b_ * T + t) * H + h;
+        for (int j = 0; j < dk; ++j) {
+            kk[j] = load_elem(J->k, tok * dk + j, J->in_dtype);
+            qq[j] = load_elem(J->q, tok * dk + j, J->in_dtype);
+            aa[j] = load_elem(J->a, tok * dk + j, J->in_dtype);
+            bb[j] = load_elem(J->b, tok * dk + j, J->in_dtype);
+            al[j] = exp((double)(J->gate_kind == OR_GATE_PER_CHANNEL ? J->g[tok * dk + j]
+                                                                      : J->g[tok]));
+        }
+        for (int i = 0; i < dv; ++i) {
+            double *Si = S + (size_t)i * dk;
+            double x = 0.0; /* S_{t-1} a, before the row changes */
+            for (int j = 0; j < dk; ++j) x += Si[j] * aa[j];
+            const double vi = load_elem(J->v, tok * dv + i, J->in_dtype);
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) {
+                Si[j] = Si[j] * al[j] + x * bb[j] + vi * kk[j];
+                acc += Si[j] * qq[j];
+            }
+            J->o[tok * dv + i] = acc;
+        }
+    }
+    if (J->S_T) memcpy(J->S_T + sidx, S, sizeof(double) * (size_t)dv * dk);
+    free(S); free(kk); free(qq); free(aa); free(bb); free(al);
+}
+
+static void *dplr_worker(void *arg) {
+    dplr_job_t *J = (dplr_job_t *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int w = J->next++;
+        pthread_mutex_unlock(&J->lock);
+        if (w >= J->B * J->H) break;
+        dplr_head(J, w / J->H, w % J->H);
+    }
+    return NULL;
+}
+
+int oracle_dplr_fwd(const void *q, const void *k, const void *v, const void *a, const void *b,
+                    int in_dtype, const float *g, int gate_kind, const double *S0, double *o,
+                    double *S_T, int B, int T, int H, int dk, int dv, int nthreads) {
+    if (!q || !k || !v || !a || !b || !g || !o) return -1;
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+    if (in_dtype != OR_F32 && in_dtype != OR_BF16) return -1;
+    if (gate_kind != OR_GATE_SCALAR && gate_kind != OR_GATE_PER_CHANNEL) return -1;
+    dplr_job_t J;
+    J.q = q; J.k = k; J.v = v; J.a = a; J.b = b; J.in_dtype = in_dtype;
+    J.g = g; J.gate_kind = gate_kind; J.S0 = S0; J.o = o; J.S_T = S_T;
+    J.B = B; J.T = T; J.H = H; J.dk = dk; J.dv = dv;
+    J.next = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    int n = nthreads;
+    if (n <= 0) n = 1;
+    if (n > B * H) n = B * H;
+    if (n <= 1) {
+        dplr_worker(&J);
+    } else {
+        pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * n);
+        for (int i = 0; i < n; ++i) pthread_create(&th[i], NULL, dplr_worker, &J);
+        for (int i = 0; i < n; ++i) pthread_join(th[i], NULL);
+        free(th);
+    }
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
