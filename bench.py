@@ -43,6 +43,7 @@ KERNEL_SOURCES = {
               "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
     "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu"],
     "bwd": ["gated_delta_rule_93_b200/csrc/gdr_bwd.cu"],
+    "dplr": ["gated_delta_rule_93_b200/csrc/gdr_dplr.cu"],
 }
 
 
@@ -56,6 +57,8 @@ def algorithmic_bytes(w):
                             + 4 * gate_elems + 4)
     beta = 0 if w.mixer == "gla" else 4
     per_tok = (2 * w.dk + w.dv) * e_in + w.dv * e_in + 4 * gate_elems + beta
+    if w.mixer == "dplr":  # q, k, a, b, v, g in; o out
+        per_tok = (4 * w.dk + w.dv) * e_in + w.dv * e_in + 4 * gate_elems
     if w.backward:  # q, k, v, g, beta, dL/do in; dq, dk, dv, dg, dbeta out (fp32)
         per_tok = ((2 * w.dk + w.dv) * e_in + 4 * gate_elems + 4 + 4 * w.dv
                    + 4 * (2 * w.dk + w.dv) + 4 * gate_elems + 4)
@@ -71,6 +74,8 @@ def algorithmic_flops(w, C=64):
         return w.B * w.H * 7.0 * w.dk * w.dv
     if w.backward:  # one recomputed forward step (5 d^2) and its reverse (16 d^2)
         return w.B * w.T * w.H * 21.0 * w.dk * w.dv
+    if w.mixer == "dplr":  # S.a and S.(alpha q) (4 d^2), S alpha + x b + v k (5 d^2)
+        return w.B * w.T * w.H * 9.0 * w.dk * w.dv
     if w.mixer == "gla":  # no correction: state update, S q, masked Q K^T and P V
         return w.B * w.T * w.H * (4 * w.dk * w.dv + C * (w.dk + w.dv))
     per = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0
@@ -243,6 +248,13 @@ def run_ours(args, rank, world, local_rank):
                 binding.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dout"], d["S0"],
                                   None, want_dS0=False, workspace=bws, out=grads)
 
+        if w.mixer == "dplr":  # recurrent DPLR forward on CUDA cores: one launch
+            launches_per_step = 1
+
+            def step():
+                binding.dplr_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["g"], d["S0"], o=o,
+                                 S_T=S_T, output_final_state=S_T is not None)
+
         if w.mixer == "gla":  # gated linear attention: one launch, no beta, no workspace
             host.pop("beta")
             d.pop("beta")
@@ -343,8 +355,9 @@ def run_ours(args, rank, world, local_rank):
     avg_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
     achieved = abytes / (avg_launch_ms / 1e3) / 1e9
     roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (tc_peak * 1e12)) * 1e3
-    if w.backward:  # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x SM clock
-        alu_peak = 148 * 128 * 2 * (clk.get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
+    alu = w.backward or w.mixer == "dplr"
+    if alu:  # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x SM clock
+        alu_peak = 148 * 128 * 2 * ((clk or {}).get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
         roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (alu_peak * 1e12)) * 1e3
     line = {
         "metric": METRIC,
@@ -373,10 +386,11 @@ def run_ours(args, rank, world, local_rank):
         "roofline": ({"bound": "alu", "achieved": aflops / (avg_launch_ms / 1e3) / 1e12,
                       "peak": alu_peak, "unit": "TFLOP/s",
                       "frac": aflops / (avg_launch_ms / 1e3) / 1e12 / alu_peak,
-                      "traffic": recorded_traffic(w.name, "bwd"),
+                      "traffic": recorded_traffic(w.name, "dplr" if w.mixer == "dplr" else "bwd"),
                       "peak_source": "CUDA-core fp32 FMA, 148 SMs x 128 lanes "
                       "x 2 flop x max SM clock", "algorithmic_flops_per_launch": aflops,
-                      "kernel": "gdr_chunk_bwd"} if w.backward else
+                      "kernel": "gdr_dplr_fwd" if w.mixer == "dplr" else "gdr_chunk_bwd"}
+                     if alu else
                      {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
                      "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
@@ -407,6 +421,8 @@ def _oracle_sample(w, inp, Tp):
         return qkv + [sl["a"].numpy(), sl["b"].numpy(), sl["gate_scale"].numpy(), S0]
     if w.backward:
         return qkv + [sl["g"].numpy(), sl["beta"].numpy(), sl["dout"].double().numpy(), S0]
+    if w.mixer == "dplr":
+        return qkv + [to_numpy_input(sl["a"]), to_numpy_input(sl["b"]), sl["g"].numpy(), S0]
     return qkv + [sl["g"].numpy(), sl["beta"].numpy(), S0]
 
 
@@ -416,6 +432,8 @@ def _oracle_fwd(oracle, w, a, n):
         return oracle.gdr_fwd_prologue(*a, gate=w.gate, nthreads=n)
     if w.backward:
         return oracle.gdr_bwd(*a, gate=w.gate, nthreads=n)
+    if w.mixer == "dplr":
+        return oracle.dplr_fwd(*a, gate=w.gate, nthreads=n)
     if w.mixer == "gla":
         return oracle.gla_fwd(a[0], a[1], a[2], a[3], a[5], gate=w.gate, nthreads=n)
     return oracle.gdr_fwd(*a, gate=w.gate, nthreads=n)

@@ -15,6 +15,7 @@ from .binding import (  # noqa: F401
     chunk_fwd_segmented,
     chunk_fwd_varlen,
     chunk_fwd_workspace_bytes,
+    dplr_fwd,
     device_status,
     lib,
     status_string,
@@ -22,5 +23,5 @@ from .binding import (  # noqa: F401
 )
 
 __all__ = ["chunk_bwd", "chunk_bwd_workspace_bytes", "chunk_fwd", "chunk_fwd_gla", "chunk_fwd_prologue", "chunk_fwd_kernel_launches", "chunk_fwd_segmented", "chunk_fwd_varlen",
-           "chunk_fwd_workspace_bytes", "step", "device_status", "lib", "status_string",
+           "chunk_fwd_workspace_bytes", "dplr_fwd", "step", "device_status", "lib", "status_string",
            "GdrError"]

@@ -34,6 +34,7 @@ EXPORTS = (
     "gdr_chunk_fwd_prologue",
     "gdr_chunk_bwd_workspace_bytes",
     "gdr_chunk_bwd",
+    "gdr_dplr_fwd",
     "gdr_step",
     "gdr_get_device_status",
     "gdr_status_string",
@@ -84,6 +85,9 @@ def lib():
             L.gdr_chunk_bwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                         vp, i, i, i, i, i, vp, sz, vp]
             L.gdr_chunk_bwd.restype = i
+            L.gdr_dplr_fwd.argtypes = [vp, vp, vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, i,
+                                       vp]
+            L.gdr_dplr_fwd.restype = i
             L.gdr_step.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, i, i, i, i, vp]
             L.gdr_step.restype = i
             L.gdr_get_device_status.argtypes = [vp]
@@ -446,3 +450,39 @@ def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, *, want_dS0=True, work
                                  if workspace is not None else 0, _stream_handle(stream))
     _check(rc)
     return out
+
+
+def dplr_fwd(q, k, v, a, b, g, S0=None, *, output_final_state=True, o=None, S_T=None,
+             stream=None):
+    """``gdr_dplr_fwd``: S_t = S_{t-1}(Diag(alpha_t) + a_t b_t^T) + v_t k_t^T,
+    o_t = S_t q_t.  q, k, a, b [B,T,H,d]; v [B,T,H,d] (one dtype); g [B,T,H]
+    or [B,T,H,d] fp32; S0 [B,H,d,d] fp32 or None.  Returns (o, S_T or None)."""
+    _need(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    for t_, n_ in ((k, "k"), (a, "a"), (b, "b")):
+        _need(t_, n_, dt, (B, T, H, dk), dev)
+    _need(v, "v", dt, (B, T, H, dv), dev)
+    if g.dim() == 4:
+        _need(g, "g", torch.float32, (B, T, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (B, T, H), dev)
+        gk = GDR_GATE_SCALAR
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _need(o, "o", dt, (B, T, H, dv), dev)
+    if output_final_state and S_T is None:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_dplr_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _in_dtype(dt),
+                                _ptr(g), gk, _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv,
+                                _stream_handle(stream))
+    _check(rc)
+    return o, S_T

@@ -326,6 +326,29 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
   return from_cuda(gdr::launch_chunk_tc(ca, s), "gdr_chunk_fwd_prologue launch");
 }
 
+gdr_status gdr_dplr_fwd(const void *q, const void *k, const void *v, const void *a,
+                        const void *b, gdr_dtype in_dtype, const float *g, gdr_gate_kind gate,
+                        const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
+                        int dv, gdr_stream_t stream) {
+  if (B < 0 || T < 0 || H < 0) return fail(GDR_ERR_INVALID_ARG, "negative B/T/H");
+  if (in_dtype != GDR_F32 && in_dtype != GDR_BF16)
+    return fail(GDR_ERR_INVALID_ARG, "in_dtype must be GDR_F32 or GDR_BF16");
+  if (gate != GDR_GATE_SCALAR && gate != GDR_GATE_PER_CHANNEL)
+    return fail(GDR_ERR_INVALID_ARG, "unknown gate kind");
+  if (dk != dv || (dk != 32 && dk != 64 && dk != 128))
+    return fail(GDR_ERR_UNSUPPORTED, "DPLR needs dk = dv in {32, 64, 128} (got %d, %d)", dk, dv);
+  if ((size_t)B * (size_t)H * (size_t)T > (size_t)1 << 40)
+    return fail(GDR_ERR_INVALID_ARG, "problem too large");
+  if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "B*H too large");
+  if ((size_t)B * H * T != 0 && (!q || !k || !v || !a || !b || !g || !o))
+    return fail(GDR_ERR_INVALID_ARG, "null q/k/v/a/b/g/o");
+  if ((size_t)B * H == 0) return ok();
+  return from_cuda(gdr::launch_dplr(q, k, v, a, b, in_dtype == GDR_BF16, g,
+                                    gate == GDR_GATE_PER_CHANNEL, S0, o, S_T, B, T, H, dk,
+                                    reinterpret_cast<cudaStream_t>(stream)),
+                   "gdr_dplr_fwd launch");
+}
+
 size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
   if (dk != dv || (dk != 32 && dk != 64 && dk != 128)) return 0;
   return gdr::bwd_ws_bytes(B, T, H, dk);

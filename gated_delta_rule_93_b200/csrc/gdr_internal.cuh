@@ -71,6 +71,11 @@ bool chunk_tc_supports(const ChunkArgs &a);
 int chunk_segments(const ChunkArgs &a, int num_sms);
 size_t chunk_segments_ws_bytes(const ChunkArgs &a, int P);
 cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStream_t stream);
+// DPLR transition, recurrent forward (CUDA cores, d_k = d_v = d in {32, 64, 128}).
+cudaError_t launch_dplr(const void *q, const void *k, const void *v, const void *a,
+                        const void *b, int bf16, const float *g, int per_channel,
+                        const float *S0, void *o, float *S_T, int B, int T, int H, int d,
+                        cudaStream_t stream);
 // Backward of the recurrence (CUDA cores, d_k = d_v = d in {32, 64, 128}).
 size_t bwd_ws_bytes(int B, int T, int H, int d);
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, int bf16, const float *g,

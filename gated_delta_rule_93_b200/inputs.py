@@ -40,7 +40,8 @@ class Workload:
     want_S_T: bool
     steps: int = 1  # decode workloads: consecutive steps
     C: int = 64
-    mixer: str = "gdr"  # "gdr" (delta rule) or "gla" (gated linear attention, beta unused)
+    mixer: str = "gdr"  # "gdr" (delta rule), "gla" (gated linear attention, beta unused)
+    #                     or "dplr" (diagonal-plus-low-rank transition)
     prologue: bool = False  # raw projections in: q, k unnormalised, gate / beta logits
     backward: bool = False  # gradients (gdr_chunk_bwd) for a seeded dL/do
     note: str = field(default="", compare=False)
@@ -68,6 +69,9 @@ WORKLOADS = {
         Workload("gla_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
                  "scalar", False, True, mixer="gla",
                  note="gated linear attention forward at the same shape (additive writes)"),
+        Workload("dplr_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
+                 "scalar", False, True, mixer="dplr",
+                 note="diagonal-plus-low-rank transition forward at the same shape"),
         Workload("gdn_bwd_b8_t4096_h16_d128", "chunk", 8, 4096, 16, 128, 128, torch.bfloat16,
                  "scalar", False, False, backward=True,
                  note="Gated DeltaNet backward at the 350M shape (dL/do ~ N(0, 1) fp32)"),
@@ -95,6 +99,21 @@ def make_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, gate="scalar", with
     beta = torch.sigmoid(torch.randn(B, T, H, generator=gen))
     S0 = 0.02 * torch.randn(B, H, dv, dk, generator=gen) if with_S0 else None
     return dict(q=q, k=k, v=v, g=g.float(), beta=beta.float(), S0=S0)
+
+
+def make_dplr_inputs(B, T, H, d, dtype=torch.bfloat16, gate="scalar", with_S0=False, seed=0):
+    """Inputs for ``gdr_dplr_fwd``: the ``make_chunk_inputs`` draws (q, k, v, g,
+    beta, S0) plus an erase direction b (unit rows of N(0, 1), its own
+    stream), and a = -beta e^{g} b (per channel, or the head's scalar gate),
+    so that each transition Diag(alpha)(I - beta b b^T) is a contraction and
+    long sequences stay bounded.  Returns dict q, k, v, a, b, g, S0."""
+    d_ = make_chunk_inputs(B, T, H, d, d, dtype, gate, with_S0, seed)
+    gen = torch.Generator().manual_seed(seed + 15485863)
+    b = _unit_rows(torch.randn(B, T, H, d, generator=gen))
+    al = torch.exp(d_["g"] if gate == "channel" else d_["g"][..., None])
+    a = -d_["beta"][..., None] * al * b
+    return dict(q=d_["q"], k=d_["k"], v=d_["v"], a=a.to(dtype), b=b.to(dtype), g=d_["g"],
+                S0=d_["S0"])
 
 
 def make_raw_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, with_S0=False, seed=0,
@@ -162,6 +181,8 @@ def make_step_inputs(N, H, dk, dv, steps, dtype=torch.bfloat16, gate="scalar", s
 def make_workload_inputs(w: Workload, seed=0, steps=None):
     if w.kind == "chunk" and w.prologue:
         return make_raw_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.with_S0, seed)
+    if w.kind == "chunk" and w.mixer == "dplr":
+        return make_dplr_inputs(w.B, w.T, w.H, w.dk, w.dtype, w.gate, w.with_S0, seed)
     if w.kind == "chunk" and w.backward:
         d = make_chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.gate, w.with_S0, seed)
         gen = torch.Generator().manual_seed(seed + 104729)

@@ -228,6 +228,29 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
                                   int norm_qk, gdr_stream_t stream);
 
 /*
+ * Diagonal-plus-low-rank (DPLR) transition, the generalised sibling of the
+ * delta rule: "Decoding Hybrid Linear Attention Architectures", section 3
+ * item 5:
+ *
+ *   S_t = S_{t-1} (Diag(alpha_t) + a_t b_t^T) + v_t k_t^T,   o_t = S_t q_t
+ *
+ * (alpha_t = e^{g_t}, one per head or one per key channel; with
+ * a = -beta (alpha . k), b = k and beta v it is the gated delta rule).
+ *
+ *   q, k, a, b  [B, T, H, dk] in_dtype;  v, o [B, T, H, dv] in_dtype
+ *   g           [B, T, H] or [B, T, H, dk] fp32
+ *   S0, S_T     [B, H, dv, dk] fp32 or NULL (zero state / not written)
+ *
+ * A recurrent forward on CUDA cores in fp32 (one CTA per (b, h)), for
+ * dk = dv in {32, 64, 128} (GDR_ERR_UNSUPPORTED otherwise).  One launch, no
+ * workspace; S0 may alias S_T.
+ */
+gdr_status gdr_dplr_fwd(const void *q, const void *k, const void *v, const void *a,
+                        const void *b, gdr_dtype in_dtype, const float *g, gdr_gate_kind gate,
+                        const float *S0, void *o, float *S_T, int B, int T, int H, int dk,
+                        int dv, gdr_stream_t stream);
+
+/*
  * Backward of the chunked forward (training): the gradients of q, k, v,
  * g = log alpha, beta and S0 from dL/do and dL/dS_T.  "Decoding Hybrid
  * Linear Attention Architectures", section 5: backpropagation through the

@@ -50,8 +50,15 @@ def test_status_strings(L):
 
 def test_workspace_query(L):
     assert L.gdr_chunk_fwd_workspace_bytes(8, 4096, 16, 128, 128, 64, 1, 0) == 0
-    # the segment path depends on the device's SM count: none without a GPU
-    assert L.gdr_chunk_fwd_workspace_bytes(1, 65536, 16, 128, 128, 64, 1, 0) == 0
+    # the segment path depends on the device's SM count: none without a GPU,
+    # three fp32 states per segment and head with one
+    import torch
+
+    ws = L.gdr_chunk_fwd_workspace_bytes(1, 65536, 16, 128, 128, 64, 1, 0)
+    if torch.cuda.is_available():
+        assert ws > 0 and ws % (3 * 16 * 128 * 128 * 4) == 0
+    else:
+        assert ws == 0
     assert L.gdr_chunk_fwd_kernel_launches(8, 4096, 16, 128, 128, 64, 1, 0) == 1
     assert L.gdr_chunk_fwd_kernel_launches(0, 4096, 16, 128, 128, 64, 1, 0) == 0
 
@@ -231,3 +238,24 @@ def test_backward_validation_rejects_before_any_launch(L):
     assert call(ws=None) == binding.GDR_ERR_WORKSPACE
     assert call(ws=_fake_ptr(4)) == binding.GDR_ERR_INVALID_ARG
     assert call(H=0) == binding.GDR_OK
+
+
+def test_dplr_validation_rejects_before_any_launch(L):
+    p = _fake_ptr()
+
+    def call(**kw):
+        a = dict(q=p, k=p, v=p, a=p, b=p, dt=1, g=p, gate=0, S0=None, o=p, ST=None, B=2, T=100,
+                 H=2, dk=64, dv=64, st=None)
+        a.update(kw)
+        return L.gdr_dplr_fwd(a["q"], a["k"], a["v"], a["a"], a["b"], a["dt"], a["g"], a["gate"],
+                              a["S0"], a["o"], a["ST"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                              a["st"])
+
+    assert call(T=-1) == binding.GDR_ERR_INVALID_ARG
+    assert call(dt=7) == binding.GDR_ERR_INVALID_ARG
+    assert call(gate=2) == binding.GDR_ERR_INVALID_ARG
+    assert call(dk=64, dv=32) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dk=48, dv=48) == binding.GDR_ERR_UNSUPPORTED
+    assert call(a=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(b=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(B=0) == binding.GDR_OK

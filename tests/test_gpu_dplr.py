@@ -1,0 +1,69 @@
+"""GPU parity of gdr_dplr_fwd (the diagonal-plus-low-rank transition) against
+the fp64 oracle.  The kernel keeps the state in fp32 and computes in fp32 on
+the same inputs; o is rounded to the input dtype.  Bars: o within 2e-2 for
+bf16 inputs (its rounding) and 1e-4 for fp32; S_T within 1e-4."""
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_93_b200 import binding
+from gated_delta_rule_93_b200.inputs import make_dplr_inputs, to_numpy_input
+from tests._gpu_util import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, dev):
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    o, S_T = binding.dplr_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["g"], d["S0"])
+    torch.cuda.synchronize(dev)
+    return o, S_T
+
+
+def _oracle(inp):
+    gate = "channel" if inp["g"].dim() == 4 else "scalar"
+    S0 = None if inp["S0"] is None else inp["S0"].double().numpy()
+    return oracle.dplr_fwd(*(to_numpy_input(inp[x]) for x in ("q", "k", "v", "a", "b")),
+                           inp["g"].numpy(), S0, gate=gate)
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("with_S0", [True, False])
+def test_dplr_matches_oracle_d128_bf16(cuda_device, gate, with_S0):
+    inp = make_dplr_inputs(2, 150, 2, 128, torch.bfloat16, gate, with_S0, seed=140)
+    o, S_T = _run(inp, cuda_device)
+    ro, rS = _oracle(inp)
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S_T, rS, 1e-4, "S_T")
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_dplr_matches_oracle_fp32(cuda_device, d):
+    inp = make_dplr_inputs(2, 70, 3, d, torch.float32, "channel", True, seed=141 + d)
+    o, S_T = _run(inp, cuda_device)
+    ro, rS = _oracle(inp)
+    assert_close(o, ro, 1e-4, "o")
+    assert_close(S_T, rS, 1e-4, "S_T")
+
+
+def test_dplr_with_delta_parameters_equals_chunked_delta_rule(cuda_device):
+    """a = -beta (alpha . k), b = k, v -> beta v gives the gated delta rule:
+    the recurrent DPLR kernel against the tensor-core chunked forward."""
+    from gated_delta_rule_93_b200.inputs import make_chunk_inputs
+    inp = make_chunk_inputs(2, 200, 2, 128, 128, torch.bfloat16, "scalar", True, seed=143)
+    d = {k: v.to(cuda_device) for k, v in inp.items()}
+    al = torch.exp(d["g"])[..., None]
+    a = (-d["beta"][..., None] * al * d["k"].float()).to(torch.bfloat16)
+    vb = (d["beta"][..., None] * d["v"].float()).to(torch.bfloat16)
+    o, S_T = binding.dplr_fwd(d["q"], d["k"], vb, a, d["k"], d["g"], d["S0"])
+    oc, Sc = binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    torch.cuda.synchronize()
+    e_o = (o.float() - oc.float()).abs().max() / oc.float().abs().max()
+    e_S = (S_T - Sc).abs().max() / Sc.abs().max()
+    assert e_o < 2e-2 and e_S < 2e-2
+
+
+def test_dplr_empty_sequence(cuda_device):
+    inp = make_dplr_inputs(1, 0, 2, 64, torch.float32, "scalar", True, seed=144)
+    _, S_T = _run(inp, cuda_device)
+    assert torch.equal(S_T.cpu(), inp["S0"])
