@@ -94,3 +94,91 @@ def chunk_fwd(q, k, v, g, beta, S0=None, C=64):
             o[b, :, h] = ob
             S_T[b, h] = sb
     return o, S_T
+
+
+def chunk_bwd_head(q, k, v, g, beta, dO, S0=None, dS_T=None, C=64):
+    """Gradients of ``chunk_fwd_head`` by reverse mode through the chunk
+    equations ("Decoding Hybrid Linear Attention Architectures", section 5:
+    backpropagation through the chunked recurrence, with the chunk's
+    quantities recomputed), written as matrix products per chunk: the form a
+    chunked backward kernel computes.  Pinned to the token-level backward
+    ``oracle.gdr_bwd``.
+
+    One (batch, head): q, k [T,dk]; v, dO [T,dv]; g [T] or [T,dk]; beta [T];
+    S0, dS_T [dv,dk] or None.  Returns dict dq, dk, dv, dg (shape of g),
+    dbeta, dS0.
+
+    Per chunk (forward notation above; Y = (I + A)^{-1}, T = Y Diag(beta)),
+    from dO and dX1 = dL/dX after the chunk:
+        dV'  = P^T dO + K- dX1
+        dX0  = Q~^T dO + Diag(b_L) dX1 - W^T dV'
+        dP   = tril_incl(dO V'^T):  dQ~ = dO X0^T + dP K^,  dK^ = dP^T Q~
+        dK-  = V' dX1^T
+        dT   = dV' V^T - dV' X0^T K~^T;  dV = T^T dV';  dK~ = -T^T dV' X0^T
+        dY   = dT Diag(beta);  dbeta += diag(Y^T dT) (column sums of Y . dT)
+        dA   = strict_tril(-Y^T dY Y^T):  dbeta_r += sum_s dA M,
+               dK~ += Diag(beta) dA K^,  dK^ += (Diag(beta) dA)^T K~   (M = K~ K^^T)
+    then through K~ = K b, K^ = K / b, Q~ = Q b, K- = K b_L / b, b = e^{gc},
+    gc = cumsum(g) (and b_L = b of the last row, which also scales X0).
+    """
+    q, k, v = _widen(q), _widen(k), _widen(v)
+    g = np.asarray(g, np.float64)
+    beta = np.asarray(beta, np.float64)
+    dO = np.asarray(dO, np.float64)
+    T, dk = q.shape
+    dv = v.shape[1]
+    scalar = g.ndim == 1
+    _, _, st = chunk_fwd_head(q, k, v, g, beta, S0, C, keep_stages=True)
+    out = dict(dq=np.zeros((T, dk)), dk=np.zeros((T, dk)), dv=np.zeros((T, dv)),
+               dg=np.zeros(g.shape), dbeta=np.zeros(T))
+    dX = np.zeros((dk, dv)) if dS_T is None else np.array(dS_T, np.float64).T.copy()
+    for ci in range(len(st) - 1, -1, -1):
+        c0 = ci * C
+        s = st[ci]
+        L = s["O"].shape[0]
+        Q, K, V, bt = q[c0:c0 + L], k[c0:c0 + L], v[c0:c0 + L], beta[c0:c0 + L]
+        b = np.exp(s["g"])
+        if b.ndim == 1:
+            b = np.repeat(b[:, None], dk, axis=1)
+        bL = b[L - 1]
+        Kt, Kh, Qt, Kb = K * b, K / b, Q * b, K * (bL[None, :] / b)
+        X0, Vp, P, W, Tm = s["X0"], s["Vp"], s["P"], s["W"], s["T"]
+        Y = np.linalg.inv(np.eye(L) + s["A"])
+        dOc = dO[c0:c0 + L]
+        dX1 = dX
+        dVp = P.T @ dOc + Kb @ dX1
+        dX0 = Qt.T @ dOc + bL[:, None] * dX1 - W.T @ dVp
+        dP = np.tril(dOc @ Vp.T, 0)
+        dQt = dOc @ X0.T + dP @ Kh
+        dKh = dP.T @ Qt
+        dKb = Vp @ dX1.T
+        dbL = np.sum(dX1 * X0, axis=1)
+        dW = -dVp @ X0.T
+        dTm = dVp @ V.T + dW @ Kt.T
+        dV = Tm.T @ dVp
+        dKt = Tm.T @ dW
+        dY = dTm * bt[None, :]
+        dbeta = np.sum(Y * dTm, axis=0)
+        dA = np.tril(-(Y.T @ dY @ Y.T), -1)
+        M = Kt @ Kh.T
+        dbeta += np.sum(dA * M, axis=1)
+        dM = bt[:, None] * dA
+        dKt += dM @ Kh
+        dKh += dM.T @ Kt
+        dK = dKt * b + dKh / b + dKb * (bL[None, :] / b)
+        dQ = dQt * b
+        db = dKt * K - dKh * K / b ** 2 + dQt * Q - dKb * K * bL[None, :] / b ** 2
+        dbL = dbL + np.sum(dKb * K / b, axis=0)
+        dgc = db * b
+        dgc[L - 1] += dbL * bL
+        if scalar:
+            dgc = dgc.sum(axis=1)
+        dgs = np.cumsum(dgc[::-1], axis=0)[::-1]  # gc = cumsum(g)
+        out["dq"][c0:c0 + L] = dQ
+        out["dk"][c0:c0 + L] = dK
+        out["dv"][c0:c0 + L] = dV
+        out["dg"][c0:c0 + L] = dgs
+        out["dbeta"][c0:c0 + L] = dbeta
+        dX = dX0
+    out["dS0"] = dX.T.copy()
+    return out

@@ -83,3 +83,23 @@ def test_backward_beta_zero_is_pure_decay():
     for t in range(T):
         want = want + np.outer(Wo[0, t, 0], q[0, t, 0].astype(np.float64) * np.exp(cum[t]))
     assert np.max(np.abs(grads["dS0"][0, 0] - want)) < 1e-12 * np.max(np.abs(want))
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_chunked_backward_matches_token_backward(gate):
+    """The chunk-level reverse mode (matrix products per chunk, the form of a
+    chunked backward kernel) equals the token-level backward: C = 16 over 40
+    tokens (two full chunks and a ragged tail)."""
+    from oracle import chunked
+
+    B, T, H, dk, dv = 1, 40, 1, 6, 5
+    q, k, v, g, beta, s0 = _inputs(B, T, H, dk, dv, gate)
+    Wo = RNG.standard_normal((B, T, H, dv))
+    WS = RNG.standard_normal((B, H, dv, dk))
+    ref = oracle.gdr_bwd(q, k, v, g, beta, Wo, s0, WS, gate=gate, nthreads=1)
+    got = chunked.chunk_bwd_head(q[0, :, 0], k[0, :, 0], v[0, :, 0], g[0, :, 0], beta[0, :, 0],
+                                 Wo[0, :, 0], s0[0, 0], WS[0, 0], C=16)
+    for name in ("dq", "dk", "dv", "dg", "dbeta"):
+        r = ref[name][0, :, 0]
+        assert np.max(np.abs(got[name] - r)) <= 1e-9 * max(1.0, np.max(np.abs(r))), name
+    assert np.max(np.abs(got["dS0"] - ref["dS0"][0, 0])) <= 1e-9 * np.max(np.abs(ref["dS0"]))
