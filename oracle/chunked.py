@@ -182,3 +182,47 @@ def chunk_bwd_head(q, k, v, g, beta, dO, S0=None, dS_T=None, C=64):
         dX = dX0
     out["dS0"] = dX.T.copy()
     return out
+
+
+def dplr_chunk_fwd_head(q, k, v, a, b, g, S0=None, C=64):
+    """Chunk form of the diagonal-plus-low-rank recurrence ("Decoding Hybrid
+    Linear Attention Architectures", section 3 item 5, chunked as section 5
+    chunks the delta rule), one (batch, head), state S [dv, dk]:
+
+        S_r = S_{r-1} (Diag(alpha_r) + a_r b_r^T) + v_r k_r^T,   o_r = S_r q_r.
+
+    Within a chunk, with e_r = prod_{u<=r} alpha_u (from the chunk start,
+    e_{-1} = 1), the low-rank reads x_r = S_{r-1} a_r satisfy
+        x_r = S_0 a^_r + sum_{s<r} x_s (b^_s . a^_r) + sum_{s<r} v_s (k^_s . a^_r),
+        a^_r = a_r e_{r-1},  b^_s = b_s / e_s,  k^_s = k_s / e_s,
+    a unit lower-triangular system (the delta rule's WY structure with the
+    erase direction b and the write key k kept apart):
+        X = (I - strict_tril(A^ B^^T))^{-1} (A^ S_0^T + strict_tril(A^ K^^T) V)
+    and then, with q~_r = q_r e_r,
+        O   = Q~ S_0^T + tril_incl(Q~ B^^T) X + tril_incl(Q~ K^^T) V
+        S_L^T = Diag(e_L) S_0^T + (B e_L / e)^T X + (K e_L / e)^T V.
+    q, k, a, b [T,dk]; v [T,dv]; g [T] or [T,dk]; S0 [dv,dk] or None.
+    Returns (o [T,dv], S_T [dv,dk]).  Pinned to ``oracle.dplr_fwd``."""
+    q, k, v, a, b = (_widen(x) for x in (q, k, v, a, b))
+    g = np.asarray(g, np.float64)
+    T, dk = q.shape
+    dv = v.shape[1]
+    St = np.zeros((dk, dv)) if S0 is None else np.array(S0, np.float64).T.copy()  # S^T
+    o = np.zeros((T, dv))
+    for c0 in range(0, T, C):
+        c1 = min(T, c0 + C)
+        L = c1 - c0
+        Q, K, V, Aa, Bb = q[c0:c1], k[c0:c1], v[c0:c1], a[c0:c1], b[c0:c1]
+        e = np.exp(np.cumsum(g[c0:c1], axis=0))
+        if e.ndim == 1:
+            e = np.repeat(e[:, None], dk, axis=1)
+        eprev = np.vstack([np.ones((1, dk)), e[:-1]])
+        Ah, Bh, Kh, Qt = Aa * eprev, Bb / e, K / e, Q * e
+        Lb = np.tril(Ah @ Bh.T, -1)
+        Lk = np.tril(Ah @ Kh.T, -1)
+        X = np.linalg.solve(np.eye(L) - Lb, Ah @ St + Lk @ V)
+        O = Qt @ St + np.tril(Qt @ Bh.T, 0) @ X + np.tril(Qt @ Kh.T, 0) @ V
+        eL = e[L - 1]
+        St = eL[:, None] * St + (Bb * (eL[None, :] / e)).T @ X + (K * (eL[None, :] / e)).T @ V
+        o[c0:c1] = O
+    return o, St.T.copy()

@@ -70,3 +70,17 @@ def test_dplr_without_low_rank_is_gla(gate):
     o, S_T = oracle.dplr_fwd(q, k, v, a, b, g, s0, gate=gate)
     ol, Sl = oracle.gla_fwd(q, k, v, g, s0, gate=gate)
     assert rel_err(o, ol) < 1e-13 and rel_err(S_T, Sl) < 1e-13
+
+
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+def test_dplr_chunk_form_matches_recurrence(gate):
+    """The chunk form (a unit lower-triangular solve for the low-rank reads,
+    then the chunk's output and end state as matrix products) equals the
+    recurrence: C = 16 over 40 tokens (two chunks and a ragged tail)."""
+    from oracle import chunked
+
+    q, k, v, a, b, g, s0 = _inputs(1, 40, 1, 6, 5, gate)
+    o, S_T = oracle.dplr_fwd(q, k, v, a, b, g, s0, gate=gate)
+    oc, Sc = chunked.dplr_chunk_fwd_head(q[0, :, 0], k[0, :, 0], v[0, :, 0], a[0, :, 0],
+                                         b[0, :, 0], g[0, :, 0], s0[0, 0], C=16)
+    assert rel_err(oc, o[0, :, 0]) < 1e-10 and rel_err(Sc, S_T[0, 0]) < 1e-10
