@@ -259,3 +259,24 @@ def test_dplr_validation_rejects_before_any_launch(L):
     assert call(a=None) == binding.GDR_ERR_INVALID_ARG
     assert call(b=None) == binding.GDR_ERR_INVALID_ARG
     assert call(B=0) == binding.GDR_OK
+
+
+def test_every_binding_refuses_cpu_tensors(L):
+    """No entry has a CPU path: each raises before reaching the library."""
+    import torch
+
+    x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
+    g = torch.zeros(1, 64, 1)
+    calls = [
+        lambda: binding.chunk_fwd_gla(x, x, x, g),
+        lambda: binding.chunk_fwd_prologue(x, x, x, g, g, torch.ones(1)),
+        lambda: binding.chunk_bwd(x, x, x, g, g, torch.zeros(1, 64, 1, 128)),
+        lambda: binding.dplr_fwd(x, x, x, x, x, g),
+        lambda: binding.chunk_fwd_segmented(x, x, x, g, g, segments=2,
+                                            workspace=torch.zeros(16, dtype=torch.uint8)),
+        lambda: binding.step(x[:, 0], x[:, 0], x[:, 0], g[:, 0], g[:, 0],
+                             torch.zeros(1, 1, 128, 128)),
+    ]
+    for i, call in enumerate(calls):
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
