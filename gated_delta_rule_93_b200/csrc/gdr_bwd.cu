@@ -20,8 +20,8 @@
 // recomputed from their checkpoint into a stash and walked in reverse.
 // Both live in the caller's workspace, element-major ([element][thread], so
 // a warp's access is one contiguous 128-byte line; each thread reads back
-// only what it wrote); the stashes of all CTAs (64 KB per token and head at
-// d = 128) stay within L2.  The token vectors of a 64-token
+// only what it wrote); a stash holds 8 states of 64 KB at d = 128, each read
+// back within 8 tokens of being written.  The token vectors of a 64-token
 // chunk (k, q, v, g, beta, dL/do) are staged in shared memory as fp32 by
 // the whole CTA with coalesced loads before the chunk is processed.
 #include "gdr_internal.cuh"
