@@ -449,15 +449,18 @@ def cpu_baseline(w, target_s=12.0):
     oracle.build()
     inp = make_workload_inputs(w)
     n = min(oracle.default_threads(), w.B * w.H)
+    # the oracle backward keeps every state of a head (2 x 128 KB per token at
+    # d = 128, per thread): its sample stops at 512 tokens
+    t_cap = min(w.T, 512) if w.backward else w.T
     Tp = 16
     while True:
         args = _oracle_sample(w, inp, Tp)
         t = time.perf_counter()
         _oracle_fwd(oracle, w, args, n)
         el = time.perf_counter() - t
-        if el >= target_s / 4 or Tp >= w.T:
+        if el >= target_s / 4 or Tp >= t_cap:
             break
-        Tp = min(w.T, max(Tp * 2, int(Tp * (target_s / 3) / max(el, 1e-3))))
+        Tp = min(t_cap, max(Tp * 2, int(Tp * (target_s / 3) / max(el, 1e-3))))
     return {"value": w.B * Tp / el, "unit": "tokens/s", "cores": n, "kind": "oracle",
             "sample": f"all {w.B}x{w.H} (b,h) pairs, first {Tp} of {w.T} tokens "
                       f"({el:.2f} s wall, fp64 C recurrence, {n} threads)"}
