@@ -426,3 +426,24 @@ def test_gla_split_and_resume(gate):
     oa, Sa = oracle.gla_fwd(q[:, :7], k[:, :7], v[:, :7], g[:, :7], s0, gate=gate)
     ob, Sb = oracle.gla_fwd(q[:, 7:], k[:, 7:], v[:, 7:], g[:, 7:], Sa, gate=gate)
     assert rel_err(np.concatenate([oa, ob], axis=1), o) < 1e-12 and rel_err(Sb, ST) < 1e-12
+
+
+def test_oracle_siblings_regression_fixture():
+    """GLA, DPLR, backward and prologue still reproduce the fixture their own
+    script wrote (guards against silent change; not an independent pin)."""
+    import json
+    import os
+    import sys
+
+    here = os.path.join(os.path.dirname(__file__), "golden")
+    sys.path.insert(0, here)
+    try:
+        import make_golden_siblings as mg
+    finally:
+        sys.path.remove(here)
+    with open(os.path.join(here, "oracle_siblings_tiny.json")) as f:
+        fx = json.load(f)
+    x = {k: np.array(v, np.float32) for k, v in fx["inputs"].items()}
+    got = mg.results(x)
+    for name, want in fx["results"].items():
+        assert np.allclose(np.asarray(got[name]), np.array(want), rtol=0, atol=1e-13), name
