@@ -103,3 +103,19 @@ def test_chunked_backward_matches_token_backward(gate):
         r = ref[name][0, :, 0]
         assert np.max(np.abs(got[name] - r)) <= 1e-9 * max(1.0, np.max(np.abs(r))), name
     assert np.max(np.abs(got["dS0"] - ref["dS0"][0, 0])) <= 1e-9 * np.max(np.abs(ref["dS0"]))
+
+
+def test_scalar_gate_gradient_is_the_channel_sum():
+    """A per-channel gate equal in every channel is the scalar gate: the same
+    dq, dk, dv, dbeta, dS0, and the scalar dg is the sum of the per-channel
+    dg over channels (the decay multiplies every channel)."""
+    B, T, H, dk, dv = 1, 9, 2, 4, 3
+    q, k, v, g, beta, s0 = _inputs(B, T, H, dk, dv, "scalar")
+    gc = np.repeat(g[..., None], dk, axis=-1)
+    Wo = RNG.standard_normal((B, T, H, dv))
+    WS = RNG.standard_normal((B, H, dv, dk))
+    a = oracle.gdr_bwd(q, k, v, g, beta, Wo, s0, WS, gate="scalar")
+    c = oracle.gdr_bwd(q, k, v, gc, beta, Wo, s0, WS, gate="channel")
+    for name in ("dq", "dk", "dv", "dbeta", "dS0"):
+        assert np.max(np.abs(a[name] - c[name])) <= 1e-12 * np.max(np.abs(c[name])), name
+    assert np.max(np.abs(a["dg"] - c["dg"].sum(axis=-1))) <= 1e-12 * np.max(np.abs(a["dg"]))

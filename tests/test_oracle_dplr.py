@@ -84,3 +84,16 @@ def test_dplr_chunk_form_matches_recurrence(gate):
     oc, Sc = chunked.dplr_chunk_fwd_head(q[0, :, 0], k[0, :, 0], v[0, :, 0], a[0, :, 0],
                                          b[0, :, 0], g[0, :, 0], s0[0, 0], C=16)
     assert rel_err(oc, o[0, :, 0]) < 1e-10 and rel_err(Sc, S_T[0, 0]) < 1e-10
+
+
+def test_constant_channel_gate_is_the_scalar_gate():
+    """DPLR and GLA with a per-channel gate equal in every channel match their
+    scalar-gate runs (the gate reaches every key channel alike)."""
+    q, k, v, a, b, g, s0 = _inputs(2, 8, 2, 4, 3, "scalar")
+    gc = np.repeat(g[..., None], 4, axis=-1)
+    o1, S1 = oracle.dplr_fwd(q, k, v, a, b, g, s0, gate="scalar")
+    o2, S2 = oracle.dplr_fwd(q, k, v, a, b, gc, s0, gate="channel")
+    assert rel_err(o1, o2) < 1e-14 and rel_err(S1, S2) < 1e-14
+    o1, S1 = oracle.gla_fwd(q, k, v, g, s0, gate="scalar")
+    o2, S2 = oracle.gla_fwd(q, k, v, gc, s0, gate="channel")
+    assert rel_err(o1, o2) < 1e-14 and rel_err(S1, S2) < 1e-14
