@@ -29,6 +29,7 @@ EXPORTS = (
     "gdr_chunk_fwd_kernel_launches",
     "gdr_chunk_fwd",
     "gdr_chunk_fwd_segmented",
+    "gdr_chunk_fwd_segmented_noalloc",
     "gdr_chunk_fwd_varlen",
     "gdr_chunk_fwd_gla",
     "gdr_chunk_fwd_prologue",
@@ -71,6 +72,9 @@ def lib():
             L.gdr_chunk_fwd_segmented.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, i, i, i, i,
                                                   i, i, i, vp, sz, vp]
             L.gdr_chunk_fwd_segmented.restype = i
+            L.gdr_chunk_fwd_segmented_noalloc.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp,
+                                                          i, i, i, i, i, i, i, vp]
+            L.gdr_chunk_fwd_segmented_noalloc.restype = i
             L.gdr_chunk_fwd_varlen.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, i, i, i,
                                                i, i, i, vp]
             L.gdr_chunk_fwd_varlen.restype = i
@@ -275,6 +279,44 @@ def chunk_fwd_segmented(q, k, v, g, beta, S0=None, *, segments, workspace,
             _ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk, _ptr(beta), _ptr(S0),
             _ptr(o), _ptr(S_T), B, T, H, dk, dv, C, int(segments), _ptr(workspace),
             workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc)
+    return o, S_T
+
+
+# Bytes of the scratch array built into the library (GDR_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
+
+
+def chunk_fwd_segmented_noalloc(q, k, v, g, beta, S0=None, *, segments, o, S_T=None, C=64,
+                                stream=None):
+    """``gdr_chunk_fwd_segmented_noalloc``: the segment path with its scratch in
+    the library's fixed array, for callers that cannot allocate device memory
+    while they run the mixer.  The caller passes every output (``o``, and
+    ``S_T`` or None); nothing is allocated here or in the library.  Calls
+    that overlap on the GPU race on the shared array.  Returns (o, S_T)."""
+    _need(q, "q")
+    dev = q.device
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", dt, (B, T, H, dk), dev)
+    _need(v, "v", dt, (B, T, H, dv), dev)
+    if g.dim() == 4:
+        _need(g, "g", torch.float32, (B, T, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(g, "g", torch.float32, (B, T, H), dev)
+        gk = GDR_GATE_SCALAR
+    _need(beta, "beta", torch.float32, (B, T, H), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    _need(o, "o", dt, (B, T, H, dv), dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
+    with torch.cuda.device(dev):
+        rc = lib().gdr_chunk_fwd_segmented_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk, _ptr(beta), _ptr(S0),
+            _ptr(o), _ptr(S_T), B, T, H, dk, dv, C, int(segments), _stream_handle(stream))
     _check(rc)
     return o, S_T
 

@@ -232,6 +232,44 @@ gdr_status gdr_chunk_fwd_segmented(const void *q, const void *k, const void *v,
                    "gdr_chunk_fwd_segmented launch");
 }
 
+// The segment path with its scratch in the library's fixed array instead of
+// a caller's workspace, for callers that cannot allocate device memory when
+// they run the mixer (see gdr.h).  Validation as gdr_chunk_fwd_segmented;
+// sizes beyond the array are refused before anything touches the device.
+gdr_status gdr_chunk_fwd_segmented_noalloc(const void *q, const void *k, const void *v,
+                                           gdr_dtype in_dtype, const float *g,
+                                           gdr_gate_kind gate, const float *beta,
+                                           const float *S0, void *o, float *S_T, int B, int T,
+                                           int H, int dk, int dv, int C, int P,
+                                           gdr_stream_t stream) {
+  gdr::ChunkArgs a;
+  gdr_status st = check_chunk(q, k, v, in_dtype, g, gate, beta, S0, o, S_T, B, T, H, dk, dv, C,
+                              &a);
+  if (st != GDR_OK) return st;
+  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128)
+    return fail(GDR_ERR_UNSUPPORTED, "segments need bf16 inputs and dk = dv = 128");
+  if (P < 2 || T <= 0 || T % (64 * P) != 0)
+    return fail(GDR_ERR_UNSUPPORTED, "P=%d segments of whole 64-token chunks (T=%d)", P, T);
+  if ((size_t)B * P * H > (size_t)1 << 31) return fail(GDR_ERR_INVALID_ARG, "B*P*H too large");
+  const size_t need = gdr::chunk_segments_ws_bytes(a, P);
+  if (need > (size_t)GDR_NOALLOC_SCRATCH_BYTES)
+    return fail(GDR_ERR_WORKSPACE,
+                "needs %zu B of scratch (B*P*H = %zu segment-heads); the library's fixed array "
+                "holds %zu B (B*P*H <= %zu)",
+                need, (size_t)B * P * H, (size_t)GDR_NOALLOC_SCRATCH_BYTES,
+                (size_t)GDR_NOALLOC_SCRATCH_BYTES / (3 * (size_t)dv * dk * sizeof(float)));
+  if ((size_t)B * H == 0) return ok();
+  a.skip_stage_chunk = -1;
+  cudaError_t e = status_word(&a.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd_segmented_noalloc status word");
+  void *scratch = nullptr;
+  e = gdr::noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_fwd_segmented_noalloc scratch address");
+  return from_cuda(gdr::launch_chunk_segments(a, P, scratch,
+                                              reinterpret_cast<cudaStream_t>(stream)),
+                   "gdr_chunk_fwd_segmented_noalloc launch");
+}
+
 gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                                 const float *g, gdr_gate_kind gate, const float *beta,
                                 const int *cu_seqlens, const float *S0, void *o, float *S_T,

@@ -71,6 +71,9 @@ bool chunk_tc_supports(const ChunkArgs &a);
 int chunk_segments(const ChunkArgs &a, int num_sms);
 size_t chunk_segments_ws_bytes(const ChunkArgs &a, int P);
 cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStream_t stream);
+// Device address, on the current device, of the library's fixed scratch
+// array (GDR_NOALLOC_SCRATCH_BYTES), looked up once per device.
+cudaError_t noalloc_scratch(void **out);
 // DPLR transition, recurrent forward (CUDA cores, d_k = d_v = d in {32, 64, 128}).
 cudaError_t launch_dplr(const void *q, const void *k, const void *v, const void *a,
                         const void *b, int bf16, const float *g, int per_channel,

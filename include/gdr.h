@@ -142,6 +142,49 @@ gdr_status gdr_chunk_fwd_segmented(const void *q, const void *k, const void *v,
                                    int B, int T, int H, int dk, int dv, int C, int P,
                                    void *workspace, size_t ws_bytes, gdr_stream_t stream);
 
+/* Size of the scratch array built into the library for
+ * gdr_chunk_fwd_segmented_noalloc: 24 MiB, enough for B*P*H <= 128
+ * segment-heads (for example one 65536-token sequence of 16 heads cut into
+ * 8 segments). */
+#define GDR_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
+
+/*
+ * gdr_chunk_fwd_segmented without a workspace argument: the same segment
+ * path and the same kernels, with the scratch taken from a fixed array that
+ * is part of the library instead of from the caller.  It is meant for
+ * callers that cannot allocate device memory when they run the mixer: a
+ * plugin inside a host framework that owns the device's memory pool and
+ * gives the plugin no allocator, or a serving loop that must not stall on
+ * cudaMalloc / cudaFree, which can synchronise the whole device.  The
+ * method on the pages has no counterpart of this entry point; the
+ * arithmetic is that of gdr_chunk_fwd_segmented.
+ *
+ * Arguments as gdr_chunk_fwd_segmented without workspace / ws_bytes.  The
+ * caller still owns and passes every input and output.
+ *
+ * Scratch: 3 * B*P*H * dv*dk * 4 bytes are needed; more than
+ * GDR_NOALLOC_SCRATCH_BYTES is refused with GDR_ERR_WORKSPACE before
+ * anything is enqueued.  The array is reserved on every GPU that loads the
+ * library and held until the process exits.  Every call uses the same
+ * array: two calls whose work overlaps on the GPU (on different streams, or
+ * from different host threads) race on it and give undefined results, so
+ * serialise them.  The array keeps whatever the last call left there; each
+ * call writes every byte it reads before reading it, so nothing has to be
+ * cleared between calls.
+ *
+ * Set-up: the first call on a device looks up that device's address of the
+ * array (cudaGetSymbolAddress, with that device current), which may load the
+ * library's module on that device; make that first call before any stream
+ * capture.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ */
+gdr_status gdr_chunk_fwd_segmented_noalloc(const void *q, const void *k, const void *v,
+                                           gdr_dtype in_dtype, const float *g,
+                                           gdr_gate_kind gate, const float *beta,
+                                           const float *S0, void *o, float *S_T, int B, int T,
+                                           int H, int dk, int dv, int C, int P,
+                                           gdr_stream_t stream);
+
 /*
  * The chunked forward over N packed sequences of different lengths (a
  * variable-length batch), one state per sequence and head.  Source as
