@@ -20,7 +20,7 @@ _lib = None
 _lock = threading.Lock()
 
 GDR_OK, GDR_ERR_INVALID_ARG, GDR_ERR_UNSUPPORTED, GDR_ERR_WORKSPACE, GDR_ERR_CUDA, \
-    GDR_ERR_TIMEOUT = range(6)
+    GDR_ERR_TIMEOUT, GDR_ERR_RANGE = range(7)
 GDR_F32, GDR_BF16 = 0, 1
 GDR_GATE_SCALAR, GDR_GATE_PER_CHANNEL = 0, 1
 
@@ -191,10 +191,12 @@ def chunk_fwd(q, k, v, g, beta, S0=None, *, output_final_state=True, o=None, S_T
         S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
     if S_T is not None:
         _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
-    ws = chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, dt, "channel" if gk else "scalar")
-    if ws and workspace is None:
-        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
     with torch.cuda.device(dev):
+        # the segment rule depends on the SM count of q's device, which the
+        # library reads from the current device
+        ws = chunk_fwd_workspace_bytes(B, T, H, dk, dv, C, dt, "channel" if gk else "scalar")
+        if ws and workspace is None:
+            workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
         rc = lib().gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(g), gk,
                                  _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv, C,
                                  _ptr(workspace), workspace.numel() if workspace is not None
