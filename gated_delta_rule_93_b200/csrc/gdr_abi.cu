@@ -112,6 +112,7 @@ const char *gdr_status_string(gdr_status s) {
     case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE";
     case GDR_ERR_CUDA: return "GDR_ERR_CUDA";
     case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT";
+    case GDR_ERR_RANGE: return "GDR_ERR_RANGE";
   }
   return "GDR_ERR_UNKNOWN";
 }
@@ -470,6 +471,12 @@ gdr_status gdr_get_device_status(gdr_stream_t stream) {
   if (e != cudaSuccess) return from_cuda(e, "gdr_get_device_status");
   if (word & gdr::kStatusTimeout)
     return fail(GDR_ERR_TIMEOUT, "a kernel gave up a bounded wait (status word 0x%x)", word);
+  if (word & gdr::kStatusRange)
+    return fail(GDR_ERR_RANGE,
+                "a per-channel gate decayed beyond the tensor-core path's range (more than "
+                "about 83 in log decay over half a chunk); those results are not valid "
+                "(status word 0x%x)",
+                word);
   return ok();
 }
 

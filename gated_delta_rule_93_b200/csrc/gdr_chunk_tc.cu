@@ -588,6 +588,11 @@ __device__ int g_dbg_chunk = 0;
   } while (0)
 #endif
 
+// Largest log2 factor the per-channel tile scaling applies (2^120, well
+// inside bf16's range for unit-norm rows); a chunk whose per-channel decay
+// over half a chunk goes beyond it (about e^{-83}) reports kStatusRange.
+constexpr float kMaxExp2 = 120.f;
+
 // 2^x with the hardware approximation (ex2.approx, the instruction __expf is
 // built on); the per-channel scaling keeps its logs in base 2.
 __device__ __forceinline__ float ex2(float x) {
@@ -725,14 +730,55 @@ __device__ __forceinline__ void scale_row(uint8_t *kt, uint8_t *qt, uint8_t *ht,
   *reinterpret_cast<uint32_t *>(ht + off) = pack_bf16(kv.x * vx, kv.y * vy);
 }
 
+// Zero the low (lo) and / or high (hi) bf16 of a pair in a tile.
+__device__ __forceinline__ void clear_pair(uint8_t *tile, uint32_t off, bool lo, bool hi) {
+  uint32_t *p = reinterpret_cast<uint32_t *>(tile + off);
+  *p &= (lo ? 0xffff0000u : 0xffffffffu) & (hi ? 0x0000ffffu : 0xffffffffu);
+}
+
+// Cold: a channel whose log2 decay factor exceeds kMaxExp2 within the chunk
+// (a per-channel decay stronger than the tile scaling can represent).  The
+// entries whose factor overflowed are set to zero, so that nothing infinite
+// reaches the tensor core; the chunk's results are then not the
+// recurrence's, which the range status bit reports.  First half (rows 0-31,
+// g0 = cumulative log2 decay): K~ and Q~ carry 2^{gc - m} >= 1.
+__device__ __noinline__ void clear_first_half(uint8_t *kt, uint8_t *qt, const float *g0, int jl,
+                                              int jc, float mx, float my) {
+  for (int t = 0; t < 32; ++t) {
+    const float2 gl = *reinterpret_cast<const float2 *>(g0 + t * 64 + jl);
+    const bool lo = gl.x - mx > kMaxExp2, hi = gl.y - my > kMaxExp2;
+    if (lo || hi) {
+      clear_pair(kt, sw128_off(t, jc), lo, hi);
+      clear_pair(qt, sw128_off(t, jc), lo, hi);
+    }
+  }
+}
+
+// Second half (rows 32-63, g1 = per-token log decay): K^ carries
+// 2^{m - gc} >= 1.
+__device__ __noinline__ void clear_second_half(uint8_t *ht, const float *g1, int jl, int jc,
+                                               int nv, float mx, float my) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  float ax = mx, ay = my;
+  for (int t = 32; t < 64; ++t) {
+    const float2 x = t < nv ? *reinterpret_cast<const float2 *>(g1 + (t - 32) * 64 + jl)
+                            : make_float2(0.f, 0.f);
+    ax += x.x * kLog2e;
+    ay += x.y * kLog2e;
+    const bool lo = mx - ax > kMaxExp2, hi = my - ay > kMaxExp2;
+    if (lo || hi) clear_pair(ht, sw128_off(t, jc), lo, hi);
+  }
+}
+
 __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, uint64_t *gf,
                               uint32_t ph, const CUtensorMap *tmG, int h, int bt, int t0n,
-                              int nv, float *gv, int j0, int lane, volatile int *abort_flag) {
+                              int nv, float *gv, int j0, int lane, volatile int *abort_flag,
+                              unsigned int *status) {
   constexpr float kLog2e = 1.4426950408889634f;
   const int jl = 2 * lane, j = j0 + jl, hh = j >> 6, jc = j & 63;
   uint8_t *kt = kq + (2 * hh) * kTileBytes, *qt = kt + kTileBytes, *ht = kh + hh * kTileBytes;
   if (!warp_wait(&gf[0], ph, abort_flag, lane)) return 0;
-  float2 acc = make_float2(0.f, 0.f);
+  float2 acc = make_float2(0.f, 0.f), first = acc;
 #pragma unroll 8
   for (int t = 0; t < 32; ++t) {
     float2 *p = reinterpret_cast<float2 *>(g0 + t * 64 + jl);
@@ -740,6 +786,7 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
     acc.x += x.x * kLog2e;
     acc.y += x.y * kLog2e;
     *p = acc;
+    if (t == 0) first = acc;
   }
   const float2 m = acc;
   gv[kGateEm + j] = ex2(m.x);
@@ -748,6 +795,12 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
   for (int t = 0; t < 32; ++t) {
     const float2 gl = *reinterpret_cast<const float2 *>(g0 + t * 64 + jl);
     scale_row(kt, qt, ht, t, jc, gl.x - m.x, gl.y - m.y);
+  }
+  // the largest factor of rows 0-31 is 2^{gc_0 - m}
+  bool out_of_range = false;
+  if (__any_sync(0xffffffffu, fmaxf(first.x - m.x, first.y - m.y) > kMaxExp2)) {
+    clear_first_half(kt, qt, g0, jl, jc, m.x, m.y);
+    out_of_range = true;
   }
   // rows 0-31 read (and written, by the generic proxy): refill
   fence_proxy_async_smem();
@@ -765,6 +818,12 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
     acc.y += x.y * kLog2e;
     scale_row(kt, qt, ht, t, jc, acc.x - m.x, acc.y - m.y);
   }
+  // the largest factor of rows 32-63 is 2^{m - gc_63}
+  if (__any_sync(0xffffffffu, fmaxf(m.x - acc.x, m.y - acc.y) > kMaxExp2)) {
+    clear_second_half(ht, g1, jl, jc, nv, m.x, m.y);
+    out_of_range = true;
+  }
+  if (out_of_range && lane == 0) atomicOr(status, kStatusRange);
   __syncwarp();
   if (lane == 0 && t0n >= 0) {
     mbar_arrive_expect_tx(&gf[1], 32 * 64 * 4);
@@ -962,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      sm + Lay::KH + s * 2 * kTileBytes, gt, gt + 32 * 64,
                                      &bars[B_GF], c & 1, &tmG, h, bt,
                                      c + 1 < n ? tb + t0 + C : -1, T - t0, gv, 0, lane,
-                                     abort_flag);
+                                     abort_flag, a.status);
         if (c + 1 < n && r >= 1) gate_req[0] = c + 1;
         if (c + 1 < n && r == 2) gate_req[1] = c + 1;
         if (r < 2) break;
@@ -1001,7 +1060,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    sm + Lay::KH + s * 2 * kTileBytes, gt, gt + 32 * 64,
                                    &bars[B_GF + 2], c & 1, &tmG, h, bt,
                                    c + 1 < n ? tb + (c + 1) * C : -1, T - c * C, gv, 64, lane,
-                                   abort_flag);
+                                   abort_flag, a.status);
       if (c + 1 < n && r >= 1) gate_req[0] = c + 1;
       if (c + 1 < n && r == 2) gate_req[1] = c + 1;
       if (r < 2) break;
@@ -1010,9 +1069,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (c >= 1 && !warp_wait(&bars[B_VEMPTY], (c - 1) & 1, abort_flag, lane)) break;
       if (lane == 0) {
         uint8_t *vv = sm + Lay::V;
-        mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
-        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, tb + c * C, bt);
-        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, tb + c * C, bt);
+        if (a.zero_v) {  // v taken as zero: the phase completes with no load
+          mbar_arrive(&bars[B_VFULL]);
+        } else {
+          mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
+          tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, tb + c * C, bt);
+          tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, tb + c * C, bt);
+        }
       }
       __syncwarp();
       last = c;
@@ -1030,9 +1093,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < n; ++c) {
         if (c >= 1 && !wait_or_abort(&bars[B_VEMPTY], (c - 1) & 1, abort_flag)) break;
         uint8_t *vv = sm + Lay::V;
-        mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
-        tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, tb + c * C, bt);
-        tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, tb + c * C, bt);
+        if (a.zero_v) {  // v taken as zero: the phase completes with no load
+          mbar_arrive(&bars[B_VFULL]);
+        } else {
+          mbar_arrive_expect_tx(&bars[B_VFULL], kVTx);
+          tma_load_4d(vv, &tmV, &bars[B_VFULL], 0, h, tb + c * C, bt);
+          tma_load_4d(vv + kTileBytes, &tmV, &bars[B_VFULL], 64, h, tb + c * C, bt);
+        }
         last = c;
       }
       if (last >= 0) drain_wait(&bars[B_VFULL], last & 1);
@@ -1075,10 +1142,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = W(B_TRDY, ph) && W(B_VFULL, ph))) break;
         {
           const uint32_t tt = PC ? a_tp + (c & 1) * kTileBytes : a_t;
+          if (!a.zero_v) {  // (v taken as zero: U = 0, the V' MMA starts the accumulator)
 #pragma unroll 1
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ss(tm + TM_UV, sdesc_sw128(a_v + kk * 2048, kTileBytes, 1024),
-                        sdesc_sw128(tt + kk * 32, 16, 1024), ID_U, kk > 0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ss(tm + TM_UV, sdesc_sw128(a_v + kk * 2048, kTileBytes, 1024),
+                          sdesc_sw128(tt + kk * 32, 16, 1024), ID_U, kk > 0);
+          }
           mma_commit(&bars[B_UF]);      // T read: the prep group may write the next T
           mma_commit(&bars[B_VEMPTY]);  // V read
         }
@@ -1086,10 +1155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ADD) {
           if (!(ok = W(B_ZR, ph))) break;
           const uint32_t tp = a_tp + (c & 1) * kTileBytes;
+          const uint32_t acc0 = a.zero_v ? 0u : 1u;
 #pragma unroll 1
           for (int kk = 0; kk < 4; ++kk)
             mma_bf16_ts(tm + TM_UV, tm + TM_Z + 8 * kk, sdesc_sw128(tp + kk * 32, 16, 1024),
-                        ID_N64, 1);
+                        ID_N64, kk > 0 ? 1u : acc0);
         }
         mma_commit(&bars[B_VPF]);
         if (!ADD) mma_commit(&bars[B_TPE + (c & 1)]);

@@ -12,6 +12,9 @@ namespace gdr {
 // Kernels OR error bits into a device status word (they never trap).  The
 // word lives in gdr_abi.cu; launchers receive its device address.
 constexpr unsigned int kStatusTimeout = 1u;
+// A per-channel gate decayed faster than the tensor-core path's tile scaling
+// can represent in some chunk (that call's results are not the recurrence's).
+constexpr unsigned int kStatusRange = 2u;
 
 struct ChunkArgs {
   const void *q, *k, *v;
@@ -29,6 +32,7 @@ struct ChunkArgs {
   // for an ordinary call):
   int s0_seg;       // > 0: sequence b reads S0[b / s0_seg] if b % s0_seg == 0, else starts at 0
   int s0_identity;  // 1: sequences without an S0 start from the identity (d_v == d_k)
+  int zero_v;       // 1: v is taken as zero (not read): the end state is the transition
   int write_o;      // 0: o is not written (may be null)
   // Packed sequences (tensor-core kernel only): B sequences, sequence b is
   // tokens [cu_seqlens[b], cu_seqlens[b + 1]) of the [1, T, H, d] tensors

@@ -10,7 +10,9 @@
 // section applies this per chunk; here it is applied per segment:
 //   pass 1a: every segment from zero (the first from S0): E_p, and for the
 //            first segment its true end state;
-//   pass 1b: every segment from the identity: end state M_p + E_p (d_v = d_k);
+//   pass 1b: every segment from the identity with v taken as zero: end state
+//            M_p (d_v = d_k), the transition itself, with no difference of
+//            two runs (which loses M_p's precision when it is not small);
 //   combine: S_start(1) = end of segment 0, S_start(p + 1) = S_start(p) M_p +
 //            E_p, in fp32; the last product is the final state S_T;
 //   pass 2:  every segment from its true start state: the output o.
@@ -41,13 +43,15 @@ __device__ __forceinline__ void cp_async_wait_all() {
 }
 
 // One CTA per (b, h) and block of 16 state rows (rows of S are independent
-// under S <- S M + E).  E_a: end states of pass 1a, E_b: of pass 1b, X: the
+// under S <- S M + E).  E_a: end states of pass 1a, E_b: of pass 1b (the
+// transitions M_p), X: the
 // start state of every segment (written), S_T: the final state (optional),
-// all [B * P, H, 128, 128] except S0 / S_T [B, H, 128, 128].  Each thread
+// all [B * P, H, 128, 128] except S0 / S_T [B, H, 128, 128] (S0 may alias
+// S_T, so neither is declared __restrict__).  Each thread
 // forms 4 rows x 2 columns of the product (a warp shares its rows), so every
 // column pair of M read from shared memory serves four rows.
 __global__ void __launch_bounds__(kCombineThreads)
-    combine_segments(const float *__restrict__ S0, const float *__restrict__ Ea,
+    combine_segments(const float *S0, const float *__restrict__ Ea,
                      const float *__restrict__ Eb, float *__restrict__ X, float *S_T, int H,
                      int P) {
   extern __shared__ float smem[];
@@ -77,8 +81,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     const float4 *ea4 = reinterpret_cast<const float4 *>(Ea + seg(p));
     const float4 *eb4 = reinterpret_cast<const float4 *>(Eb + seg(p));
     float4 *m4 = reinterpret_cast<float4 *>(M), *a4 = reinterpret_cast<float4 *>(MA);
-    // E_b and E_a of the segment into shared memory, every copy in flight at
-    // once, then M = E_b - E_a in place
+    // M = E_b and E_a of the segment into shared memory, every copy in
+    // flight at once
 #pragma unroll 8
     for (int j = 0; j < kDim * kDim / 4 / kCombineThreads; ++j) {
       const int i = t + j * kCombineThreads;
@@ -86,13 +90,6 @@ __global__ void __launch_bounds__(kCombineThreads)
       cp_async16(a4 + i, ea4 + i);
     }
     cp_async_wait_all();
-    __syncthreads();
-#pragma unroll 8
-    for (int j = 0; j < kDim * kDim / 4 / kCombineThreads; ++j) {
-      const int i = t + j * kCombineThreads;
-      const float4 x = m4[i], y = a4[i];
-      m4[i] = make_float4(x.x - y.x, x.y - y.y, x.z - y.z, x.w - y.w);
-    }
     __syncthreads();
     float2 acc[4];
 #pragma unroll
@@ -171,13 +168,15 @@ cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStrea
   s.write_o = 0;
   cudaError_t e = launch_chunk_tc(s, stream);
   if (e != cudaSuccess) return e;
-  // pass 1b: identity start, end states = transition + the same writes
+  // pass 1b: identity start with v taken as zero, end states = transitions
   s.S0 = nullptr;
   s.s0_seg = 0;
   s.s0_identity = 1;
+  s.zero_v = 1;
   s.S_T = Eb;
   e = launch_chunk_tc(s, stream);
   if (e != cudaSuccess) return e;
+  s.zero_v = 0;
   combine_segments<<<dim3(a.B * a.H, kRowBlocks), kCombineThreads, kCombineSmem, stream>>>(
       a.S0, Ea, Eb, X, a.S_T, a.H, P);
   e = cudaGetLastError();

@@ -29,7 +29,9 @@
  *   the call returns GDR_ERR_INVALID_ARG or GDR_ERR_UNSUPPORTED and launches
  *   nothing; gdr_last_error_message() then describes the problem.
  * - A kernel that gives up a bounded wait records GDR_ERR_TIMEOUT in a
- *   device status word; gdr_get_device_status() reads and clears it.
+ *   device status word; gdr_get_device_status() reads and clears it.  The
+ *   tensor-core path records GDR_ERR_RANGE there when a per-channel gate
+ *   decays beyond what it can represent (see gdr_chunk_fwd).
  * - Gate: `g` holds log(alpha) in fp32 (finite, <= 0).  A scalar gate has one
  *   value per (token, head); a per-channel gate has d_k values.
  * - Dtypes: q, k, v and o share `in_dtype` (fp32 or bf16); g, beta and the
@@ -54,7 +56,9 @@ typedef enum {
   GDR_ERR_UNSUPPORTED = 2, /* valid request this build does not implement   */
   GDR_ERR_WORKSPACE = 3,   /* workspace pointer/size too small              */
   GDR_ERR_CUDA = 4,        /* a CUDA runtime call failed                    */
-  GDR_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (device word) */
+  GDR_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (device word) */
+  GDR_ERR_RANGE = 6        /* per-channel decay beyond the tensor-core path's
+                              range in some chunk (device word)             */
 } gdr_status;
 
 typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
@@ -105,9 +109,18 @@ int gdr_chunk_fwd_kernel_launches(int B, int T, int H, int dk, int dv, int C,
  *
  * T may be any value >= 0 (a ragged last chunk is masked); B*H may be 0.
  * S0 may alias S_T (each (b, h) reads all of S0 before writing S_T); o must
- * not alias any input.  Per-channel gates must keep the decay accumulated
- * over one chunk within about 80 (|sum of g| per channel) so that the
- * intermediate exp(-sum g) stays finite in fp32; scalar gates have no limit.
+ * not alias any input.
+ *
+ * Range of per-channel gates on the tensor-core path (bf16, dk = dv = 128):
+ * a chunk's K and Q tiles are scaled per key channel by e^{+-(gc - m)}
+ * around the cumulative decay m at the chunk's row 31, so in every channel
+ * the decay accumulated over each half chunk (32 tokens) must stay above
+ * about -83 (|sum of g| <= 83, e.g. a decay of e^{-2.6} per token held for
+ * 32 tokens).  A chunk beyond that has its overflowing tile entries zeroed
+ * (the outputs stay finite but are not the recurrence's) and the call
+ * records GDR_ERR_RANGE in the device status word (gdr_get_device_status).
+ * Scalar gates and the CUDA-core path (fp32 inputs, dk or dv < 128) have no
+ * limit.
  */
 gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                          const float *g, gdr_gate_kind gate, const float *beta,
@@ -121,10 +134,10 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
  * workspace.  Source: "Decoding Hybrid Linear Attention Architectures",
  * section 5, whose inter-chunk recursion (end state = start state times the
  * chunk's transition plus what the chunk writes) is applied per segment:
- * every segment runs from a zero state (the first from S0) and from the
- * identity, the segments' start states follow in fp32
- * (S_start(p+1) = S_start(p) M_p + E_p, M_p = the identity run's end state
- * minus the zero run's), and a last pass writes o.  gdr_chunk_fwd takes
+ * every segment runs from a zero state (the first from S0), giving E_p, and
+ * from the identity with v taken as zero, giving its transition M_p; the
+ * segments' start states follow in fp32 (S_start(p+1) = S_start(p) M_p +
+ * E_p), and a last pass writes o.  gdr_chunk_fwd takes
  * this path by itself for long sequences with few heads; this entry point
  * fixes P (for example to capture a fixed shape in a CUDA graph).
  *
@@ -348,7 +361,10 @@ gdr_status gdr_step(const void *q, const void *k, const void *v, gdr_dtype in_dt
 /*
  * Synchronises `stream`, then reads and clears the device status word.
  * Returns GDR_OK, GDR_ERR_TIMEOUT (a kernel gave up a bounded wait since the
- * last call) or GDR_ERR_CUDA (the synchronisation itself failed).
+ * last call), GDR_ERR_RANGE (a per-channel gate decayed beyond the
+ * tensor-core path's range in some chunk since the last call; a time-out
+ * takes precedence when both happened) or GDR_ERR_CUDA (the
+ * synchronisation itself failed).
  */
 gdr_status gdr_get_device_status(gdr_stream_t stream);
 

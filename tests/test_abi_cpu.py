@@ -44,7 +44,8 @@ def test_no_driver_dependency(L):
 
 def test_status_strings(L):
     for code, name in enumerate(["GDR_OK", "GDR_ERR_INVALID_ARG", "GDR_ERR_UNSUPPORTED",
-                                 "GDR_ERR_WORKSPACE", "GDR_ERR_CUDA", "GDR_ERR_TIMEOUT"]):
+                                 "GDR_ERR_WORKSPACE", "GDR_ERR_CUDA", "GDR_ERR_TIMEOUT",
+                                 "GDR_ERR_RANGE"]):
         assert binding.status_string(code) == name
 
 

@@ -183,6 +183,34 @@ def test_segment_path_matches_oracle(cuda_device, gate, with_S0):
     assert_close(S_T, rS, 2e-2, "S_T")
 
 
+@pytest.mark.parametrize("gscale", [0.0, 0.0125])
+@pytest.mark.parametrize("P", [None, 8])
+def test_segment_path_weak_decay(cuda_device, gscale, P):
+    """Weak decay, where a segment's transition M_p is far from zero: g = 0
+    (the delta rule, "Decoding Hybrid Linear Attention Architectures",
+    section 3 item 2) and g of about -0.001 per token (the default gates
+    times 0.0125).  The segment path recovers M_p = (M_p + E_p) - E_p from
+    two runs; here that difference is not damped.  B1 H2 T4096 d128 with S0,
+    the automatic segment path (4 segments) and the segmented entry point
+    with 8 segments."""
+    B, T, H, d = 1, 4096, 2, 128
+    inp = make_chunk_inputs(B, T, H, d, d, torch.bfloat16, "scalar", True, seed=17)
+    inp["g"] = (inp["g"] * gscale).contiguous()
+    dd = {k: v.to(cuda_device) for k, v in inp.items()}
+    if P is None:
+        assert binding.chunk_fwd_kernel_launches(B, T, H, d, d) == 4
+        o, S_T = binding.chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"])
+    else:
+        ws = torch.empty(3 * B * P * H * d * d * 4, dtype=torch.uint8, device=cuda_device)
+        o, S_T = binding.chunk_fwd_segmented(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
+                                             dd["S0"], segments=P, workspace=ws)
+    torch.cuda.synchronize()
+    assert binding.device_status() == 0
+    ro, rS = oracle_chunk(inp)
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S_T, rS, 2e-2, "S_T")
+
+
 def test_segment_path_initial_state_may_alias_final_state(cuda_device):
     inp = make_chunk_inputs(1, 4096, 2, 128, 128, torch.bfloat16, "scalar", True, seed=12)
     d = {k: v.to(cuda_device) for k, v in inp.items()}
@@ -240,3 +268,51 @@ def test_segmented_entry_point_rejects_short_workspace(cuda_device):
         binding.chunk_fwd_segmented(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], None,
                                     segments=4, workspace=ws)
     assert ei.value.status == binding.GDR_ERR_WORKSPACE
+
+
+def _one_channel_decay(inp, g_channel, channel=5, head=0):
+    g = inp["g"].clone()
+    g[:, :, head, channel] = g_channel
+    return dict(inp, g=g.contiguous())
+
+
+def test_per_channel_strong_decay_within_range(cuda_device):
+    """One key channel forgetting fast, e^{-2.5} per token (-80 over half a
+    chunk), inside the tensor-core path's range: oracle parity, clean status."""
+    inp = _one_channel_decay(make_chunk_inputs(1, 256, 2, 128, 128, torch.bfloat16, "channel",
+                                               True, seed=61), -2.5)
+    o, S_T = gpu_chunk(inp, cuda_device)
+    assert binding.device_status() == binding.GDR_OK
+    ro, rS = oracle_chunk(inp)
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S_T, rS, 2e-2, "S_T")
+
+
+def test_per_channel_rapid_forgetting_reports_range(cuda_device):
+    """One key channel at g = -30 per token ("one-step rapid forgetting",
+    "Decoding Hybrid Linear Attention Architectures", section 4) is beyond
+    what the tensor-core path's tile scaling represents: the call records
+    GDR_ERR_RANGE in the device status word and its outputs stay finite."""
+    inp = _one_channel_decay(make_chunk_inputs(1, 256, 2, 128, 128, torch.bfloat16, "channel",
+                                               True, seed=62), -30.0)
+    o, S_T = gpu_chunk(inp, cuda_device)
+    assert binding.device_status() == binding.GDR_ERR_RANGE
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S_T).all()
+    # the status word was cleared by the read; a call within range is clean
+    inp2 = make_chunk_inputs(1, 128, 2, 128, 128, torch.bfloat16, "channel", False, seed=63)
+    gpu_chunk(inp2, cuda_device)
+    assert binding.device_status() == binding.GDR_OK
+
+
+@pytest.mark.parametrize("d,dtype", [(64, torch.bfloat16), (128, torch.float32)])
+def test_per_channel_rapid_forgetting_cuda_core_path(cuda_device, d, dtype):
+    """The CUDA-core path (d < 128 or fp32 inputs) forms exact pairwise decays
+    and takes any finite g <= 0: g = -30 per token in one channel matches
+    the oracle."""
+    inp = _one_channel_decay(make_chunk_inputs(1, 200, 2, d, d, dtype, "channel", True,
+                                               seed=64), -30.0)
+    o, S_T = gpu_chunk(inp, cuda_device)
+    assert binding.device_status() == binding.GDR_OK
+    ro, rS = oracle_chunk(inp)
+    assert_close(o, ro, TOL[dtype], "o")
+    assert_close(S_T, rS, TOL[dtype], "S_T")
