@@ -101,17 +101,25 @@ def make_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, gate="scalar", with
     return dict(q=q, k=k, v=v, g=g.float(), beta=beta.float(), S0=S0)
 
 
-def make_dplr_inputs(B, T, H, d, dtype=torch.bfloat16, gate="scalar", with_S0=False, seed=0):
+def make_dplr_inputs(B, T, H, d, dtype=torch.bfloat16, gate="scalar", with_S0=False, seed=0,
+                     independent=False):
     """Inputs for ``gdr_dplr_fwd``: the ``make_chunk_inputs`` draws (q, k, v, g,
     beta, S0) plus an erase direction b (unit rows of N(0, 1), its own
     stream), and a = -beta e^{g} b (per channel, or the head's scalar gate),
     so that each transition Diag(alpha)(I - beta b b^T) is a contraction and
-    long sequences stay bounded.  Returns dict q, k, v, a, b, g, S0."""
+    long sequences stay bounded.  independent=True draws a on its own instead
+    (unit rows of N(0, 1) times 0.5, a third stream): a general low-rank
+    term, not tied to b (its transitions need not contract, so keep T short).
+    Returns dict q, k, v, a, b, g, S0."""
     d_ = make_chunk_inputs(B, T, H, d, d, dtype, gate, with_S0, seed)
     gen = torch.Generator().manual_seed(seed + 15485863)
     b = _unit_rows(torch.randn(B, T, H, d, generator=gen))
-    al = torch.exp(d_["g"] if gate == "channel" else d_["g"][..., None])
-    a = -d_["beta"][..., None] * al * b
+    if independent:
+        gen_a = torch.Generator().manual_seed(seed + 32452843)
+        a = 0.5 * _unit_rows(torch.randn(B, T, H, d, generator=gen_a))
+    else:
+        al = torch.exp(d_["g"] if gate == "channel" else d_["g"][..., None])
+        a = -d_["beta"][..., None] * al * b
     return dict(q=d_["q"], k=d_["k"], v=d_["v"], a=a.to(dtype), b=b.to(dtype), g=d_["g"],
                 S0=d_["S0"])
 

@@ -46,6 +46,18 @@ def test_dplr_matches_oracle_fp32(cuda_device, d):
     assert_close(S_T, rS, 1e-4, "S_T")
 
 
+@pytest.mark.parametrize("gate", ["scalar", "channel"])
+@pytest.mark.parametrize("d,dtype,tol_o", [(128, torch.bfloat16, 2e-2), (64, torch.float32, 1e-4)])
+def test_dplr_independent_low_rank_matches_oracle(cuda_device, gate, d, dtype, tol_o):
+    """a and b drawn independently (a general low-rank read, not the delta
+    rule's contraction a = -beta alpha b): 100 tokens, with S0."""
+    inp = make_dplr_inputs(2, 100, 2, d, dtype, gate, True, seed=150 + d, independent=True)
+    o, S_T = _run(inp, cuda_device)
+    ro, rS = _oracle(inp)
+    assert_close(o, ro, tol_o, "o")
+    assert_close(S_T, rS, 1e-4, "S_T")
+
+
 def test_dplr_with_delta_parameters_equals_chunked_delta_rule(cuda_device):
     """a = -beta (alpha . k), b = k, v -> beta v gives the gated delta rule:
     the recurrent DPLR kernel against the tensor-core chunked forward."""
