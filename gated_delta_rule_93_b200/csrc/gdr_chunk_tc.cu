@@ -24,7 +24,13 @@
 //
 // W is never formed: S_b W^T = (S_b K^T) T'^T moves that product onto the
 // state side, where it costs one small MMA and one TMEM conversion.  S_b is
-// the bf16 copy of the fp32 state, kept in TMEM as the A operand.
+// the bf16 copy of the fp32 state, kept in TMEM as the A operand; V'^T's two
+// bf16 copies (plain, and decayed to the chunk end) are written back into
+// TMEM as well, so every MMA of the state side takes A from TMEM.  Measured
+// on the B200: consecutive k-steps into one accumulator wait on each other
+// (about 73 cycles each with A in TMEM, 165 with A in shared memory, for
+// N = 64 as for N = 128), while independent accumulators overlap; Z and O_a
+// are therefore issued with their k-steps interleaved.
 //
 // The fp32 state is held as S = sigma * S_tmem.  A chunk's decay only
 // changes sigma (and scales the next update by 1 / sigma), so S_tmem is
@@ -36,13 +42,17 @@
 //
 // Warp roles (one CTA per (b, h), 384 threads):
 //   warps 0-3  "state" group (TMEM lanes = value channels): Z -> bf16 in
-//              TMEM, V'^T -> bf16 operands, S -> S_b, O epilogue (each warp
-//              stages its 32 channels and stores them with one TMA store);
+//              TMEM, O_a scaled in place (O_b then accumulates onto it),
+//              V'^T -> bf16 operands in TMEM, S -> S_b, O epilogue (each
+//              warp stages its 32 channels and stores them with one TMA
+//              store); O, T, T' and P have two buffers, so that neither the
+//              epilogue of a chunk nor the prep group's next T waits on the
+//              state side's progress;
 //   warps 4-7  "prep" group, one chunk ahead: gate cumsum, A/P epilogue,
 //              (I + A)^{-1} with T/T' written straight from it;
 //   warp 8     TMA producer of the K/Q stages (three) + g/beta loads;
-//   warp 9     state-side MMA issuer (U^T = V^T T^T, Z, V'^T, O_a, S, O_b;
-//              one thread);
+//   warp 9     state-side MMA issuer (Z with O_a, U^T = V^T T^T, V'^T, S,
+//              O_b; one thread);
 //   warp 10    TMA producer of V (one stage);
 //   warp 11    prep-side MMA issuer (D1, one thread): an issue can stall
 //              while the tensor core's queue is full, which must not hold up
@@ -101,8 +111,9 @@ constexpr int kSvEg = 0, kSvEgl = 64, kSvEm = 128, kSvEgm = 256;
 // stage, the scaled K~, Q~ tiles in place of K, Q and K^ in its own tiles,
 // each scaling warp's fp32 gate rows (its 64 channels, rows 0-31 and 32-63
 // of the chunk being scaled, each half refilled with the next chunk's as
-// soon as it has been read), and shares T with T' and V'^T with its decayed
-// copy (both identical without a scalar decay).
+// soon as it has been read), and shares T with T' (identical without a
+// scalar decay).  V'^T never goes to shared memory: its bf16 operand copies
+// are written back into TMEM (the MMAs that read it take A from TMEM).
 template <bool PC>
 struct Cfg {
   static constexpr int kStages = PC ? 2 : 3;
@@ -112,20 +123,19 @@ struct Cfg {
   static constexpr uint32_t KH = KQ + kStages * 4 * kTileBytes;              // PC: [Kh_h0|Kh_h1]
   static constexpr uint32_t GT = KH + (PC ? kStages * 2 * kTileBytes : 0);   // PC: g [2][2][32][64]
   static constexpr uint32_t V = GT + (PC ? 64 * 128 * 4 : 0);                // [V_h0|V_h1]
-  static constexpr uint32_t T = V + 2 * kTileBytes;                          // T  K-major [r][s]
-  static constexpr uint32_t TP = T + (PC ? 0 : kTileBytes);                  // T' K-major, x2
+  static constexpr uint32_t T = V + 2 * kTileBytes;                          // T  K-major [r][s], x2
+  static constexpr uint32_t TP = T + (PC ? 0 : 2 * kTileBytes);              // T' K-major, x2
   static constexpr uint32_t P = TP + 2 * kTileBytes;                         // P  K-major, x2
-  static constexpr uint32_t VP = P + 2 * kTileBytes;                         // V'^T K-major [dv][C]
-  static constexpr uint32_t VPD = VP + (PC ? 0 : 2 * kTileBytes);            // decayed / sigma
-  static constexpr uint32_t AF = VPD + 2 * kTileBytes;                       // fp32 A, D blocks
+  static constexpr uint32_t STG = P + 2 * kTileBytes;                        // o staging (4 x 4 KB)
+  static constexpr uint32_t AF = STG + 2 * kTileBytes;                       // fp32 A, D blocks
   static constexpr uint32_t SCR = AF + 64 * LDA * 4;                         // inverse scratch
   static constexpr uint32_t GS = SCR + (512 + 4 * 256) * 4;                  // gate vectors
   static constexpr uint32_t SVEC = GS + kStages * kGateBytes;                // x3 (state group)
   static constexpr uint32_t BAR = SVEC + 3 * kSvecBytes;                     // mbarriers
-  static constexpr uint32_t MISC = BAR + 32 * 8;                             // tmem base, abort
+  static constexpr uint32_t MISC = BAR + 40 * 8;                             // tmem base, abort
   static constexpr uint32_t END = MISC + 16;
   static constexpr size_t kSmemBytes = END + 1024;
-  static_assert(V % 1024 == 0 && T % 1024 == 0 && VPD % 1024 == 0 && AF % 1024 == 0 &&
+  static_assert(V % 1024 == 0 && T % 1024 == 0 && STG % 1024 == 0 && AF % 1024 == 0 &&
                     GT % 1024 == 0,
                 "tile alignment");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -139,17 +149,17 @@ enum {
   B_VEMPTY,            // V free (commit after U)                       (commit)
   B_D1F,               // D1 written                                    (commit, prep side)
   B_D1E,               // D1 read by the prep group                     (4 warps)
-  B_TRDY,              // T, T' and P of a chunk written                (4 warps)
-  B_UF,                // U^T written (T read)                          (commit)
-  B_ZF,                // Z written                                     (commit)
+  B_TRDY,              // [2] T, T' and P of a chunk written (buffer c % 2) (4 warps)
+  B_UF = B_TRDY + 2,   // [2] U^T written (T buffer c % 2 read)         (commit)
+  B_ZF = B_UF + 2,     // Z and O_a written                             (commit)
   B_ZR,                // Z (or -Z) bf16 operand in TMEM                (4 warps)
   B_VPF,               // V'^T complete                                 (commit)
-  B_VPR,               // V'^T bf16 operands in smem                    (4 warps)
+  B_VPR,               // V'^T bf16 operands (and O_a scaled) in TMEM   (4 warps)
   B_SF,                // state update complete                         (commit)
-  B_OF,                // O_a, O_b complete                             (commit)
+  B_OF,                // O (O_a scaled + O_b) complete                 (commit)
   B_SBR,               // S_b in TMEM for the next chunk                (4 warps)
-  B_OE,                // O_a, O_b read by the epilogue                 (4 warps)
-  B_PE,                // [2] P buffer free (after O_b)                 (commit)
+  B_OE,                // [2] O buffer c % 2 read by the epilogue       (4 warps)
+  B_PE = B_OE + 2,     // [2] P buffer free (after O_b)                 (commit)
   B_TPE = B_PE + 2,    // [2] T' buffer free (after V')                 (commit)
   B_FIN = B_TPE + 2,   // final drain, state-side issuer                (commit)
   B_FIN2,              // final drain, prep-side issuer                 (commit)
@@ -160,10 +170,14 @@ enum {
                        //     stage folded into its vectors (prep-side MMA warp)
   B_COUNT = B_GF + 4
 };
-static_assert(B_COUNT <= 32, "barrier slots");
+static_assert(B_COUNT <= 40, "barrier slots");
 
-// TMEM column map (512 allocated; 1 CTA per SM).
-constexpr uint32_t TM_S = 0, TM_SB = 128, TM_Z = 192, TM_UV = 256, TM_O = 320, TM_OA = 384,
+// TMEM column map (512 allocated; 1 CTA per SM).  UV holds U^T, then V'^T
+// in fp32, then its two bf16 operand copies (plain in columns 0-31, decayed
+// in 32-63), converted in place.  O has two buffers (chunk c in c % 2):
+// O_a = S_b Q^T, scaled in place by the state group, then O_b accumulated
+// onto it, so the epilogue of chunk c never holds up chunk c + 1.
+constexpr uint32_t TM_S = 0, TM_SB = 128, TM_Z = 192, TM_O0 = 256, TM_UV = 320, TM_O1 = 384,
                    TM_D1 = 448;
 
 constexpr uint32_t ID_D1 = idesc_bf16(128, 64, 0, 0);
@@ -884,8 +898,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[B_VEMPTY], 1);
     mbar_init(&bars[B_D1F], 1);
     mbar_init(&bars[B_D1E], 4);
-    mbar_init(&bars[B_TRDY], 4);
-    mbar_init(&bars[B_UF], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars[B_TRDY + s], 4);
+      mbar_init(&bars[B_UF + s], 1);
+      mbar_init(&bars[B_OE + s], 4);
+    }
     mbar_init(&bars[B_ZF], 1);
     mbar_init(&bars[B_ZR], 4);
     mbar_init(&bars[B_VPF], 1);
@@ -893,7 +910,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[B_SF], 1);
     mbar_init(&bars[B_OF], 1);
     mbar_init(&bars[B_SBR], 4);
-    mbar_init(&bars[B_OE], 4);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[B_PE + s], 1);
       mbar_init(&bars[B_TPE + s], 1);
@@ -905,14 +921,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // T and both T' tiles start at zero: their blocks above the block diagonal
-  // are never written afterwards.  Additive writes (ADD): T = I for good (in
-  // the T tile, or both T' tiles that per-channel gates use for T), so that
-  // the U MMA yields V'^T = V^T.
-  for (uint32_t off = 16 * tid; off < (PC ? 2 : 3) * kTileBytes; off += 16 * kThreads) {
+  // Both T and both T' tiles start at zero: their blocks above the block
+  // diagonal are never written afterwards.  Additive writes (ADD): T = I for
+  // good (in both T tiles, or both T' tiles that per-channel gates use for
+  // T), so that the U MMA yields V'^T = V^T.
+  for (uint32_t off = 16 * tid; off < (PC ? 2 : 4) * kTileBytes; off += 16 * kThreads) {
     uint4 z = make_uint4(0u, 0u, 0u, 0u);
     const uint32_t tile = off / kTileBytes, row = (off % kTileBytes) / 128;
-    if (ADD && (PC ? tile < 2 : tile == 0) && ((off % 128) / 16 ^ (row & 7)) == row / 8) {
+    if (ADD && tile < 2 && ((off % 128) / 16 ^ (row & 7)) == row / 8) {
       // this 16-byte chunk holds columns 8 (row / 8) .. + 7 of its row: the
       // diagonal element is number row % 8 (bf16 1.0 = 0x3f80)
       const uint32_t e = row & 7, one = 0x3f80u << (16 * (e & 1));
@@ -1109,7 +1125,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_tp = smem_u32(sm + Lay::TP);
       const uint32_t a_p = smem_u32(sm + Lay::P);
-      const uint32_t a_vp = smem_u32(sm + Lay::VP), a_vpd = smem_u32(sm + Lay::VPD);
       const uint32_t a_kh = smem_u32(sm + Lay::KH), a_v = smem_u32(sm + Lay::V);
       const uint32_t a_t = smem_u32(sm + Lay::T);
       auto W = [&](int slot, uint32_t parity) {
@@ -1126,29 +1141,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = c & 1;
         const int st = c % kStages;
         const uint32_t kq = a_kq + st * 4 * kTileBytes;
-        // Z = S_b K^T  (ADD: no correction, no Z)
+        // Z = S_b K^T and O_a = S_b Q^T, their k-steps interleaved: two
+        // independent accumulators share the tensor pipe while each waits on
+        // its own previous k-step.  O_a goes to buffer c % 2, free once the
+        // epilogue has read chunk c - 2's O.  The SF commit below also covers
+        // these last reads of S_b (the state group overwrites S_b once SF
+        // completes).  (ADD: no correction; no Z.)
         if (!(ok = W(B_SBR, ph) && W(B_FULL + st, (c / kStages) & 1))) break;
-        if (!ADD) {
+        if (c >= 2 && !(ok = W(B_OE + (c & 1), ((c >> 1) - 1) & 1))) break;
+        const uint32_t tmo = tm + ((c & 1) ? TM_O1 : TM_O0);
 #pragma unroll 1
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tm + TM_Z, tm + TM_SB + 8 * kk,
-                        sdesc_sw128(kq + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32, 16, 1024),
-                        ID_N64, kk > 0);
-          mma_commit(&bars[B_ZF]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = kq + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32;
+          if (!ADD)
+            mma_bf16_ts(tm + TM_Z, tm + TM_SB + 8 * kk, sdesc_sw128(koff, 16, 1024), ID_N64,
+                        kk > 0);
+          mma_bf16_ts(tmo, tm + TM_SB + 8 * kk, sdesc_sw128(koff + kTileBytes, 16, 1024),
+                      ID_N64, kk > 0);
         }
+        mma_commit(&bars[B_ZF]);
         // U^T = V^T T^T into the V' accumulator, once T of the chunk is
         // written and V has landed (the previous V' was converted: its VPR
-        // wait precedes in this thread).  PC: T is in the T' buffer.
-        if (!(ok = W(B_TRDY, ph) && W(B_VFULL, ph))) break;
+        // wait precedes in this thread).  T buffer c % 2 (PC: T is in the T'
+        // buffer).
+        if (!(ok = W(B_TRDY + (c & 1), (c >> 1) & 1) && W(B_VFULL, ph))) break;
         {
-          const uint32_t tt = PC ? a_tp + (c & 1) * kTileBytes : a_t;
+          const uint32_t tt = (PC ? a_tp : a_t) + (c & 1) * kTileBytes;
           if (!a.zero_v) {  // (v taken as zero: U = 0, the V' MMA starts the accumulator)
 #pragma unroll 1
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_ss(tm + TM_UV, sdesc_sw128(a_v + kk * 2048, kTileBytes, 1024),
                           sdesc_sw128(tt + kk * 32, 16, 1024), ID_U, kk > 0);
           }
-          mma_commit(&bars[B_UF]);      // T read: the prep group may write the next T
+          mma_commit(&bars[B_UF + (c & 1)]);  // T read: the prep group may write chunk c + 2's
           mma_commit(&bars[B_VEMPTY]);  // V read
         }
         // V'^T = U^T + Z (-T')^T, or (-Z) T'^T  (ADD: V'^T = U^T = V^T)
@@ -1163,31 +1188,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars[B_VPF]);
         if (!ADD) mma_commit(&bars[B_TPE + (c & 1)]);
-        // O_a = S_b Q^T, once the epilogue has read the previous chunk's O.
-        // Issued before the SF commit, which then also covers this last read
-        // of S_b (the state group overwrites S_b once SF completes).
-        if (c >= 1 && !(ok = W(B_OE, (c - 1) & 1))) break;
-#pragma unroll 1
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tm + TM_OA, tm + TM_SB + 8 * kk,
-                      sdesc_sw128(kq + kTileBytes + (kk >> 2) * 2 * kTileBytes + (kk & 3) * 32,
-                                  16, 1024),
-                      ID_N64, kk > 0);
-        // S_tmem += (V'^T decayed / sigma) K ;  O_b = V'^T P^T
+        // S_tmem += (V'^T decayed / sigma) K ;  O_b = V'^T P^T, with the bf16
+        // copies of V'^T in TMEM as A (PC: the plain copy serves both)
         if (!(ok = W(B_VPR, ph))) break;
         // B = K (MN-major); PC: K^ of the stage
         const uint32_t kb = PC ? a_kh + st * 2 * kTileBytes : kq;
         const uint32_t kb_lbo = PC ? kTileBytes : 2 * kTileBytes;
+        const uint32_t vpd = tm + TM_UV + (PC ? 0 : 32);
 #pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tm + TM_S, sdesc_sw128(a_vpd + kk * 32, 16, 1024),
-                      sdesc_sw128(kb + kk * 2048, kb_lbo, 1024), ID_S, 1);
+          mma_bf16_ts(tm + TM_S, vpd + 8 * kk, sdesc_sw128(kb + kk * 2048, kb_lbo, 1024), ID_S,
+                      1);
         mma_commit(&bars[B_SF]);
+        // O_b accumulated onto the scaled O_a (its scaling precedes the
+        // state group's VPR arrival)
         const uint32_t pp = a_p + (c & 1) * kTileBytes;
 #pragma unroll 1
         for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ss(tm + TM_O, sdesc_sw128(a_vp + kk * 32, 16, 1024),
-                      sdesc_sw128(pp + kk * 32, 16, 1024), ID_N64, kk > 0);
+          mma_bf16_ts(tmo, tm + TM_UV + 8 * kk, sdesc_sw128(pp + kk * 32, 16, 1024), ID_N64, 1);
         mma_commit(&bars[B_OF]);
         mma_commit(&bars[B_PE + (c & 1)]);
         mma_commit(&bars[B_EMPTY + st]);
@@ -1273,9 +1291,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool a_rows = !ADD && pt < 64;
       // (prologue: also the chunk's token norms, in place of the stage)
       bool bad = !wait_all<4>({PRO ? &bars[B_NORM + st] : &bars[B_FULL + st], &bars[B_D1F],
-                               &bars[B_PE + (c & 1)], a_rows ? &bars[B_TRDY] : &bars[B_D1F]},
+                               &bars[B_PE + (c & 1)],
+                               a_rows ? &bars[B_TRDY + ((c - 1) & 1)] : &bars[B_D1F]},
                               {uint32_t((c / kStages) & 1), ph, uint32_t(((c >> 1) - 1) & 1),
-                               a_rows ? uint32_t((c - 1) & 1) : ph},
+                               a_rows ? uint32_t(((c - 1) >> 1) & 1) : ph},
                               abort_flag);
       if (!bad && (!ADD || rl >= 64)) {
         const bool factored = -gcv[63] < kSafeDecay;
@@ -1343,20 +1362,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         warp_arrive(&bars[B_D1E]);  // this thread's D1 reads are done
       }
       if (ADD) {
-        // T = I throughout: only P is handed on, once U of the previous chunk
-        // has completed (which keeps TRDY within one phase of its waiter).
-        bad = bad || !warp_wait(&bars[B_UF], (c - 1) & 1, abort_flag, lane);
+        // T = I throughout: only P is handed on, once U of chunk c - 2 has
+        // completed (which keeps TRDY buffer c % 2 within one phase of its
+        // waiter).
+        bad = bad || !warp_wait(&bars[B_UF + (c & 1)], ((c >> 1) - 1) & 1, abort_flag, lane);
         if (group_any(kBar, bad)) { ok = false; break; }
-        warp_arrive(&bars[B_TRDY]);
+        warp_arrive(&bars[B_TRDY + (c & 1)]);
         continue;
       }
-      // ---- Y = (I + A)^{-1} -> T, T'.  T is free once U of the previous
-      //      chunk has completed, this T' buffer once V' of chunk c - 2 has.
+      // ---- Y = (I + A)^{-1} -> T, T' (buffers c % 2): free once U (T) and
+      //      V' (T') of chunk c - 2 have completed.
       uint8_t *tpc = sm + Lay::TP + (c & 1) * kTileBytes;
-      const TOut to{PC ? tpc : sm + Lay::T, tpc, bs,
+      const TOut to{PC ? tpc : sm + Lay::T + (c & 1) * kTileBytes, tpc, bs,
                     PC ? egv : gv + (PRO ? kGateSEgK : kGateSEg)};
-      bad = bad || !wait_all<2>({&bars[B_UF], &bars[B_TPE + (c & 1)]},
-                                {uint32_t((c - 1) & 1), uint32_t(((c >> 1) - 1) & 1)}, abort_flag);
+      bad = bad || !wait_all<2>({&bars[B_UF + (c & 1)], &bars[B_TPE + (c & 1)]},
+                                {uint32_t(((c >> 1) - 1) & 1), uint32_t(((c >> 1) - 1) & 1)},
+                                abort_flag);
       if (!bad && rl < 64) {  // the warps that wrote A invert its diagonal blocks
         __syncwarp();
         invert_diag(AF, to, rl >> 5, lane);
@@ -1372,7 +1393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         invert_level2<!PC>(AF, ysc, wscr, to, pt);
       }
       fence_proxy_async_smem();
-      warp_arrive(&bars[B_TRDY]);  // this thread's T, T', P writes are done
+      warp_arrive(&bars[B_TRDY + (c & 1)]);  // this thread's T, T', P writes are done
     }
     if (!ok && pt == 0) atomicOr(a.status, kStatusTimeout);
   } else if (warp < 4) {
@@ -1543,11 +1564,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = c & 1;
       const float *sv = reinterpret_cast<const float *>(svec(c));
       const float *egv = sv + kSvEg, *eglv = sv + kSvEgl;
+      const uint32_t tmo = lane_base + ((c & 1) ? TM_O1 : TM_O0);
       // ---- Z (scalar gates: T' is stored negated) or -Z (per-channel gates,
       //      whose T' buffer is T itself) -> bf16 A operand, in place in TMEM
-      if (!ADD) {
+      //      (ZF also covers O_a)
       if (!warp_wait(&bars[B_ZF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
+      if (!ADD) {
       {
         // both halves are loaded before either is overwritten in place
         float z0[32], z1[32];
@@ -1569,29 +1592,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       warp_arrive(&bars[B_ZR]);
       }
-      // ---- V'^T -> bf16 operands (plain, and decayed to the chunk end / sigma)
+      // ---- O_a Diag(sigma e^{gc}) in place (fp32), off the chain: the
+      //      state group would otherwise wait for V' here.  O_b is then
+      //      accumulated onto it.  (PC: the factors are 1, Q~ carries the
+      //      decay.)  Stored before the VPR arrival below.
+      if (!PC) {
+#pragma unroll 1
+        for (int q = 0; q < 2; ++q) {
+          float x[32];
+          tmem_ld32(tmo + 32 * q, x);
+          const float4 *e4 = reinterpret_cast<const float4 *>(egv + 32 * q);
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const float4 e = e4[s4];
+            x[4 * s4] *= e.x;
+            x[4 * s4 + 1] *= e.y;
+            x[4 * s4 + 2] *= e.z;
+            x[4 * s4 + 3] *= e.w;
+          }
+          tmem_st16(tmo + 32 * q, *reinterpret_cast<float(*)[16]>(x));
+          tmem_st16(tmo + 32 * q + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+        }
+      }
+      // ---- V'^T -> its bf16 A operands, in place in TMEM: plain in columns
+      //      0-31, decayed to the chunk end / sigma in 32-63 (PC: the plain
+      //      copy serves both)
       if (!warp_wait(&bars[B_VPF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
-      if (lane == 0) tma_store_wait_read0();  // the previous o store has read VPD
-      __syncwarp();
-#pragma unroll 1
-      for (int q = 0; q < 2; ++q) {
-        float x[32];
-        tmem_ld32(lane_base + TM_UV + 32 * q, x);
-        DBG_ROW(40960 + 32 * q, 64, x);
-        st_row32_sw128(sm + Lay::VP, i, q, x);
-        const float4 *e4 = reinterpret_cast<const float4 *>(eglv + 32 * q);
+      {
+        // both halves are loaded before either is overwritten in place
+        float x0[32], x1[32];
+        tmem_ld32(lane_base + TM_UV, x0);
+        tmem_ld32(lane_base + TM_UV + 32, x1);
+        DBG_ROW(40960, 64, x0);
+        DBG_ROW(40960 + 32, 64, x1);
+        uint32_t u[16];
 #pragma unroll
-        for (int s4 = 0; s4 < 8; ++s4) {
-          const float4 e = e4[s4];
-          x[4 * s4] *= e.x;
-          x[4 * s4 + 1] *= e.y;
-          x[4 * s4 + 2] *= e.z;
-          x[4 * s4 + 3] *= e.w;
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x0[2 * e], x0[2 * e + 1]);
+        tmem_st16u(lane_base + TM_UV, u);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x1[2 * e], x1[2 * e + 1]);
+        tmem_st16u(lane_base + TM_UV + 16, u);
+        if (!PC) {
+          const float4 *e4 = reinterpret_cast<const float4 *>(eglv);
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const float4 e = e4[s4];
+            u[2 * s4] = pack_bf16(x0[4 * s4] * e.x, x0[4 * s4 + 1] * e.y);
+            u[2 * s4 + 1] = pack_bf16(x0[4 * s4 + 2] * e.z, x0[4 * s4 + 3] * e.w);
+          }
+          tmem_st16u(lane_base + TM_UV + 32, u);
+#pragma unroll
+          for (int s4 = 0; s4 < 8; ++s4) {
+            const float4 e = e4[8 + s4];
+            u[2 * s4] = pack_bf16(x1[4 * s4] * e.x, x1[4 * s4 + 1] * e.y);
+            u[2 * s4 + 1] = pack_bf16(x1[4 * s4 + 2] * e.z, x1[4 * s4 + 3] * e.w);
+          }
+          tmem_st16u(lane_base + TM_UV + 48, u);
         }
-        st_row32_sw128(sm + Lay::VPD, i, q, x);
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       warp_arrive(&bars[B_VPR]);
       // next chunk's gate factors, while the state update runs
@@ -1644,17 +1704,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
         }
       }
-      // ---- O = O_a Diag(e^{gc}) + O_b -> bf16, stored straight to o
+      // ---- O (= O_a Diag(sigma e^{gc}) + O_b, in buffer c % 2) -> bf16 -> o
       if (!warp_wait(&bars[B_OF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
         // The warp stages its 32 channels x 64 tokens (bf16, [token][channel],
-        // 64-byte rows) in its own rows of VPD, free once the state update
-        // has read them, and one lane stores the box with TMA (rows past T
-        // are clipped).  O is read in the 16-lane shape, which gives each
+        // 64-byte rows) in its own quarter of STG, free once the warp's
+        // previous store has read it, and one lane stores the box with TMA
+        // (rows past T are clipped).  O is read in the 16-lane shape, which gives each
         // thread two adjacent tokens of a channel, so one transposing matrix
         // store writes 8 tokens x 32 channels per warp.
-        const uint32_t stg = smem_u32(sm + Lay::VPD + 4096 * warp);
+        if (lane == 0) tma_store_wait_read0();  // the previous o store has read STG
+        __syncwarp();
+        const uint32_t stg = smem_u32(sm + Lay::STG + 4096 * warp);
         // row address of this thread in a matrix store: token 8 k + lane % 8
         // of channel group lane / 8 (matrix j = lane / 8 holds channels
         // 8 j .. 8 j + 7).  The staging tile is 64-byte swizzled (16-byte
@@ -1662,30 +1724,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // expects), so the 8 rows of a matrix fall in distinct banks.
         const int r8 = lane & 7;
         const uint32_t row_addr = stg + r8 * 64 + 16 * ((lane >> 3) ^ ((r8 >> 1) & 3));
-        const int tq = lane & 3;
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
           // lanes 0-15 / 16-31 of the warp's quarter, tokens 32 q .. 32 q + 31
-          float a0[16], a1[16], b0[16], b1[16];
-          tmem_ld16x256b_x4(lane_base + TM_OA + 32 * q, a0);
-          tmem_ld16x256b_x4(lane_base + (16u << 16) + TM_OA + 32 * q, a1);
-          tmem_ld16x256b_x4(lane_base + TM_O + 32 * q, b0);
-          tmem_ld16x256b_x4(lane_base + (16u << 16) + TM_O + 32 * q, b1);
+          float a0[16], a1[16];
+          tmem_ld16x256b_x4(tmo + 32 * q, a0);
+          tmem_ld16x256b_x4(tmo + (16u << 16) + 32 * q, a1);
           tmem_wait_ld();
-          if (q == 1) {  // every read of O_a / O_b is done
+          if (q == 1) {  // every read of this O buffer is done
             tc_fence_before();
-            warp_arrive(&bars[B_OE]);
+            warp_arrive(&bars[B_OE + (c & 1)]);
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k) {  // tokens 32 q + 8 k + 2 tq, + 1
-            const float2 ev = *reinterpret_cast<const float2 *>(egv + 32 * q + 8 * k + 2 * tq);
             const int e = 4 * k;
-            stmatrix_x4_trans(
-                row_addr + (4 * q + k) * 512,
-                pack_bf16(ev.x * a0[e] + b0[e], ev.y * a0[e + 1] + b0[e + 1]),
-                pack_bf16(ev.x * a0[e + 2] + b0[e + 2], ev.y * a0[e + 3] + b0[e + 3]),
-                pack_bf16(ev.x * a1[e] + b1[e], ev.y * a1[e + 1] + b1[e + 1]),
-                pack_bf16(ev.x * a1[e + 2] + b1[e + 2], ev.y * a1[e + 3] + b1[e + 3]));
+            stmatrix_x4_trans(row_addr + (4 * q + k) * 512, pack_bf16(a0[e], a0[e + 1]),
+                              pack_bf16(a0[e + 2], a0[e + 3]), pack_bf16(a1[e], a1[e + 1]),
+                              pack_bf16(a1[e + 2], a1[e + 3]));
           }
         }
         fence_proxy_async_smem();
@@ -1696,7 +1751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the next sequence's rows, so the valid rows go out with plain
           // 16-byte stores (chunk j of staging row r sits at j ^ ((r / 2) % 4)).
           if (a.write_o) {
-            const uint8_t *st = sm + Lay::VPD + 4096 * warp;
+            const uint8_t *st = sm + Lay::STG + 4096 * warp;
             for (int r = lane; r < rows; r += 32) {
               uint4 *dst = reinterpret_cast<uint4 *>(
                   reinterpret_cast<__nv_bfloat16 *>(a.o) +
@@ -1708,7 +1763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else if (lane == 0) {
           if (a.write_o)
-            tma_store_4d(&tmO, sm + Lay::VPD + 4096 * warp, 32 * warp, h, tb + c * C, bt);
+            tma_store_4d(&tmO, sm + Lay::STG + 4096 * warp, 32 * warp, h, tb + c * C, bt);
           tma_store_commit();
         }
       }
