@@ -183,98 +183,111 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, rank, world, local_rank):
+def make_step(w, dev, rank, nsteps):
+    """The workload's inputs on the device and one step of it through the
+    binding.  Returns a dict: step (callable), host (CPU inputs), d (device
+    inputs), o, S_T, S (decode state), grads, results (what a step returns to
+    its caller), launches (kernels per step)."""
     from gated_delta_rule_93_b200 import binding
 
-    w = WORKLOADS[args.workload]
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream(dev)
+    r = {"grads": None, "S": None, "S_T": None}
     if w.kind == "step":
         # decode: one gdr_step over all N x H states per step, inputs of the
-        # first (warmup + steps) steps resident, the state updated in place
-        nsteps = args.warmup + args.steps + 3
+        # first nsteps steps resident, the state updated in place
         host = make_workload_inputs(w, seed=rank, steps=nsteps)
         d = {k: v.to(dev) for k, v in host.items()}
         S = d["S0"].clone()
         o = torch.empty(w.B, w.H, w.dv, dtype=w.dtype, device=dev)
         it = [0]
-        launches_per_step = 1
 
         def step():
             i = it[0] % nsteps
             it[0] += 1
             binding.step(d["q"][i], d["k"][i], d["v"][i], d["g"][i], d["beta"][i], S, o=o)
 
-        S_T = None
-    else:
-        host = make_workload_inputs(w, seed=rank)
-        d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
-        o = torch.empty(w.B, w.T, w.H, w.dv, dtype=w.dtype, device=dev)
-        S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev) \
-            if w.want_S_T else None
-        # scratch of the segment path (long sequences with few heads), if any
-        ws_bytes = binding.chunk_fwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.C, w.dtype,
-                                                     w.gate)
-        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
-        launches_per_step = binding.chunk_fwd_kernel_launches(w.B, w.T, w.H, w.dk, w.dv, w.C,
-                                                              w.dtype, w.gate)
+        r.update(step=step, host=host, d=d, o=o, S=S, launches=1, results=[o])
+        return r
+    host = make_workload_inputs(w, seed=rank)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
+    o = torch.empty(w.B, w.T, w.H, w.dv, dtype=w.dtype, device=dev)
+    S_T = torch.empty(w.B, w.H, w.dv, w.dk, dtype=torch.float32, device=dev) \
+        if w.want_S_T else None
+    # scratch of the segment path (long sequences with few heads), if any
+    ws_bytes = binding.chunk_fwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.C, w.dtype,
+                                                 w.gate)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    launches = binding.chunk_fwd_kernel_launches(w.B, w.T, w.H, w.dk, w.dv, w.C, w.dtype,
+                                                 w.gate)
+
+    def step():
+        binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o,
+                          S_T=S_T, output_final_state=S_T is not None, workspace=ws)
+
+    if w.prologue:  # raw projections in: one launch, no workspace
+        launches = 1
 
         def step():
-            binding.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o=o,
-                              S_T=S_T, output_final_state=S_T is not None, workspace=ws)
+            binding.chunk_fwd_prologue(d["q"], d["k"], d["v"], d["a"], d["b"],
+                                       d["gate_scale"], d["S0"], o=o, S_T=S_T,
+                                       output_final_state=S_T is not None)
 
-        if w.prologue:  # raw projections in: one launch, no workspace
-            launches_per_step = 1
+    grads = None
+    if w.backward:  # gradients for a seeded dL/do; preallocated outputs and workspace
+        launches = 1
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = dict(dq=torch.empty(w.B, w.T, w.H, w.dk, **f32),
+                     dk=torch.empty(w.B, w.T, w.H, w.dk, **f32),
+                     dv=torch.empty(w.B, w.T, w.H, w.dv, **f32),
+                     dg=torch.empty(tuple(d["g"].shape), **f32),
+                     dbeta=torch.empty(w.B, w.T, w.H, **f32), dS0=None)
+        bws = torch.empty(binding.chunk_bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv),
+                          dtype=torch.uint8, device=dev)
+        o, S_T = grads["dq"], None
 
-            def step():
-                binding.chunk_fwd_prologue(d["q"], d["k"], d["v"], d["a"], d["b"],
-                                           d["gate_scale"], d["S0"], o=o, S_T=S_T,
-                                           output_final_state=S_T is not None)
+        def step():
+            binding.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dout"], d["S0"],
+                              None, want_dS0=False, workspace=bws, out=grads)
 
-        if w.backward:  # gradients for a seeded dL/do; preallocated outputs and workspace
-            launches_per_step = 1
-            f32 = dict(dtype=torch.float32, device=dev)
-            grads = dict(dq=torch.empty(w.B, w.T, w.H, w.dk, **f32),
-                         dk=torch.empty(w.B, w.T, w.H, w.dk, **f32),
-                         dv=torch.empty(w.B, w.T, w.H, w.dv, **f32),
-                         dg=torch.empty(tuple(d["g"].shape), **f32),
-                         dbeta=torch.empty(w.B, w.T, w.H, **f32), dS0=None)
-            bws = torch.empty(binding.chunk_bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv),
-                              dtype=torch.uint8, device=dev)
-            o, S_T = grads["dq"], None
+    if w.mixer == "dplr":  # recurrent DPLR forward on CUDA cores: one launch
+        launches = 1
 
-            def step():
-                binding.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dout"], d["S0"],
-                                  None, want_dS0=False, workspace=bws, out=grads)
+        def step():
+            binding.dplr_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["g"], d["S0"], o=o,
+                             S_T=S_T, output_final_state=S_T is not None)
 
-        if w.mixer == "dplr":  # recurrent DPLR forward on CUDA cores: one launch
-            launches_per_step = 1
+    if w.mixer == "gla":  # gated linear attention: one launch, no beta, no workspace
+        host.pop("beta")
+        d.pop("beta")
+        launches = 1
 
-            def step():
-                binding.dplr_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["g"], d["S0"], o=o,
-                                 S_T=S_T, output_final_state=S_T is not None)
+        def step():
+            binding.chunk_fwd_gla(d["q"], d["k"], d["v"], d["g"], d["S0"], o=o, S_T=S_T,
+                                  output_final_state=S_T is not None)
 
-        if w.mixer == "gla":  # gated linear attention: one launch, no beta, no workspace
-            host.pop("beta")
-            d.pop("beta")
-            launches_per_step = 1
+    results = [grads[n] for n in ("dq", "dk", "dv", "dg", "dbeta")] if w.backward else \
+        [o] + ([S_T] if S_T is not None else [])
+    r.update(step=step, host=host, d=d, o=o, S_T=S_T, grads=grads, launches=launches,
+             results=results)
+    return r
 
-            def step():
-                binding.chunk_fwd_gla(d["q"], d["k"], d["v"], d["g"], d["S0"], o=o, S_T=S_T,
-                                      output_final_state=S_T is not None)
+
+def time_device(step, steps, warmup, dev, world, local_rank):
+    """W untimed steps, then K steps timed with CUDA events on the launching
+    stream between barriers and synchronisations, SM clocks sampled during
+    the region.  Returns (total ms, per-step ms list, clocks)."""
+    from gated_delta_rule_93_b200 import binding
+
+    stream = torch.cuda.current_stream(dev)
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
     if binding.device_status() != 0:
         raise RuntimeError("device status word set during warm-up")
-
-    # ---- device-timed region: inputs resident in HBM, one launch per step
     vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
     clocks = ClockSampler(vis[local_rank].strip() if local_rank < len(vis) else local_rank)
     clocks.start()
@@ -282,11 +295,16 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize(dev)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+          for _ in range(steps)]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    # Hold the stream with a short spin (torch's, before the timed region)
+    # while the host enqueues the K steps, so that the events time the
+    # device's back-to-back execution and not the host's per-call latency
+    # (which would dominate small workloads).
+    torch.cuda._sleep(int(1e6 * (steps + 2)))
     t0.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
@@ -294,12 +312,95 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     barrier()
     clk = clocks.stop()
-    total_ms = t0.elapsed_time(t1)
-    per_launch_ms = [a.elapsed_time(b) for a, b in ev]
     if binding.device_status() != 0:
         raise RuntimeError("device status word set during the timed region")
+    return t0.elapsed_time(t1), [a.elapsed_time(b) for a, b in ev], clk
+
+
+def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk):
+    """tokens/s, TFLOP/s and the roofline of one timed workload."""
+    ms_step = total_ms / steps
+    tokens_step = w.B * w.T if w.kind == "chunk" else w.B  # tokens one step processes
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    abytes = algorithmic_bytes(w)
+    aflops = algorithmic_flops(w, w.C)
+    avg_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
+    achieved = abytes / (avg_launch_ms / 1e3) / 1e9
+    roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (tc_peak * 1e12)) * 1e3
+    alu = w.backward or w.mixer == "dplr"
+    alu_peak = None
+    if alu:  # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x SM clock
+        alu_peak = 148 * 128 * 2 * ((clk or {}).get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
+        roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (alu_peak * 1e12)) * 1e3
+    if alu:
+        roof = {"bound": "alu", "achieved": aflops / (avg_launch_ms / 1e3) / 1e12,
+                "peak": alu_peak, "unit": "TFLOP/s",
+                "frac": aflops / (avg_launch_ms / 1e3) / 1e12 / alu_peak,
+                "traffic": recorded_traffic(w.name, "dplr" if w.mixer == "dplr" else "bwd"),
+                "peak_source": "CUDA-core fp32 FMA, 148 SMs x 128 lanes x 2 flop x max SM "
+                               "clock", "algorithmic_flops_per_launch": aflops,
+                "kernel": "gdr_dplr_fwd" if w.mixer == "dplr" else "gdr_chunk_bwd"}
+    else:
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
+                "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
+                "kernel": ("gdr_chunk_fwd_prologue" if w.prologue else
+                           "gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
+                if w.kind == "chunk" else "gdr_step"}
+    return {"value": world * tokens_step * steps / (total_ms / 1e3), "ms_per_step": ms_step,
+            "tflops": aflops * world * steps / (total_ms / 1e3) / 1e12,
+            "roofline_time_ms": roof_ms, "roofline_fraction": roof_ms / ms_step,
+            "roofline": roof, "tokens_step": tokens_step}
+
+
+# The other workloads of the benchmark, timed in the same process after the
+# headline one (one GPU): the long sequence (segment path), the per-channel
+# gate, the decode step and the tiny fp32 forward.
+EXTRA_WORKLOADS = ("gdn_b1_t65536_h16_d128", "kda_b8_t4096_h16_d128",
+                   "decode_n256_h16_d128_x1024", "tiny_fp32")
+
+
+def time_extra(name, args, rank, world, local_rank, dev):
+    w = WORKLOADS[name]
+    steps, warmup = max(5, min(args.steps, 20)), 3
+    r = make_step(w, dev, rank, warmup + steps + 3)
+    total_ms, per_launch, clk = time_device(r["step"], steps, warmup, dev, world, local_rank)
+    f = roofline_fields(w, total_ms, per_launch, steps, world, clk)
+    out = {"metric_value": f["value"], "unit": "tokens/s", "ms_per_step": f["ms_per_step"],
+           "steps": steps, "warmup": warmup, "tflops": f["tflops"],
+           "roofline_fraction": f["roofline_fraction"], "roofline": f["roofline"],
+           "gpu_launches": steps * r["launches"], "clocks": clk,
+           "config": {"B": w.B, "T": w.T if w.kind == "chunk" else 1, "H": w.H, "d_k": w.dk,
+                      "d_v": w.dv, "gate": w.gate, "S0": w.with_S0, "S_T": w.want_S_T,
+                      "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32"}}
+    if w.kind == "step":
+        out["config"]["note"] = ("one gdr_step over all 256 x 16 states per step; the state "
+                                 "is updated in place (%d consecutive steps timed)" % steps)
+    del r
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    r = make_step(w, dev, rank, args.warmup + args.steps + 3)
+    step, host, d, o, S_T, S = r["step"], r["host"], r["d"], r["o"], r["S_T"], r["S"]
+    launches_per_step = r["launches"]
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    # ---- device-timed region: inputs resident in HBM
+    total_ms, per_launch_ms, clk = time_device(step, args.steps, args.warmup, dev, world,
+                                               local_rank)
 
     # ---- end to end through the same API with host buffers (pinned)
+    from gated_delta_rule_93_b200 import binding
+
     if w.kind == "step":
         # per step: that step's q, k, v, g, beta go host -> device, o comes back;
         # the state stays resident (it is the decoder's cache)
@@ -309,8 +410,7 @@ def run_ours(args, rank, world, local_rank):
         pin = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
         dev_in = d
     # the step's results read back: o (and S_T), or every gradient
-    results = [grads[n] for n in ("dq", "dk", "dv", "dg", "dbeta")] if w.backward else \
-        [o] + ([S_T] if S_T is not None else [])
+    results = r["results"]
     res_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in results]
     h2d = sum(v.numel() * v.element_size() for v in pin.values() if v is not None)
     d2h = sum(t.numel() * t.element_size() for t in res_h)
@@ -343,30 +443,26 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- max over ranks
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
+    f = roofline_fields(w, total_ms, per_launch_ms, args.steps, world, clk)
+
+    # ---- the other workloads, each timed on its own after the headline one
+    extras = {}
+    if world == 1 and not args.no_extra and w.name == DEFAULT_WORKLOAD:
+        del r, step, host, d, dev_in, pin, results, res_h
+        torch.cuda.empty_cache()
+        for name in EXTRA_WORKLOADS:
+            extras[name] = time_extra(name, args, rank, world, local_rank, dev)
 
     if rank != 0:
         return None
-    ms_step = total_ms / args.steps
-    tokens_step = w.B * w.T if w.kind == "chunk" else w.B  # tokens one step processes
-    value = world * tokens_step * args.steps / (total_ms / 1e3)
-    hbm_peak, tc_peak, peak_kind = measured_peaks()
-    abytes = algorithmic_bytes(w)
-    aflops = algorithmic_flops(w, w.C)
-    avg_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
-    achieved = abytes / (avg_launch_ms / 1e3) / 1e9
-    roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (tc_peak * 1e12)) * 1e3
-    alu = w.backward or w.mixer == "dplr"
-    if alu:  # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x SM clock
-        alu_peak = 148 * 128 * 2 * ((clk or {}).get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
-        roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (alu_peak * 1e12)) * 1e3
     line = {
         "metric": METRIC,
-        "value": value,
+        "value": f["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": ms_step,
+        "ms_per_step": f["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -380,29 +476,20 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"independent (b,h) shards x{world}",
                    "l2": "inputs exceed L2 (%.0f MB > 126 MB); no flush" %
                          (algorithmic_bytes(w) / 1e6)},
-        "tflops": aflops * world * args.steps / (total_ms / 1e3) / 1e12,
-        "roofline_time_ms": roof_ms,
-        "roofline_fraction": roof_ms / ms_step,
-        "roofline": ({"bound": "alu", "achieved": aflops / (avg_launch_ms / 1e3) / 1e12,
-                      "peak": alu_peak, "unit": "TFLOP/s",
-                      "frac": aflops / (avg_launch_ms / 1e3) / 1e12 / alu_peak,
-                      "traffic": recorded_traffic(w.name, "dplr" if w.mixer == "dplr" else "bwd"),
-                      "peak_source": "CUDA-core fp32 FMA, 148 SMs x 128 lanes "
-                      "x 2 flop x max SM clock", "algorithmic_flops_per_launch": aflops,
-                      "kernel": "gdr_dplr_fwd" if w.mixer == "dplr" else "gdr_chunk_bwd"}
-                     if alu else
-                     {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
-                     "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
-                     "kernel": ("gdr_chunk_fwd_prologue" if w.prologue else
-                                "gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
-                     if w.kind == "chunk" else "gdr_step"}),
-        "e2e": {"value": world * tokens_step * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        "tflops": f["tflops"],
+        "roofline_time_ms": f["roofline_time_ms"],
+        "roofline_fraction": f["roofline_fraction"],
+        "roofline": f["roofline"],
+        "e2e": {"value": world * f["tokens_step"] * e2e_steps / (e2e_ms / 1e3),
+                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": args.steps * launches_per_step,
         "clocks": clk,
     }
+    if extras:
+        line["configs"] = extras
+        line["gpu_launches_all"] = line["gpu_launches"] + sum(
+            x["gpu_launches"] for x in extras.values())
     if rank == 0 and world == 1 and not args.no_cpu_baseline and w.kind == "chunk":
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     return line
@@ -509,6 +596,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the chosen workload (not the other workloads after it)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-tokens", type=int, default=64)
     args = ap.parse_args()

@@ -1148,7 +1148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // these last reads of S_b (the state group overwrites S_b once SF
         // completes).  (ADD: no correction; no Z.)
         if (!(ok = W(B_SBR, ph) && W(B_FULL + st, (c / kStages) & 1))) break;
-        if (c >= 2 && !(ok = W(B_OE + (c & 1), ((c >> 1) - 1) & 1))) break;
+        // (segment passes that write no o skip O_a and O_b altogether)
+        const bool wo = a.write_o != 0;
+        if (wo && c >= 2 && !(ok = W(B_OE + (c & 1), ((c >> 1) - 1) & 1))) break;
         const uint32_t tmo = tm + ((c & 1) ? TM_O1 : TM_O0);
 #pragma unroll 1
         for (int kk = 0; kk < 8; ++kk) {
@@ -1156,8 +1158,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ADD)
             mma_bf16_ts(tm + TM_Z, tm + TM_SB + 8 * kk, sdesc_sw128(koff, 16, 1024), ID_N64,
                         kk > 0);
-          mma_bf16_ts(tmo, tm + TM_SB + 8 * kk, sdesc_sw128(koff + kTileBytes, 16, 1024),
-                      ID_N64, kk > 0);
+          if (wo)
+            mma_bf16_ts(tmo, tm + TM_SB + 8 * kk, sdesc_sw128(koff + kTileBytes, 16, 1024),
+                        ID_N64, kk > 0);
         }
         mma_commit(&bars[B_ZF]);
         // U^T = V^T T^T into the V' accumulator, once T of the chunk is
@@ -1203,10 +1206,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O_b accumulated onto the scaled O_a (its scaling precedes the
         // state group's VPR arrival)
         const uint32_t pp = a_p + (c & 1) * kTileBytes;
+        if (wo) {
 #pragma unroll 1
-        for (int kk = 0; kk < 4; ++kk)
-          mma_bf16_ts(tmo, tm + TM_UV + 8 * kk, sdesc_sw128(pp + kk * 32, 16, 1024), ID_N64, 1);
-        mma_commit(&bars[B_OF]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tmo, tm + TM_UV + 8 * kk, sdesc_sw128(pp + kk * 32, 16, 1024), ID_N64,
+                        1);
+          mma_commit(&bars[B_OF]);
+        }
         mma_commit(&bars[B_PE + (c & 1)]);
         mma_commit(&bars[B_EMPTY + st]);
       }
@@ -1296,7 +1302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                               {uint32_t((c / kStages) & 1), ph, uint32_t(((c >> 1) - 1) & 1),
                                a_rows ? uint32_t(((c - 1) >> 1) & 1) : ph},
                               abort_flag);
-      if (!bad && (!ADD || rl >= 64)) {
+      if (!bad && (!ADD || rl >= 64) && (rl < 64 || a.write_o)) {
         const bool factored = -gcv[63] < kSafeDecay;
         // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns at a time
         tc_fence_after();
@@ -1596,7 +1602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       //      state group would otherwise wait for V' here.  O_b is then
       //      accumulated onto it.  (PC: the factors are 1, Q~ carries the
       //      decay.)  Stored before the VPR arrival below.
-      if (!PC) {
+      if (!PC && a.write_o) {
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
           float x[32];
@@ -1705,6 +1711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // ---- O (= O_a Diag(sigma e^{gc}) + O_b, in buffer c % 2) -> bf16 -> o
+      if (!a.write_o) continue;
       if (!warp_wait(&bars[B_OF], ph, abort_flag, lane)) { ok = false; break; }
       tc_fence_after();
       {
