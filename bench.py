@@ -42,7 +42,9 @@ KERNEL_SOURCES = {
               "gated_delta_rule_93_b200/csrc/gdr_segments.cu",
               "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
     "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu"],
-    "bwd": ["gated_delta_rule_93_b200/csrc/gdr_bwd.cu"],
+    "bwd": ["gated_delta_rule_93_b200/csrc/gdr_bwd.cu",
+            "gated_delta_rule_93_b200/csrc/gdr_bwd_tc.cu",
+            "gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu"],
     "dplr": ["gated_delta_rule_93_b200/csrc/gdr_dplr.cu"],
 }
 
@@ -80,6 +82,12 @@ def algorithmic_flops(w, C=64):
         return w.B * w.T * w.H * (4 * w.dk * w.dv + C * (w.dk + w.dv))
     per = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0
     return w.B * w.T * w.H * per
+
+
+def backward_on_tensor_cores(w):
+    """The backward's tensor-core path: bf16, d_k = d_v = 128, scalar gate."""
+    return (w.backward and w.dtype == torch.bfloat16 and w.dk == 128 and w.dv == 128
+            and w.gate == "scalar" and w.T > 0)
 
 
 def measured_peaks():
@@ -233,14 +241,17 @@ def make_step(w, dev, rank, nsteps):
 
     grads = None
     if w.backward:  # gradients for a seeded dL/do; preallocated outputs and workspace
-        launches = 1
+        # (tensor cores: the forward rerun with a stash, the reverse state
+        # pass and the chunk-parallel gradient pass; else one CUDA-core launch)
+        launches = 3 if backward_on_tensor_cores(w) else 1
         f32 = dict(dtype=torch.float32, device=dev)
         grads = dict(dq=torch.empty(w.B, w.T, w.H, w.dk, **f32),
                      dk=torch.empty(w.B, w.T, w.H, w.dk, **f32),
                      dv=torch.empty(w.B, w.T, w.H, w.dv, **f32),
                      dg=torch.empty(tuple(d["g"].shape), **f32),
                      dbeta=torch.empty(w.B, w.T, w.H, **f32), dS0=None)
-        bws = torch.empty(binding.chunk_bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv),
+        bws = torch.empty(binding.chunk_bwd_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.dtype,
+                                                            w.gate),
                           dtype=torch.uint8, device=dev)
         o, S_T = grads["dq"], None
 
@@ -327,7 +338,7 @@ def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk):
     avg_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
     achieved = abytes / (avg_launch_ms / 1e3) / 1e9
     roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (tc_peak * 1e12)) * 1e3
-    alu = w.backward or w.mixer == "dplr"
+    alu = (w.backward and not backward_on_tensor_cores(w)) or w.mixer == "dplr"
     alu_peak = None
     if alu:  # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x SM clock
         alu_peak = 148 * 128 * 2 * ((clk or {}).get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
@@ -342,9 +353,11 @@ def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk):
                 "kernel": "gdr_dplr_fwd" if w.mixer == "dplr" else "gdr_chunk_bwd"}
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": recorded_traffic(w.name, w.kind),
+                "frac": achieved / hbm_peak,
+                "traffic": recorded_traffic(w.name, "bwd" if w.backward else w.kind),
                 "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
-                "kernel": ("gdr_chunk_fwd_prologue" if w.prologue else
+                "kernel": ("gdr_chunk_bwd (tensor cores, 3 launches)" if w.backward else
+                           "gdr_chunk_fwd_prologue" if w.prologue else
                            "gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
                 if w.kind == "chunk" else "gdr_step"}
     return {"value": world * tokens_step * steps / (total_ms / 1e3), "ms_per_step": ms_step,

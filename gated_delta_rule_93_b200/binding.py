@@ -84,7 +84,7 @@ def lib():
             L.gdr_chunk_fwd_prologue.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, i, i,
                                                  i, i, i, i, i, vp]
             L.gdr_chunk_fwd_prologue.restype = i
-            L.gdr_chunk_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
+            L.gdr_chunk_bwd_workspace_bytes.argtypes = [i, i, i, i, i, i, i]
             L.gdr_chunk_bwd_workspace_bytes.restype = sz
             L.gdr_chunk_bwd.argtypes = [vp, vp, vp, i, vp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                         vp, i, i, i, i, i, vp, sz, vp]
@@ -440,8 +440,10 @@ def chunk_fwd_prologue(q, k, v, a, b, gate_scale, S0=None, *, norm_q=True, norm_
     return o, S_T
 
 
-def chunk_bwd_workspace_bytes(B, T, H, dk, dv):
-    return int(lib().gdr_chunk_bwd_workspace_bytes(B, T, H, dk, dv))
+def chunk_bwd_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, gate="scalar"):
+    """Workspace ``chunk_bwd`` needs for this shape, input dtype and gate kind."""
+    gk = GDR_GATE_PER_CHANNEL if gate == "channel" else GDR_GATE_SCALAR
+    return int(lib().gdr_chunk_bwd_workspace_bytes(B, T, H, dk, dv, _in_dtype(dtype), gk))
 
 
 def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, *, want_dS0=True, workspace=None,
@@ -481,7 +483,7 @@ def chunk_bwd(q, k, v, g, beta, dout, S0=None, dS_T=None, *, want_dS0=True, work
         _need(out[name], name, torch.float32, shape, dev)
     if out.get("dS0") is not None:
         _need(out["dS0"], "dS0", torch.float32, (B, H, dv, dk), dev)
-    ws = chunk_bwd_workspace_bytes(B, T, H, dk, dv)
+    ws = chunk_bwd_workspace_bytes(B, T, H, dk, dv, dt, "channel" if gk else "scalar")
     if workspace is None and ws:
         workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
     with torch.cuda.device(dev):

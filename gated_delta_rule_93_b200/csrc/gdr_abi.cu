@@ -388,8 +388,18 @@ gdr_status gdr_dplr_fwd(const void *q, const void *k, const void *v, const void 
                    "gdr_dplr_fwd launch");
 }
 
-size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv) {
+namespace {
+// The backward's path for a shape: the tensor-core chunked backward, or the
+// per-step recurrence on CUDA cores.
+bool bwd_on_tensor_cores(int T, int d, gdr_dtype in_dtype, gdr_gate_kind gate) {
+  return T > 0 && gdr::bwd_tc_supports(in_dtype == GDR_BF16, gate == GDR_GATE_PER_CHANNEL, d);
+}
+}  // namespace
+
+size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype in_dtype,
+                                     gdr_gate_kind gate) {
   if (dk != dv || (dk != 32 && dk != 64 && dk != 128)) return 0;
+  if (bwd_on_tensor_cores(T, dk, in_dtype, gate)) return gdr::bwd_tc_ws_bytes(B, T, H);
   return gdr::bwd_ws_bytes(B, T, H, dk);
 }
 
@@ -413,15 +423,28 @@ gdr_status gdr_chunk_bwd(const void *q, const void *k, const void *v, gdr_dtype 
     if (!q || !k || !v || !g || !beta || !dout || !dq || !dk || !dv || !dg || !dbeta)
       return fail(GDR_ERR_INVALID_ARG, "null input or gradient pointer");
   }
-  const size_t need = gdr::bwd_ws_bytes(B, T, H, dk_);
+  const size_t need = gdr_chunk_bwd_workspace_bytes(B, T, H, dk_, dv_, in_dtype, gate);
   if ((size_t)B * H != 0 && (ws_bytes < need || !workspace))
     return fail(GDR_ERR_WORKSPACE, "workspace %zu B < required %zu B", ws_bytes, need);
   if (workspace && !aligned16(workspace))
     return fail(GDR_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   if ((size_t)B * H == 0) return ok();
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (bwd_on_tensor_cores(T, dk_, in_dtype, gate)) {
+    if ((size_t)B * H * ((T + 63) / 64) > 0x7fffffffu)
+      return fail(GDR_ERR_INVALID_ARG, "B*H*chunks too large");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout))
+      return fail(GDR_ERR_INVALID_ARG, "q/k/v/dout must be 16-byte aligned");
+    unsigned int *status = nullptr;
+    cudaError_t e = status_word(&status);
+    if (e != cudaSuccess) return from_cuda(e, "gdr_chunk_bwd status word");
+    return from_cuda(gdr::launch_bwd_tc(q, k, v, g, beta, S0, dout, dS_T, dq, dk, dv, dg, dbeta,
+                                        dS0, B, T, H, workspace, status, s),
+                     "gdr_chunk_bwd launch (tensor cores)");
+  }
   return from_cuda(gdr::launch_bwd(q, k, v, in_dtype == GDR_BF16, g, gate == GDR_GATE_PER_CHANNEL,
                                    beta, S0, dout, dS_T, dq, dk, dv, dg, dbeta, dS0, B, T, H,
-                                   dk_, workspace, reinterpret_cast<cudaStream_t>(stream)),
+                                   dk_, workspace, s),
                    "gdr_chunk_bwd launch");
 }
 

@@ -850,7 +850,7 @@ __device__ int scale_channels(uint8_t *kq, uint8_t *kh, float *g0, float *g1, ui
 
 // Each SM sub-partition holds a quarter of the register file and three of
 // the block's twelve warps: the launch bound caps registers at 168.
-template <bool PC, bool ADD, bool PRO>
+template <bool PC, bool ADD, bool PRO, bool STASH>
 __global__ void __launch_bounds__(kThreads, 1)
     gdr_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -1170,6 +1170,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = W(B_TRDY + (c & 1), (c >> 1) & 1) && W(B_VFULL, ph))) break;
         {
           const uint32_t tt = (PC ? a_tp : a_t) + (c & 1) * kTileBytes;
+          if (STASH) {  // backward stash: this chunk's T (map in tmO's slot)
+            tma_store_3d(&tmO, sm + Lay::T + (c & 1) * kTileBytes, 0, 0, bh * n + c);
+            tma_store_commit();
+            tma_store_wait_read0();  // read before the prep group may rewrite the buffer
+          }
           if (!a.zero_v) {  // (v taken as zero: U = 0, the V' MMA starts the accumulator)
 #pragma unroll 1
             for (int kk = 0; kk < 4; ++kk)
@@ -1485,7 +1490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the O epilogue carry sigma).  While sigma * dl (dl: the chunk's decay)
     // stays above the floor only sigma changes; otherwise (fold) S_tmem <-
     // f S_tmem with f = sigma * dl and sigma restarts at 1.
-    auto pass_from_tmem = [&](bool fold, float f) {
+    // (backward stash: xst = row i of the next chunk's X0, xs = sigma, the
+    // scale that takes S_tmem to the true state)
+    auto pass_from_tmem = [&](bool fold, float f, uint4 *xst, float xs) {
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float x[32];
@@ -1494,6 +1501,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
         tmem_st16u(lane_base + TM_SB + 16 * q, u);
+        if (xst) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            xst[4 * q + e] = make_uint4(pack_bf16(xs * x[8 * e], xs * x[8 * e + 1]),
+                                        pack_bf16(xs * x[8 * e + 2], xs * x[8 * e + 3]),
+                                        pack_bf16(xs * x[8 * e + 4], xs * x[8 * e + 5]),
+                                        pack_bf16(xs * x[8 * e + 6], xs * x[8 * e + 7]));
+        }
         if (fold) {  // rare: write back S_tmem * f
 #pragma unroll
           for (int e = 0; e < 32; ++e) x[e] *= f;
@@ -1551,6 +1566,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x[2 * e], x[2 * e + 1]);
           tmem_st16u(lane_base + TM_SB + 16 * q, u);
+          if (STASH) {  // backward stash: row i of chunk 0's X0 (the start state)
+            uint4 *xst = reinterpret_cast<uint4 *>(a.stash_x + (((size_t)bh * n) * DV + i) * DK);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              xst[4 * q + e] = make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+          }
           float y0[16], y1[16];
           const float dl0 = PC ? 1.f : dl;
 #pragma unroll
@@ -1633,12 +1654,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         DBG_ROW(40960, 64, x0);
         DBG_ROW(40960 + 32, 64, x1);
         uint32_t u[16];
+        // (backward stash: row i of V'^T, tokens 0-63)
+        uint4 *vst = STASH ? reinterpret_cast<uint4 *>(a.stash_v + (((size_t)bh * n + c) *
+                                                                      DV + i) * C)
+                           : nullptr;
 #pragma unroll
         for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x0[2 * e], x0[2 * e + 1]);
         tmem_st16u(lane_base + TM_UV, u);
+        if (vst) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) vst[e] = make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+        }
 #pragma unroll
         for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x1[2 * e], x1[2 * e + 1]);
         tmem_st16u(lane_base + TM_UV + 16, u);
+        if (vst) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            vst[4 + e] = make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+        }
         if (!PC) {
           const float4 *e4 = reinterpret_cast<const float4 *>(eglv);
 #pragma unroll
@@ -1680,7 +1714,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const float nxt = sig * dl;
           const bool fold = !(nxt >= kScaleFloor);  // also when dl underflows to 0
-          pass_from_tmem(fold, nxt);
+          pass_from_tmem(fold, nxt,
+                         STASH ? reinterpret_cast<uint4 *>(
+                                     a.stash_x + (((size_t)bh * n + c + 1) * DV + i) * DK)
+                               : nullptr,
+                         sig);
           sig = fold ? 1.f : nxt;
           // next chunk's e^{gc_last - gc} / sigma for its update (every warp
           // writes the same values, from the stage, after its own pass)
@@ -1848,15 +1886,19 @@ bool make_map_gate(CUtensorMap *m, const float *base, int B, int T, int H, int d
   return r == CUDA_SUCCESS;
 }
 
-template <bool PC, bool ADD, bool PRO>
+bool make_map_stash_t(CUtensorMap *m, void *base, long long nchunks) {
+  return tc_map_stash(m, base, nchunks, 64, 64);
+}
+
+template <bool PC, bool ADD, bool PRO, bool STASH = false>
 cudaError_t launch_variant(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                            const CUtensorMap &mv, const CUtensorMap &mg, const CUtensorMap &mo,
                            cudaStream_t stream) {
   constexpr size_t smem = Cfg<PC>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC, ADD, PRO>,
+  cudaError_t e = cudaFuncSetAttribute(gdr_chunk_tc_kernel<PC, ADD, PRO, STASH>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gdr_chunk_tc_kernel<PC, ADD, PRO>
+  gdr_chunk_tc_kernel<PC, ADD, PRO, STASH>
       <<<(unsigned)((size_t)a.B * a.H), kThreads, smem, stream>>>(mq, mk, mv, mg, mo, a);
   return cudaGetLastError();
 }
@@ -1876,6 +1918,26 @@ cudaError_t launch_pc(const ChunkArgs &a, const CUtensorMap &mq, const CUtensorM
 
 }  // namespace
 
+bool tc_map_bf16(CUtensorMap *m, const void *base, int B, int T, int H, int d) {
+  return make_map(m, base, B, T, H, d);
+}
+
+// 3-D map over a per-chunk array [nchunks][rows][cols] bf16 (row-major), box
+// 64 columns x 64 rows of one chunk, 128-byte swizzle (the tile layout of
+// the tensor-core kernels).
+bool tc_map_stash(CUtensorMap *m, const void *base, long long nchunks, int rows, int cols) {
+  auto fn = encode_fn();
+  if (!fn || nchunks <= 0 || nchunks > 0x7fffffffLL || rows < 64 || cols < 64) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)nchunks};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)rows * cols * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool chunk_tc_supports(const ChunkArgs &a) {
   return a.bf16 && a.dk == DK && a.dv == DV && a.T > 0 && (size_t)a.B * a.H <= 0x7fffffffu;
 }
@@ -1891,6 +1953,15 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
       !make_map(&mv, a.v, mb, a.T, a.H, DV) ||
       !make_map_out(&mo, a.write_o ? a.o : const_cast<void *>(a.q), mb, a.T, a.H, DV))
     return cudaErrorInvalidValue;
+  if (a.stash_t) {  // backward stash (no o): the T tiles go out through the output map's slot
+    if (a.per_channel || a.write_o || a.cu_seqlens) return cudaErrorNotSupported;
+    if (!make_map_stash_t(&mo, a.stash_t, (long long)a.B * a.H * ((a.T + C - 1) / C)))
+      return cudaErrorInvalidValue;
+  }
+  if (a.stash_t) {
+    if (!a.stash_x || !a.stash_v || a.additive || a.prologue) return cudaErrorNotSupported;
+    return launch_variant<false, false, false, true>(a, mq, mk, mv, mq, mo, stream);
+  }
   if (a.per_channel) {
     if (!make_map_gate(&mg, a.g, mb, a.T, a.H, DK)) return cudaErrorInvalidValue;
     return launch_pc<true>(a, mq, mk, mv, mg, mo, stream);

@@ -1,6 +1,7 @@
 // Internal declarations shared by the gated delta-rule CUDA sources.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -47,6 +48,12 @@ struct ChunkArgs {
   int prologue;
   int norm_qk;
   const float *gate_scale;  // [H]
+  // Stash for the backward (tensor-core kernel, scalar gates, write_o = 0):
+  // per (b, h) and chunk c, in bf16, row-major: the state at the chunk's
+  // start X0 = S_c [128][128] (value channel, key channel), V'^T [128][64]
+  // (value channel, token) and T = (I + A)^{-1} Diag(beta) [64][64].
+  // Null: nothing is stashed.
+  __nv_bfloat16 *stash_x, *stash_v, *stash_t;
 };
 
 struct StepArgs {
@@ -68,6 +75,11 @@ cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
 // the shape is outside what it handles, so the caller can pick another path.
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 bool chunk_tc_supports(const ChunkArgs &a);
+// Tensor maps of the tensor-core kernels (host): a [B, T, H, d] bf16 tensor
+// in 64 x 64 boxes, and a per-chunk array [nchunks][rows][cols] bf16 in
+// 64 x 64 boxes, both with the 128-byte swizzle.
+bool tc_map_bf16(CUtensorMap *m, const void *base, int B, int T, int H, int d);
+bool tc_map_stash(CUtensorMap *m, const void *base, long long nchunks, int rows, int cols);
 
 // Long sequences with few (b, h): each sequence is cut into P segments that
 // run as separate (b, h) units (two passes of the tensor-core kernel, a
@@ -90,6 +102,17 @@ cudaError_t launch_bwd(const void *q, const void *k, const void *v, int bf16, co
                        const float *dST, float *dq, float *dk, float *dv, float *dg,
                        float *dbeta, float *dS0, int B, int T, int H, int d, void *ws,
                        cudaStream_t stream);
+
+// Backward on the tensor cores (bf16, d_k = d_v = 128, scalar gate): the
+// forward rerun with a per-chunk stash, a reverse pass for the state
+// gradient and a chunk-parallel pass for the token gradients (3 launches).
+bool bwd_tc_supports(int bf16, int per_channel, int d);
+size_t bwd_tc_ws_bytes(int B, int T, int H);
+cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *S0, const float *dout,
+                          const float *dST, float *dq, float *dk, float *dv, float *dg,
+                          float *dbeta, float *dS0, int B, int T, int H, void *ws,
+                          unsigned int *status, cudaStream_t stream);
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ float load_in(const void *p, size_t i, int bf16) {

@@ -142,6 +142,16 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap *m, const void *s
       : "memory");
 }
 
+// 3-D tiled store shared -> global.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *m, const void *src, int c0,
+                                             int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], "
+      "[%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_store_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

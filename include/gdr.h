@@ -324,15 +324,27 @@ gdr_status gdr_dplr_fwd(const void *q, const void *k, const void *v, const void 
  *   dq, dk [B, T, H, dk] fp32;  dv [B, T, H, dv] fp32 (written)
  *   dg     [B, T, H] fp32 (scalar gate) or [B, T, H, dk] (per channel)
  *   dbeta  [B, T, H] fp32;  dS0 [B, H, dv, dk] fp32 or NULL (not written)
- *   workspace  device memory of gdr_chunk_bwd_workspace_bytes() bytes,
- *              16-byte aligned, owned by the caller (overwritten): the
- *              state at every 8th token and an 8-token stash per (b, h)
+ *   workspace  device memory of gdr_chunk_bwd_workspace_bytes() bytes for
+ *              the same shape, dtype and gate, 16-byte aligned, owned by the
+ *              caller (overwritten)
  *
- * Needs dk = dv in {32, 64, 128} (GDR_ERR_UNSUPPORTED otherwise); fp32 or
- * bf16 inputs; arithmetic in fp32 on CUDA cores, one CTA per (b, h).  One
- * launch on `stream`.
+ * Two paths, chosen by shape:
+ * - bf16 inputs, dk = dv = 128, scalar gate, T > 0: the chunked backward on
+ *   the tensor cores (tcgen05), as section 5 has it (chunked and
+ *   parallelised, with recomputation), in three launches: the forward again,
+ *   stashing per chunk its start state, V'^T and T (bf16); a reverse pass
+ *   over the chunks of each (b, h) carrying dL/dS in fp32 (stashing it and
+ *   dV'^T per chunk, and writing dS0); a chunk-parallel pass forming dq,
+ *   dk, dv, dg and dbeta.  Workspace: 104 KB per 64-token chunk and head.
+ * - any other shape (dk = dv in {32, 64, 128}, fp32 or bf16 inputs, scalar
+ *   or per-channel gate, T >= 0): the per-step reverse recurrence above in
+ *   fp32 on CUDA cores, one CTA per (b, h), with the state checkpointed every
+ *   8 tokens (workspace: those states and an 8-token stash per (b, h)); one
+ *   launch.
+ * GDR_ERR_UNSUPPORTED for dk != dv or a head size outside {32, 64, 128}.
  */
-size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv);
+size_t gdr_chunk_bwd_workspace_bytes(int B, int T, int H, int dk, int dv, gdr_dtype in_dtype,
+                                     gdr_gate_kind gate);
 gdr_status gdr_chunk_bwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                          const float *g, gdr_gate_kind gate, const float *beta, const float *S0,
                          const float *dout, const float *dS_T, float *dq, float *dk, float *dv,

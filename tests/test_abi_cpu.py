@@ -214,12 +214,16 @@ def test_prologue_validation_rejects_before_any_launch(L):
 def test_backward_validation_rejects_before_any_launch(L):
     """gdr_chunk_bwd: square heads of 32, 64 or 128; workspace required."""
     p = _fake_ptr()
-    ws = L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128)
-    assert ws == 2 * 2 * (38 + 1 + 8) * 128 * 128 * 4  # every 8th state + an 8-token stash
-    assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 64) == 0
+    # CUDA cores (fp32 inputs, or a per-channel gate): every 8th state + an 8-token stash
+    ws = L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128, 0, 0)
+    assert ws == 2 * 2 * (38 + 1 + 8) * 128 * 128 * 4
+    assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128, 1, 1) == ws
+    # tensor cores (bf16, d = 128, scalar gate): 104 KB of bf16 stash per chunk and head
+    assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128, 1, 0) == 2 * 2 * 5 * 106496
+    assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 64, 1, 0) == 0
 
     def call(**kw):
-        a = dict(q=p, k=p, v=p, dt=1, g=p, gate=0, beta=p, S0=None, do=p, dST=None, dq=p, dk=p,
+        a = dict(q=p, k=p, v=p, dt=0, g=p, gate=0, beta=p, S0=None, do=p, dST=None, dq=p, dk=p,
                  dv=p, dg=p, db=p, dS0=None, B=2, T=300, H=2, dk_=128, dv_=128, ws=p, wsb=ws,
                  st=None)
         a.update(kw)
