@@ -131,6 +131,19 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
       : "memory");
 }
 
+// 16-byte global -> shared copy through the asynchronous copy unit, the
+// commit of this thread's copies, and the wait for them.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 // Bounded wait of every thread, then a CTA-wide agreement (a thread that
 // timed out makes every thread leave together).
 __device__ __forceinline__ bool wait_all_threads(uint64_t *bar, uint32_t parity, bool ok) {
@@ -166,11 +179,14 @@ struct StateArgs {
   unsigned int *status;
 };
 
-// Shared memory (bytes from a 1024-byte aligned base): [K_h0|Q_h0|K_h1|Q_h1],
-// T~, [dO_h0|dO_h1], P, [K-bar_h0|K-bar_h1], gate vectors, barriers.
-constexpr uint32_t R_KQ = 0, R_TT = 4 * kTile, R_DO = 5 * kTile, R_P = 7 * kTile,
-                   R_KB = 8 * kTile, R_VEC = 10 * kTile, R_BAR = R_VEC + 1024,
-                   R_MISC = R_BAR + 64, R_END = R_MISC + 64;
+// Shared memory (bytes from a 1024-byte aligned base): two stages of
+// [K_h0|Q_h0|K_h1|Q_h1] and of T (T~ once scaled) so that the next chunk's
+// loads run under this one's work, [dO_h0|dO_h1] (bf16), P,
+// [K-bar_h0|K-bar_h1], the next chunk's dO in fp32 (asynchronous copies),
+// gate vectors, barriers.
+constexpr uint32_t R_KQ = 0, R_TT = 8 * kTile, R_DO = 10 * kTile, R_P = 12 * kTile,
+                   R_KB = 13 * kTile, R_STG = 15 * kTile, R_VEC = 19 * kTile,  // STG: 32 KB
+                   R_BAR = R_VEC + 1024, R_MISC = R_BAR + 64, R_END = R_MISC + 64;
 constexpr size_t kStateSmem = R_END + 1024;
 // TMEM columns: dS (fp32), its bf16 copy, dV'^T, Zc = dV'^T T~, D1 = [K; Q] K^T
 constexpr uint32_t TR_DS = 0, TR_DSB = 128, TR_DVP = 192, TR_ZC = 256, TR_D1 = 320;
@@ -184,13 +200,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             ~uintptr_t(1023));
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, H = a.H, n = a.n;
-  uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + R_BAR), *bar_mma = bar_ld + 1;
+  uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + R_BAR), *bar_mma = bar_ld + 2;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + R_MISC);
   float *gcv = reinterpret_cast<float *>(sm + R_VEC);  // [64] cumulative log decay
   float *bv = gcv + 64;                                 // [64] e^{gc}
   float *kbv = gcv + 128;                               // [64] e^{gc_last - gc}
   if (t == 0) {
     mbar_init(bar_ld, 1);
+    mbar_init(bar_ld + 1, 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
   }
@@ -216,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tmem_wait_st();
 
-  const uint32_t kq = smem_u32(sm + R_KQ), tt = smem_u32(sm + R_TT), dq = smem_u32(sm + R_DO);
+  const uint32_t dq = smem_u32(sm + R_DO);
   const uint32_t pp = smem_u32(sm + R_P), kb = smem_u32(sm + R_KB);
   constexpr uint32_t ID_D1 = idesc_bf16(128, 64, 0, 0);
   constexpr uint32_t ID_DOP = idesc_bf16(128, 64, 1, 1);   // A = dO^T, B = P (both MN-major)
@@ -224,20 +241,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t ID_ZC = idesc_bf16(128, 64, 0, 1);    // A = dV'^T (TMEM), B = T~
   constexpr uint32_t ID_DOQ = idesc_bf16(128, 128, 1, 1);  // A = dO^T, B = Q~
   constexpr uint32_t ID_ZK = idesc_bf16(128, 128, 0, 1);   // A = -Zc (TMEM), B = K
-  uint32_t ph_ld = 0, ph_mma = 0;
-  bool ok = true;
-#pragma unroll 1
-  for (int ci = n - 1; ci >= 0 && ok; --ci) {
-    const int t0 = ci * C, L = min(C, a.T - t0);
-    // ---- loads: K, Q, T (TMA; rows past T are zero); dO -> bf16; gates
-    if (t == 0) {
-      mbar_arrive_expect_tx(bar_ld, 5 * kTile);
-      tma_load_4d(sm + R_KQ + 0 * kTile, &tmK, bar_ld, 0, h, t0, b);
-      tma_load_4d(sm + R_KQ + 1 * kTile, &tmQ, bar_ld, 0, h, t0, b);
-      tma_load_4d(sm + R_KQ + 2 * kTile, &tmK, bar_ld, 64, h, t0, b);
-      tma_load_4d(sm + R_KQ + 3 * kTile, &tmQ, bar_ld, 64, h, t0, b);
-      tma_load_3d(sm + R_TT, &tmT, bar_ld, 0, 0, bh * n + ci);
+  // Chunk c's K, Q and T into stage st by TMA (rows past T read as zero);
+  // thread 0 only.  ld_n counts the loads each stage has received.
+  int ld_n0 = 0, ld_n1 = 0;
+  auto load_tiles = [&](int c, int st) {
+    uint64_t *bl = bar_ld + st;
+    uint8_t *kqs = sm + R_KQ + st * 4 * kTile;
+    const int c0 = c * C;
+    mbar_arrive_expect_tx(bl, 5 * kTile);
+    tma_load_4d(kqs + 0 * kTile, &tmK, bl, 0, h, c0, b);
+    tma_load_4d(kqs + 1 * kTile, &tmQ, bl, 0, h, c0, b);
+    tma_load_4d(kqs + 2 * kTile, &tmK, bl, 64, h, c0, b);
+    tma_load_4d(kqs + 3 * kTile, &tmQ, bl, 64, h, c0, b);
+    tma_load_3d(sm + R_TT + st * kTile, &tmT, bl, 0, 0, bh * n + c);
+    if (st) ++ld_n1; else ++ld_n0;
+  };
+  // Chunk c's dO rows into the fp32 staging area through the asynchronous
+  // copy unit: this thread's row t / 2, channel half t % 2 (rows past T are
+  // not copied).  Only the thread that copies a row half reads it back.
+  auto load_dout = [&](int c) {
+    const int c0 = c * C, Lc = min(C, a.T - c0), r = t >> 1, hh = t & 1;
+    if (r < Lc) {
+      const float *src = a.dout + (((size_t)b * a.T + c0 + r) * H + h) * D + 64 * hh;
+      uint8_t *dst = sm + R_STG + r * 512 + hh * 256;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) cp_async16(dst + 16 * e, src + 4 * e);
     }
+    cp_async_commit();
+  };
+  uint32_t ph_mma = 0;
+  bool ok = true;
+  if (t == 0) load_tiles(n - 1, 0);
+  load_dout(n - 1);
+#pragma unroll 1
+  for (int it = 0; it < n && ok; ++it) {
+    const int ci = n - 1 - it, st = it & 1;
+    const int t0 = ci * C, L = min(C, a.T - t0);
+    uint8_t *kqp = sm + R_KQ + st * 4 * kTile, *ttp = sm + R_TT + st * kTile;
+    const uint32_t kq = smem_u32(kqp), tt = smem_u32(ttp);
+    // the next chunk's K, Q, T into the other stage: every MMA and every
+    // thread's access of the chunk before this one, which used it, is done
+    if (ci >= 1 && t == 0) load_tiles(ci - 1, st ^ 1);
     if (warp == 0) {
       const size_t tok = ((size_t)b * a.T + t0 + lane) * H + h;
       float x0 = lane < L ? a.g[tok] : 0.f;
@@ -250,23 +294,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       kbv[lane] = __expf(gl - x0);
       kbv[lane + 32] = __expf(gl - x1);
     }
-    {  // dO rows -> bf16 tile (thread: row t / 2, channel half t % 2)
+    {  // dO rows (this thread's own asynchronous copies) -> bf16 tile
       const int r = t >> 1, hh = t & 1;
+      cp_async_wait_all();
       uint8_t *tile = sm + R_DO + hh * kTile;
-      const float4 *src =
-          r < L ? reinterpret_cast<const float4 *>(a.dout + (((size_t)b * a.T + t0 + r) * H + h) *
-                                                                D + 64 * hh)
-                : nullptr;
+      const float4 *src = reinterpret_cast<const float4 *>(sm + R_STG + r * 512 + hh * 256);
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const float4 v0 = src ? src[2 * ch] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 v1 = src ? src[2 * ch + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const int ch = (c8 + r) & 7;  // rotated: the lanes' reads spread over the banks
+        const float4 v0 = r < L ? src[2 * ch] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v1 = r < L ? src[2 * ch + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<uint4 *>(tile + sw128_off(r, 8 * ch)) =
             make_uint4(pack_bf16(v0.x, v0.y), pack_bf16(v0.z, v0.w), pack_bf16(v1.x, v1.y),
                        pack_bf16(v1.z, v1.w));
       }
     }
     __syncthreads();  // gate vectors written
+    if (ci >= 1) load_dout(ci - 1);
     {  // dS1 -> its bf16 copy (TMEM) and the stash; dS <- e^{gl} dS1
       const float bl = bv[63];
       uint4 *dst = reinterpret_cast<uint4 *>(a.stash_ds + (((size_t)bh * n + ci) * D + i) * D);
@@ -287,8 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
     }
-    ok = wait_all_threads(bar_ld, ph_ld, ok);
-    ph_ld ^= 1;
+    ok = wait_all_threads(bar_ld + st, (it >> 1) & 1, ok);
     if (!ok) break;
     // ---- D1 = [K; Q] K^T (rows 64-127: Q K^T for P)
     tc_fence_before();
@@ -306,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     {  // meanwhile: K-bar = K e^{gl - gc} (new tiles); T~ = T Diag(e^{gc}) in place
       const int r = t >> 1, hh = t & 1;
       const float f = kbv[r];
-      const uint8_t *src = sm + R_KQ + 2 * hh * kTile;
+      const uint8_t *src = kqp + 2 * hh * kTile;
       uint8_t *dst = sm + R_KB + hh * kTile;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
@@ -318,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         const int col = 32 * hh + 8 * ch;
-        uint8_t *p = sm + R_TT + sw128_off(r, col);
+        uint8_t *p = ttp + sw128_off(r, col);
         uint4 v = *reinterpret_cast<uint4 *>(p);
         uint32_t *w = &v.x;
 #pragma unroll
@@ -351,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     {
       const int r = t >> 1, hh = t & 1;
-      uint8_t *qt = sm + R_KQ + (2 * hh + 1) * kTile;
+      uint8_t *qt = kqp + (2 * hh + 1) * kTile;
       const float f = bv[r];
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) scale_chunk(qt + sw128_off(r, 8 * ch), f);
@@ -454,7 +497,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
     }
   }
-  if (!ok && t == 0) atomicOr(a.status, kStatusTimeout);
+  cp_async_wait_all();
+  if (!ok && t == 0) {  // a load still in flight lands before the CTA ends
+    atomicOr(a.status, kStatusTimeout);
+    if (ld_n0) mbar_wait_bounded(bar_ld, (uint32_t)(ld_n0 - 1) & 1u, kWaitNs);
+    if (ld_n1) mbar_wait_bounded(bar_ld + 1, (uint32_t)(ld_n1 - 1) & 1u, kWaitNs);
+  }
   if (t == 0) {  // every issued MMA has completed before TMEM is released
     mma_commit(bar_mma);
     mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
@@ -520,6 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *betav = gcv + 192;                             // beta
   float *dbeta1 = gcv + 256;                            // column sums of dT . Y
   float *red = gcv + 320;                               // [4] block reduction
+  float *rbeta = gcv + 448;                             // 1 / beta (0 where beta = 0)
   if (t == 0) {
     mbar_init(bar_ld, 1);
     mbar_init(bar_mma, 1);
@@ -591,24 +640,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     bv[lane + 32] = __expf(x1);
     kbv[lane] = __expf(gl - x0);
     kbv[lane + 32] = __expf(gl - x1);
-    betav[lane] = lane < L ? a.beta[tok] : 0.f;
-    betav[lane + 32] = lane + 32 < L ? a.beta[tok + (size_t)32 * H] : 0.f;
+    const float b0 = lane < L ? a.beta[tok] : 0.f;
+    const float b1 = lane + 32 < L ? a.beta[tok + (size_t)32 * H] : 0.f;
+    betav[lane] = b0;
+    betav[lane + 32] = b1;
+    rbeta[lane] = b0 > 0.f ? 1.f / b0 : 0.f;
+    rbeta[lane + 32] = b1 > 0.f ? 1.f / b1 : 0.f;
   }
-  {  // dO rows -> bf16 tile
-    const int r = t >> 1, hh = t & 1;
-    uint8_t *tile = sm + G_DO + hh * kTile;
-    const float4 *src =
-        r < L ? reinterpret_cast<const float4 *>(a.dout + (((size_t)b * a.T + t0 + r) * H + h) *
-                                                              D + 64 * hh)
-              : nullptr;
+  {  // dO rows -> bf16 tile: warp w takes rows w, w + 4, ...; lane l channels
+     // 4l .. 4l + 3 (each row one coalesced 512-byte read)
+    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint8_t *tile = sm + G_DO + (lane >> 4) * kTile;
+    const int col = (4 * lane) & 63;
+    float4 v[16];
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const float4 v0 = src ? src[2 * ch] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 v1 = src ? src[2 * ch + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<uint4 *>(tile + sw128_off(r, 8 * ch)) =
-          make_uint4(pack_bf16(v0.x, v0.y), pack_bf16(v0.z, v0.w), pack_bf16(v1.x, v1.y),
-                     pack_bf16(v1.z, v1.w));
+    for (int k = 0; k < 16; ++k) {
+      const int r = warp + 4 * k;
+      v[k] = r < L ? reinterpret_cast<const float4 *>(
+                         a.dout + (((size_t)b * a.T + t0 + r) * H + h) * D)[lane]
+                   : z4;
     }
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      *reinterpret_cast<uint2 *>(tile + sw128_off(warp + 4 * k, col)) =
+          make_uint2(pack_bf16(v[k].x, v[k].y), pack_bf16(v[k].z, v[k].w));
   }
   ok = wait_all_threads(bar_ld, 0, ok);
   sync_for_mma();
@@ -650,12 +705,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(lb + TG0, x0);
       tmem_ld32(lb + TG0 + 32, x1);
       float *dst = a.dv + row0 * D + i;
-#pragma unroll 4
+      const size_t rs = (size_t)H * D;
+#pragma unroll
       for (int r = 0; r < 32; ++r)
-        if (r < L) dst[(size_t)r * H * D] = x0[r];
-#pragma unroll 4
+        if (r < L) dst[r * rs] = x0[r];
+#pragma unroll
       for (int r = 0; r < 32; ++r)
-        if (r + 32 < L) dst[(size_t)(r + 32) * H * D] = x1[r];
+        if (r + 32 < L) dst[(r + 32) * rs] = x1[r];
     }
     {
       float x0[32], x1[32];
@@ -686,8 +742,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = 32 * hp + 8 * ch + 2 * e;
             const float2 x = unpack_bf16(w[e]);
             const float b0 = betav[s], b1 = betav[s + 1];
-            y[8 * ch + 2 * e] = b0 > 0.f ? x.x / b0 : (r == s ? 1.f : 0.f);
-            y[8 * ch + 2 * e + 1] = b1 > 0.f ? x.y / b1 : (r == s + 1 ? 1.f : 0.f);
+            y[8 * ch + 2 * e] = b0 > 0.f ? x.x * rbeta[s] : (r == s ? 1.f : 0.f);
+            y[8 * ch + 2 * e + 1] = b1 > 0.f ? x.y * rbeta[s + 1] : (r == s + 1 ? 1.f : 0.f);
           }
         }
         st_row32(sm + G_Y, r, hp, y);
@@ -870,7 +926,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // lanes = key channels j: dq = AccQ, dk = AccT + AccH + AccB; gate
     // partials p[j][r] = (AccT - AccH - AccB) K[r][j] + AccQ Q[r][j] into the
-    // (now dead) V and dW^T tiles, fp32 [128][64]
+    // (now dead) V and dW^T tiles, fp32 [128][64], entry (j, r) at column
+    // r ^ (j % 32) (writes by lanes j and reads by lanes r hit distinct banks)
     const int j = t;
     float *part = reinterpret_cast<float *>(sm + G_V);
     const uint8_t *kt = sm + G_KQ + 2 * (j >> 6) * kTile, *qt = kt + kTile;
@@ -882,14 +939,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(lb + TG1 + 32 * hp, at);
       tmem_ld32(lb + TG7 + 32 * hp, ah);
       tmem_ld32(lb + TG3 + 32 * hp, ab);
-#pragma unroll 4
+#pragma unroll
       for (int e = 0; e < 32; ++e) {
         const int r = 32 * hp + e;
         const float kv = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(
                                              kt + sw128_off(r, j & 63)) << 16);
         const float qv = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(
                                              qt + sw128_off(r, j & 63)) << 16);
-        part[j * 64 + r] = (at[e] - ah[e] - ab[e]) * kv + aq[e] * qv;
+        part[j * 64 + (r ^ (j & 31))] = (at[e] - ah[e] - ab[e]) * kv + aq[e] * qv;
         dbl += ab[e] * kv;
         if (r < L) {
           const size_t o = (row0 + (size_t)r * H) * D + j;
@@ -926,7 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = t;
       float s = 0.f;
 #pragma unroll 8
-      for (int jj = 0; jj < 128; ++jj) s += part[jj * 64 + r];
+      for (int jj = 0; jj < 128; ++jj) s += part[jj * 64 + (r ^ (jj & 31))];
       if (r == 63) s += red[0] + red[1] + red[2] + red[3];
       // reverse inclusive scan over r within two warps (rows 0-31, 32-63)
       float x = s;
