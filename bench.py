@@ -38,7 +38,8 @@ DEFAULT_WORKLOAD = "gdn_b8_t4096_h16_d128"
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = {
     "chunk": ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
-              "gated_delta_rule_93_b200/csrc/gdr_chunk_simt.cu",
+              "gated_delta_rule_93_b200/csrc/gdr_chunk_split.cu",
+              "gated_delta_rule_93_b200/csrc/gdr_tc_util.cuh",
               "gated_delta_rule_93_b200/csrc/gdr_segments.cu",
               "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
     "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu"],

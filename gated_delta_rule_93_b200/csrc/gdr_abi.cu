@@ -202,7 +202,7 @@ gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype 
   else if (gdr::chunk_tc_supports(a))
     e = gdr::launch_chunk_tc(a, s);
   else
-    e = gdr::launch_chunk_simt(a, s);
+    e = gdr::launch_chunk_split(a, s);
   return from_cuda(e, "gdr_chunk_fwd launch");
 }
 

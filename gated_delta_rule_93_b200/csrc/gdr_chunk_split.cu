@@ -1,0 +1,588 @@
+// Chunkwise gated delta-rule forward on the sm_100a tensor cores for the
+// shapes the warp-specialised bf16 kernel does not take: fp32 inputs, and
+// head dims d_k, d_v in {32, 64, 128} other than bf16 with d_k = d_v = 128.
+//
+// Source: "Decoding Hybrid Linear Attention Architectures", section 5
+// (inter-chunk state recursion, intra-chunk output, log-space gates) and the
+// WY/UT form of the delta rule from "Linear Attention Variants (RetNet, GLA,
+// DeltaNet, Based)", DeltaNet section.  In the state's own orientation (S is
+// d_v x d_k, one TMEM lane per value channel i) and for one chunk of C = 64
+// tokens, with gc_r the cumulative log decay from the chunk start and m a
+// per-key-channel reference (gc at row 31 for a per-channel gate, 0 for a
+// scalar gate):
+//
+//   K~ = K e^{gc - m},  Q~ = Q e^{gc - m},  K^ = K e^{m - gc}
+//   D1  = [K~; Q~] K^^T                   (tcgen05, M = 128, N = 64)
+//   A   = strict_tril(beta_r D1_KK Gamma),  P = tril_incl(D1_QK Gamma)
+//         (Gamma_rs = e^{gc_r - gc_s} for a scalar gate, 1 per channel)
+//   [Z | O_a] = S' [K~; Q~]^T,  S' = S Diag(e^{m})     (tcgen05, A = S' in TMEM)
+//   T   = (I + A)^{-1} Diag(beta)         (forward substitution, fp32)
+//   U^T = (V^T - zf Z) T^T                 (zf_r = e^{gc_r} scalar gate, 1 per channel)
+//   O^T = zf O_a + U^T P^T
+//   S   = S Diag(e^{gc_last}) + U^T (K e^{gc_last - gc})
+//
+// Every operand is carried as two bf16 terms, x = hi + lo with
+// |x - hi - lo| <= 2^-18 |x|, and each product as three bf16 MMAs (hi hi,
+// hi lo, lo hi) into one fp32 accumulator, so the contractions keep close to
+// fp32 accuracy (the dropped lo lo term and the split are below 2^-16
+// relative) on the bf16 tensor-core path.  The state stays fp32 in TMEM;
+// T is solved in fp32 on the CUDA cores.
+//
+// A per-channel gate's factors e^{+-(gc - m)} are bounded by 2^100 (the lo
+// terms of the split stay normal numbers); a chunk whose decay within 32
+// tokens exceeds that has those factors zeroed and sets the range bit of the
+// status word, so the call reports GDR_ERR_RANGE instead of a wrong result.
+// The scalar gate's factors are pairwise and never exceed 1.
+//
+// One CTA per (b, h), 128 threads, sequential phases (load and split ->
+// D1, Z, O_a -> A, P, U's right-hand side, decay of S -> T -> U -> O_b and
+// the state update -> output), each MMA group waited on with a bounded
+// mbarrier wait.  d_k = 32 is zero-padded to 64 on chip; d_v < 128 leaves
+// the upper TMEM lanes at zero.  A ragged last chunk is zero-padded
+// (k = q = v = 0, beta = 0, g = 0), which leaves the state untouched; its
+// padded output rows are not stored.
+#include "gdr_internal.cuh"
+#include "gdr_tc_util.cuh"
+
+namespace gdr {
+namespace {
+
+using namespace sm100;
+using namespace tcu;
+
+constexpr int C = 64;
+constexpr int kThreads = 128;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kMaxExp = 100.f * kLn2;  // largest |gc - m| of a scaled factor
+
+// Shared memory (bytes from a 1024-byte aligned base).  bf16 tiles in the
+// 128-byte swizzle, K-major, 64 columns per block:
+//   KQ    [K~; Q~] 128 rows x DK (hi, lo)
+//   KH    K^ 64 rows x DK (hi, lo); after D1: A in fp32 [64][64]
+//   KB    (K e^{gl - gc})^T  DK rows x 64 (hi, lo)
+//   TT, PP  T and P 64 x 64 (hi, lo)
+//   GC    per-channel cumulative log decays [64][DK] fp32
+template <int DK>
+struct Layout {
+  static constexpr uint32_t kKQBlk = 128 * 128, kKHBlk = 64 * 128;
+  static constexpr uint32_t KQ_HI = 0, KQ_LO = KQ_HI + (DK / 64) * kKQBlk;
+  static constexpr uint32_t KH_HI = KQ_LO + (DK / 64) * kKQBlk,
+                            KH_LO = KH_HI + (DK / 64) * kKHBlk;
+  static constexpr uint32_t KB_HI = KH_LO + (DK / 64) * kKHBlk, KB_LO = KB_HI + DK * 128;
+  static constexpr uint32_t TT_HI = KB_LO + DK * 128, TT_LO = TT_HI + 8192;
+  static constexpr uint32_t PP_HI = TT_LO + 8192, PP_LO = PP_HI + 8192;
+  static constexpr uint32_t GC = PP_LO + 8192;
+  static constexpr uint32_t VEC = GC + 64 * DK * 4;  // 768 floats
+  static constexpr uint32_t BAR = VEC + 768 * 4, MISC = BAR + 16, END = MISC + 16;
+  static constexpr size_t bytes = END + 1024;
+  static_assert(2 * (DK / 64) * kKHBlk >= 64 * 64 * 4, "A overlays K^");
+  static_assert(bytes <= 232448, "shared memory budget");
+};
+
+// TMEM columns: S fp32 [DK], S' hi / lo as bf16 pairs [DK/2 each], D1 (then
+// O_b) [64], Z (then U's right-hand side, hi | lo) and O_a [128], U [64].
+template <int DK>
+struct Cols {
+  static constexpr uint32_t S = 0, SH = DK, SL = DK + DK / 2, D1 = 2 * DK, ZO = 2 * DK + 64,
+                            U = 2 * DK + 192;
+  static_assert(U + 64 <= 512, "TMEM columns");
+};
+
+// 8 consecutive input elements (fp32 or bf16) of row `row`, columns c0.. of
+// a [B, T, H, d] tensor; zero past the row's d or the sequence.
+__device__ __forceinline__ void load8(const void *p, int bf16, size_t row_off, int c0, int d,
+                                      bool valid, float (&x)[8]) {
+  if (!valid || c0 >= d) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = 0.f;
+    return;
+  }
+  if (bf16) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(
+        reinterpret_cast<const __nv_bfloat16 *>(p) + row_off + c0);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf16(w[e]);
+      x[2 * e] = f.x;
+      x[2 * e + 1] = f.y;
+    }
+  } else {
+    const float4 *q = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p) +
+                                                       row_off + c0);
+    const float4 a = q[0], b = q[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+}
+
+// hi / lo bf16 of 8 values into the 16-byte chunk at `off` of two tiles.
+__device__ __forceinline__ void put8(uint8_t *hi_tile, uint8_t *lo_tile, uint32_t off,
+                                     const float (&x)[8]) {
+  float h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) split_bf16(x[e], h[e], l[e]);
+  *reinterpret_cast<uint4 *>(hi_tile + off) =
+      make_uint4(pack_bf16(h[0], h[1]), pack_bf16(h[2], h[3]), pack_bf16(h[4], h[5]),
+                 pack_bf16(h[6], h[7]));
+  *reinterpret_cast<uint4 *>(lo_tile + off) =
+      make_uint4(pack_bf16(l[0], l[1]), pack_bf16(l[2], l[3]), pack_bf16(l[4], l[5]),
+                 pack_bf16(l[6], l[7]));
+}
+
+// 64 fp32 values as hi | lo bf16 pairs into 64 TMEM columns at `taddr`
+// (hi in the first 32 columns, lo in the next 32).
+__device__ __forceinline__ void tmem_put_split64(uint32_t taddr, const float (&x)[64]) {
+  uint32_t hu[16], lu[16];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float h0, l0, h1, l1;
+      split_bf16(x[32 * half + 2 * e], h0, l0);
+      split_bf16(x[32 * half + 2 * e + 1], h1, l1);
+      hu[e] = pack_bf16(h0, h1);
+      lu[e] = pack_bf16(l0, l1);
+    }
+    tmem_st16u(taddr + 16 * half, hu);
+    tmem_st16u(taddr + 32 + 16 * half, lu);
+  }
+}
+
+__device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, bool ok) {
+  ok = ok && mbar_wait_bounded(bar, parity, kWaitNs);
+  return __syncthreads_and(ok) != 0;
+}
+
+// Generic shared-memory and TMEM writes of every thread -> the next MMA.
+__device__ __forceinline__ void sync_for_mma() {
+  fence_proxy_async_smem();
+  tmem_wait_st();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+}
+
+template <int DK, bool PC>
+__global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs a) {
+  using LY = Layout<DK>;
+  using TC = Cols<DK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~uintptr_t(1023));
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, H = a.H;
+  const int dk = a.dk, dv = a.dv, bf = a.bf16;
+  const int n = (a.T + C - 1) / C;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + LY::BAR);
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + LY::MISC);
+  float *vec = reinterpret_cast<float *>(sm + LY::VEC);
+  float *gcs = vec;          // [64] scalar gate: cumulative log decay
+  float *zf = vec + 64;      // [64] e^{gc_r} (scalar gate) or 1
+  float *ebar = vec + 128;   // [64] scalar gate: e^{gl - gc_r}
+  float *betav = vec + 192;  // [64]
+  float *mref = vec + 256;   // [128] per channel: m_j
+  float *em = vec + 384;     // [128] per channel: e^{m_j}
+  float *egl = vec + 512;    // [128] e^{gl_j} (scalar gate: every entry e^{gl})
+  float *glv = vec + 640;    // [128] per channel: gl_j
+  float *gcm = reinterpret_cast<float *>(sm + LY::GC);  // [64][DK]
+  if (t == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tslot;
+  const uint32_t lb = tm + ((uint32_t)(warp * 32) << 16);  // this warp's lanes
+  const int i = t;                                         // value channel (TMEM lane)
+
+  // S = S0 (or 0); lanes >= d_v and columns >= d_k stay 0
+#pragma unroll 1
+  for (int q = 0; q < DK / 32; ++q) {
+    float x[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = 32 * q + e;
+      x[e] = (a.S0 && i < dv && j < dk) ? a.S0[((size_t)bh * dv + i) * dk + j] : 0.f;
+    }
+    tmem_st32(lb + TC::S + 32 * q, x);
+  }
+  tmem_wait_st();
+
+  constexpr uint32_t ID_D1 = idesc_bf16(128, 64, 0, 0);
+  constexpr uint32_t ID_ZO = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t ID_64 = idesc_bf16(128, 64, 0, 0);
+  constexpr uint32_t ID_S = idesc_bf16(128, DK, 0, 0);
+  const uint32_t s_kqh = smem_u32(sm + LY::KQ_HI), s_kql = smem_u32(sm + LY::KQ_LO);
+  const uint32_t s_khh = smem_u32(sm + LY::KH_HI), s_khl = smem_u32(sm + LY::KH_LO);
+  const uint32_t s_kbh = smem_u32(sm + LY::KB_HI), s_kbl = smem_u32(sm + LY::KB_LO);
+  const uint32_t s_tth = smem_u32(sm + LY::TT_HI), s_ttl = smem_u32(sm + LY::TT_LO);
+  const uint32_t s_pph = smem_u32(sm + LY::PP_HI), s_ppl = smem_u32(sm + LY::PP_LO);
+  float4 *Af4 = reinterpret_cast<float4 *>(sm + LY::KH_HI);  // A [64][16 float4], swizzled
+
+  uint32_t ph = 0;
+  bool ok = true;
+  auto mma_wait = [&]() {
+    if (t == 0) mma_commit(bar);
+    ok = wait_all(bar, ph, ok);
+    ph ^= 1;
+    tc_fence_after();
+  };
+
+#pragma unroll 1
+  for (int c = 0; c < n && ok; ++c) {
+    const int t0 = c * C, L = min(C, a.T - t0);
+    const size_t tok0 = ((size_t)b * a.T + t0) * H + h;  // token index of row 0
+    // ---- gates
+    if (PC) {
+      if (t < DK) {
+        const int j = t;
+        float acc = 0.f, m = 0.f;
+#pragma unroll 8
+        for (int r = 0; r < C; ++r) {
+          acc += (r < L && j < dk) ? a.g[(tok0 + (size_t)r * H) * dk + j] : 0.f;
+          gcm[r * DK + j] = acc;
+          if (r == 31) m = acc;
+        }
+        mref[j] = m;
+        em[j] = __expf(m);
+        egl[j] = __expf(acc);
+        glv[j] = acc;
+      }
+      if (warp == 3) {
+        betav[lane] = lane < L ? a.beta[tok0 + (size_t)lane * H] : 0.f;
+        betav[lane + 32] = lane + 32 < L ? a.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
+      }
+      if (t < 64) zf[t] = 1.f;
+    } else {
+      if (warp == 0) {
+        float x0 = lane < L ? a.g[tok0 + (size_t)lane * H] : 0.f;
+        float x1 = lane + 32 < L ? a.g[tok0 + (size_t)(lane + 32) * H] : 0.f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+          const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+          if (lane >= off) {
+            x0 += y0;
+            x1 += y1;
+          }
+        }
+        x1 += __shfl_sync(0xffffffffu, x0, 31);
+        const float gl = __shfl_sync(0xffffffffu, x1, 31);
+        gcs[lane] = x0;
+        gcs[lane + 32] = x1;
+        zf[lane] = __expf(x0);
+        zf[lane + 32] = __expf(x1);
+        ebar[lane] = __expf(gl - x0);
+        ebar[lane + 32] = __expf(gl - x1);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) egl[lane + 32 * e] = __expf(gl);
+      }
+      if (warp == 1) {
+        betav[lane] = lane < L ? a.beta[tok0 + (size_t)lane * H] : 0.f;
+        betav[lane + 32] = lane + 32 < L ? a.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
+      }
+    }
+    __syncthreads();
+    // ---- S' = S Diag(e^{m}) as hi / lo bf16 in TMEM
+#pragma unroll 1
+    for (int q = 0; q < DK / 32; ++q) {
+      float x[32];
+      tmem_ld32(lb + TC::S + 32 * q, x);
+      uint32_t hu[16], lu[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float f0 = PC ? em[32 * q + 2 * e] : 1.f, f1 = PC ? em[32 * q + 2 * e + 1] : 1.f;
+        float h0, l0, h1, l1;
+        split_bf16(x[2 * e] * f0, h0, l0);
+        split_bf16(x[2 * e + 1] * f1, h1, l1);
+        hu[e] = pack_bf16(h0, h1);
+        lu[e] = pack_bf16(l0, l1);
+      }
+      tmem_st16u(lb + TC::SH + 16 * q, hu);
+      tmem_st16u(lb + TC::SL + 16 * q, lu);
+    }
+    // ---- K~, Q~, K^, (K e^{gl - gc})^T tiles: row r = t / 2, half t % 2 of the columns
+    {
+      const int r = t >> 1, hf = t & 1;
+      const bool valid = r < L;
+      const size_t rk = (tok0 + (size_t)r * H) * dk;
+      bool range_bad = false;
+#pragma unroll 1
+      for (int g8 = 0; g8 < DK / 16; ++g8) {
+        const int c0 = hf * (DK / 2) + 8 * g8;
+        float kx[8], qx[8];
+        load8(a.k, bf, rk, c0, dk, valid, kx);
+        load8(a.q, bf, rk, c0, dk, valid, qx);
+        float kt[8], qt[8], kh[8], kb[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = c0 + e;
+          if (PC) {
+            const float x = gcm[r * DK + j] - mref[j];
+            const bool inr = fabsf(x) <= kMaxExp;
+            range_bad |= !inr && (kx[e] != 0.f || qx[e] != 0.f);
+            const float up = inr ? __expf(x) : 0.f, dn = inr ? __expf(-x) : 0.f;
+            kt[e] = kx[e] * up;
+            qt[e] = qx[e] * up;
+            kh[e] = kx[e] * dn;
+            kb[e] = kx[e] * __expf(glv[j] - gcm[r * DK + j]);
+          } else {
+            kt[e] = kx[e];
+            qt[e] = qx[e];
+            kh[e] = kx[e];
+            kb[e] = kx[e] * ebar[r];
+          }
+        }
+        const uint32_t blk = (uint32_t)(c0 >> 6), cc = (uint32_t)(c0 & 63);
+        put8(sm + LY::KQ_HI + blk * LY::kKQBlk, sm + LY::KQ_LO + blk * LY::kKQBlk,
+             sw128_off(r, cc), kt);
+        put8(sm + LY::KQ_HI + blk * LY::kKQBlk, sm + LY::KQ_LO + blk * LY::kKQBlk,
+             sw128_off(64 + r, cc), qt);
+        put8(sm + LY::KH_HI + blk * LY::kKHBlk, sm + LY::KH_LO + blk * LY::kKHBlk,
+             sw128_off(r, cc), kh);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {  // transposed: row j, column r
+          float hi, lo;
+          split_bf16(kb[e], hi, lo);
+          const uint32_t off = sw128_off(c0 + e, r);
+          *reinterpret_cast<__nv_bfloat16 *>(sm + LY::KB_HI + off) = __float2bfloat16_rn(hi);
+          *reinterpret_cast<__nv_bfloat16 *>(sm + LY::KB_LO + off) = __float2bfloat16_rn(lo);
+        }
+      }
+      if (PC && range_bad) atomicOr(a.status, kStatusRange);
+    }
+    sync_for_mma();
+    // ---- D1 = [K~; Q~] K^^T ;  [Z | O_a] = S' [K~; Q~]^T
+    if (t == 0) {
+#pragma unroll 1
+      for (int kk = 0; kk < DK / 16; ++kk) {
+        const uint32_t ka = (kk >> 2) * LY::kKQBlk + (kk & 3) * 32;
+        const uint32_t kh = (kk >> 2) * LY::kKHBlk + (kk & 3) * 32;
+        const uint64_t ah = sdesc_sw128(s_kqh + ka, 16, 1024), al = sdesc_sw128(s_kql + ka, 16, 1024);
+        mma_bf16_ss(tm + TC::D1, ah, sdesc_sw128(s_khh + kh, 16, 1024), ID_D1, kk > 0);
+        mma_bf16_ss(tm + TC::D1, ah, sdesc_sw128(s_khl + kh, 16, 1024), ID_D1, 1);
+        mma_bf16_ss(tm + TC::D1, al, sdesc_sw128(s_khh + kh, 16, 1024), ID_D1, 1);
+        mma_ts(tm + TC::ZO, tm + TC::SH + 8 * kk, ah, ID_ZO, kk > 0);
+        mma_ts(tm + TC::ZO, tm + TC::SH + 8 * kk, al, ID_ZO, 1);
+        mma_ts(tm + TC::ZO, tm + TC::SL + 8 * kk, ah, ID_ZO, 1);
+      }
+    }
+    mma_wait();
+    if (!ok) break;
+    // ---- A (fp32, over K^) and P (hi / lo tiles) from D1; U's right-hand
+    //      side V^T - zf Z into TMEM; S <- S Diag(e^{gl})
+    if (t < 64) {
+      const int r = t;
+      const float br = betav[r], gr = gcs[r];
+#pragma unroll 1
+      for (int hp = 0; hp < 2; ++hp) {
+        float x[32];
+        tmem_ld32(lb + TC::D1 + 32 * hp, x);
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          float y[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int s = 32 * hp + 4 * e4 + e;
+            const float gam = PC ? 1.f : __expf(gr - gcs[s]);
+            y[e] = (s < r && r < L) ? br * x[4 * e4 + e] * gam : 0.f;
+          }
+          Af4[r * 16 + ((8 * hp + e4) ^ (r & 15))] = make_float4(y[0], y[1], y[2], y[3]);
+        }
+      }
+    } else {
+      const int r = t - 64;
+      const float gr = gcs[r];
+#pragma unroll 1
+      for (int hp = 0; hp < 2; ++hp) {
+        float x[32], hi[32], lo[32];
+        tmem_ld32(lb + TC::D1 + 32 * hp, x);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int s = 32 * hp + e;
+          const float gam = PC ? 1.f : __expf(gr - gcs[s]);
+          split_bf16((s <= r && r < L) ? x[e] * gam : 0.f, hi[e], lo[e]);
+        }
+        st_row32(sm + LY::PP_HI, r, hp, hi);
+        st_row32(sm + LY::PP_LO, r, hp, lo);
+      }
+    }
+    {
+      float z[64];
+      {
+        float z0[32], z1[32];
+        tmem_ld32(lb + TC::ZO, z0);
+        tmem_ld32(lb + TC::ZO + 32, z1);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          z[e] = z0[e];
+          z[32 + e] = z1[e];
+        }
+      }
+      const size_t vi = tok0 * dv + i;
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        const float vr = (r < L && i < dv) ? load_in(a.v, vi + (size_t)r * H * dv, bf) : 0.f;
+        z[r] = vr - zf[r] * z[r];
+      }
+      tmem_put_split64(lb + TC::ZO, z);
+    }
+#pragma unroll 1
+    for (int q = 0; q < DK / 32; ++q) {
+      float x[32];
+      tmem_ld32(lb + TC::S + 32 * q, x);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] *= egl[32 * q + e];
+      tmem_st32(lb + TC::S + 32 * q, x);
+    }
+    tmem_wait_st();
+    __syncthreads();
+    // ---- T = (I + A)^{-1} Diag(beta): column c by forward substitution
+    if (t < 64) {
+      const int cl = t;
+      float y[64];
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        float acc = (r == cl) ? 1.f : 0.f;
+#pragma unroll
+        for (int s4 = 0; s4 < (r + 3) / 4; ++s4) {
+          const float4 a4 = Af4[r * 16 + (s4 ^ (r & 15))];
+          if (4 * s4 + 0 < r) acc -= a4.x * y[4 * s4 + 0];
+          if (4 * s4 + 1 < r) acc -= a4.y * y[4 * s4 + 1];
+          if (4 * s4 + 2 < r) acc -= a4.z * y[4 * s4 + 2];
+          if (4 * s4 + 3 < r) acc -= a4.w * y[4 * s4 + 3];
+        }
+        y[r] = acc;
+      }
+      const float bc = betav[cl];
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        float hi, lo;
+        split_bf16(y[r] * bc, hi, lo);
+        const uint32_t off = sw128_off(r, cl);
+        *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_HI + off) = __float2bfloat16_rn(hi);
+        *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_LO + off) = __float2bfloat16_rn(lo);
+      }
+    }
+    sync_for_mma();
+    // ---- U^T = R T^T
+    if (t == 0) {
+#pragma unroll 1
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bh_ = sdesc_sw128(s_tth + kk * 32, 16, 1024);
+        mma_ts(tm + TC::U, tm + TC::ZO + 8 * kk, bh_, ID_64, kk > 0);
+        mma_ts(tm + TC::U, tm + TC::ZO + 8 * kk, sdesc_sw128(s_ttl + kk * 32, 16, 1024), ID_64, 1);
+        mma_ts(tm + TC::U, tm + TC::ZO + 32 + 8 * kk, bh_, ID_64, 1);
+      }
+    }
+    mma_wait();
+    if (!ok) break;
+    {
+      float u[64];
+      {
+        float u0[32], u1[32];
+        tmem_ld32(lb + TC::U, u0);
+        tmem_ld32(lb + TC::U + 32, u1);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          u[e] = u0[e];
+          u[32 + e] = u1[e];
+        }
+      }
+      tmem_put_split64(lb + TC::U, u);
+    }
+    sync_for_mma();
+    // ---- O_b = U^T P^T (over D1) ;  S += U^T (K e^{gl - gc})
+    if (t == 0) {
+#pragma unroll 1
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t uh = tm + TC::U + 8 * kk, ul = tm + TC::U + 32 + 8 * kk;
+        const uint64_t ph_ = sdesc_sw128(s_pph + kk * 32, 16, 1024);
+        const uint64_t kb_ = sdesc_sw128(s_kbh + kk * 32, 16, 1024);
+        mma_ts(tm + TC::D1, uh, ph_, ID_64, kk > 0);
+        mma_ts(tm + TC::D1, uh, sdesc_sw128(s_ppl + kk * 32, 16, 1024), ID_64, 1);
+        mma_ts(tm + TC::D1, ul, ph_, ID_64, 1);
+        mma_ts(tm + TC::S, uh, kb_, ID_S, 1);
+        mma_ts(tm + TC::S, uh, sdesc_sw128(s_kbl + kk * 32, 16, 1024), ID_S, 1);
+        mma_ts(tm + TC::S, ul, kb_, ID_S, 1);
+      }
+    }
+    mma_wait();
+    if (!ok) break;
+    // ---- o_r = zf_r O_a + O_b (lane = value channel)
+#pragma unroll 1
+    for (int hp = 0; hp < 2; ++hp) {
+      float oa[32], ob[32];
+      tmem_ld32(lb + TC::ZO + 64 + 32 * hp, oa);
+      tmem_ld32(lb + TC::D1 + 32 * hp, ob);
+      if (i < dv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int r = 32 * hp + e;
+          if (r < L) store_out(a.o, (tok0 + (size_t)r * H) * dv + i, zf[r] * oa[e] + ob[e], bf);
+        }
+      }
+    }
+    __syncthreads();  // the vectors and tiles of this chunk are read
+  }
+  if (ok && a.S_T) {
+#pragma unroll 1
+    for (int q = 0; q < DK / 32; ++q) {
+      float x[32];
+      tmem_ld32(lb + TC::S + 32 * q, x);
+      if (i < dv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = 32 * q + e;
+          if (j < dk) a.S_T[((size_t)bh * dv + i) * dk + j] = x[e];
+        }
+      }
+    }
+  }
+  if (!ok && t == 0) atomicOr(a.status, kStatusTimeout);
+  if (t == 0) {  // every issued MMA has completed before TMEM is released
+    mma_commit(bar);
+    mbar_wait_bounded(bar, ph, kWaitNs);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+template <int DK, bool PC>
+cudaError_t launch_split(const ChunkArgs &a, cudaStream_t stream) {
+  auto kern = gdr_chunk_split_kernel<DK, PC>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Layout<DK>::bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)(a.B * a.H), kThreads, Layout<DK>::bytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_split_supports(const ChunkArgs &a) {
+  const bool dims = (a.dk == 32 || a.dk == 64 || a.dk == 128) &&
+                    (a.dv == 32 || a.dv == 64 || a.dv == 128);
+  return dims && !a.cu_seqlens && !a.additive && !a.prologue && !a.stash_x && !a.stash_v &&
+         !a.stash_t && a.s0_seg == 0 && !a.s0_identity && !a.zero_v && a.write_o &&
+         a.skip_stage_chunk < 0;
+}
+
+cudaError_t launch_chunk_split(const ChunkArgs &a, cudaStream_t stream) {
+  if (!chunk_split_supports(a)) return cudaErrorNotSupported;
+  if (a.B * a.H == 0) return cudaSuccess;
+  if (a.dk == 128)
+    return a.per_channel ? launch_split<128, true>(a, stream) : launch_split<128, false>(a, stream);
+  return a.per_channel ? launch_split<64, true>(a, stream) : launch_split<64, false>(a, stream);
+}
+
+}  // namespace gdr

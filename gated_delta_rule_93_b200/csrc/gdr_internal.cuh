@@ -70,7 +70,12 @@ struct StepArgs {
 
 // Launchers return cudaSuccess or the launch error.
 cudaError_t launch_step(const StepArgs &a, cudaStream_t stream);
-cudaError_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t stream);
+// Split-operand tensor-core forward (fp32 inputs, and head dims the
+// warp-specialised kernel does not take): every operand as two bf16 terms,
+// every product as three MMAs; returns cudaErrorNotSupported outside its
+// shapes.
+cudaError_t launch_chunk_split(const ChunkArgs &a, cudaStream_t stream);
+bool chunk_split_supports(const ChunkArgs &a);
 // Tensor-core (tcgen05) chunked forward; returns cudaErrorNotSupported when
 // the shape is outside what it handles, so the caller can pick another path.
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);

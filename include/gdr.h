@@ -111,16 +111,20 @@ int gdr_chunk_fwd_kernel_launches(int B, int T, int H, int dk, int dv, int C,
  * S0 may alias S_T (each (b, h) reads all of S0 before writing S_T); o must
  * not alias any input.
  *
- * Range of per-channel gates on the tensor-core path (bf16, dk = dv = 128):
- * a chunk's K and Q tiles are scaled per key channel by e^{+-(gc - m)}
- * around the cumulative decay m at the chunk's row 31, so in every channel
- * the decay accumulated over each half chunk (32 tokens) must stay above
- * about -83 (|sum of g| <= 83, e.g. a decay of e^{-2.6} per token held for
- * 32 tokens).  A chunk beyond that has its overflowing tile entries zeroed
- * (the outputs stay finite but are not the recurrence's) and the call
- * records GDR_ERR_RANGE in the device status word (gdr_get_device_status).
- * Scalar gates and the CUDA-core path (fp32 inputs, dk or dv < 128) have no
- * limit.
+ * Two tensor-core kernels serve this call: bf16 with dk = dv = 128 runs the
+ * warp-specialised kernel (bf16 operands); fp32 inputs and every other
+ * (dk, dv) run the split-operand kernel, which carries each operand as two
+ * bf16 terms and each product as three MMAs (close to fp32 accuracy).
+ *
+ * Range of per-channel gates: a chunk's K and Q tiles are scaled per key
+ * channel by e^{+-(gc - m)} around the cumulative decay m at the chunk's
+ * row 31, so in every channel the decay accumulated over each half chunk
+ * (32 tokens) must stay above about -83 (bf16, dk = dv = 128; e.g. a decay
+ * of e^{-2.6} per token held for 32 tokens) or -69 (split-operand kernel,
+ * whose low terms must stay normal numbers).  A chunk beyond that has its
+ * overflowing tile entries zeroed (the outputs stay finite but are not the
+ * recurrence's) and the call records GDR_ERR_RANGE in the device status
+ * word (gdr_get_device_status).  Scalar gates have no limit.
  */
 gdr_status gdr_chunk_fwd(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                          const float *g, gdr_gate_kind gate, const float *beta,

@@ -143,7 +143,9 @@ def test_split_and_resume_on_gpu(cuda_device):
 
 
 def test_linearity_in_values(cuda_device):
-    """o(S0, V1 + V2) = o(S0, V1) + o(0, V2) for fixed q, k, gates (fp32)."""
+    """o(S0, V1 + V2) = o(S0, V1) + o(0, V2) for fixed q, k, gates (fp32).
+    Three runs of the split-operand path, each within a few 2^-18 per product
+    of exact (two bf16 terms per operand, three MMAs per product): bar 5e-5."""
     a = make_chunk_inputs(1, 130, 2, 64, 64, torch.float32, "scalar", True, seed=8)
     b = make_chunk_inputs(1, 130, 2, 64, 64, torch.float32, "scalar", True, seed=9)
     d = {k: v.to(cuda_device) for k, v in a.items()}
@@ -152,8 +154,8 @@ def test_linearity_in_values(cuda_device):
     o2, s2 = binding.chunk_fwd(d["q"], d["k"], v2, d["g"], d["beta"], None)
     o12, s12 = binding.chunk_fwd(d["q"], d["k"], d["v"] + v2, d["g"], d["beta"], d["S0"])
     torch.cuda.synchronize()
-    assert ((o1 + o2 - o12).abs().max() / o12.abs().max()).item() < 1e-5
-    assert ((s1 + s2 - s12).abs().max() / s12.abs().max()).item() < 1e-5
+    assert ((o1 + o2 - o12).abs().max() / o12.abs().max()).item() < 5e-5
+    assert ((s1 + s2 - s12).abs().max() / s12.abs().max()).item() < 5e-5
 
 
 def test_misaligned_pointer_is_rejected(cuda_device):
@@ -304,15 +306,26 @@ def test_per_channel_rapid_forgetting_reports_range(cuda_device):
     assert binding.device_status() == binding.GDR_OK
 
 
-@pytest.mark.parametrize("d,dtype", [(64, torch.bfloat16), (128, torch.float32)])
-def test_per_channel_rapid_forgetting_cuda_core_path(cuda_device, d, dtype):
-    """The CUDA-core path (d < 128 or fp32 inputs) forms exact pairwise decays
-    and takes any finite g <= 0: g = -30 per token in one channel matches
-    the oracle."""
+@pytest.mark.parametrize("d,dtype", [(64, torch.bfloat16), (128, torch.float32), (32, torch.float32)])
+def test_per_channel_strong_decay_split_path(cuda_device, d, dtype):
+    """The split-operand path (d < 128 or fp32 inputs): one key channel at
+    g = -2 per token (-62 over half a chunk, inside its 2^100 factor range)
+    matches the oracle at the dtype's bar, with a clean status."""
     inp = _one_channel_decay(make_chunk_inputs(1, 200, 2, d, d, dtype, "channel", True,
-                                               seed=64), -30.0)
+                                               seed=64), -2.0)
     o, S_T = gpu_chunk(inp, cuda_device)
     assert binding.device_status() == binding.GDR_OK
     ro, rS = oracle_chunk(inp)
     assert_close(o, ro, TOL[dtype], "o")
     assert_close(S_T, rS, TOL[dtype], "S_T")
+
+
+@pytest.mark.parametrize("d,dtype", [(64, torch.bfloat16), (128, torch.float32)])
+def test_per_channel_rapid_forgetting_split_path_reports_range(cuda_device, d, dtype):
+    """g = -30 per token in one channel is beyond the split-operand path's
+    factor range too: GDR_ERR_RANGE in the status word, finite outputs."""
+    inp = _one_channel_decay(make_chunk_inputs(1, 200, 2, d, d, dtype, "channel", True,
+                                               seed=65), -30.0)
+    o, S_T = gpu_chunk(inp, cuda_device)
+    assert binding.device_status() == binding.GDR_ERR_RANGE
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S_T).all()
