@@ -46,7 +46,8 @@ KERNEL_SOURCES = {
     "bwd": ["gated_delta_rule_93_b200/csrc/gdr_bwd.cu",
             "gated_delta_rule_93_b200/csrc/gdr_bwd_tc.cu",
             "gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu"],
-    "dplr": ["gated_delta_rule_93_b200/csrc/gdr_dplr.cu"],
+    "dplr": ["gated_delta_rule_93_b200/csrc/gdr_chunk_split.cu",
+             "gated_delta_rule_93_b200/csrc/gdr_tc_util.cuh"],
 }
 
 
@@ -77,8 +78,10 @@ def algorithmic_flops(w, C=64):
         return w.B * w.H * 7.0 * w.dk * w.dv
     if w.backward:  # one recomputed forward step (5 d^2) and its reverse (16 d^2)
         return w.B * w.T * w.H * 21.0 * w.dk * w.dv
-    if w.mixer == "dplr":  # S.a and S.(alpha q) (4 d^2), S alpha + x b + v k (5 d^2)
-        return w.B * w.T * w.H * 9.0 * w.dk * w.dv
+    if w.mixer == "dplr":  # chunked: two state reads and two state updates (8 d_k d_v),
+        # four masked intra-chunk products, three masked products with values
+        per = 8 * w.dk * w.dv + C * (4 * w.dk + 3 * w.dv) + C * C / 3.0
+        return w.B * w.T * w.H * per
     if w.mixer == "gla":  # no correction: state update, S q, masked Q K^T and P V
         return w.B * w.T * w.H * (4 * w.dk * w.dv + C * (w.dk + w.dv))
     per = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0
@@ -260,7 +263,7 @@ def make_step(w, dev, rank, nsteps):
             binding.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["dout"], d["S0"],
                               None, want_dS0=False, workspace=bws, out=grads)
 
-    if w.mixer == "dplr":  # recurrent DPLR forward on CUDA cores: one launch
+    if w.mixer == "dplr":  # chunked DPLR forward on the tensor cores: one launch
         launches = 1
 
         def step():
@@ -339,7 +342,7 @@ def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk):
     avg_launch_ms = sum(per_launch_ms) / len(per_launch_ms)
     achieved = abytes / (avg_launch_ms / 1e3) / 1e9
     roof_ms = max(abytes / (hbm_peak * 1e9), aflops / (tc_peak * 1e12)) * 1e3
-    alu = (w.backward and not backward_on_tensor_cores(w)) or w.mixer == "dplr"
+    alu = w.backward and not backward_on_tensor_cores(w)
     alu_peak = None
     if alu:  # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 flop x SM clock
         alu_peak = 148 * 128 * 2 * ((clk or {}).get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
@@ -348,18 +351,20 @@ def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk):
         roof = {"bound": "alu", "achieved": aflops / (avg_launch_ms / 1e3) / 1e12,
                 "peak": alu_peak, "unit": "TFLOP/s",
                 "frac": aflops / (avg_launch_ms / 1e3) / 1e12 / alu_peak,
-                "traffic": recorded_traffic(w.name, "dplr" if w.mixer == "dplr" else "bwd"),
+                "traffic": recorded_traffic(w.name, "bwd"),
                 "peak_source": "CUDA-core fp32 FMA, 148 SMs x 128 lanes x 2 flop x max SM "
                                "clock", "algorithmic_flops_per_launch": aflops,
-                "kernel": "gdr_dplr_fwd" if w.mixer == "dplr" else "gdr_chunk_bwd"}
+                "kernel": "gdr_chunk_bwd"}
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak,
-                "traffic": recorded_traffic(w.name, "bwd" if w.backward else w.kind),
+                "traffic": recorded_traffic(w.name, "bwd" if w.backward else
+                                            "dplr" if w.mixer == "dplr" else w.kind),
                 "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
                 "kernel": ("gdr_chunk_bwd (tensor cores, 3 launches)" if w.backward else
                            "gdr_chunk_fwd_prologue" if w.prologue else
-                           "gdr_chunk_fwd_gla" if w.mixer == "gla" else "gdr_chunk_fwd")
+                           "gdr_chunk_fwd_gla" if w.mixer == "gla" else
+                           "gdr_dplr_fwd" if w.mixer == "dplr" else "gdr_chunk_fwd")
                 if w.kind == "chunk" else "gdr_step"}
     return {"value": world * tokens_step * steps / (total_ms / 1e3), "ms_per_step": ms_step,
             "tflops": aflops * world * steps / (total_ms / 1e3) / 1e12,

@@ -374,17 +374,29 @@ gdr_status gdr_dplr_fwd(const void *q, const void *k, const void *v, const void 
     return fail(GDR_ERR_INVALID_ARG, "in_dtype must be GDR_F32 or GDR_BF16");
   if (gate != GDR_GATE_SCALAR && gate != GDR_GATE_PER_CHANNEL)
     return fail(GDR_ERR_INVALID_ARG, "unknown gate kind");
-  if (dk != dv || (dk != 32 && dk != 64 && dk != 128))
-    return fail(GDR_ERR_UNSUPPORTED, "DPLR needs dk = dv in {32, 64, 128} (got %d, %d)", dk, dv);
+  if (!head_dim_ok(dk) || !head_dim_ok(dv))
+    return fail(GDR_ERR_UNSUPPORTED, "DPLR head dims dk=%d dv=%d (need 32, 64 or 128)", dk, dv);
   if ((size_t)B * (size_t)H * (size_t)T > (size_t)1 << 40)
     return fail(GDR_ERR_INVALID_ARG, "problem too large");
   if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "B*H too large");
-  if ((size_t)B * H * T != 0 && (!q || !k || !v || !a || !b || !g || !o))
-    return fail(GDR_ERR_INVALID_ARG, "null q/k/v/a/b/g/o");
+  if ((size_t)B * H * T != 0) {
+    if (!q || !k || !v || !a || !b || !g || !o)
+      return fail(GDR_ERR_INVALID_ARG, "null q/k/v/a/b/g/o");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned16(b) ||
+        !aligned16(g) || !aligned16(o))
+      return fail(GDR_ERR_INVALID_ARG, "q/k/v/a/b/g/o must be 16-byte aligned");
+  }
+  if ((S0 && !aligned16(S0)) || (S_T && !aligned16(S_T)))
+    return fail(GDR_ERR_INVALID_ARG, "S0/S_T must be 16-byte aligned");
   if ((size_t)B * H == 0) return ok();
-  return from_cuda(gdr::launch_dplr(q, k, v, a, b, in_dtype == GDR_BF16, g,
-                                    gate == GDR_GATE_PER_CHANNEL, S0, o, S_T, B, T, H, dk,
-                                    reinterpret_cast<cudaStream_t>(stream)),
+  gdr::DplrChunkArgs p;
+  p.q = q; p.k = k; p.v = v; p.a = a; p.b = b; p.g = g; p.S0 = S0; p.o = o; p.S_T = S_T;
+  p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv;
+  p.bf16 = in_dtype == GDR_BF16;
+  p.per_channel = gate == GDR_GATE_PER_CHANNEL;
+  cudaError_t e = status_word(&p.status);
+  if (e != cudaSuccess) return from_cuda(e, "gdr_dplr_fwd status word");
+  return from_cuda(gdr::launch_dplr_chunk(p, reinterpret_cast<cudaStream_t>(stream)),
                    "gdr_dplr_fwd launch");
 }
 

@@ -34,6 +34,9 @@
 // status word, so the call reports GDR_ERR_RANGE instead of a wrong result.
 // The scalar gate's factors are pairwise and never exceed 1.
 //
+// The same file holds the chunked DPLR transition (below), built the same
+// way.
+//
 // One CTA per (b, h), 128 threads, sequential phases (load and split ->
 // D1, Z, O_a -> A, P, U's right-hand side, decay of S -> T -> U -> O_b and
 // the state update -> output), each MMA group waited on with a bounded
@@ -567,6 +570,506 @@ cudaError_t launch_split(const ChunkArgs &a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+
+// ====================================================================== DPLR
+// S_t = S_{t-1} (Diag(alpha_t) + a_t b_t^T) + v_t k_t^T,  o_t = S_t q_t
+// ("Decoding Hybrid Linear Attention Architectures", section 3 item 5),
+// chunked as that page's section 5 chunks the delta rule.  With e_r the
+// decay from the chunk start (e_{-1} = 1), the low-rank reads x_r = S_{r-1}
+// a_r of one chunk solve a unit lower-triangular system,
+//   X^T = (S_0 A^^T + V^T Lk^T) T^T,  T = (I - Lb)^{-1},
+//   Lb = strict_tril(A^ B^^T),  Lk = strict_tril(A^ K^^T),
+//   a^_r = a_r e_{r-1},  b^_s = b_s / e_s,  k^_s = k_s / e_s,
+// and then, with q~_r = q_r e_r,
+//   O^T = S_0 Q~^T + X^T tril_incl(Q~ B^^T)^T + V^T tril_incl(Q~ K^^T)^T
+//   S   = S_0 Diag(e_L) + X^T (B e_L / e) + V^T (K e_L / e).
+// The four intra-chunk products come from one MMA group,
+// [A^; Q~] [B^; K^]^T (M = 128, N = 128), and S_0 [A^; Q~]^T gives both
+// state reads; the decay factors follow the delta-rule kernel above (per
+// channel around the row-31 reference m, with the same range bound; a
+// scalar gate's pairwise factors on the products).  Operands are split into
+// two bf16 terms and products into three MMAs as above.
+template <int DK>
+struct DLayout {
+  static constexpr uint32_t kBlk = 128 * 128;  // 128 rows x 64 bf16
+  static constexpr uint32_t AQ_HI = 0, AQ_LO = AQ_HI + (DK / 64) * kBlk;
+  static constexpr uint32_t BK_HI = AQ_LO + (DK / 64) * kBlk, BK_LO = BK_HI + (DK / 64) * kBlk;
+  // after D1: Lb (fp32) and the Lk, P_b, P_k tiles over [A^; Q~] when it is
+  // large enough (DK = 128), else in their own region; the transposed
+  // B-bar, K-bar tiles over [B^; K^]
+  static constexpr uint32_t POST = DK == 128 ? AQ_HI : BK_LO + (DK / 64) * kBlk;
+  static constexpr uint32_t LB = POST, LK_HI = POST + 16384, LK_LO = LK_HI + 8192,
+                            PB_HI = LK_LO + 8192, PB_LO = PB_HI + 8192, PK_HI = PB_LO + 8192,
+                            PK_LO = PK_HI + 8192;
+  static constexpr uint32_t BB_HI = BK_HI, BB_LO = BB_HI + DK * 128, KB_HI = BB_LO + DK * 128,
+                            KB_LO = KB_HI + DK * 128;
+  static constexpr uint32_t TT_HI = DK == 128 ? BK_LO + (DK / 64) * kBlk : PK_LO + 8192,
+                            TT_LO = TT_HI + 8192;
+  static constexpr uint32_t GC = TT_LO + 8192;
+  static constexpr uint32_t VEC = GC + 64 * DK * 4;  // 768 floats
+  static constexpr uint32_t BAR = VEC + 768 * 4, MISC = BAR + 16, END = MISC + 16;
+  static constexpr size_t bytes = END + 1024;
+  static_assert(PK_LO + 8192 <= (DK == 128 ? BK_HI : TT_HI), "post-D1 tiles fit");
+  static_assert(KB_LO + DK * 128 <= BK_HI + 2 * (DK / 64) * kBlk, "B-bar, K-bar fit");
+  static_assert(bytes <= 232448, "shared memory budget");
+};
+
+template <int DK, bool PC>
+__global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkArgs p) {
+  using LY = DLayout<DK>;
+  // TMEM: S [DK], S' hi / lo [DK/2 each], D1 [128] (then W / X in its first
+  // 64 columns and V^T hi | lo in the last 64), ZO [128] (Z_a, then U's
+  // right-hand side, then O_b, in the first 64; O_a in the last 64)
+  constexpr uint32_t TS = 0, TSH = DK, TSL = DK + DK / 2, TD1 = 2 * DK, TZO = 2 * DK + 128;
+  static_assert(TZO + 128 <= 512, "TMEM columns");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~uintptr_t(1023));
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H, H = p.H;
+  const int dk = p.dk, dv = p.dv, bf = p.bf16;
+  const int n = (p.T + C - 1) / C;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + LY::BAR);
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + LY::MISC);
+  float *vec = reinterpret_cast<float *>(sm + LY::VEC);
+  float *gcs = vec;         // [64] scalar gate: cumulative log decay
+  float *zfo = vec + 64;    // [64] e^{gc_r} (scalar gate) or 1
+  float *ebar = vec + 128;  // [64] scalar gate: e^{gl - gc_r}
+  float *zfa = vec + 192;   // [64] e^{gc_{r-1}} (scalar gate) or 1
+  float *mref = vec + 256, *em = vec + 384, *egl = vec + 512, *glv = vec + 640;  // [128] each
+  float *gcm = reinterpret_cast<float *>(sm + LY::GC);  // [64][DK]
+  if (t == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *tslot;
+  const uint32_t lb = tm + ((uint32_t)(warp * 32) << 16);
+  const int i = t;
+
+#pragma unroll 1
+  for (int q = 0; q < DK / 32; ++q) {
+    float x[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int j = 32 * q + e;
+      x[e] = (p.S0 && i < dv && j < dk) ? p.S0[((size_t)bh * dv + i) * dk + j] : 0.f;
+    }
+    tmem_st32(lb + TS + 32 * q, x);
+  }
+  tmem_wait_st();
+
+  constexpr uint32_t ID_128 = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t ID_64 = idesc_bf16(128, 64, 0, 0);
+  constexpr uint32_t ID_S = idesc_bf16(128, DK, 0, 0);
+  const uint32_t s_aqh = smem_u32(sm + LY::AQ_HI), s_aql = smem_u32(sm + LY::AQ_LO);
+  const uint32_t s_bkh = smem_u32(sm + LY::BK_HI), s_bkl = smem_u32(sm + LY::BK_LO);
+  const uint32_t s_lkh = smem_u32(sm + LY::LK_HI), s_lkl = smem_u32(sm + LY::LK_LO);
+  const uint32_t s_pbh = smem_u32(sm + LY::PB_HI), s_pbl = smem_u32(sm + LY::PB_LO);
+  const uint32_t s_pkh = smem_u32(sm + LY::PK_HI), s_pkl = smem_u32(sm + LY::PK_LO);
+  const uint32_t s_bbh = smem_u32(sm + LY::BB_HI), s_bbl = smem_u32(sm + LY::BB_LO);
+  const uint32_t s_kbh = smem_u32(sm + LY::KB_HI), s_kbl = smem_u32(sm + LY::KB_LO);
+  const uint32_t s_tth = smem_u32(sm + LY::TT_HI), s_ttl = smem_u32(sm + LY::TT_LO);
+  float4 *Lb4 = reinterpret_cast<float4 *>(sm + LY::LB);  // [64][16 float4], swizzled
+
+  uint32_t ph = 0;
+  bool ok = true;
+  auto mma_wait = [&]() {
+    if (t == 0) mma_commit(bar);
+    ok = wait_all(bar, ph, ok);
+    ph ^= 1;
+    tc_fence_after();
+  };
+
+#pragma unroll 1
+  for (int c = 0; c < n && ok; ++c) {
+    const int t0 = c * C, L = min(C, p.T - t0);
+    const size_t tok0 = ((size_t)b * p.T + t0) * H + h;
+    // ---- gates
+    if (PC) {
+      if (t < DK) {
+        const int j = t;
+        float acc = 0.f, m = 0.f;
+#pragma unroll 8
+        for (int r = 0; r < C; ++r) {
+          acc += (r < L && j < dk) ? p.g[(tok0 + (size_t)r * H) * dk + j] : 0.f;
+          gcm[r * DK + j] = acc;
+          if (r == 31) m = acc;
+        }
+        mref[j] = m;
+        em[j] = __expf(m);
+        egl[j] = __expf(acc);
+        glv[j] = acc;
+      }
+      if (t < 64) {
+        zfo[t] = 1.f;
+        zfa[t] = 1.f;
+      }
+    } else if (warp == 0) {
+      float x0 = lane < L ? p.g[tok0 + (size_t)lane * H] : 0.f;
+      float x1 = lane + 32 < L ? p.g[tok0 + (size_t)(lane + 32) * H] : 0.f;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+        const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+        if (lane >= off) {
+          x0 += y0;
+          x1 += y1;
+        }
+      }
+      const float c31 = __shfl_sync(0xffffffffu, x0, 31);  // every lane takes part
+      x1 += c31;
+      const float gl = __shfl_sync(0xffffffffu, x1, 31);
+      const float p0 = __shfl_up_sync(0xffffffffu, x0, 1), p1 = __shfl_up_sync(0xffffffffu, x1, 1);
+      const float x0m = lane == 0 ? 0.f : p0;  // gc_{r-1}, r = lane
+      const float x1m = lane == 0 ? c31 : p1;  // r = lane + 32
+      gcs[lane] = x0;
+      gcs[lane + 32] = x1;
+      zfo[lane] = __expf(x0);
+      zfo[lane + 32] = __expf(x1);
+      zfa[lane] = __expf(x0m);
+      zfa[lane + 32] = __expf(x1m);
+      ebar[lane] = __expf(gl - x0);
+      ebar[lane + 32] = __expf(gl - x1);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) egl[lane + 32 * e] = __expf(gl);
+    }
+    __syncthreads();
+    // ---- S' = S Diag(e^{m}) as hi / lo bf16 in TMEM
+#pragma unroll 1
+    for (int q = 0; q < DK / 32; ++q) {
+      float x[32];
+      tmem_ld32(lb + TS + 32 * q, x);
+      uint32_t hu[16], lu[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float f0 = PC ? em[32 * q + 2 * e] : 1.f, f1 = PC ? em[32 * q + 2 * e + 1] : 1.f;
+        float h0, l0, h1, l1;
+        split_bf16(x[2 * e] * f0, h0, l0);
+        split_bf16(x[2 * e + 1] * f1, h1, l1);
+        hu[e] = pack_bf16(h0, h1);
+        lu[e] = pack_bf16(l0, l1);
+      }
+      tmem_st16u(lb + TSH + 16 * q, hu);
+      tmem_st16u(lb + TSL + 16 * q, lu);
+    }
+    // ---- [A^; Q~] and [B^; K^] tiles: row r = t / 2, half t % 2 of the columns
+    {
+      const int r = t >> 1, hf = t & 1;
+      const bool valid = r < L;
+      const size_t rk = (tok0 + (size_t)r * H) * dk;
+      bool range_bad = false;
+#pragma unroll 1
+      for (int g8 = 0; g8 < DK / 16; ++g8) {
+        const int c0 = hf * (DK / 2) + 8 * g8;
+        float ax[8], qx[8], bx[8], kx[8];
+        load8(p.a, bf, rk, c0, dk, valid, ax);
+        load8(p.q, bf, rk, c0, dk, valid, qx);
+        load8(p.b, bf, rk, c0, dk, valid, bx);
+        load8(p.k, bf, rk, c0, dk, valid, kx);
+        if (PC) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int j = c0 + e;
+            const float m = mref[j], gr = gcm[r * DK + j];
+            const float xa = (r > 0 ? gcm[(r - 1) * DK + j] : 0.f) - m, xq = gr - m;
+            const bool ia = fabsf(xa) <= kMaxExp, iq = fabsf(xq) <= kMaxExp;
+            range_bad |= (!ia && ax[e] != 0.f) || (!iq && (qx[e] != 0.f || bx[e] != 0.f ||
+                                                            kx[e] != 0.f));
+            const float fa = ia ? __expf(xa) : 0.f, fq = iq ? __expf(xq) : 0.f,
+                        fb = iq ? __expf(-xq) : 0.f;
+            ax[e] *= fa;
+            qx[e] *= fq;
+            bx[e] *= fb;
+            kx[e] *= fb;
+          }
+        }
+        const uint32_t blk = (uint32_t)(c0 >> 6) * LY::kBlk, cc = (uint32_t)(c0 & 63);
+        put8(sm + LY::AQ_HI + blk, sm + LY::AQ_LO + blk, sw128_off(r, cc), ax);
+        put8(sm + LY::AQ_HI + blk, sm + LY::AQ_LO + blk, sw128_off(64 + r, cc), qx);
+        put8(sm + LY::BK_HI + blk, sm + LY::BK_LO + blk, sw128_off(r, cc), bx);
+        put8(sm + LY::BK_HI + blk, sm + LY::BK_LO + blk, sw128_off(64 + r, cc), kx);
+      }
+      if (PC && range_bad) atomicOr(p.status, kStatusRange);
+    }
+    sync_for_mma();
+    // ---- D1 = [A^; Q~] [B^; K^]^T ;  [Z_a | O_a] = S' [A^; Q~]^T
+    if (t == 0) {
+#pragma unroll 1
+      for (int kk = 0; kk < DK / 16; ++kk) {
+        const uint32_t ko = (kk >> 2) * LY::kBlk + (kk & 3) * 32;
+        const uint64_t ah = sdesc_sw128(s_aqh + ko, 16, 1024), al = sdesc_sw128(s_aql + ko, 16, 1024);
+        const uint64_t bh_ = sdesc_sw128(s_bkh + ko, 16, 1024);
+        mma_bf16_ss(tm + TD1, ah, bh_, ID_128, kk > 0);
+        mma_bf16_ss(tm + TD1, ah, sdesc_sw128(s_bkl + ko, 16, 1024), ID_128, 1);
+        mma_bf16_ss(tm + TD1, al, bh_, ID_128, 1);
+        mma_ts(tm + TZO, tm + TSH + 8 * kk, ah, ID_128, kk > 0);
+        mma_ts(tm + TZO, tm + TSH + 8 * kk, al, ID_128, 1);
+        mma_ts(tm + TZO, tm + TSL + 8 * kk, ah, ID_128, 1);
+      }
+    }
+    mma_wait();
+    if (!ok) break;
+    // ---- from D1: Lb (fp32), Lk, P_b, P_k (hi / lo tiles)
+    if (t < 64) {
+      const int r = t;
+      const float gr = r > 0 ? gcs[r - 1] : 0.f;
+#pragma unroll 1
+      for (int hp = 0; hp < 4; ++hp) {  // D1 columns 32 hp .. 32 hp + 31
+        float x[32];
+        tmem_ld32(lb + TD1 + 32 * hp, x);
+        float hi[32], lo[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int s = 32 * (hp & 1) + e;
+          const float gam = PC ? 1.f : __expf(gr - gcs[s]);
+          x[e] = (s < r && r < L) ? x[e] * gam : 0.f;
+          split_bf16(x[e], hi[e], lo[e]);
+        }
+        if (hp < 2) {
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4)
+            Lb4[r * 16 + ((8 * hp + e4) ^ (r & 15))] =
+                make_float4(x[4 * e4], x[4 * e4 + 1], x[4 * e4 + 2], x[4 * e4 + 3]);
+        } else {
+          st_row32(sm + LY::LK_HI, r, hp & 1, hi);
+          st_row32(sm + LY::LK_LO, r, hp & 1, lo);
+        }
+      }
+    } else {
+      const int r = t - 64;
+      const float gr = gcs[r];
+#pragma unroll 1
+      for (int hp = 0; hp < 4; ++hp) {
+        float x[32], hi[32], lo[32];
+        tmem_ld32(lb + TD1 + 32 * hp, x);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int s = 32 * (hp & 1) + e;
+          const float gam = PC ? 1.f : __expf(gr - gcs[s]);
+          split_bf16((s <= r && r < L) ? x[e] * gam : 0.f, hi[e], lo[e]);
+        }
+        st_row32(sm + (hp < 2 ? LY::PB_HI : LY::PK_HI), r, hp & 1, hi);
+        st_row32(sm + (hp < 2 ? LY::PB_LO : LY::PK_LO), r, hp & 1, lo);
+      }
+    }
+    {  // V^T (lane = value channel) as hi | lo into D1 columns 64-127
+      float vt[64];
+      const size_t vi = tok0 * dv + i;
+#pragma unroll
+      for (int r = 0; r < C; ++r)
+        vt[r] = (r < L && i < dv) ? load_in(p.v, vi + (size_t)r * H * dv, bf) : 0.f;
+      tmem_put_split64(lb + TD1 + 64, vt);
+    }
+    {  // (B e^{gl - gc})^T and (K e^{gl - gc})^T over [B^; K^] (dead after D1)
+      const int r = t >> 1, hf = t & 1;
+      const bool valid = r < L;
+      const size_t rk = (tok0 + (size_t)r * H) * dk;
+#pragma unroll 1
+      for (int g8 = 0; g8 < DK / 16; ++g8) {
+        const int c0 = hf * (DK / 2) + 8 * g8;
+        float bx[8], kx[8];
+        load8(p.b, bf, rk, c0, dk, valid, bx);
+        load8(p.k, bf, rk, c0, dk, valid, kx);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int j = c0 + e;
+          const float f = PC ? __expf(glv[j] - gcm[r * DK + j]) : ebar[r];
+          float hi, lo;
+          const uint32_t off = sw128_off(j, r);
+          split_bf16(bx[e] * f, hi, lo);
+          *reinterpret_cast<__nv_bfloat16 *>(sm + LY::BB_HI + off) = __float2bfloat16_rn(hi);
+          *reinterpret_cast<__nv_bfloat16 *>(sm + LY::BB_LO + off) = __float2bfloat16_rn(lo);
+          split_bf16(kx[e] * f, hi, lo);
+          *reinterpret_cast<__nv_bfloat16 *>(sm + LY::KB_HI + off) = __float2bfloat16_rn(hi);
+          *reinterpret_cast<__nv_bfloat16 *>(sm + LY::KB_LO + off) = __float2bfloat16_rn(lo);
+        }
+      }
+    }
+    sync_for_mma();
+    // ---- W = V^T Lk^T (over D1 columns 0-63)
+    if (t == 0) {
+#pragma unroll 1
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t lh = sdesc_sw128(s_lkh + kk * 32, 16, 1024);
+        mma_ts(tm + TD1, tm + TD1 + 64 + 8 * kk, lh, ID_64, kk > 0);
+        mma_ts(tm + TD1, tm + TD1 + 64 + 8 * kk, sdesc_sw128(s_lkl + kk * 32, 16, 1024), ID_64, 1);
+        mma_ts(tm + TD1, tm + TD1 + 96 + 8 * kk, lh, ID_64, 1);
+      }
+    }
+    mma_wait();
+    if (!ok) break;
+    // ---- R = zfa Z_a + W -> hi | lo over Z_a;  S <- S Diag(e^{gl})
+    {
+      float z[64], w[64];
+      {
+        float z0[32], z1[32];
+        tmem_ld32(lb + TZO, z0);
+        tmem_ld32(lb + TZO + 32, z1);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          z[e] = z0[e];
+          z[32 + e] = z1[e];
+        }
+        tmem_ld32(lb + TD1, z0);
+        tmem_ld32(lb + TD1 + 32, z1);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          w[e] = z0[e];
+          w[32 + e] = z1[e];
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < C; ++r) z[r] = zfa[r] * z[r] + w[r];
+      tmem_put_split64(lb + TZO, z);
+    }
+#pragma unroll 1
+    for (int q = 0; q < DK / 32; ++q) {
+      float x[32];
+      tmem_ld32(lb + TS + 32 * q, x);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) x[e] *= egl[32 * q + e];
+      tmem_st32(lb + TS + 32 * q, x);
+    }
+    tmem_wait_st();
+    // ---- T = (I - Lb)^{-1}: column c by forward substitution
+    if (t < 64) {
+      const int cl = t;
+      float y[64];
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        float acc = (r == cl) ? 1.f : 0.f;
+#pragma unroll
+        for (int s4 = 0; s4 < (r + 3) / 4; ++s4) {
+          const float4 a4 = Lb4[r * 16 + (s4 ^ (r & 15))];
+          if (4 * s4 + 0 < r) acc += a4.x * y[4 * s4 + 0];
+          if (4 * s4 + 1 < r) acc += a4.y * y[4 * s4 + 1];
+          if (4 * s4 + 2 < r) acc += a4.z * y[4 * s4 + 2];
+          if (4 * s4 + 3 < r) acc += a4.w * y[4 * s4 + 3];
+        }
+        y[r] = acc;
+      }
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        float hi, lo;
+        split_bf16(y[r], hi, lo);
+        const uint32_t off = sw128_off(r, cl);
+        *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_HI + off) = __float2bfloat16_rn(hi);
+        *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_LO + off) = __float2bfloat16_rn(lo);
+      }
+    }
+    sync_for_mma();
+    // ---- X^T = R T^T (over D1 columns 0-63)
+    if (t == 0) {
+#pragma unroll 1
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t th = sdesc_sw128(s_tth + kk * 32, 16, 1024);
+        mma_ts(tm + TD1, tm + TZO + 8 * kk, th, ID_64, kk > 0);
+        mma_ts(tm + TD1, tm + TZO + 8 * kk, sdesc_sw128(s_ttl + kk * 32, 16, 1024), ID_64, 1);
+        mma_ts(tm + TD1, tm + TZO + 32 + 8 * kk, th, ID_64, 1);
+      }
+    }
+    mma_wait();
+    if (!ok) break;
+    {
+      float x[64];
+      {
+        float x0[32], x1[32];
+        tmem_ld32(lb + TD1, x0);
+        tmem_ld32(lb + TD1 + 32, x1);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          x[e] = x0[e];
+          x[32 + e] = x1[e];
+        }
+      }
+      tmem_put_split64(lb + TD1, x);
+    }
+    sync_for_mma();
+    // ---- O_b = X^T P_b^T + V^T P_k^T (over ZO columns 0-63);
+    //      S += X^T (B e^{gl - gc}) + V^T (K e^{gl - gc})
+    if (t == 0) {
+#pragma unroll 1
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t xh = tm + TD1 + 8 * kk, xl = tm + TD1 + 32 + 8 * kk;
+        const uint32_t vh = tm + TD1 + 64 + 8 * kk, vl = tm + TD1 + 96 + 8 * kk;
+        const uint64_t pb = sdesc_sw128(s_pbh + kk * 32, 16, 1024);
+        const uint64_t pk = sdesc_sw128(s_pkh + kk * 32, 16, 1024);
+        const uint64_t bb = sdesc_sw128(s_bbh + kk * 32, 16, 1024);
+        const uint64_t kb = sdesc_sw128(s_kbh + kk * 32, 16, 1024);
+        mma_ts(tm + TZO, xh, pb, ID_64, kk > 0);
+        mma_ts(tm + TZO, xh, sdesc_sw128(s_pbl + kk * 32, 16, 1024), ID_64, 1);
+        mma_ts(tm + TZO, xl, pb, ID_64, 1);
+        mma_ts(tm + TZO, vh, pk, ID_64, 1);
+        mma_ts(tm + TZO, vh, sdesc_sw128(s_pkl + kk * 32, 16, 1024), ID_64, 1);
+        mma_ts(tm + TZO, vl, pk, ID_64, 1);
+        mma_ts(tm + TS, xh, bb, ID_S, 1);
+        mma_ts(tm + TS, xh, sdesc_sw128(s_bbl + kk * 32, 16, 1024), ID_S, 1);
+        mma_ts(tm + TS, xl, bb, ID_S, 1);
+        mma_ts(tm + TS, vh, kb, ID_S, 1);
+        mma_ts(tm + TS, vh, sdesc_sw128(s_kbl + kk * 32, 16, 1024), ID_S, 1);
+        mma_ts(tm + TS, vl, kb, ID_S, 1);
+      }
+    }
+    mma_wait();
+    if (!ok) break;
+    // ---- o_r = zfo_r O_a + O_b
+#pragma unroll 1
+    for (int hp = 0; hp < 2; ++hp) {
+      float oa[32], ob[32];
+      tmem_ld32(lb + TZO + 64 + 32 * hp, oa);
+      tmem_ld32(lb + TZO + 32 * hp, ob);
+      if (i < dv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int r = 32 * hp + e;
+          if (r < L) store_out(p.o, (tok0 + (size_t)r * H) * dv + i, zfo[r] * oa[e] + ob[e], bf);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (ok && p.S_T) {
+#pragma unroll 1
+    for (int q = 0; q < DK / 32; ++q) {
+      float x[32];
+      tmem_ld32(lb + TS + 32 * q, x);
+      if (i < dv) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int j = 32 * q + e;
+          if (j < dk) p.S_T[((size_t)bh * dv + i) * dk + j] = x[e];
+        }
+      }
+    }
+  }
+  if (!ok && t == 0) atomicOr(p.status, kStatusTimeout);
+  if (t == 0) {
+    mma_commit(bar);
+    mbar_wait_bounded(bar, ph, kWaitNs);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+template <int DK, bool PC>
+cudaError_t launch_dplr_split(const DplrChunkArgs &a, cudaStream_t stream) {
+  auto kern = gdr_dplr_split_kernel<DK, PC>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)DLayout<DK>::bytes);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)(a.B * a.H), kThreads, DLayout<DK>::bytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool chunk_split_supports(const ChunkArgs &a) {
@@ -583,6 +1086,18 @@ cudaError_t launch_chunk_split(const ChunkArgs &a, cudaStream_t stream) {
   if (a.dk == 128)
     return a.per_channel ? launch_split<128, true>(a, stream) : launch_split<128, false>(a, stream);
   return a.per_channel ? launch_split<64, true>(a, stream) : launch_split<64, false>(a, stream);
+}
+
+cudaError_t launch_dplr_chunk(const DplrChunkArgs &a, cudaStream_t stream) {
+  const bool dims = (a.dk == 32 || a.dk == 64 || a.dk == 128) &&
+                    (a.dv == 32 || a.dv == 64 || a.dv == 128);
+  if (!dims) return cudaErrorNotSupported;
+  if (a.B * a.H == 0) return cudaSuccess;
+  if (a.dk == 128)
+    return a.per_channel ? launch_dplr_split<128, true>(a, stream)
+                         : launch_dplr_split<128, false>(a, stream);
+  return a.per_channel ? launch_dplr_split<64, true>(a, stream)
+                       : launch_dplr_split<64, false>(a, stream);
 }
 
 }  // namespace gdr

@@ -95,11 +95,19 @@ cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStrea
 // Device address, on the current device, of the library's fixed scratch
 // array (GDR_NOALLOC_SCRATCH_BYTES), looked up once per device.
 cudaError_t noalloc_scratch(void **out);
-// DPLR transition, recurrent forward (CUDA cores, d_k = d_v = d in {32, 64, 128}).
-cudaError_t launch_dplr(const void *q, const void *k, const void *v, const void *a,
-                        const void *b, int bf16, const float *g, int per_channel,
-                        const float *S0, void *o, float *S_T, int B, int T, int H, int d,
-                        cudaStream_t stream);
+// DPLR transition, chunked forward on the tensor cores (split operands):
+// S_t = S_{t-1} (Diag(alpha_t) + a_t b_t^T) + v_t k_t^T, o_t = S_t q_t.
+struct DplrChunkArgs {
+  const void *q, *k, *v, *a, *b;  // [B, T, H, dk] (v: dv), bf16 or fp32
+  const float *g;                 // [B, T, H] or [B, T, H, dk]
+  const float *S0;                // [B, H, dv, dk] or null
+  void *o;                        // [B, T, H, dv]
+  float *S_T;                     // [B, H, dv, dk] or null
+  int B, T, H, dk, dv;
+  int bf16, per_channel;
+  unsigned int *status;
+};
+cudaError_t launch_dplr_chunk(const DplrChunkArgs &a, cudaStream_t stream);
 // Backward of the recurrence (CUDA cores, d_k = d_v = d in {32, 64, 128}).
 size_t bwd_ws_bytes(int B, int T, int H, int d);
 cudaError_t launch_bwd(const void *q, const void *k, const void *v, int bf16, const float *g,

@@ -301,9 +301,17 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
  *   g           [B, T, H] or [B, T, H, dk] fp32
  *   S0, S_T     [B, H, dv, dk] fp32 or NULL (zero state / not written)
  *
- * A recurrent forward on CUDA cores in fp32 (one CTA per (b, h)), for
- * dk = dv in {32, 64, 128} (GDR_ERR_UNSUPPORTED otherwise).  One launch, no
- * workspace; S0 may alias S_T.
+ * Chunked on the tensor cores (C = 64, one CTA per (b, h), one launch, no
+ * workspace), the way section 5 of that page chunks the delta rule: per
+ * chunk the low-rank reads x_r = S_{r-1} a_r solve a unit lower-triangular
+ * system (the delta rule's WY form with the erase direction b and the write
+ * key k kept apart), then o and the end state follow from three intra-chunk
+ * products and two state products.  Operands are carried as two bf16 terms
+ * and products as three MMAs (close to fp32 accuracy); the state is fp32.
+ * dk, dv in {32, 64, 128} (GDR_ERR_UNSUPPORTED otherwise); pointers 16-byte
+ * aligned; S0 may alias S_T.  A per-channel gate has the split-operand
+ * range of gdr_chunk_fwd (decay over each half chunk above about -69 per
+ * channel), beyond which the call records GDR_ERR_RANGE.
  */
 gdr_status gdr_dplr_fwd(const void *q, const void *k, const void *v, const void *a,
                         const void *b, gdr_dtype in_dtype, const float *g, gdr_gate_kind gate,

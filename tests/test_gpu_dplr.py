@@ -1,7 +1,8 @@
-"""GPU parity of gdr_dplr_fwd (the diagonal-plus-low-rank transition) against
-the fp64 oracle.  The kernel keeps the state in fp32 and computes in fp32 on
-the same inputs; o is rounded to the input dtype.  Bars: o within 2e-2 for
-bf16 inputs (its rounding) and 1e-4 for fp32; S_T within 1e-4."""
+"""GPU parity of gdr_dplr_fwd (the diagonal-plus-low-rank transition, chunked
+on the tensor cores with split bf16 operands) against the fp64 oracle.  The
+state is fp32 and every product is carried to near fp32 accuracy on the same
+inputs; o is rounded to the input dtype.  Bars: o within 2e-2 for bf16
+inputs (its rounding) and 1e-4 for fp32; S_T within 1e-4."""
 import pytest
 import torch
 
@@ -79,3 +80,59 @@ def test_dplr_empty_sequence(cuda_device):
     inp = make_dplr_inputs(1, 0, 2, 64, torch.float32, "scalar", True, seed=144)
     _, S_T = _run(inp, cuda_device)
     assert torch.equal(S_T.cpu(), inp["S0"])
+
+
+@pytest.mark.parametrize("dk,dv,dtype", [(64, 128, torch.float32), (128, 32, torch.bfloat16),
+                                         (32, 64, torch.float32)])
+def test_dplr_unequal_head_dims(cuda_device, dk, dv, dtype):
+    """d_k != d_v: q, k, a, b [.., dk], v and o [.., dv], state [dv, dk];
+    a ragged tail (130 = 2 x 64 + 2), per-channel gate, S0 given."""
+    inp = make_dplr_inputs(2, 130, 2, dk, dtype, "channel", True, seed=160 + dk + dv)
+    gen = torch.Generator().manual_seed(161 + dv)
+    v = torch.randn(2, 130, 2, dv, generator=gen).to(dtype)
+    S0 = 0.02 * torch.randn(2, 2, dv, dk, generator=gen)
+    inp = dict(inp, v=v, S0=S0)
+    o, S_T = _run(inp, cuda_device)
+    ro, rS = _oracle(inp)
+    assert_close(o, ro, 2e-2 if dtype == torch.bfloat16 else 1e-4, "o")
+    assert_close(S_T, rS, 1e-4, "S_T")
+
+
+def _one_channel_decay(inp, g_channel, channel=5, head=0):
+    g = inp["g"].clone()
+    g[:, :, head, channel] = g_channel
+    return dict(inp, g=g.contiguous())
+
+
+def test_dplr_per_channel_strong_decay_in_range(cuda_device):
+    """One key channel at g = -2 per token (-62 over half a chunk, inside the
+    split-operand range): oracle parity at the fp32 bar, clean status."""
+    inp = _one_channel_decay(make_dplr_inputs(1, 200, 2, 64, torch.float32, "channel", True,
+                                              seed=170), -2.0)
+    o, S_T = _run(inp, cuda_device)
+    assert binding.device_status() == binding.GDR_OK
+    ro, rS = _oracle(inp)
+    assert_close(o, ro, 1e-4, "o")
+    assert_close(S_T, rS, 1e-4, "S_T")
+
+
+def test_dplr_per_channel_rapid_forgetting_reports_range(cuda_device):
+    """g = -30 per token in one channel is outside the factor range: the call
+    records GDR_ERR_RANGE and its outputs stay finite."""
+    inp = _one_channel_decay(make_dplr_inputs(1, 200, 2, 64, torch.float32, "channel", True,
+                                              seed=171), -30.0)
+    o, S_T = _run(inp, cuda_device)
+    assert binding.device_status() == binding.GDR_ERR_RANGE
+    assert torch.isfinite(o).all() and torch.isfinite(S_T).all()
+
+
+def test_dplr_full_size_workload(cuda_device):
+    """The DPLR workload (B8 T4096 H16 d128, bf16, scalar gate), whole
+    tensors against the full oracle."""
+    from gated_delta_rule_93_b200.inputs import WORKLOADS, make_workload_inputs
+    inp = make_workload_inputs(WORKLOADS["dplr_b8_t4096_h16_d128"])
+    o, S_T = _run(inp, cuda_device)
+    assert binding.device_status() == binding.GDR_OK
+    ro, rS = _oracle(inp)
+    assert_close(o, ro, 2e-2, "o")
+    assert_close(S_T, rS, 1e-4, "S_T")
