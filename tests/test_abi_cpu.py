@@ -259,9 +259,11 @@ def test_dplr_validation_rejects_before_any_launch(L):
     assert call(T=-1) == binding.GDR_ERR_INVALID_ARG
     assert call(dt=7) == binding.GDR_ERR_INVALID_ARG
     assert call(gate=2) == binding.GDR_ERR_INVALID_ARG
-    assert call(dk=64, dv=32) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dk=64, dv=48) == binding.GDR_ERR_UNSUPPORTED
     assert call(dk=48, dv=48) == binding.GDR_ERR_UNSUPPORTED
     assert call(a=None) == binding.GDR_ERR_INVALID_ARG
+    assert call(a=_fake_ptr(4)) == binding.GDR_ERR_INVALID_ARG
+    assert call(S0=_fake_ptr(8)) == binding.GDR_ERR_INVALID_ARG
     assert call(b=None) == binding.GDR_ERR_INVALID_ARG
     assert call(B=0) == binding.GDR_OK
 
