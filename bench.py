@@ -37,18 +37,37 @@ METRIC = "tokens/s and TFLOP/s per gated-delta layer fwd (1 B200), % of roofline
 DEFAULT_WORKLOAD = "gdn_b8_t4096_h16_d128"
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = {
+    # the kernel each kind of workload times, for the profile's source hash
     "chunk": ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
-              "gated_delta_rule_93_b200/csrc/gdr_chunk_split.cu",
+              "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
+    "seg": ["gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
+            "gated_delta_rule_93_b200/csrc/gdr_segments.cu",
+            "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
+    "split": ["gated_delta_rule_93_b200/csrc/gdr_chunk_split.cu",
               "gated_delta_rule_93_b200/csrc/gdr_tc_util.cuh",
-              "gated_delta_rule_93_b200/csrc/gdr_segments.cu",
               "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
     "step": ["gated_delta_rule_93_b200/csrc/gdr_step.cu"],
-    "bwd": ["gated_delta_rule_93_b200/csrc/gdr_bwd.cu",
-            "gated_delta_rule_93_b200/csrc/gdr_bwd_tc.cu",
-            "gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu"],
+    "bwd": ["gated_delta_rule_93_b200/csrc/gdr_bwd_tc.cu",
+            "gated_delta_rule_93_b200/csrc/gdr_tc_util.cuh",
+            "gated_delta_rule_93_b200/csrc/gdr_chunk_tc.cu",
+            "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
     "dplr": ["gated_delta_rule_93_b200/csrc/gdr_chunk_split.cu",
-             "gated_delta_rule_93_b200/csrc/gdr_tc_util.cuh"],
+             "gated_delta_rule_93_b200/csrc/gdr_tc_util.cuh",
+             "gated_delta_rule_93_b200/csrc/gdr_sm100.cuh"],
 }
+
+
+def kernel_kind(w, launches=1):
+    """Which kernel a workload times: the KERNEL_SOURCES key."""
+    if w.backward:
+        return "bwd"
+    if w.mixer == "dplr":
+        return "dplr"
+    if w.kind == "step":
+        return "step"
+    if w.dtype != torch.bfloat16 or w.dk != 128 or w.dv != 128:
+        return "split"
+    return "seg" if launches > 1 else "chunk"
 
 
 # ------------------------------------------------------------------ work model
@@ -332,7 +351,7 @@ def time_device(step, steps, warmup, dev, world, local_rank):
     return t0.elapsed_time(t1), [a.elapsed_time(b) for a, b in ev], clk
 
 
-def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk):
+def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk, launches=1):
     """tokens/s, TFLOP/s and the roofline of one timed workload."""
     ms_step = total_ms / steps
     tokens_step = w.B * w.T if w.kind == "chunk" else w.B  # tokens one step processes
@@ -351,15 +370,14 @@ def roofline_fields(w, total_ms, per_launch_ms, steps, world, clk):
         roof = {"bound": "alu", "achieved": aflops / (avg_launch_ms / 1e3) / 1e12,
                 "peak": alu_peak, "unit": "TFLOP/s",
                 "frac": aflops / (avg_launch_ms / 1e3) / 1e12 / alu_peak,
-                "traffic": recorded_traffic(w.name, "bwd"),
+                "traffic": recorded_traffic(w.name, kernel_kind(w, launches)),
                 "peak_source": "CUDA-core fp32 FMA, 148 SMs x 128 lanes x 2 flop x max SM "
                                "clock", "algorithmic_flops_per_launch": aflops,
                 "kernel": "gdr_chunk_bwd"}
     else:
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak,
-                "traffic": recorded_traffic(w.name, "bwd" if w.backward else
-                                            "dplr" if w.mixer == "dplr" else w.kind),
+                "traffic": recorded_traffic(w.name, kernel_kind(w, launches)),
                 "peak_source": peak_kind, "algorithmic_bytes_per_launch": abytes,
                 "kernel": ("gdr_chunk_bwd (tensor cores, 3 launches)" if w.backward else
                            "gdr_chunk_fwd_prologue" if w.prologue else
@@ -384,7 +402,7 @@ def time_extra(name, args, rank, world, local_rank, dev):
     steps, warmup = max(5, min(args.steps, 20)), 3
     r = make_step(w, dev, rank, warmup + steps + 3)
     total_ms, per_launch, clk = time_device(r["step"], steps, warmup, dev, world, local_rank)
-    f = roofline_fields(w, total_ms, per_launch, steps, world, clk)
+    f = roofline_fields(w, total_ms, per_launch, steps, world, clk, r["launches"])
     out = {"metric_value": f["value"], "unit": "tokens/s", "ms_per_step": f["ms_per_step"],
            "steps": steps, "warmup": warmup, "tflops": f["tflops"],
            "roofline_fraction": f["roofline_fraction"], "roofline": f["roofline"],
@@ -462,7 +480,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- max over ranks
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], device=dev)
-    f = roofline_fields(w, total_ms, per_launch_ms, args.steps, world, clk)
+    f = roofline_fields(w, total_ms, per_launch_ms, args.steps, world, clk, launches_per_step)
 
     # ---- the other workloads, each timed on its own after the headline one
     extras = {}
