@@ -92,18 +92,16 @@ struct Cols {
   static_assert(U + 64 <= 512, "TMEM columns");
 };
 
-// 8 consecutive input elements (fp32 or bf16) of row `row`, columns c0.. of
-// a [B, T, H, d] tensor; zero past the row's d or the sequence.
-__device__ __forceinline__ void load8(const void *p, int bf16, size_t row_off, int c0, int d,
-                                      bool valid, float (&x)[8]) {
-  if (!valid || c0 >= d) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = 0.f;
-    return;
-  }
-  if (bf16) {
-    const uint4 u = *reinterpret_cast<const uint4 *>(
-        reinterpret_cast<const __nv_bfloat16 *>(p) + row_off + c0);
+// 8 consecutive input elements (fp32 if !BF, else bf16) of a [B, T, H, d]
+// tensor at element offset `off`.  Callers pass an in-range offset for
+// every lane (a clamped one where the element is padding) and select zero
+// afterwards, so that the loads carry no branch and all of a phase's loads
+// can be in flight together.
+template <bool BF>
+__device__ __forceinline__ void ld8(const void *p, size_t off, float (&x)[8]) {
+  if (BF) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(p) +
+                                                     off);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -112,11 +110,138 @@ __device__ __forceinline__ void load8(const void *p, int bf16, size_t row_off, i
       x[2 * e + 1] = f.y;
     }
   } else {
-    const float4 *q = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p) +
-                                                       row_off + c0);
+    const float4 *q = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p) + off);
     const float4 a = q[0], b = q[1];
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
     x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+}
+
+template <bool BF>
+__device__ __forceinline__ float ld1(const void *p, size_t off) {
+  if (BF) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[off]);
+  return reinterpret_cast<const float *>(p)[off];
+}
+
+template <bool BF>
+__device__ __forceinline__ void st1(void *p, size_t off, float x) {
+  if (BF)
+    reinterpret_cast<__nv_bfloat16 *>(p)[off] = __float2bfloat16_rn(x);
+  else
+    reinterpret_cast<float *>(p)[off] = x;
+}
+
+// Element (row r, column c0) of a chunk's [64][d] input block starting at
+// token row offset `tok0` (token stride H): the offset of the element when
+// it exists (r < L, c0 < d), else of the chunk's first element.
+__device__ __forceinline__ size_t in_off(size_t tok0, int r, int c0, int H, int d, bool valid) {
+  return valid ? (tok0 + (size_t)r * H) * d + c0 : tok0 * d;
+}
+
+// 16 consecutive fp32 of row r of a swizzled [64][16 float4] matrix,
+// columns 16 q .. 16 q + 15.
+__device__ __forceinline__ void ld_row16(const float4 *N4, int r, int q, float (&x)[16]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float4 v = N4[r * 16 + ((4 * q + u) ^ (r & 15))];
+    x[4 * u] = v.x;
+    x[4 * u + 1] = v.y;
+    x[4 * u + 2] = v.z;
+    x[4 * u + 3] = v.w;
+  }
+}
+
+// X = (I + s N)^{-1} for a strictly lower-triangular 64 x 64 N (s = +1 or
+// -1), by 16 x 16 blocks; threads 0-63 (the other warps do not take part;
+// 64-thread named barrier 1).  N is fp32 [64][16 float4] with float4 k of
+// row r at k ^ (r % 16); X goes to Y [64][64] fp32 ([row][column]: a warp's
+// lanes hit distinct banks).  With L = I + s N:
+//   X_ii = L_ii^{-1}   (four blocks at once, one column per thread, by
+//                       forward substitution)
+//   X_ij = -s X_ii sum_{k=j}^{i-1} N_ik X_kj   (i > j, in three levels
+//                       i - j = 1, 2, 3; 48, 32, then 16 threads, one column
+//                       each)
+// The products' loops stay rolled over blocks, so the code is small: a
+// fully unrolled 64-row substitution is ~40 KB of straight-line code and
+// ran from instruction-cache misses.
+template <int S>
+__device__ __forceinline__ void block_solve(const float4 *N4, float *Y, int t) {
+  {  // diagonal blocks: block i = t / 16, column c = 16 i + t % 16
+    const int i = t >> 4, cc = t & 15, c = 16 * i + cc;
+    float y[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float nr[16];
+      ld_row16(N4, 16 * i + k, i, nr);
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < k; ++j) sum = fmaf(nr[j], y[j], sum);
+      y[k] = (k == cc ? 1.f : 0.f) - (float)S * sum;
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) Y[(16 * i + k) * 64 + c] = y[k];
+#pragma unroll 1
+    for (int r = 0; r < 16 * i; ++r) Y[r * 64 + c] = 0.f;  // above the diagonal blocks
+  }
+  asm volatile("bar.sync 1, 64;" ::: "memory");
+#pragma unroll 1
+  for (int lvl = 1; lvl < 4; ++lvl) {
+    if (t < 16 * (4 - lvl)) {
+      const int j = t >> 4, i = j + lvl, c = 16 * j + (t & 15);
+      float m[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) m[u] = 0.f;
+#pragma unroll 1
+      for (int k = j; k < i; ++k) {  // m += N_ik X_kj[:, c], four rows of N_ik at a time
+        float xk[16];
+#pragma unroll
+        for (int p = 0; p < 16; ++p) xk[p] = Y[(16 * k + p) * 64 + c];
+#pragma unroll
+        for (int ug = 0; ug < 4; ++ug) {
+          float n0[16], n1[16], n2[16], n3[16];
+          ld_row16(N4, 16 * i + 4 * ug + 0, k, n0);
+          ld_row16(N4, 16 * i + 4 * ug + 1, k, n1);
+          ld_row16(N4, 16 * i + 4 * ug + 2, k, n2);
+          ld_row16(N4, 16 * i + 4 * ug + 3, k, n3);
+#pragma unroll
+          for (int p = 0; p < 16; ++p) {  // four independent chains, interleaved
+            m[4 * ug + 0] = fmaf(n0[p], xk[p], m[4 * ug + 0]);
+            m[4 * ug + 1] = fmaf(n1[p], xk[p], m[4 * ug + 1]);
+            m[4 * ug + 2] = fmaf(n2[p], xk[p], m[4 * ug + 2]);
+            m[4 * ug + 3] = fmaf(n3[p], xk[p], m[4 * ug + 3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int ug = 0; ug < 4; ++ug) {  // X_ij[:, c] = -s X_ii m, four rows at a time
+        float x0[16], x1[16], x2[16], x3[16];
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        const float4 *r0 = reinterpret_cast<const float4 *>(Y + (16 * i + 4 * ug + 0) * 64 + 16 * i);
+        const float4 *r1 = reinterpret_cast<const float4 *>(Y + (16 * i + 4 * ug + 1) * 64 + 16 * i);
+        const float4 *r2 = reinterpret_cast<const float4 *>(Y + (16 * i + 4 * ug + 2) * 64 + 16 * i);
+        const float4 *r3 = reinterpret_cast<const float4 *>(Y + (16 * i + 4 * ug + 3) * 64 + 16 * i);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 v0 = r0[q], v1 = r1[q], v2 = r2[q], v3 = r3[q];
+          x0[4 * q] = v0.x; x0[4 * q + 1] = v0.y; x0[4 * q + 2] = v0.z; x0[4 * q + 3] = v0.w;
+          x1[4 * q] = v1.x; x1[4 * q + 1] = v1.y; x1[4 * q + 2] = v1.z; x1[4 * q + 3] = v1.w;
+          x2[4 * q] = v2.x; x2[4 * q + 1] = v2.y; x2[4 * q + 2] = v2.z; x2[4 * q + 3] = v2.w;
+          x3[4 * q] = v3.x; x3[4 * q + 1] = v3.y; x3[4 * q + 2] = v3.z; x3[4 * q + 3] = v3.w;
+        }
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          a0 = fmaf(x0[p], m[p], a0);
+          a1 = fmaf(x1[p], m[p], a1);
+          a2 = fmaf(x2[p], m[p], a2);
+          a3 = fmaf(x3[p], m[p], a3);
+        }
+        Y[(16 * i + 4 * ug + 0) * 64 + c] = -(float)S * a0;
+        Y[(16 * i + 4 * ug + 1) * 64 + c] = -(float)S * a1;
+        Y[(16 * i + 4 * ug + 2) * 64 + c] = -(float)S * a2;
+        Y[(16 * i + 4 * ug + 3) * 64 + c] = -(float)S * a3;
+      }
+    }
+    asm volatile("bar.sync 1, 64;" ::: "memory");
   }
 }
 
@@ -167,7 +292,7 @@ __device__ __forceinline__ void sync_for_mma() {
   tc_fence_after();
 }
 
-template <int DK, bool PC>
+template <int DK, bool PC, bool BF>
 __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs a) {
   using LY = Layout<DK>;
   using TC = Cols<DK>;
@@ -176,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
                                             ~uintptr_t(1023));
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, H = a.H;
-  const int dk = a.dk, dv = a.dv, bf = a.bf16;
+  const int dk = a.dk, dv = a.dv;
   const int n = (a.T + C - 1) / C;
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + LY::BAR);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + LY::MISC);
@@ -314,15 +439,20 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     // ---- K~, Q~, K^, (K e^{gl - gc})^T tiles: row r = t / 2, half t % 2 of the columns
     {
       const int r = t >> 1, hf = t & 1;
-      const bool valid = r < L;
-      const size_t rk = (tok0 + (size_t)r * H) * dk;
       bool range_bad = false;
-#pragma unroll 1
+#pragma unroll
       for (int g8 = 0; g8 < DK / 16; ++g8) {
         const int c0 = hf * (DK / 2) + 8 * g8;
+        const bool valid = r < L && c0 < dk;
+        const size_t off = in_off(tok0, r, c0, H, dk, valid);
         float kx[8], qx[8];
-        load8(a.k, bf, rk, c0, dk, valid, kx);
-        load8(a.q, bf, rk, c0, dk, valid, qx);
+        ld8<BF>(a.k, off, kx);
+        ld8<BF>(a.q, off, qx);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          kx[e] = valid ? kx[e] : 0.f;
+          qx[e] = valid ? qx[e] : 0.f;
+        }
         float kt[8], qt[8], kh[8], kb[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -429,12 +559,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
           z[32 + e] = z1[e];
         }
       }
-      const size_t vi = tok0 * dv + i;
+      const int ic = i < dv ? i : 0;
+      float vr[64];
 #pragma unroll
-      for (int r = 0; r < C; ++r) {
-        const float vr = (r < L && i < dv) ? load_in(a.v, vi + (size_t)r * H * dv, bf) : 0.f;
-        z[r] = vr - zf[r] * z[r];
-      }
+      for (int r = 0; r < C; ++r) vr[r] = ld1<BF>(a.v, (tok0 + (size_t)(r < L ? r : 0) * H) * dv + ic);
+#pragma unroll
+      for (int r = 0; r < C; ++r) z[r] = ((r < L && i < dv) ? vr[r] : 0.f) - zf[r] * z[r];
       tmem_put_split64(lb + TC::ZO, z);
     }
 #pragma unroll 1
@@ -448,27 +578,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     tmem_wait_st();
     __syncthreads();
     // ---- T = (I + A)^{-1} Diag(beta): column c by forward substitution
-    if (t < 64) {
+    if (t < 64) {  // Y over the per-channel decays (read only before D1)
       const int cl = t;
-      float y[64];
-#pragma unroll
-      for (int r = 0; r < C; ++r) {
-        float acc = (r == cl) ? 1.f : 0.f;
-#pragma unroll
-        for (int s4 = 0; s4 < (r + 3) / 4; ++s4) {
-          const float4 a4 = Af4[r * 16 + (s4 ^ (r & 15))];
-          if (4 * s4 + 0 < r) acc -= a4.x * y[4 * s4 + 0];
-          if (4 * s4 + 1 < r) acc -= a4.y * y[4 * s4 + 1];
-          if (4 * s4 + 2 < r) acc -= a4.z * y[4 * s4 + 2];
-          if (4 * s4 + 3 < r) acc -= a4.w * y[4 * s4 + 3];
-        }
-        y[r] = acc;
-      }
+      float *Y = gcm;
+      block_solve<1>(Af4, Y, cl);
       const float bc = betav[cl];
-#pragma unroll
+#pragma unroll 8
       for (int r = 0; r < C; ++r) {
         float hi, lo;
-        split_bf16(y[r] * bc, hi, lo);
+        split_bf16(Y[r * 64 + cl] * bc, hi, lo);
         const uint32_t off = sw128_off(r, cl);
         *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_HI + off) = __float2bfloat16_rn(hi);
         *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_LO + off) = __float2bfloat16_rn(lo);
@@ -529,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int r = 32 * hp + e;
-          if (r < L) store_out(a.o, (tok0 + (size_t)r * H) * dv + i, zf[r] * oa[e] + ob[e], bf);
+          if (r < L) st1<BF>(a.o, (tok0 + (size_t)r * H) * dv + i, zf[r] * oa[e] + ob[e]);
         }
       }
     }
@@ -560,9 +678,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
   if (warp == 0) tmem_dealloc(tm, 512);
 }
 
-template <int DK, bool PC>
+template <int DK, bool PC, bool BF>
 cudaError_t launch_split(const ChunkArgs &a, cudaStream_t stream) {
-  auto kern = gdr_chunk_split_kernel<DK, PC>;
+  auto kern = gdr_chunk_split_kernel<DK, PC, BF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Layout<DK>::bytes);
   if (e != cudaSuccess) return e;
@@ -614,7 +732,7 @@ struct DLayout {
   static_assert(bytes <= 232448, "shared memory budget");
 };
 
-template <int DK, bool PC>
+template <int DK, bool PC, bool BF>
 __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkArgs p) {
   using LY = DLayout<DK>;
   // TMEM: S [DK], S' hi / lo [DK/2 each], D1 [128] (then W / X in its first
@@ -627,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
                                             ~uintptr_t(1023));
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H, H = p.H;
-  const int dk = p.dk, dv = p.dv, bf = p.bf16;
+  const int dk = p.dk, dv = p.dv;
   const int n = (p.T + C - 1) / C;
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + LY::BAR);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + LY::MISC);
@@ -762,17 +880,24 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     // ---- [A^; Q~] and [B^; K^] tiles: row r = t / 2, half t % 2 of the columns
     {
       const int r = t >> 1, hf = t & 1;
-      const bool valid = r < L;
-      const size_t rk = (tok0 + (size_t)r * H) * dk;
       bool range_bad = false;
-#pragma unroll 1
+#pragma unroll
       for (int g8 = 0; g8 < DK / 16; ++g8) {
         const int c0 = hf * (DK / 2) + 8 * g8;
+        const bool valid = r < L && c0 < dk;
+        const size_t off = in_off(tok0, r, c0, H, dk, valid);
         float ax[8], qx[8], bx[8], kx[8];
-        load8(p.a, bf, rk, c0, dk, valid, ax);
-        load8(p.q, bf, rk, c0, dk, valid, qx);
-        load8(p.b, bf, rk, c0, dk, valid, bx);
-        load8(p.k, bf, rk, c0, dk, valid, kx);
+        ld8<BF>(p.a, off, ax);
+        ld8<BF>(p.q, off, qx);
+        ld8<BF>(p.b, off, bx);
+        ld8<BF>(p.k, off, kx);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          ax[e] = valid ? ax[e] : 0.f;
+          qx[e] = valid ? qx[e] : 0.f;
+          bx[e] = valid ? bx[e] : 0.f;
+          kx[e] = valid ? kx[e] : 0.f;
+        }
         if (PC) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -861,22 +986,28 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     }
     {  // V^T (lane = value channel) as hi | lo into D1 columns 64-127
       float vt[64];
-      const size_t vi = tok0 * dv + i;
+      const int ic = i < dv ? i : 0;
 #pragma unroll
-      for (int r = 0; r < C; ++r)
-        vt[r] = (r < L && i < dv) ? load_in(p.v, vi + (size_t)r * H * dv, bf) : 0.f;
+      for (int r = 0; r < C; ++r) vt[r] = ld1<BF>(p.v, (tok0 + (size_t)(r < L ? r : 0) * H) * dv + ic);
+#pragma unroll
+      for (int r = 0; r < C; ++r) vt[r] = (r < L && i < dv) ? vt[r] : 0.f;
       tmem_put_split64(lb + TD1 + 64, vt);
     }
     {  // (B e^{gl - gc})^T and (K e^{gl - gc})^T over [B^; K^] (dead after D1)
       const int r = t >> 1, hf = t & 1;
-      const bool valid = r < L;
-      const size_t rk = (tok0 + (size_t)r * H) * dk;
-#pragma unroll 1
+#pragma unroll
       for (int g8 = 0; g8 < DK / 16; ++g8) {
         const int c0 = hf * (DK / 2) + 8 * g8;
+        const bool valid = r < L && c0 < dk;
+        const size_t off = in_off(tok0, r, c0, H, dk, valid);
         float bx[8], kx[8];
-        load8(p.b, bf, rk, c0, dk, valid, bx);
-        load8(p.k, bf, rk, c0, dk, valid, kx);
+        ld8<BF>(p.b, off, bx);
+        ld8<BF>(p.k, off, kx);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          bx[e] = valid ? bx[e] : 0.f;
+          kx[e] = valid ? kx[e] : 0.f;
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int j = c0 + e;
@@ -939,26 +1070,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     }
     tmem_wait_st();
     // ---- T = (I - Lb)^{-1}: column c by forward substitution
-    if (t < 64) {
+    if (t < 64) {  // Y over the per-channel decays (read only before this)
       const int cl = t;
-      float y[64];
-#pragma unroll
-      for (int r = 0; r < C; ++r) {
-        float acc = (r == cl) ? 1.f : 0.f;
-#pragma unroll
-        for (int s4 = 0; s4 < (r + 3) / 4; ++s4) {
-          const float4 a4 = Lb4[r * 16 + (s4 ^ (r & 15))];
-          if (4 * s4 + 0 < r) acc += a4.x * y[4 * s4 + 0];
-          if (4 * s4 + 1 < r) acc += a4.y * y[4 * s4 + 1];
-          if (4 * s4 + 2 < r) acc += a4.z * y[4 * s4 + 2];
-          if (4 * s4 + 3 < r) acc += a4.w * y[4 * s4 + 3];
-        }
-        y[r] = acc;
-      }
-#pragma unroll
+      float *Y = gcm;
+      block_solve<-1>(Lb4, Y, cl);
+#pragma unroll 8
       for (int r = 0; r < C; ++r) {
         float hi, lo;
-        split_bf16(y[r], hi, lo);
+        split_bf16(Y[r * 64 + cl], hi, lo);
         const uint32_t off = sw128_off(r, cl);
         *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_HI + off) = __float2bfloat16_rn(hi);
         *reinterpret_cast<__nv_bfloat16 *>(sm + LY::TT_LO + off) = __float2bfloat16_rn(lo);
@@ -1029,7 +1148,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int r = 32 * hp + e;
-          if (r < L) store_out(p.o, (tok0 + (size_t)r * H) * dv + i, zfo[r] * oa[e] + ob[e], bf);
+          if (r < L) st1<BF>(p.o, (tok0 + (size_t)r * H) * dv + i, zfo[r] * oa[e] + ob[e]);
         }
       }
     }
@@ -1060,9 +1179,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
   if (warp == 0) tmem_dealloc(tm, 512);
 }
 
-template <int DK, bool PC>
+template <int DK, bool PC, bool BF>
 cudaError_t launch_dplr_split(const DplrChunkArgs &a, cudaStream_t stream) {
-  auto kern = gdr_dplr_split_kernel<DK, PC>;
+  auto kern = gdr_dplr_split_kernel<DK, PC, BF>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)DLayout<DK>::bytes);
   if (e != cudaSuccess) return e;
@@ -1083,9 +1202,17 @@ bool chunk_split_supports(const ChunkArgs &a) {
 cudaError_t launch_chunk_split(const ChunkArgs &a, cudaStream_t stream) {
   if (!chunk_split_supports(a)) return cudaErrorNotSupported;
   if (a.B * a.H == 0) return cudaSuccess;
-  if (a.dk == 128)
-    return a.per_channel ? launch_split<128, true>(a, stream) : launch_split<128, false>(a, stream);
-  return a.per_channel ? launch_split<64, true>(a, stream) : launch_split<64, false>(a, stream);
+  const int key = (a.dk == 128 ? 4 : 0) | (a.per_channel ? 2 : 0) | (a.bf16 ? 1 : 0);
+  switch (key) {
+    case 0: return launch_split<64, false, false>(a, stream);
+    case 1: return launch_split<64, false, true>(a, stream);
+    case 2: return launch_split<64, true, false>(a, stream);
+    case 3: return launch_split<64, true, true>(a, stream);
+    case 4: return launch_split<128, false, false>(a, stream);
+    case 5: return launch_split<128, false, true>(a, stream);
+    case 6: return launch_split<128, true, false>(a, stream);
+    default: return launch_split<128, true, true>(a, stream);
+  }
 }
 
 cudaError_t launch_dplr_chunk(const DplrChunkArgs &a, cudaStream_t stream) {
@@ -1093,11 +1220,17 @@ cudaError_t launch_dplr_chunk(const DplrChunkArgs &a, cudaStream_t stream) {
                     (a.dv == 32 || a.dv == 64 || a.dv == 128);
   if (!dims) return cudaErrorNotSupported;
   if (a.B * a.H == 0) return cudaSuccess;
-  if (a.dk == 128)
-    return a.per_channel ? launch_dplr_split<128, true>(a, stream)
-                         : launch_dplr_split<128, false>(a, stream);
-  return a.per_channel ? launch_dplr_split<64, true>(a, stream)
-                       : launch_dplr_split<64, false>(a, stream);
+  const int key = (a.dk == 128 ? 4 : 0) | (a.per_channel ? 2 : 0) | (a.bf16 ? 1 : 0);
+  switch (key) {
+    case 0: return launch_dplr_split<64, false, false>(a, stream);
+    case 1: return launch_dplr_split<64, false, true>(a, stream);
+    case 2: return launch_dplr_split<64, true, false>(a, stream);
+    case 3: return launch_dplr_split<64, true, true>(a, stream);
+    case 4: return launch_dplr_split<128, false, false>(a, stream);
+    case 5: return launch_dplr_split<128, false, true>(a, stream);
+    case 6: return launch_dplr_split<128, true, false>(a, stream);
+    default: return launch_dplr_split<128, true, true>(a, stream);
+  }
 }
 
 }  // namespace gdr
