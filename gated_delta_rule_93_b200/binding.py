@@ -407,9 +407,10 @@ def chunk_fwd_prologue(q, k, v, a, b, gate_scale, S0=None, *, norm_q=True, norm_
                        output_final_state=True, o=None, S_T=None, C=64, stream=None):
     """``gdr_chunk_fwd_prologue``: the chunked forward from raw projections.
 
-    q, k [B,T,H,dk] (raw, bf16); v [B,T,H,dv]; a, b [B,T,H] fp32 gate and
-    beta logits; gate_scale [H] fp32.  In the kernel: q, k L2-normalised (per
-    the flags), beta = sigmoid(b), g = -gate_scale[h] softplus(a).
+    q, k [B,T,H,dk] (raw; bf16 or fp32); v [B,T,H,dv]; a [B,T,H] (scalar
+    gate) or [B,T,H,dk] (per-channel gate) and b [B,T,H] fp32 gate and beta
+    logits; gate_scale [H] fp32.  In the kernel: q, k L2-normalised (per the
+    flags), beta = sigmoid(b), g = -gate_scale[h] softplus(a).
     Returns (o, S_T or None)."""
     _need(q, "q")
     dev = q.device
@@ -418,7 +419,12 @@ def chunk_fwd_prologue(q, k, v, a, b, gate_scale, S0=None, *, norm_q=True, norm_
     dt = q.dtype
     _need(k, "k", dt, (B, T, H, dk), dev)
     _need(v, "v", dt, (B, T, H, dv), dev)
-    _need(a, "a", torch.float32, (B, T, H), dev)
+    if a.dim() == 4:
+        _need(a, "a", torch.float32, (B, T, H, dk), dev)
+        gk = GDR_GATE_PER_CHANNEL
+    else:
+        _need(a, "a", torch.float32, (B, T, H), dev)
+        gk = GDR_GATE_SCALAR
     _need(b, "b", torch.float32, (B, T, H), dev)
     _need(gate_scale, "gate_scale", torch.float32, (H,), dev)
     if S0 is not None:
@@ -433,7 +439,7 @@ def chunk_fwd_prologue(q, k, v, a, b, gate_scale, S0=None, *, norm_q=True, norm_
     flags = (1 if norm_q else 0) | (2 if norm_k else 0)
     with torch.cuda.device(dev):
         rc = lib().gdr_chunk_fwd_prologue(_ptr(q), _ptr(k), _ptr(v), _in_dtype(dt), _ptr(a),
-                                          GDR_GATE_SCALAR, _ptr(gate_scale), _ptr(b), _ptr(S0),
+                                          gk, _ptr(gate_scale), _ptr(b), _ptr(S0),
                                           _ptr(o), _ptr(S_T), B, T, H, dk, dv, C, flags,
                                           _stream_handle(stream))
     _check(rc)

@@ -281,8 +281,6 @@ gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr
   gdr_status st = check_chunk(q, k, v, in_dtype, g, gate, beta, S0, o, S_T, 1, total_T, H, dk,
                               dv, C, &a);
   if (st != GDR_OK) return st;
-  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128)
-    return fail(GDR_ERR_UNSUPPORTED, "packed sequences need bf16 inputs and dk = dv = 128");
   if ((size_t)N * H == 0) return ok();
   if (!cu_seqlens) return fail(GDR_ERR_INVALID_ARG, "null cu_seqlens");
   if ((size_t)N * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "N*H too large");
@@ -299,7 +297,9 @@ gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr
   }
   a.B = N;
   a.cu_seqlens = cu_seqlens;
-  return from_cuda(gdr::launch_chunk_tc(a, s), "gdr_chunk_fwd_varlen launch");
+  return from_cuda(gdr::chunk_tc_supports(a) ? gdr::launch_chunk_tc(a, s)
+                                             : gdr::launch_chunk_split(a, s),
+                   "gdr_chunk_fwd_varlen launch");
 }
 
 gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
@@ -310,8 +310,6 @@ gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dt
   gdr_status st = check_chunk(q, k, v, in_dtype, g, gate, nullptr, S0, o, S_T, B, T, H, dk, dv,
                               C, &a, false);
   if (st != GDR_OK) return st;
-  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128)
-    return fail(GDR_ERR_UNSUPPORTED, "gated linear attention needs bf16 inputs and dk = dv = 128");
   if ((size_t)B * H == 0) return ok();
   if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "B*H too large");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -327,7 +325,9 @@ gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dt
   }
   a.beta = nullptr;
   a.additive = 1;
-  return from_cuda(gdr::launch_chunk_tc(a, s), "gdr_chunk_fwd_gla launch");
+  return from_cuda(gdr::chunk_tc_supports(a) ? gdr::launch_chunk_tc(a, s)
+                                             : gdr::launch_chunk_split(a, s),
+                   "gdr_chunk_fwd_gla launch");
 }
 
 gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
@@ -340,9 +340,6 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
                               &ca);
   if (st != GDR_OK) return st;
   if (norm_qk < 0 || norm_qk > 3) return fail(GDR_ERR_INVALID_ARG, "norm_qk must be 0..3");
-  if (in_dtype != GDR_BF16 || dk != 128 || dv != 128 || gate != GDR_GATE_SCALAR)
-    return fail(GDR_ERR_UNSUPPORTED,
-                "the fused prologue needs bf16 inputs, dk = dv = 128 and a scalar gate");
   if ((size_t)B * H == 0) return ok();
   if (!gate_scale) return fail(GDR_ERR_INVALID_ARG, "null gate_scale");
   if ((size_t)B * H > 0x7fffffffu) return fail(GDR_ERR_INVALID_ARG, "B*H too large");
@@ -360,9 +357,13 @@ gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
   ca.prologue = 1;
   ca.norm_qk = norm_qk;
   ca.gate_scale = gate_scale;
-  ca.skip_stage_chunk = t_skip_stage_chunk;
+  // the warp-specialised kernel takes bf16, d = 128 with a scalar gate; every
+  // other shape and per-channel gates run the split-operand kernel
+  const bool tc = gdr::chunk_tc_supports(ca) && gate == GDR_GATE_SCALAR;
+  ca.skip_stage_chunk = tc ? t_skip_stage_chunk : -1;
   t_skip_stage_chunk = -1;
-  return from_cuda(gdr::launch_chunk_tc(ca, s), "gdr_chunk_fwd_prologue launch");
+  return from_cuda(tc ? gdr::launch_chunk_tc(ca, s) : gdr::launch_chunk_split(ca, s),
+                   "gdr_chunk_fwd_prologue launch");
 }
 
 gdr_status gdr_dplr_fwd(const void *q, const void *k, const void *v, const void *a,

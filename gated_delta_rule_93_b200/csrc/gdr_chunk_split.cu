@@ -292,6 +292,58 @@ __device__ __forceinline__ void sync_for_mma() {
   tc_fence_after();
 }
 
+// Prologue maps (raw projections in): "Decoding Hybrid Linear Attention
+// Architectures", section 4 (beta in (0, 1), alpha in (0, 1], gates in log
+// space) and section 3 item 2 (the erase is a projector along a unit key):
+// beta = sigmoid(b), g = -s_h softplus(a), q, k <- x / sqrt(|x|^2 + eps).
+constexpr float kNormEps = 1e-6f;
+__device__ __forceinline__ float softplus_f(float x) {
+  return fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
+
+// beta of rows lane, lane + 32 (one warp); from logits when `logit`.
+__device__ __forceinline__ void load_beta(float *betav, const float *beta, size_t tok0, int H,
+                                          int L, int lane, bool logit) {
+  float b0 = lane < L ? beta[tok0 + (size_t)lane * H] : 0.f;
+  float b1 = lane + 32 < L ? beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
+  if (logit) {
+    b0 = lane < L ? sigmoid_f(b0) : 0.f;
+    b1 = lane + 32 < L ? sigmoid_f(b1) : 0.f;
+  }
+  betav[lane] = b0;
+  betav[lane + 32] = b1;
+}
+
+// 1 / sqrt(|x|^2 + eps) of row r of k (flags & 2) and q (flags & 1); this
+// thread holds the columns [hf DK/2, hf DK/2 + DK/2) and its partner
+// (thread ^ 1) the others, so the sums meet with one shuffle.  Every lane
+// of the warp calls this.
+template <bool BF, int DK>
+__device__ __forceinline__ void row_inv_norms(const void *k, const void *q, size_t tok0, int r,
+                                              int hf, int H, int dk, int L, int flags, float &rk,
+                                              float &rq) {
+  float sk = 0.f, sq = 0.f;
+#pragma unroll
+  for (int g8 = 0; g8 < DK / 16; ++g8) {
+    const int c0 = hf * (DK / 2) + 8 * g8;
+    const bool valid = r < L && c0 < dk;
+    const size_t off = in_off(tok0, r, c0, H, dk, valid);
+    float kx[8], qx[8];
+    ld8<BF>(k, off, kx);
+    ld8<BF>(q, off, qx);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      sk = fmaf(valid ? kx[e] : 0.f, valid ? kx[e] : 0.f, sk);
+      sq = fmaf(valid ? qx[e] : 0.f, valid ? qx[e] : 0.f, sq);
+    }
+  }
+  sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+  rk = (flags & 2) ? rsqrtf(sk + kNormEps) : 1.f;
+  rq = (flags & 1) ? rsqrtf(sq + kNormEps) : 1.f;
+}
+
 template <int DK, bool PC, bool BF>
 __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs a) {
   using LY = Layout<DK>;
@@ -302,7 +354,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, H = a.H;
   const int dk = a.dk, dv = a.dv;
-  const int n = (a.T + C - 1) / C;
+  // sequence b: token rows [seq0, seq0 + Tb) of the [B, T] (or packed [1, total]) layout
+  // (packed: cu_seqlens clamped into [0, total] and non-decreasing)
+  const int seq0 = a.cu_seqlens ? min(max(a.cu_seqlens[b], 0), a.T) : b * a.T;
+  const int Tb = a.cu_seqlens ? min(max(a.cu_seqlens[b + 1], seq0), a.T) - seq0 : a.T;
+  const int n = (Tb + C - 1) / C;
+  const bool add = a.additive != 0, pro = a.prologue != 0;
+  const float gsc = pro ? a.gate_scale[h] : 0.f;
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + LY::BAR);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + LY::MISC);
   float *vec = reinterpret_cast<float *>(sm + LY::VEC);
@@ -365,8 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
 
 #pragma unroll 1
   for (int c = 0; c < n && ok; ++c) {
-    const int t0 = c * C, L = min(C, a.T - t0);
-    const size_t tok0 = ((size_t)b * a.T + t0) * H + h;  // token index of row 0
+    const int t0 = c * C, L = min(C, Tb - t0);
+    const size_t tok0 = ((size_t)seq0 + t0) * H + h;  // token index of row 0
     // ---- gates
     if (PC) {
       if (t < DK) {
@@ -374,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
         float acc = 0.f, m = 0.f;
 #pragma unroll 8
         for (int r = 0; r < C; ++r) {
-          acc += (r < L && j < dk) ? a.g[(tok0 + (size_t)r * H) * dk + j] : 0.f;
+          const float x = (r < L && j < dk) ? a.g[(tok0 + (size_t)r * H) * dk + j] : 0.f;
+          acc += pro ? ((r < L && j < dk) ? -gsc * softplus_f(x) : 0.f) : x;
           gcm[r * DK + j] = acc;
           if (r == 31) m = acc;
         }
@@ -383,15 +442,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
         egl[j] = __expf(acc);
         glv[j] = acc;
       }
-      if (warp == 3) {
-        betav[lane] = lane < L ? a.beta[tok0 + (size_t)lane * H] : 0.f;
-        betav[lane + 32] = lane + 32 < L ? a.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
-      }
+      if (warp == 3 && !add) load_beta(betav, a.beta, tok0, H, L, lane, pro);
       if (t < 64) zf[t] = 1.f;
     } else {
       if (warp == 0) {
         float x0 = lane < L ? a.g[tok0 + (size_t)lane * H] : 0.f;
         float x1 = lane + 32 < L ? a.g[tok0 + (size_t)(lane + 32) * H] : 0.f;
+        if (pro) {  // logits -> g = -s_h softplus(a)
+          x0 = lane < L ? -gsc * softplus_f(x0) : 0.f;
+          x1 = lane + 32 < L ? -gsc * softplus_f(x1) : 0.f;
+        }
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
           const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
@@ -412,10 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
 #pragma unroll
         for (int e = 0; e < 4; ++e) egl[lane + 32 * e] = __expf(gl);
       }
-      if (warp == 1) {
-        betav[lane] = lane < L ? a.beta[tok0 + (size_t)lane * H] : 0.f;
-        betav[lane + 32] = lane + 32 < L ? a.beta[tok0 + (size_t)(lane + 32) * H] : 0.f;
-      }
+      if (warp == 1 && !add) load_beta(betav, a.beta, tok0, H, L, lane, pro);
     }
     __syncthreads();
     // ---- S' = S Diag(e^{m}) as hi / lo bf16 in TMEM
@@ -440,6 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     {
       const int r = t >> 1, hf = t & 1;
       bool range_bad = false;
+      float rk = 1.f, rq = 1.f;  // prologue: 1 / |k_r|, 1 / |q_r| (the pair t, t ^ 1 holds the row)
+      if (pro && a.norm_qk) row_inv_norms<BF, DK>(a.k, a.q, tok0, r, hf, H, dk, L, a.norm_qk, rk, rq);
 #pragma unroll
       for (int g8 = 0; g8 < DK / 16; ++g8) {
         const int c0 = hf * (DK / 2) + 8 * g8;
@@ -450,8 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
         ld8<BF>(a.q, off, qx);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          kx[e] = valid ? kx[e] : 0.f;
-          qx[e] = valid ? qx[e] : 0.f;
+          kx[e] = valid ? kx[e] * rk : 0.f;
+          qx[e] = valid ? qx[e] * rq : 0.f;
         }
         float kt[8], qt[8], kh[8], kb[8];
 #pragma unroll
@@ -512,6 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     // ---- A (fp32, over K^) and P (hi / lo tiles) from D1; U's right-hand
     //      side V^T - zf Z into TMEM; S <- S Diag(e^{gl})
     if (t < 64) {
+      if (!add) {
       const int r = t;
       const float br = betav[r], gr = gcs[r];
 #pragma unroll 1
@@ -529,6 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
           }
           Af4[r * 16 + ((8 * hp + e4) ^ (r & 15))] = make_float4(y[0], y[1], y[2], y[3]);
         }
+      }
       }
     } else {
       const int r = t - 64;
@@ -564,7 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
 #pragma unroll
       for (int r = 0; r < C; ++r) vr[r] = ld1<BF>(a.v, (tok0 + (size_t)(r < L ? r : 0) * H) * dv + ic);
 #pragma unroll
-      for (int r = 0; r < C; ++r) z[r] = ((r < L && i < dv) ? vr[r] : 0.f) - zf[r] * z[r];
+      for (int r = 0; r < C; ++r)
+        z[r] = ((r < L && i < dv) ? vr[r] : 0.f) - (add ? 0.f : zf[r] * z[r]);
       tmem_put_split64(lb + TC::ZO, z);
     }
 #pragma unroll 1
@@ -578,6 +640,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     tmem_wait_st();
     __syncthreads();
     // ---- T = (I + A)^{-1} Diag(beta): column c by forward substitution
+    //      (additive writes: T = I, U = V, none of this)
+    if (!add) {
     if (t < 64) {  // Y over the per-channel decays (read only before D1)
       const int cl = t;
       float *Y = gcm;
@@ -619,12 +683,14 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
       }
       tmem_put_split64(lb + TC::U, u);
     }
+    }  // !add
     sync_for_mma();
     // ---- O_b = U^T P^T (over D1) ;  S += U^T (K e^{gl - gc})
     if (t == 0) {
 #pragma unroll 1
       for (int kk = 0; kk < 4; ++kk) {
-        const uint32_t uh = tm + TC::U + 8 * kk, ul = tm + TC::U + 32 + 8 * kk;
+        const uint32_t ucol = add ? TC::ZO : TC::U;  // U^T (= V^T for additive writes)
+        const uint32_t uh = tm + ucol + 8 * kk, ul = tm + ucol + 32 + 8 * kk;
         const uint64_t ph_ = sdesc_sw128(s_pph + kk * 32, 16, 1024);
         const uint64_t kb_ = sdesc_sw128(s_kbh + kk * 32, 16, 1024);
         mma_ts(tm + TC::D1, uh, ph_, ID_64, kk > 0);
@@ -1194,9 +1260,8 @@ cudaError_t launch_dplr_split(const DplrChunkArgs &a, cudaStream_t stream) {
 bool chunk_split_supports(const ChunkArgs &a) {
   const bool dims = (a.dk == 32 || a.dk == 64 || a.dk == 128) &&
                     (a.dv == 32 || a.dv == 64 || a.dv == 128);
-  return dims && !a.cu_seqlens && !a.additive && !a.prologue && !a.stash_x && !a.stash_v &&
-         !a.stash_t && a.s0_seg == 0 && !a.s0_identity && !a.zero_v && a.write_o &&
-         a.skip_stage_chunk < 0;
+  return dims && !a.stash_x && !a.stash_v && !a.stash_t && a.s0_seg == 0 && !a.s0_identity &&
+         !a.zero_v && a.write_o && a.skip_stage_chunk < 0 && (!a.prologue || a.gate_scale);
 }
 
 cudaError_t launch_chunk_split(const ChunkArgs &a, cudaStream_t stream) {

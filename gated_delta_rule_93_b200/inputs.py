@@ -125,15 +125,16 @@ def make_dplr_inputs(B, T, H, d, dtype=torch.bfloat16, gate="scalar", with_S0=Fa
 
 
 def make_raw_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, with_S0=False, seed=0,
-                          gate_scale=None):
-    """Raw-projection inputs for ``gdr_chunk_fwd_prologue`` (scalar gate).
+                          gate_scale=None, gate="scalar"):
+    """Raw-projection inputs for ``gdr_chunk_fwd_prologue``.
 
     Returns dict of q, k [B,T,H,dk] ~ N(0,1) not normalised, v [B,T,H,dv], a
     (gate logits) and b (beta logits) [B,T,H] ~ N(0,1) fp32, gate_scale [H]
     fp32 (default 0.1 for every head) and S0 (or None).  Same draws, in the
     same order, as ``make_chunk_inputs`` with the same seed, before its
     normalisation and gate maps: with gate_scale 0.1 the prologue yields that
-    workload's distribution.
+    workload's distribution.  gate="channel": a is [B,T,H,dk] ~ N(0,1), drawn
+    from a stream of its own (the other draws unchanged).
     """
     gen = torch.Generator().manual_seed(seed)
     q = torch.randn(B, T, H, dk, generator=gen).to(dtype)
@@ -143,6 +144,8 @@ def make_raw_chunk_inputs(B, T, H, dk, dv, dtype=torch.bfloat16, with_S0=False, 
     b = torch.randn(B, T, H, generator=gen)
     S0 = 0.02 * torch.randn(B, H, dv, dk, generator=gen) if with_S0 else None
     gs = torch.full((H,), 0.1) if gate_scale is None else torch.as_tensor(gate_scale).float()
+    if gate == "channel":
+        a = torch.randn(B, T, H, dk, generator=torch.Generator().manual_seed(seed + 49979687))
     return dict(q=q, k=k, v=v, a=a.float(), b=b.float(), gate_scale=gs.float().contiguous(),
                 S0=S0)
 

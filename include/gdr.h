@@ -208,8 +208,8 @@ gdr_status gdr_chunk_fwd_segmented_noalloc(const void *q, const void *k, const v
  * gdr_chunk_fwd: each sequence runs the recurrence of "Decoding Hybrid
  * Linear Attention Architectures", sections 3 and 5, from its own S0.
  *
- *   q, k        [total_T, H, dk]  bf16     the sequences back to back
- *   v, o        [total_T, H, dv]  bf16
+ *   q, k        [total_T, H, dk]  in_dtype the sequences back to back
+ *   v, o        [total_T, H, dv]  in_dtype
  *   g           [total_T, H] fp32 (scalar gate) or [total_T, H, dk] (per
  *               channel); beta [total_T, H] fp32
  *   cu_seqlens  device int32 [N + 1]: sequence i is tokens
@@ -218,8 +218,9 @@ gdr_status gdr_chunk_fwd_segmented_noalloc(const void *q, const void *k, const v
  *   S0, S_T     [N, H, dv, dk] fp32 or NULL, as in gdr_chunk_fwd (S0 may
  *               alias S_T); an empty sequence gets S_T = S0 (or 0)
  *
- * S_T feeds gdr_step directly (same layout): prefill, then decode.  Needs
- * bf16 inputs and dk = dv = 128 (GDR_ERR_UNSUPPORTED otherwise).  One
+ * S_T feeds gdr_step directly (same layout): prefill, then decode.  Any
+ * shape gdr_chunk_fwd takes (bf16 with dk = dv = 128 on the
+ * warp-specialised kernel, the rest on the split-operand kernel).  One
  * launch; no workspace.
  */
 gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
@@ -239,14 +240,15 @@ gdr_status gdr_chunk_fwd_varlen(const void *q, const void *k, const void *v, gdr
  * erase term and no beta.  Computed chunkwise as gdr_chunk_fwd with the
  * correction W S dropped (T = I).
  *
- *   q, k   [B, T, H, dk] bf16;  v, o [B, T, H, dv] bf16
+ *   q, k   [B, T, H, dk] in_dtype;  v, o [B, T, H, dv] in_dtype
  *   g      [B, T, H] fp32 (scalar gate) or [B, T, H, dk] (per channel)
  *   S0     [B, H, dv, dk] fp32 or NULL (zero state); may alias S_T
  *   S_T    [B, H, dv, dk] fp32 or NULL (not written)
  *
- * Needs dk = dv = 128, C = 64 and bf16 inputs (GDR_ERR_UNSUPPORTED
- * otherwise).  T = 0 copies S0 (or zeros) to S_T.  One launch on `stream`,
- * no workspace; o must not alias an input.
+ * Any shape gdr_chunk_fwd takes, C = 64 (GDR_ERR_UNSUPPORTED otherwise):
+ * bf16 with dk = dv = 128 runs the warp-specialised kernel, the rest the
+ * split-operand kernel.  T = 0 copies S0 (or zeros) to S_T.  One launch on
+ * `stream`, no workspace; o must not alias an input.
  */
 gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dtype in_dtype,
                              const float *g, gdr_gate_kind gate, const float *S0, void *o,
@@ -270,16 +272,19 @@ gdr_status gdr_chunk_fwd_gla(const void *q, const void *k, const void *v, gdr_dt
  *
  * then the recurrence of gdr_chunk_fwd.
  *
- *   q, k        [B, T, H, dk] bf16   raw (not normalised) projections
- *   v, o        [B, T, H, dv] bf16
- *   a, b        [B, T, H] fp32       gate and write-strength logits
+ *   q, k        [B, T, H, dk] in_dtype  raw (not normalised) projections
+ *   v, o        [B, T, H, dv] in_dtype
+ *   a           [B, T, H] fp32 (scalar gate) or [B, T, H, dk] (per channel)
+ *               gate logits;  b [B, T, H] fp32 write-strength logits
  *   gate_scale  [H] fp32, > 0        per-head decay scale
  *   S0, S_T     as gdr_chunk_fwd
  *
- * Needs bf16 inputs, dk = dv = 128, C = 64 and gate = GDR_GATE_SCALAR
- * (GDR_ERR_UNSUPPORTED otherwise).  One launch, no workspace (long sequences
- * with few heads are not split into segments on this entry).  The inputs
- * are not modified.
+ * Any shape gdr_chunk_fwd takes, C = 64 (GDR_ERR_UNSUPPORTED otherwise):
+ * bf16 with dk = dv = 128 and a scalar gate runs the warp-specialised
+ * kernel; fp32 inputs, other head dims and per-channel gates (with the
+ * range limit of gdr_chunk_fwd) run the split-operand kernel.  One launch,
+ * no workspace (long sequences with few heads are not split into segments
+ * on this entry).  The inputs are not modified.
  */
 gdr_status gdr_chunk_fwd_prologue(const void *q, const void *k, const void *v,
                                   gdr_dtype in_dtype, const float *a, gdr_gate_kind gate,

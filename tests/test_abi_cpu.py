@@ -143,7 +143,7 @@ def test_binding_refuses_cpu_tensors(L):
 
 
 def test_varlen_validation_rejects_before_any_launch(L):
-    """gdr_chunk_fwd_varlen: packed sequences, tensor-core shapes only."""
+    """gdr_chunk_fwd_varlen: packed sequences, the shapes gdr_chunk_fwd takes."""
     p = _fake_ptr()
 
     def call(**kw):
@@ -156,8 +156,8 @@ def test_varlen_validation_rejects_before_any_launch(L):
 
     assert call(N=-1) == binding.GDR_ERR_INVALID_ARG
     assert call(cu=None) == binding.GDR_ERR_INVALID_ARG
-    assert call(dt=0) == binding.GDR_ERR_UNSUPPORTED
-    assert call(dk=64, dv=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dt=5) == binding.GDR_ERR_INVALID_ARG
+    assert call(dk=48, dv=64) == binding.GDR_ERR_UNSUPPORTED
     assert call(C=32) == binding.GDR_ERR_UNSUPPORTED
     assert call(q=None) == binding.GDR_ERR_INVALID_ARG
     assert call(o=_fake_ptr(2)) == binding.GDR_ERR_INVALID_ARG
@@ -165,7 +165,7 @@ def test_varlen_validation_rejects_before_any_launch(L):
 
 
 def test_gla_validation_rejects_before_any_launch(L):
-    """gdr_chunk_fwd_gla: no beta; tensor-core shapes only."""
+    """gdr_chunk_fwd_gla: no beta; the shapes gdr_chunk_fwd takes."""
     p = _fake_ptr()
 
     def call(**kw):
@@ -178,8 +178,8 @@ def test_gla_validation_rejects_before_any_launch(L):
 
     assert call(B=-1) == binding.GDR_ERR_INVALID_ARG
     assert call(gate=7) == binding.GDR_ERR_INVALID_ARG
-    assert call(dt=0) == binding.GDR_ERR_UNSUPPORTED
-    assert call(dk=64, dv=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dt=5) == binding.GDR_ERR_INVALID_ARG
+    assert call(dk=48, dv=64) == binding.GDR_ERR_UNSUPPORTED
     assert call(C=32) == binding.GDR_ERR_UNSUPPORTED
     assert call(q=None) == binding.GDR_ERR_INVALID_ARG
     assert call(g=None) == binding.GDR_ERR_INVALID_ARG
@@ -188,7 +188,7 @@ def test_gla_validation_rejects_before_any_launch(L):
 
 
 def test_prologue_validation_rejects_before_any_launch(L):
-    """gdr_chunk_fwd_prologue: raw projections; scalar gate, tensor-core shapes."""
+    """gdr_chunk_fwd_prologue: raw projections; the shapes gdr_chunk_fwd takes."""
     p = _fake_ptr()
 
     def call(**kw):
@@ -201,9 +201,9 @@ def test_prologue_validation_rejects_before_any_launch(L):
 
     assert call(B=-1) == binding.GDR_ERR_INVALID_ARG
     assert call(flags=4) == binding.GDR_ERR_INVALID_ARG
-    assert call(dt=0) == binding.GDR_ERR_UNSUPPORTED
-    assert call(gate=1) == binding.GDR_ERR_UNSUPPORTED
-    assert call(dk=64, dv=64) == binding.GDR_ERR_UNSUPPORTED
+    assert call(dt=5) == binding.GDR_ERR_INVALID_ARG
+    assert call(gate=7) == binding.GDR_ERR_INVALID_ARG
+    assert call(dk=48, dv=64) == binding.GDR_ERR_UNSUPPORTED
     assert call(C=32) == binding.GDR_ERR_UNSUPPORTED
     assert call(gs=None) == binding.GDR_ERR_INVALID_ARG
     assert call(b=None) == binding.GDR_ERR_INVALID_ARG

@@ -95,3 +95,17 @@ def test_gla_empty_sequence_copies_state(cuda_device):
     inp["S0"] = None
     _, S_T = _gpu(inp, cuda_device)
     assert torch.count_nonzero(S_T).item() == 0
+
+
+# the split-operand kernel: fp32 inputs (bar 1e-4) and other head dims
+@pytest.mark.parametrize("dk,dv,dtype,gate", [(64, 64, torch.float32, "scalar"),
+                                              (32, 128, torch.float32, "channel"),
+                                              (128, 64, torch.bfloat16, "channel")])
+def test_gla_split_operand_shapes(cuda_device, dk, dv, dtype, gate):
+    inp = make_chunk_inputs(2, 150, 3, dk, dv, dtype, gate, True, seed=75 + dk + dv)
+    o, S_T = _gpu(inp, cuda_device)
+    assert binding.device_status() == 0
+    ro, rS = _oracle(inp)
+    tol = 1e-4 if dtype == torch.float32 else TOL
+    assert_close(o, ro, tol, "o")
+    assert_close(S_T, rS, tol, "S_T")

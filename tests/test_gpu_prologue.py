@@ -34,9 +34,11 @@ def _gpu(inp, dev, **kw):
 
 def _oracle(inp, norm_q=True, norm_k=True):
     S0 = None if inp["S0"] is None else inp["S0"].double().numpy()
+    gate = "channel" if inp["a"].dim() == 4 else "scalar"
     return oracle.gdr_fwd_prologue(to_numpy_input(inp["q"]), to_numpy_input(inp["k"]),
                                    to_numpy_input(inp["v"]), inp["a"].numpy(), inp["b"].numpy(),
-                                   inp["gate_scale"].numpy(), S0, norm_q=norm_q, norm_k=norm_k)
+                                   inp["gate_scale"].numpy(), S0, gate=gate, norm_q=norm_q,
+                                   norm_k=norm_k)
 
 
 # several chunks + a ragged tail; one exact chunk; a single token
@@ -107,3 +109,30 @@ def test_prologue_skipped_load_times_out_and_reports(cuda_device):
     ro, rS = _oracle(inp)
     assert_close(o, ro, TOL, "o after recovery")
     assert binding.device_status() == binding.GDR_OK
+
+
+# the split-operand kernel: fp32 inputs (bar 1e-4), other head dims, and
+# per-channel gate logits (any dtype); several chunks and a ragged tail
+@pytest.mark.parametrize("dk,dv,dtype,gate", [(128, 128, torch.bfloat16, "channel"),
+                                              (64, 64, torch.float32, "scalar"),
+                                              (32, 64, torch.float32, "channel"),
+                                              (128, 32, torch.bfloat16, "scalar")])
+def test_prologue_split_operand_shapes(cuda_device, dk, dv, dtype, gate):
+    inp = make_raw_chunk_inputs(2, 150, 3, dk, dv, dtype, True, seed=98 + dk + dv,
+                                gate_scale=[0.05 + 0.1 * h for h in range(3)], gate=gate)
+    o, S_T = _gpu(inp, cuda_device)
+    assert binding.device_status() == 0
+    ro, rS = _oracle(inp)
+    tol = 1e-4 if dtype == torch.float32 else TOL
+    assert_close(o, ro, tol, "o")
+    assert_close(S_T, rS, tol, "S_T")
+
+
+def test_prologue_split_operand_flags(cuda_device):
+    """norm_q only, fp32 d = 64: the flags on the split-operand kernel."""
+    inp = make_raw_chunk_inputs(1, 100, 2, 64, 64, torch.float32, True, seed=99)
+    inp["k"] = inp["k"] * 0.12
+    o, S_T = _gpu(inp, cuda_device, norm_q=True, norm_k=False)
+    ro, rS = _oracle(inp, norm_q=True, norm_k=False)
+    assert_close(o, ro, 1e-4, "o")
+    assert_close(S_T, rS, 1e-4, "S_T")

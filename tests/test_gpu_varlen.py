@@ -107,7 +107,24 @@ def test_prefill_then_decode(cuda_device):
 
 
 def test_varlen_rejects_unsupported_shapes(cuda_device):
-    inp = make_varlen_inputs([10, 20], 2, 64, 64, torch.bfloat16, "scalar", False, seed=44)
+    inp = make_varlen_inputs([10, 20], 2, 48, 48, torch.bfloat16, "scalar", False, seed=44)
     with pytest.raises(binding.GdrError) as ei:
         _run(inp, cuda_device)
     assert ei.value.status == binding.GDR_ERR_UNSUPPORTED
+
+
+# the split-operand kernel: fp32 inputs (bar 1e-4) and other head dims
+@pytest.mark.parametrize("dk,dv,dtype,gate", [(64, 64, torch.float32, "scalar"),
+                                              (32, 64, torch.float32, "channel"),
+                                              (128, 64, torch.bfloat16, "scalar")])
+def test_varlen_split_operand_shapes(cuda_device, dk, dv, dtype, gate):
+    inp = make_varlen_inputs(LENS, 2, dk, dv, dtype, gate, True, seed=45 + dk + dv)
+    o, S_T = _run(inp, cuda_device)
+    assert binding.device_status() == 0
+    tol = 1e-4 if dtype == torch.float32 else 2e-2
+    cu = inp["cu_seqlens"].tolist()
+    for i, n in enumerate(LENS):
+        ro, rS = _oracle_seq(inp, i)
+        if n:
+            assert_close(o[cu[i]:cu[i + 1]].unsqueeze(0), ro, tol, f"o of sequence {i}")
+        assert_close(S_T[i:i + 1], rS, tol, f"S_T of sequence {i}")
