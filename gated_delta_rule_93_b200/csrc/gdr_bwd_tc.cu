@@ -71,6 +71,31 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
       : "memory");
 }
 
+// Bulk copies of contiguous bytes (sizes and addresses multiples of 16):
+// shared -> global with a bulk group (this thread waits for its reads of
+// shared memory, or for completion), and global -> shared completing on an
+// mbarrier's transaction count.
+__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(smem_u32(ssrc)), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_load(void *sdst, const void *gsrc, uint32_t bytes,
+                                          uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(sdst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 16-byte global -> shared copy through the asynchronous copy unit, the
 // commit of this thread's copies, and the wait for them.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -115,6 +140,7 @@ struct StateArgs {
   float *dS0;         // [B, H, D, D] or null
   __nv_bfloat16 *stash_ds;  // [B H n][D][D]: dS1 of every chunk (written)
   __nv_bfloat16 *stash_dv;  // [B H n][D][C]: dV'^T of every chunk (written)
+  uint8_t *stash_do;        // [B H n][16 KB]: dO of every chunk, bf16, as the swizzled tiles
   int B, T, H, n;
   unsigned int *status;
 };
@@ -249,7 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                        pack_bf16(v1.z, v1.w));
       }
     }
-    __syncthreads();  // gate vectors written
+    fence_proxy_async_smem();  // the dO tiles -> the bulk copy's reads
+    __syncthreads();           // gate vectors written
+    if (t == 0)  // the bf16 dO tiles of this chunk, for the gradient pass
+      bulk_store(a.stash_do + ((size_t)bh * n + ci) * 2 * kTile, sm + R_DO, 2 * kTile);
     if (ci >= 1) load_dout(ci - 1);
     {  // dS1 -> its bf16 copy (TMEM) and the stash; dS <- e^{gl} dS1
       const float bl = bv[63];
@@ -421,6 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_ts(tm + TR_DS, tm + TR_ZC + 8 * kk, sdesc_sw128(kq + kk * 2048, 2 * kTile, 1024),
                ID_ZK, 1);
       mma_commit(bar_mma);
+      bulk_wait_read();  // the dO tiles are rewritten by the next chunk (after this barrier)
     }
     ok = wait_all_threads(bar_mma, ph_mma, ok);
     ph_mma ^= 1;
@@ -438,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   cp_async_wait_all();
+  if (t == 0) bulk_wait_all();
   if (!ok && t == 0) {  // a load still in flight lands before the CTA ends
     atomicOr(a.status, kStatusTimeout);
     if (ld_n0) mbar_wait_bounded(bar_ld, (uint32_t)(ld_n0 - 1) & 1u, kWaitNs);
@@ -462,7 +493,7 @@ namespace {
 // ====================================================================== gradients
 struct GradArgs {
   const float *g, *beta;  // [B, T, H]
-  const float *dout;      // [B, T, H, D] fp32
+  const uint8_t *stash_do;  // [B H n][16 KB]: the state pass's bf16 dO tiles
   float *dq, *dk, *dv;    // [B, T, H, D] fp32 (written)
   float *dg, *dbeta;      // [B, T, H] fp32 (written)
   int B, T, H, n;
@@ -549,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- loads
   if (t == 0) {
-    mbar_arrive_expect_tx(bar_ld, 19 * kTile);  // K, Q, V, X0, dS1, V'^T, dV'^T, T
+    mbar_arrive_expect_tx(bar_ld, 21 * kTile);  // K, Q, V, X0, dS1, V'^T, dV'^T, T, dO
     tma_load_4d(sm + G_KQ + 0 * kTile, &tmK, bar_ld, 0, h, t0, b);
     tma_load_4d(sm + G_KQ + 1 * kTile, &tmQ, bar_ld, 0, h, t0, b);
     tma_load_4d(sm + G_KQ + 2 * kTile, &tmK, bar_ld, 64, h, t0, b);
@@ -568,6 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_load_3d(sm + G_DV + 0 * kTile, &tmDV, bar_ld, 0, 0, chunk);
     tma_load_3d(sm + G_DV + 1 * kTile, &tmDV, bar_ld, 0, 64, chunk);
     tma_load_3d(sm + G_T, &tmT, bar_ld, 0, 0, chunk);
+    // dO (bf16, already in the tiles' swizzled layout, from the state pass)
+    bulk_load(sm + G_DO, a.stash_do + (size_t)chunk * 2 * kTile, 2 * kTile, bar_ld);
   }
   if (warp == 0) {  // gates
     const size_t tok = ((size_t)b * a.T + t0 + lane) * H + h;
@@ -586,24 +619,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     betav[lane + 32] = b1;
     rbeta[lane] = b0 > 0.f ? 1.f / b0 : 0.f;
     rbeta[lane + 32] = b1 > 0.f ? 1.f / b1 : 0.f;
-  }
-  {  // dO rows -> bf16 tile: warp w takes rows w, w + 4, ...; lane l channels
-     // 4l .. 4l + 3 (each row one coalesced 512-byte read)
-    const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    uint8_t *tile = sm + G_DO + (lane >> 4) * kTile;
-    const int col = (4 * lane) & 63;
-    float4 v[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int r = warp + 4 * k;
-      v[k] = r < L ? reinterpret_cast<const float4 *>(
-                         a.dout + (((size_t)b * a.T + t0 + r) * H + h) * D)[lane]
-                   : z4;
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-      *reinterpret_cast<uint2 *>(tile + sw128_off(warp + 4 * k, col)) =
-          make_uint2(pack_bf16(v[k].x, v[k].y), pack_bf16(v[k].z, v[k].w));
   }
   ok = wait_all_threads(bar_ld, 0, ok);
   sync_for_mma();
@@ -960,10 +975,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 namespace gdr {
 
 // Per-chunk stash of the tensor-core backward, bytes: X0 [128][128], V'^T
-// [128][64], T [64][64], dS1 [128][128], dV'^T [128][64], all bf16.
+// [128][64], T [64][64], dS1 [128][128], dV'^T [128][64], dO [64][128], all
+// bf16 (dO as the two 128-byte-swizzled tiles the state pass converted).
 constexpr size_t kStashX = (size_t)D * D * 2, kStashV = (size_t)D * C * 2,
-                 kStashT = (size_t)C * C * 2;
-constexpr size_t kStashPerChunk = 2 * kStashX + 2 * kStashV + kStashT;
+                 kStashT = (size_t)C * C * 2, kStashO = (size_t)C * D * 2;
+constexpr size_t kStashPerChunk = 2 * kStashX + 2 * kStashV + kStashT + kStashO;
 
 bool bwd_tc_supports(int bf16, int per_channel, int d) {
   return bf16 && !per_channel && d == D;
@@ -988,6 +1004,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   __nv_bfloat16 *st = reinterpret_cast<__nv_bfloat16 *>(w + nch * (kStashX + kStashV));
   __nv_bfloat16 *sds = reinterpret_cast<__nv_bfloat16 *>(w + nch * (kStashX + kStashV + kStashT));
   __nv_bfloat16 *sdv = reinterpret_cast<__nv_bfloat16 *>(w + nch * (2 * kStashX + kStashV + kStashT));
+  uint8_t *sdo = w + nch * (2 * kStashX + 2 * kStashV + kStashT);
   // 1. the forward again, stashing X0, V'^T and T per chunk (no o)
   ChunkArgs fa{};
   fa.q = q; fa.k = k; fa.v = v; fa.g = g; fa.beta = beta; fa.S0 = S0;
@@ -1008,7 +1025,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   e = cudaFuncSetAttribute(gdr_bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kStateSmem);
   if (e != cudaSuccess) return e;
-  StateArgs ra{g, dout, dST, dS0, sds, sdv, B, T, H, (int)n, status};
+  StateArgs ra{g, dout, dST, dS0, sds, sdv, sdo, B, T, H, (int)n, status};
   gdr_bwd_state_kernel<<<(unsigned)(B * H), kThreads, kStateSmem, stream>>>(mk, mq, mt, ra);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1016,7 +1033,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
   e = cudaFuncSetAttribute(gdr_bwd_grad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kGradSmem);
   if (e != cudaSuccess) return e;
-  GradArgs ga{g, beta, dout, dq, dk, dv, dg, dbeta, B, T, H, (int)n};
+  GradArgs ga{g, beta, sdo, dq, dk, dv, dg, dbeta, B, T, H, (int)n};
   gdr_bwd_grad_kernel<<<(unsigned)nch, kThreads, kGradSmem, stream>>>(mq, mk, mv, mx, mds, mvp,
                                                                       mdv, mt, ga);
   return cudaGetLastError();

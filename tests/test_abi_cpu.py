@@ -219,7 +219,7 @@ def test_backward_validation_rejects_before_any_launch(L):
     assert ws == 2 * 2 * (38 + 1 + 8) * 128 * 128 * 4
     assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128, 1, 1) == ws
     # tensor cores (bf16, d = 128, scalar gate): 104 KB of bf16 stash per chunk and head
-    assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128, 1, 0) == 2 * 2 * 5 * 106496
+    assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 128, 1, 0) == 2 * 2 * 5 * 122880
     assert L.gdr_chunk_bwd_workspace_bytes(2, 300, 2, 128, 64, 1, 0) == 0
 
     def call(**kw):
