@@ -1261,6 +1261,7 @@ bool chunk_split_supports(const ChunkArgs &a) {
   const bool dims = (a.dk == 32 || a.dk == 64 || a.dk == 128) &&
                     (a.dv == 32 || a.dv == 64 || a.dv == 128);
   return dims && !a.stash_x && !a.stash_v && !a.stash_t && a.s0_seg == 0 && !a.s0_identity &&
+         a.seg_n == 0 &&
          !a.zero_v && a.write_o && a.skip_stage_chunk < 0 && (!a.prologue || a.gate_scale);
 }
 

@@ -877,6 +877,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tb = s0;
     bt = 0;
     T = s1 - s0;
+  } else if (a.seg_n > 0) {  // segment b % seg_n of sequence b / seg_n, whole chunks
+    const int b0 = b / a.seg_n, p = b % a.seg_n, nc = (a.seg_T + C - 1) / C;
+    const int c0 = (int)((long long)p * nc / a.seg_n);
+    const int c1 = (int)((long long)(p + 1) * nc / a.seg_n);
+    tb = b0 * a.seg_T + c0 * C;
+    bt = 0;
+    T = min(c1 * C, a.seg_T) - c0 * C;
   }
   const int n = (T + C - 1) / C;
 
@@ -1791,7 +1798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         const int rows = T - c * C;  // valid rows of the chunk
-        if (a.cu_seqlens && rows < C) {
+        if ((a.cu_seqlens || a.seg_n > 0) && rows < C) {
           // The last chunk of a packed sequence: the TMA box would run into
           // the next sequence's rows, so the valid rows go out with plain
           // 16-byte stores (chunk j of staging row r sits at j ^ ((r / 2) % 4)).
@@ -1948,7 +1955,7 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream) {
   // Without an output (segment passes) the output map is never used; it is
   // built over q so that it is a valid map.
   // (packed sequences: the tensors are [1, total, H, d]; one CTA per sequence and head)
-  const int mb = a.cu_seqlens ? 1 : a.B;
+  const int mb = (a.cu_seqlens || a.seg_n > 0) ? 1 : a.B;
   if (!make_map(&mq, a.q, mb, a.T, a.H, DK) || !make_map(&mk, a.k, mb, a.T, a.H, DK) ||
       !make_map(&mv, a.v, mb, a.T, a.H, DV) ||
       !make_map_out(&mo, a.write_o ? a.o : const_cast<void *>(a.q), mb, a.T, a.H, DV))

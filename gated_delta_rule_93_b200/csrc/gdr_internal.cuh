@@ -35,6 +35,12 @@ struct ChunkArgs {
   int s0_identity;  // 1: sequences without an S0 start from the identity (d_v == d_k)
   int zero_v;       // 1: v is taken as zero (not read): the end state is the transition
   int write_o;      // 0: o is not written (may be null)
+  // Segment passes with uneven segments (tensor-core kernel only; 0: off):
+  // the tensors are read as packed rows [1, total, H, d], and sequence
+  // b is segment b % seg_n of original sequence b / seg_n (seg_T tokens),
+  // chunks split as evenly as whole chunks allow; a.T is then the packed
+  // total and a.B the number of segments.
+  int seg_n, seg_T;
   // Packed sequences (tensor-core kernel only): B sequences, sequence b is
   // tokens [cu_seqlens[b], cu_seqlens[b + 1]) of the [1, T, H, d] tensors
   // (device int32 [B + 1]); null: dense [B, T, H, d].

@@ -16,8 +16,9 @@
 //   combine: S_start(1) = end of segment 0, S_start(p + 1) = S_start(p) M_p +
 //            E_p, in fp32; the last product is the final state S_T;
 //   pass 2:  every segment from its true start state: the output o.
-// The passes reuse the kernel on the same tensors: [B, T, H, d] is
-// [B * P, T / P, H, d] with segment p of sequence b as sequence b * P + p.
+// The passes reuse the kernel on the same tensors, read as packed rows: segment
+// p of sequence b is unit b * P + p, chunks [p nc / P, (p + 1) nc / P) of the
+// sequence's nc chunks (so P need not divide them).
 #include "gdr_internal.cuh"
 
 namespace gdr {
@@ -126,13 +127,13 @@ int chunk_segments(const ChunkArgs &a, int num_sms) {
   if (!chunk_tc_supports(a) || a.dk != kDim || a.dv != kDim || a.skip_stage_chunk >= 0)
     return 1;
   const long long bh = (long long)a.B * a.H;
-  if (bh <= 0 || num_sms <= 0) return 1;
-  // Largest power of two P with B * H * P CTAs in one wave, segments of whole
-  // chunks, at least 16 chunks each; three passes pay off only from P = 4.
+  if (bh <= 0 || num_sms <= 0 || (long long)a.B * a.T > 0x7fffffffLL) return 1;
+  // Largest P with B * H * P CTAs in one wave and at least 16 chunks per
+  // segment (segments of whole chunks, as even as that allows); three passes
+  // pay off only from P = 4.
+  const long long nc = ((long long)a.T + 63) / 64;
   int P = 1;
-  while (P < 64 && bh * 2 * P <= num_sms && a.T % (64 * 2 * P) == 0 &&
-         a.T / (64 * 2 * P) >= 16)
-    P *= 2;
+  while (P < 64 && bh * (P + 1) <= num_sms && nc / (P + 1) >= 16) ++P;
   return P >= 4 ? P : 1;
 }
 
@@ -156,9 +157,14 @@ cudaError_t launch_chunk_segments(const ChunkArgs &a, int P, void *ws, cudaStrea
   }
   const size_t n_state = (size_t)a.B * P * a.H * a.dv * a.dk;
   float *X = static_cast<float *>(ws), *Ea = X + n_state, *Eb = Ea + n_state;
+  if ((long long)a.B * a.T > 0x7fffffffLL || P < 1) return cudaErrorInvalidValue;
+  // the passes read the [B, T] tensors as packed rows, segment p of
+  // sequence b being unit b * P + p (whole chunks, as even as they go)
   ChunkArgs s = a;
   s.B = a.B * P;
-  s.T = a.T / P;
+  s.T = a.B * a.T;
+  s.seg_n = P;
+  s.seg_T = a.T;
   // pass 1a: zero start (the first segment of a sequence from S0), end states
   s.S0 = a.S0;
   s.s0_seg = P;
