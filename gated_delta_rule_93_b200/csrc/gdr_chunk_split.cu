@@ -54,7 +54,8 @@ using namespace sm100;
 using namespace tcu;
 
 constexpr int C = 64;
-constexpr int kThreads = 128;
+constexpr int kThreads = 128;   // the delta-rule split kernel
+constexpr int kThreadsD = 256;  // the DPLR kernel
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kMaxExp = 100.f * kLn2;  // largest |gc - m| of a scaled factor
@@ -276,6 +277,21 @@ __device__ __forceinline__ void tmem_put_split64(uint32_t taddr, const float (&x
     tmem_st16u(taddr + 16 * half, hu);
     tmem_st16u(taddr + 32 + 16 * half, lu);
   }
+}
+
+// 32 fp32 values as hi / lo bf16 pairs: 16 TMEM columns each at th and tl.
+__device__ __forceinline__ void tmem_put_split32(uint32_t th, uint32_t tl, const float (&x)[32]) {
+  uint32_t hu[16], lu[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    float h0, l0, h1, l1;
+    split_bf16(x[2 * e], h0, l0);
+    split_bf16(x[2 * e + 1], h1, l1);
+    hu[e] = pack_bf16(h0, h1);
+    lu[e] = pack_bf16(l0, l1);
+  }
+  tmem_st16u(th, hu);
+  tmem_st16u(tl, lu);
 }
 
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t parity, bool ok) {
@@ -799,7 +815,7 @@ struct DLayout {
 };
 
 template <int DK, bool PC, bool BF>
-__global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkArgs p) {
+__global__ void __launch_bounds__(kThreadsD, 1) gdr_dplr_split_kernel(DplrChunkArgs p) {
   using LY = DLayout<DK>;
   // TMEM: S [DK], S' hi / lo [DK/2 each], D1 [128] (then W / X in its first
   // 64 columns and V^T hi | lo in the last 64), ZO [128] (Z_a, then U's
@@ -809,7 +825,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~uintptr_t(1023));
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // 8 warps: warp w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (value
+  // channels) and split that lane quarter's columns or rows between them (hs)
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, lq = warp & 3, hs = warp >> 2;
   const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H, H = p.H;
   const int dk = p.dk, dv = p.dv;
   const int n = (p.T + C - 1) / C;
@@ -834,11 +852,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
-  const uint32_t lb = tm + ((uint32_t)(warp * 32) << 16);
-  const int i = t;
+  const uint32_t lb = tm + ((uint32_t)(lq * 32) << 16);
+  const int i = lq * 32 + lane;  // value channel (TMEM lane)
 
 #pragma unroll 1
-  for (int q = 0; q < DK / 32; ++q) {
+  for (int q = hs; q < DK / 32; q += 2) {
     float x[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
@@ -927,7 +945,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     __syncthreads();
     // ---- S' = S Diag(e^{m}) as hi / lo bf16 in TMEM
 #pragma unroll 1
-    for (int q = 0; q < DK / 32; ++q) {
+    for (int q = hs; q < DK / 32; q += 2) {
       float x[32];
       tmem_ld32(lb + TS + 32 * q, x);
       uint32_t hu[16], lu[16];
@@ -943,13 +961,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
       tmem_st16u(lb + TSH + 16 * q, hu);
       tmem_st16u(lb + TSL + 16 * q, lu);
     }
-    // ---- [A^; Q~] and [B^; K^] tiles: row r = t / 2, half t % 2 of the columns
+    // ---- [A^; Q~] and [B^; K^] tiles: row r = t / 4, quarter t % 4 of the columns
     {
-      const int r = t >> 1, hf = t & 1;
+      const int r = t >> 2, hf = t & 3;
       bool range_bad = false;
 #pragma unroll
-      for (int g8 = 0; g8 < DK / 16; ++g8) {
-        const int c0 = hf * (DK / 2) + 8 * g8;
+      for (int g8 = 0; g8 < DK / 32; ++g8) {
+        const int c0 = hf * (DK / 4) + 8 * g8;
         const bool valid = r < L && c0 < dk;
         const size_t off = in_off(tok0, r, c0, H, dk, valid);
         float ax[8], qx[8], bx[8], kx[8];
@@ -1008,11 +1026,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     mma_wait();
     if (!ok) break;
     // ---- from D1: Lb (fp32), Lk, P_b, P_k (hi / lo tiles)
-    if (t < 64) {
-      const int r = t;
+    if (lq < 2) {  // rows 0-63: Lb (hs = 0) and Lk (hs = 1)
+      const int r = i;
       const float gr = r > 0 ? gcs[r - 1] : 0.f;
 #pragma unroll 1
-      for (int hp = 0; hp < 4; ++hp) {  // D1 columns 32 hp .. 32 hp + 31
+      for (int hp = 2 * hs; hp < 2 * hs + 2; ++hp) {  // D1 columns 32 hp .. 32 hp + 31
         float x[32];
         tmem_ld32(lb + TD1 + 32 * hp, x);
         float hi[32], lo[32];
@@ -1033,11 +1051,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
           st_row32(sm + LY::LK_LO, r, hp & 1, lo);
         }
       }
-    } else {
-      const int r = t - 64;
+    } else {  // rows 64-127: P_b (hs = 0) and P_k (hs = 1)
+      const int r = i - 64;
       const float gr = gcs[r];
 #pragma unroll 1
-      for (int hp = 0; hp < 4; ++hp) {
+      for (int hp = 2 * hs; hp < 2 * hs + 2; ++hp) {
         float x[32], hi[32], lo[32];
         tmem_ld32(lb + TD1 + 32 * hp, x);
 #pragma unroll
@@ -1050,20 +1068,24 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
         st_row32(sm + (hp < 2 ? LY::PB_LO : LY::PK_LO), r, hp & 1, lo);
       }
     }
-    {  // V^T (lane = value channel) as hi | lo into D1 columns 64-127
-      float vt[64];
+    __syncthreads();  // every lane's D1 columns 64-127 read before V^T goes there
+    {  // V^T (lane = value channel) as hi | lo into D1 columns 64-127; rows 32 hs ..
+      float vt[32];
       const int ic = i < dv ? i : 0;
 #pragma unroll
-      for (int r = 0; r < C; ++r) vt[r] = ld1<BF>(p.v, (tok0 + (size_t)(r < L ? r : 0) * H) * dv + ic);
+      for (int e = 0; e < 32; ++e) {
+        const int r = 32 * hs + e;
+        vt[e] = ld1<BF>(p.v, (tok0 + (size_t)(r < L ? r : 0) * H) * dv + ic);
+      }
 #pragma unroll
-      for (int r = 0; r < C; ++r) vt[r] = (r < L && i < dv) ? vt[r] : 0.f;
-      tmem_put_split64(lb + TD1 + 64, vt);
+      for (int e = 0; e < 32; ++e) vt[e] = (32 * hs + e < L && i < dv) ? vt[e] : 0.f;
+      tmem_put_split32(lb + TD1 + 64 + 16 * hs, lb + TD1 + 96 + 16 * hs, vt);
     }
     {  // (B e^{gl - gc})^T and (K e^{gl - gc})^T over [B^; K^] (dead after D1)
-      const int r = t >> 1, hf = t & 1;
+      const int r = t >> 2, hf = t & 3;
 #pragma unroll
-      for (int g8 = 0; g8 < DK / 16; ++g8) {
-        const int c0 = hf * (DK / 2) + 8 * g8;
+      for (int g8 = 0; g8 < DK / 32; ++g8) {
+        const int c0 = hf * (DK / 4) + 8 * g8;
         const bool valid = r < L && c0 < dk;
         const size_t off = in_off(tok0, r, c0, H, dk, valid);
         float bx[8], kx[8];
@@ -1103,31 +1125,17 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     mma_wait();
     if (!ok) break;
     // ---- R = zfa Z_a + W -> hi | lo over Z_a;  S <- S Diag(e^{gl})
-    {
-      float z[64], w[64];
-      {
-        float z0[32], z1[32];
-        tmem_ld32(lb + TZO, z0);
-        tmem_ld32(lb + TZO + 32, z1);
+    {  // rows 32 hs .. 32 hs + 31 of this lane; all reads before any write
+      float z[32], w[32];
+      tmem_ld32(lb + TZO + 32 * hs, z);
+      tmem_ld32(lb + TD1 + 32 * hs, w);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          z[e] = z0[e];
-          z[32 + e] = z1[e];
-        }
-        tmem_ld32(lb + TD1, z0);
-        tmem_ld32(lb + TD1 + 32, z1);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          w[e] = z0[e];
-          w[32 + e] = z1[e];
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < C; ++r) z[r] = zfa[r] * z[r] + w[r];
-      tmem_put_split64(lb + TZO, z);
+      for (int e = 0; e < 32; ++e) z[e] = zfa[32 * hs + e] * z[e] + w[e];
+      __syncthreads();
+      tmem_put_split32(lb + TZO + 16 * hs, lb + TZO + 32 + 16 * hs, z);
     }
 #pragma unroll 1
-    for (int q = 0; q < DK / 32; ++q) {
+    for (int q = hs; q < DK / 32; q += 2) {
       float x[32];
       tmem_ld32(lb + TS + 32 * q, x);
 #pragma unroll
@@ -1162,19 +1170,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     }
     mma_wait();
     if (!ok) break;
-    {
-      float x[64];
-      {
-        float x0[32], x1[32];
-        tmem_ld32(lb + TD1, x0);
-        tmem_ld32(lb + TD1 + 32, x1);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          x[e] = x0[e];
-          x[32 + e] = x1[e];
-        }
-      }
-      tmem_put_split64(lb + TD1, x);
+    {  // rows 32 hs .. 32 hs + 31 of this lane; all reads before any write
+      float x[32];
+      tmem_ld32(lb + TD1 + 32 * hs, x);
+      __syncthreads();
+      tmem_put_split32(lb + TD1 + 16 * hs, lb + TD1 + 32 + 16 * hs, x);
     }
     sync_for_mma();
     // ---- O_b = X^T P_b^T + V^T P_k^T (over ZO columns 0-63);
@@ -1204,9 +1204,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
     }
     mma_wait();
     if (!ok) break;
-    // ---- o_r = zfo_r O_a + O_b
-#pragma unroll 1
-    for (int hp = 0; hp < 2; ++hp) {
+    // ---- o_r = zfo_r O_a + O_b (rows 32 hs .. 32 hs + 31)
+    {
+      const int hp = hs;
       float oa[32], ob[32];
       tmem_ld32(lb + TZO + 64 + 32 * hp, oa);
       tmem_ld32(lb + TZO + 32 * hp, ob);
@@ -1222,7 +1222,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_dplr_split_kernel(DplrChunkAr
   }
   if (ok && p.S_T) {
 #pragma unroll 1
-    for (int q = 0; q < DK / 32; ++q) {
+    for (int q = hs; q < DK / 32; q += 2) {
       float x[32];
       tmem_ld32(lb + TS + 32 * q, x);
       if (i < dv) {
@@ -1251,7 +1251,7 @@ cudaError_t launch_dplr_split(const DplrChunkArgs &a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)DLayout<DK>::bytes);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(a.B * a.H), kThreads, DLayout<DK>::bytes, stream>>>(a);
+  kern<<<(unsigned)(a.B * a.H), kThreadsD, DLayout<DK>::bytes, stream>>>(a);
   return cudaGetLastError();
 }
 
