@@ -46,7 +46,8 @@ using namespace sm100;
 using namespace tcu;
 
 constexpr int C = 64, D = 128;
-constexpr int kThreads = 128;
+constexpr int kThreads = 128;      // the reverse state pass
+constexpr int kGradThreads = 256;  // the gradient pass
 constexpr uint32_t kTile = 8192;             // one 64 x 64 bf16 tile (128-byte swizzle)
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
@@ -507,7 +508,7 @@ struct GradArgs {
 constexpr uint32_t G_KQ = 0, G_V = 4 * kTile, G_DWT = 6 * kTile, G_X = 8 * kTile,
                    G_DS = 12 * kTile, G_VP = 16 * kTile, G_DV = 18 * kTile, G_T = 20 * kTile,
                    G_DO = 21 * kTile, G_Y = 23 * kTile, G_DYT = 24 * kTile, G_DPS = 25 * kTile,
-                   G_DMS = 26 * kTile, G_VEC = 27 * kTile, G_BAR = G_VEC + 2048,
+                   G_DMS = 26 * kTile, G_VEC = 27 * kTile, G_BAR = G_VEC + 4096,
                    G_MISC = G_BAR + 64, G_END = G_MISC + 64;
 constexpr size_t kGradSmem = G_END + 1024;
 static_assert(kGradSmem <= 232448, "shared memory budget");
@@ -515,7 +516,7 @@ static_assert(kGradSmem <= 232448, "shared memory budget");
 constexpr uint32_t TG0 = 0, TG1 = 64, TG2 = 128, TG3 = 192, TG4 = 256, TG5 = 320, TG6 = 384,
                    TG7 = 448;
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kGradThreads, 1)
     gdr_bwd_grad_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
@@ -527,7 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~uintptr_t(1023));
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // 8 warps: warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 and
+  // split each per-lane phase's columns between them (hs)
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, lq = warp & 3, hs = warp >> 2;
   const int ci = blockIdx.x % a.n, bh = blockIdx.x / a.n, b = bh / a.H, h = bh % a.H;
   const int H = a.H, t0 = ci * C, L = min(C, a.T - t0);
   const int chunk = bh * a.n + ci;
@@ -537,9 +540,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *bv = gcv + 64;                                 // e^{gc}
   float *kbv = gcv + 128;                               // e^{gl - gc}
   float *betav = gcv + 192;                             // beta
-  float *dbeta1 = gcv + 256;                            // column sums of dT . Y
-  float *red = gcv + 320;                               // [4] block reduction
-  float *rbeta = gcv + 448;                             // 1 / beta (0 where beta = 0)
+  float *rbeta = gcv + 256;                             // 1 / beta (0 where beta = 0)
+  float *dbeta1 = gcv + 320;                            // [2][64] column sums of dT . Y
+  float *dbeta2s = gcv + 448;                           // [2][64] sums of dA M
+  float *red = gcv + 576;                               // [8] block reduction
+  float *scan = gcv + 640;                              // [64] scan scratch
+  float *psum = gcv + 704;                              // [4][64] gate partial sums
   if (t == 0) {
     mbar_init(bar_ld, 1);
     mbar_init(bar_mma, 1);
@@ -553,7 +559,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
-  const uint32_t lb = tm + ((uint32_t)(warp * 32) << 16);
+  const uint32_t lb = tm + ((uint32_t)(lq * 32) << 16);
+  const int i = lq * 32 + lane;  // this thread's TMEM lane
   const uint32_t s_kq = smem_u32(sm + G_KQ), s_v = smem_u32(sm + G_V), s_x = smem_u32(sm + G_X);
   const uint32_t s_ds = smem_u32(sm + G_DS), s_vp = smem_u32(sm + G_VP);
   const uint32_t s_dv = smem_u32(sm + G_DV), s_t = smem_u32(sm + G_T), s_do = smem_u32(sm + G_DO);
@@ -654,40 +661,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // dv (lanes = value channels); dW^T -> bf16 (TMEM in place, and the smem
     // tile [j][r]); Y = T Diag(1 / beta) (rows r < 64)
-    const int i = t;
-    {
-      float x0[32], x1[32];
-      tmem_ld32(lb + TG0, x0);
-      tmem_ld32(lb + TG0 + 32, x1);
+    {  // tokens 32 hs .. 32 hs + 31
+      float x0[32];
+      tmem_ld32(lb + TG0 + 32 * hs, x0);
       float *dst = a.dv + row0 * D + i;
       const size_t rs = (size_t)H * D;
 #pragma unroll
       for (int r = 0; r < 32; ++r)
-        if (r < L) dst[r * rs] = x0[r];
-#pragma unroll
-      for (int r = 0; r < 32; ++r)
-        if (r + 32 < L) dst[(r + 32) * rs] = x1[r];
+        if (32 * hs + r < L) dst[(32 * hs + r) * rs] = x0[r];
     }
-    {
-      float x0[32], x1[32];
-      tmem_ld32(lb + TG2, x0);
-      tmem_ld32(lb + TG2 + 32, x1);
+    {  // columns 32 hs ..: all reads of the fp32 dW^T before its bf16 copy overwrites it
+      float x0[32];
+      tmem_ld32(lb + TG2 + 32 * hs, x0);
       uint32_t u[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x0[2 * e], x0[2 * e + 1]);
-      tmem_st16u(lb + TG2, u);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x1[2 * e], x1[2 * e + 1]);
-      tmem_st16u(lb + TG2 + 16, u);
-      uint8_t *tile = sm + G_DWT + (i >> 6) * kTile;
-      st_row32(tile, i & 63, 0, x0);
-      st_row32(tile, i & 63, 1, x1);
+      __syncthreads();
+      tmem_st16u(lb + TG2 + 16 * hs, u);
+      st_row32(sm + G_DWT + (i >> 6) * kTile, i & 63, hs, x0);
     }
-    if (t < 64) {  // row r of Y from row r of T
-      const int r = t;
+    if (t < 128) {  // row r of Y from row r of T, half t / 64 of the columns
+      const int r = t & 63;
       float y[32];
-#pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
+      {
+        const int hp = t >> 6;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           const uint4 v = *reinterpret_cast<const uint4 *>(sm + G_T + sw128_off(r, 32 * hp + 8 * ch));
@@ -718,13 +715,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     // dT^T [s][r] = dT^T_1 + e^{gc_s} dT^T_2 (rows s < 64): dbeta_s (part 1) =
     // sum_r dT[r][s] Y[r][s]; dY^T [s][r] = beta_s dT^T[s][r]
-    if (t < 64) {
-      const int s = t;
+    if (lq < 2) {  // rows s = lanes 0-63, columns 32 hs ..
+      const int s = i;
       float x[32], y2[32];
       float acc = 0.f;
       const float bs = bv[s], bes = betav[s];
-#pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
+      {
+        const int hp = hs;
         tmem_ld32(lb + TG1 + 32 * hp, x);
         tmem_ld32(lb + TG3 + 32 * hp, y2);
 #pragma unroll
@@ -737,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         st_row32(sm + G_DYT, s, hp, x);
       }
-      dbeta1[s] = acc;
+      dbeta1[64 * hs + s] = acc;
     }
     sync_for_mma();
     // ---- G5: E = Y^T dY [s][q]
@@ -750,17 +747,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mma_wait();
   }
   if (ok) {
-    {  // E -> bf16 in place (A of G6)
-      float x0[32], x1[32];
-      tmem_ld32(lb + TG1, x0);
-      tmem_ld32(lb + TG1 + 32, x1);
+    {  // E -> bf16 in place (A of G6): columns 32 hs .., all reads before the writes
+      float x0[32];
+      tmem_ld32(lb + TG1 + 32 * hs, x0);
       uint32_t u[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x0[2 * e], x0[2 * e + 1]);
-      tmem_st16u(lb + TG1, u);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x1[2 * e], x1[2 * e + 1]);
-      tmem_st16u(lb + TG1 + 16, u);
+      __syncthreads();
+      tmem_st16u(lb + TG1 + 16 * hs, u);
     }
     sync_for_mma();
     // ---- G6: F = E Y^T [s][p];  G8a: dP = dO V'^T [r][s]
@@ -782,12 +776,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // rows s < 64: dA = strict_tril(-F); dbeta_s (part 2) = sum_p dA M, M =
     // KK e^{gc_s - gc_p}; dMs[s][p] = beta_s dA[s][p] e^{gc_s - gc_p};
     // dPs[r][s] = tril(dP)[r][s] e^{gc_r - gc_s}
-    if (t < 64) {
-      const int r = t;
+    if (lq < 2) {  // rows r = lanes 0-63, columns 32 hs ..
+      const int r = i;
       const float gr = gcv[r], br = betav[r];
       float f[32], kk2[32], p[32];
-#pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
+      {
+        const int hp = hs;
         tmem_ld32(lb + TG3 + 32 * hp, f);
         tmem_ld32(lb + TG4 + 32 * hp, kk2);
         tmem_ld32(lb + TG5 + 32 * hp, p);
@@ -803,19 +797,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_row32(sm + G_DMS, r, hp, f);
         st_row32(sm + G_DPS, r, hp, p);
       }
+      dbeta2s[64 * hs + r] = dbeta2;
     }
     // dO -> dO~ = Diag(e^{gc}) dO; V'^T columns scaled by e^{gl - gc};
     // T -> T~ = T Diag(e^{gc}) (all in place; their unscaled uses are done)
     {
-      const int r = t >> 1, hh = t & 1;
-      const float fb = bv[r];
+      // dO~: 64 rows x 2 tiles x 8 chunks, four 16-byte chunks per thread
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) scale_chunk(sm + G_DO + hh * kTile + sw128_off(r, 8 * ch), fb);
-      // V'^T: rows i (128), columns r: thread t handles row t, 64 columns
-      uint8_t *vp = sm + G_VP + (t >> 6) * kTile;
+      for (int k = 0; k < 4; ++k) {
+        const int id = t + 256 * k, r = id >> 4, hh = (id >> 3) & 1, ch = id & 7;
+        scale_chunk(sm + G_DO + hh * kTile + sw128_off(r, 8 * ch), bv[r]);
+      }
+      // V'^T: rows i (128) x 8 chunks of columns r, four per thread
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint8_t *p = vp + sw128_off(t & 63, 8 * ch);
+      for (int k = 0; k < 4; ++k) {
+        const int id = t + 256 * k, row = id >> 3, ch = id & 7;
+        uint8_t *p = sm + G_VP + (row >> 6) * kTile + sw128_off(row & 63, 8 * ch);
         uint4 v = *reinterpret_cast<uint4 *>(p);
         uint32_t *w = &v.x;
 #pragma unroll
@@ -825,19 +822,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         *reinterpret_cast<uint4 *>(p) = v;
       }
-      if (t < 64) {  // T row t: columns scaled by e^{gc_col}
+      // T: 64 rows x 8 chunks, columns scaled by e^{gc_col}, two per thread
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint8_t *p = sm + G_T + sw128_off(t, 8 * ch);
-          uint4 v = *reinterpret_cast<uint4 *>(p);
-          uint32_t *w = &v.x;
+      for (int k = 0; k < 2; ++k) {
+        const int id = t + 256 * k, row = id >> 3, ch = id & 7;
+        uint8_t *p = sm + G_T + sw128_off(row, 8 * ch);
+        uint4 v = *reinterpret_cast<uint4 *>(p);
+        uint32_t *w = &v.x;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 x = unpack_bf16(w[e]);
-            w[e] = pack_bf16(x.x * bv[8 * ch + 2 * e], x.y * bv[8 * ch + 2 * e + 1]);
-          }
-          *reinterpret_cast<uint4 *>(p) = v;
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = unpack_bf16(w[e]);
+          w[e] = pack_bf16(x.x * bv[8 * ch + 2 * e], x.y * bv[8 * ch + 2 * e + 1]);
         }
+        *reinterpret_cast<uint4 *>(p) = v;
       }
     }
     sync_for_mma();
@@ -883,12 +880,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // partials p[j][r] = (AccT - AccH - AccB) K[r][j] + AccQ Q[r][j] into the
     // (now dead) V and dW^T tiles, fp32 [128][64], entry (j, r) at column
     // r ^ (j % 32) (writes by lanes j and reads by lanes r hit distinct banks)
-    const int j = t;
+    const int j = lq * 32 + lane;
     float *part = reinterpret_cast<float *>(sm + G_V);
     const uint8_t *kt = sm + G_KQ + 2 * (j >> 6) * kTile, *qt = kt + kTile;
     float dbl = 0.f;  // sum over r of AccB K
-#pragma unroll 1
-    for (int hp = 0; hp < 2; ++hp) {
+    {  // tokens 32 hs .. 32 hs + 31
+      const int hp = hs;
       float aq[32], at[32], ah[32], ab[32];
       tmem_ld32(lb + TG6 + 32 * hp, aq);
       tmem_ld32(lb + TG1 + 32 * hp, at);
@@ -914,8 +911,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       const uint8_t *dsr = sm + G_DS + 2 * (j >> 6) * kTile, *xr = sm + G_X + 2 * (j >> 6) * kTile;
       float acc = 0.f;
-#pragma unroll 1
-      for (int hc = 0; hc < 2; ++hc)
+      {
+        const int hc = hs;  // columns 64 hs .. 64 hs + 63 of the row
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const uint32_t off = hc * kTile + sw128_off(j & 63, 8 * ch);
@@ -928,18 +925,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc += p.x * q.x + p.y * q.y;
           }
         }
+      }
       dbl += bv[63] * acc;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dbl += __shfl_xor_sync(0xffffffffu, dbl, off);
     if (lane == 0) red[warp] = dbl;
     __syncthreads();
+    {  // partial sums of the gate partials over 32 key channels each
+      const int r = t & 63, qj = t >> 6;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 2
+      for (int jj = 32 * qj; jj < 32 * qj + 32; jj += 4) {
+        s0 += part[(jj + 0) * 64 + (r ^ ((jj + 0) & 31))];
+        s1 += part[(jj + 1) * 64 + (r ^ ((jj + 1) & 31))];
+        s2 += part[(jj + 2) * 64 + (r ^ ((jj + 2) & 31))];
+        s3 += part[(jj + 3) * 64 + (r ^ ((jj + 3) & 31))];
+      }
+      psum[64 * qj + r] = (s0 + s1) + (s2 + s3);
+    }
+    __syncthreads();
     if (t < 64) {  // dgc_r, then the reverse cumsum within the chunk; dbeta
       const int r = t;
-      float s = 0.f;
-#pragma unroll 8
-      for (int jj = 0; jj < 128; ++jj) s += part[jj * 64 + (r ^ (jj & 31))];
-      if (r == 63) s += red[0] + red[1] + red[2] + red[3];
+      float s = (psum[r] + psum[64 + r]) + (psum[128 + r] + psum[192 + r]);
+      if (r == 63)
+        s += ((red[0] + red[1]) + (red[2] + red[3])) + ((red[4] + red[5]) + (red[6] + red[7]));
       // reverse inclusive scan over r within two warps (rows 0-31, 32-63)
       float x = s;
 #pragma unroll
@@ -947,15 +957,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float y = __shfl_down_sync(0xffffffffu, x, off);
         if (lane + off < 32) x += y;
       }
-      gcv[320 + 64 + r] = x;  // scratch (after red)
-      dbeta2 += dbeta1[r];
-      if (r < L) a.dbeta[row0 + (size_t)r * H] = dbeta2;
+      scan[r] = x;
+      const float db = (dbeta2s[r] + dbeta2s[64 + r]) + (dbeta1[r] + dbeta1[64 + r]);
+      if (r < L) a.dbeta[row0 + (size_t)r * H] = db;
     }
     __syncthreads();
     if (t < 64) {
       const int r = t;
-      float x = gcv[320 + 64 + r];
-      if (r < 32) x += gcv[320 + 64 + 32];  // rows 32-63's total
+      float x = scan[r];
+      if (r < 32) x += scan[32];  // rows 32-63's total
       if (r < L) a.dg[row0 + (size_t)r * H] = x;
     }
   }
@@ -1034,7 +1044,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
                            (int)kGradSmem);
   if (e != cudaSuccess) return e;
   GradArgs ga{g, beta, sdo, dq, dk, dv, dg, dbeta, B, T, H, (int)n};
-  gdr_bwd_grad_kernel<<<(unsigned)nch, kThreads, kGradSmem, stream>>>(mq, mk, mv, mx, mds, mvp,
+  gdr_bwd_grad_kernel<<<(unsigned)nch, kGradThreads, kGradSmem, stream>>>(mq, mk, mv, mx, mds, mvp,
                                                                       mdv, mt, ga);
   return cudaGetLastError();
 }
