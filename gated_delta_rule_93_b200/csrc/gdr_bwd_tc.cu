@@ -46,8 +46,8 @@ using namespace sm100;
 using namespace tcu;
 
 constexpr int C = 64, D = 128;
-constexpr int kThreads = 128;      // the reverse state pass
-constexpr int kGradThreads = 256;  // the gradient pass
+constexpr int kStateThreads = 256;  // the reverse state pass
+constexpr int kGradThreads = 256;   // the gradient pass
 constexpr uint32_t kTile = 8192;             // one 64 x 64 bf16 tile (128-byte swizzle)
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
@@ -158,14 +158,16 @@ constexpr size_t kStateSmem = R_END + 1024;
 // TMEM columns: dS (fp32), its bf16 copy, dV'^T, Zc = dV'^T T~, D1 = [K; Q] K^T
 constexpr uint32_t TR_DS = 0, TR_DSB = 128, TR_DVP = 192, TR_ZC = 256, TR_D1 = 320;
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kStateThreads, 1)
     gdr_bwd_state_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmT, StateArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~uintptr_t(1023));
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // 8 warps: warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (value
+  // channels) and split each per-lane phase's columns between them (hs)
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, lq = warp & 3, hs = warp >> 2;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, H = a.H, n = a.n;
   uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + R_BAR), *bar_mma = bar_ld + 2;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + R_MISC);
@@ -186,12 +188,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
-  const uint32_t lb = tm + ((uint32_t)(warp * 32) << 16);  // this warp's 32 lanes
-  const int i = t;                                         // TMEM lane = value channel
+  const uint32_t lb = tm + ((uint32_t)(lq * 32) << 16);  // this warp's 32 lanes
+  const int i = lq * 32 + lane;                          // TMEM lane = value channel
 
   // dS = dL/dS_T (or 0)
 #pragma unroll 1
-  for (int q = 0; q < 4; ++q) {
+  for (int q = hs; q < 4; q += 2) {
     float x[32];
     const float *src = a.dST ? a.dST + ((size_t)bh * D + i) * D + 32 * q : nullptr;
 #pragma unroll
@@ -227,12 +229,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   // copy unit: this thread's row t / 2, channel half t % 2 (rows past T are
   // not copied).  Only the thread that copies a row half reads it back.
   auto load_dout = [&](int c) {
-    const int c0 = c * C, Lc = min(C, a.T - c0), r = t >> 1, hh = t & 1;
+    const int c0 = c * C, Lc = min(C, a.T - c0), r = t >> 2, qq = t & 3;
     if (r < Lc) {
-      const float *src = a.dout + (((size_t)b * a.T + c0 + r) * H + h) * D + 64 * hh;
-      uint8_t *dst = sm + R_STG + r * 512 + hh * 256;
+      const float *src = a.dout + (((size_t)b * a.T + c0 + r) * H + h) * D + 32 * qq;
+      uint8_t *dst = sm + R_STG + r * 512 + qq * 128;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) cp_async16(dst + 16 * e, src + 4 * e);
+      for (int e = 0; e < 8; ++e) cp_async16(dst + 16 * e, src + 4 * e);
     }
     cp_async_commit();
   };
@@ -261,14 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       kbv[lane] = __expf(gl - x0);
       kbv[lane + 32] = __expf(gl - x1);
     }
-    {  // dO rows (this thread's own asynchronous copies) -> bf16 tile
-      const int r = t >> 1, hh = t & 1;
+    {  // dO rows (this thread's own asynchronous copies) -> bf16 tile: row t / 4,
+       // channels 32 (t % 4) .. + 31 (tile (t % 4) / 2, 16-byte chunks 4 ((t % 4) % 2) ..)
+      const int r = t >> 2, qq = t & 3, hh = qq >> 1;
       cp_async_wait_all();
       uint8_t *tile = sm + R_DO + hh * kTile;
       const float4 *src = reinterpret_cast<const float4 *>(sm + R_STG + r * 512 + hh * 256);
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const int ch = (c8 + r) & 7;  // rotated: the lanes' reads spread over the banks
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const int ch = 4 * (qq & 1) + ((c4 + r) & 3);  // rotated: reads spread over the banks
         const float4 v0 = r < L ? src[2 * ch] : make_float4(0.f, 0.f, 0.f, 0.f);
         const float4 v1 = r < L ? src[2 * ch + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
         *reinterpret_cast<uint4 *>(tile + sw128_off(r, 8 * ch)) =
@@ -285,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float bl = bv[63];
       uint4 *dst = reinterpret_cast<uint4 *>(a.stash_ds + (((size_t)bh * n + ci) * D + i) * D);
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
+      for (int q = hs; q < 4; q += 2) {
         float x[32];
         tmem_ld32(lb + TR_DS + 32 * q, x);
         uint32_t u[16];
@@ -317,20 +320,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar_mma);
     }
     {  // meanwhile: K-bar = K e^{gl - gc} (new tiles); T~ = T Diag(e^{gc}) in place
-      const int r = t >> 1, hh = t & 1;
+      const int r = t >> 2, qq = t & 3, hh = qq >> 1;
       const float f = kbv[r];
       const uint8_t *src = kqp + 2 * hh * kTile;
       uint8_t *dst = sm + R_KB + hh * kTile;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t off = sw128_off(r, 8 * ch);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        const uint32_t off = sw128_off(r, 8 * (4 * (qq & 1) + c4));
         *reinterpret_cast<uint4 *>(dst + off) = *reinterpret_cast<const uint4 *>(src + off);
         scale_chunk(dst + off, f);
       }
-      // T~: row s = t / 2, columns 32 (t % 2) .. + 31 scaled by e^{gc_col}
+      // T~: row s = t / 4, columns 16 (t % 4) .. + 15 scaled by e^{gc_col}
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int col = 32 * hh + 8 * ch;
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col = 16 * qq + 8 * ch;
         uint8_t *p = ttp + sw128_off(r, col);
         uint4 v = *reinterpret_cast<uint4 *>(p);
         uint32_t *w = &v.x;
@@ -347,11 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) break;
     tc_fence_after();
     // ---- P = tril(Q K^T e^{gc_r - gc_s}) (TMEM lanes 64-127); Q~ = Q Diag(e^{gc}) in place
-    if (t >= 64) {
-      const int r = t - 64;
+    if (lq >= 2) {  // TMEM lanes 64-127 (rows r of Q K^T), columns 32 hs ..
+      const int r = i - 64;
       float x[32];
-#pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
+      {
+        const int hp = hs;
         tmem_ld32(lb + TR_D1 + 32 * hp, x);
         const float gr = gcv[r];
 #pragma unroll
@@ -363,11 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     {
-      const int r = t >> 1, hh = t & 1;
+      const int r = t >> 2, qq = t & 3, hh = qq >> 1;
       uint8_t *qt = kqp + (2 * hh + 1) * kTile;
       const float f = bv[r];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) scale_chunk(qt + sw128_off(r, 8 * ch), f);
+      for (int c4 = 0; c4 < 4; ++c4) scale_chunk(qt + sw128_off(r, 8 * (4 * (qq & 1) + c4)), f);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -389,24 +392,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     ph_mma ^= 1;
     if (!ok) break;
     tc_fence_after();
-    {  // dV'^T -> the stash and its bf16 copy in place
-      float x0[32], x1[32];
-      tmem_ld32(lb + TR_DVP, x0);
-      tmem_ld32(lb + TR_DVP + 32, x1);
+    {  // dV'^T -> the stash and its bf16 copy in place: columns 32 hs .., all
+       // reads before the writes
+      float x0[32];
+      tmem_ld32(lb + TR_DVP + 32 * hs, x0);
       uint32_t u[16];
       uint4 *dst = reinterpret_cast<uint4 *>(a.stash_dv + (((size_t)bh * n + ci) * D + i) * C);
 #pragma unroll
       for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x0[2 * e], x0[2 * e + 1]);
-      tmem_st16u(lb + TR_DVP, u);
+      __syncthreads();
+      tmem_st16u(lb + TR_DVP + 16 * hs, u);
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        dst[e] = make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) u[e] = pack_bf16(x1[2 * e], x1[2 * e + 1]);
-      tmem_st16u(lb + TR_DVP + 16, u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        dst[4 + e] = make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
+        dst[4 * hs + e] = make_uint4(u[4 * e], u[4 * e + 1], u[4 * e + 2], u[4 * e + 3]);
       tmem_wait_st();
     }
     tc_fence_before();
@@ -428,17 +426,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     ph_mma ^= 1;
     if (!ok) break;
     tc_fence_after();
-    {  // -Zc -> bf16 in place
-      float x0[32], x1[32];
-      tmem_ld32(lb + TR_ZC, x0);
-      tmem_ld32(lb + TR_ZC + 32, x1);
+    {  // -Zc -> bf16 in place: columns 32 hs .., all reads before the writes
+      float x0[32];
+      tmem_ld32(lb + TR_ZC + 32 * hs, x0);
       uint32_t u[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e) u[e] = pack_bf16(-x0[2 * e], -x0[2 * e + 1]);
-      tmem_st16u(lb + TR_ZC, u);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) u[e] = pack_bf16(-x1[2 * e], -x1[2 * e + 1]);
-      tmem_st16u(lb + TR_ZC + 16, u);
+      __syncthreads();
+      tmem_st16u(lb + TR_ZC + 16 * hs, u);
       tmem_wait_st();
     }
     tc_fence_before();
@@ -459,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (ok && a.dS0) {
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
+    for (int q = hs; q < 4; q += 2) {
       float x[32];
       tmem_ld32(lb + TR_DS + 32 * q, x);
       float4 *dst = reinterpret_cast<float4 *>(a.dS0 + ((size_t)bh * D + i) * D + 32 * q);
@@ -1036,7 +1031,7 @@ cudaError_t launch_bwd_tc(const void *q, const void *k, const void *v, const flo
                            (int)kStateSmem);
   if (e != cudaSuccess) return e;
   StateArgs ra{g, dout, dST, dS0, sds, sdv, sdo, B, T, H, (int)n, status};
-  gdr_bwd_state_kernel<<<(unsigned)(B * H), kThreads, kStateSmem, stream>>>(mk, mq, mt, ra);
+  gdr_bwd_state_kernel<<<(unsigned)(B * H), kStateThreads, kStateSmem, stream>>>(mk, mq, mt, ra);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // 3. the token gradients, one CTA per chunk and head
