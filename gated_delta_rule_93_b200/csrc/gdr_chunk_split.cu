@@ -54,8 +54,7 @@ using namespace sm100;
 using namespace tcu;
 
 constexpr int C = 64;
-constexpr int kThreads = 128;   // the delta-rule split kernel
-constexpr int kThreadsD = 256;  // the DPLR kernel
+constexpr int kThreadsD = 256;  // both kernels: 8 warps, two per TMEM lane quarter
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kMaxExp = 100.f * kLn2;  // largest |gc - m| of a scaled factor
@@ -260,25 +259,6 @@ __device__ __forceinline__ void put8(uint8_t *hi_tile, uint8_t *lo_tile, uint32_
                  pack_bf16(l[6], l[7]));
 }
 
-// 64 fp32 values as hi | lo bf16 pairs into 64 TMEM columns at `taddr`
-// (hi in the first 32 columns, lo in the next 32).
-__device__ __forceinline__ void tmem_put_split64(uint32_t taddr, const float (&x)[64]) {
-  uint32_t hu[16], lu[16];
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      float h0, l0, h1, l1;
-      split_bf16(x[32 * half + 2 * e], h0, l0);
-      split_bf16(x[32 * half + 2 * e + 1], h1, l1);
-      hu[e] = pack_bf16(h0, h1);
-      lu[e] = pack_bf16(l0, l1);
-    }
-    tmem_st16u(taddr + 16 * half, hu);
-    tmem_st16u(taddr + 32 + 16 * half, lu);
-  }
-}
-
 // 32 fp32 values as hi / lo bf16 pairs: 16 TMEM columns each at th and tl.
 __device__ __forceinline__ void tmem_put_split32(uint32_t th, uint32_t tl, const float (&x)[32]) {
   uint32_t hu[16], lu[16];
@@ -332,17 +312,17 @@ __device__ __forceinline__ void load_beta(float *betav, const float *beta, size_
 }
 
 // 1 / sqrt(|x|^2 + eps) of row r of k (flags & 2) and q (flags & 1); this
-// thread holds the columns [hf DK/2, hf DK/2 + DK/2) and its partner
-// (thread ^ 1) the others, so the sums meet with one shuffle.  Every lane
-// of the warp calls this.
+// thread holds the columns [hf DK/4, hf DK/4 + DK/4) and the three threads
+// beside it (thread ^ 1, ^ 2, ^ 3) the others, so the sums meet with two
+// shuffles.  Every lane of the warp calls this.
 template <bool BF, int DK>
 __device__ __forceinline__ void row_inv_norms(const void *k, const void *q, size_t tok0, int r,
                                               int hf, int H, int dk, int L, int flags, float &rk,
                                               float &rq) {
   float sk = 0.f, sq = 0.f;
 #pragma unroll
-  for (int g8 = 0; g8 < DK / 16; ++g8) {
-    const int c0 = hf * (DK / 2) + 8 * g8;
+  for (int g8 = 0; g8 < DK / 32; ++g8) {
+    const int c0 = hf * (DK / 4) + 8 * g8;
     const bool valid = r < L && c0 < dk;
     const size_t off = in_off(tok0, r, c0, H, dk, valid);
     float kx[8], qx[8];
@@ -356,18 +336,22 @@ __device__ __forceinline__ void row_inv_norms(const void *k, const void *q, size
   }
   sk += __shfl_xor_sync(0xffffffffu, sk, 1);
   sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+  sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 2);
   rk = (flags & 2) ? rsqrtf(sk + kNormEps) : 1.f;
   rq = (flags & 1) ? rsqrtf(sq + kNormEps) : 1.f;
 }
 
 template <int DK, bool PC, bool BF>
-__global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs a) {
+__global__ void __launch_bounds__(kThreadsD, 1) gdr_chunk_split_kernel(ChunkArgs a) {
   using LY = Layout<DK>;
   using TC = Cols<DK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~uintptr_t(1023));
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // 8 warps: warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31 (value
+  // channels) and split each per-lane phase's columns or rows between them (hs)
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, lq = warp & 3, hs = warp >> 2;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H, H = a.H;
   const int dk = a.dk, dv = a.dv;
   // sequence b: token rows [seq0, seq0 + Tb) of the [B, T] (or packed [1, total]) layout
@@ -401,12 +385,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
-  const uint32_t lb = tm + ((uint32_t)(warp * 32) << 16);  // this warp's lanes
-  const int i = t;                                         // value channel (TMEM lane)
+  const uint32_t lb = tm + ((uint32_t)(lq * 32) << 16);  // this warp's lanes
+  const int i = lq * 32 + lane;                          // value channel (TMEM lane)
 
   // S = S0 (or 0); lanes >= d_v and columns >= d_k stay 0
 #pragma unroll 1
-  for (int q = 0; q < DK / 32; ++q) {
+  for (int q = hs; q < DK / 32; q += 2) {
     float x[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
@@ -493,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     __syncthreads();
     // ---- S' = S Diag(e^{m}) as hi / lo bf16 in TMEM
 #pragma unroll 1
-    for (int q = 0; q < DK / 32; ++q) {
+    for (int q = hs; q < DK / 32; q += 2) {
       float x[32];
       tmem_ld32(lb + TC::S + 32 * q, x);
       uint32_t hu[16], lu[16];
@@ -509,15 +493,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
       tmem_st16u(lb + TC::SH + 16 * q, hu);
       tmem_st16u(lb + TC::SL + 16 * q, lu);
     }
-    // ---- K~, Q~, K^, (K e^{gl - gc})^T tiles: row r = t / 2, half t % 2 of the columns
+    // ---- K~, Q~, K^, (K e^{gl - gc})^T tiles: row r = t / 4, quarter t % 4 of the columns
     {
-      const int r = t >> 1, hf = t & 1;
+      const int r = t >> 2, hf = t & 3;
       bool range_bad = false;
-      float rk = 1.f, rq = 1.f;  // prologue: 1 / |k_r|, 1 / |q_r| (the pair t, t ^ 1 holds the row)
+      float rk = 1.f, rq = 1.f;  // prologue: 1 / |k_r|, 1 / |q_r| (threads 4 r .. 4 r + 3 hold the row)
       if (pro && a.norm_qk) row_inv_norms<BF, DK>(a.k, a.q, tok0, r, hf, H, dk, L, a.norm_qk, rk, rq);
 #pragma unroll
-      for (int g8 = 0; g8 < DK / 16; ++g8) {
-        const int c0 = hf * (DK / 2) + 8 * g8;
+      for (int g8 = 0; g8 < DK / 32; ++g8) {
+        const int c0 = hf * (DK / 4) + 8 * g8;
         const bool valid = r < L && c0 < dk;
         const size_t off = in_off(tok0, r, c0, H, dk, valid);
         float kx[8], qx[8];
@@ -586,12 +570,12 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     if (!ok) break;
     // ---- A (fp32, over K^) and P (hi / lo tiles) from D1; U's right-hand
     //      side V^T - zf Z into TMEM; S <- S Diag(e^{gl})
-    if (t < 64) {
+    if (lq < 2) {  // TMEM lanes 0-63: rows of A, columns 32 hs ..
       if (!add) {
-      const int r = t;
+      const int r = i;
       const float br = betav[r], gr = gcs[r];
-#pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
+      {
+        const int hp = hs;
         float x[32];
         tmem_ld32(lb + TC::D1 + 32 * hp, x);
 #pragma unroll
@@ -607,11 +591,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
         }
       }
       }
-    } else {
-      const int r = t - 64;
+    } else {  // TMEM lanes 64-127: rows of P, columns 32 hs ..
+      const int r = i - 64;
       const float gr = gcs[r];
-#pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
+      {
+        const int hp = hs;
         float x[32], hi[32], lo[32];
         tmem_ld32(lb + TC::D1 + 32 * hp, x);
 #pragma unroll
@@ -624,29 +608,26 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
         st_row32(sm + LY::PP_LO, r, hp, lo);
       }
     }
-    {
-      float z[64];
-      {
-        float z0[32], z1[32];
-        tmem_ld32(lb + TC::ZO, z0);
-        tmem_ld32(lb + TC::ZO + 32, z1);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          z[e] = z0[e];
-          z[32 + e] = z1[e];
-        }
-      }
+    {  // rows 32 hs .. 32 hs + 31 of this lane; all reads before any write
+      float z[32];
+      tmem_ld32(lb + TC::ZO + 32 * hs, z);
       const int ic = i < dv ? i : 0;
-      float vr[64];
+      float vr[32];
 #pragma unroll
-      for (int r = 0; r < C; ++r) vr[r] = ld1<BF>(a.v, (tok0 + (size_t)(r < L ? r : 0) * H) * dv + ic);
+      for (int e = 0; e < 32; ++e) {
+        const int r = 32 * hs + e;
+        vr[e] = ld1<BF>(a.v, (tok0 + (size_t)(r < L ? r : 0) * H) * dv + ic);
+      }
 #pragma unroll
-      for (int r = 0; r < C; ++r)
-        z[r] = ((r < L && i < dv) ? vr[r] : 0.f) - (add ? 0.f : zf[r] * z[r]);
-      tmem_put_split64(lb + TC::ZO, z);
+      for (int e = 0; e < 32; ++e) {
+        const int r = 32 * hs + e;
+        z[e] = ((r < L && i < dv) ? vr[e] : 0.f) - (add ? 0.f : zf[r] * z[e]);
+      }
+      __syncthreads();
+      tmem_put_split32(lb + TC::ZO + 16 * hs, lb + TC::ZO + 32 + 16 * hs, z);
     }
 #pragma unroll 1
-    for (int q = 0; q < DK / 32; ++q) {
+    for (int q = hs; q < DK / 32; q += 2) {
       float x[32];
       tmem_ld32(lb + TC::S + 32 * q, x);
 #pragma unroll
@@ -685,19 +666,11 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     }
     mma_wait();
     if (!ok) break;
-    {
-      float u[64];
-      {
-        float u0[32], u1[32];
-        tmem_ld32(lb + TC::U, u0);
-        tmem_ld32(lb + TC::U + 32, u1);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          u[e] = u0[e];
-          u[32 + e] = u1[e];
-        }
-      }
-      tmem_put_split64(lb + TC::U, u);
+    {  // rows 32 hs .. of this lane; all reads before any write
+      float u[32];
+      tmem_ld32(lb + TC::U + 32 * hs, u);
+      __syncthreads();
+      tmem_put_split32(lb + TC::U + 16 * hs, lb + TC::U + 32 + 16 * hs, u);
     }
     }  // !add
     sync_for_mma();
@@ -719,9 +692,9 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
     }
     mma_wait();
     if (!ok) break;
-    // ---- o_r = zf_r O_a + O_b (lane = value channel)
-#pragma unroll 1
-    for (int hp = 0; hp < 2; ++hp) {
+    // ---- o_r = zf_r O_a + O_b (lane = value channel; rows 32 hs ..)
+    {
+      const int hp = hs;
       float oa[32], ob[32];
       tmem_ld32(lb + TC::ZO + 64 + 32 * hp, oa);
       tmem_ld32(lb + TC::D1 + 32 * hp, ob);
@@ -737,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdr_chunk_split_kernel(ChunkArgs 
   }
   if (ok && a.S_T) {
 #pragma unroll 1
-    for (int q = 0; q < DK / 32; ++q) {
+    for (int q = hs; q < DK / 32; q += 2) {
       float x[32];
       tmem_ld32(lb + TC::S + 32 * q, x);
       if (i < dv) {
@@ -766,7 +739,7 @@ cudaError_t launch_split(const ChunkArgs &a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Layout<DK>::bytes);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(a.B * a.H), kThreads, Layout<DK>::bytes, stream>>>(a);
+  kern<<<(unsigned)(a.B * a.H), kThreadsD, Layout<DK>::bytes, stream>>>(a);
   return cudaGetLastError();
 }
 
