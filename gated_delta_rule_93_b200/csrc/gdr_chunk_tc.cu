@@ -167,7 +167,7 @@ enum {
   B_GF = B_SCALED + 2, // [4] PC: gate rows of a scaling warp landed    (1 + tx)
                        //     (warp w, rows 0-31 / 32-63: 2 w + half)
   B_NORM = B_GF,       // [3] prologue (scalar gates): token norms of a
-                       //     stage folded into its vectors (prep-side MMA warp)
+                       //     stage folded into its vectors (prep group, 1 thread)
   B_COUNT = B_GF + 4
 };
 static_assert(B_COUNT <= 40, "barrier slots");
@@ -626,13 +626,9 @@ __device__ __forceinline__ float softplus_f(float x) {
 }
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + __expf(-x)); }
 
-// L2-normalise the K rows (nk) and Q rows (nq) of a landed K/Q stage in
-// place, one warp: lane l takes row l and l + 32 of each.  A row's 128
-// channels are its 128-byte row in the h0 tile and in the h1 tile; the sum
-// of squares and the scaling do not depend on the order of the 16-byte
-// chunks, so the swizzle is ignored and each lane starts at chunk l % 8,
-// which puts the 8 lanes of a 16-byte access phase on distinct banks.
-// Rows past the sequence's end were filled with zeros and stay zero.
+// Token norms (prologue), in the prep group.  |k_s|^2 is the diagonal of
+// K K^T, which D1 already holds (rows 0-63); |q_r|^2 is summed from the
+// landed Q tiles, two threads per token.
 __device__ __forceinline__ float sumsq_bf16x8(uint4 x, float ss) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -644,42 +640,30 @@ __device__ __forceinline__ float sumsq_bf16x8(uint4 x, float ss) {
   return ss;
 }
 
-// 1 / sqrt(|x|^2 + eps) of one 128-channel row of a landed K/Q stage: its
-// 128-byte row in the h0 tile (p0) and in the h1 tile (p0 + 2 tiles).  The
+// Sum of squares of one 128-byte row of a swizzled 64-channel tile.  The
 // sum does not depend on the order of the 16-byte chunks, so the swizzle is
 // ignored and lane l starts at chunk l % 8, which puts the 8 lanes of a
-// 16-byte access phase on distinct banks.  Zero rows (past the sequence's
-// end) give a finite factor.
-__device__ __forceinline__ float row_inv_norm(const uint8_t *p0, int lane) {
-  const uint8_t *p1 = p0 + 2 * kTileBytes;
-  float s0 = 0.f, s1 = 0.f;
+// 16-byte access phase on distinct banks.
+__device__ __forceinline__ float row_sumsq_half(const uint8_t *row, int lane) {
+  float s = 0.f;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int ch = ((p + lane) & 7) * 16;
-    s0 = sumsq_bf16x8(*reinterpret_cast<const uint4 *>(p0 + ch), s0);
-    s1 = sumsq_bf16x8(*reinterpret_cast<const uint4 *>(p1 + ch), s1);
-  }
-  return rsqrtf(s0 + s1 + kNormEps);
+  for (int p = 0; p < 8; ++p)
+    s = sumsq_bf16x8(*reinterpret_cast<const uint4 *>(row + ((p + lane) & 7) * 16), s);
+  return s;
 }
 
-// Prologue, one warp, once a stage has landed (lane l: tokens l and l + 32):
-// 1 / |k| into Rk and folded into the vectors that meet K (Ieg, Egl in
-// place, SEgK = SEg rk), 1 / |q| into Rq and SEgQ = SEg rq.
-__device__ __forceinline__ void fold_token_norms(const uint8_t *kq, float *gv, int lane, bool nq,
-                                                 bool nk) {
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    const int t = lane + 32 * half;
-    const float rk = nk ? row_inv_norm(kq + t * 128, lane) : 1.f;
-    const float rq = nq ? row_inv_norm(kq + kTileBytes + t * 128, lane) : 1.f;
-    const float seg = gv[kGateSEg + t];
-    gv[kGateRk + t] = rk;
-    gv[kGateRq + t] = rq;
-    gv[kGateSEgK + t] = seg * rk;
-    gv[kGateSEgQ + t] = seg * rq;
-    gv[kGateIeg + t] *= rk;
-    gv[kGateEgl + t] *= rk;
-  }
+// x[lane] of a register row, by a select tree on the lane's bits.
+__device__ __forceinline__ float pick_lane(const float (&x)[32], int lane) {
+  float y[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) y[e] = (lane & 1) ? x[2 * e + 1] : x[2 * e];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] = (lane & 2) ? y[2 * e + 1] : y[2 * e];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) y[e] = (lane & 4) ? y[2 * e + 1] : y[2 * e];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) y[e] = (lane & 8) ? y[2 * e + 1] : y[2 * e];
+  return (lane & 16) ? y[1] : y[0];
 }
 
 // Scalar gates of one stage from the per-token log decays (gl0: token lane,
@@ -1235,10 +1219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kPrepMmaWarp) {
     // ================================================================ prep-side MMAs
-    // (prologue: after issuing D1 of a chunk, the whole warp folds the
-    // chunk's token norms into its vectors, off the K/Q load's path; the
-    // prep group next needs them about an inverse later)
-    if (PRO || lane == 0) {
+    if (lane == 0) {
       const uint32_t a_kq = smem_u32(sm + Lay::KQ), a_kh = smem_u32(sm + Lay::KH);
       auto W = [&](int slot, uint32_t parity) {
         const bool ok = wait_or_abort(&bars[slot], parity, abort_flag);
@@ -1262,31 +1243,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bars[B_D1F]);
       };
-      auto norms = [&](int c) {
-        if (!PRO) return;
-        __syncwarp();
-        const int s = c % kStages;
-        fold_token_norms(sm + Lay::KQ + s * 4 * kTileBytes, gate_slot(c), lane,
-                         (a.norm_qk & 1) != 0, (a.norm_qk & 2) != 0);
-        warp_arrive(&bars[B_NORM + s]);
-      };
       // D1 of chunk c + 1 goes out as soon as the prep group has read D1 of
       // chunk c and the chunk's operands are ready.
       bool ok = ready(0);
-      if (ok) {
-        if (lane == 0) issue_d1(0);
-        norms(0);
-      }
+      if (ok) issue_d1(0);
       for (int c = 0; c + 1 < n && ok; ++c) {
         if (!(ok = W(B_D1E, c & 1) && ready(c + 1))) break;
-        if (lane == 0) issue_d1(c + 1);
-        norms(c + 1);
+        issue_d1(c + 1);
       }
-      if (lane == 0) {
-        mma_commit(&bars[B_FIN2]);
-        drain_wait(&bars[B_FIN2], 0);
-        if (!ok) atomicOr(a.status, kStatusTimeout);
-      }
+      mma_commit(&bars[B_FIN2]);
+      drain_wait(&bars[B_FIN2], 0);
+      if (!ok) atomicOr(a.status, kStatusTimeout);
     }
   } else if (warp >= 4 && warp < 8) {
     // ================================================================ prep group
@@ -1307,13 +1274,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       // four prep warps; the P warps probe D1 again in its place).
       // (ADD: no A, so no wait on AF)
       const bool a_rows = !ADD && pt < 64;
-      // (prologue: also the chunk's token norms, in place of the stage)
-      bool bad = !wait_all<4>({PRO ? &bars[B_NORM + st] : &bars[B_FULL + st], &bars[B_D1F],
+      bool bad = !wait_all<4>({&bars[B_FULL + st], &bars[B_D1F],
                                &bars[B_PE + (c & 1)],
                                a_rows ? &bars[B_TRDY + ((c - 1) & 1)] : &bars[B_D1F]},
                               {uint32_t((c / kStages) & 1), ph, uint32_t(((c >> 1) - 1) & 1),
                                a_rows ? uint32_t(((c - 1) >> 1) & 1) : ph},
                               abort_flag);
+      if (PRO) {
+        // Token norms: 1 / |k| into Rk and folded into the vectors that meet
+        // K (Ieg, Egl in place, SEgK = SEg rk), 1 / |q| into Rq and SEgQ =
+        // SEg rq.  Thread pt sums half a Q row (token pt / 2, channels
+        // 64 (pt % 2) ..); the A rows' threads read their own |k|^2 off D1.
+        // Nothing here is skipped on a failed wait: the loads stay in
+        // bounds and the shuffle needs every lane; only the writes are.
+        float *gw = gate_slot(c);
+        const uint8_t *kq = sm + Lay::KQ + st * 4 * kTileBytes;
+        float sq = row_sumsq_half(kq + (1 + 2 * (pt & 1)) * kTileBytes + (pt >> 1) * 128, lane);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        tc_fence_after();
+        if (rl < 64) {  // warps 4, 5: D1[rl][rl] is column lane of half rl / 32
+          float x[32];
+          tmem_ld32(lane_base + TM_D1 + 32 * (rl >> 5), x);
+          const float rk = (a.norm_qk & 2) ? rsqrtf(pick_lane(x, lane) + kNormEps) : 1.f;
+          if (!bad) {
+            gw[kGateRk + rl] = rk;
+            gw[kGateSEgK + rl] = gw[kGateSEg + rl] * rk;
+            gw[kGateIeg + rl] *= rk;
+            gw[kGateEgl + rl] *= rk;
+          }
+        }
+        if (!bad && (pt & 1) == 0) {
+          const float rq = (a.norm_qk & 1) ? rsqrtf(sq + kNormEps) : 1.f;
+          gw[kGateRq + (pt >> 1)] = rq;
+          gw[kGateSEgQ + (pt >> 1)] = gw[kGateSEg + (pt >> 1)] * rq;
+        }
+        // The group's norms are in; the state group waits for them on the
+        // stage's norm barrier.
+        if (!group_any(kBar, bad) && pt == 0) mbar_arrive(&bars[B_NORM + st]);
+      }
       if (!bad && (!ADD || rl >= 64) && (rl < 64 || a.write_o)) {
         const bool factored = -gcv[63] < kSafeDecay;
         // ---- A (lanes 0-63) and P (lanes 64-127) from D1, 32 columns at a time
