@@ -99,3 +99,26 @@ def test_roofline_fields_arithmetic(monkeypatch):
     # two ranks: the whole job's tokens over the (max-over-ranks) time
     f2 = bench.roofline_fields(w, total, per_launch, steps, 2, None)
     assert f2["value"] == pytest.approx(2 * f["value"])
+
+
+def test_reference_arm_prints_one_json_line():
+    """`bench.py --impl reference` times the oracle on the host and prints the
+    contract's line: impl, cpu_baseline, a zero-copy e2e and no GPU launch."""
+    import json
+    import subprocess
+    import sys
+
+    r = subprocess.run([sys.executable, bench.__file__, "--impl", "reference", "--workload",
+                        "tiny_fp32", "--steps", "2", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["gpu_launches"] == 0
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["warmup"] >= 3 and d["steps"] == 2
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == "tiny_fp32"
