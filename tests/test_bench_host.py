@@ -1,8 +1,8 @@
 """Host logic of bench.py, on CPU: which kernel's sources a workload's
 profile is tied to, the algorithmic bytes each roofline divides by (counted
 here tensor by tensor from the workload's shapes), the rule that a recorded
-DRAM figure is reported only while its source hash still matches, and the
-roofline arithmetic of one timed workload."""
+DRAM figure is reported only while its source hash still matches, the
+roofline arithmetic of one timed workload, and the reference arm's line."""
 import pytest
 import torch
 
